@@ -1,0 +1,231 @@
+/*
+ * paged_kv.h — C ABI of libpagedkv: a paged KV cache and PagedAttention decode
+ * for NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (sources cited by page title and section):
+ *
+ *  - "vLLM's 'memory paging' — PagedAttention illustrated", §2: the KV cache is
+ *    cut into fixed-size pages (blocks of 8/16/... tokens); every sequence
+ *    keeps a page table of physical blocks that need not be contiguous; a
+ *    scheduler hands blocks out from a free list and takes them back.
+ *  - same page, §3 phase 1: a new token goes into the sequence's current
+ *    block; when that block is full the next token takes a fresh block from
+ *    the free list and the table grows by one entry (no copy of old data).
+ *  - same page, §3 phase 2: attention reads the table, treats the scattered
+ *    blocks as one logically contiguous K and V, and runs ordinary attention
+ *    (scores q·Kᵀ, softmax, weighted sum of V).
+ *  - same page, §3 phase 3 and §4: blocks shared by several sequences carry a
+ *    reference count and are freed by the last sharer; writing into a shared
+ *    block goes to a private copy first; admission refuses work that does not
+ *    fit instead of running out of memory; abort frees a request's blocks.
+ *  - "LLM inference optimisation: principles overview", §3.3: page layout and
+ *    block sizes 8/16/32.
+ *
+ * Conventions
+ *  - Every function returns an int status: PKV_OK (0) or a negative PKV_ERR_*.
+ *    pkv_last_error_string() gives the text of the calling thread's last error.
+ *  - Argument errors are reported synchronously, before anything is launched.
+ *  - Device pointers are owned by the caller (allocated e.g. by PyTorch); the
+ *    library never allocates or frees device memory.  Device buffers must be
+ *    16-byte aligned and densely packed in the layouts stated below.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Kernels are launched asynchronously on it; returning PKV_OK means the
+ *    launch was accepted.  Faults found by the kernels themselves (a block id
+ *    outside the pool, a wait that ran out) are recorded in a device status
+ *    word read with pkv_device_status().
+ *  - dtype: PKV_F32, PKV_BF16 or PKV_F16 — the element type of q, the new K/V
+ *    rows and the K/V pools.  Attention output is always float32.
+ *
+ * KV pool layout: K and V are separate pools, each
+ *     [num_blocks][num_kv_heads][block_size][head_dim]   (head_dim fastest)
+ * so one (block, kv head) is a contiguous block_size*head_dim tile.  Slot
+ * s = block*block_size + offset names token row `offset` of physical block
+ * `block`.  Supported: head_dim in {64, 128}, block_size in {8, 16, 32},
+ * num_q_heads / num_kv_heads in {1, 2, 4, 8}.
+ */
+#ifndef PAGED_KV_H
+#define PAGED_KV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum pkv_status {
+  PKV_OK = 0,
+  PKV_ERR_INVALID_ARG = -1,    /* bad size, null pointer, misalignment */
+  PKV_ERR_OUT_OF_BLOCKS = -2,  /* not enough free blocks; nothing changed */
+  PKV_ERR_UNKNOWN_SEQ = -3,    /* sequence id not present */
+  PKV_ERR_UNSUPPORTED = -4,    /* dtype / head_dim / block_size / group size */
+  PKV_ERR_CUDA = -5,           /* a CUDA runtime call failed */
+  PKV_ERR_DEVICE_TIMEOUT = -6, /* a bounded device wait gave up */
+  PKV_ERR_SEQ_EXISTS = -7,     /* sequence id already present */
+  PKV_ERR_BAD_BLOCK = -8       /* a kernel met a block id / slot outside the pool */
+};
+
+enum pkv_dtype { PKV_F32 = 0, PKV_BF16 = 1, PKV_F16 = 2 };
+
+/* Text of the calling thread's most recent error ("" if none).  The pointer
+ * stays valid until the thread's next library call. */
+const char* pkv_last_error_string(void);
+
+/* Library version string, e.g. "1.0.0". */
+const char* pkv_version(void);
+
+/* ------------------------------------------------------------------------ */
+/* Host block allocator (vLLM paging page §2, §3 phases 1 and 3, §4).       */
+/* All of it runs on the host in integers.  A pkv_alloc_t is not thread-safe:
+ * one thread at a time.  Every failing call leaves the allocator unchanged. */
+/* ------------------------------------------------------------------------ */
+
+typedef struct pkv_alloc pkv_alloc_t;
+
+typedef struct pkv_stats {
+  int64_t num_blocks;
+  int64_t block_size;
+  int64_t free_blocks;
+  int64_t used_blocks;    /* num_blocks - free_blocks */
+  int64_t num_seqs;
+  int64_t cow_copies;     /* copy-on-write pairs issued since creation */
+  int64_t logical_tokens; /* sum of sequence lengths (shared tokens counted per sharer) */
+  int64_t waste_tokens;   /* over distinct used blocks: block_size - the fullest sharer's fill */
+} pkv_stats_t;
+
+/* Create an allocator over blocks 0..num_blocks-1.  The free list is a LIFO
+ * stack; `free_order` (num_blocks distinct ids, may be NULL for 0,1,2,...)
+ * gives the order in which blocks are first handed out: free_order[0] first.
+ * Callers pass a seeded permutation to scatter sequences across the pool.
+ * Errors: INVALID_ARG (sizes <= 0, free_order not a permutation). */
+int pkv_alloc_create(int32_t num_blocks, int32_t block_size, const int32_t* free_order,
+                     pkv_alloc_t** out);
+
+/* Free the allocator (NULL is ignored). */
+void pkv_alloc_destroy(pkv_alloc_t* a);
+
+/* Admit a sequence that already holds n_tokens tokens (e.g. a prompt):
+ * reserves ceil(n_tokens / block_size) blocks at once, or none
+ * (admission control, vLLM paging page §4).
+ * Errors: SEQ_EXISTS, OUT_OF_BLOCKS, INVALID_ARG (n_tokens < 0). */
+int pkv_seq_add(pkv_alloc_t* a, int64_t seq_id, int32_t n_tokens);
+
+/* Make `child` share every block of `parent` (refcount + 1 each); child gets
+ * parent's length.  Prefix sharing, vLLM paging page §3 phase 3.
+ * Errors: UNKNOWN_SEQ (parent), SEQ_EXISTS (child). */
+int pkv_seq_fork(pkv_alloc_t* a, int64_t parent, int64_t child);
+
+/* Reserve the slot of one new token for each listed sequence, in list order
+ * (vLLM paging page §3 phase 1).  For a sequence of length L the new token is
+ * position L:
+ *   - if L % block_size == 0 a block is popped from the free list and
+ *     appended to its table;
+ *   - else if its last block is shared (refcount > 1) a block is popped, the
+ *     pair (old, new) is written to cow_pairs_out (copy the old block's K/V
+ *     into the new one before writing the token: pkv_copy_blocks), the old
+ *     block's refcount drops by one and the table entry now names the new one;
+ *   - the slot table[L / block_size] * block_size + L % block_size is written
+ *     to slot_out[i] and the length becomes L + 1.
+ * slot_out: int32[n].  cow_pairs_out: int32[cow_capacity][2] (src, dst);
+ * *n_cow receives the number of pairs.  At most n pairs are produced, so
+ * cow_capacity >= n always suffices.
+ * All-or-nothing: on OUT_OF_BLOCKS, UNKNOWN_SEQ or INVALID_ARG (cow_capacity
+ * too small) no sequence changes. */
+int pkv_seq_append_slots(pkv_alloc_t* a, const int64_t* seq_ids, int32_t n,
+                         int32_t* slot_out, int32_t* cow_pairs_out, int32_t cow_capacity,
+                         int32_t* n_cow);
+
+/* End (or abort) a sequence: each of its blocks loses one reference, and a
+ * block reaching zero goes back on the free stack, in table order (vLLM paging
+ * page §3 phase 3, §4 abort).  Errors: UNKNOWN_SEQ. */
+int pkv_seq_free(pkv_alloc_t* a, int64_t seq_id);
+
+/* Current length (tokens) of a sequence.  Errors: UNKNOWN_SEQ. */
+int pkv_seq_len(const pkv_alloc_t* a, int64_t seq_id, int32_t* len);
+
+/* Write the block tables of the listed sequences as rows of
+ * tables_out[n][max_blocks] (unused entries = -1) and their lengths to
+ * seq_lens_out[n] (may be NULL).  Errors: UNKNOWN_SEQ, INVALID_ARG (a table
+ * longer than max_blocks). */
+int pkv_block_tables(const pkv_alloc_t* a, const int64_t* seq_ids, int32_t n, int32_t max_blocks,
+                     int32_t* tables_out, int32_t* seq_lens_out);
+
+/* Usage counters (vLLM paging page §5 lists KV cache usage as the metric to
+ * watch).  Errors: INVALID_ARG. */
+int pkv_alloc_stats(const pkv_alloc_t* a, pkv_stats_t* out);
+
+/* ------------------------------------------------------------------------ */
+/* Device operations (sm_100a).                                             */
+/* ------------------------------------------------------------------------ */
+
+/* KV append ("reshape_and_cache"): for each i < n_tokens with
+ * slot_mapping[i] >= 0, copy rows k_new[i][h][:] and v_new[i][h][:] (all
+ * heads) into slot slot_mapping[i] of k_pool / v_pool; slot < 0 is a padding
+ * token and writes nothing.  Bit-exact copy (vLLM paging page §3 phase 1;
+ * optimisation-overview page §2.2: O(1) append, no copy of old data).
+ * k_new, v_new: dtype[n_tokens][num_kv_heads][head_dim]; slot_mapping:
+ * int32[n_tokens] on the device.  A slot >= num_blocks*block_size is skipped
+ * and recorded as PKV_ERR_BAD_BLOCK in the device status.
+ * Two tokens given the same slot: which write wins is unspecified. */
+int pkv_kv_append(const void* k_new, const void* v_new, const int32_t* slot_mapping,
+                  int32_t n_tokens, void* k_pool, void* v_pool, int32_t num_blocks,
+                  int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t dtype,
+                  void* stream);
+
+/* Copy whole blocks (every head and offset of K and V) src -> dst for each
+ * pair in block_pairs: int32[n_pairs][2] on the device — the copy-on-write
+ * step of the vLLM paging page §3 phase 3.  Pairs must not chain (no dst is
+ * another pair's src) and dsts must be distinct; pairs from
+ * pkv_seq_append_slots satisfy both.  Ids outside the pool are skipped and
+ * recorded as PKV_ERR_BAD_BLOCK. */
+int pkv_copy_blocks(void* k_pool, void* v_pool, const int32_t* block_pairs, int32_t n_pairs,
+                    int32_t num_blocks, int32_t num_kv_heads, int32_t head_dim,
+                    int32_t block_size, int32_t dtype, void* stream);
+
+/* Bytes of device workspace pkv_paged_attention_decode needs for these sizes
+ * (split-partition partials and the work list).  partition_tokens as for the
+ * decode call (0 = automatic); the value depends only on the arguments. */
+int pkv_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                              int32_t head_dim, int32_t max_blocks_per_seq, int32_t block_size,
+                              int32_t partition_tokens, size_t* bytes);
+
+/* PagedAttention decode (vLLM paging page §3 phase 2): for every sequence b
+ * and query head h, with G = num_q_heads / num_kv_heads and g = h / G,
+ *     out[b][h][:] = sum_t softmax_t(scale * q[b][h]·K_b[t][g]) * V_b[t][g][:]
+ * over the seq_lens[b] tokens t of sequence b, where token t of b lives in
+ * physical block block_tables[b][t / block_size] at offset t % block_size.
+ * No mask: the decode query is the newest position and sees every cached
+ * token (call pkv_kv_append first to include the new token itself).
+ * seq_lens[b] == 0 gives zeros.
+ *
+ * q: dtype[num_seqs][num_q_heads][head_dim]; block_tables:
+ * int32[num_seqs][max_blocks_per_seq]; seq_lens: int32[num_seqs], each in
+ * [0, max_blocks_per_seq*block_size]; out: float32[num_seqs][num_q_heads][head_dim].
+ * The softmax is single-pass (online max and sum, fp32 accumulation).
+ * Sequences longer than partition_tokens are split into partitions of that
+ * many tokens (a multiple of block_size; 0 = automatic), whose partial
+ * results are merged by a second kernel with the max/sum rescaling.
+ * workspace: at least pkv_decode_workspace_size(...) bytes of device memory,
+ * 256-byte aligned, used as scratch for the duration of the call (do not
+ * share one workspace between calls that may run concurrently).
+ * Table entries outside [0, num_blocks) are not read; they are recorded as
+ * PKV_ERR_BAD_BLOCK and block 0 is read in their place. */
+int pkv_paged_attention_decode(const void* q, const void* k_pool, const void* v_pool,
+                               const int32_t* block_tables, const int32_t* seq_lens,
+                               int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                               int32_t head_dim, int32_t num_blocks, int32_t max_blocks_per_seq,
+                               int32_t block_size, float scale, int32_t dtype,
+                               int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                               float* out, void* stream);
+
+/* Synchronise `stream`, then read the device status word of the current
+ * device into *status: PKV_OK, or the first PKV_ERR_BAD_BLOCK /
+ * PKV_ERR_DEVICE_TIMEOUT a kernel recorded since the last clear.  clear != 0
+ * resets it to PKV_OK.  Returns PKV_ERR_CUDA if the synchronisation failed. */
+int pkv_device_status(void* stream, int32_t* status, int32_t clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGED_KV_H */

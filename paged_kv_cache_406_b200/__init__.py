@@ -1,0 +1,13 @@
+"""paged_kv_cache_406_b200 — a paged KV cache and PagedAttention decode for
+NVIDIA B200 (sm_100a).
+
+The work is done by ``libpagedkv.so`` (hand-written CUDA kernels plus a C++
+host block allocator, C ABI in ``include/paged_kv.h``); this package is its
+thin Python binding.  Build the library with
+``python -m paged_kv_cache_406_b200.build``.
+"""
+from .binding import (Allocator, PagedKVError, pkv_copy_blocks, pkv_decode_workspace_size,  # noqa: F401
+                      pkv_device_status, pkv_kv_append, pkv_paged_attention_decode)
+from ._native import LIB_PATH, lib  # noqa: F401
+
+__version__ = "1.0.0"

@@ -1,0 +1,217 @@
+"""Tensor-level binding: the C entry points under their own names, taking
+PyTorch tensors.
+
+Each function checks dtypes, devices, shapes and contiguity, then passes
+``data_ptr()`` values and ``torch.cuda.current_stream().cuda_stream`` to the
+library.  PyTorch supplies device memory and streams; every step of the
+paged-KV path runs in libpagedkv's kernels (device) or allocator (host).
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+from . import _native as N
+from ._native import PagedKVError, check, lib
+
+_DTYPES = {torch.float32: N.PKV_F32, torch.bfloat16: N.PKV_BF16, torch.float16: N.PKV_F16}
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype not in _DTYPES:
+        raise TypeError(f"unsupported dtype {t.dtype}; expected float32, bfloat16 or float16")
+    return _DTYPES[t.dtype]
+
+
+def _cuda(t: torch.Tensor, name: str, dtype=None) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _pool_dims(k_pool: torch.Tensor, v_pool: torch.Tensor):
+    if k_pool.dim() != 4 or k_pool.shape != v_pool.shape or k_pool.dtype != v_pool.dtype:
+        raise ValueError("k_pool and v_pool must both be [num_blocks, num_kv_heads, block_size, head_dim], same dtype")
+    nb, hkv, bs, d = k_pool.shape
+    return nb, hkv, bs, d
+
+
+# ----------------------------------------------------------------------------
+# device operations
+# ----------------------------------------------------------------------------
+
+def pkv_kv_append(k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: torch.Tensor,
+                  k_pool: torch.Tensor, v_pool: torch.Tensor) -> None:
+    """Write each new token's K/V rows into its slot (``slot < 0`` = padding)."""
+    nb, hkv, bs, d = _pool_dims(_cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"))
+    for name, t in (("k_new", k_new), ("v_new", v_new)):
+        _cuda(t, name, k_pool.dtype)
+        if t.dim() != 3 or t.shape[1:] != (hkv, d):
+            raise ValueError(f"{name} must be [n_tokens, {hkv}, {d}]")
+    if k_new.shape != v_new.shape:
+        raise ValueError("k_new and v_new differ in shape")
+    _cuda(slot_mapping, "slot_mapping", torch.int32)
+    if slot_mapping.numel() != k_new.shape[0]:
+        raise ValueError("slot_mapping must hold one slot per new token")
+    check(lib().pkv_kv_append(k_new.data_ptr(), v_new.data_ptr(), slot_mapping.data_ptr(), k_new.shape[0],
+                              k_pool.data_ptr(), v_pool.data_ptr(), nb, hkv, d, bs, _dtype_code(k_pool),
+                              _stream()))
+
+
+def pkv_copy_blocks(k_pool: torch.Tensor, v_pool: torch.Tensor, block_pairs: torch.Tensor) -> None:
+    """Copy whole blocks src → dst for each ``(src, dst)`` row of ``block_pairs``."""
+    nb, hkv, bs, d = _pool_dims(_cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"))
+    _cuda(block_pairs, "block_pairs", torch.int32)
+    if block_pairs.numel() % 2:
+        raise ValueError("block_pairs must be [n_pairs, 2]")
+    n = block_pairs.numel() // 2
+    check(lib().pkv_copy_blocks(k_pool.data_ptr(), v_pool.data_ptr(), block_pairs.data_ptr(), n, nb, hkv, d, bs,
+                                _dtype_code(k_pool), _stream()))
+
+
+def pkv_decode_workspace_size(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                              max_blocks_per_seq: int, block_size: int, partition_tokens: int = 0) -> int:
+    out = ctypes.c_size_t(0)
+    check(lib().pkv_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                                          block_size, partition_tokens, ctypes.byref(out)))
+    return out.value
+
+
+def pkv_paged_attention_decode(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                               block_tables: torch.Tensor, seq_lens: torch.Tensor, scale: float,
+                               out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                               partition_tokens: int = 0) -> torch.Tensor:
+    """PagedAttention decode; returns ``out`` (float32 ``[num_seqs, num_q_heads, head_dim]``)."""
+    nb, hkv, bs, d = _pool_dims(_cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"))
+    _cuda(q, "q", k_pool.dtype)
+    if q.dim() != 3 or q.shape[2] != d:
+        raise ValueError(f"q must be [num_seqs, num_q_heads, {d}]")
+    B, hq, _ = q.shape
+    _cuda(block_tables, "block_tables", torch.int32)
+    _cuda(seq_lens, "seq_lens", torch.int32)
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.numel() != B:
+        raise ValueError("block_tables must be [num_seqs, max_blocks_per_seq] and seq_lens [num_seqs]")
+    maxb = block_tables.shape[1]
+    if out is None:
+        out = torch.empty((B, hq, d), dtype=torch.float32, device=q.device)
+    else:
+        _cuda(out, "out", torch.float32)
+        if tuple(out.shape) != (B, hq, d):
+            raise ValueError("out has the wrong shape")
+    need = pkv_decode_workspace_size(B, hq, hkv, d, maxb, bs, partition_tokens)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    else:
+        _cuda(workspace, "workspace", torch.uint8)
+    check(lib().pkv_paged_attention_decode(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
+                                           block_tables.data_ptr(), seq_lens.data_ptr(), B, hq, hkv, d, nb, maxb,
+                                           bs, float(scale), _dtype_code(k_pool), partition_tokens,
+                                           workspace.data_ptr(), workspace.numel(), out.data_ptr(), _stream()))
+    return out
+
+
+def pkv_device_status(clear: bool = True) -> int:
+    """Synchronise the current stream and return the device status word."""
+    st = ctypes.c_int32(0)
+    check(lib().pkv_device_status(_stream(), ctypes.byref(st), 1 if clear else 0))
+    return st.value
+
+
+# ----------------------------------------------------------------------------
+# host block allocator
+# ----------------------------------------------------------------------------
+
+def _i64_array(ids: Sequence[int]):
+    a = np.ascontiguousarray(np.asarray(ids, dtype=np.int64))
+    return a, a.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
+
+
+class Allocator:
+    """The library's host block allocator (pkv_alloc_*): free stack, refcounts,
+    copy-on-write; every failing call leaves it unchanged."""
+
+    def __init__(self, num_blocks: int, block_size: int, free_order=None):
+        self._h = ctypes.c_void_p()
+        self.num_blocks, self.block_size = int(num_blocks), int(block_size)
+        if free_order is not None:
+            fo = np.ascontiguousarray(np.asarray(free_order, dtype=np.int32))
+            if fo.size != num_blocks:
+                raise ValueError("free_order must list every block once")
+            ptr = fo.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+        else:
+            ptr = None
+        check(lib().pkv_alloc_create(num_blocks, block_size, ptr, ctypes.byref(self._h)))
+        self._slot_buf = np.zeros(0, dtype=np.int32)
+        self._cow_buf = np.zeros(0, dtype=np.int32)
+
+    def close(self) -> None:
+        if self._h:
+            lib().pkv_alloc_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def add(self, seq_id: int, n_tokens: int) -> None:
+        check(lib().pkv_seq_add(self._h, seq_id, n_tokens))
+
+    def fork(self, parent: int, child: int) -> None:
+        check(lib().pkv_seq_fork(self._h, parent, child))
+
+    def free(self, seq_id: int) -> None:
+        check(lib().pkv_seq_free(self._h, seq_id))
+
+    def seq_len(self, seq_id: int) -> int:
+        n = ctypes.c_int32(0)
+        check(lib().pkv_seq_len(self._h, seq_id, ctypes.byref(n)))
+        return n.value
+
+    def append_slots(self, seq_ids: Sequence[int], slot_out: Optional[np.ndarray] = None):
+        """Reserve one slot per sequence; returns ``(slots int32[n], cow_pairs int32[k, 2])``."""
+        ids, ip = _i64_array(seq_ids)
+        n = ids.size
+        if slot_out is None:
+            slot_out = np.empty(n, dtype=np.int32)
+        if self._cow_buf.size < 2 * n:
+            self._cow_buf = np.empty(2 * max(n, 1), dtype=np.int32)
+        ncow = ctypes.c_int32(0)
+        check(lib().pkv_seq_append_slots(self._h, ip, n, slot_out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                         self._cow_buf.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), n,
+                                         ctypes.byref(ncow)))
+        return slot_out, self._cow_buf[: 2 * ncow.value].reshape(-1, 2).copy()
+
+    def block_tables(self, seq_ids: Sequence[int], max_blocks: int, tables_out=None, seq_lens_out=None):
+        """``(tables int32[n, max_blocks] padded with -1, seq_lens int32[n])``."""
+        ids, ip = _i64_array(seq_ids)
+        n = ids.size
+        if tables_out is None:
+            tables_out = np.empty((n, max_blocks), dtype=np.int32)
+        if seq_lens_out is None:
+            seq_lens_out = np.empty(n, dtype=np.int32)
+        check(lib().pkv_block_tables(self._h, ip, n, max_blocks,
+                                     tables_out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                     seq_lens_out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))))
+        return tables_out, seq_lens_out
+
+    def stats(self) -> dict:
+        s = N.pkv_stats_t()
+        check(lib().pkv_alloc_stats(self._h, ctypes.byref(s)))
+        return {name: getattr(s, name) for name, _ in s._fields_}
+
+
+__all__ = ["Allocator", "PagedKVError", "pkv_kv_append", "pkv_copy_blocks", "pkv_decode_workspace_size",
+           "pkv_paged_attention_decode", "pkv_device_status"]

@@ -1,0 +1,129 @@
+"""PagedKVCache: one layer's paged K/V pools on a GPU plus the host allocator,
+and the decode step that ties them together.
+
+One call of :meth:`PagedKVCache.decode_step` is the whole hot path of a decode
+step for one layer ("vLLM's 'memory paging' — PagedAttention illustrated", §3):
+
+1. slot reservation on the host (pkv_seq_append_slots): a new block when the
+   last one is full, a private copy when it is shared;
+2. one host→device copy of the step's metadata (slots, copy pairs, block
+   tables, lengths) from pinned memory;
+3. pkv_copy_blocks for the copy-on-write pairs, if any;
+4. pkv_kv_append of the new tokens' K/V;
+5. pkv_paged_attention_decode (plus its partition merge) over every sequence,
+   new token included.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+from . import binding as B
+from ._native import check, lib
+
+
+class PagedKVCache:
+    def __init__(self, num_blocks: int, num_kv_heads: int, head_dim: int, block_size: int,
+                 dtype: torch.dtype, max_blocks_per_seq: int, device="cuda", free_order=None,
+                 k_pool: Optional[torch.Tensor] = None, v_pool: Optional[torch.Tensor] = None):
+        self.device = torch.device(device)
+        self.num_blocks, self.num_kv_heads = int(num_blocks), int(num_kv_heads)
+        self.head_dim, self.block_size = int(head_dim), int(block_size)
+        self.dtype = dtype
+        self.max_blocks = int(max_blocks_per_seq)
+        shape = (num_blocks, num_kv_heads, block_size, head_dim)
+        self.k_pool = k_pool if k_pool is not None else torch.empty(shape, dtype=dtype, device=self.device)
+        self.v_pool = v_pool if v_pool is not None else torch.empty(shape, dtype=dtype, device=self.device)
+        if tuple(self.k_pool.shape) != shape or tuple(self.v_pool.shape) != shape:
+            raise ValueError(f"pools must be {shape}")
+        self.alloc = B.Allocator(num_blocks, block_size, free_order)
+        self._meta_cap = 0
+        self._ws = None
+        self._out = None
+
+    # -- sequence lifecycle (host) -----------------------------------------
+    def add(self, seq_id: int, n_tokens: int) -> None:
+        self.alloc.add(seq_id, n_tokens)
+
+    def fork(self, parent: int, child: int) -> None:
+        self.alloc.fork(parent, child)
+
+    def free(self, seq_id: int) -> None:
+        self.alloc.free(seq_id)
+
+    # -- metadata staging ----------------------------------------------------
+    def _ensure_meta(self, n: int) -> None:
+        # layout (int32): slots[n] | seq_lens[n] | cow[2n] | tables[n * max_blocks]
+        need = n * (4 + self.max_blocks)
+        if need <= self._meta_cap:
+            return
+        self._meta_host = torch.empty(need, dtype=torch.int32, pin_memory=True)
+        self._meta_dev = torch.empty(need, dtype=torch.int32, device=self.device)
+        self._meta_np = self._meta_host.numpy()
+        self._meta_cap = need
+        self._h2d_done = None
+
+    def prepare_step(self, seq_ids: Sequence[int]):
+        """Host part of a decode step: reserve slots and build the metadata
+        (numpy views into pinned memory).  Returns ``(n_cow, views)``."""
+        n = len(seq_ids)
+        self._ensure_meta(n)
+        if self._h2d_done is not None:
+            self._h2d_done.synchronize()  # the previous copy no longer reads the pinned buffer
+        m = self._meta_np
+        slots = m[:n]
+        lens = m[n:2 * n]
+        cow = m[2 * n:4 * n]
+        tables = m[4 * n:4 * n + n * self.max_blocks].reshape(n, self.max_blocks)
+        ids = np.ascontiguousarray(np.asarray(seq_ids, dtype=np.int64))
+        ip = ids.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
+        ncow = ctypes.c_int32(0)
+        i32p = lambda a: a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))  # noqa: E731
+        check(lib().pkv_seq_append_slots(self.alloc._h, ip, n, i32p(slots), i32p(cow), n, ctypes.byref(ncow)))
+        check(lib().pkv_block_tables(self.alloc._h, ip, n, self.max_blocks, i32p(tables), i32p(lens)))
+        return ncow.value, (slots, lens, cow, tables)
+
+    def upload_step(self, n: int):
+        """Copy the staged metadata to the device; returns device views."""
+        used = n * (4 + self.max_blocks)
+        self._meta_dev[:used].copy_(self._meta_host[:used], non_blocking=True)
+        ev = torch.cuda.Event()
+        ev.record()
+        self._h2d_done = ev
+        d = self._meta_dev
+        return (d[:n], d[n:2 * n], d[2 * n:4 * n], d[4 * n:4 * n + n * self.max_blocks].view(n, self.max_blocks))
+
+    def _buffers(self, n: int, num_q_heads: int, partition_tokens: int):
+        ws = B.pkv_decode_workspace_size(n, num_q_heads, self.num_kv_heads, self.head_dim, self.max_blocks,
+                                         self.block_size, partition_tokens)
+        if self._ws is None or self._ws.numel() < ws:
+            self._ws = torch.empty(ws, dtype=torch.uint8, device=self.device)
+        shape = (n, num_q_heads, self.head_dim)
+        if self._out is None or tuple(self._out.shape) != shape:
+            self._out = torch.empty(shape, dtype=torch.float32, device=self.device)
+        return self._ws, self._out
+
+    # -- the decode step -----------------------------------------------------
+    def decode_step(self, seq_ids: Sequence[int], q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                    scale: float, partition_tokens: int = 0) -> torch.Tensor:
+        """Append one token per sequence and attend over every cached token.
+
+        ``q`` [n, Hq, D], ``k_new``/``v_new`` [n, Hkv, D] in the pool dtype, on
+        the device or in (pinned) host memory.  Returns float32 [n, Hq, D] on
+        the device (valid until the next step)."""
+        n = len(seq_ids)
+        ncow, _ = self.prepare_step(seq_ids)
+        slots, lens, cow, tables = self.upload_step(n)
+        q, k_new, v_new = (t.to(self.device, non_blocking=True) for t in (q, k_new, v_new))
+        if ncow:
+            B.pkv_copy_blocks(self.k_pool, self.v_pool, cow[:2 * ncow].view(ncow, 2))
+        B.pkv_kv_append(k_new, v_new, slots, self.k_pool, self.v_pool)
+        ws, out = self._buffers(n, q.shape[1], partition_tokens)
+        return B.pkv_paged_attention_decode(q, self.k_pool, self.v_pool, tables, lens, scale, out=out,
+                                            workspace=ws, partition_tokens=partition_tokens)
+
+    def stats(self) -> dict:
+        return self.alloc.stats()

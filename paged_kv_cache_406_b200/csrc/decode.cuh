@@ -1,0 +1,534 @@
+// PagedAttention decode for sm_100a.
+//
+// What is computed ("vLLM's 'memory paging' — PagedAttention illustrated",
+// §3 phase 2): for every sequence b and query head h the kernel follows b's
+// block table, treats the scattered physical blocks as one logically
+// contiguous K and V, and returns softmax(scale · q·Kᵀ)·V, with query head h
+// reading KV head h / G (grouped-query attention, contiguous groups).
+//
+// How (B200 design, not the page's):
+//   plan kernel    one CTA turns seq_lens into a work list of partitions of
+//                  `partition_tokens` tokens, largest first;
+//   decode kernel  persistent CTAs (grid = SMs x resident CTAs) walk the list
+//                  with a stride; per work unit (sequence, partition, KV
+//                  head) a producer warp streams each block's K and V tiles
+//                  (one contiguous block_size x head_dim tile each) into a
+//                  shared-memory ring with 1-D bulk copies completing on
+//                  mbarriers; four consumer warps take every fourth block and
+//                  keep their own online softmax state (running max m, sum l,
+//                  fp32 accumulator), and merge at the end of the unit;
+//   reduce kernel  merges the per-partition (m, l, o) of sequences that were
+//                  split, with the max/sum rescaling
+//                      out = Σ_p 2^(m_p-M) o_p / Σ_p 2^(m_p-M) l_p.
+// Scores are kept in log2 units (q is pre-multiplied by scale·log2 e).  The
+// running max is only moved when a new score exceeds it by more than
+// kRescaleThreshold (2^8 headroom in fp32), which leaves the result unchanged
+// because every accumulator and sum is always taken against the same m.
+#pragma once
+
+#include "device_common.cuh"
+
+namespace pkv {
+
+constexpr int kConsumerWarps = 4;
+constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
+constexpr float kRescaleThreshold = 8.0f;
+constexpr unsigned kFull = 0xffffffffu;
+
+struct DecodeParams {
+  const void* q;
+  const void* k_pool;
+  const void* v_pool;
+  const int32_t* block_tables;
+  int32_t num_q_heads, num_kv_heads, num_blocks, max_blocks, block_size, partition_tokens, max_parts;
+  int32_t n_stages;
+  float scale_log2;
+  const int4* items;  // {b, partition, partitions of b, end token}
+  const int32_t* n_items;
+  float* part_m;
+  float* part_l;
+  float* part_o;
+  float* out;
+};
+
+// ---------------------------------------------------------------------------
+// plan: seq_lens -> work list, partitions sorted by block count, largest first
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ seq_lens, int32_t num_seqs,
+                                                    int32_t max_tokens, int32_t part_tokens, int32_t block_size,
+                                                    int4* __restrict__ items, int32_t* __restrict__ n_items) {
+  extern __shared__ int32_t hist[];  // [kmax + 1] counts, then [kmax + 1] cursors
+  const int kmax = part_tokens / block_size;
+  int32_t* cursor = hist + kmax + 1;
+  for (int i = threadIdx.x; i <= kmax; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  for (int b = threadIdx.x; b < num_seqs; b += blockDim.x) {
+    int L = seq_lens[b];
+    if (L < 0 || L > max_tokens) {
+      record_error(PKV_ERR_BAD_BLOCK);
+      L = L < 0 ? 0 : max_tokens;
+    }
+    const int nfull = L / part_tokens, rem = L % part_tokens;
+    if (nfull) atomicAdd(&hist[kmax], nfull);
+    if (rem) atomicAdd(&hist[(rem + block_size - 1) / block_size], 1);
+    if (L == 0) atomicAdd(&hist[0], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int k = kmax; k >= 0; --k) {
+      cursor[k] = run;
+      run += hist[k];
+    }
+    *n_items = run;
+  }
+  __syncthreads();
+  for (int b = threadIdx.x; b < num_seqs; b += blockDim.x) {
+    int L = seq_lens[b];
+    L = L < 0 ? 0 : (L > max_tokens ? max_tokens : L);
+    const int nfull = L / part_tokens, rem = L % part_tokens;
+    if (nfull) {
+      int pos = atomicAdd(&cursor[kmax], nfull);
+      for (int p = 0; p < nfull; ++p)
+        items[pos + p] = make_int4(b, p, nfull + (rem ? 1 : 0), (p + 1) * part_tokens);
+    }
+    if (rem) {
+      int pos = atomicAdd(&cursor[(rem + block_size - 1) / block_size], 1);
+      items[pos] = make_int4(b, nfull, nfull + 1, L);
+    }
+    if (L == 0) {
+      int pos = atomicAdd(&cursor[0], 1);
+      items[pos] = make_int4(b, 0, 1, 0);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// cross-lane helpers within a group of 8 lanes that share one token row
+// ---------------------------------------------------------------------------
+
+// Sums G per-lane partial dot products over the 8 lanes of a token group and
+// leaves each lane with the full score of one head, head_of<G>(r8).
+template <int G>
+__device__ __forceinline__ float reduce_scatter(const float (&v)[G], int r8) {
+  if constexpr (G == 1) {
+    float x = v[0];
+    x += __shfl_xor_sync(kFull, x, 4);
+    x += __shfl_xor_sync(kFull, x, 2);
+    x += __shfl_xor_sync(kFull, x, 1);
+    return x;
+  } else if constexpr (G == 2) {
+    const bool u4 = r8 & 4;
+    float x = (u4 ? v[1] : v[0]) + __shfl_xor_sync(kFull, u4 ? v[0] : v[1], 4);
+    x += __shfl_xor_sync(kFull, x, 2);
+    x += __shfl_xor_sync(kFull, x, 1);
+    return x;
+  } else {
+    static_assert(G == 4, "group size");
+    const bool u4 = r8 & 4, u2 = r8 & 2;
+    float a0 = (u4 ? v[2] : v[0]) + __shfl_xor_sync(kFull, u4 ? v[0] : v[2], 4);
+    float a1 = (u4 ? v[3] : v[1]) + __shfl_xor_sync(kFull, u4 ? v[1] : v[3], 4);
+    float x = (u2 ? a1 : a0) + __shfl_xor_sync(kFull, u2 ? a0 : a1, 2);
+    x += __shfl_xor_sync(kFull, x, 1);
+    return x;
+  }
+}
+
+template <int G>
+__device__ __forceinline__ int head_of(int r8) {
+  if constexpr (G == 1) return 0;
+  else if constexpr (G == 2) return (r8 >> 2) & 1;
+  else return ((r8 >> 2) & 1) * 2 + ((r8 >> 1) & 1);
+}
+
+// The lane of each head that writes per-head values (one per duplicate set).
+template <int G>
+__device__ __forceinline__ bool head_writer(int r8) {
+  if constexpr (G == 1) return r8 == 0;
+  else if constexpr (G == 2) return (r8 & 3) == 0;
+  else return (r8 & 1) == 0;
+}
+
+// Inverse of reduce_scatter's layout: every lane of the token group ends with
+// all G values, out[h] = value held by the lanes of head h.
+template <int G>
+__device__ __forceinline__ void all_gather(float x, float (&out)[G], int r8) {
+  if constexpr (G == 1) {
+    out[0] = x;
+  } else if constexpr (G == 2) {
+    const bool u4 = r8 & 4;
+    float y = __shfl_xor_sync(kFull, x, 4);
+    out[0] = u4 ? y : x;
+    out[1] = u4 ? x : y;
+  } else {
+    const bool u4 = r8 & 4, u2 = r8 & 2;
+    float y = __shfl_xor_sync(kFull, x, 2);
+    float lo = u2 ? y : x, hi = u2 ? x : y;
+    float y0 = __shfl_xor_sync(kFull, lo, 4);
+    float y1 = __shfl_xor_sync(kFull, hi, 4);
+    out[0] = u4 ? y0 : lo;
+    out[1] = u4 ? y1 : hi;
+    out[2] = u4 ? lo : y0;
+    out[3] = u4 ? hi : y1;
+  }
+}
+
+// v[head_of<G>(r8)] without dynamic register indexing.
+template <int G>
+__device__ __forceinline__ float pick(const float (&v)[G], int r8) {
+  if constexpr (G == 1) return v[0];
+  else if constexpr (G == 2) return (r8 & 4) ? v[1] : v[0];
+  else {
+    const bool u4 = r8 & 4, u2 = r8 & 2;
+    return u4 ? (u2 ? v[3] : v[2]) : (u2 ? v[1] : v[0]);
+  }
+}
+
+struct WorkUnit {
+  int b, part, nparts, t0, t1, g, nblk;
+};
+
+__device__ __forceinline__ WorkUnit load_unit(const DecodeParams& p, int w) {
+  WorkUnit u;
+  const int idx = w / p.num_kv_heads;
+  u.g = w - idx * p.num_kv_heads;
+  const int4 it = p.items[idx];
+  u.b = it.x;
+  u.part = it.y;
+  u.nparts = it.z;
+  u.t0 = it.y * p.partition_tokens;
+  u.t1 = it.w;
+  u.nblk = (u.t1 - u.t0 + p.block_size - 1) / p.block_size;
+  return u;
+}
+
+// Shared memory: [n_stages][K tile | V tile] ring, 2 x kConsumerWarps merge
+// records, full/empty mbarriers, abort flag.
+template <typename T, int D, int G>
+struct DecodeSmem {
+  static constexpr int kMergeFloats = G * D + 2 * G;  // acc[G][D], m[G], l[G]
+  __host__ __device__ static size_t ring_bytes(int bs, int ns) { return size_t(ns) * 2 * bs * D * sizeof(T); }
+  __host__ __device__ static size_t bytes(int bs, int ns) {
+    return ring_bytes(bs, ns) + 2 * kConsumerWarps * kMergeFloats * sizeof(float) + 2 * ns * sizeof(uint64_t) + 16;
+  }
+};
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeParams p) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  constexpr int kVec = Elem<T>::kVec;       // elements per 16-byte chunk
+  constexpr int kChunksPerLane = D / kVec / 8;  // 8 lanes cover one token row
+  constexpr int kPairs = kChunksPerLane * kVec / 2;  // fp32 pairs per lane
+  constexpr int kMF = DecodeSmem<T, D, G>::kMergeFloats;
+  static_assert(kChunksPerLane >= 1, "head_dim too small");
+
+  const int BS = p.block_size;
+  const int NS = p.n_stages;
+  const uint32_t tile_bytes = BS * D * sizeof(T);
+  const uint32_t stage_bytes = 2 * tile_bytes;
+  float* merge = reinterpret_cast<float*>(smem + DecodeSmem<T, D, G>::ring_bytes(BS, NS));
+  uint64_t* full = reinterpret_cast<uint64_t*>(merge + 2 * kConsumerWarps * kMF);
+  uint64_t* empty = full + NS;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + NS);
+  const uint32_t ring_s = smem_addr(smem);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(smem_addr(full + s), 1);
+      mbar_init(smem_addr(empty + s), 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const int n_work = *p.n_items * p.num_kv_heads;
+  const int Hq = p.num_q_heads;
+
+  if (warp == kConsumerWarps) {
+    // ----------------------------- producer -----------------------------
+    const uint64_t policy = l2_evict_first_policy();
+    const unsigned char* kbase = static_cast<const unsigned char*>(p.k_pool);
+    const unsigned char* vbase = static_cast<const unsigned char*>(p.v_pool);
+    uint32_t c = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < n_work && ok; w += gridDim.x) {
+      const WorkUnit u = load_unit(p, w);
+      const int32_t* trow = p.block_tables + static_cast<int64_t>(u.b) * p.max_blocks + u.t0 / BS;
+      for (int jb = 0; jb < u.nblk && ok; jb += 32) {
+        const int cnt = min(32, u.nblk - jb);
+        const int mine = lane < cnt ? trow[jb + lane] : 0;
+        for (int j = 0; j < cnt; ++j, ++c) {
+          int phys = __shfl_sync(kFull, mine, j);
+          if (lane == 0) {
+            const int s = c % NS;
+            const uint32_t r = c / NS;
+            ok = mbar_wait(smem_addr(empty + s), (r & 1) ^ 1, abort_flag);
+            if (ok) {
+              if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_blocks)) {
+                record_error(PKV_ERR_BAD_BLOCK);
+                phys = 0;
+              }
+              const size_t off = (static_cast<size_t>(phys) * p.num_kv_heads + u.g) * tile_bytes;
+              const uint32_t bar = smem_addr(full + s);
+              mbar_arrive_expect_tx(bar, stage_bytes);
+              bulk_g2s(ring_s + s * stage_bytes, kbase + off, tile_bytes, bar, policy);
+              bulk_g2s(ring_s + s * stage_bytes + tile_bytes, vbase + off, tile_bytes, bar, policy);
+            } else {
+              record_error(PKV_ERR_DEVICE_TIMEOUT);
+              *abort_flag = 1;
+            }
+          }
+          ok = __shfl_sync(kFull, ok, 0);
+          if (!ok) break;
+        }
+      }
+    }
+    // Before the CTA exits no copy may still be landing in its shared memory:
+    // wait (bounded) for the last copy issued into every stage.
+    __syncwarp();
+    if (lane == 0) {
+      const uint32_t issued = c;  // blocks issued (a failed wait issued nothing)
+      for (int s = 0; s < NS && s < static_cast<int>(issued); ++s) {
+        const uint32_t last_round = (issued - 1 - s) / NS;
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(smem_addr(full + s), last_round & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+    return;
+  }
+
+  // ------------------------------ consumers ------------------------------
+  const int r8 = lane & 7, tg = lane >> 3;
+  const int hs = head_of<G>(r8);
+  const bool writer = head_writer<G>(r8);
+  uint32_t c = 0;
+  int iter = 0;
+  bool ok = true;
+  for (int w = blockIdx.x; w < n_work; w += gridDim.x, ++iter) {
+    const WorkUnit u = load_unit(p, w);
+
+    // q rows of this KV head's G query heads, my dims, scaled to log2 units
+    float2 q2[G][kPairs];
+    {
+      const T* qrow = static_cast<const T*>(p.q) + (static_cast<int64_t>(u.b) * Hq + u.g * G) * D;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+#pragma unroll
+        for (int i = 0; i < kChunksPerLane; ++i) {
+          const uint4 raw = __ldg(reinterpret_cast<const uint4*>(qrow + h * D + (r8 + 8 * i) * kVec));
+          float2 f[kVec / 2];
+          Elem<T>::widen(raw, f);
+#pragma unroll
+          for (int e = 0; e < kVec / 2; ++e)
+            q2[h][i * kVec / 2 + e] = make_float2(f[e].x * p.scale_log2, f[e].y * p.scale_log2);
+        }
+      }
+    }
+
+    float m[G];
+    float2 acc[G][kPairs];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      m[h] = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < kPairs; ++e) acc[h][e] = make_float2(0.f, 0.f);
+    }
+    float m_own = -INFINITY, l_own = 0.f;
+
+    const int j0 = (warp - static_cast<int>(c % kConsumerWarps) + kConsumerWarps) % kConsumerWarps;
+    for (int j = j0; j < u.nblk && ok; j += kConsumerWarps) {
+      const uint32_t cc = c + j;
+      const int s = cc % NS;
+      const bool landed = __all_sync(kFull, mbar_wait(smem_addr(full + s), (cc / NS) & 1, abort_flag));
+      if (!landed) {
+        if (lane == 0) {
+          record_error(PKV_ERR_DEVICE_TIMEOUT);
+          *abort_flag = 1;
+        }
+        ok = false;
+        break;
+      }
+      const unsigned char* ks = smem + s * stage_bytes;
+      const unsigned char* vs = ks + tile_bytes;
+      const int nv = min(BS, u.t1 - (u.t0 + j * BS));
+      const int nrows = (nv + 3) >> 2;
+      for (int rr = 0; rr < nrows; ++rr) {
+        const int tt = rr * 4 + tg;
+        const bool valid = tt < nv;
+        const unsigned char* krow = ks + tt * (D * sizeof(T));
+        float part[G];
+        {
+          float2 pp[G];
+#pragma unroll
+          for (int h = 0; h < G; ++h) pp[h] = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int i = 0; i < kChunksPerLane; ++i) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(krow + (r8 + 8 * i) * 16);
+            float2 kf[kVec / 2];
+            Elem<T>::widen(raw, kf);
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+#pragma unroll
+              for (int e = 0; e < kVec / 2; ++e) pp[h] = __ffma2_rn(q2[h][i * kVec / 2 + e], kf[e], pp[h]);
+          }
+#pragma unroll
+          for (int h = 0; h < G; ++h) part[h] = pp[h].x + pp[h].y;
+        }
+        float s_own = reduce_scatter<G>(part, r8);
+        s_own = valid ? s_own : -INFINITY;
+
+        if (__any_sync(kFull, s_own > m_own + kRescaleThreshold)) {
+          float mx = s_own;
+          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+          float mall[G], fac[G];
+          all_gather<G>(mx, mall, r8);
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float mn = fmaxf(m[h], mall[h]);
+            fac[h] = (mn == -INFINITY) ? 1.f : fast_exp2(m[h] - mn);
+            m[h] = mn;
+#pragma unroll
+            for (int e = 0; e < kPairs; ++e) acc[h][e] = __fmul2_rn(acc[h][e], make_float2(fac[h], fac[h]));
+          }
+          l_own *= pick<G>(fac, r8);
+          m_own = pick<G>(m, r8);
+        }
+        const float p_own = fast_exp2(s_own - m_own);
+        l_own += p_own;
+        float pv[G];
+        all_gather<G>(p_own, pv, r8);
+        if (valid) {
+          const unsigned char* vrow = vs + tt * (D * sizeof(T));
+#pragma unroll
+          for (int i = 0; i < kChunksPerLane; ++i) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(vrow + (r8 + 8 * i) * 16);
+            float2 vf[kVec / 2];
+            Elem<T>::widen(raw, vf);
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+#pragma unroll
+              for (int e = 0; e < kVec / 2; ++e)
+                acc[h][i * kVec / 2 + e] = __ffma2_rn(make_float2(pv[h], pv[h]), vf[e], acc[h][i * kVec / 2 + e]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(empty + s));
+    }
+    c += u.nblk;
+
+    // ---- merge the 4 token groups of this warp, then the 4 warps ----
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int e = 0; e < kPairs; ++e) {
+        acc[h][e].x += __shfl_xor_sync(kFull, acc[h][e].x, 8);
+        acc[h][e].y += __shfl_xor_sync(kFull, acc[h][e].y, 8);
+        acc[h][e].x += __shfl_xor_sync(kFull, acc[h][e].x, 16);
+        acc[h][e].y += __shfl_xor_sync(kFull, acc[h][e].y, 16);
+      }
+    l_own += __shfl_xor_sync(kFull, l_own, 8);
+    l_own += __shfl_xor_sync(kFull, l_own, 16);
+
+    float* mb = merge + ((iter & 1) * kConsumerWarps + warp) * kMF;
+    if (tg == 0) {
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int i = 0; i < kChunksPerLane; ++i)
+#pragma unroll
+          for (int e = 0; e < kVec / 2; ++e)
+            *reinterpret_cast<float2*>(mb + h * D + (r8 + 8 * i) * kVec + 2 * e) = acc[h][i * kVec / 2 + e];
+      if (writer) mb[G * D + G + hs] = l_own;
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) mb[G * D + h] = m[h];
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+
+    const float* m0 = merge + (iter & 1) * kConsumerWarps * kMF;
+    const bool single = u.nparts == 1;
+    for (int idx = threadIdx.x; idx < G * D; idx += kConsumerWarps * 32) {
+      const int h = idx / D, d = idx - h * D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w2 = 0; w2 < kConsumerWarps; ++w2) M = fmaxf(M, m0[w2 * kMF + G * D + h]);
+      float num = 0.f, den = 0.f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int w2 = 0; w2 < kConsumerWarps; ++w2) {
+          const float f = fast_exp2(m0[w2 * kMF + G * D + h] - M);
+          num += f * m0[w2 * kMF + h * D + d];
+          den += f * m0[w2 * kMF + G * D + G + h];
+        }
+      }
+      const int64_t row = static_cast<int64_t>(u.b) * Hq + u.g * G + h;
+      if (single) {
+        p.out[row * D + d] = den > 0.f ? num / den : 0.f;
+      } else {
+        const int64_t pr = row * p.max_parts + u.part;
+        p.part_o[pr * D + d] = num;
+        if (d == 0) {
+          p.part_m[pr] = M;
+          p.part_l[pr] = den;
+        }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// reduce: merge the partitions of split sequences; one warp per (seq, q head)
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) reduce_kernel(const int32_t* __restrict__ seq_lens, int32_t num_seqs,
+                                                     int32_t num_q_heads, int32_t max_tokens, int32_t part_tokens,
+                                                     int32_t max_parts, const float* __restrict__ part_m,
+                                                     const float* __restrict__ part_l,
+                                                     const float* __restrict__ part_o, float* __restrict__ out) {
+  constexpr int kPer = D / 32;
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= num_seqs * num_q_heads) return;
+  const int b = row / num_q_heads;
+  int L = seq_lens[b];
+  L = L < 0 ? 0 : (L > max_tokens ? max_tokens : L);
+  if (L <= part_tokens) return;  // written directly by the decode kernel
+  const int np = (L + part_tokens - 1) / part_tokens;
+  const int64_t base = static_cast<int64_t>(row) * max_parts;
+  float M = -INFINITY;
+  for (int p = lane; p < np; p += 32) M = fmaxf(M, part_m[base + p]);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+  float num[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) num[i] = 0.f;
+  float den = 0.f;
+  for (int p = 0; p < np; ++p) {
+    const float f = fast_exp2(part_m[base + p] - M);
+    den += f * part_l[base + p];
+    const float* o = part_o + (base + p) * D + lane * kPer;
+    if constexpr (kPer == 4) {
+      const float4 v = *reinterpret_cast<const float4*>(o);
+      num[0] += f * v.x;
+      num[1] += f * v.y;
+      num[2] += f * v.z;
+      num[3] += f * v.w;
+    } else {
+      const float2 v = *reinterpret_cast<const float2*>(o);
+      num[0] += f * v.x;
+      num[1] += f * v.y;
+    }
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  float* dst = out + static_cast<int64_t>(row) * D + lane * kPer;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) dst[i] = num[i] * inv;
+}
+
+}  // namespace pkv

@@ -1,0 +1,336 @@
+// Device entry points of libpagedkv (sm_100a): KV append, block copy,
+// PagedAttention decode (plan + decode + reduce) and the device status word.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+
+#include "decode.cuh"
+#include "device_common.cuh"
+#include "pkv_internal.h"
+
+namespace pkv {
+
+// ---------------------------------------------------------------------------
+// KV append: one thread per 16-byte chunk of one (token, kv head) row, K and V.
+// vLLM paging page §3 phase 1: the new token is written into its slot.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) kv_append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+                                                        const int32_t* __restrict__ slots, int64_t n_chunks,
+                                                        uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
+                                                        int32_t num_blocks, int32_t num_kv_heads, int32_t row_chunks,
+                                                        int32_t block_size) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n_chunks) return;
+  const int32_t chunk = static_cast<int32_t>(i % row_chunks);
+  const int64_t row = i / row_chunks;  // token * num_kv_heads + head
+  const int32_t h = static_cast<int32_t>(row % num_kv_heads);
+  const int64_t tok = row / num_kv_heads;
+  const int32_t slot = slots[tok];
+  if (slot < 0) return;  // padding token
+  const int32_t blk = slot / block_size, off = slot - blk * block_size;
+  if (blk >= num_blocks) {
+    if (chunk == 0 && h == 0) record_error(PKV_ERR_BAD_BLOCK);
+    return;
+  }
+  const int64_t dst = ((static_cast<int64_t>(blk) * num_kv_heads + h) * block_size + off) * row_chunks + chunk;
+  k_pool[dst] = k_new[i];
+  v_pool[dst] = v_new[i];
+}
+
+// ---------------------------------------------------------------------------
+// Block copy for copy-on-write (vLLM paging page §3 phase 3): pair y copies
+// one whole block of K and of V, every head and offset.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
+                                                          const int32_t* __restrict__ pairs, int32_t num_blocks,
+                                                          int64_t block_chunks) {
+  const int32_t src = pairs[2 * blockIdx.y], dst = pairs[2 * blockIdx.y + 1];
+  if (static_cast<unsigned>(src) >= static_cast<unsigned>(num_blocks) ||
+      static_cast<unsigned>(dst) >= static_cast<unsigned>(num_blocks)) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) record_error(PKV_ERR_BAD_BLOCK);
+    return;
+  }
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < block_chunks;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    k_pool[dst * block_chunks + i] = k_pool[src * block_chunks + i];
+    v_pool[dst * block_chunks + i] = v_pool[src * block_chunks + i];
+  }
+}
+
+}  // namespace pkv
+
+// ===========================================================================
+// host side
+// ===========================================================================
+namespace {
+
+using pkv::fail;
+
+constexpr int kMaxDevices = 64;
+constexpr int kAutoPartitionTokens = 256;
+constexpr int kMaxPartitionTokens = 8192;
+
+size_t elem_size(int dtype) { return dtype == PKV_F32 ? 4 : 2; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(PKV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int check_common(int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t dtype, const char* fn) {
+  if (dtype != PKV_F32 && dtype != PKV_BF16 && dtype != PKV_F16)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: dtype %d not supported", fn, dtype);
+  if (head_dim != 64 && head_dim != 128)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: head_dim %d not supported (64 or 128)", fn, head_dim);
+  if (block_size != 8 && block_size != 16 && block_size != 32)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: block_size %d not supported (8, 16 or 32)", fn, block_size);
+  if (num_kv_heads <= 0) return fail(PKV_ERR_INVALID_ARG, "%s: num_kv_heads %d <= 0", fn, num_kv_heads);
+  return PKV_OK;
+}
+
+int sm_count(int dev) {
+  static std::atomic<int> cache[kMaxDevices];
+  if (dev < kMaxDevices) {
+    int v = cache[dev].load(std::memory_order_relaxed);
+    if (v) return v;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev < kMaxDevices) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+int resolve_partition(int32_t partition_tokens, int32_t block_size, int32_t* out) {
+  int32_t pt = partition_tokens == 0 ? kAutoPartitionTokens : partition_tokens;
+  if (pt < block_size || pt % block_size != 0 || pt > kMaxPartitionTokens)
+    return fail(PKV_ERR_INVALID_ARG,
+                "partition_tokens %d must be a positive multiple of block_size %d and at most %d",
+                partition_tokens, block_size, kMaxPartitionTokens);
+  *out = pt;
+  return PKV_OK;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct WsLayout {
+  int32_t max_parts;
+  size_t items, m, l, o, total;  // byte offsets; n_items lives at offset 0
+};
+
+WsLayout ws_layout(int64_t num_seqs, int64_t num_q_heads, int64_t head_dim, int64_t max_tokens, int32_t pt) {
+  WsLayout w;
+  w.max_parts = static_cast<int32_t>(std::max<int64_t>(1, (max_tokens + pt - 1) / pt));
+  const int64_t rows = num_seqs * num_q_heads * w.max_parts;
+  w.items = 256;
+  w.m = w.items + round256(num_seqs * w.max_parts * sizeof(int4));
+  w.l = w.m + round256(rows * sizeof(float));
+  w.o = w.l + round256(rows * sizeof(float));
+  w.total = w.o + round256(rows * head_dim * sizeof(float));
+  return w;
+}
+
+int ring_stages(size_t stage_bytes) {
+  // about 64 KB of K/V in flight per CTA; a multiple of the consumer warps
+  int ns = static_cast<int>((64 * 1024) / stage_bytes);
+  ns = std::max(pkv::kConsumerWarps, std::min(16, ns));
+  return ns - ns % pkv::kConsumerWarps;
+}
+
+template <typename T, int D, int G>
+int launch_decode(const pkv::DecodeParams& base, const int32_t* seq_lens, int32_t num_seqs, int32_t max_tokens,
+                  cudaStream_t stream) {
+  pkv::DecodeParams p = base;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  p.n_stages = ring_stages(size_t(2) * p.block_size * D * sizeof(T));
+  const size_t smem = pkv::DecodeSmem<T, D, G>::bytes(p.block_size, p.n_stages);
+  auto kern = pkv::decode_kernel<T, D, G>;
+
+  // per device: opt in to the largest dynamic shared memory any block size
+  // needs (once), then cache resident CTAs per SM for this block size
+  static std::atomic<int> occ_cache[kMaxDevices][3];
+  const int bs_idx = p.block_size == 8 ? 0 : (p.block_size == 16 ? 1 : 2);
+  int occ = dev < kMaxDevices ? occ_cache[dev][bs_idx].load(std::memory_order_relaxed) : 0;
+  if (occ == 0) {
+    size_t smem_max = 0;
+    for (int bs : {8, 16, 32})
+      smem_max = std::max(smem_max, pkv::DecodeSmem<T, D, G>::bytes(bs, ring_stages(size_t(2) * bs * D * sizeof(T))));
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_max));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, pkv::kDecodeThreads, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    if (occ <= 0) return fail(PKV_ERR_CUDA, "decode kernel does not fit on an SM (smem %zu)", smem);
+    if (dev < kMaxDevices) occ_cache[dev][bs_idx].store(occ, std::memory_order_relaxed);
+  }
+
+  const int kmax = p.partition_tokens / p.block_size;
+  pkv::plan_kernel<<<1, 1024, 2 * (kmax + 1) * sizeof(int32_t), stream>>>(
+      seq_lens, num_seqs, max_tokens, p.partition_tokens, p.block_size, const_cast<int4*>(p.items),
+      const_cast<int32_t*>(p.n_items));
+  const int64_t work_upper = int64_t(num_seqs) * p.max_parts * p.num_kv_heads;
+  const int grid = static_cast<int>(std::min<int64_t>(int64_t(sm_count(dev)) * occ, work_upper));
+  kern<<<grid, pkv::kDecodeThreads, smem, stream>>>(p);
+  if (p.max_parts > 1) {
+    const int rows = num_seqs * p.num_q_heads;
+    pkv::reduce_kernel<D><<<(rows + 7) / 8, 256, 0, stream>>>(seq_lens, num_seqs, p.num_q_heads, max_tokens,
+                                                              p.partition_tokens, p.max_parts, p.part_m, p.part_l,
+                                                              p.part_o, p.out);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return pkv::ok();
+}
+
+template <typename T>
+int dispatch_decode(int32_t head_dim, int32_t group, const pkv::DecodeParams& p, const int32_t* seq_lens,
+                    int32_t num_seqs, int32_t max_tokens, cudaStream_t s) {
+  if (head_dim == 128) {
+    if (group == 1) return launch_decode<T, 128, 1>(p, seq_lens, num_seqs, max_tokens, s);
+    if (group == 2) return launch_decode<T, 128, 2>(p, seq_lens, num_seqs, max_tokens, s);
+    return launch_decode<T, 128, 4>(p, seq_lens, num_seqs, max_tokens, s);
+  }
+  if (group == 1) return launch_decode<T, 64, 1>(p, seq_lens, num_seqs, max_tokens, s);
+  if (group == 2) return launch_decode<T, 64, 2>(p, seq_lens, num_seqs, max_tokens, s);
+  return launch_decode<T, 64, 4>(p, seq_lens, num_seqs, max_tokens, s);
+}
+
+}  // namespace
+
+extern "C" int pkv_kv_append(const void* k_new, const void* v_new, const int32_t* slot_mapping, int32_t n_tokens,
+                             void* k_pool, void* v_pool, int32_t num_blocks, int32_t num_kv_heads,
+                             int32_t head_dim, int32_t block_size, int32_t dtype, void* stream) {
+  int rc = check_common(num_kv_heads, head_dim, block_size, dtype, "pkv_kv_append");
+  if (rc) return rc;
+  if (n_tokens < 0 || num_blocks <= 0) return fail(PKV_ERR_INVALID_ARG, "pkv_kv_append: n_tokens/num_blocks");
+  if (n_tokens == 0) return pkv::ok();
+  if (!k_new || !v_new || !slot_mapping || !k_pool || !v_pool)
+    return fail(PKV_ERR_INVALID_ARG, "pkv_kv_append: NULL pointer");
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pool) || !aligned16(v_pool))
+    return fail(PKV_ERR_INVALID_ARG, "pkv_kv_append: K/V buffers must be 16-byte aligned");
+  const int32_t row_chunks = static_cast<int32_t>(head_dim * elem_size(dtype) / 16);
+  const int64_t n_chunks = int64_t(n_tokens) * num_kv_heads * row_chunks;
+  const int64_t blocks = (n_chunks + 255) / 256;
+  pkv::kv_append_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), slot_mapping, n_chunks,
+      static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), num_blocks, num_kv_heads, row_chunks, block_size);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pkv_kv_append launch");
+  return pkv::ok();
+}
+
+extern "C" int pkv_copy_blocks(void* k_pool, void* v_pool, const int32_t* block_pairs, int32_t n_pairs,
+                               int32_t num_blocks, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                               int32_t dtype, void* stream) {
+  int rc = check_common(num_kv_heads, head_dim, block_size, dtype, "pkv_copy_blocks");
+  if (rc) return rc;
+  if (n_pairs < 0 || num_blocks <= 0) return fail(PKV_ERR_INVALID_ARG, "pkv_copy_blocks: n_pairs/num_blocks");
+  if (n_pairs == 0) return pkv::ok();
+  if (n_pairs > 65535) return fail(PKV_ERR_INVALID_ARG, "pkv_copy_blocks: at most 65535 pairs per call");
+  if (!k_pool || !v_pool || !block_pairs) return fail(PKV_ERR_INVALID_ARG, "pkv_copy_blocks: NULL pointer");
+  if (!aligned16(k_pool) || !aligned16(v_pool))
+    return fail(PKV_ERR_INVALID_ARG, "pkv_copy_blocks: pools must be 16-byte aligned");
+  const int64_t block_chunks = int64_t(num_kv_heads) * block_size * head_dim * elem_size(dtype) / 16;
+  const int64_t xb = std::min<int64_t>((block_chunks + 255) / 256, 64);
+  dim3 grid(static_cast<unsigned>(xb), static_cast<unsigned>(n_pairs));
+  pkv::copy_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), block_pairs, num_blocks, block_chunks);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pkv_copy_blocks launch");
+  return pkv::ok();
+}
+
+extern "C" int pkv_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                         int32_t head_dim, int32_t max_blocks_per_seq, int32_t block_size,
+                                         int32_t partition_tokens, size_t* bytes) {
+  if (!bytes) return fail(PKV_ERR_INVALID_ARG, "pkv_decode_workspace_size: bytes is NULL");
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_blocks_per_seq < 0 ||
+      block_size <= 0)
+    return fail(PKV_ERR_INVALID_ARG, "pkv_decode_workspace_size: bad sizes");
+  int32_t pt = 0;
+  int rc = resolve_partition(partition_tokens, block_size, &pt);
+  if (rc) return rc;
+  *bytes = ws_layout(num_seqs, num_q_heads, head_dim, int64_t(max_blocks_per_seq) * block_size, pt).total;
+  return pkv::ok();
+}
+
+extern "C" int pkv_paged_attention_decode(const void* q, const void* k_pool, const void* v_pool,
+                                          const int32_t* block_tables, const int32_t* seq_lens, int32_t num_seqs,
+                                          int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                          int32_t num_blocks, int32_t max_blocks_per_seq, int32_t block_size,
+                                          float scale, int32_t dtype, int32_t partition_tokens, void* workspace,
+                                          size_t workspace_bytes, float* out, void* stream) {
+  const char* fn = "pkv_paged_attention_decode";
+  int rc = check_common(num_kv_heads, head_dim, block_size, dtype, fn);
+  if (rc) return rc;
+  if (num_seqs < 0 || num_q_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq < 0)
+    return fail(PKV_ERR_INVALID_ARG, "%s: bad sizes", fn);
+  if (num_q_heads % num_kv_heads != 0)
+    return fail(PKV_ERR_INVALID_ARG, "%s: num_q_heads %d not a multiple of num_kv_heads %d", fn, num_q_heads,
+                num_kv_heads);
+  const int32_t group = num_q_heads / num_kv_heads;
+  if (group != 1 && group != 2 && group != 4)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: group size %d not supported (1, 2 or 4)", fn, group);
+  if (!std::isfinite(scale)) return fail(PKV_ERR_INVALID_ARG, "%s: scale is not finite", fn);
+  int32_t pt = 0;
+  rc = resolve_partition(partition_tokens, block_size, &pt);
+  if (rc) return rc;
+  if (num_seqs == 0) return pkv::ok();
+  if (!q || !k_pool || !v_pool || !block_tables || !seq_lens || !workspace || !out)
+    return fail(PKV_ERR_INVALID_ARG, "%s: NULL pointer", fn);
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out))
+    return fail(PKV_ERR_INVALID_ARG, "%s: q, pools and out must be 16-byte aligned", fn);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(PKV_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", fn);
+  const int64_t max_tokens = int64_t(max_blocks_per_seq) * block_size;
+  if (max_tokens > (int64_t(1) << 30)) return fail(PKV_ERR_INVALID_ARG, "%s: max_blocks_per_seq too large", fn);
+  const WsLayout w = ws_layout(num_seqs, num_q_heads, head_dim, max_tokens, pt);
+  if (workspace_bytes < w.total)
+    return fail(PKV_ERR_INVALID_ARG, "%s: workspace %zu bytes < %zu needed", fn, workspace_bytes, w.total);
+
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  pkv::DecodeParams p{};
+  p.q = q;
+  p.k_pool = k_pool;
+  p.v_pool = v_pool;
+  p.block_tables = block_tables;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.num_blocks = num_blocks;
+  p.max_blocks = max_blocks_per_seq;
+  p.block_size = block_size;
+  p.partition_tokens = pt;
+  p.max_parts = w.max_parts;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.items = reinterpret_cast<const int4*>(ws + w.items);
+  p.n_items = reinterpret_cast<const int32_t*>(ws);
+  p.part_m = reinterpret_cast<float*>(ws + w.m);
+  p.part_l = reinterpret_cast<float*>(ws + w.l);
+  p.part_o = reinterpret_cast<float*>(ws + w.o);
+  p.out = out;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int32_t mt = static_cast<int32_t>(max_tokens);
+  switch (dtype) {
+    case PKV_F32: return dispatch_decode<float>(head_dim, group, p, seq_lens, num_seqs, mt, s);
+    case PKV_BF16: return dispatch_decode<__nv_bfloat16>(head_dim, group, p, seq_lens, num_seqs, mt, s);
+    default: return dispatch_decode<__half>(head_dim, group, p, seq_lens, num_seqs, mt, s);
+  }
+}
+
+extern "C" int pkv_device_status(void* stream, int32_t* status, int32_t clear) {
+  if (!status) return fail(PKV_ERR_INVALID_ARG, "pkv_device_status: status is NULL");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "pkv_device_status: cudaStreamSynchronize");
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, pkv::g_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "pkv_device_status: read");
+  if (clear) {
+    const int zero = PKV_OK;
+    e = cudaMemcpyToSymbol(pkv::g_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "pkv_device_status: clear");
+  }
+  *status = v;
+  return pkv::ok();
+}

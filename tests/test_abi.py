@@ -1,0 +1,110 @@
+"""The C-ABI library loads, exports every entry point the header declares,
+and rejects bad arguments on the host before anything is launched (CPU only:
+no call here reaches a kernel launch)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_406_b200 import _native as N
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "paged_kv.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pkv_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_documented_entry_points():
+    names = declared_functions()
+    for must in ("pkv_kv_append", "pkv_paged_attention_decode", "pkv_copy_blocks", "pkv_alloc_create",
+                 "pkv_seq_append_slots", "pkv_seq_free", "pkv_seq_fork", "pkv_decode_workspace_size"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(native):
+    for name in declared_functions():
+        assert hasattr(native, name), f"{name} declared in include/paged_kv.h but not exported"
+        assert name in N.SIGNATURES, f"{name} has no binding signature"
+
+
+def test_version_and_error_string(native):
+    assert native.pkv_version().decode() == "1.0.0"
+    rc = native.pkv_alloc_create(0, 16, None, ctypes.byref(ctypes.c_void_p()))
+    assert rc == N.PKV_ERR_INVALID_ARG
+    assert b"num_blocks" in native.pkv_last_error_string()
+
+
+def _ws(native, *args):
+    out = ctypes.c_size_t(0)
+    rc = native.pkv_decode_workspace_size(*args, ctypes.byref(out))
+    return rc, out.value
+
+
+def test_workspace_size_host_only(native):
+    rc, a = _ws(native, 64, 32, 8, 128, 257, 16, 0)
+    assert rc == 0 and a > 0
+    rc, b = _ws(native, 64, 32, 8, 128, 257, 16, 512)
+    assert rc == 0 and b < a  # fewer partitions, smaller partials
+    rc, _ = _ws(native, 64, 32, 8, 128, 257, 16, 100)  # not a multiple of the block size
+    assert rc == N.PKV_ERR_INVALID_ARG
+    rc, _ = _ws(native, -1, 32, 8, 128, 257, 16, 0)
+    assert rc == N.PKV_ERR_INVALID_ARG
+
+
+FAKE = 1 << 20  # an aligned non-null address; every call below fails validation before using it
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=7), N.PKV_ERR_UNSUPPORTED),
+    (dict(head_dim=96), N.PKV_ERR_UNSUPPORTED),
+    (dict(block_size=12), N.PKV_ERR_UNSUPPORTED),
+    (dict(hq=24, hkv=8), N.PKV_ERR_UNSUPPORTED),        # group size 3
+    (dict(hq=30, hkv=8), N.PKV_ERR_INVALID_ARG),        # not a multiple
+    (dict(pt=100), N.PKV_ERR_INVALID_ARG),
+    (dict(ws_bytes=16), N.PKV_ERR_INVALID_ARG),         # workspace too small
+    (dict(q=FAKE + 4), N.PKV_ERR_INVALID_ARG),          # misaligned q
+    (dict(ws=FAKE + 16), N.PKV_ERR_INVALID_ARG),        # workspace not 256-aligned
+    (dict(q=0), N.PKV_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), N.PKV_ERR_INVALID_ARG),
+])
+def test_decode_rejects_bad_arguments_before_launch(native, kw, code):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, t=FAKE, l=FAKE, B=4, hq=32, hkv=8, head_dim=128, nb=64, maxb=8,
+             block_size=16, scale=0.1, dtype=N.PKV_BF16, pt=0, ws=FAKE, ws_bytes=1 << 30, out=FAKE)
+    a.update(kw)
+    rc = native.pkv_paged_attention_decode(a["q"], a["k"], a["v"], a["t"], a["l"], a["B"], a["hq"], a["hkv"],
+                                           a["head_dim"], a["nb"], a["maxb"], a["block_size"], a["scale"],
+                                           a["dtype"], a["pt"], a["ws"], a["ws_bytes"], a["out"], None)
+    assert rc == code, native.pkv_last_error_string()
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=9), N.PKV_ERR_UNSUPPORTED),
+    (dict(head_dim=80), N.PKV_ERR_UNSUPPORTED),
+    (dict(kn=FAKE + 8), N.PKV_ERR_INVALID_ARG),
+    (dict(n=-1), N.PKV_ERR_INVALID_ARG),
+    (dict(slots=0), N.PKV_ERR_INVALID_ARG),
+])
+def test_append_rejects_bad_arguments_before_launch(native, kw, code):
+    a = dict(kn=FAKE, vn=FAKE, slots=FAKE, n=3, kp=FAKE, vp=FAKE, nb=8, hkv=8, head_dim=128, bs=16,
+             dtype=N.PKV_BF16)
+    a.update(kw)
+    rc = native.pkv_kv_append(a["kn"], a["vn"], a["slots"], a["n"], a["kp"], a["vp"], a["nb"], a["hkv"],
+                              a["head_dim"], a["bs"], a["dtype"], None)
+    assert rc == code
+
+
+def test_zero_sized_calls_are_no_ops(native):
+    assert native.pkv_kv_append(None, None, None, 0, None, None, 8, 8, 128, 16, N.PKV_BF16, None) == 0
+    assert native.pkv_copy_blocks(None, None, None, 0, 8, 8, 128, 16, N.PKV_BF16, None) == 0
+    assert native.pkv_paged_attention_decode(None, None, None, None, None, 0, 32, 8, 128, 8, 8, 16, 0.1,
+                                             N.PKV_BF16, 0, None, 0, None, None) == 0
+
+
+def test_copy_blocks_rejects_bad_arguments_before_launch(native):
+    assert native.pkv_copy_blocks(FAKE, FAKE, FAKE, 2, 8, 8, 128, 16, 5, None) == N.PKV_ERR_UNSUPPORTED
+    assert native.pkv_copy_blocks(FAKE + 4, FAKE, FAKE, 2, 8, 8, 128, 16, N.PKV_F16, None) == N.PKV_ERR_INVALID_ARG
+    assert native.pkv_copy_blocks(FAKE, FAKE, 0, 2, 8, 8, 128, 16, N.PKV_F16, None) == N.PKV_ERR_INVALID_ARG
