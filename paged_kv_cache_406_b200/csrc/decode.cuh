@@ -202,6 +202,44 @@ __device__ __forceinline__ WorkUnit load_unit(const DecodeParams& p, int w) {
   return u;
 }
 
+// Final merge of one work unit: the kConsumerWarps per-warp records in `rec`
+// (acc[G][D], m[G], l[G] each, taken against each warp's own running max)
+// are rescaled to their common max and either normalised into `out` (the
+// sequence has one partition) or stored as the partition's (m, l, o) partial.
+// Called by the consumer threads (0 .. kConsumerWarps*32-1) after the named
+// barrier that publishes the records.
+template <int G, int D>
+__device__ __forceinline__ void merge_store(const float* rec, const WorkUnit& u, const DecodeParams& p) {
+  constexpr int kMF = G * D + 2 * G;
+  const bool single = u.nparts == 1;
+  for (int idx = threadIdx.x; idx < G * D; idx += kConsumerWarps * 32) {
+    const int h = idx / D, d = idx - h * D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w2 = 0; w2 < kConsumerWarps; ++w2) M = fmaxf(M, rec[w2 * kMF + G * D + h]);
+    float num = 0.f, den = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w2 = 0; w2 < kConsumerWarps; ++w2) {
+        const float f = fast_exp2(rec[w2 * kMF + G * D + h] - M);
+        num += f * rec[w2 * kMF + h * D + d];
+        den += f * rec[w2 * kMF + G * D + G + h];
+      }
+    }
+    const int64_t row = static_cast<int64_t>(u.b) * p.num_q_heads + u.g * G + h;
+    if (single) {
+      p.out[row * D + d] = den > 0.f ? num / den : 0.f;
+    } else {
+      const int64_t pr = row * p.max_parts + u.part;
+      p.part_o[pr * D + d] = num;
+      if (d == 0) {
+        p.part_m[pr] = M;
+        p.part_l[pr] = den;
+      }
+    }
+  }
+}
+
 // Shared memory: [n_stages][K tile | V tile] ring, 2 x kConsumerWarps merge
 // records, full/empty mbarriers, abort flag.
 template <typename T, int D, int G>
@@ -451,34 +489,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
     }
     asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
 
-    const float* m0 = merge + (iter & 1) * kConsumerWarps * kMF;
-    const bool single = u.nparts == 1;
-    for (int idx = threadIdx.x; idx < G * D; idx += kConsumerWarps * 32) {
-      const int h = idx / D, d = idx - h * D;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w2 = 0; w2 < kConsumerWarps; ++w2) M = fmaxf(M, m0[w2 * kMF + G * D + h]);
-      float num = 0.f, den = 0.f;
-      if (M != -INFINITY) {
-#pragma unroll
-        for (int w2 = 0; w2 < kConsumerWarps; ++w2) {
-          const float f = fast_exp2(m0[w2 * kMF + G * D + h] - M);
-          num += f * m0[w2 * kMF + h * D + d];
-          den += f * m0[w2 * kMF + G * D + G + h];
-        }
-      }
-      const int64_t row = static_cast<int64_t>(u.b) * Hq + u.g * G + h;
-      if (single) {
-        p.out[row * D + d] = den > 0.f ? num / den : 0.f;
-      } else {
-        const int64_t pr = row * p.max_parts + u.part;
-        p.part_o[pr * D + d] = num;
-        if (d == 0) {
-          p.part_m[pr] = M;
-          p.part_l[pr] = den;
-        }
-      }
-    }
+    merge_store<G, D>(merge + (iter & 1) * kConsumerWarps * kMF, u, p);
   }
 }
 

@@ -1,0 +1,317 @@
+// PagedAttention decode on tensor cores, for 16-bit K/V with grouped-query
+// heads (G = num_q_heads / num_kv_heads in {2, 4, 8}).
+//
+// Same work list, ring and merge as decode_kernel (decode.cuh); what changes
+// is how a consumer warp turns a 16-token chunk into scores and outputs:
+//
+//   S^T[16 tokens][8 heads] = K[16][D] · Q^T[D][8]     (mma m16n8k16, D/16 steps)
+//   O^T[D][8 heads]        += V^T[D][16] · P^T[16][8]  (mma m16n8k16, D/16 tiles)
+//
+// Query heads of one KV head fill the 8 columns (G of them real, the rest
+// zero), so q·Kᵀ of a GQA group is a dense [tokens x dims] x [dims x heads]
+// product.  P is rounded to a pair of 16-bit values hi + lo (two mmas) so the
+// weights keep about 16 significant bits; accumulation is fp32.
+//
+// K and V chunks arrive by 2-D tensor-map TMA loads with 128-byte swizzle
+// (16-byte chunk c of row r is stored at chunk c ^ (r mod 8)), so the
+// ldmatrix reads of 8 consecutive rows hit 8 different bank groups.  A chunk
+// is 16 tokens: one block (block_size 16), two blocks (8) or half a block (32).
+// Token rows past the end of the sequence are masked out of the softmax and
+// their V rows are zeroed in shared memory before the P·V product, so stale
+// pool contents (possibly NaN) never reach the accumulators.
+#pragma once
+
+#include <cuda.h>
+
+#include "decode.cuh"
+
+namespace pkv {
+
+constexpr int kChunkTokens = 16;
+
+template <int D>
+struct MmaLayout {
+  static constexpr int kHalves = D / 64;                      // 128-byte column halves
+  static constexpr int kHalfBytes = kChunkTokens * 128;       // 16 rows x 128 B
+  static constexpr int kTileBytes = kHalves * kHalfBytes;     // one K (or V) chunk
+  static constexpr int kStageBytes = 2 * kTileBytes;
+};
+
+template <typename T, int D, int G>
+struct MmaSmem {
+  static constexpr int kMergeFloats = G * D + 2 * G;
+  __host__ __device__ static size_t ring_bytes(int ns) { return size_t(ns) * MmaLayout<D>::kStageBytes; }
+  __host__ __device__ static size_t bytes(int ns) {
+    // + 1024: the dynamic shared memory base is aligned up to the 1024-byte swizzle atom
+    return 1024 + ring_bytes(ns) + 2 * kConsumerWarps * kMergeFloats * sizeof(float) + 2 * ns * sizeof(uint64_t) +
+           16;
+  }
+};
+
+// Byte offset of the 16-byte chunk `chunk` (0..7) of row `row` in a
+// 128B-swizzled [rows][128 B] tile whose base is 1024-byte aligned.
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const DecodeParams p,
+                                                                    const __grid_constant__ CUtensorMap tmap_k,
+                                                                    const __grid_constant__ CUtensorMap tmap_v) {
+  static_assert(G == 2 || G == 4 || G == 8, "group size");
+  using L = MmaLayout<D>;
+  constexpr int kSteps = D / 16;  // k-steps of q·Kᵀ and m-tiles of P·V
+  constexpr int kMF = MmaSmem<T, D, G>::kMergeFloats;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int BS = p.block_size;
+  const int NS = p.n_stages;
+  float* merge = reinterpret_cast<float*>(smem + MmaSmem<T, D, G>::ring_bytes(NS));
+  uint64_t* full = reinterpret_cast<uint64_t*>(merge + 2 * kConsumerWarps * kMF);
+  uint64_t* empty = full + NS;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + NS);
+  const uint32_t ring_s = smem_addr(smem);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(smem_addr(full + s), 1);
+      mbar_init(smem_addr(empty + s), 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const int n_work = *p.n_items * p.num_kv_heads;
+
+  if (warp == kConsumerWarps) {
+    // ----------------------------- producer -----------------------------
+    if (lane == 0) {
+      prefetch_tensormap(&tmap_k);
+      prefetch_tensormap(&tmap_v);
+    }
+    const uint64_t policy = l2_evict_first_policy();
+    const int box_rows = BS < kChunkTokens ? BS : kChunkTokens;
+    uint32_t c = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < n_work && ok; w += gridDim.x) {
+      const WorkUnit u = load_unit(p, w);
+      const int32_t* trow = p.block_tables + static_cast<int64_t>(u.b) * p.max_blocks + u.t0 / BS;
+      const int nch = (u.t1 - u.t0 + kChunkTokens - 1) / kChunkTokens;
+      int wb = -64, mine = 0;  // window of 32 table entries starting at block wb
+      for (int k = 0; k < nch; ++k, ++c) {
+        const int jb0 = (k * kChunkTokens) / BS;  // first block of the chunk (unit-relative)
+        const int nb_here = BS < kChunkTokens ? min(kChunkTokens / BS, u.nblk - jb0) : 1;
+        if (jb0 + nb_here > wb + 32) {
+          wb = jb0;
+          mine = wb + lane < u.nblk ? trow[wb + lane] : 0;
+        }
+        int phys0 = __shfl_sync(kFull, mine, jb0 - wb);
+        int phys1 = __shfl_sync(kFull, mine, min(jb0 + 1 - wb, 31));
+        if (lane == 0) {
+          const int s = c % NS;
+          const uint32_t r = c / NS;
+          ok = mbar_wait(smem_addr(empty + s), (r & 1) ^ 1, abort_flag);
+          if (ok) {
+            const uint32_t bar = smem_addr(full + s);
+            const uint32_t kdst = ring_s + s * L::kStageBytes;
+            const uint32_t vdst = kdst + L::kTileBytes;
+            const int row_in_block = BS > kChunkTokens ? (k * kChunkTokens) % BS : 0;
+            mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nb_here * box_rows * D * 2 * 2));
+            for (int i = 0; i < nb_here; ++i) {
+              int phys = i == 0 ? phys0 : phys1;
+              if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_blocks)) {
+                record_error(PKV_ERR_BAD_BLOCK);
+                phys = 0;
+              }
+              const int32_t y = (phys * p.num_kv_heads + u.g) * BS + row_in_block;
+#pragma unroll
+              for (int h = 0; h < L::kHalves; ++h) {
+                const uint32_t off = h * L::kHalfBytes + i * box_rows * 128;
+                tma_load_2d(kdst + off, &tmap_k, 64 * h, y, bar, policy);
+                tma_load_2d(vdst + off, &tmap_v, 64 * h, y, bar, policy);
+              }
+            }
+          } else {
+            record_error(PKV_ERR_DEVICE_TIMEOUT);
+            *abort_flag = 1;
+          }
+        }
+        ok = __shfl_sync(kFull, ok, 0);
+        if (!ok) break;
+      }
+    }
+    // No copy may still be landing in shared memory when the CTA exits.
+    __syncwarp();
+    if (lane == 0) {
+      for (int s = 0; s < NS && s < static_cast<int>(c); ++s) {
+        const uint32_t last_round = (c - 1 - s) / NS;
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(smem_addr(full + s), last_round & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+    return;
+  }
+
+  // ------------------------------ consumers ------------------------------
+  const int gq = lane >> 2;  // fragment row group: token (S^T) / dim (O^T) / head (B operands)
+  const int tq = lane & 3;   // fragment column pair: heads 2tq, 2tq+1
+  // lanes that feed ldmatrix rows
+  const int ld_row_a = (lane & 7) + ((lane >> 3) & 1) * 8, ld_col_a = lane >> 4;  // K (A = K chunk)
+  const int ld_row_v = (lane & 7) + (lane >> 4) * 8, ld_col_v = (lane >> 3) & 1;  // V (A = V^T, .trans)
+  const int src0 = 4 * (2 * tq) + (gq >> 1), src1 = src0 + 4;  // P^T transpose sources
+  const uint32_t sel = (gq & 1) ? 0x7632u : 0x5410u;
+  const float sl = p.scale_log2;
+  uint32_t c = 0;
+  int iter = 0;
+  bool ok = true;
+  for (int w = blockIdx.x; w < n_work; w += gridDim.x, ++iter) {
+    const WorkUnit u = load_unit(p, w);
+    const int nch = (u.t1 - u.t0 + kChunkTokens - 1) / kChunkTokens;
+
+    // B fragments of Qᵀ: column n = head gq (zero for the padding heads >= G)
+    uint32_t qb[kSteps][2];
+    {
+      const T* qrow = static_cast<const T*>(p.q) + (static_cast<int64_t>(u.b) * p.num_q_heads + u.g * G + gq) * D;
+#pragma unroll
+      for (int ks = 0; ks < kSteps; ++ks) {
+        qb[ks][0] = gq < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq)) : 0u;
+        qb[ks][1] = gq < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq + 8)) : 0u;
+      }
+    }
+    float acc[kSteps][4];
+#pragma unroll
+    for (int mt = 0; mt < kSteps; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // heads 2tq, 2tq+1
+
+    const int k0 = (warp - static_cast<int>(c % kConsumerWarps) + kConsumerWarps) % kConsumerWarps;
+    for (int k = k0; k < nch && ok; k += kConsumerWarps) {
+      const uint32_t cc = c + k;
+      const int s = cc % NS;
+      const bool landed = __all_sync(kFull, mbar_wait(smem_addr(full + s), (cc / NS) & 1, abort_flag));
+      if (!landed) {
+        if (lane == 0) {
+          record_error(PKV_ERR_DEVICE_TIMEOUT);
+          *abort_flag = 1;
+        }
+        ok = false;
+        break;
+      }
+      const uint32_t kbase = ring_s + s * L::kStageBytes;
+      const uint32_t vbase = kbase + L::kTileBytes;
+      const int nv = min(kChunkTokens, u.t1 - (u.t0 + k * kChunkTokens));
+
+      // ---- scores: S^T = K · Qᵀ ----
+      float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < kSteps; ++ks) {
+        uint32_t a[4];
+        ldmatrix_x4(kbase + (ks / 4) * L::kHalfBytes + swz(ld_row_a, 2 * (ks % 4) + ld_col_a), a);
+        mma_16816<T>(sc, a, qb[ks][0], qb[ks][1]);
+      }
+      const bool v0 = gq < nv, v1 = gq + 8 < nv;  // tokens gq and gq + 8 of the chunk
+      const float s0 = v0 ? sc[0] * sl : -INFINITY, s1 = v0 ? sc[1] * sl : -INFINITY;
+      const float s2 = v1 ? sc[2] * sl : -INFINITY, s3 = v1 ? sc[3] * sl : -INFINITY;
+
+      // ---- online softmax (the running max moves only by more than the threshold) ----
+      float bm0 = fmaxf(s0, s2), bm1 = fmaxf(s1, s3);
+      if (__any_sync(kFull, bm0 > m0 + kRescaleThreshold || bm1 > m1 + kRescaleThreshold)) {
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          bm0 = fmaxf(bm0, __shfl_xor_sync(kFull, bm0, o));
+          bm1 = fmaxf(bm1, __shfl_xor_sync(kFull, bm1, o));
+        }
+        const float n0 = fmaxf(m0, bm0), n1 = fmaxf(m1, bm1);
+        const float f0 = n0 == -INFINITY ? 1.f : fast_exp2(m0 - n0);
+        const float f1 = n1 == -INFINITY ? 1.f : fast_exp2(m1 - n1);
+#pragma unroll
+        for (int mt = 0; mt < kSteps; ++mt) {
+          acc[mt][0] *= f0;
+          acc[mt][2] *= f0;
+          acc[mt][1] *= f1;
+          acc[mt][3] *= f1;
+        }
+        l0 *= f0;
+        l1 *= f1;
+        m0 = n0;
+        m1 = n1;
+      }
+      const float p0 = fast_exp2(s0 - m0), p1 = fast_exp2(s1 - m1);
+      const float p2 = fast_exp2(s2 - m0), p3 = fast_exp2(s3 - m1);
+      l0 += p0 + p2;
+      l1 += p1 + p3;
+
+      // ---- P as hi + lo 16-bit pairs, transposed into B fragments of Pᵀ ----
+      uint32_t ha, la, hb, lb;
+      split_pack<T>(p0, p1, ha, la);  // token gq:     heads 2tq, 2tq+1
+      split_pack<T>(p2, p3, hb, lb);  // token gq + 8
+      const uint32_t bh0 = __byte_perm(__shfl_sync(kFull, ha, src0), __shfl_sync(kFull, ha, src1), sel);
+      const uint32_t bh1 = __byte_perm(__shfl_sync(kFull, hb, src0), __shfl_sync(kFull, hb, src1), sel);
+      const uint32_t bl0 = __byte_perm(__shfl_sync(kFull, la, src0), __shfl_sync(kFull, la, src1), sel);
+      const uint32_t bl1 = __byte_perm(__shfl_sync(kFull, lb, src0), __shfl_sync(kFull, lb, src1), sel);
+
+      // ---- rows past the sequence end: zero V so stale values cannot reach P·V ----
+      if (nv < kChunkTokens) {
+        const int per_row = 8 * L::kHalves;
+        const int total = (kChunkTokens - nv) * per_row;
+        for (int i = lane; i < total; i += 32) {
+          const int row = nv + i / per_row, rem = i % per_row;
+          const uint32_t addr = vbase + (rem / 8) * L::kHalfBytes + row * 128 + (rem % 8) * 16;
+          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0) : "memory");
+        }
+        __syncwarp();
+      }
+
+      // ---- O^T += V^T · P^T ----
+#pragma unroll
+      for (int mt = 0; mt < kSteps; ++mt) {
+        uint32_t a[4];
+        ldmatrix_x4_trans(vbase + (mt / 4) * L::kHalfBytes + swz(ld_row_v, 2 * (mt % 4) + ld_col_v), a);
+        mma_16816<T>(acc[mt], a, bh0, bh1);
+        mma_16816<T>(acc[mt], a, bl0, bl1);
+      }
+      if (nv < kChunkTokens) fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(empty + s));
+    }
+    c += nch;
+
+    // ---- publish this warp's record, then merge the warps ----
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      l0 += __shfl_xor_sync(kFull, l0, o);
+      l1 += __shfl_xor_sync(kFull, l1, o);
+    }
+    float* mb = merge + ((iter & 1) * kConsumerWarps + warp) * kMF;
+    const int h0 = 2 * tq, h1 = 2 * tq + 1;
+#pragma unroll
+    for (int mt = 0; mt < kSteps; ++mt) {
+      const int d = 16 * mt + gq;
+      if (h0 < G) {
+        mb[h0 * D + d] = acc[mt][0];
+        mb[h0 * D + d + 8] = acc[mt][2];
+      }
+      if (h1 < G) {
+        mb[h1 * D + d] = acc[mt][1];
+        mb[h1 * D + d + 8] = acc[mt][3];
+      }
+    }
+    if (gq == 0) {
+      if (h0 < G) {
+        mb[G * D + h0] = m0;
+        mb[G * D + G + h0] = l0;
+      }
+      if (h1 < G) {
+        mb[G * D + h1] = m1;
+        mb[G * D + G + h1] = l1;
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+    merge_store<G, D>(merge + (iter & 1) * kConsumerWarps * kMF, u, p);
+  }
+}
+
+}  // namespace pkv

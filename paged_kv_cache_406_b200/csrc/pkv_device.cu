@@ -4,8 +4,11 @@
 
 #include <atomic>
 #include <cmath>
+#include <cstring>
+#include <mutex>
 
 #include "decode.cuh"
+#include "decode_mma.cuh"
 #include "device_common.cuh"
 #include "pkv_internal.h"
 
@@ -160,6 +163,8 @@ int launch_decode(const pkv::DecodeParams& base, const int32_t* seq_lens, int32_
       smem_max = std::max(smem_max, pkv::DecodeSmem<T, D, G>::bytes(bs, ring_stages(size_t(2) * bs * D * sizeof(T))));
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_max));
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(carveout)");
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, pkv::kDecodeThreads, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
     if (occ <= 0) return fail(PKV_ERR_CUDA, "decode kernel does not fit on an SM (smem %zu)", smem);
@@ -182,6 +187,129 @@ int launch_decode(const pkv::DecodeParams& base, const int32_t* seq_lens, int32_
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return pkv::ok();
+}
+
+// ---- tensor maps over the K/V pools for the tensor-core kernel ----
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// Pool viewed as a 2-D tensor [rows = num_blocks * Hkv * block_size][head_dim]
+// of 16-bit elements; boxes of 64 elements (128 B) x box_rows, 128-byte swizzle.
+int make_pool_map(CUtensorMap* m, const void* pool, int dtype, int64_t rows, int head_dim, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                   const_cast<void*>(pool), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return PKV_OK;
+}
+
+// Small cache of encoded maps: a decode step reuses the same pools every call.
+struct MapCacheEntry {
+  const void* pool;
+  int64_t rows;
+  int dtype, head_dim, box_rows;
+  CUtensorMap map;
+};
+
+int pool_map(CUtensorMap* out, const void* pool, int dtype, int64_t rows, int head_dim, int box_rows) {
+  static std::mutex mu;
+  static MapCacheEntry cache[8];
+  static int next = 0, used = 0;
+  std::lock_guard<std::mutex> g(mu);
+  for (int i = 0; i < used; ++i) {
+    const MapCacheEntry& e = cache[i];
+    if (e.pool == pool && e.rows == rows && e.dtype == dtype && e.head_dim == head_dim && e.box_rows == box_rows) {
+      *out = e.map;
+      return PKV_OK;
+    }
+  }
+  int rc = make_pool_map(out, pool, dtype, rows, head_dim, box_rows);
+  if (rc) return rc;
+  cache[next] = MapCacheEntry{pool, rows, dtype, head_dim, box_rows, *out};
+  next = (next + 1) % 8;
+  used = used < 8 ? used + 1 : 8;
+  return PKV_OK;
+}
+
+template <typename T, int D, int G>
+int launch_decode_mma(const pkv::DecodeParams& base, const int32_t* seq_lens, int32_t num_seqs, int32_t max_tokens,
+                      int dtype, cudaStream_t stream) {
+  pkv::DecodeParams p = base;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  p.n_stages = 8;
+  const size_t smem = pkv::MmaSmem<T, D, G>::bytes(p.n_stages);
+  auto kern = pkv::decode_mma_kernel<T, D, G>;
+  static std::atomic<int> occ_cache[kMaxDevices];
+  int occ = dev < kMaxDevices ? occ_cache[dev].load(std::memory_order_relaxed) : 0;
+  if (occ == 0) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_mma)");
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(carveout)");
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, pkv::kDecodeThreads, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    if (occ <= 0) return fail(PKV_ERR_CUDA, "decode_mma kernel does not fit on an SM (smem %zu)", smem);
+    if (dev < kMaxDevices) occ_cache[dev].store(occ, std::memory_order_relaxed);
+  }
+  const int64_t rows = int64_t(p.num_blocks) * p.num_kv_heads * p.block_size;
+  const int box_rows = p.block_size < pkv::kChunkTokens ? p.block_size : pkv::kChunkTokens;
+  CUtensorMap mk, mv;
+  int rc = pool_map(&mk, p.k_pool, dtype, rows, D, box_rows);
+  if (rc) return rc;
+  rc = pool_map(&mv, p.v_pool, dtype, rows, D, box_rows);
+  if (rc) return rc;
+
+  const int kmax = p.partition_tokens / p.block_size;
+  pkv::plan_kernel<<<1, 1024, 2 * (kmax + 1) * sizeof(int32_t), stream>>>(
+      seq_lens, num_seqs, max_tokens, p.partition_tokens, p.block_size, const_cast<int4*>(p.items),
+      const_cast<int32_t*>(p.n_items));
+  const int64_t work_upper = int64_t(num_seqs) * p.max_parts * p.num_kv_heads;
+  const int grid = static_cast<int>(std::min<int64_t>(int64_t(sm_count(dev)) * occ, work_upper));
+  kern<<<grid, pkv::kDecodeThreads, smem, stream>>>(p, mk, mv);
+  if (p.max_parts > 1) {
+    const int rows_out = num_seqs * p.num_q_heads;
+    pkv::reduce_kernel<D><<<(rows_out + 7) / 8, 256, 0, stream>>>(seq_lens, num_seqs, p.num_q_heads, max_tokens,
+                                                                  p.partition_tokens, p.max_parts, p.part_m,
+                                                                  p.part_l, p.part_o, p.out);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode_mma launch");
+  return pkv::ok();
+}
+
+template <typename T>
+int dispatch_decode_mma(int32_t head_dim, int32_t group, const pkv::DecodeParams& p, const int32_t* seq_lens,
+                        int32_t num_seqs, int32_t max_tokens, int dtype, cudaStream_t s) {
+  if (head_dim == 128) {
+    if (group == 2) return launch_decode_mma<T, 128, 2>(p, seq_lens, num_seqs, max_tokens, dtype, s);
+    if (group == 4) return launch_decode_mma<T, 128, 4>(p, seq_lens, num_seqs, max_tokens, dtype, s);
+    return launch_decode_mma<T, 128, 8>(p, seq_lens, num_seqs, max_tokens, dtype, s);
+  }
+  if (group == 2) return launch_decode_mma<T, 64, 2>(p, seq_lens, num_seqs, max_tokens, dtype, s);
+  if (group == 4) return launch_decode_mma<T, 64, 4>(p, seq_lens, num_seqs, max_tokens, dtype, s);
+  return launch_decode_mma<T, 64, 8>(p, seq_lens, num_seqs, max_tokens, dtype, s);
 }
 
 template <typename T>
@@ -271,8 +399,10 @@ extern "C" int pkv_paged_attention_decode(const void* q, const void* k_pool, con
     return fail(PKV_ERR_INVALID_ARG, "%s: num_q_heads %d not a multiple of num_kv_heads %d", fn, num_q_heads,
                 num_kv_heads);
   const int32_t group = num_q_heads / num_kv_heads;
-  if (group != 1 && group != 2 && group != 4)
-    return fail(PKV_ERR_UNSUPPORTED, "%s: group size %d not supported (1, 2 or 4)", fn, group);
+  if (group != 1 && group != 2 && group != 4 && group != 8)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: group size %d not supported (1, 2, 4 or 8)", fn, group);
+  if (group == 8 && dtype == PKV_F32)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: group size 8 needs 16-bit K/V", fn);
   if (!std::isfinite(scale)) return fail(PKV_ERR_INVALID_ARG, "%s: scale is not finite", fn);
   int32_t pt = 0;
   rc = resolve_partition(partition_tokens, block_size, &pt);
@@ -312,6 +442,15 @@ extern "C" int pkv_paged_attention_decode(const void* q, const void* k_pool, con
   p.out = out;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int32_t mt = static_cast<int32_t>(max_tokens);
+  // 16-bit K/V with grouped heads: tensor-core kernel (16-token chunks);
+  // otherwise the CUDA-core kernel
+  if (dtype != PKV_F32 && group >= 2 && pt % pkv::kChunkTokens == 0) {
+    if (int64_t(num_blocks) * num_kv_heads * block_size > INT32_MAX)
+      return fail(PKV_ERR_INVALID_ARG, "%s: pool has more than 2^31 token rows", fn);
+    if (dtype == PKV_BF16) return dispatch_decode_mma<__nv_bfloat16>(head_dim, group, p, seq_lens, num_seqs, mt, dtype, s);
+    return dispatch_decode_mma<__half>(head_dim, group, p, seq_lens, num_seqs, mt, dtype, s);
+  }
+  if (group == 8) return fail(PKV_ERR_UNSUPPORTED, "%s: group size 8 needs partition_tokens %% 16 == 0", fn);
   switch (dtype) {
     case PKV_F32: return dispatch_decode<float>(head_dim, group, p, seq_lens, num_seqs, mt, s);
     case PKV_BF16: return dispatch_decode<__nv_bfloat16>(head_dim, group, p, seq_lens, num_seqs, mt, s);

@@ -43,9 +43,13 @@ def _ragged(bs):
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("g", [1, 2, 4])
+@pytest.mark.parametrize("g", [1, 2, 4, 8])
 @pytest.mark.parametrize("bs", [8, 16, 32])
 def test_decode_matches_oracle(dtype, d, g, bs):
+    """16-bit K/V with G >= 2 runs on the tensor-core kernel, the rest on the
+    CUDA-core kernel; both against the oracle on ragged lengths."""
+    if dtype == "f32" and g == 8:
+        pytest.skip("group size 8 needs 16-bit K/V (rejected: see test_unsupported_group)")
     hkv = 2
     case = Case(_ragged(bs), g * hkv, hkv, d, bs, dtype, seed=zlib.crc32(f"{dtype}{d}{g}{bs}".encode()) % 1000)
     ref = case.oracle()
@@ -62,6 +66,39 @@ def test_partition_sizes_agree(pt_blocks):
     assert_close(out, ref, "bf16", f"partition {bs * pt_blocks}")
     single = _decode(case, pt=8192)
     assert torch.max(torch.abs(out - single)).item() < 1e-4
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("g", [2, 4, 8])
+def test_tensor_core_and_cuda_core_kernels_agree(dtype, g):
+    """partition_tokens 24 (not a multiple of 16) sends 16-bit GQA work to the
+    CUDA-core kernel; 32 to the tensor-core kernel.  Both match the oracle."""
+    if g == 8:
+        pytest.skip("the CUDA-core kernel covers group sizes 1, 2, 4")
+    case = Case([1, 7, 8, 9, 23, 24, 25, 200, 777], 2 * g, 2, 128, 8, dtype, seed=21)
+    ref = case.oracle()
+    simt = _decode(case, pt=24)
+    mma = _decode(case, pt=32)
+    assert_close(simt, ref, dtype, "cuda-core kernel")
+    assert_close(mma, ref, dtype, "tensor-core kernel")
+    assert torch.max(torch.abs(simt - mma)).item() < 2e-3
+
+
+def test_unsupported_group():
+    case = Case([5], 8, 1, 64, 16, "f32", seed=22)
+    with pytest.raises(pkv.PagedKVError) as e:
+        _decode(case)
+    assert e.value.code == pkv._native.PKV_ERR_UNSUPPORTED
+
+
+def test_softmax_peaked_two_tokens_meets_tolerance():
+    """Two tokens with scores far apart and large V: the hi + lo split of P
+    keeps the weighted sum within tolerance where a single 16-bit P would not."""
+    case = Case([2, 3, 2], 8, 2, 128, 16, "bf16", seed=23)
+    case.v_pool.mul_(8.0)
+    case.q.mul_(3.0)
+    ref = case.oracle()
+    assert_close(_decode(case), ref, "bf16", "peaked")
 
 
 def test_zero_length_gives_zeros_and_single_token_gives_v():
