@@ -26,8 +26,10 @@
  *    pkv_last_error_string() gives the text of the calling thread's last error.
  *  - Argument errors are reported synchronously, before anything is launched.
  *  - Device pointers are owned by the caller (allocated e.g. by PyTorch); the
- *    library never allocates or frees device memory.  Device buffers must be
- *    16-byte aligned and densely packed in the layouts stated below.
+ *    library never allocates or frees device memory at run time (the one fixed
+ *    exception is the static scratch of pkv_paged_attention_decode_static,
+ *    held from library load to process exit).  Device buffers must be 16-byte
+ *    aligned and densely packed in the layouts stated below.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *    Kernels are launched asynchronously on it; returning PKV_OK means the
  *    launch was accepted.  Faults found by the kernels themselves (a block id
@@ -217,6 +219,37 @@ int pkv_paged_attention_decode(const void* q, const void* k_pool, const void* v_
                                int32_t block_size, float scale, int32_t dtype,
                                int32_t partition_tokens, void* workspace, size_t workspace_bytes,
                                float* out, void* stream);
+
+/* PagedAttention decode exactly as pkv_paged_attention_decode, for callers
+ * that cannot allocate device memory when they decode: serving runtimes that
+ * have reserved nearly all of HBM for their KV pool up front, framework
+ * plugins whose host owns every allocation, hot loops that must not pay a
+ * synchronising cudaMalloc/cudaFree.  (The source pages have no counterpart:
+ * this is a library convenience.)  The scratch space comes from a static
+ * device array inside the library, pkv_static_workspace_bytes() bytes
+ * (64 MiB) on every GPU that loads the library, held until the process exits;
+ * this call allocates nothing.
+ *  - Sizes whose scratch (pkv_decode_workspace_size) exceeds that limit are
+ *    rejected with PKV_ERR_INVALID_ARG before anything is launched.
+ *  - The first call on a device looks up the array's device address with
+ *    cudaGetSymbolAddress (once per device); make that first call before any
+ *    stream capture.
+ *  - All calls share the one array, and it keeps the last call's contents
+ *    (every value a call reads it writes first, so nothing needs clearing).
+ *    Calls that overlap on the GPU (different streams, no ordering between
+ *    them) race on it: serialise them, or use pkv_paged_attention_decode with
+ *    separate workspaces.
+ * Arguments, layouts and results as for pkv_paged_attention_decode. */
+int pkv_paged_attention_decode_static(const void* q, const void* k_pool, const void* v_pool,
+                                      const int32_t* block_tables, const int32_t* seq_lens, int32_t num_seqs,
+                                      int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                      int32_t num_blocks, int32_t max_blocks_per_seq, int32_t block_size,
+                                      float scale, int32_t dtype, int32_t partition_tokens, float* out,
+                                      void* stream);
+
+/* Size in bytes of the static workspace used by
+ * pkv_paged_attention_decode_static. */
+size_t pkv_static_workspace_bytes(void);
 
 /* Synchronise `stream`, then read the device status word of the current
  * device into *status: PKV_OK, or the first PKV_ERR_BAD_BLOCK /

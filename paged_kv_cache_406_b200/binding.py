@@ -121,6 +121,36 @@ def pkv_paged_attention_decode(q: torch.Tensor, k_pool: torch.Tensor, v_pool: to
     return out
 
 
+def pkv_paged_attention_decode_static(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                                      block_tables: torch.Tensor, seq_lens: torch.Tensor, scale: float,
+                                      out: Optional[torch.Tensor] = None, partition_tokens: int = 0) -> torch.Tensor:
+    """Decode with the library's static scratch instead of a workspace tensor,
+    for callers that cannot allocate device memory while decoding (pass
+    ``out`` to allocate nothing here either).  Same result as
+    :func:`pkv_paged_attention_decode`; calls overlapping on the GPU race on
+    the shared scratch."""
+    nb, hkv, bs, d = _pool_dims(_cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"))
+    _cuda(q, "q", k_pool.dtype)
+    if q.dim() != 3 or q.shape[2] != d:
+        raise ValueError(f"q must be [num_seqs, num_q_heads, {d}]")
+    B, hq, _ = q.shape
+    _cuda(block_tables, "block_tables", torch.int32)
+    _cuda(seq_lens, "seq_lens", torch.int32)
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.numel() != B:
+        raise ValueError("block_tables must be [num_seqs, max_blocks_per_seq] and seq_lens [num_seqs]")
+    if out is None:
+        out = torch.empty((B, hq, d), dtype=torch.float32, device=q.device)
+    else:
+        _cuda(out, "out", torch.float32)
+        if tuple(out.shape) != (B, hq, d):
+            raise ValueError("out has the wrong shape")
+    check(lib().pkv_paged_attention_decode_static(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
+                                                  block_tables.data_ptr(), seq_lens.data_ptr(), B, hq, hkv, d, nb,
+                                                  block_tables.shape[1], bs, float(scale), _dtype_code(k_pool),
+                                                  partition_tokens, out.data_ptr(), _stream()))
+    return out
+
+
 def pkv_device_status(clear: bool = True) -> int:
     """Synchronise the current stream and return the device status word."""
     st = ctypes.c_int32(0)
@@ -214,4 +244,4 @@ class Allocator:
 
 
 __all__ = ["Allocator", "PagedKVError", "pkv_kv_append", "pkv_copy_blocks", "pkv_decode_workspace_size",
-           "pkv_paged_attention_decode", "pkv_device_status"]
+           "pkv_paged_attention_decode", "pkv_paged_attention_decode_static", "pkv_device_status"]

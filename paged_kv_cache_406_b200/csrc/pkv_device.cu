@@ -473,3 +473,68 @@ extern "C" int pkv_device_status(void* stream, int32_t* status, int32_t clear) {
   *status = v;
   return pkv::ok();
 }
+
+// ===========================================================================
+// Decode without caller-provided workspace.
+//
+// Some callers cannot allocate device memory at the point where they decode:
+// serving runtimes that reserve nearly all of HBM for their KV pool up front
+// (a later cudaMalloc can fail or fragment that reservation), framework
+// plugins whose host owns every allocation and forbids direct cudaMalloc, and
+// hot loops that must not pay a synchronising cudaMalloc / cudaFree.  For
+// them the split-partition scratch lives in this file-scope array instead.
+// Every GPU that loads the library holds it (kStaticWorkspaceBytes) until the
+// process exits.
+// ===========================================================================
+namespace {
+
+constexpr size_t kStaticWorkspaceBytes = size_t(64) << 20;  // 64 MiB
+static __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
+
+// Device address of g_static_workspace on the current device, looked up once
+// per device (the host-side name is only a stand-in for the device array).
+int static_workspace_ptr(void** out) {
+  static std::mutex mu;
+  static void* ptrs[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev >= kMaxDevices) return fail(PKV_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kMaxDevices);
+  std::lock_guard<std::mutex> g(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_workspace);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static workspace)");
+    ptrs[dev] = p;
+  }
+  *out = ptrs[dev];
+  return PKV_OK;
+}
+
+}  // namespace
+
+extern "C" size_t pkv_static_workspace_bytes(void) { return kStaticWorkspaceBytes; }
+
+extern "C" int pkv_paged_attention_decode_static(const void* q, const void* k_pool, const void* v_pool,
+                                                 const int32_t* block_tables, const int32_t* seq_lens,
+                                                 int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                                 int32_t head_dim, int32_t num_blocks, int32_t max_blocks_per_seq,
+                                                 int32_t block_size, float scale, int32_t dtype,
+                                                 int32_t partition_tokens, float* out, void* stream) {
+  size_t need = 0;
+  int rc = pkv_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, block_size,
+                                     partition_tokens, &need);
+  if (rc) return rc;
+  if (need > kStaticWorkspaceBytes)
+    return fail(PKV_ERR_INVALID_ARG,
+                "pkv_paged_attention_decode_static: these sizes need %zu bytes of scratch, more than the %zu-byte "
+                "static workspace; use pkv_paged_attention_decode with a caller-provided workspace",
+                need, kStaticWorkspaceBytes);
+  if (num_seqs == 0) return pkv::ok();
+  void* ws = nullptr;
+  rc = static_workspace_ptr(&ws);
+  if (rc) return rc;
+  return pkv_paged_attention_decode(q, k_pool, v_pool, block_tables, seq_lens, num_seqs, num_q_heads, num_kv_heads,
+                                    head_dim, num_blocks, max_blocks_per_seq, block_size, scale, dtype,
+                                    partition_tokens, ws, kStaticWorkspaceBytes, out, stream);
+}
