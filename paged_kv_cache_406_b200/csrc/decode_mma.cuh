@@ -12,9 +12,10 @@
 // product.  P is rounded to a pair of 16-bit values hi + lo (two mmas) so the
 // weights keep about 16 significant bits; accumulation is fp32.
 //
-// K and V chunks arrive by 2-D tensor-map TMA loads with 128-byte swizzle
-// (16-byte chunk c of row r is stored at chunk c ^ (r mod 8)), so the
-// ldmatrix reads of 8 consecutive rows hit 8 different bank groups.  A chunk
+// K and V chunks arrive by 3-D tensor-map TMA loads (one per block and per K
+// or V: all 128-byte column halves of br rows) with 128-byte swizzle (16-byte
+// chunk c of row r is stored at chunk c ^ (r mod 8)), so the ldmatrix reads of
+// 8 consecutive rows hit 8 different bank groups.  A chunk
 // is 16 tokens: one block (block_size 16), two blocks (8) or half a block (32).
 // Token rows past the end of the sequence are masked out of the softmax and
 // their V rows are zeroed in shared memory before the P·V product, so stale
@@ -31,9 +32,8 @@ constexpr int kChunkTokens = 16;
 
 template <int D>
 struct MmaLayout {
-  static constexpr int kHalves = D / 64;                      // 128-byte column halves
-  static constexpr int kHalfBytes = kChunkTokens * 128;       // 16 rows x 128 B
-  static constexpr int kTileBytes = kHalves * kHalfBytes;     // one K (or V) chunk
+  static constexpr int kHalves = D / 64;                       // 128-byte column halves of a row
+  static constexpr int kTileBytes = kChunkTokens * D * 2;       // one 16-token K (or V) chunk
   static constexpr int kStageBytes = 2 * kTileBytes;
 };
 
@@ -42,16 +42,21 @@ struct MmaSmem {
   static constexpr int kMergeFloats = G * D + 2 * G;
   __host__ __device__ static size_t ring_bytes(int ns) { return size_t(ns) * MmaLayout<D>::kStageBytes; }
   __host__ __device__ static size_t bytes(int ns) {
-    // + 1024: the dynamic shared memory base is aligned up to the 1024-byte swizzle atom
+    // + 1024: the dynamic shared memory base is aligned up to the 1024-byte swizzle atom;
+    // + 128: the producer's window of 32 block-table entries
     return 1024 + ring_bytes(ns) + 2 * kConsumerWarps * kMergeFloats * sizeof(float) + 2 * ns * sizeof(uint64_t) +
-           16;
+           16 + 128;
   }
 };
 
-// Byte offset of the 16-byte chunk `chunk` (0..7) of row `row` in a
-// 128B-swizzled [rows][128 B] tile whose base is 1024-byte aligned.
-__device__ __forceinline__ uint32_t swz(int row, int chunk) {
-  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+// A chunk tile in shared memory is built from TMA boxes of `br` rows (br = 16,
+// or 8 when block_size is 8 and a chunk spans two blocks).  Each box holds,
+// for every 128-byte column half h, br rows of 128 B with the 128-byte
+// swizzle (16-byte chunk c of row r at chunk position c ^ (r mod 8)):
+//     byte offset of (row r, half h) = (r / br) * (halves * br * 128) + h * br * 128 + (r % br) * 128
+__device__ __forceinline__ uint32_t row_offset(int r, int h, int br_shift, int halves) {
+  const int br = 1 << br_shift;
+  return static_cast<uint32_t>(((r >> br_shift) * halves * br + h * br + (r & (br - 1))) * 128);
 }
 
 template <typename T, int D, int G>
@@ -61,16 +66,20 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
   static_assert(G == 2 || G == 4 || G == 8, "group size");
   using L = MmaLayout<D>;
   constexpr int kSteps = D / 16;  // k-steps of q·Kᵀ and m-tiles of P·V
+  constexpr int kHalves = L::kHalves;
   constexpr int kMF = MmaSmem<T, D, G>::kMergeFloats;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
   const int BS = p.block_size;
   const int NS = p.n_stages;
+  const int bs_shift = BS == 8 ? 3 : (BS == 16 ? 4 : 5);
+  const int br_shift = BS == 8 ? 3 : 4;  // rows per TMA box: 8 or 16
   float* merge = reinterpret_cast<float*>(smem + MmaSmem<T, D, G>::ring_bytes(NS));
   uint64_t* full = reinterpret_cast<uint64_t*>(merge + 2 * kConsumerWarps * kMF);
   uint64_t* empty = full + NS;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + NS);
+  int32_t* tab = reinterpret_cast<int32_t*>(empty + NS) + 4;  // 32 block-table entries
   const uint32_t ring_s = smem_addr(smem);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -88,68 +97,70 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
 
   if (warp == kConsumerWarps) {
     // ----------------------------- producer -----------------------------
+    // All lanes walk the units and refill the table window; lane 0 alone
+    // issues the chunks of each window, so the per-chunk path has no
+    // warp-wide synchronisation.
     if (lane == 0) {
       prefetch_tensormap(&tmap_k);
       prefetch_tensormap(&tmap_v);
     }
     const uint64_t policy = l2_evict_first_policy();
-    const int box_rows = BS < kChunkTokens ? BS : kChunkTokens;
-    uint32_t c = 0;
+    const uint32_t box_bytes = (1u << br_shift) * D * 2;           // one K (or V) box
+    const uint32_t blk_off = kHalves * (1u << br_shift) * 128;     // second box of a chunk (block_size 8)
+    int s = 0;
+    uint32_t ph = 0, issued = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < n_work && ok; w += gridDim.x) {
       const WorkUnit u = load_unit(p, w);
-      const int32_t* trow = p.block_tables + static_cast<int64_t>(u.b) * p.max_blocks + u.t0 / BS;
+      const int32_t* trow = p.block_tables + static_cast<int64_t>(u.b) * p.max_blocks + (u.t0 >> bs_shift);
       const int nch = (u.t1 - u.t0 + kChunkTokens - 1) / kChunkTokens;
-      int wb = -64, mine = 0;  // window of 32 table entries starting at block wb
-      for (int k = 0; k < nch; ++k, ++c) {
-        const int jb0 = (k * kChunkTokens) / BS;  // first block of the chunk (unit-relative)
-        const int nb_here = BS < kChunkTokens ? min(kChunkTokens / BS, u.nblk - jb0) : 1;
-        if (jb0 + nb_here > wb + 32) {
-          wb = jb0;
-          mine = wb + lane < u.nblk ? trow[wb + lane] : 0;
-        }
-        int phys0 = __shfl_sync(kFull, mine, jb0 - wb);
-        int phys1 = __shfl_sync(kFull, mine, min(jb0 + 1 - wb, 31));
+      const int ybase = u.g * BS;
+      for (int wb = 0; wb < u.nblk && ok; wb += 32) {
+        tab[lane] = wb + lane < u.nblk ? trow[wb + lane] : 0;
+        __syncwarp();
         if (lane == 0) {
-          const int s = c % NS;
-          const uint32_t r = c / NS;
-          ok = mbar_wait(smem_addr(empty + s), (r & 1) ^ 1, abort_flag);
-          if (ok) {
+          const int k_end = min(nch, ((wb + 32) << bs_shift) >> 4);
+          for (int k = (wb << bs_shift) >> 4; k < k_end; ++k) {
+            if (!mbar_wait(smem_addr(empty + s), ph ^ 1, abort_flag)) {
+              record_error(PKV_ERR_DEVICE_TIMEOUT);
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
+            const int jb = (k << 4) >> bs_shift;  // unit-relative block of the chunk
+            const int nb_here = BS == 8 ? min(2, u.nblk - jb) : 1;
+            const int row0 = BS == 32 ? (k & 1) << 4 : 0;
             const uint32_t bar = smem_addr(full + s);
             const uint32_t kdst = ring_s + s * L::kStageBytes;
-            const uint32_t vdst = kdst + L::kTileBytes;
-            const int row_in_block = BS > kChunkTokens ? (k * kChunkTokens) % BS : 0;
-            mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nb_here * box_rows * D * 2 * 2));
+            mbar_arrive_expect_tx(bar, nb_here * 2 * box_bytes);
             for (int i = 0; i < nb_here; ++i) {
-              int phys = i == 0 ? phys0 : phys1;
+              int phys = tab[jb - wb + i];
               if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_blocks)) {
                 record_error(PKV_ERR_BAD_BLOCK);
                 phys = 0;
               }
-              const int32_t y = (phys * p.num_kv_heads + u.g) * BS + row_in_block;
-#pragma unroll
-              for (int h = 0; h < L::kHalves; ++h) {
-                const uint32_t off = h * L::kHalfBytes + i * box_rows * 128;
-                tma_load_2d(kdst + off, &tmap_k, 64 * h, y, bar, policy);
-                tma_load_2d(vdst + off, &tmap_v, 64 * h, y, bar, policy);
-              }
+              const int32_t y = phys * p.num_kv_heads * BS + ybase + row0;
+              tma_load_3d(kdst + i * blk_off, &tmap_k, 0, y, 0, bar, policy);
+              tma_load_3d(kdst + L::kTileBytes + i * blk_off, &tmap_v, 0, y, 0, bar, policy);
             }
-          } else {
-            record_error(PKV_ERR_DEVICE_TIMEOUT);
-            *abort_flag = 1;
+            ++issued;
+            if (++s == NS) {
+              s = 0;
+              ph ^= 1;
+            }
           }
         }
+        __syncwarp();
         ok = __shfl_sync(kFull, ok, 0);
-        if (!ok) break;
       }
     }
-    // No copy may still be landing in shared memory when the CTA exits.
-    __syncwarp();
+    // No copy may still be landing in shared memory when the CTA exits: wait
+    // (bounded) for the last phase issued into every stage.
     if (lane == 0) {
-      for (int s = 0; s < NS && s < static_cast<int>(c); ++s) {
-        const uint32_t last_round = (c - 1 - s) / NS;
+      for (int st = 0; st < NS && st < static_cast<int>(issued); ++st) {
+        const uint32_t uses = (issued - st + NS - 1) / NS;
         const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(smem_addr(full + s), last_round & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
+        while (!mbar_try_wait(smem_addr(full + st), (uses - 1) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
         }
       }
     }
@@ -159,10 +170,17 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
   // ------------------------------ consumers ------------------------------
   const int gq = lane >> 2;  // fragment row group: token (S^T) / dim (O^T) / head (B operands)
   const int tq = lane & 3;   // fragment column pair: heads 2tq, 2tq+1
-  // lanes that feed ldmatrix rows
-  const int ld_row_a = (lane & 7) + ((lane >> 3) & 1) * 8, ld_col_a = lane >> 4;  // K (A = K chunk)
-  const int ld_row_v = (lane & 7) + (lane >> 4) * 8, ld_col_v = (lane >> 3) & 1;  // V (A = V^T, .trans)
-  const int src0 = 4 * (2 * tq) + (gq >> 1), src1 = src0 + 4;  // P^T transpose sources
+  // ldmatrix row addresses of this lane: K chunk (A operand) and V chunk (A = Vᵀ via .trans)
+  const int ra = (lane & 7) + ((lane >> 3) & 1) * 8, ca = lane >> 4;
+  const int rv = (lane & 7) + (lane >> 4) * 8, cv = (lane >> 3) & 1;
+  uint32_t offa[kHalves], offv[kHalves];
+#pragma unroll
+  for (int h = 0; h < kHalves; ++h) {
+    offa[h] = row_offset(ra, h, br_shift, kHalves);
+    offv[h] = row_offset(rv, h, br_shift, kHalves);
+  }
+  const int xa = ra & 7, xv = rv & 7;
+  const int src0 = 4 * (2 * tq) + (gq >> 1), src1 = src0 + 4;  // Pᵀ transpose sources
   const uint32_t sel = (gq & 1) ? 0x7632u : 0x5410u;
   const float sl = p.scale_log2;
   uint32_t c = 0;
@@ -188,10 +206,10 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // heads 2tq, 2tq+1
 
     const int k0 = (warp - static_cast<int>(c % kConsumerWarps) + kConsumerWarps) % kConsumerWarps;
+    int s = (c + k0) % NS;
+    uint32_t ph = ((c + k0) / NS) & 1;
     for (int k = k0; k < nch && ok; k += kConsumerWarps) {
-      const uint32_t cc = c + k;
-      const int s = cc % NS;
-      const bool landed = __all_sync(kFull, mbar_wait(smem_addr(full + s), (cc / NS) & 1, abort_flag));
+      const bool landed = __all_sync(kFull, mbar_wait(smem_addr(full + s), ph, abort_flag));
       if (!landed) {
         if (lane == 0) {
           record_error(PKV_ERR_DEVICE_TIMEOUT);
@@ -209,7 +227,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
 #pragma unroll
       for (int ks = 0; ks < kSteps; ++ks) {
         uint32_t a[4];
-        ldmatrix_x4(kbase + (ks / 4) * L::kHalfBytes + swz(ld_row_a, 2 * (ks % 4) + ld_col_a), a);
+        ldmatrix_x4(kbase + offa[ks / 4] + (((2 * (ks % 4) + ca) ^ xa) << 4), a);
         mma_16816<T>(sc, a, qb[ks][0], qb[ks][1]);
       }
       const bool v0 = gq < nv, v1 = gq + 8 < nv;  // tokens gq and gq + 8 of the chunk
@@ -255,11 +273,11 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
 
       // ---- rows past the sequence end: zero V so stale values cannot reach P·V ----
       if (nv < kChunkTokens) {
-        const int per_row = 8 * L::kHalves;
+        const int per_row = 8 * kHalves;
         const int total = (kChunkTokens - nv) * per_row;
         for (int i = lane; i < total; i += 32) {
           const int row = nv + i / per_row, rem = i % per_row;
-          const uint32_t addr = vbase + (rem / 8) * L::kHalfBytes + row * 128 + (rem % 8) * 16;
+          const uint32_t addr = vbase + row_offset(row, rem / 8, br_shift, kHalves) + (rem % 8) * 16;
           asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0) : "memory");
         }
         __syncwarp();
@@ -269,13 +287,18 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
 #pragma unroll
       for (int mt = 0; mt < kSteps; ++mt) {
         uint32_t a[4];
-        ldmatrix_x4_trans(vbase + (mt / 4) * L::kHalfBytes + swz(ld_row_v, 2 * (mt % 4) + ld_col_v), a);
+        ldmatrix_x4_trans(vbase + offv[mt / 4] + (((2 * (mt % 4) + cv) ^ xv) << 4), a);
         mma_16816<T>(acc[mt], a, bh0, bh1);
         mma_16816<T>(acc[mt], a, bl0, bl1);
       }
       if (nv < kChunkTokens) fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_addr(empty + s));
+      s += kConsumerWarps;
+      if (s >= NS) {
+        s -= NS;
+        ph ^= 1;
+      }
     }
     c += nch;
 

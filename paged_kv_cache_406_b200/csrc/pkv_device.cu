@@ -207,16 +207,20 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Pool viewed as a 2-D tensor [rows = num_blocks * Hkv * block_size][head_dim]
-// of 16-bit elements; boxes of 64 elements (128 B) x box_rows, 128-byte swizzle.
+// Pool viewed as a 3-D tensor of 16-bit elements: x = 64 elements (one 128-byte
+// column half), y = token row (num_blocks * Hkv * block_size rows, head_dim * 2
+// bytes apart), z = column half (head_dim / 64 of them, 128 bytes apart).  A
+// box of 64 x box_rows x halves lands in shared memory as [half][row][128 B]
+// with 128-byte swizzle.
 int make_pool_map(CUtensorMap* m, const void* pool, int dtype, int64_t rows, int head_dim, int box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * 2};
-  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
-  const cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+  const cuuint32_t halves = static_cast<cuuint32_t>(head_dim / 64);
+  const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), halves};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2, 128};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), halves};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
                    const_cast<void*>(pool), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
