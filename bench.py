@@ -269,8 +269,7 @@ def run_ours(args):
                                      out=out, workspace=workspace, partition_tokens=w.partition_tokens)
         if ev is not None:
             ev[1].record()
-        pt = w.partition_tokens or 256
-        n += 2 + (1 if int(st["lens_host"].max()) > pt else 0)  # plan + decode (+ merge)
+        n += 2  # plan + decode (partition merge runs inside the decode kernel)
         return n
 
     for i in range(args.warmup):
@@ -394,7 +393,7 @@ def run_ours(args):
                        "l2": "inputs larger than L2: %.0f MB of K/V read per step vs 126 MB L2, no flush"
                              % (np.mean(step_kv) / 1e6),
                        "parallelism": f"replicas x{ws} (independent batches per GPU)"},
-            "roofline": {"kernel": "pkv_paged_attention_decode (plan + attention + merge kernels)",
+            "roofline": {"kernel": "pkv_paged_attention_decode (plan + decode kernels)",
                          "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
                          "traffic": traffic, "algorithmic_bytes_per_launch": int(np.mean(step_algo)),

@@ -17,8 +17,9 @@
 //                  mbarriers; four consumer warps take every fourth block and
 //                  keep their own online softmax state (running max m, sum l,
 //                  fp32 accumulator), and merge at the end of the unit;
-//   reduce kernel  merges the per-partition (m, l, o) of sequences that were
-//                  split, with the max/sum rescaling
+//   merge kernel   for sequences that were split, one warp per (sequence,
+//                  query head) merges the per-partition (m, l, o) with the
+//                  max/sum rescaling
 //                      out = Σ_p 2^(m_p-M) o_p / Σ_p 2^(m_p-M) l_p.
 // Scores are kept in log2 units (q is pre-multiplied by scale·log2 e).  The
 // running max is only moved when a new score exceeds it by more than
@@ -57,6 +58,9 @@ struct DecodeParams {
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ seq_lens, int32_t num_seqs,
                                                     int32_t max_tokens, int32_t part_tokens, int32_t block_size,
                                                     int4* __restrict__ items, int32_t* __restrict__ n_items) {
+  // the decode grid may be scheduled now; it waits for this grid's results
+  // (griddepcontrol.wait) before reading them
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ int32_t hist[];  // [kmax + 1] counts, then [kmax + 1] cursors
   const int kmax = part_tokens / block_size;
   int32_t* cursor = hist + kmax + 1;
@@ -205,9 +209,9 @@ __device__ __forceinline__ WorkUnit load_unit(const DecodeParams& p, int w) {
 // Final merge of one work unit: the kConsumerWarps per-warp records in `rec`
 // (acc[G][D], m[G], l[G] each, taken against each warp's own running max)
 // are rescaled to their common max and either normalised into `out` (the
-// sequence has one partition) or stored as the partition's (m, l, o) partial.
-// Called by the consumer threads (0 .. kConsumerWarps*32-1) after the named
-// barrier that publishes the records.
+// sequence has one partition) or stored as the partition's (m, l, o) partial
+// for merge_kernel.  Called by the consumer threads (0 .. kConsumerWarps*32-1)
+// after the named barrier that publishes the records.
 template <int G, int D>
 __device__ __forceinline__ void merge_store(const float* rec, const WorkUnit& u, const DecodeParams& p) {
   constexpr int kMF = G * D + 2 * G;
@@ -247,7 +251,9 @@ struct DecodeSmem {
   static constexpr int kMergeFloats = G * D + 2 * G;  // acc[G][D], m[G], l[G]
   __host__ __device__ static size_t ring_bytes(int bs, int ns) { return size_t(ns) * 2 * bs * D * sizeof(T); }
   __host__ __device__ static size_t bytes(int bs, int ns) {
-    return ring_bytes(bs, ns) + 2 * kConsumerWarps * kMergeFloats * sizeof(float) + 2 * ns * sizeof(uint64_t) + 16;
+    // + 16: abort and merge flags; + 128: the producer's window of 32 block-table entries
+    return ring_bytes(bs, ns) + 2 * kConsumerWarps * kMergeFloats * sizeof(float) + 2 * ns * sizeof(uint64_t) + 16 +
+           128;
   }
 };
 
@@ -268,6 +274,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
   uint64_t* full = reinterpret_cast<uint64_t*>(merge + 2 * kConsumerWarps * kMF);
   uint64_t* empty = full + NS;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + NS);
+  int32_t* tab = reinterpret_cast<int32_t*>(empty + NS) + 4;  // 32 block-table entries
   const uint32_t ring_s = smem_addr(smem);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -280,58 +287,66 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
     fence_mbar_init();
   }
   __syncthreads();
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the plan kernel's work list is complete
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // let merge_kernel be scheduled
 
   const int n_work = *p.n_items * p.num_kv_heads;
   const int Hq = p.num_q_heads;
 
   if (warp == kConsumerWarps) {
     // ----------------------------- producer -----------------------------
+    // All lanes walk the units and refill a 32-entry block-table window in
+    // shared memory; lane 0 alone issues the window's blocks (no warp-wide
+    // synchronisation on the per-block path).
     const uint64_t policy = l2_evict_first_policy();
     const unsigned char* kbase = static_cast<const unsigned char*>(p.k_pool);
     const unsigned char* vbase = static_cast<const unsigned char*>(p.v_pool);
-    uint32_t c = 0;
+    int s = 0;
+    uint32_t ph = 0, issued = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < n_work && ok; w += gridDim.x) {
       const WorkUnit u = load_unit(p, w);
       const int32_t* trow = p.block_tables + static_cast<int64_t>(u.b) * p.max_blocks + u.t0 / BS;
       for (int jb = 0; jb < u.nblk && ok; jb += 32) {
-        const int cnt = min(32, u.nblk - jb);
-        const int mine = lane < cnt ? trow[jb + lane] : 0;
-        for (int j = 0; j < cnt; ++j, ++c) {
-          int phys = __shfl_sync(kFull, mine, j);
-          if (lane == 0) {
-            const int s = c % NS;
-            const uint32_t r = c / NS;
-            ok = mbar_wait(smem_addr(empty + s), (r & 1) ^ 1, abort_flag);
-            if (ok) {
-              if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_blocks)) {
-                record_error(PKV_ERR_BAD_BLOCK);
-                phys = 0;
-              }
-              const size_t off = (static_cast<size_t>(phys) * p.num_kv_heads + u.g) * tile_bytes;
-              const uint32_t bar = smem_addr(full + s);
-              mbar_arrive_expect_tx(bar, stage_bytes);
-              bulk_g2s(ring_s + s * stage_bytes, kbase + off, tile_bytes, bar, policy);
-              bulk_g2s(ring_s + s * stage_bytes + tile_bytes, vbase + off, tile_bytes, bar, policy);
-            } else {
+        tab[lane] = jb + lane < u.nblk ? trow[jb + lane] : 0;
+        __syncwarp();
+        if (lane == 0) {
+          const int cnt = min(32, u.nblk - jb);
+          for (int j = 0; j < cnt; ++j) {
+            if (!mbar_wait(smem_addr(empty + s), ph ^ 1, abort_flag)) {
               record_error(PKV_ERR_DEVICE_TIMEOUT);
               *abort_flag = 1;
+              ok = false;
+              break;
+            }
+            int phys = tab[j];
+            if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_blocks)) {
+              record_error(PKV_ERR_BAD_BLOCK);
+              phys = 0;
+            }
+            const size_t off = (static_cast<size_t>(phys) * p.num_kv_heads + u.g) * tile_bytes;
+            const uint32_t bar = smem_addr(full + s);
+            mbar_arrive_expect_tx(bar, stage_bytes);
+            bulk_g2s(ring_s + s * stage_bytes, kbase + off, tile_bytes, bar, policy);
+            bulk_g2s(ring_s + s * stage_bytes + tile_bytes, vbase + off, tile_bytes, bar, policy);
+            ++issued;
+            if (++s == NS) {
+              s = 0;
+              ph ^= 1;
             }
           }
-          ok = __shfl_sync(kFull, ok, 0);
-          if (!ok) break;
         }
+        __syncwarp();
+        ok = __shfl_sync(kFull, ok, 0);
       }
     }
     // Before the CTA exits no copy may still be landing in its shared memory:
-    // wait (bounded) for the last copy issued into every stage.
-    __syncwarp();
+    // wait (bounded) for the last phase issued into every stage.
     if (lane == 0) {
-      const uint32_t issued = c;  // blocks issued (a failed wait issued nothing)
-      for (int s = 0; s < NS && s < static_cast<int>(issued); ++s) {
-        const uint32_t last_round = (issued - 1 - s) / NS;
+      for (int st = 0; st < NS && st < static_cast<int>(issued); ++st) {
+        const uint32_t uses = (issued - st + NS - 1) / NS;
         const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(smem_addr(full + s), last_round & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
+        while (!mbar_try_wait(smem_addr(full + st), (uses - 1) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
         }
       }
     }
@@ -377,10 +392,10 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
     float m_own = -INFINITY, l_own = 0.f;
 
     const int j0 = (warp - static_cast<int>(c % kConsumerWarps) + kConsumerWarps) % kConsumerWarps;
+    int s = (c + j0) % NS;
+    uint32_t ph = ((c + j0) / NS) & 1;
     for (int j = j0; j < u.nblk && ok; j += kConsumerWarps) {
-      const uint32_t cc = c + j;
-      const int s = cc % NS;
-      const bool landed = __all_sync(kFull, mbar_wait(smem_addr(full + s), (cc / NS) & 1, abort_flag));
+      const bool landed = __all_sync(kFull, mbar_wait(smem_addr(full + s), ph, abort_flag));
       if (!landed) {
         if (lane == 0) {
           record_error(PKV_ERR_DEVICE_TIMEOUT);
@@ -456,6 +471,11 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_addr(empty + s));
+      s += kConsumerWarps;
+      if (s >= NS) {
+        s -= NS;
+        ph ^= 1;
+      }
     }
     c += u.nblk;
 
@@ -494,52 +514,74 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
 }
 
 // ---------------------------------------------------------------------------
-// reduce: merge the partitions of split sequences; one warp per (seq, q head)
+// merge: partitions of split sequences; one warp per (sequence, query head).
+// Lanes first hold the rescale weight 2^(m_p - M) and l_p of 32 partitions
+// each; the weighted rows o_p are then summed with several partitions' loads
+// in flight.  Launched with programmatic serialisation after the decode
+// kernel: it waits (griddepcontrol.wait) for all partials before reading.
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(256) reduce_kernel(const int32_t* __restrict__ seq_lens, int32_t num_seqs,
-                                                     int32_t num_q_heads, int32_t max_tokens, int32_t part_tokens,
-                                                     int32_t max_parts, const float* __restrict__ part_m,
-                                                     const float* __restrict__ part_l,
-                                                     const float* __restrict__ part_o, float* __restrict__ out) {
-  constexpr int kPer = D / 32;
+__global__ void __launch_bounds__(256) merge_kernel(const int32_t* __restrict__ seq_lens, int32_t num_seqs,
+                                                    int32_t num_q_heads, int32_t max_tokens, int32_t part_tokens,
+                                                    int32_t max_parts, const float* __restrict__ part_m,
+                                                    const float* __restrict__ part_l,
+                                                    const float* __restrict__ part_o, float* __restrict__ out) {
+  constexpr int kPer = D / 32;  // output columns per lane
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= num_seqs * num_q_heads) return;
   const int b = row / num_q_heads;
   int L = seq_lens[b];
   L = L < 0 ? 0 : (L > max_tokens ? max_tokens : L);
-  if (L <= part_tokens) return;  // written directly by the decode kernel
+  if (L <= part_tokens) return;  // one partition: written by the decode kernel
   const int np = (L + part_tokens - 1) / part_tokens;
   const int64_t base = static_cast<int64_t>(row) * max_parts;
   float M = -INFINITY;
-  for (int p = lane; p < np; p += 32) M = fmaxf(M, part_m[base + p]);
+  for (int q = lane; q < np; q += 32) M = fmaxf(M, part_m[base + q]);
 #pragma unroll
   for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
-  float num[kPer];
+  float acc[kPer];
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) num[i] = 0.f;
+  for (int i = 0; i < kPer; ++i) acc[i] = 0.f;
   float den = 0.f;
-  for (int p = 0; p < np; ++p) {
-    const float f = fast_exp2(part_m[base + p] - M);
-    den += f * part_l[base + p];
-    const float* o = part_o + (base + p) * D + lane * kPer;
-    if constexpr (kPer == 4) {
-      const float4 v = *reinterpret_cast<const float4*>(o);
-      num[0] += f * v.x;
-      num[1] += f * v.y;
-      num[2] += f * v.z;
-      num[3] += f * v.w;
-    } else {
-      const float2 v = *reinterpret_cast<const float2*>(o);
-      num[0] += f * v.x;
-      num[1] += f * v.y;
+  for (int q0 = 0; q0 < np; q0 += 32) {
+    const int nq = min(32, np - q0);
+    const float f_mine = lane < nq ? fast_exp2(part_m[base + q0 + lane] - M) : 0.f;
+    den += lane < nq ? f_mine * part_l[base + q0 + lane] : 0.f;
+    const float* o = part_o + (base + q0) * D + lane * kPer;
+    int j = 0;
+    for (; j + 4 <= nq; j += 4) {
+      float v[4][kPer];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        if constexpr (kPer == 4) {
+          const float4 x = *reinterpret_cast<const float4*>(o + (j + t) * D);
+          v[t][0] = x.x; v[t][1] = x.y; v[t][2] = x.z; v[t][3] = x.w;
+        } else {
+          const float2 x = *reinterpret_cast<const float2*>(o + (j + t) * D);
+          v[t][0] = x.x; v[t][1] = x.y;
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float f = __shfl_sync(kFull, f_mine, j + t);
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) acc[i] += f * v[t][i];
+      }
+    }
+    for (; j < nq; ++j) {
+      const float f = __shfl_sync(kFull, f_mine, j);
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) acc[i] += f * o[j * D + i];
     }
   }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(kFull, den, o);
   const float inv = den > 0.f ? 1.f / den : 0.f;
   float* dst = out + static_cast<int64_t>(row) * D + lane * kPer;
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) dst[i] = num[i] * inv;
+  for (int i = 0; i < kPer; ++i) dst[i] = acc[i] * inv;
 }
 
 }  // namespace pkv

@@ -92,6 +92,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
     fence_mbar_init();
   }
   __syncthreads();
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the plan kernel's work list is complete
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // let merge_kernel be scheduled
 
   const int n_work = *p.n_items * p.num_kv_heads;
 

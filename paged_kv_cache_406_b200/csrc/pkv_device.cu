@@ -1,5 +1,6 @@
 // Device entry points of libpagedkv (sm_100a): KV append, block copy,
-// PagedAttention decode (plan + decode + reduce) and the device status word.
+// PagedAttention decode (plan, decode and partition-merge kernels) and the
+// device status word.
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -122,11 +123,13 @@ struct WsLayout {
   size_t items, m, l, o, total;  // byte offsets; n_items lives at offset 0
 };
 
-WsLayout ws_layout(int64_t num_seqs, int64_t num_q_heads, int64_t head_dim, int64_t max_tokens, int32_t pt) {
+WsLayout ws_layout(int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim, int64_t max_tokens,
+                   int32_t pt) {
   WsLayout w;
   w.max_parts = static_cast<int32_t>(std::max<int64_t>(1, (max_tokens + pt - 1) / pt));
   const int64_t rows = num_seqs * num_q_heads * w.max_parts;
   w.items = 256;
+  (void)num_kv_heads;
   w.m = w.items + round256(num_seqs * w.max_parts * sizeof(int4));
   w.l = w.m + round256(rows * sizeof(float));
   w.o = w.l + round256(rows * sizeof(float));
@@ -139,6 +142,49 @@ int ring_stages(size_t stage_bytes) {
   int ns = static_cast<int>((64 * 1024) / stage_bytes);
   ns = std::max(pkv::kConsumerWarps, std::min(16, ns));
   return ns - ns % pkv::kConsumerWarps;
+}
+
+// Launches `kern` with programmatic stream serialisation: the grid may be
+// scheduled while the previous kernel in the stream runs; it waits for that
+// kernel's results with griddepcontrol.wait before reading them.
+template <typename Kernel, typename... Args>
+cudaError_t launch_pdl(Kernel kern, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+// plan kernel -> decode kernel -> merge kernel (the last only when some
+// sequence can span more than one partition)
+template <int D, typename Kernel, typename... Args>
+int launch_plan_decode_merge(const pkv::DecodeParams& p, const int32_t* seq_lens, int32_t num_seqs,
+                             int32_t max_tokens, Kernel kern, int grid, size_t smem, cudaStream_t stream,
+                             Args... args) {
+  const int kmax = p.partition_tokens / p.block_size;
+  pkv::plan_kernel<<<1, 1024, 2 * (kmax + 1) * sizeof(int32_t), stream>>>(
+      seq_lens, num_seqs, max_tokens, p.partition_tokens, p.block_size, const_cast<int4*>(p.items),
+      const_cast<int32_t*>(p.n_items));
+  cudaError_t e = launch_pdl(kern, dim3(grid), dim3(pkv::kDecodeThreads), smem, stream, p, args...);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  if (p.max_parts > 1) {
+    const int rows = num_seqs * p.num_q_heads;
+    e = launch_pdl(pkv::merge_kernel<D>, dim3((rows + 7) / 8), dim3(256), 0, stream, seq_lens, num_seqs,
+                   p.num_q_heads, max_tokens, p.partition_tokens, p.max_parts,
+                   static_cast<const float*>(p.part_m), static_cast<const float*>(p.part_l),
+                   static_cast<const float*>(p.part_o), p.out);
+    if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return pkv::ok();
 }
 
 template <typename T, int D, int G>
@@ -171,22 +217,9 @@ int launch_decode(const pkv::DecodeParams& base, const int32_t* seq_lens, int32_
     if (dev < kMaxDevices) occ_cache[dev][bs_idx].store(occ, std::memory_order_relaxed);
   }
 
-  const int kmax = p.partition_tokens / p.block_size;
-  pkv::plan_kernel<<<1, 1024, 2 * (kmax + 1) * sizeof(int32_t), stream>>>(
-      seq_lens, num_seqs, max_tokens, p.partition_tokens, p.block_size, const_cast<int4*>(p.items),
-      const_cast<int32_t*>(p.n_items));
   const int64_t work_upper = int64_t(num_seqs) * p.max_parts * p.num_kv_heads;
   const int grid = static_cast<int>(std::min<int64_t>(int64_t(sm_count(dev)) * occ, work_upper));
-  kern<<<grid, pkv::kDecodeThreads, smem, stream>>>(p);
-  if (p.max_parts > 1) {
-    const int rows = num_seqs * p.num_q_heads;
-    pkv::reduce_kernel<D><<<(rows + 7) / 8, 256, 0, stream>>>(seq_lens, num_seqs, p.num_q_heads, max_tokens,
-                                                              p.partition_tokens, p.max_parts, p.part_m, p.part_l,
-                                                              p.part_o, p.out);
-  }
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-  return pkv::ok();
+  return launch_plan_decode_merge<D>(p, seq_lens, num_seqs, max_tokens, kern, grid, smem, stream);
 }
 
 // ---- tensor maps over the K/V pools for the tensor-core kernel ----
@@ -285,22 +318,9 @@ int launch_decode_mma(const pkv::DecodeParams& base, const int32_t* seq_lens, in
   rc = pool_map(&mv, p.v_pool, dtype, rows, D, box_rows);
   if (rc) return rc;
 
-  const int kmax = p.partition_tokens / p.block_size;
-  pkv::plan_kernel<<<1, 1024, 2 * (kmax + 1) * sizeof(int32_t), stream>>>(
-      seq_lens, num_seqs, max_tokens, p.partition_tokens, p.block_size, const_cast<int4*>(p.items),
-      const_cast<int32_t*>(p.n_items));
   const int64_t work_upper = int64_t(num_seqs) * p.max_parts * p.num_kv_heads;
   const int grid = static_cast<int>(std::min<int64_t>(int64_t(sm_count(dev)) * occ, work_upper));
-  kern<<<grid, pkv::kDecodeThreads, smem, stream>>>(p, mk, mv);
-  if (p.max_parts > 1) {
-    const int rows_out = num_seqs * p.num_q_heads;
-    pkv::reduce_kernel<D><<<(rows_out + 7) / 8, 256, 0, stream>>>(seq_lens, num_seqs, p.num_q_heads, max_tokens,
-                                                                  p.partition_tokens, p.max_parts, p.part_m,
-                                                                  p.part_l, p.part_o, p.out);
-  }
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "decode_mma launch");
-  return pkv::ok();
+  return launch_plan_decode_merge<D>(p, seq_lens, num_seqs, max_tokens, kern, grid, smem, stream, mk, mv);
 }
 
 template <typename T>
@@ -384,7 +404,7 @@ extern "C" int pkv_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, 
   int32_t pt = 0;
   int rc = resolve_partition(partition_tokens, block_size, &pt);
   if (rc) return rc;
-  *bytes = ws_layout(num_seqs, num_q_heads, head_dim, int64_t(max_blocks_per_seq) * block_size, pt).total;
+  *bytes = ws_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, int64_t(max_blocks_per_seq) * block_size, pt).total;
   return pkv::ok();
 }
 
@@ -420,7 +440,7 @@ extern "C" int pkv_paged_attention_decode(const void* q, const void* k_pool, con
     return fail(PKV_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", fn);
   const int64_t max_tokens = int64_t(max_blocks_per_seq) * block_size;
   if (max_tokens > (int64_t(1) << 30)) return fail(PKV_ERR_INVALID_ARG, "%s: max_blocks_per_seq too large", fn);
-  const WsLayout w = ws_layout(num_seqs, num_q_heads, head_dim, max_tokens, pt);
+  const WsLayout w = ws_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_tokens, pt);
   if (workspace_bytes < w.total)
     return fail(PKV_ERR_INVALID_ARG, "%s: workspace %zu bytes < %zu needed", fn, workspace_bytes, w.total);
 
