@@ -41,23 +41,25 @@ STAGED_STEPS = 16  # distinct steps of metadata resident on the device, cycled
 # from the ncu capture summarised in profiles/ (dram__bytes_read.sum +
 # dram__bytes_write.sum over its kernels).  Valid only while the kernel
 # sources hash to TRAFFIC_SOURCE_SHA; otherwise reported as null.
-TRAFFIC_BYTES = None
-TRAFFIC_SOURCE_SHA = None
+TRAFFIC_BYTES = 607263488  # plan + decode + merge kernels, mean of two captured calls
+TRAFFIC_SOURCE_SHA = "62c7be410db53362"
 
 
 def kernel_source_sha() -> str:
+    """Hash of the device sources (every .cu / .cuh file of the library)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_406_b200", "csrc")
-    for name in ("decode.cuh", "device_common.cuh", "pkv_device.cu"):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(f.read())
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=8000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama3_8b")
@@ -74,6 +76,25 @@ def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return ws, rank, local
+
+
+def combine_ranks(elapsed_ms: float, nbytes: float, ntokens: float, device) -> tuple:
+    """Whole-job totals over the ranks of the default process group: the
+    slowest rank's time (max), and the sums of bytes and tokens processed."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return elapsed_ms, nbytes, ntokens
+    mx = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+    sm = torch.tensor([nbytes, ntokens], dtype=torch.float64, device=device)
+    dist.all_reduce(sm, op=dist.ReduceOp.SUM)
+    return float(mx[0]), float(sm[0]), float(sm[1])
+
+
+def rank_workload(w, rank: int):
+    """Rank r runs its own batch of the same shape (weak scaling): seeds offset by 1000·r."""
+    from dataclasses import replace
+    return replace(w, seed=w.seed + 1000 * rank) if rank else w
 
 
 def measured_peaks():
@@ -187,13 +208,11 @@ def make_units(w, k_pool, v_pool, tables, lens, q, order, count):
 
 
 # ---------------------------------------------------------------------------
-def setup(w, device, horizon, seed_offset=0):
+def setup(w, device, horizon):
     """Pools, allocator and admitted batch; ``horizon`` = tokens each sequence
     may still gain (staged + end-to-end steps), covered by pool and tables."""
     from paged_kv_cache_406_b200 import workloads as W
     from paged_kv_cache_406_b200.cache import PagedKVCache
-    from dataclasses import replace
-    w = replace(w, seed=w.seed + seed_offset) if seed_offset else w
     lens = W.seq_lens(w)
     nb = W.pool_blocks(w, lens + horizon)
     shape = (nb, w.num_kv_heads, w.block_size, w.head_dim)
@@ -223,7 +242,7 @@ def run_ours(args):
         from dataclasses import replace
         w0 = replace(w0, partition_tokens=args.partition_tokens)
     horizon = STAGED_STEPS + 3 + max(0, args.e2e_steps) + 8
-    w, cache, lens0 = setup(w0, dev, horizon, seed_offset=1000 * rank)
+    w, cache, lens0 = setup(rank_workload(w0, rank), dev, horizon)
     B, hq, hkv, d, bs = w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size
     esz = torch.tensor([], dtype=w.torch_dtype).element_size()
     ids = list(range(B))
@@ -248,10 +267,14 @@ def run_ours(args):
     def kv_bytes(lens):
         return int(lens.astype(np.int64).sum()) * hkv * d * 2 * esz
 
+    pt_eff = w.partition_tokens or 512
+
     def algo_bytes(lens):
-        # KV rows once per (sequence, KV head) + block-table entries + q + out
+        # K/V rows once per (sequence, KV head) + block-table entries + q + out,
+        # + the split-partition partials (m, l, o per query head), written once and read once
         tab = int(sum(-(-int(L) // bs) for L in lens)) * 4
-        return kv_bytes(lens) + tab + B * hq * d * esz + B * hq * d * 4
+        parts = int(sum(-(-int(L) // pt_eff) for L in lens if L > pt_eff))
+        return kv_bytes(lens) + tab + B * hq * d * esz + B * hq * d * 4 + 2 * parts * hq * (d + 2) * 4
 
     launches_per = []
 
@@ -302,15 +325,7 @@ def run_ours(args):
     step_kv = [kv_bytes(staged[(args.warmup + i) % STAGED_STEPS]["lens_host"]) for i in range(K)]
     step_algo = [algo_bytes(staged[(args.warmup + i) % STAGED_STEPS]["lens_host"]) for i in range(K)]
     my_bytes = float(sum(step_kv))
-    t = torch.tensor([elapsed_ms, my_bytes, float(B * K)], dtype=torch.float64, device=dev)
-    if ws > 1:
-        mx = t[:1].clone()
-        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
-        sm = t[1:].clone()
-        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
-        elapsed_all, bytes_all, tokens_all = float(mx[0]), float(sm[0]), float(sm[1])
-    else:
-        elapsed_all, bytes_all, tokens_all = elapsed_ms, my_bytes, float(B * K)
+    elapsed_all, bytes_all, tokens_all = combine_ranks(elapsed_ms, my_bytes, float(B * K), dev)
     value = bytes_all / (elapsed_all * 1e-3) / 1e9
     tok_s = tokens_all / (elapsed_all * 1e-3)
 
@@ -350,21 +365,18 @@ def run_ours(args):
         e1.record()
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
-        te = torch.tensor([e2e_ms, float(sum(e_lens))], dtype=torch.float64, device=dev)
-        if ws > 1:
-            mx = te[:1].clone()
-            dist.all_reduce(mx, op=dist.ReduceOp.MAX)
-            sm = te[1:].clone()
-            dist.all_reduce(sm, op=dist.ReduceOp.SUM)
-            e2e_ms_all, e2e_bytes_all = float(mx[0]), float(sm[0])
-        else:
-            e2e_ms_all, e2e_bytes_all = e2e_ms, float(sum(e_lens))
+        e2e_ms_all, e2e_bytes_all, _ = combine_ranks(e2e_ms, float(sum(e_lens)), float(B * E), dev)
         h2d = (B * hq * d + 2 * B * hkv * d) * esz + meta_bytes // E
         e2e = {"value": round(e2e_bytes_all / (e2e_ms_all * 1e-3) / 1e9, 2), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(B * hq * d * 4),
                "ms_per_step": round(e2e_ms_all / E, 4),
                "tokens_per_s_per_layer": round(ws * B * E / (e2e_ms_all * 1e-3), 1),
                "includes": "host slot reservation, pinned H2D of q/K/V rows and metadata, kernels, D2H of out"}
+
+    st_a = cache.stats()
+    alloc_stats = {"used_blocks": st_a["used_blocks"], "free_blocks": st_a["free_blocks"],
+                   "logical_tokens": st_a["logical_tokens"], "waste_tokens": st_a["waste_tokens"],
+                   "waste_frac": round(st_a["waste_tokens"] / max(1, st_a["used_blocks"] * bs), 5)}
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -373,10 +385,12 @@ def run_ours(args):
         st = staged[(args.warmup + K - 1) % STAGED_STEPS]
         units = make_units(w, cache.k_pool, cache.v_pool, st["tables"].cpu().numpy(), st["lens_host"], st["q"],
                            order, count=min(len(order), 64))
-        nbytes, secs, done = time_oracle(units, args.cpu_seconds)
+        cycle = (units[i % len(units)] for i in range(10 ** 9))  # repeat the sample until the budget is spent
+        nbytes, secs, done = time_oracle(cycle, args.cpu_seconds)
         cpu = {"value": round(nbytes / secs / 1e9, 4), "unit": "GB/s", "cores": oracle_threads(),
                "kind": "oracle", "host_cpus": os.cpu_count(),
-               "sample": f"{done} (sequence, KV head) units of the same batch, fp64 numpy oracle, {secs:.1f} s"}
+               "sample": f"{done} (sequence, KV head) units drawn from the same batch (64 distinct, cycled), "
+                         f"fp64 numpy oracle, {secs:.1f} s"}
 
     if rank == 0:
         res = {
@@ -388,17 +402,18 @@ def run_ours(args):
             "config": {"workload": w.name, "num_seqs": B, "num_q_heads": hq, "num_kv_heads": hkv,
                        "head_dim": d, "block_size": bs, "seq_lens": "U[512,4096]" if w.name == "llama3_8b" else "",
                        "mean_seq_len": round(float(np.mean(staged[0]["lens_host"])), 1),
-                       "partition_tokens": w.partition_tokens or 256, "pool_blocks": cache.num_blocks,
+                       "partition_tokens": w.partition_tokens or 512, "pool_blocks": cache.num_blocks,
                        "kv_bytes_per_step": int(np.mean(step_kv)),
                        "l2": "inputs larger than L2: %.0f MB of K/V read per step vs 126 MB L2, no flush"
                              % (np.mean(step_kv) / 1e6),
                        "parallelism": f"replicas x{ws} (independent batches per GPU)"},
-            "roofline": {"kernel": "pkv_paged_attention_decode (plan + decode kernels)",
+            "roofline": {"kernel": "pkv_paged_attention_decode (plan + decode + partition-merge kernels)",
                          "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
                          "traffic": traffic, "algorithmic_bytes_per_launch": int(np.mean(step_algo)),
                          "avg_launch_ms": round(dec_avg_ms, 5), "kernel_source_sha": sha},
             "gpu_launches": launches, "clocks": clk, "cpu_baseline": cpu, "e2e": e2e,
+            "allocator": alloc_stats,
         }
         print(json.dumps(res), flush=True)
     if ws > 1:

@@ -72,7 +72,7 @@ namespace {
 using pkv::fail;
 
 constexpr int kMaxDevices = 64;
-constexpr int kAutoPartitionTokens = 256;
+constexpr int kAutoPartitionTokens = 512;
 constexpr int kMaxPartitionTokens = 8192;
 
 size_t elem_size(int dtype) { return dtype == PKV_F32 ? 4 : 2; }

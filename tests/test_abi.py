@@ -45,10 +45,12 @@ def _ws(native, *args):
 
 
 def test_workspace_size_host_only(native):
-    rc, a = _ws(native, 64, 32, 8, 128, 257, 16, 0)
+    rc, a = _ws(native, 64, 32, 8, 128, 257, 16, 256)
     assert rc == 0 and a > 0
     rc, b = _ws(native, 64, 32, 8, 128, 257, 16, 512)
     assert rc == 0 and b < a  # fewer partitions, smaller partials
+    rc, c = _ws(native, 64, 32, 8, 128, 257, 16, 0)  # automatic: 512-token partitions
+    assert rc == 0 and c == b
     rc, _ = _ws(native, 64, 32, 8, 128, 257, 16, 100)  # not a multiple of the block size
     assert rc == N.PKV_ERR_INVALID_ARG
     rc, _ = _ws(native, -1, 32, 8, 128, 257, 16, 0)

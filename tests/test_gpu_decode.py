@@ -38,7 +38,7 @@ def _decode(case: Case, pt=0, lens=None):
 
 
 def _ragged(bs):
-    return [0, 1, bs - 1, bs, bs + 1, 2 * bs + 3, 100, 255, 256, 257, 511, 512, 513]
+    return [0, 1, bs - 1, bs, bs + 1, 2 * bs + 3, 100, 255, 256, 257, 511, 512, 513, 1025]
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
@@ -53,7 +53,7 @@ def test_decode_matches_oracle(dtype, d, g, bs):
     hkv = 2
     case = Case(_ragged(bs), g * hkv, hkv, d, bs, dtype, seed=zlib.crc32(f"{dtype}{d}{g}{bs}".encode()) % 1000)
     ref = case.oracle()
-    out = _decode(case)  # automatic partitions: the 257..513-token sequences are split
+    out = _decode(case)  # automatic 512-token partitions: the 513- and 1025-token sequences are split
     assert_close(out, ref, dtype, f"{dtype} D{d} G{g} bs{bs}")
 
 
