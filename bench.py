@@ -45,6 +45,16 @@ TRAFFIC_BYTES = 607263488  # plan + decode + merge kernels, mean of two captured
 TRAFFIC_SOURCE_SHA = "62c7be410db53362"
 
 
+SEQ_LEN_RECIPES = {
+    "tiny": "{1,7,16,33} before the step's append",
+    "llama3_8b": "U[512,4096]",
+    "prefix_shared": "1024-token shared prefix (refcount = num_seqs) + U[64,512] tails; KV bytes are logical "
+                     "(the prefix counted once per sequence)",
+    "long_splitk": "7 x 32768 + 1 x 131072",
+    "mha_7b": "lognormal(median 1000, sigma 1) clipped to [16, 8192]",
+}
+
+
 def kernel_source_sha() -> str:
     """Hash of the device sources (every .cu / .cuh file of the library)."""
     h = hashlib.sha256()
@@ -214,15 +224,29 @@ def setup(w, device, horizon):
     from paged_kv_cache_406_b200 import workloads as W
     from paged_kv_cache_406_b200.cache import PagedKVCache
     lens = W.seq_lens(w)
-    nb = W.pool_blocks(w, lens + horizon)
+    nb = W.pool_blocks(w, lens + horizon) + (w.num_seqs if w.prefix_tokens else 0)
     shape = (nb, w.num_kv_heads, w.block_size, w.head_dim)
     k_pool = W.normal(shape, w.torch_dtype, W.pool_seed(w, 0), device=device)
     v_pool = W.normal(shape, w.torch_dtype, W.pool_seed(w, 1), device=device)
     maxb = -(-(int(lens.max()) + horizon) // w.block_size)
     cache = PagedKVCache(nb, w.num_kv_heads, w.head_dim, w.block_size, w.torch_dtype, maxb, device=device,
                          free_order=W.free_order(nb, w.seed), k_pool=k_pool, v_pool=v_pool)
-    for b, L in enumerate(lens):
-        cache.add(b, int(L))
+    if w.prefix_tokens:
+        # one sequence holds the shared prefix, the others fork it (refcount =
+        # num_seqs), then every sequence appends its own tail token by token
+        from paged_kv_cache_406_b200 import pkv_copy_blocks
+        cache.add(0, w.prefix_tokens)
+        for b in range(1, w.num_seqs):
+            cache.fork(0, b)
+        tails = lens - w.prefix_tokens
+        for r in range(int(tails.max())):
+            ids = [b for b in range(w.num_seqs) if tails[b] > r]
+            _, cow = cache.alloc.append_slots(ids)
+            if cow.size:
+                pkv_copy_blocks(cache.k_pool, cache.v_pool, torch.from_numpy(cow).to(device))
+    else:
+        for b, L in enumerate(lens):
+            cache.add(b, int(L))
     return w, cache, lens
 
 
@@ -400,7 +424,7 @@ def run_ours(args):
             "tokens_per_s_per_layer": round(tok_s, 1),
             "hbm_fraction": round(value / peak, 4),
             "config": {"workload": w.name, "num_seqs": B, "num_q_heads": hq, "num_kv_heads": hkv,
-                       "head_dim": d, "block_size": bs, "seq_lens": "U[512,4096]" if w.name == "llama3_8b" else "",
+                       "head_dim": d, "block_size": bs, "seq_lens": SEQ_LEN_RECIPES.get(w.name.split("_bs")[0], ""),
                        "mean_seq_len": round(float(np.mean(staged[0]["lens_host"])), 1),
                        "partition_tokens": w.partition_tokens or 512, "pool_blocks": cache.num_blocks,
                        "kv_bytes_per_step": int(np.mean(step_kv)),

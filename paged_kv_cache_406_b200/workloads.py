@@ -97,15 +97,15 @@ def seq_lens(w: Workload) -> np.ndarray:
 
 def pool_blocks(w: Workload, lens: np.ndarray) -> int:
     """Physical blocks in the pool: the blocks every sequence reaches by the
-    last step (shared prefix counted once, one spare per sequence for a
-    copied shared block), times the slack factor; at least 16."""
+    last step (shared prefix counted once), times the slack factor; at least
+    16 (the tiny workload's fixed 16-block pool when its slack is 0)."""
     bs = w.block_size
     if w.prefix_tokens:
         prefix_blocks = -(-w.prefix_tokens // bs)
         need = prefix_blocks + int(sum(-(-(int(L) + w.steps) // bs) - w.prefix_tokens // bs for L in lens))
     else:
         need = int(sum(-(-(int(L) + w.steps) // bs) for L in lens))
-    return max(16, int(math.ceil(need * w.pool_slack)) if w.pool_slack else 16)
+    return max(16, int(math.ceil(need * w.pool_slack)) if w.pool_slack else need)
 
 
 def free_order(num_blocks: int, seed: int) -> np.ndarray:
