@@ -24,9 +24,14 @@ Modules:
   copy, and the split-partition (m, l, o) rescaling identity.
 * :mod:`oracle.block_allocator` — a pure-Python model of the host block
   allocator (free stack, refcounts, copy-on-write, all-or-nothing errors).
+* :mod:`oracle.fp8` — e4m3 codes (decode, round-to-nearest-even saturating
+  encode), the quantising append and decode attention over e4m3 pools with
+  per-pool scales ("LLM inference optimisation: principles overview" §5.1:
+  an FP8 KV cache).
 
 Parity status: every function here is pinned by ``tests/test_oracle.py`` or
 ``tests/test_allocator_oracle.py`` against something other than itself
 (brute force, a library special case, closed forms, invariants, the worked
-paging example of the vLLM paging page); none is "parity unpinned".
+paging example of the vLLM paging page; for e4m3, torch's float8_e4m3fn and
+closed-form code values); none is "parity unpinned".
 """

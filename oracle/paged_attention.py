@@ -37,7 +37,7 @@ from __future__ import annotations
 import numpy as np
 
 LAYOUTS = ("NHBD", "NBHD")
-DTYPES = ("f32", "f16", "bf16")
+DTYPES = ("f32", "f16", "bf16", "f64")
 
 
 def to_f64(raw: np.ndarray, dtype: str) -> np.ndarray:
@@ -53,6 +53,8 @@ def to_f64(raw: np.ndarray, dtype: str) -> np.ndarray:
     if dtype == "bf16":
         bits = np.asarray(raw, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
         return bits.view(np.float32).astype(np.float64)
+    if dtype == "f64":
+        return np.asarray(raw, dtype=np.float64)
     raise ValueError(f"unknown dtype {dtype!r}")
 
 
