@@ -67,7 +67,7 @@ enum pkv_status {
   PKV_ERR_BAD_BLOCK = -8       /* a kernel met a block id / slot outside the pool */
 };
 
-enum pkv_dtype { PKV_F32 = 0, PKV_BF16 = 1, PKV_F16 = 2 };
+enum pkv_dtype { PKV_F32 = 0, PKV_BF16 = 1, PKV_F16 = 2, PKV_FP8_E4M3 = 3 };
 
 /* Text of the calling thread's most recent error ("" if none).  The pointer
  * stays valid until the thread's next library call. */
@@ -176,7 +176,7 @@ int pkv_kv_append(const void* k_new, const void* v_new, const int32_t* slot_mapp
 
 /* Copy whole blocks (every head and offset of K and V) src -> dst for each
  * pair in block_pairs: int32[n_pairs][2] on the device — the copy-on-write
- * step of the vLLM paging page §3 phase 3.  Pairs must not chain (no dst is
+ * step of the vLLM paging page §3 phase 3.  dtype may also be PKV_FP8_E4M3.  Pairs must not chain (no dst is
  * another pair's src) and dsts must be distinct; pairs from
  * pkv_seq_append_slots satisfy both.  Ids outside the pool are skipped and
  * recorded as PKV_ERR_BAD_BLOCK. */
@@ -250,6 +250,41 @@ int pkv_paged_attention_decode_static(const void* q, const void* k_pool, const v
 /* Size in bytes of the static workspace used by
  * pkv_paged_attention_decode_static. */
 size_t pkv_static_workspace_bytes(void);
+
+/* ------------------------------------------------------------------------ */
+/* FP8 (e4m3) KV cache ("LLM inference optimisation: principles overview"   */
+/* §5.1: storing the KV cache as FP8 halves its bytes).                     */
+/* Pools hold e4m3 codes (uint8, same [num_blocks][num_kv_heads][block_size] */
+/* [head_dim] layout); element value = k_scale * e4m3(code) for K and        */
+/* v_scale * e4m3(code) for V (one fp32 scale per pool).  e4m3: 1 sign, 4    */
+/* exponent (bias 7), 3 mantissa bits, no infinities, 0x7F/0xFF = NaN,       */
+/* largest finite 448.                                                       */
+/* ------------------------------------------------------------------------ */
+
+/* Append into e4m3 pools: each element x of the new rows (src_dtype PKV_F32,
+ * PKV_BF16 or PKV_F16, layout as pkv_kv_append) is stored as the e4m3 code
+ * nearest to x * (1/scale), the product taken in fp32 with the fp32
+ * reciprocal of the scale, ties to even, saturating to +-448.  Slots as for
+ * pkv_kv_append (slot < 0 skipped, out-of-pool recorded as BAD_BLOCK).
+ * Errors: INVALID_ARG (scales not positive/finite, misalignment),
+ * UNSUPPORTED (head_dim, block_size, src_dtype). */
+int pkv_kv_append_fp8(const void* k_new, const void* v_new, int32_t src_dtype, const int32_t* slot_mapping,
+                      int32_t n_tokens, void* k_pool, void* v_pool, int32_t num_blocks, int32_t num_kv_heads,
+                      int32_t head_dim, int32_t block_size, float k_scale, float v_scale, void* stream);
+
+/* PagedAttention decode over e4m3 pools: the result of
+ * pkv_paged_attention_decode on the dequantised values (scores
+ * scale * k_scale * q·code, output v_scale * the softmax-weighted codes).
+ * q is float16 [num_seqs][num_q_heads][head_dim] (e4m3 widens to f16
+ * exactly); head_dim must be 128; group sizes 1, 2, 4, 8; partition_tokens a
+ * multiple of 16 (0 = automatic).  Workspace as sized by
+ * pkv_decode_workspace_size with the same arguments. */
+int pkv_paged_attention_decode_fp8(const void* q, const void* k_pool, const void* v_pool,
+                                   const int32_t* block_tables, const int32_t* seq_lens, int32_t num_seqs,
+                                   int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks,
+                                   int32_t max_blocks_per_seq, int32_t block_size, float scale, float k_scale,
+                                   float v_scale, int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                                   float* out, void* stream);
 
 /* Synchronise `stream`, then read the device status word of the current
  * device into *status: PKV_OK, or the first PKV_ERR_BAD_BLOCK /

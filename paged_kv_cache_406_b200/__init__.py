@@ -7,8 +7,8 @@ thin Python binding.  Build the library with
 ``python -m paged_kv_cache_406_b200.build``.
 """
 from .binding import (Allocator, PagedKVError, pkv_copy_blocks, pkv_decode_workspace_size,  # noqa: F401
-                      pkv_device_status, pkv_kv_append, pkv_paged_attention_decode,
-                      pkv_paged_attention_decode_static)
+                      pkv_device_status, pkv_kv_append, pkv_kv_append_fp8, pkv_paged_attention_decode,
+                      pkv_paged_attention_decode_fp8, pkv_paged_attention_decode_static)
 from ._native import LIB_PATH, lib  # noqa: F401
 
 __version__ = "1.0.0"

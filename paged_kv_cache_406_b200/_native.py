@@ -23,7 +23,7 @@ PKV_ERR_DEVICE_TIMEOUT = -6
 PKV_ERR_SEQ_EXISTS = -7
 PKV_ERR_BAD_BLOCK = -8
 
-PKV_F32, PKV_BF16, PKV_F16 = 0, 1, 2
+PKV_F32, PKV_BF16, PKV_F16, PKV_FP8_E4M3 = 0, 1, 2, 3
 
 # Every entry point include/paged_kv.h declares, with its ctypes signature.
 _i32, _i64, _f32, _vp, _sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
@@ -58,6 +58,10 @@ SIGNATURES = {
     "pkv_paged_attention_decode_static": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                                                          _i32, _i32, _f32, _i32, _i32, _vp, _vp]),
     "pkv_static_workspace_bytes": (ctypes.c_size_t, []),
+    "pkv_kv_append_fp8": (ctypes.c_int, [_vp, _vp, _i32, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _f32, _f32,
+                                         _vp]),
+    "pkv_paged_attention_decode_fp8": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
+                                                      _i32, _f32, _f32, _f32, _i32, _vp, _sz, _vp, _vp]),
 }
 
 

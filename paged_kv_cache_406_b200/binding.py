@@ -17,12 +17,13 @@ import torch
 from . import _native as N
 from ._native import PagedKVError, check, lib
 
-_DTYPES = {torch.float32: N.PKV_F32, torch.bfloat16: N.PKV_BF16, torch.float16: N.PKV_F16}
+_DTYPES = {torch.float32: N.PKV_F32, torch.bfloat16: N.PKV_BF16, torch.float16: N.PKV_F16,
+           torch.float8_e4m3fn: N.PKV_FP8_E4M3, torch.uint8: N.PKV_FP8_E4M3}
 
 
 def _dtype_code(t: torch.Tensor) -> int:
     if t.dtype not in _DTYPES:
-        raise TypeError(f"unsupported dtype {t.dtype}; expected float32, bfloat16 or float16")
+        raise TypeError(f"unsupported dtype {t.dtype}; expected float32, bfloat16, float16 or e4m3 codes")
     return _DTYPES[t.dtype]
 
 
@@ -151,6 +152,65 @@ def pkv_paged_attention_decode_static(q: torch.Tensor, k_pool: torch.Tensor, v_p
     return out
 
 
+def _fp8_pool(t: torch.Tensor, name: str) -> torch.Tensor:
+    _cuda(t, name)
+    if t.dtype not in (torch.uint8, torch.float8_e4m3fn):
+        raise TypeError(f"{name} must hold e4m3 codes (torch.uint8 or torch.float8_e4m3fn), got {t.dtype}")
+    return t
+
+
+def pkv_kv_append_fp8(k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: torch.Tensor, k_pool: torch.Tensor,
+                      v_pool: torch.Tensor, k_scale: float, v_scale: float) -> None:
+    """Quantise each new token's K/V rows to e4m3 (x / scale, nearest, saturating)
+    and write them into their slots of the e4m3 pools."""
+    _fp8_pool(k_pool, "k_pool")
+    _fp8_pool(v_pool, "v_pool")
+    if k_pool.dim() != 4 or k_pool.shape != v_pool.shape:
+        raise ValueError("pools must be [num_blocks, num_kv_heads, block_size, head_dim]")
+    nb, hkv, bs, d = k_pool.shape
+    for name, t in (("k_new", k_new), ("v_new", v_new)):
+        _cuda(t, name)
+        if t.dim() != 3 or t.shape[1:] != (hkv, d):
+            raise ValueError(f"{name} must be [n_tokens, {hkv}, {d}]")
+    if k_new.shape != v_new.shape or k_new.dtype != v_new.dtype:
+        raise ValueError("k_new and v_new differ in shape or dtype")
+    _cuda(slot_mapping, "slot_mapping", torch.int32)
+    if slot_mapping.numel() != k_new.shape[0]:
+        raise ValueError("slot_mapping must hold one slot per new token")
+    check(lib().pkv_kv_append_fp8(k_new.data_ptr(), v_new.data_ptr(), _dtype_code(k_new), slot_mapping.data_ptr(),
+                                  k_new.shape[0], k_pool.data_ptr(), v_pool.data_ptr(), nb, hkv, d, bs,
+                                  float(k_scale), float(v_scale), _stream()))
+
+
+def pkv_paged_attention_decode_fp8(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                                   block_tables: torch.Tensor, seq_lens: torch.Tensor, scale: float, k_scale: float,
+                                   v_scale: float, out: Optional[torch.Tensor] = None,
+                                   workspace: Optional[torch.Tensor] = None, partition_tokens: int = 0) -> torch.Tensor:
+    """PagedAttention decode over e4m3 pools (q float16); float32 output."""
+    _fp8_pool(k_pool, "k_pool")
+    _fp8_pool(v_pool, "v_pool")
+    nb, hkv, bs, d = k_pool.shape
+    _cuda(q, "q", torch.float16)
+    B, hq, _ = q.shape
+    _cuda(block_tables, "block_tables", torch.int32)
+    _cuda(seq_lens, "seq_lens", torch.int32)
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.numel() != B:
+        raise ValueError("block_tables must be [num_seqs, max_blocks_per_seq] and seq_lens [num_seqs]")
+    maxb = block_tables.shape[1]
+    if out is None:
+        out = torch.empty((B, hq, d), dtype=torch.float32, device=q.device)
+    else:
+        _cuda(out, "out", torch.float32)
+    need = pkv_decode_workspace_size(B, hq, hkv, d, maxb, bs, partition_tokens)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    check(lib().pkv_paged_attention_decode_fp8(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
+                                               block_tables.data_ptr(), seq_lens.data_ptr(), B, hq, hkv, d, nb, maxb,
+                                               bs, float(scale), float(k_scale), float(v_scale), partition_tokens,
+                                               workspace.data_ptr(), workspace.numel(), out.data_ptr(), _stream()))
+    return out
+
+
 def pkv_device_status(clear: bool = True) -> int:
     """Synchronise the current stream and return the device status word."""
     st = ctypes.c_int32(0)
@@ -244,4 +304,5 @@ class Allocator:
 
 
 __all__ = ["Allocator", "PagedKVError", "pkv_kv_append", "pkv_copy_blocks", "pkv_decode_workspace_size",
-           "pkv_paged_attention_decode", "pkv_paged_attention_decode_static", "pkv_device_status"]
+           "pkv_paged_attention_decode", "pkv_paged_attention_decode_static", "pkv_device_status",
+           "pkv_kv_append_fp8", "pkv_paged_attention_decode_fp8"]

@@ -28,8 +28,14 @@ from ._native import check, lib
 class PagedKVCache:
     def __init__(self, num_blocks: int, num_kv_heads: int, head_dim: int, block_size: int,
                  dtype: torch.dtype, max_blocks_per_seq: int, device="cuda", free_order=None,
-                 k_pool: Optional[torch.Tensor] = None, v_pool: Optional[torch.Tensor] = None):
+                 k_pool: Optional[torch.Tensor] = None, v_pool: Optional[torch.Tensor] = None,
+                 k_scale: float = 1.0, v_scale: float = 1.0):
+        """``dtype`` torch.float8_e4m3fn (or torch.uint8) keeps the pools as e4m3
+        codes with per-pool scales ``k_scale`` / ``v_scale`` (the overview page's
+        FP8 KV cache); new rows are quantised on append and q must be float16."""
         self.device = torch.device(device)
+        self.fp8 = dtype in (torch.float8_e4m3fn, torch.uint8)
+        self.k_scale, self.v_scale = float(k_scale), float(v_scale)
         self.num_blocks, self.num_kv_heads = int(num_blocks), int(num_kv_heads)
         self.head_dim, self.block_size = int(head_dim), int(block_size)
         self.dtype = dtype
@@ -120,8 +126,13 @@ class PagedKVCache:
         q, k_new, v_new = (t.to(self.device, non_blocking=True) for t in (q, k_new, v_new))
         if ncow:
             B.pkv_copy_blocks(self.k_pool, self.v_pool, cow[:2 * ncow].view(ncow, 2))
-        B.pkv_kv_append(k_new, v_new, slots, self.k_pool, self.v_pool)
         ws, out = self._buffers(n, q.shape[1], partition_tokens)
+        if self.fp8:
+            B.pkv_kv_append_fp8(k_new, v_new, slots, self.k_pool, self.v_pool, self.k_scale, self.v_scale)
+            return B.pkv_paged_attention_decode_fp8(q, self.k_pool, self.v_pool, tables, lens, scale, self.k_scale,
+                                                    self.v_scale, out=out, workspace=ws,
+                                                    partition_tokens=partition_tokens)
+        B.pkv_kv_append(k_new, v_new, slots, self.k_pool, self.v_pool)
         return B.pkv_paged_attention_decode(q, self.k_pool, self.v_pool, tables, lens, scale, out=out,
                                             workspace=ws, partition_tokens=partition_tokens)
 

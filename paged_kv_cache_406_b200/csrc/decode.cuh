@@ -44,6 +44,7 @@ struct DecodeParams {
   int32_t num_q_heads, num_kv_heads, num_blocks, max_blocks, block_size, partition_tokens, max_parts;
   int32_t n_stages;
   float scale_log2;
+  float v_scale;  // multiplies the output (e4m3 V pools; 1 otherwise)
   const int4* items;  // {b, partition, partitions of b, end token}
   const int32_t* n_items;
   float* part_m;
@@ -232,10 +233,10 @@ __device__ __forceinline__ void merge_store(const float* rec, const WorkUnit& u,
     }
     const int64_t row = static_cast<int64_t>(u.b) * p.num_q_heads + u.g * G + h;
     if (single) {
-      p.out[row * D + d] = den > 0.f ? num / den : 0.f;
+      p.out[row * D + d] = den > 0.f ? p.v_scale * num / den : 0.f;
     } else {
       const int64_t pr = row * p.max_parts + u.part;
-      p.part_o[pr * D + d] = num;
+      p.part_o[pr * D + d] = p.v_scale * num;
       if (d == 0) {
         p.part_m[pr] = M;
         p.part_l[pr] = den;

@@ -23,6 +23,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_fp8.h>
 
 #include "decode.cuh"
 
@@ -30,24 +31,46 @@ namespace pkv {
 
 constexpr int kChunkTokens = 16;
 
-template <int D>
+// kKVBytes = bytes per stored K/V element: 2 (bf16 / f16) or 1 (e4m3).
+template <int D, int kKVBytes = 2>
 struct MmaLayout {
-  static constexpr int kHalves = D / 64;                       // 128-byte column halves of a row
-  static constexpr int kTileBytes = kChunkTokens * D * 2;       // one 16-token K (or V) chunk
-  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kHalves = D / 64;                           // 128-byte column halves of a 16-bit row
+  static constexpr int kTileBytes = kChunkTokens * D * 2;           // 16-bit 16-token K (or V) chunk
+  static constexpr int kRingHalves = D * kKVBytes / 128;            // 128-byte column halves of a stored row
+  static constexpr int kRingTileBytes = kChunkTokens * D * kKVBytes;  // stored 16-token chunk in the ring
+  static constexpr int kStageBytes = 2 * kRingTileBytes;
+  // e4m3 chunks are widened into a per-warp 16-bit K and V tile
+  static constexpr int kStagingBytes = kKVBytes == 1 ? 2 * kTileBytes : 0;
 };
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, int kKVBytes = 2>
 struct MmaSmem {
+  using L = MmaLayout<D, kKVBytes>;
   static constexpr int kMergeFloats = G * D + 2 * G;
-  __host__ __device__ static size_t ring_bytes(int ns) { return size_t(ns) * MmaLayout<D>::kStageBytes; }
+  __host__ __device__ static size_t ring_bytes(int ns) {
+    return size_t(ns) * L::kStageBytes + size_t(kConsumerWarps) * L::kStagingBytes;
+  }
   __host__ __device__ static size_t bytes(int ns) {
-    // + 1024: the dynamic shared memory base is aligned up to the 1024-byte swizzle atom;
-    // + 128: the producer's window of 32 block-table entries
+    // + 1024: the dynamic shared memory base is aligned up to the 1024-byte swizzle atom
     return 1024 + ring_bytes(ns) + 2 * kConsumerWarps * kMergeFloats * sizeof(float) + 2 * ns * sizeof(uint64_t) +
            16 + 128;
   }
 };
+
+// 16 e4m3 codes (one 16-byte chunk) widened exactly to 16 f16 values.
+__device__ __forceinline__ void widen_e4m3x16(const uint4& in, uint4& lo, uint4& hi) {
+  const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] & 0xffffu), __NV_E4M3);
+    const __half2_raw b = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] >> 16), __NV_E4M3);
+    o[2 * i] = static_cast<uint32_t>(a.x) | (static_cast<uint32_t>(a.y) << 16);
+    o[2 * i + 1] = static_cast<uint32_t>(b.x) | (static_cast<uint32_t>(b.y) << 16);
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
 
 // A chunk tile in shared memory is built from TMA boxes of `br` rows (br = 16,
 // or 8 when block_size is 8 and a chunk spans two blocks).  Each box holds,
@@ -59,15 +82,20 @@ __device__ __forceinline__ uint32_t row_offset(int r, int h, int br_shift, int h
   return static_cast<uint32_t>(((r >> br_shift) * halves * br + h * br + (r & (br - 1))) * 128);
 }
 
-template <typename T, int D, int G>
+// kKVBytes = 1: the pools hold e4m3 codes (T must be __half: e4m3 widens to
+// f16 exactly); the consumer warp widens each landed chunk into its own
+// 16-bit staging tile and frees the ring stage before the MMAs.
+template <typename T, int D, int G, int kKVBytes = 2>
 __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const DecodeParams p,
                                                                     const __grid_constant__ CUtensorMap tmap_k,
                                                                     const __grid_constant__ CUtensorMap tmap_v) {
-  static_assert(G == 2 || G == 4 || G == 8, "group size");
-  using L = MmaLayout<D>;
+  static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
+  static_assert(kKVBytes == 2 || (kKVBytes == 1 && D == 128), "e4m3 pools need head_dim 128");
+  using L = MmaLayout<D, kKVBytes>;
+  constexpr bool kFp8 = kKVBytes == 1;
   constexpr int kSteps = D / 16;  // k-steps of q·Kᵀ and m-tiles of P·V
   constexpr int kHalves = L::kHalves;
-  constexpr int kMF = MmaSmem<T, D, G>::kMergeFloats;
+  constexpr int kMF = MmaSmem<T, D, G, kKVBytes>::kMergeFloats;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -75,7 +103,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
   const int NS = p.n_stages;
   const int bs_shift = BS == 8 ? 3 : (BS == 16 ? 4 : 5);
   const int br_shift = BS == 8 ? 3 : 4;  // rows per TMA box: 8 or 16
-  float* merge = reinterpret_cast<float*>(smem + MmaSmem<T, D, G>::ring_bytes(NS));
+  float* merge = reinterpret_cast<float*>(smem + MmaSmem<T, D, G, kKVBytes>::ring_bytes(NS));
   uint64_t* full = reinterpret_cast<uint64_t*>(merge + 2 * kConsumerWarps * kMF);
   uint64_t* empty = full + NS;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + NS);
@@ -107,8 +135,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
       prefetch_tensormap(&tmap_v);
     }
     const uint64_t policy = l2_evict_first_policy();
-    const uint32_t box_bytes = (1u << br_shift) * D * 2;           // one K (or V) box
-    const uint32_t blk_off = kHalves * (1u << br_shift) * 128;     // second box of a chunk (block_size 8)
+    const uint32_t box_bytes = (1u << br_shift) * D * kKVBytes;        // one K (or V) box
+    const uint32_t blk_off = L::kRingHalves * (1u << br_shift) * 128;  // second box of a chunk (block_size 8)
     int s = 0;
     uint32_t ph = 0, issued = 0;
     bool ok = true;
@@ -143,7 +171,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
               }
               const int32_t y = phys * p.num_kv_heads * BS + ybase + row0;
               tma_load_3d(kdst + i * blk_off, &tmap_k, 0, y, 0, bar, policy);
-              tma_load_3d(kdst + L::kTileBytes + i * blk_off, &tmap_v, 0, y, 0, bar, policy);
+              tma_load_3d(kdst + L::kRingTileBytes + i * blk_off, &tmap_v, 0, y, 0, bar, policy);
             }
             ++issued;
             if (++s == NS) {
@@ -175,12 +203,16 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
   // ldmatrix row addresses of this lane: K chunk (A operand) and V chunk (A = Vᵀ via .trans)
   const int ra = (lane & 7) + ((lane >> 3) & 1) * 8, ca = lane >> 4;
   const int rv = (lane & 7) + (lane >> 4) * 8, cv = (lane >> 3) & 1;
+  // the tiles the MMAs read: the ring chunk itself (16-bit pools, boxes of
+  // br rows) or the warp's staging tile (e4m3 pools, always 16-row layout)
+  const int tile_shift = kFp8 ? 4 : br_shift;
   uint32_t offa[kHalves], offv[kHalves];
 #pragma unroll
   for (int h = 0; h < kHalves; ++h) {
-    offa[h] = row_offset(ra, h, br_shift, kHalves);
-    offv[h] = row_offset(rv, h, br_shift, kHalves);
+    offa[h] = row_offset(ra, h, tile_shift, kHalves);
+    offv[h] = row_offset(rv, h, tile_shift, kHalves);
   }
+  const uint32_t staging = ring_s + NS * L::kStageBytes + warp * L::kStagingBytes;
   const int xa = ra & 7, xv = rv & 7;
   const int src0 = 4 * (2 * tq) + (gq >> 1), src1 = src0 + 4;  // Pᵀ transpose sources
   const uint32_t sel = (gq & 1) ? 0x7632u : 0x5410u;
@@ -220,9 +252,39 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
         ok = false;
         break;
       }
-      const uint32_t kbase = ring_s + s * L::kStageBytes;
-      const uint32_t vbase = kbase + L::kTileBytes;
+      uint32_t kbase = ring_s + s * L::kStageBytes;
+      uint32_t vbase = kbase + L::kRingTileBytes;
       const int nv = min(kChunkTokens, u.t1 - (u.t0 + k * kChunkTokens));
+      if constexpr (kFp8) {
+        // widen the e4m3 chunk (rows of 128 B, 128-byte swizzle) into the
+        // 16-bit staging layout, then hand the ring stage back at once
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int i = lane + 32 * j, row = i >> 3, c = i & 7;  // 16 codes: dims 16c .. 16c+15
+          const uint32_t src = static_cast<uint32_t>(row * 128 + ((c ^ (row & 7)) << 4));
+          const uint32_t d0 = row_offset(row, c >> 2, 4, kHalves) + ((((c & 3) << 1) ^ (row & 7)) << 4);
+          const uint32_t d1 = row_offset(row, c >> 2, 4, kHalves) + (((((c & 3) << 1) + 1) ^ (row & 7)) << 4);
+          uint4 raw, lo, hi;
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(raw.x), "=r"(raw.y), "=r"(raw.z), "=r"(raw.w) : "r"(kbase + src));
+          widen_e4m3x16(raw, lo, hi);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(staging + d0), "r"(lo.x), "r"(lo.y),
+                       "r"(lo.z), "r"(lo.w) : "memory");
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(staging + d1), "r"(hi.x), "r"(hi.y),
+                       "r"(hi.z), "r"(hi.w) : "memory");
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(raw.x), "=r"(raw.y), "=r"(raw.z), "=r"(raw.w) : "r"(vbase + src));
+          widen_e4m3x16(raw, lo, hi);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(staging + L::kTileBytes + d0), "r"(lo.x),
+                       "r"(lo.y), "r"(lo.z), "r"(lo.w) : "memory");
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(staging + L::kTileBytes + d1), "r"(hi.x),
+                       "r"(hi.y), "r"(hi.z), "r"(hi.w) : "memory");
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_addr(empty + s));
+        kbase = staging;
+        vbase = staging + L::kTileBytes;
+      }
 
       // ---- scores: S^T = K · Qᵀ ----
       float sc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -279,7 +341,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
         const int total = (kChunkTokens - nv) * per_row;
         for (int i = lane; i < total; i += 32) {
           const int row = nv + i / per_row, rem = i % per_row;
-          const uint32_t addr = vbase + row_offset(row, rem / 8, br_shift, kHalves) + (rem % 8) * 16;
+          const uint32_t addr = vbase + row_offset(row, rem / 8, tile_shift, kHalves) + (rem % 8) * 16;
           asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0) : "memory");
         }
         __syncwarp();
@@ -293,9 +355,13 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
         mma_16816<T>(acc[mt], a, bh0, bh1);
         mma_16816<T>(acc[mt], a, bl0, bl1);
       }
-      if (nv < kChunkTokens) fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_addr(empty + s));
+      if (!kFp8) {
+        if (nv < kChunkTokens) fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_addr(empty + s));
+      } else {
+        __syncwarp();  // the staging tile is rewritten by this warp's next chunk
+      }
       s += kConsumerWarps;
       if (s >= NS) {
         s -= NS;

@@ -8,6 +8,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <cuda_fp8.h>
+
 #include "decode.cuh"
 #include "decode_mma.cuh"
 #include "device_common.cuh"
@@ -62,6 +64,76 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ k_
   }
 }
 
+// ---------------------------------------------------------------------------
+// KV append into e4m3 pools: each thread quantises 8 elements of one (token,
+// head) row, x * (1 / scale) in fp32, rounded to nearest e4m3 (ties to even,
+// saturating to +-448), and stores 8 bytes.
+// ---------------------------------------------------------------------------
+template <typename Src>
+__device__ __forceinline__ void load8_f32(const Src* p, float (&x)[8]);
+
+template <>
+__device__ __forceinline__ void load8_f32<float>(const float* p, float (&x)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
+template <>
+__device__ __forceinline__ void load8_f32<__nv_bfloat16>(const __nv_bfloat16* p, float (&x)[8]) {
+  const uint4 r = *reinterpret_cast<const uint4*>(p);
+  float2 f[4];
+  Elem<__nv_bfloat16>::widen(r, f);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) { x[2 * i] = f[i].x; x[2 * i + 1] = f[i].y; }
+}
+
+template <>
+__device__ __forceinline__ void load8_f32<__half>(const __half* p, float (&x)[8]) {
+  const uint4 r = *reinterpret_cast<const uint4*>(p);
+  float2 f[4];
+  Elem<__half>::widen(r, f);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) { x[2 * i] = f[i].x; x[2 * i + 1] = f[i].y; }
+}
+
+template <typename Src>
+__global__ void __launch_bounds__(256) kv_append_fp8_kernel(const Src* __restrict__ k_new, const Src* __restrict__ v_new,
+                                                            const int32_t* __restrict__ slots, int64_t n_groups,
+                                                            uint8_t* __restrict__ k_pool, uint8_t* __restrict__ v_pool,
+                                                            int32_t num_blocks, int32_t num_kv_heads, int32_t head_dim,
+                                                            int32_t block_size, float k_inv, float v_inv) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n_groups) return;
+  const int32_t per_row = head_dim / 8;
+  const int32_t grp = static_cast<int32_t>(i % per_row);
+  const int64_t row = i / per_row;  // token * num_kv_heads + head
+  const int32_t h = static_cast<int32_t>(row % num_kv_heads);
+  const int64_t tok = row / num_kv_heads;
+  const int32_t slot = slots[tok];
+  if (slot < 0) return;
+  const int32_t blk = slot / block_size, off = slot - blk * block_size;
+  if (blk >= num_blocks) {
+    if (grp == 0 && h == 0) record_error(PKV_ERR_BAD_BLOCK);
+    return;
+  }
+  const int64_t dst = ((static_cast<int64_t>(blk) * num_kv_heads + h) * block_size + off) * head_dim + grp * 8;
+  const int64_t src = row * head_dim + grp * 8;
+#pragma unroll
+  for (int kv = 0; kv < 2; ++kv) {
+    float x[8];
+    load8_f32<Src>((kv ? v_new : k_new) + src, x);
+    const float inv = kv ? v_inv : k_inv;
+    uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __nv_fp8x2_storage_t q2 =
+          __nv_cvt_float2_to_fp8x2(make_float2(x[2 * j] * inv, x[2 * j + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+      packed[j >> 1] |= static_cast<uint32_t>(q2) << (16 * (j & 1));
+    }
+    *reinterpret_cast<uint2*>((kv ? v_pool : k_pool) + dst) = make_uint2(packed[0], packed[1]);
+  }
+}
+
 }  // namespace pkv
 
 // ===========================================================================
@@ -75,7 +147,7 @@ constexpr int kMaxDevices = 64;
 constexpr int kAutoPartitionTokens = 512;
 constexpr int kMaxPartitionTokens = 8192;
 
-size_t elem_size(int dtype) { return dtype == PKV_F32 ? 4 : 2; }
+size_t elem_size(int dtype) { return dtype == PKV_F32 ? 4 : (dtype == PKV_FP8_E4M3 ? 1 : 2); }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -248,6 +320,18 @@ EncodeTiledFn encode_fn() {
 int make_pool_map(CUtensorMap* m, const void* pool, int dtype, int64_t rows, int head_dim, int box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  if (dtype == PKV_FP8_E4M3) {
+    // e4m3 codes: a row of head_dim bytes is one box column (head_dim = 128: 128 B)
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows), 1};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(head_dim)};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(head_dim), static_cast<cuuint32_t>(box_rows), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(pool), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled (e4m3) failed (%d)", static_cast<int>(r));
+    return PKV_OK;
+  }
   const cuuint32_t halves = static_cast<cuuint32_t>(head_dim / 64);
   const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), halves};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2, 128};
@@ -288,7 +372,7 @@ int pool_map(CUtensorMap* out, const void* pool, int dtype, int64_t rows, int he
   return PKV_OK;
 }
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, int kKVBytes = 2>
 int launch_decode_mma(const pkv::DecodeParams& base, const int32_t* seq_lens, int32_t num_seqs, int32_t max_tokens,
                       int dtype, cudaStream_t stream) {
   pkv::DecodeParams p = base;
@@ -296,8 +380,8 @@ int launch_decode_mma(const pkv::DecodeParams& base, const int32_t* seq_lens, in
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   p.n_stages = 8;
-  const size_t smem = pkv::MmaSmem<T, D, G>::bytes(p.n_stages);
-  auto kern = pkv::decode_mma_kernel<T, D, G>;
+  const size_t smem = pkv::MmaSmem<T, D, G, kKVBytes>::bytes(p.n_stages);
+  auto kern = pkv::decode_mma_kernel<T, D, G, kKVBytes>;
   static std::atomic<int> occ_cache[kMaxDevices];
   int occ = dev < kMaxDevices ? occ_cache[dev].load(std::memory_order_relaxed) : 0;
   if (occ == 0) {
@@ -376,7 +460,8 @@ extern "C" int pkv_kv_append(const void* k_new, const void* v_new, const int32_t
 extern "C" int pkv_copy_blocks(void* k_pool, void* v_pool, const int32_t* block_pairs, int32_t n_pairs,
                                int32_t num_blocks, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                                int32_t dtype, void* stream) {
-  int rc = check_common(num_kv_heads, head_dim, block_size, dtype, "pkv_copy_blocks");
+  // a byte copy: e4m3 pools are copied like 16-bit ones, at one byte per element
+  int rc = check_common(num_kv_heads, head_dim, block_size, dtype == PKV_FP8_E4M3 ? PKV_F16 : dtype, "pkv_copy_blocks");
   if (rc) return rc;
   if (n_pairs < 0 || num_blocks <= 0) return fail(PKV_ERR_INVALID_ARG, "pkv_copy_blocks: n_pairs/num_blocks");
   if (n_pairs == 0) return pkv::ok();
@@ -458,6 +543,7 @@ extern "C" int pkv_paged_attention_decode(const void* q, const void* k_pool, con
   p.partition_tokens = pt;
   p.max_parts = w.max_parts;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.v_scale = 1.0f;
   p.items = reinterpret_cast<const int4*>(ws + w.items);
   p.n_items = reinterpret_cast<const int32_t*>(ws);
   p.part_m = reinterpret_cast<float*>(ws + w.m);
@@ -496,6 +582,122 @@ extern "C" int pkv_device_status(void* stream, int32_t* status, int32_t clear) {
   }
   *status = v;
   return pkv::ok();
+}
+
+// ===========================================================================
+// FP8 (e4m3) KV cache
+// ===========================================================================
+extern "C" int pkv_kv_append_fp8(const void* k_new, const void* v_new, int32_t src_dtype,
+                                 const int32_t* slot_mapping, int32_t n_tokens, void* k_pool, void* v_pool,
+                                 int32_t num_blocks, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                 float k_scale, float v_scale, void* stream) {
+  const char* fn = "pkv_kv_append_fp8";
+  int rc = check_common(num_kv_heads, head_dim, block_size, src_dtype, fn);
+  if (rc) return rc;
+  if (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
+    return fail(PKV_ERR_INVALID_ARG, "%s: scales must be positive and finite", fn);
+  if (n_tokens < 0 || num_blocks <= 0) return fail(PKV_ERR_INVALID_ARG, "%s: n_tokens/num_blocks", fn);
+  if (n_tokens == 0) return pkv::ok();
+  if (!k_new || !v_new || !slot_mapping || !k_pool || !v_pool) return fail(PKV_ERR_INVALID_ARG, "%s: NULL pointer", fn);
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pool) || !aligned16(v_pool))
+    return fail(PKV_ERR_INVALID_ARG, "%s: buffers must be 16-byte aligned", fn);
+  const float k_inv = static_cast<float>(1.0 / static_cast<double>(k_scale));
+  const float v_inv = static_cast<float>(1.0 / static_cast<double>(v_scale));
+  const int64_t n_groups = int64_t(n_tokens) * num_kv_heads * (head_dim / 8);
+  const unsigned blocks = static_cast<unsigned>((n_groups + 255) / 256);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* kp = static_cast<uint8_t*>(k_pool);
+  uint8_t* vp = static_cast<uint8_t*>(v_pool);
+  switch (src_dtype) {
+    case PKV_F32:
+      pkv::kv_append_fp8_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(k_new),
+                                                              static_cast<const float*>(v_new), slot_mapping, n_groups,
+                                                              kp, vp, num_blocks, num_kv_heads, head_dim, block_size,
+                                                              k_inv, v_inv);
+      break;
+    case PKV_BF16:
+      pkv::kv_append_fp8_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+          static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new), slot_mapping, n_groups,
+          kp, vp, num_blocks, num_kv_heads, head_dim, block_size, k_inv, v_inv);
+      break;
+    default:
+      pkv::kv_append_fp8_kernel<__half><<<blocks, 256, 0, s>>>(static_cast<const __half*>(k_new),
+                                                               static_cast<const __half*>(v_new), slot_mapping,
+                                                               n_groups, kp, vp, num_blocks, num_kv_heads, head_dim,
+                                                               block_size, k_inv, v_inv);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pkv_kv_append_fp8 launch");
+  return pkv::ok();
+}
+
+extern "C" int pkv_paged_attention_decode_fp8(const void* q, const void* k_pool, const void* v_pool,
+                                              const int32_t* block_tables, const int32_t* seq_lens, int32_t num_seqs,
+                                              int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                              int32_t num_blocks, int32_t max_blocks_per_seq, int32_t block_size,
+                                              float scale, float k_scale, float v_scale, int32_t partition_tokens,
+                                              void* workspace, size_t workspace_bytes, float* out, void* stream) {
+  const char* fn = "pkv_paged_attention_decode_fp8";
+  int rc = check_common(num_kv_heads, head_dim, block_size, PKV_F16, fn);
+  if (rc) return rc;
+  if (head_dim != 128) return fail(PKV_ERR_UNSUPPORTED, "%s: e4m3 pools need head_dim 128", fn);
+  if (num_seqs < 0 || num_q_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq < 0)
+    return fail(PKV_ERR_INVALID_ARG, "%s: bad sizes", fn);
+  if (num_q_heads % num_kv_heads != 0) return fail(PKV_ERR_INVALID_ARG, "%s: num_q_heads % num_kv_heads != 0", fn);
+  const int32_t group = num_q_heads / num_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: group size %d not supported (1, 2, 4 or 8)", fn, group);
+  if (!std::isfinite(scale) || !(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) ||
+      !std::isfinite(v_scale))
+    return fail(PKV_ERR_INVALID_ARG, "%s: scale must be finite and k_scale, v_scale positive", fn);
+  int32_t pt = 0;
+  rc = resolve_partition(partition_tokens, block_size, &pt);
+  if (rc) return rc;
+  if (pt % pkv::kChunkTokens != 0) return fail(PKV_ERR_INVALID_ARG, "%s: partition_tokens must be a multiple of 16", fn);
+  if (num_seqs == 0) return pkv::ok();
+  if (!q || !k_pool || !v_pool || !block_tables || !seq_lens || !workspace || !out)
+    return fail(PKV_ERR_INVALID_ARG, "%s: NULL pointer", fn);
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out))
+    return fail(PKV_ERR_INVALID_ARG, "%s: q, pools and out must be 16-byte aligned", fn);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(PKV_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", fn);
+  const int64_t max_tokens = int64_t(max_blocks_per_seq) * block_size;
+  if (max_tokens > (int64_t(1) << 30)) return fail(PKV_ERR_INVALID_ARG, "%s: max_blocks_per_seq too large", fn);
+  if (int64_t(num_blocks) * num_kv_heads * block_size > INT32_MAX)
+    return fail(PKV_ERR_INVALID_ARG, "%s: pool has more than 2^31 token rows", fn);
+  const WsLayout w = ws_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_tokens, pt);
+  if (workspace_bytes < w.total)
+    return fail(PKV_ERR_INVALID_ARG, "%s: workspace %zu bytes < %zu needed", fn, workspace_bytes, w.total);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  pkv::DecodeParams p{};
+  p.q = q;
+  p.k_pool = k_pool;
+  p.v_pool = v_pool;
+  p.block_tables = block_tables;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.num_blocks = num_blocks;
+  p.max_blocks = max_blocks_per_seq;
+  p.block_size = block_size;
+  p.partition_tokens = pt;
+  p.max_parts = w.max_parts;
+  // scores = scale * k_scale * q·codes; output = v_scale * softmax-weighted codes
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * static_cast<double>(k_scale) * 1.4426950408889634);
+  p.v_scale = v_scale;
+  p.items = reinterpret_cast<const int4*>(ws + w.items);
+  p.n_items = reinterpret_cast<const int32_t*>(ws);
+  p.part_m = reinterpret_cast<float*>(ws + w.m);
+  p.part_l = reinterpret_cast<float*>(ws + w.l);
+  p.part_o = reinterpret_cast<float*>(ws + w.o);
+  p.out = out;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int32_t mt = static_cast<int32_t>(max_tokens);
+  switch (group) {
+    case 1: return launch_decode_mma<__half, 128, 1, 1>(p, seq_lens, num_seqs, mt, PKV_FP8_E4M3, s);
+    case 2: return launch_decode_mma<__half, 128, 2, 1>(p, seq_lens, num_seqs, mt, PKV_FP8_E4M3, s);
+    case 4: return launch_decode_mma<__half, 128, 4, 1>(p, seq_lens, num_seqs, mt, PKV_FP8_E4M3, s);
+    default: return launch_decode_mma<__half, 128, 8, 1>(p, seq_lens, num_seqs, mt, PKV_FP8_E4M3, s);
+  }
 }
 
 // ===========================================================================
