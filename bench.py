@@ -48,6 +48,7 @@ TRAFFIC_SOURCE_SHA = "62c7be410db53362"
 SEQ_LEN_RECIPES = {
     "tiny": "{1,7,16,33} before the step's append",
     "llama3_8b": "U[512,4096]",
+    "llama3_8b_fp8": "U[512,4096]; e4m3 K/V (scale 1/32), q and new rows float16",
     "prefix_shared": "1024-token shared prefix (refcount = num_seqs) + U[64,512] tails; KV bytes are logical "
                      "(the prefix counted once per sequence)",
     "long_splitk": "7 x 32768 + 1 x 131072",
@@ -182,12 +183,16 @@ def oracle_threads() -> int:
 def time_oracle(units, budget_s: float):
     """Runs the oracle on (q rows, K, V raw blocks, table, L, scale, dtype)
     units until the budget is spent; returns (KV bytes, seconds, units done)."""
+    from oracle import fp8 as of8
     from oracle import paged_attention as pa
     done, nbytes, t0 = 0, 0, time.perf_counter()
     for u in units:
         q, kb, vb, L, scale, dtype, kv_bytes = u
         table = np.arange(kb.shape[0], dtype=np.int32)[None]
-        pa.paged_decode_attention(q, kb, vb, table, np.array([L]), scale, dtype)
+        if isinstance(dtype, tuple):  # ("e4m3", k_scale, v_scale)
+            of8.paged_decode_attention_fp8(q, kb, vb, table, np.array([L]), scale, dtype[1], dtype[2])
+        else:
+            pa.paged_decode_attention(q, kb, vb, table, np.array([L]), scale, dtype)
         done += 1
         nbytes += kv_bytes
         if time.perf_counter() - t0 > budget_s:
@@ -199,6 +204,8 @@ def _raw(t: torch.Tensor) -> np.ndarray:
     t = t.detach().cpu().contiguous()
     if t.dtype == torch.bfloat16:
         return t.view(torch.int16).numpy().view(np.uint16)
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8).numpy()
     return t.numpy()
 
 
@@ -213,7 +220,8 @@ def make_units(w, k_pool, v_pool, tables, lens, q, order, count):
         kb = _raw(k_pool[idx, g:g + 1])
         vb = _raw(v_pool[idx, g:g + 1])
         qb = _raw(q[b:b + 1, g * G:(g + 1) * G])
-        units.append((qb, kb, vb, L, w.scale, w.dtype, L * w.head_dim * 2 * e))
+        dt = ("e4m3", w.kv_scale, w.kv_scale) if w.dtype == "e4m3" else w.dtype
+        units.append((qb, kb, vb, L, w.scale, dt, L * w.head_dim * 2 * e))
     return units
 
 
@@ -226,11 +234,12 @@ def setup(w, device, horizon):
     lens = W.seq_lens(w)
     nb = W.pool_blocks(w, lens + horizon) + (w.num_seqs if w.prefix_tokens else 0)
     shape = (nb, w.num_kv_heads, w.block_size, w.head_dim)
-    k_pool = W.normal(shape, w.torch_dtype, W.pool_seed(w, 0), device=device)
-    v_pool = W.normal(shape, w.torch_dtype, W.pool_seed(w, 1), device=device)
+    k_pool = W.pool_values(shape, w, 0, device=device)
+    v_pool = W.pool_values(shape, w, 1, device=device)
     maxb = -(-(int(lens.max()) + horizon) // w.block_size)
     cache = PagedKVCache(nb, w.num_kv_heads, w.head_dim, w.block_size, w.torch_dtype, maxb, device=device,
-                         free_order=W.free_order(nb, w.seed), k_pool=k_pool, v_pool=v_pool)
+                         free_order=W.free_order(nb, w.seed), k_pool=k_pool, v_pool=v_pool,
+                         k_scale=w.kv_scale, v_scale=w.kv_scale)
     if w.prefix_tokens:
         # one sequence holds the shared prefix, the others fork it (refcount =
         # num_seqs), then every sequence appends its own tail token by token
@@ -268,7 +277,9 @@ def run_ours(args):
     horizon = STAGED_STEPS + 3 + max(0, args.e2e_steps) + 8
     w, cache, lens0 = setup(rank_workload(w0, rank), dev, horizon)
     B, hq, hkv, d, bs = w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size
-    esz = torch.tensor([], dtype=w.torch_dtype).element_size()
+    esz = torch.tensor([], dtype=w.torch_dtype).element_size()   # stored K/V element
+    qsz = torch.tensor([], dtype=w.io_dtype).element_size()      # q and new rows
+    fp8 = w.dtype == "e4m3"
     ids = list(range(B))
     alloc = cache.alloc
 
@@ -281,9 +292,9 @@ def run_ours(args):
             slots=torch.from_numpy(slots.copy()).to(dev), cow=torch.from_numpy(cow.copy()).to(dev),
             ncow=cow.shape[0], tables=torch.from_numpy(tables.copy()).to(dev),
             lens=torch.from_numpy(lens.copy()).to(dev), lens_host=lens.copy(),
-            q=W.normal((B, hq, d), w.torch_dtype, W.step_seed(w, s, 0), device=dev),
-            kn=W.normal((B, hkv, d), w.torch_dtype, W.step_seed(w, s, 1), device=dev),
-            vn=W.normal((B, hkv, d), w.torch_dtype, W.step_seed(w, s, 2), device=dev)))
+            q=W.normal((B, hq, d), w.io_dtype, W.step_seed(w, s, 0), device=dev),
+            kn=W.normal((B, hkv, d), w.io_dtype, W.step_seed(w, s, 1), device=dev),
+            vn=W.normal((B, hkv, d), w.io_dtype, W.step_seed(w, s, 2), device=dev)))
     wsb = P.pkv_decode_workspace_size(B, hq, hkv, d, cache.max_blocks, bs, w.partition_tokens)
     workspace = torch.empty(wsb, dtype=torch.uint8, device=dev)
     out = torch.empty((B, hq, d), dtype=torch.float32, device=dev)
@@ -298,7 +309,7 @@ def run_ours(args):
         # + the split-partition partials (m, l, o per query head), written once and read once
         tab = int(sum(-(-int(L) // bs) for L in lens)) * 4
         parts = int(sum(-(-int(L) // pt_eff) for L in lens if L > pt_eff))
-        return kv_bytes(lens) + tab + B * hq * d * esz + B * hq * d * 4 + 2 * parts * hq * (d + 2) * 4
+        return kv_bytes(lens) + tab + B * hq * d * qsz + B * hq * d * 4 + 2 * parts * hq * (d + 2) * 4
 
     launches_per = []
 
@@ -308,12 +319,20 @@ def run_ours(args):
         if st["ncow"]:
             P.pkv_copy_blocks(cache.k_pool, cache.v_pool, st["cow"])
             n += 1
-        P.pkv_kv_append(st["kn"], st["vn"], st["slots"], cache.k_pool, cache.v_pool)
+        if fp8:
+            P.pkv_kv_append_fp8(st["kn"], st["vn"], st["slots"], cache.k_pool, cache.v_pool, w.kv_scale, w.kv_scale)
+        else:
+            P.pkv_kv_append(st["kn"], st["vn"], st["slots"], cache.k_pool, cache.v_pool)
         n += 1
         if ev is not None:
             ev[0].record()
-        P.pkv_paged_attention_decode(st["q"], cache.k_pool, cache.v_pool, st["tables"], st["lens"], w.scale,
-                                     out=out, workspace=workspace, partition_tokens=w.partition_tokens)
+        if fp8:
+            P.pkv_paged_attention_decode_fp8(st["q"], cache.k_pool, cache.v_pool, st["tables"], st["lens"], w.scale,
+                                             w.kv_scale, w.kv_scale, out=out, workspace=workspace,
+                                             partition_tokens=w.partition_tokens)
+        else:
+            P.pkv_paged_attention_decode(st["q"], cache.k_pool, cache.v_pool, st["tables"], st["lens"], w.scale,
+                                         out=out, workspace=workspace, partition_tokens=w.partition_tokens)
         if ev is not None:
             ev[1].record()
         n += 2  # plan + decode (partition merge runs inside the decode kernel)
@@ -365,7 +384,7 @@ def run_ours(args):
         E = args.e2e_steps
         host_in = []
         for s in range(min(E, STAGED_STEPS)):
-            host_in.append(tuple(W.normal(shape, w.torch_dtype, W.step_seed(w, 100 + s, k)).pin_memory()
+            host_in.append(tuple(W.normal(shape, w.io_dtype, W.step_seed(w, 100 + s, k)).pin_memory()
                                  for k, shape in ((0, (B, hq, d)), (1, (B, hkv, d)), (2, (B, hkv, d)))))
         out_host = torch.empty((B, hq, d), dtype=torch.float32, pin_memory=True)
         for s in range(3):  # warm-up
@@ -390,7 +409,7 @@ def run_ours(args):
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
         e2e_ms_all, e2e_bytes_all, _ = combine_ranks(e2e_ms, float(sum(e_lens)), float(B * E), dev)
-        h2d = (B * hq * d + 2 * B * hkv * d) * esz + meta_bytes // E
+        h2d = (B * hq * d + 2 * B * hkv * d) * qsz + meta_bytes // E
         e2e = {"value": round(e2e_bytes_all / (e2e_ms_all * 1e-3) / 1e9, 2), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(B * hq * d * 4),
                "ms_per_step": round(e2e_ms_all / E, 4),

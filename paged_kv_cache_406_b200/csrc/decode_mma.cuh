@@ -30,6 +30,12 @@
 namespace pkv {
 
 constexpr int kChunkTokens = 16;
+// Two producer warps share the issuing: warp kConsumerWarps + pr issues the
+// chunks whose CTA-wide index has parity pr (the ring stages of that parity).
+// One lane issuing every TMA load (~150 cycles each plus its bookkeeping) was
+// the measured limit of the single-producer kernel.
+constexpr int kMmaProducers = 2;
+constexpr int kMmaThreads = (kConsumerWarps + kMmaProducers) * 32;
 
 // kKVBytes = bytes per stored K/V element: 2 (bf16 / f16) or 1 (e4m3).
 template <int D, int kKVBytes = 2>
@@ -53,23 +59,27 @@ struct MmaSmem {
   __host__ __device__ static size_t bytes(int ns) {
     // + 1024: the dynamic shared memory base is aligned up to the 1024-byte swizzle atom
     return 1024 + ring_bytes(ns) + 2 * kConsumerWarps * kMergeFloats * sizeof(float) + 2 * ns * sizeof(uint64_t) +
-           16 + 128;
+           16 + kMmaProducers * 128;
   }
 };
 
+// Two e4m3 codes (low byte first) widened exactly to a packed f16 pair.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t codes) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(codes));
+  return r;
+}
+
 // 16 e4m3 codes (one 16-byte chunk) widened exactly to 16 f16 values.
 __device__ __forceinline__ void widen_e4m3x16(const uint4& in, uint4& lo, uint4& hi) {
-  const uint32_t w[4] = {in.x, in.y, in.z, in.w};
-  uint32_t o[8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] & 0xffffu), __NV_E4M3);
-    const __half2_raw b = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] >> 16), __NV_E4M3);
-    o[2 * i] = static_cast<uint32_t>(a.x) | (static_cast<uint32_t>(a.y) << 16);
-    o[2 * i + 1] = static_cast<uint32_t>(b.x) | (static_cast<uint32_t>(b.y) << 16);
-  }
-  lo = make_uint4(o[0], o[1], o[2], o[3]);
-  hi = make_uint4(o[4], o[5], o[6], o[7]);
+  lo.x = e4m3x2_to_f16x2(static_cast<uint16_t>(in.x));
+  lo.y = e4m3x2_to_f16x2(static_cast<uint16_t>(in.x >> 16));
+  lo.z = e4m3x2_to_f16x2(static_cast<uint16_t>(in.y));
+  lo.w = e4m3x2_to_f16x2(static_cast<uint16_t>(in.y >> 16));
+  hi.x = e4m3x2_to_f16x2(static_cast<uint16_t>(in.z));
+  hi.y = e4m3x2_to_f16x2(static_cast<uint16_t>(in.z >> 16));
+  hi.z = e4m3x2_to_f16x2(static_cast<uint16_t>(in.w));
+  hi.w = e4m3x2_to_f16x2(static_cast<uint16_t>(in.w >> 16));
 }
 
 // A chunk tile in shared memory is built from TMA boxes of `br` rows (br = 16,
@@ -86,7 +96,7 @@ __device__ __forceinline__ uint32_t row_offset(int r, int h, int br_shift, int h
 // f16 exactly); the consumer warp widens each landed chunk into its own
 // 16-bit staging tile and frees the ring stage before the MMAs.
 template <typename T, int D, int G, int kKVBytes = 2>
-__global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const DecodeParams p,
+__global__ void __launch_bounds__(kMmaThreads) decode_mma_kernel(const DecodeParams p,
                                                                     const __grid_constant__ CUtensorMap tmap_k,
                                                                     const __grid_constant__ CUtensorMap tmap_v) {
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
@@ -107,7 +117,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
   uint64_t* full = reinterpret_cast<uint64_t*>(merge + 2 * kConsumerWarps * kMF);
   uint64_t* empty = full + NS;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + NS);
-  int32_t* tab = reinterpret_cast<int32_t*>(empty + NS) + 4;  // 32 block-table entries
+  int32_t* tab = reinterpret_cast<int32_t*>(empty + NS) + 4;  // 32 block-table entries per producer
   const uint32_t ring_s = smem_addr(smem);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -125,11 +135,14 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
 
   const int n_work = *p.n_items * p.num_kv_heads;
 
-  if (warp == kConsumerWarps) {
-    // ----------------------------- producer -----------------------------
-    // All lanes walk the units and refill the table window; lane 0 alone
-    // issues the chunks of each window, so the per-chunk path has no
-    // warp-wide synchronisation.
+  if (warp >= kConsumerWarps) {
+    // ----------------------------- producers -----------------------------
+    // Both producer warps walk every unit and refill their own 32-entry
+    // block-table window; lane 0 of producer pr alone issues the window's
+    // chunks of parity pr, so the per-chunk path has no warp-wide
+    // synchronisation.
+    const int pr = warp - kConsumerWarps;
+    int32_t* mytab = tab + 32 * pr;
     if (lane == 0) {
       prefetch_tensormap(&tmap_k);
       prefetch_tensormap(&tmap_v);
@@ -137,8 +150,9 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
     const uint64_t policy = l2_evict_first_policy();
     const uint32_t box_bytes = (1u << br_shift) * D * kKVBytes;        // one K (or V) box
     const uint32_t blk_off = L::kRingHalves * (1u << br_shift) * 128;  // second box of a chunk (block_size 8)
-    int s = 0;
+    int s = pr;           // this producer's stages: pr, pr + 2, ...
     uint32_t ph = 0, issued = 0;
+    uint32_t cg = 0;      // CTA-wide chunk index of the unit's first chunk
     bool ok = true;
     for (int w = blockIdx.x; w < n_work && ok; w += gridDim.x) {
       const WorkUnit u = load_unit(p, w);
@@ -146,11 +160,12 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
       const int nch = (u.t1 - u.t0 + kChunkTokens - 1) / kChunkTokens;
       const int ybase = u.g * BS;
       for (int wb = 0; wb < u.nblk && ok; wb += 32) {
-        tab[lane] = wb + lane < u.nblk ? trow[wb + lane] : 0;
+        mytab[lane] = wb + lane < u.nblk ? trow[wb + lane] : 0;
         __syncwarp();
         if (lane == 0) {
+          const int k_begin = (wb << bs_shift) >> 4;
           const int k_end = min(nch, ((wb + 32) << bs_shift) >> 4);
-          for (int k = (wb << bs_shift) >> 4; k < k_end; ++k) {
+          for (int k = k_begin + ((pr - static_cast<int>(cg) - k_begin) & 1); k < k_end; k += kMmaProducers) {
             if (!mbar_wait(smem_addr(empty + s), ph ^ 1, abort_flag)) {
               record_error(PKV_ERR_DEVICE_TIMEOUT);
               *abort_flag = 1;
@@ -164,7 +179,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
             const uint32_t kdst = ring_s + s * L::kStageBytes;
             mbar_arrive_expect_tx(bar, nb_here * 2 * box_bytes);
             for (int i = 0; i < nb_here; ++i) {
-              int phys = tab[jb - wb + i];
+              int phys = mytab[jb - wb + i];
               if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_blocks)) {
                 record_error(PKV_ERR_BAD_BLOCK);
                 phys = 0;
@@ -174,8 +189,9 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
               tma_load_3d(kdst + L::kRingTileBytes + i * blk_off, &tmap_v, 0, y, 0, bar, policy);
             }
             ++issued;
-            if (++s == NS) {
-              s = 0;
+            s += kMmaProducers;
+            if (s >= NS) {
+              s -= NS;
               ph ^= 1;
             }
           }
@@ -183,12 +199,15 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
         __syncwarp();
         ok = __shfl_sync(kFull, ok, 0);
       }
+      cg += nch;
     }
     // No copy may still be landing in shared memory when the CTA exits: wait
-    // (bounded) for the last phase issued into every stage.
+    // (bounded) for the last phase issued into each of this producer's stages.
     if (lane == 0) {
-      for (int st = 0; st < NS && st < static_cast<int>(issued); ++st) {
-        const uint32_t uses = (issued - st + NS - 1) / NS;
+      const int mine = NS / kMmaProducers;  // stages pr, pr + 2, ...
+      for (int j = 0; j < mine && j < static_cast<int>(issued); ++j) {
+        const uint32_t uses = (issued - j + mine - 1) / mine;
+        const int st = pr + kMmaProducers * j;
         const uint64_t t0 = global_timer_ns();
         while (!mbar_try_wait(smem_addr(full + st), (uses - 1) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
         }
@@ -257,28 +276,32 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(const Decode
       const int nv = min(kChunkTokens, u.t1 - (u.t0 + k * kChunkTokens));
       if constexpr (kFp8) {
         // widen the e4m3 chunk (rows of 128 B, 128-byte swizzle) into the
-        // 16-bit staging layout, then hand the ring stage back at once
+        // 16-bit staging layout, then hand the ring stage back at once; plain
+        // shared-memory accesses so all eight loads are in flight together
+        const unsigned char* ksrc = smem + (kbase - ring_s);
+        const unsigned char* vsrc = smem + (vbase - ring_s);
+        unsigned char* dst = smem + (staging - ring_s);
+        uint4 rk[4], rv[4];
+        uint32_t d0[4], d1[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int i = lane + 32 * j, row = i >> 3, c = i & 7;  // 16 codes: dims 16c .. 16c+15
-          const uint32_t src = static_cast<uint32_t>(row * 128 + ((c ^ (row & 7)) << 4));
-          const uint32_t d0 = row_offset(row, c >> 2, 4, kHalves) + ((((c & 3) << 1) ^ (row & 7)) << 4);
-          const uint32_t d1 = row_offset(row, c >> 2, 4, kHalves) + (((((c & 3) << 1) + 1) ^ (row & 7)) << 4);
-          uint4 raw, lo, hi;
-          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(raw.x), "=r"(raw.y), "=r"(raw.z), "=r"(raw.w) : "r"(kbase + src));
-          widen_e4m3x16(raw, lo, hi);
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(staging + d0), "r"(lo.x), "r"(lo.y),
-                       "r"(lo.z), "r"(lo.w) : "memory");
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(staging + d1), "r"(hi.x), "r"(hi.y),
-                       "r"(hi.z), "r"(hi.w) : "memory");
-          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(raw.x), "=r"(raw.y), "=r"(raw.z), "=r"(raw.w) : "r"(vbase + src));
-          widen_e4m3x16(raw, lo, hi);
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(staging + L::kTileBytes + d0), "r"(lo.x),
-                       "r"(lo.y), "r"(lo.z), "r"(lo.w) : "memory");
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(staging + L::kTileBytes + d1), "r"(hi.x),
-                       "r"(hi.y), "r"(hi.z), "r"(hi.w) : "memory");
+          const int src = row * 128 + ((c ^ (row & 7)) << 4);
+          rk[j] = *reinterpret_cast<const uint4*>(ksrc + src);
+          rv[j] = *reinterpret_cast<const uint4*>(vsrc + src);
+          const uint32_t base = row_offset(row, c >> 2, 4, kHalves);
+          d0[j] = base + ((((c & 3) << 1) ^ (row & 7)) << 4);
+          d1[j] = base + (((((c & 3) << 1) + 1) ^ (row & 7)) << 4);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint4 lo, hi;
+          widen_e4m3x16(rk[j], lo, hi);
+          *reinterpret_cast<uint4*>(dst + d0[j]) = lo;
+          *reinterpret_cast<uint4*>(dst + d1[j]) = hi;
+          widen_e4m3x16(rv[j], lo, hi);
+          *reinterpret_cast<uint4*>(dst + L::kTileBytes + d0[j]) = lo;
+          *reinterpret_cast<uint4*>(dst + L::kTileBytes + d1[j]) = hi;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_addr(empty + s));

@@ -238,13 +238,13 @@ cudaError_t launch_pdl(Kernel kern, dim3 grid, dim3 block, size_t smem, cudaStre
 // sequence can span more than one partition)
 template <int D, typename Kernel, typename... Args>
 int launch_plan_decode_merge(const pkv::DecodeParams& p, const int32_t* seq_lens, int32_t num_seqs,
-                             int32_t max_tokens, Kernel kern, int grid, size_t smem, cudaStream_t stream,
+                             int32_t max_tokens, Kernel kern, int grid, int threads, size_t smem, cudaStream_t stream,
                              Args... args) {
   const int kmax = p.partition_tokens / p.block_size;
   pkv::plan_kernel<<<1, 1024, 2 * (kmax + 1) * sizeof(int32_t), stream>>>(
       seq_lens, num_seqs, max_tokens, p.partition_tokens, p.block_size, const_cast<int4*>(p.items),
       const_cast<int32_t*>(p.n_items));
-  cudaError_t e = launch_pdl(kern, dim3(grid), dim3(pkv::kDecodeThreads), smem, stream, p, args...);
+  cudaError_t e = launch_pdl(kern, dim3(grid), dim3(threads), smem, stream, p, args...);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   if (p.max_parts > 1) {
     const int rows = num_seqs * p.num_q_heads;
@@ -291,7 +291,7 @@ int launch_decode(const pkv::DecodeParams& base, const int32_t* seq_lens, int32_
 
   const int64_t work_upper = int64_t(num_seqs) * p.max_parts * p.num_kv_heads;
   const int grid = static_cast<int>(std::min<int64_t>(int64_t(sm_count(dev)) * occ, work_upper));
-  return launch_plan_decode_merge<D>(p, seq_lens, num_seqs, max_tokens, kern, grid, smem, stream);
+  return launch_plan_decode_merge<D>(p, seq_lens, num_seqs, max_tokens, kern, grid, pkv::kDecodeThreads, smem, stream);
 }
 
 // ---- tensor maps over the K/V pools for the tensor-core kernel ----
@@ -389,7 +389,7 @@ int launch_decode_mma(const pkv::DecodeParams& base, const int32_t* seq_lens, in
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_mma)");
     e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(carveout)");
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, pkv::kDecodeThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, pkv::kMmaThreads, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
     if (occ <= 0) return fail(PKV_ERR_CUDA, "decode_mma kernel does not fit on an SM (smem %zu)", smem);
     if (dev < kMaxDevices) occ_cache[dev].store(occ, std::memory_order_relaxed);
@@ -404,7 +404,8 @@ int launch_decode_mma(const pkv::DecodeParams& base, const int32_t* seq_lens, in
 
   const int64_t work_upper = int64_t(num_seqs) * p.max_parts * p.num_kv_heads;
   const int grid = static_cast<int>(std::min<int64_t>(int64_t(sm_count(dev)) * occ, work_upper));
-  return launch_plan_decode_merge<D>(p, seq_lens, num_seqs, max_tokens, kern, grid, smem, stream, mk, mv);
+  return launch_plan_decode_merge<D>(p, seq_lens, num_seqs, max_tokens, kern, grid, pkv::kMmaThreads, smem, stream, mk,
+                                     mv);
 }
 
 template <typename T>

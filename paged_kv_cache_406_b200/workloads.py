@@ -22,7 +22,7 @@ from dataclasses import dataclass, replace
 import numpy as np
 import torch
 
-TORCH_DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}
+TORCH_DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16, "e4m3": torch.float8_e4m3fn}
 
 
 @dataclass(frozen=True)
@@ -33,16 +33,22 @@ class Workload:
     num_kv_heads: int
     head_dim: int
     block_size: int
-    dtype: str            # "f32" | "bf16" | "f16"
+    dtype: str            # pool element type: "f32" | "bf16" | "f16" | "e4m3"
     seed: int
     steps: int = 1        # decode steps (one appended token per sequence each)
     partition_tokens: int = 0  # 0 = library default
     prefix_tokens: int = 0     # tokens shared by every sequence (refcount = num_seqs)
     pool_slack: float = 1.2    # pool size as a multiple of the blocks needed
+    kv_scale: float = 1.0 / 32  # e4m3 pools: value = kv_scale * code value (K and V)
 
     @property
     def torch_dtype(self) -> torch.dtype:
         return TORCH_DTYPES[self.dtype]
+
+    @property
+    def io_dtype(self) -> torch.dtype:
+        """Element type of q and of the new K/V rows (float16 for e4m3 pools)."""
+        return torch.float16 if self.dtype == "e4m3" else TORCH_DTYPES[self.dtype]
 
     @property
     def group(self) -> int:
@@ -58,6 +64,8 @@ WORKLOADS = {
     "tiny": Workload("tiny", 4, 4, 4, 64, 16, "f32", 406001, pool_slack=0.0),
     # Llama-3-8B-shaped layer: 64 sequences of U[512, 4096] tokens, GQA 32/8, bf16
     "llama3_8b": Workload("llama3_8b", 64, 32, 8, 128, 16, "bf16", 406002),
+    # the same batch with an e4m3 KV cache (scale 1/32), q and new rows float16
+    "llama3_8b_fp8": Workload("llama3_8b_fp8", 64, 32, 8, 128, 16, "e4m3", 406002),
     # 32 sequences sharing a 1024-token prefix plus U[64, 512]-token tails
     "prefix_shared_bs8": Workload("prefix_shared_bs8", 32, 32, 8, 128, 8, "bf16", 406003, prefix_tokens=1024),
     "prefix_shared_bs16": Workload("prefix_shared_bs16", 32, 32, 8, 128, 16, "bf16", 406003, prefix_tokens=1024),
@@ -121,6 +129,15 @@ def normal(shape, dtype: torch.dtype, seed: int, device="cpu") -> torch.Tensor:
         return torch.randn(shape, generator=g, device=device, dtype=dtype)
     x = np.random.Generator(np.random.PCG64(seed)).standard_normal(size=shape, dtype=np.float32)
     return torch.from_numpy(x).to(dtype)
+
+
+def pool_values(shape, w: Workload, which: int, device="cpu") -> torch.Tensor:
+    """Initial pool contents: N(0, 1) in the pool dtype; for e4m3 pools the
+    codes of N(0, 1) / kv_scale (torch's float8 cast, round to nearest even)."""
+    if w.dtype == "e4m3":
+        x = normal(shape, torch.float32, pool_seed(w, which), device)
+        return (x / w.kv_scale).to(torch.float8_e4m3fn)
+    return normal(shape, w.torch_dtype, pool_seed(w, which), device)
 
 
 def step_seed(w: Workload, step: int, what: int) -> int:
