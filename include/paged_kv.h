@@ -93,6 +93,9 @@ typedef struct pkv_stats {
   int64_t cow_copies;     /* copy-on-write pairs issued since creation */
   int64_t logical_tokens; /* sum of sequence lengths (shared tokens counted per sharer) */
   int64_t waste_tokens;   /* over distinct used blocks: block_size - the fullest sharer's fill */
+  int64_t cached_blocks;  /* blocks indexed by the prefix cache (in use or cached-free) */
+  int64_t cache_queries;  /* full prompt blocks looked up by pkv_seq_add_cached */
+  int64_t cache_hits;     /* of those, blocks reused */
 } pkv_stats_t;
 
 /* Create an allocator over blocks 0..num_blocks-1.  The free list is a LIFO
@@ -112,6 +115,23 @@ void pkv_alloc_destroy(pkv_alloc_t* a);
  * Errors: SEQ_EXISTS, OUT_OF_BLOCKS, INVALID_ARG (n_tokens < 0). */
 int pkv_seq_add(pkv_alloc_t* a, int64_t seq_id, int32_t n_tokens);
 
+/* Admit a sequence whose n_tokens prompt token ids are known, reusing cached
+ * blocks of an identical prefix (prefix caching: vLLM paging page §3 phase 3
+ * and §5 "enable_prefix_caching"; vLLM production page §5).  Each full block
+ * of the prompt is identified by the token ids of the whole prefix through
+ * it (64-bit FNV-1a chain hash, verified against stored tokens on every
+ * hit).  The longest run of leading full blocks found in the cache is reused
+ * (refcount + 1); the rest, including a partial last block, are fresh, and
+ * fresh full blocks are registered.  A registered block whose refcount
+ * reaches zero stays cached ("cached-free", still counted as free) until a
+ * hit revives it or the free stack runs dry and it is evicted, least
+ * recently freed first.  *n_cached_tokens (may be NULL) receives the number
+ * of leading tokens whose K/V are already in the pool (reused blocks x
+ * block_size); the caller computes and appends the rest.  All-or-nothing.
+ * Errors: SEQ_EXISTS, OUT_OF_BLOCKS, INVALID_ARG. */
+int pkv_seq_add_cached(pkv_alloc_t* a, int64_t seq_id, const int32_t* tokens, int32_t n_tokens,
+                       int32_t* n_cached_tokens);
+
 /* Make `child` share every block of `parent` (refcount + 1 each); child gets
  * parent's length.  Prefix sharing, vLLM paging page §3 phase 3.
  * Errors: UNKNOWN_SEQ (parent), SEQ_EXISTS (child). */
@@ -120,8 +140,9 @@ int pkv_seq_fork(pkv_alloc_t* a, int64_t parent, int64_t child);
 /* Reserve the slot of one new token for each listed sequence, in list order
  * (vLLM paging page §3 phase 1).  For a sequence of length L the new token is
  * position L:
- *   - if L % block_size == 0 a block is popped from the free list and
- *     appended to its table;
+ *   - if L % block_size == 0 a block is popped from the free list (or a
+ *     cached-free block is evicted when the list is empty) and appended to
+ *     its table;
  *   - else if its last block is shared (refcount > 1) a block is popped, the
  *     pair (old, new) is written to cow_pairs_out (copy the old block's K/V
  *     into the new one before writing the token: pkv_copy_blocks), the old

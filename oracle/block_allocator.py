@@ -26,6 +26,25 @@ Readings where the page is silent (the C++ allocator implements the same):
 * every failing call leaves the state exactly as it was (all-or-nothing);
 * a freed sequence returns its blocks in table order, so its last block ends
   on top of the stack.
+
+Prefix caching (vLLM paging page §3 phase 3 and §5 "enable_prefix_caching";
+vLLM production page §5: reusing blocks costs hashing time and helps only
+repeated prefixes) — readings taken:
+
+* a *full* block admitted with known token ids is identified by the token ids
+  of the whole prefix up to and including it (the chain of its predecessors);
+  a sequence admitted with ``add_cached`` reuses the longest run of leading
+  full blocks whose identities are cached (refcount + 1) and takes fresh blocks
+  for the rest; its partial last block is always fresh;
+* fresh full blocks of an ``add_cached`` admission are registered under their
+  identity unless that identity is already registered (a later block of a
+  prefix can outlive an evicted earlier one); blocks filled later by appends
+  are not registered;
+* a registered block whose refcount drops to zero stays registered as
+  *cached-free*: a later hit revives it; it is evicted (unregistered and handed
+  out) only when the free stack is empty, least recently freed first;
+* a registered block is never written (appends go to partial blocks, which are
+  never registered).
 """
 from __future__ import annotations
 
@@ -57,21 +76,38 @@ class BlockAllocatorModel:
         self.refcount = [0] * num_blocks
         self.seqs: dict[int, list] = {}  # id -> [table, length]
         self.cow_copies = 0
+        self.cache: dict[tuple, int] = {}  # prefix token tuple -> block
+        self.block_key: dict[int, tuple] = {}
+        self.lru: list[int] = []           # cached-free blocks, least recently freed first
+        self.cache_queries = 0
+        self.cache_hits = 0
 
     # -- helpers --------------------------------------------------------
     def _pop(self) -> int:
-        if not self.free:
+        if self.free:
+            b = self.free.pop()
+        elif self.lru:  # evict the least recently freed cached block
+            b = self.lru.pop(0)
+            del self.cache[self.block_key.pop(b)]
+        else:
             raise AllocatorError(ERR_OUT_OF_BLOCKS, "no free block")
-        b = self.free.pop()
         self.refcount[b] = 1
         return b
 
+    def _available(self) -> int:
+        return len(self.free) + len(self.lru)
+
+    def _state(self):
+        return (self.free, self.refcount, self.seqs, self.cow_copies, self.cache, self.block_key, self.lru,
+                self.cache_queries, self.cache_hits)
+
     def _atomic(self, fn):
-        saved = copy.deepcopy((self.free, self.refcount, self.seqs, self.cow_copies))
+        saved = copy.deepcopy(self._state())
         try:
             return fn()
         except AllocatorError:
-            self.free, self.refcount, self.seqs, self.cow_copies = saved
+            (self.free, self.refcount, self.seqs, self.cow_copies, self.cache, self.block_key, self.lru,
+             self.cache_queries, self.cache_hits) = saved
             raise
 
     # -- operations ------------------------------------------------------
@@ -81,10 +117,46 @@ class BlockAllocatorModel:
         if seq_id in self.seqs:
             raise AllocatorError(ERR_SEQ_EXISTS, "sequence exists")
         need = -(-n_tokens // self.block_size)
-        if need > len(self.free):
+        if need > self._available():
             raise AllocatorError(ERR_OUT_OF_BLOCKS, "admission refused")
         table = [self._pop() for _ in range(need)]
         self.seqs[seq_id] = [table, n_tokens]
+
+    def add_cached(self, seq_id: int, tokens) -> int:
+        """Admit a sequence holding ``tokens``, reusing cached full blocks of its
+        prefix; returns the number of leading tokens whose blocks were reused."""
+        tokens = [int(t) for t in tokens]
+        if seq_id in self.seqs:
+            raise AllocatorError(ERR_SEQ_EXISTS, "sequence exists")
+        bs = self.block_size
+        n = len(tokens)
+        nfull = n // bs
+        hits = 0
+        while hits < nfull and tuple(tokens[:(hits + 1) * bs]) in self.cache:
+            hits += 1
+        need = -(-n // bs) - hits
+        # revived cached-free blocks leave the evictable set, so they do not count as available
+        revived = sum(1 for i in range(hits) if self.refcount[self.cache[tuple(tokens[:(i + 1) * bs])]] == 0)
+        if need > self._available() - revived:
+            raise AllocatorError(ERR_OUT_OF_BLOCKS, "admission refused")
+        self.cache_queries += nfull
+        self.cache_hits += hits
+        table = []
+        for i in range(hits):
+            b = self.cache[tuple(tokens[:(i + 1) * bs])]
+            if self.refcount[b] == 0:
+                self.lru.remove(b)
+            self.refcount[b] += 1
+            table.append(b)
+        for i in range(hits, -(-n // bs)):
+            b = self._pop()
+            table.append(b)
+            key = tuple(tokens[:(i + 1) * bs])
+            if i < nfull and key not in self.cache:  # a later block may still be cached after an eviction
+                self.cache[key] = b
+                self.block_key[b] = key
+        self.seqs[seq_id] = [table, n]
+        return hits * bs
 
     def fork(self, parent: int, child: int) -> None:
         if parent not in self.seqs:
@@ -128,7 +200,10 @@ class BlockAllocatorModel:
         for b in table:
             self.refcount[b] -= 1
             if self.refcount[b] == 0:
-                self.free.append(b)
+                if b in self.block_key:
+                    self.lru.append(b)  # stays cached until evicted
+                else:
+                    self.free.append(b)
 
     def block_table(self, seq_id: int) -> list:
         return list(self.seqs[seq_id][0])
@@ -144,12 +219,15 @@ class BlockAllocatorModel:
                 fill[b] = max(fill.get(b, 0), used)
         return {
             "num_blocks": self.num_blocks,
-            "free_blocks": len(self.free),
-            "used_blocks": self.num_blocks - len(self.free),
+            "free_blocks": len(self.free) + len(self.lru),
+            "used_blocks": self.num_blocks - len(self.free) - len(self.lru),
             "num_seqs": len(self.seqs),
             "cow_copies": self.cow_copies,
             "logical_tokens": sum(n for _, n in self.seqs.values()),
             "waste_tokens": sum(self.block_size - f for f in fill.values()),
+            "cached_blocks": len(self.block_key),
+            "cache_queries": self.cache_queries,
+            "cache_hits": self.cache_hits,
         }
 
     def check_invariants(self) -> None:
@@ -161,8 +239,14 @@ class BlockAllocatorModel:
                 count[b] += table.count(b)
         assert count == self.refcount, "refcount != number of tables holding the block"
         free = set(self.free)
+        lru = set(self.lru)
         assert len(free) == len(self.free), "block twice on the free list"
+        assert len(lru) == len(self.lru), "block twice on the cached-free list"
+        assert not free & lru
         for b in range(self.num_blocks):
-            assert (self.refcount[b] == 0) == (b in free)
+            assert (self.refcount[b] == 0) == (b in free or b in lru)
+        assert lru <= set(self.block_key), "cached-free blocks are registered"
+        assert not free & set(self.block_key), "stack blocks are not registered"
+        assert all(self.cache[k] == b for b, k in self.block_key.items())
         used = sum(1 for r in self.refcount if r > 0)
-        assert used + len(self.free) == self.num_blocks
+        assert used + len(self.free) + len(self.lru) == self.num_blocks

@@ -34,7 +34,7 @@ _pi64 = ctypes.POINTER(ctypes.c_int64)
 class pkv_stats_t(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int64) for n in (
         "num_blocks", "block_size", "free_blocks", "used_blocks", "num_seqs", "cow_copies",
-        "logical_tokens", "waste_tokens")]
+        "logical_tokens", "waste_tokens", "cached_blocks", "cache_queries", "cache_hits")]
 
 
 SIGNATURES = {
@@ -44,6 +44,7 @@ SIGNATURES = {
     "pkv_alloc_destroy": (None, [_vp]),
     "pkv_seq_add": (ctypes.c_int, [_vp, _i64, _i32]),
     "pkv_seq_fork": (ctypes.c_int, [_vp, _i64, _i64]),
+    "pkv_seq_add_cached": (ctypes.c_int, [_vp, _i64, _pi32, _i32, _pi32]),
     "pkv_seq_append_slots": (ctypes.c_int, [_vp, _pi64, _i32, _pi32, _pi32, _i32, _pi32]),
     "pkv_seq_free": (ctypes.c_int, [_vp, _i64]),
     "pkv_seq_len": (ctypes.c_int, [_vp, _i64, _pi32]),

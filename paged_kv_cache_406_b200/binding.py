@@ -259,6 +259,15 @@ class Allocator:
     def add(self, seq_id: int, n_tokens: int) -> None:
         check(lib().pkv_seq_add(self._h, seq_id, n_tokens))
 
+    def add_cached(self, seq_id: int, tokens) -> int:
+        """Admit a sequence with known prompt token ids, reusing cached blocks of
+        an identical prefix; returns the number of leading tokens already cached."""
+        t = np.ascontiguousarray(np.asarray(tokens, dtype=np.int32))
+        n = ctypes.c_int32(0)
+        check(lib().pkv_seq_add_cached(self._h, seq_id, t.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), t.size,
+                                       ctypes.byref(n)))
+        return n.value
+
     def fork(self, parent: int, child: int) -> None:
         check(lib().pkv_seq_fork(self._h, parent, child))
 

@@ -54,6 +54,12 @@ class PagedKVCache:
     def add(self, seq_id: int, n_tokens: int) -> None:
         self.alloc.add(seq_id, n_tokens)
 
+    def add_cached(self, seq_id: int, tokens) -> int:
+        """Admit a sequence by its token ids, reusing cached full blocks of its
+        prefix; returns how many leading tokens already sit in the pool (the
+        caller writes K/V only for the rest)."""
+        return self.alloc.add_cached(seq_id, tokens)
+
     def fork(self, parent: int, child: int) -> None:
         self.alloc.fork(parent, child)
 

@@ -154,3 +154,61 @@ def test_errors_leave_state_unchanged(native):
     with pytest.raises(PagedKVError) as e:
         nat.block_tables([0], 0)
     assert e.value.code == -1
+
+
+@pytest.mark.parametrize("seed", [3, 4])
+def test_prefix_cache_matches_model(native, seed):
+    """add_cached, appends, forks and frees on the C++ allocator and the model:
+    identical reuse counts, tables, slots, statistics and error codes, with
+    eviction of cached-free blocks when the pool runs dry."""
+    rng = np.random.default_rng(seed)
+    bs, nb = 4, 50
+    order = rng.permutation(nb)
+    model = BlockAllocatorModel(nb, bs, order)
+    nat = Allocator(nb, bs, order)
+    prefixes = [list(rng.integers(0, 4, size=16)) for _ in range(3)]
+    live, nxt = [], 0
+    for _ in range(1500):
+        op = int(rng.integers(0, 5))
+        m_err = n_err = m_res = n_res = None
+        if op <= 1 or not live:
+            toks = prefixes[int(rng.integers(3))][: int(rng.integers(0, 17))] + \
+                [int(x) for x in rng.integers(0, 4, size=int(rng.integers(0, 7)))]
+            try:
+                m_res = model.add_cached(nxt, toks)
+            except AllocatorError as e:
+                m_err = e.code
+            try:
+                n_res = nat.add_cached(nxt, toks)
+            except PagedKVError as e:
+                n_err = e.code
+            assert m_res == n_res
+            if m_err is None:
+                live.append(nxt)
+            nxt += 1
+        elif op == 2:
+            ids = [int(x) for x in rng.choice(live, size=int(rng.integers(1, len(live) + 1)))]
+            try:
+                ms, mc = model.append_slots(ids)
+            except AllocatorError as e:
+                m_err = e.code
+            try:
+                ns, nc = nat.append_slots(ids)
+            except PagedKVError as e:
+                n_err = e.code
+            if m_err is None and n_err is None:
+                assert ns.tolist() == ms and [tuple(x) for x in nc.tolist()] == mc
+        elif op == 3:
+            p = live[int(rng.integers(len(live)))]
+            model.fork(p, nxt)
+            nat.fork(p, nxt)
+            live.append(nxt)
+            nxt += 1
+        else:
+            v = live.pop(int(rng.integers(len(live))))
+            model.free_seq(v)
+            nat.free(v)
+        assert m_err == n_err
+        model.check_invariants()
+        _same(model, nat, live)
+    assert nat.stats()["cache_hits"] > 0

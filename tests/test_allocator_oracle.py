@@ -3,8 +3,10 @@
 Pinned by the worked paging example of the vLLM paging page (§3 phases 1 and
 3, stored in ``tests/golden/paging_example.json``), by closed-form block counts
 (``ceil(n / block_size)`` blocks per sequence, ``n - 1`` copies when ``n``
-sharers each append into a shared partial block), and by the bookkeeping
-invariants checked after every operation of a seeded random workload.
+sharers each append into a shared partial block; for prefix caching the
+number of reused blocks, the prefix property, revival and eviction order, and
+blocks used by a shared system prompt), and by the bookkeeping invariants
+checked after every operation of seeded random workloads.
 """
 import json
 import os
@@ -167,3 +169,124 @@ def test_waste_accounting():
     a.fork(0, 2)  # shared blocks counted once
     assert a.stats()["waste_tokens"] == 15
     assert a.stats()["logical_tokens"] == 17 + 32 + 17
+
+
+# ---------------------------------------------------------------------------
+# prefix caching (vLLM paging page §3 phase 3, §5; vLLM production page §5)
+# ---------------------------------------------------------------------------
+
+def test_prefix_cache_reuses_full_blocks_of_identical_prefix():
+    bs = 4
+    a = BlockAllocatorModel(64, bs)
+    toks = list(range(100, 114))  # 14 tokens: 3 full blocks + 2
+    assert a.add_cached(0, toks) == 0
+    assert a.add_cached(1, toks) == 12  # the 3 full blocks, never the partial one
+    t0, t1 = a.block_table(0), a.block_table(1)
+    assert t1[:3] == t0[:3] and t1[3] != t0[3]
+    assert all(a.refcount[b] == 2 for b in t0[:3])
+    st = a.stats()
+    assert (st["cache_queries"], st["cache_hits"], st["cached_blocks"]) == (6, 3, 3)
+    a.check_invariants()
+
+
+def test_prefix_cache_stops_at_first_difference():
+    bs = 4
+    a = BlockAllocatorModel(64, bs)
+    base = list(range(16))
+    a.add_cached(0, base)
+    other = base[:4] + [99] + base[5:]  # differs inside block 1
+    assert a.add_cached(1, other) == 4
+    assert a.block_table(1)[0] == a.block_table(0)[0]
+    assert a.block_table(1)[1:] != a.block_table(0)[1:]
+    # a prefix of a block is not a hit: 3 tokens of block 0 only
+    assert a.add_cached(2, base[:3]) == 0
+    a.check_invariants()
+
+
+def test_cached_blocks_survive_free_and_are_revived():
+    bs = 4
+    a = BlockAllocatorModel(16, bs)
+    toks = list(range(8))
+    a.add_cached(0, toks)
+    t0 = a.block_table(0)
+    a.free_seq(0)
+    st = a.stats()
+    assert st["free_blocks"] == 16 and st["cached_blocks"] == 2  # free to use, still cached
+    assert a.add_cached(1, toks) == 8
+    assert a.block_table(1) == t0
+    a.check_invariants()
+
+
+def test_cached_free_blocks_are_evicted_least_recently_freed_first():
+    bs = 2
+    a = BlockAllocatorModel(4, bs, free_order=[0, 1, 2, 3])
+    a.add_cached(0, [1, 2])      # block 0
+    a.add_cached(1, [3, 4])      # block 1
+    a.free_seq(1)                # freed first
+    a.free_seq(0)
+    a.add(2, 4)                  # takes the two stack blocks 2, 3
+    assert a.block_table(2) == [2, 3]
+    a.add(3, 2)                  # stack empty: evicts block 1 (freed first)
+    assert a.block_table(3) == [1]
+    assert a.add_cached(5, [1, 2]) == 2   # block 0 is still cached-free: revived, no new block
+    assert a.block_table(5) == [0]
+    with pytest.raises(AllocatorError) as e:  # [3, 4] was evicted with block 1 and the pool is full
+        a.add_cached(4, [3, 4])
+    assert e.value.code == ERR_OUT_OF_BLOCKS
+    a.check_invariants()
+
+
+def test_prefix_cache_eviction_then_readmission_consistent():
+    bs = 2
+    a = BlockAllocatorModel(4, bs, free_order=[0, 1, 2, 3])
+    a.add_cached(0, [1, 2, 3, 4])  # blocks 0 (prefix [1,2]), 1 (prefix [1,2,3,4])
+    a.free_seq(0)                  # both cached-free: 0 then 1
+    a.add(1, 4)                    # stack blocks 2, 3
+    a.add(2, 2)                    # evicts block 0: the first prefix block
+    # [1,2] is gone but [1,2,3,4] is still cached: no hit (the chain starts with a miss)
+    a.free_seq(2)
+    assert a.add_cached(3, [1, 2, 3, 4]) == 0
+    a.check_invariants()
+
+
+def test_system_prompt_blocks_counted_once():
+    """32 requests with a shared 1024-token system prompt and distinct
+    100-token questions, admitted with prefix caching: the pool holds the
+    prompt once plus each request's own blocks."""
+    bs, n, prompt = 16, 32, 1024
+    a = BlockAllocatorModel(4000, bs)
+    rng = np.random.default_rng(3)
+    sys_prompt = list(rng.integers(0, 32000, size=prompt))
+    reused = [a.add_cached(i, sys_prompt + list(rng.integers(0, 32000, size=100))) for i in range(n)]
+    assert reused == [0] + [prompt] * (n - 1)
+    own = -(-(prompt + 100) // bs) - prompt // bs
+    assert a.stats()["used_blocks"] == prompt // bs + n * own
+    a.check_invariants()
+
+
+def test_random_workload_with_prefix_cache_keeps_invariants():
+    rng = np.random.default_rng(77)
+    bs = 4
+    a = BlockAllocatorModel(60, bs, rng.permutation(60))
+    prefixes = [list(rng.integers(0, 5, size=12)) for _ in range(3)]
+    live, nxt = [], 0
+    for _ in range(2000):
+        op = int(rng.integers(0, 5))
+        try:
+            if op <= 1 or not live:
+                toks = prefixes[int(rng.integers(3))][: int(rng.integers(0, 13))] + \
+                    list(rng.integers(0, 5, size=int(rng.integers(0, 6))))
+                a.add_cached(nxt, toks)
+                live.append(nxt)
+                nxt += 1
+            elif op == 2:
+                a.append_slots([int(x) for x in rng.choice(live, size=int(rng.integers(1, len(live) + 1)))])
+            elif op == 3:
+                a.fork(live[int(rng.integers(len(live)))], nxt)
+                live.append(nxt)
+                nxt += 1
+            else:
+                a.free_seq(live.pop(int(rng.integers(len(live)))))
+        except AllocatorError as e:
+            assert e.code == ERR_OUT_OF_BLOCKS
+        a.check_invariants()
