@@ -15,13 +15,18 @@ Sources (cited by page title and section):
   §4 (admission control, abort).
 * "LLM inference optimisation: principles overview" (LLM 推理优化：技术原理解析总览),
   §2.2 domain three and §3.3 (KV cache cut into fixed-size physical pages of
-  16 tokens, logical-to-physical page table, O(1) append).
+  16 tokens, logical-to-physical page table, O(1) append), §2.3 (chunked
+  prefill of long inputs).
+* the vLLM production-deployment page, §2 (chunked prefill and decode steps
+  batched together; prefix blocks shared between requests) and §5 (prefix
+  caching).
 
 Modules:
 
 * :mod:`oracle.paged_attention` — gather through the block table, two-pass fp64
   softmax attention with GQA head grouping, KV append by slot mapping, block
-  copy, and the split-partition (m, l, o) rescaling identity.
+  copy, the split-partition (m, l, o) rescaling identity, and causal chunked
+  prefill attention over the pool (each new row sees its own prefix).
 * :mod:`oracle.block_allocator` — a pure-Python model of the host block
   allocator (free stack, refcounts, copy-on-write, all-or-nothing errors).
 * :mod:`oracle.fp8` — e4m3 codes (decode, round-to-nearest-even saturating
@@ -29,7 +34,8 @@ Modules:
   per-pool scales ("LLM inference optimisation: principles overview" §5.1:
   an FP8 KV cache).
 
-Parity status: every function here is pinned by ``tests/test_oracle.py`` or
+Parity status: every function here is pinned by ``tests/test_oracle.py``,
+``tests/test_oracle_prefill.py``, ``tests/test_oracle_fp8.py`` or
 ``tests/test_allocator_oracle.py`` against something other than itself
 (brute force, a library special case, closed forms, invariants, the worked
 paging example of the vLLM paging page; for e4m3, torch's float8_e4m3fn and

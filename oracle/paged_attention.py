@@ -181,3 +181,49 @@ def combine_partials(partials):
     num = sum(np.exp(m - M) * o for m, _, o in partials)
     den = sum(np.exp(m - M) * l for m, l, _ in partials)
     return num / den
+
+
+def paged_prefill_attention(q, k_pool, v_pool, block_tables, seq_lens, q_lens, scale,
+                            dtype: str, layout: str = "NHBD") -> np.ndarray:
+    """Causal attention of a prefill chunk over a paged KV pool, float64 ``[T, Hq, D]``.
+
+    Chunked prefill (vLLM production page §2: long prompts are fed in chunks
+    and share a batch with decode steps; optimisation-overview page §2.3:
+    ``enable_chunked_prefill``): sequence ``b`` brings ``n_b = q_lens[b]`` new
+    query rows, packed one sequence after another in ``q`` (``T = Σ n_b``).
+    Their K/V are already in the pool (written by :func:`kv_append`), so the
+    pool holds ``seq_lens[b]`` tokens of which the last ``n_b`` are the
+    chunk's.  Query ``i`` of the chunk sits at position
+    ``p = seq_lens[b] - n_b + i`` and, causally, sees the tokens ``0 … p``
+    (earlier context plus the chunk's rows up to itself).  Each row is then
+    the decode computation of :func:`paged_decode_attention` over its
+    visible prefix: gather through the table, scores scaled by ``scale``,
+    two-pass softmax, weighted sum of V, KV head ``h // G``.
+    """
+    T, Hq, D = q.shape
+    q_lens = [int(x) for x in np.asarray(q_lens).tolist()]
+    if sum(q_lens) != T:
+        raise ValueError("q rows must equal the sum of q_lens")
+    Hkv = k_pool.shape[1] if layout == "NHBD" else k_pool.shape[2]
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    G = Hq // Hkv
+    qf = to_f64(q, dtype)
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    row = 0
+    for b, n in enumerate(q_lens):
+        L = int(seq_lens[b])
+        if n > L:
+            raise ValueError("a chunk cannot be longer than its sequence")
+        if n == 0:
+            continue
+        K = to_f64(gather_sequence(k_pool, block_tables[b], L, layout), dtype)
+        V = to_f64(gather_sequence(v_pool, block_tables[b], L, layout), dtype)
+        for i in range(n):
+            p = L - n + i
+            for h in range(Hq):
+                g = h // G
+                w = attention_weights(qf[row + i, h], K[:p + 1, g, :], scale)
+                out[row + i, h] = w @ V[:p + 1, g, :]
+        row += n
+    return out
