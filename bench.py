@@ -35,6 +35,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "paged decode attention: KV GB/s (fraction of B200 HBM peak), tokens/s per layer"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_SUSTAINED = 1400.0  # TFLOP/s, dense bf16 under the power cap
 STAGED_STEPS = 16  # distinct steps of metadata resident on the device, cycled
 
 # DRAM traffic of one pkv_paged_attention_decode call on the default workload,
@@ -106,6 +107,14 @@ def rank_workload(w, rank: int):
     """Rank r runs its own batch of the same shape (weak scaling): seeds offset by 1000·r."""
     from dataclasses import replace
     return replace(w, seed=w.seed + 1000 * rank) if rank else w
+
+
+def measured_peak_file() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if not os.path.exists(p):
+        return {}
+    with open(p) as f:
+        return json.load(f)
 
 
 def measured_peaks():
@@ -259,6 +268,14 @@ def setup(w, device, horizon):
     return w, cache, lens
 
 
+def decode_launches(max_blocks: int, block_size: int, partition_tokens: int) -> int:
+    """Kernels one pkv_paged_attention_decode call launches: the plan and
+    decode kernels, plus the partition merge when a sequence of the table's
+    capacity can span more than one partition."""
+    pt = partition_tokens or 512
+    return 2 + (1 if max_blocks * block_size > pt else 0)
+
+
 def run_ours(args):
     import torch.distributed as dist
     import paged_kv_cache_406_b200 as P
@@ -335,8 +352,7 @@ def run_ours(args):
                                          out=out, workspace=workspace, partition_tokens=w.partition_tokens)
         if ev is not None:
             ev[1].record()
-        n += 2  # plan + decode (partition merge runs inside the decode kernel)
-        return n
+        return n + decode_launches(cache.max_blocks, bs, w.partition_tokens)
 
     for i in range(args.warmup):
         step(i)
@@ -463,6 +479,312 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+PREFILL_METRIC = "paged prefill attention: TFLOP/s (fraction of B200 dense bf16 peak), prompt tokens/s per layer"
+
+
+def prefill_flops(ctx, n: int, hq: int, d: int) -> int:
+    """Algorithmic FLOPs of causal attention for chunks of n rows behind ctx
+    cached tokens: q·Kᵀ and P·V, 2·d each per visible (row, key) pair."""
+    keys = sum(int(c) * n + n * (n + 1) // 2 for c in ctx)
+    return 4 * d * hq * keys
+
+
+def time_prefill_oracle(units, budget_s: float):
+    """Runs the prefill oracle on (q rows, K, V, table, L, n, scale, dtype)
+    units until the budget is spent; returns (FLOPs, seconds, units done)."""
+    from oracle import paged_attention as pa
+    done, flops, t0 = 0, 0, time.perf_counter()
+    for q, kb, vb, L, n, scale, dtype, fl in units:
+        table = np.arange(kb.shape[0], dtype=np.int32)[None]
+        pa.paged_prefill_attention(q, kb, vb, table, np.array([L]), np.array([n]), scale, dtype)
+        done += 1
+        flops += fl
+        if time.perf_counter() - t0 > budget_s:
+            break
+    return flops, time.perf_counter() - t0, done
+
+
+def run_prefill(args, w0):
+    """A step is one chunked-prefill pass over the batch: the chunk's K/V
+    rows appended through their slots, then causal paged prefill attention
+    of the chunk's query rows over the pool."""
+    import torch.distributed as dist
+    import paged_kv_cache_406_b200 as P
+    from paged_kv_cache_406_b200 import workloads as W
+    from paged_kv_cache_406_b200.cache import PagedKVCache
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = rank_workload(w0, rank)
+    B, hq, hkv, d, bs, n = w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, w.chunk_tokens
+    ctx = W.seq_lens(w)
+    L = ctx + n
+    nb = W.pool_blocks(w, L)
+    shape = (nb, hkv, bs, d)
+    maxb = -(-int(L.max()) // bs)
+    cache = PagedKVCache(nb, hkv, d, bs, w.torch_dtype, maxb, device=dev, free_order=W.free_order(nb, w.seed),
+                         k_pool=W.pool_values(shape, w, 0, device=dev), v_pool=W.pool_values(shape, w, 1, device=dev))
+    ids = list(range(B))
+    for b in ids:
+        cache.add(b, int(ctx[b]))
+    # the chunk's slots (host allocator), row r of sequence b at q row b·n + r
+    slots = np.stack([cache.alloc.append_slots(ids)[0].copy() for _ in range(n)], axis=1).reshape(-1)
+    tables, lens = cache.alloc.block_tables(ids, maxb)
+    slot_d = torch.from_numpy(slots.astype(np.int32)).to(dev)
+    tables_d, lens_d = torch.from_numpy(tables.copy()).to(dev), torch.from_numpy(lens.copy()).to(dev)
+    q_start = torch.arange(0, B * n + 1, n, dtype=torch.int32, device=dev)
+    T = B * n
+    q = W.normal((T, hq, d), w.torch_dtype, W.step_seed(w, 0, 0), device=dev)
+    kn = W.normal((T, hkv, d), w.torch_dtype, W.step_seed(w, 0, 1), device=dev)
+    vn = W.normal((T, hkv, d), w.torch_dtype, W.step_seed(w, 0, 2), device=dev)
+    out = torch.empty((T, hq, d), dtype=torch.float32, device=dev)
+
+    def step(ev=None):
+        P.pkv_kv_append(kn, vn, slot_d, cache.k_pool, cache.v_pool)
+        if ev is not None:
+            ev[0].record()
+        P.pkv_paged_attention_prefill(q, cache.k_pool, cache.v_pool, tables_d, lens_d, q_start, n, w.scale, out=out)
+        if ev is not None:
+            ev[1].record()
+        return 2
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert P.pkv_device_status(clear=True) == 0
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local, not args.no_clocks)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record()
+    launches = 0
+    for i in range(K):
+        launches += step(evs[i])
+    end.record()
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    status = P.pkv_device_status(clear=True)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+    elapsed_ms = start.elapsed_time(end)
+    attn_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    flops = prefill_flops(ctx, n, hq, d)
+    elapsed_all, flops_all, tokens_all = combine_ranks(elapsed_ms, float(flops) * K, float(T * K), dev)
+    value = flops_all / (elapsed_all * 1e-3) / 1e12
+    peaks = measured_peak_file()
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_BF16_SUSTAINED))
+    peak_kind = "measured bf16_tflops_sustained" if "bf16_tflops_sustained" in peaks else "fallback sustained"
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+
+    # ---- end to end: host q / K / V rows and metadata in, out back to host ----
+    e2e = None
+    if args.e2e_steps > 0:
+        E = args.e2e_steps
+        hq_in, hk_in, hv_in = (t.cpu().pin_memory() for t in (q, kn, vn))
+        meta_h = torch.from_numpy(np.concatenate([slots.astype(np.int32), tables.reshape(-1), lens,
+                                                  np.arange(0, T + 1, n, dtype=np.int32)])).pin_memory()
+        meta_d = torch.empty_like(meta_h, device=dev)
+        out_h = torch.empty((T, hq, d), dtype=torch.float32, pin_memory=True)
+        qd, kd, vd = torch.empty_like(q), torch.empty_like(kn), torch.empty_like(vn)
+        ns, nt = slots.size, tables.size
+
+        def e2e_step():
+            meta_d.copy_(meta_h, non_blocking=True)
+            qd.copy_(hq_in, non_blocking=True)
+            kd.copy_(hk_in, non_blocking=True)
+            vd.copy_(hv_in, non_blocking=True)
+            P.pkv_kv_append(kd, vd, meta_d[:ns], cache.k_pool, cache.v_pool)
+            P.pkv_paged_attention_prefill(qd, cache.k_pool, cache.v_pool, meta_d[ns:ns + nt].view(B, maxb),
+                                          meta_d[ns + nt:ns + nt + B], meta_d[ns + nt + B:], n, w.scale, out=out)
+            out_h.copy_(out, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(E):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        e2e_all, e2e_flops, _ = combine_ranks(e2e_ms, float(flops) * E, float(T * E), dev)
+        e2e = {"value": round(e2e_flops / (e2e_all * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int((q.numel() + kn.numel() + vn.numel()) * q.element_size() + meta_h.numel() * 4),
+               "d2h_bytes_per_step": int(out.numel() * 4), "ms_per_step": round(e2e_all / E, 4),
+               "tokens_per_s_per_layer": round(ws * T * E / (e2e_all * 1e-3), 1),
+               "includes": "pinned H2D of the chunk's q/K/V rows and metadata, append, prefill, D2H of out"}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        rng = np.random.default_rng(7)
+        G = w.group
+        units = []
+        for b in rng.permutation(B)[:4]:
+            g = int(rng.integers(hkv))
+            nblk = -(-int(L[b]) // bs)
+            idx = torch.as_tensor(tables[b, :nblk], device=dev, dtype=torch.long)
+            kb, vb = _raw(cache.k_pool[idx, g:g + 1]), _raw(cache.v_pool[idx, g:g + 1])
+            rows = 4  # the chunk's last rows: the most keys per row
+            qb = _raw(q[b * n + n - rows:b * n + n, g * G:(g + 1) * G])
+            fl = 4 * d * G * sum(int(L[b]) - rows + 1 + r for r in range(rows))
+            units.append((qb, kb, vb, int(L[b]), rows, w.scale, w.dtype, fl))
+        cycle = (units[i % len(units)] for i in range(10 ** 9))
+        fl, secs, done = time_prefill_oracle(cycle, args.cpu_seconds)
+        cpu = {"value": round(fl / secs / 1e12, 6), "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+               "host_cpus": os.cpu_count(),
+               "sample": f"{done} units of 4 query rows x {G} heads (one KV head, full causal context) from the same "
+                         f"batch, 4 distinct, cycled; fp64 numpy oracle, {secs:.1f} s"}
+
+    if rank == 0:
+        res = {
+            "metric": PREFILL_METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": ws, "steps": K,
+            "warmup": args.warmup, "ms_per_step": round(elapsed_all / K, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "tokens_per_s_per_layer": round(tokens_all / (elapsed_all * 1e-3), 1),
+            "config": {"workload": w.name, "num_seqs": B, "num_q_heads": hq, "num_kv_heads": hkv, "head_dim": d,
+                       "block_size": bs, "chunk_tokens": n,
+                       "cached_context": "U[0,3584]" if int(ctx.max()) else "0 (whole prompts)",
+                       "flops_per_step": flops,
+                       "l2": "inputs larger than L2: %.0f MB of K/V + %.0f MB of q and out per step, no flush"
+                             % (int(L.sum()) * hkv * d * 4 / 1e6, T * hq * d * 6 / 1e6),
+                       "parallelism": f"replicas x{ws} (independent batches per GPU)"},
+            "roofline": {"kernel": "pkv_paged_attention_prefill (prefill_tc_kernel)", "bound": "tensor",
+                         "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(achieved / peak, 4), "peak_source": peak_kind,
+                         "burst_peak": peaks.get("bf16_tflops"),
+                         "traffic": None, "algorithmic_flops_per_launch": flops,
+                         "tensor_flops_issued_per_launch": "1.5x algorithmic (P·V runs on P hi and P lo) plus the "
+                                                          "masked part of diagonal chunks",
+                         "avg_launch_ms": round(attn_ms, 5), "kernel_source_sha": kernel_source_sha()},
+            "gpu_launches": launches, "clocks": clk, "cpu_baseline": cpu, "e2e": e2e,
+        }
+        print(json.dumps(res), flush=True)
+    if ws > 1:
+        dist.destroy_process_group()
+
+
+def run_adaptive(args, w):
+    """Adaptive block size (optimisation-overview page §3.3) against one
+    fixed 16-token pool on the same batch: a step appends one token per
+    sequence and runs paged decode attention; the adaptive arm does that
+    once per block-size class (32 / 16 / 8)."""
+    import paged_kv_cache_406_b200 as P
+    from paged_kv_cache_406_b200 import workloads as W
+    from paged_kv_cache_406_b200.cache import AdaptivePagedKVCache, PagedKVCache, block_size_for
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = rank_workload(w, rank)
+    B, hq, hkv, d = w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim
+    lens0 = W.seq_lens(w)
+    horizon = STAGED_STEPS + 8
+    maxtok = int(lens0.max()) + horizon
+    per_class = {}
+    for L in lens0:
+        bs = block_size_for(int(L))
+        per_class[bs] = per_class.get(bs, 0) + -(-(int(L) + horizon) // bs)
+    per_class = {bs: int(np.ceil(1.2 * nb)) for bs, nb in per_class.items()}
+    ad = AdaptivePagedKVCache(per_class, hkv, d, w.torch_dtype, maxtok, device=dev, seed=w.seed)
+    nb16 = int(np.ceil(1.2 * sum(-(-(int(L) + horizon) // 16) for L in lens0)))
+    fixed = PagedKVCache(nb16, hkv, d, 16, w.torch_dtype, -(-maxtok // 16), device=dev,
+                         free_order=W.free_order(nb16, w.seed))
+    for k, c in enumerate(list(ad.caches.values()) + [fixed]):
+        c.k_pool.copy_(W.normal(c.k_pool.shape, w.torch_dtype, W.pool_seed(w, 0) + 17 * k, device=dev))
+        c.v_pool.copy_(W.normal(c.v_pool.shape, w.torch_dtype, W.pool_seed(w, 1) + 17 * k, device=dev))
+    for i, L in enumerate(lens0):
+        ad.add(i, int(L))
+        fixed.add(i, int(L))
+    ids = ad.order()
+    e = torch.tensor([], dtype=w.torch_dtype).element_size()
+    q = W.normal((B, hq, d), w.torch_dtype, W.step_seed(w, 0, 0), device=dev)
+    kn = W.normal((B, hkv, d), w.torch_dtype, W.step_seed(w, 0, 1), device=dev)
+    vn = W.normal((B, hkv, d), w.torch_dtype, W.step_seed(w, 0, 2), device=dev)
+
+    def stage(cache, members):
+        out = []
+        for _ in range(STAGED_STEPS):
+            slots, _ = cache.alloc.append_slots(members)
+            tables, lens = cache.alloc.block_tables(members, cache.max_blocks)
+            out.append((torch.from_numpy(slots.copy()).to(dev), torch.from_numpy(tables.copy()).to(dev),
+                        torch.from_numpy(lens.copy()).to(dev), lens.copy()))
+        wsb = P.pkv_decode_workspace_size(len(members), hq, hkv, d, cache.max_blocks, cache.block_size, 0)
+        return out, torch.empty(wsb, dtype=torch.uint8, device=dev)
+
+    arms = {"adaptive": [], "fixed_bs16": []}
+    a = 0
+    for bs in ad.CLASSES:
+        members = [i for i in ids if ad.cls[i] == bs]
+        if members:
+            st, wsp = stage(ad.caches[bs], members)
+            arms["adaptive"].append((ad.caches[bs], st, wsp, slice(a, a + len(members))))
+            a += len(members)
+    st, wsp = stage(fixed, ids)
+    arms["fixed_bs16"].append((fixed, st, wsp, slice(0, B)))
+    out = torch.empty((B, hq, d), dtype=torch.float32, device=dev)
+
+    def step(arm, i):
+        for cache, st, wsp, sl in arms[arm]:
+            slots, tables, lens, _ = st[i % STAGED_STEPS]
+            P.pkv_kv_append(kn[sl], vn[sl], slots, cache.k_pool, cache.v_pool)
+            P.pkv_paged_attention_decode(q[sl], cache.k_pool, cache.v_pool, tables, lens, w.scale, out=out[sl],
+                                         workspace=wsp)
+        return sum(1 + decode_launches(c.max_blocks, c.block_size, 0) for c, _, _, _ in arms[arm])
+
+    res_arms = {}
+    clocks = ClockSampler(local, not args.no_clocks)
+    launches = 0
+    for arm in arms:
+        for i in range(args.warmup):
+            step(arm, i)
+        torch.cuda.synchronize()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for i in range(args.steps):
+            launches += step(arm, args.warmup + i)
+        s1.record()
+        torch.cuda.synchronize()
+        ms = s0.elapsed_time(s1)
+        nbytes = sum(int(st[(args.warmup + i) % STAGED_STEPS][3].astype(np.int64).sum()) * hkv * d * 2 * e
+                     for i in range(args.steps) for _, st, _, _ in arms[arm])
+        res_arms[arm] = {"kv_gb_s": round(nbytes / (ms * 1e-3) / 1e9, 1), "ms_per_step": round(ms / args.steps, 5),
+                         "tokens_per_s_per_layer": round(B * args.steps / (ms * 1e-3), 1),
+                         "calls_per_step": len(arms[arm]),
+                         "pool_blocks": {str(c.block_size): c.num_blocks for c, _, _, _ in arms[arm]},
+                         "waste_tokens": sum(c.stats()["waste_tokens"] for c, _, _, _ in arms[arm])}
+    clk = clocks.stop()
+    assert P.pkv_device_status(clear=True) == 0
+    peak, peak_kind = measured_peaks()
+    r = res_arms["adaptive"]
+    if rank == 0:
+        res = {"metric": METRIC, "value": r["kv_gb_s"], "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+               "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True,
+               "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+               "tokens_per_s_per_layer": r["tokens_per_s_per_layer"], "hbm_fraction": round(r["kv_gb_s"] / peak, 4),
+               "config": {"workload": w.name, "num_seqs": B, "num_q_heads": hq, "num_kv_heads": hkv, "head_dim": d,
+                          "block_size": "adaptive: 32 below 1024 tokens, 16 below 8192, 8 above",
+                          "seq_lens": "80% U[128,1023], 19% U[1024,8191], 1 U[8192,16384]",
+                          "class_sizes": {str(bs): sum(1 for i in ids if ad.cls[i] == bs) for bs in ad.CLASSES},
+                          "l2": "no flush; K/V per step %.0f MB" % (sum(int(L) for L in lens0) * hkv * d * 2 * e / 1e6),
+                          "parallelism": f"replicas x{ws}"},
+               "arms": res_arms, "peak": peak, "peak_source": f"{peak_kind} hbm_gbs",
+               "gpu_launches": launches, "clocks": clk, "cpu_baseline": None, "e2e": None}
+        print(json.dumps(res), flush=True)
+
+
 def run_reference(args):
     """The reference arm: the fp64 CPU oracle, on this arm's workload, each
     step a bounded sample of it (rank 0 only)."""
@@ -471,6 +793,8 @@ def run_reference(args):
         return
     from paged_kv_cache_406_b200 import workloads as W
     w = W.WORKLOADS[args.workload]
+    if w.chunk_tokens:
+        return run_reference_prefill(args, w, ws)
     lens = W.seq_lens(w)
     rng = np.random.default_rng(w.seed)
     G, e = w.group, torch.tensor([], dtype=w.torch_dtype).element_size()
@@ -510,6 +834,51 @@ def run_reference(args):
     print(json.dumps(res), flush=True)
 
 
+def run_reference_prefill(args, w, ws):
+    """Reference arm for a prefill workload: each step, the fp64 oracle on the
+    last 4 chunk rows x G query heads of one (sequence, KV head) over its full
+    causal context."""
+    from paged_kv_cache_406_b200 import workloads as W
+    L = W.seq_lens(w) + w.chunk_tokens
+    rng = np.random.default_rng(w.seed)
+    G, rows = w.group, 4
+    order = [(int(b), int(rng.integers(w.num_kv_heads))) for b in rng.permutation(w.num_seqs)]
+    cache = {}
+
+    def unit(i):
+        b, g = order[i % len(order)]
+        if (b, g) not in cache:
+            nblk = -(-int(L[b]) // w.block_size)
+            shp = (nblk, 1, w.block_size, w.head_dim)
+            kb = _raw(W.normal(shp, w.torch_dtype, W.pool_seed(w, 0) + 7919 * b + g))
+            vb = _raw(W.normal(shp, w.torch_dtype, W.pool_seed(w, 1) + 7919 * b + g))
+            qb = _raw(W.normal((rows, G, w.head_dim), w.torch_dtype, W.step_seed(w, 0, 0) + b))
+            fl = 4 * w.head_dim * G * sum(int(L[b]) - rows + 1 + r for r in range(rows))
+            cache[(b, g)] = (qb, kb, vb, int(L[b]), rows, w.scale, w.dtype, fl)
+        return cache[(b, g)]
+
+    K, Wm = args.steps, args.warmup
+    for i in range(Wm):
+        time_prefill_oracle([unit(i)], 1e9)
+    total_fl, total_s = 0, 0.0
+    for i in range(K):
+        fl, s, _ = time_prefill_oracle([unit(Wm + i)], 1e9)
+        total_fl += fl
+        total_s += s
+    value = total_fl / total_s / 1e12
+    res = {"impl": "reference", "metric": PREFILL_METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+           "n_gpus": ws, "steps": K, "warmup": Wm, "ms_per_step": round(total_s / K * 1e3, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": w.name, "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads,
+                      "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
+                      "chunk_tokens": w.chunk_tokens},
+           "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "kind": "oracle", "cores": oracle_threads(),
+                            "sample": f"{rows} chunk rows x {G} heads of one (sequence, KV head) per step, "
+                                      "full causal context, fp64 numpy oracle"},
+           "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -517,7 +886,14 @@ def main():
     else:
         if not torch.cuda.is_available():
             raise SystemExit("bench.py needs a CUDA GPU (B200); use --impl reference for the CPU oracle")
-        run_ours(args)
+        from paged_kv_cache_406_b200 import workloads as W
+        w = W.WORKLOADS[args.workload]
+        if w.chunk_tokens:
+            run_prefill(args, w)
+        elif w.name == "adaptive_mix":
+            run_adaptive(args, w)
+        else:
+            run_ours(args)
 
 
 if __name__ == "__main__":

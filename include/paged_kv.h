@@ -241,6 +241,39 @@ int pkv_paged_attention_decode(const void* q, const void* k_pool, const void* v_
                                int32_t partition_tokens, void* workspace, size_t workspace_bytes,
                                float* out, void* stream);
 
+/* Paged prefill attention (chunked prefill: vLLM production page §2;
+ * optimisation-overview page §2.3): sequence b brings
+ * n_b = q_start[b+1] - q_start[b] new query rows, stored at rows
+ * q_start[b] .. q_start[b+1]-1 of q, whose K/V are already in the pool
+ * (written by pkv_kv_append), so the pool holds seq_lens[b] tokens of which
+ * the last n_b are the chunk's.  Row i of the chunk sits at position
+ * p = seq_lens[b] - n_b + i and attends causally to tokens 0 .. p:
+ *     out[q_start[b]+i][h][:] = sum_{t<=p} softmax_t(scale * q·K_b[t][g]) * V_b[t][g][:]
+ * with g = h / G, G = num_q_heads / num_kv_heads, tokens reached through the
+ * block table as in pkv_paged_attention_decode.  A one-row chunk is a decode
+ * query.
+ *
+ * q: dtype[num_q_tokens][num_q_heads][128]; q_start: int32[num_seqs + 1],
+ * non-decreasing, q_start[0] >= 0, q_start[num_seqs] <= num_q_tokens;
+ * max_q_len: an upper bound of every n_b (sets the launch grid);
+ * block_tables / seq_lens as for decode; out: float32[num_q_tokens][num_q_heads][128]
+ * (rows outside every chunk are not written).  dtype PKV_BF16 or PKV_F16,
+ * head_dim 128, G in {1, 2, 4, 8}, block_size 8, 16 or 32; others return
+ * PKV_ERR_UNSUPPORTED.  q, pools and out 16-byte aligned.
+ * Computed on the tcgen05 tensor cores with fp32 accumulation; P enters the
+ * P·V product as two 16-bit halves (hi + lo), so the result stays within
+ * about 1e-5 of the exact softmax.  A sequence whose chunk is longer than
+ * seq_lens[b] or max_q_len is skipped and recorded as PKV_ERR_INVALID_ARG;
+ * table entries outside [0, num_blocks) as PKV_ERR_BAD_BLOCK (block 0 read
+ * instead), both in the device status. */
+int pkv_paged_attention_prefill(const void* q, const void* k_pool, const void* v_pool,
+                                const int32_t* block_tables, const int32_t* seq_lens,
+                                const int32_t* q_start, int32_t num_seqs, int32_t num_q_tokens,
+                                int32_t max_q_len, int32_t num_q_heads, int32_t num_kv_heads,
+                                int32_t head_dim, int32_t num_blocks, int32_t max_blocks_per_seq,
+                                int32_t block_size, float scale, int32_t dtype, float* out,
+                                void* stream);
+
 /* PagedAttention decode exactly as pkv_paged_attention_decode, for callers
  * that cannot allocate device memory when they decode: serving runtimes that
  * have reserved nearly all of HBM for their KV pool up front, framework

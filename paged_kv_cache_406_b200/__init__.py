@@ -1,5 +1,5 @@
-"""paged_kv_cache_406_b200 — a paged KV cache and PagedAttention decode for
-NVIDIA B200 (sm_100a).
+"""paged_kv_cache_406_b200 — a paged KV cache, PagedAttention decode and paged
+prefill attention for NVIDIA B200 (sm_100a).
 
 The work is done by ``libpagedkv.so`` (hand-written CUDA kernels plus a C++
 host block allocator, C ABI in ``include/paged_kv.h``); this package is its
@@ -8,7 +8,8 @@ thin Python binding.  Build the library with
 """
 from .binding import (Allocator, PagedKVError, pkv_copy_blocks, pkv_decode_workspace_size,  # noqa: F401
                       pkv_device_status, pkv_kv_append, pkv_kv_append_fp8, pkv_paged_attention_decode,
-                      pkv_paged_attention_decode_fp8, pkv_paged_attention_decode_static)
+                      pkv_paged_attention_decode_fp8, pkv_paged_attention_decode_static,
+                      pkv_paged_attention_prefill)
 from ._native import LIB_PATH, lib  # noqa: F401
 
 __version__ = "1.0.0"

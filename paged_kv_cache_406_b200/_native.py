@@ -63,6 +63,8 @@ SIGNATURES = {
                                          _vp]),
     "pkv_paged_attention_decode_fp8": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                                                       _i32, _f32, _f32, _f32, _i32, _vp, _sz, _vp, _vp]),
+    "pkv_paged_attention_prefill": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
+                                                   _i32, _i32, _i32, _f32, _i32, _vp, _vp]),
 }
 
 

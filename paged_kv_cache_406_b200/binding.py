@@ -122,6 +122,38 @@ def pkv_paged_attention_decode(q: torch.Tensor, k_pool: torch.Tensor, v_pool: to
     return out
 
 
+def pkv_paged_attention_prefill(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                                block_tables: torch.Tensor, seq_lens: torch.Tensor, q_start: torch.Tensor,
+                                max_q_len: int, scale: float, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Causal paged prefill attention; returns ``out`` (float32
+    ``[num_q_tokens, num_q_heads, head_dim]``).  Sequence ``b`` owns q rows
+    ``q_start[b] .. q_start[b+1]-1`` (int32 ``[num_seqs + 1]`` on the device);
+    ``max_q_len`` bounds every chunk length."""
+    nb, hkv, bs, d = _pool_dims(_cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"))
+    _cuda(q, "q", k_pool.dtype)
+    if q.dim() != 3 or q.shape[2] != d:
+        raise ValueError(f"q must be [num_q_tokens, num_q_heads, {d}]")
+    T, hq, _ = q.shape
+    _cuda(block_tables, "block_tables", torch.int32)
+    _cuda(seq_lens, "seq_lens", torch.int32)
+    _cuda(q_start, "q_start", torch.int32)
+    B = seq_lens.numel()
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or q_start.numel() != B + 1:
+        raise ValueError("block_tables must be [num_seqs, max_blocks_per_seq] and q_start [num_seqs + 1]")
+    maxb = block_tables.shape[1]
+    if out is None:
+        out = torch.empty((T, hq, d), dtype=torch.float32, device=q.device)
+    else:
+        _cuda(out, "out", torch.float32)
+        if tuple(out.shape) != (T, hq, d):
+            raise ValueError("out has the wrong shape")
+    check(lib().pkv_paged_attention_prefill(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
+                                            block_tables.data_ptr(), seq_lens.data_ptr(), q_start.data_ptr(), B, T,
+                                            int(max_q_len), hq, hkv, d, nb, maxb, bs, float(scale),
+                                            _dtype_code(k_pool), out.data_ptr(), _stream()))
+    return out
+
+
 def pkv_paged_attention_decode_static(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
                                       block_tables: torch.Tensor, seq_lens: torch.Tensor, scale: float,
                                       out: Optional[torch.Tensor] = None, partition_tokens: int = 0) -> torch.Tensor:

@@ -120,19 +120,21 @@ class PagedKVCache:
 
     # -- the decode step -----------------------------------------------------
     def decode_step(self, seq_ids: Sequence[int], q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
-                    scale: float, partition_tokens: int = 0) -> torch.Tensor:
+                    scale: float, partition_tokens: int = 0, out: Optional[torch.Tensor] = None) -> torch.Tensor:
         """Append one token per sequence and attend over every cached token.
 
         ``q`` [n, Hq, D], ``k_new``/``v_new`` [n, Hkv, D] in the pool dtype, on
         the device or in (pinned) host memory.  Returns float32 [n, Hq, D] on
-        the device (valid until the next step)."""
+        the device: ``out`` if given (a contiguous device tensor), else a
+        buffer of this cache valid until the next step."""
         n = len(seq_ids)
         ncow, _ = self.prepare_step(seq_ids)
         slots, lens, cow, tables = self.upload_step(n)
         q, k_new, v_new = (t.to(self.device, non_blocking=True) for t in (q, k_new, v_new))
         if ncow:
             B.pkv_copy_blocks(self.k_pool, self.v_pool, cow[:2 * ncow].view(ncow, 2))
-        ws, out = self._buffers(n, q.shape[1], partition_tokens)
+        ws, own = self._buffers(n, q.shape[1], partition_tokens)
+        out = own if out is None else out
         if self.fp8:
             B.pkv_kv_append_fp8(k_new, v_new, slots, self.k_pool, self.v_pool, self.k_scale, self.v_scale)
             return B.pkv_paged_attention_decode_fp8(q, self.k_pool, self.v_pool, tables, lens, scale, self.k_scale,
@@ -144,3 +146,69 @@ class PagedKVCache:
 
     def stats(self) -> dict:
         return self.alloc.stats()
+
+
+def block_size_for(seq_len: int) -> int:
+    """The optimisation-overview page's block-size classes (§3.3): 32 below
+    1024 tokens, 16 from 1024 to below 8192, 8 from 8192 on."""
+    if seq_len < 1024:
+        return 32
+    if seq_len < 8192:
+        return 16
+    return 8
+
+
+class AdaptivePagedKVCache:
+    """Adaptive block size (optimisation-overview page §3.3): one paged pool
+    per block-size class (32, 16, 8 tokens); a sequence joins the class of
+    its length at admission and keeps it for life (the page leaves migration
+    open; none is done).  A decode step runs the paged path once per class.
+
+    ``seq_ids`` passed to :meth:`decode_step` must be grouped by class in the
+    order 32, 16, 8 (:meth:`order` returns live ids that way), so that each
+    class works on a contiguous slice of q, the new rows and the output."""
+
+    CLASSES = (32, 16, 8)
+
+    def __init__(self, blocks_per_class: dict, num_kv_heads: int, head_dim: int, dtype: torch.dtype,
+                 max_tokens: int, device="cuda", seed: int = 0):
+        self.caches = {}
+        for bs in self.CLASSES:
+            nb = int(blocks_per_class.get(bs, 0))
+            if nb <= 0:
+                continue
+            order = np.random.Generator(np.random.PCG64(seed + bs)).permutation(nb).astype(np.int32)
+            self.caches[bs] = PagedKVCache(nb, num_kv_heads, head_dim, bs, dtype, -(-max_tokens // bs),
+                                           device=device, free_order=order)
+        self.cls: dict = {}
+
+    def add(self, seq_id: int, n_tokens: int) -> int:
+        bs = block_size_for(n_tokens)
+        if bs not in self.caches:
+            raise ValueError(f"no pool for block size {bs}")
+        self.caches[bs].add(seq_id, n_tokens)
+        self.cls[seq_id] = bs
+        return bs
+
+    def free(self, seq_id: int) -> None:
+        self.caches[self.cls.pop(seq_id)].free(seq_id)
+
+    def order(self) -> list:
+        return [s for bs in self.CLASSES for s in self.cls if self.cls[s] == bs]
+
+    def decode_step(self, seq_ids: Sequence[int], q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                    scale: float, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        n = len(seq_ids)
+        ranks = [self.CLASSES.index(self.cls[s]) for s in seq_ids]
+        if any(a > b for a, b in zip(ranks, ranks[1:])):
+            raise ValueError("seq_ids must be grouped by block-size class (32, 16, 8)")
+        if out is None:
+            out = torch.empty((n, q.shape[1], q.shape[2]), dtype=torch.float32, device=next(iter(self.caches.values())).device)
+        a = 0
+        for bs in self.CLASSES:
+            m = sum(1 for r in ranks if self.CLASSES[r] == bs)
+            if m:
+                self.caches[bs].decode_step(seq_ids[a:a + m], q[a:a + m], k_new[a:a + m], v_new[a:a + m], scale,
+                                            out=out[a:a + m])
+            a += m
+        return out

@@ -13,6 +13,7 @@
 #include "decode.cuh"
 #include "decode_mma.cuh"
 #include "device_common.cuh"
+#include "prefill.cuh"
 #include "pkv_internal.h"
 
 namespace pkv {
@@ -764,4 +765,140 @@ extern "C" int pkv_paged_attention_decode_static(const void* q, const void* k_po
   return pkv_paged_attention_decode(q, k_pool, v_pool, block_tables, seq_lens, num_seqs, num_q_heads, num_kv_heads,
                                     head_dim, num_blocks, max_blocks_per_seq, block_size, scale, dtype,
                                     partition_tokens, ws, kStaticWorkspaceBytes, out, stream);
+}
+
+// =============================================================================
+// Paged prefill attention (tcgen05 tensor cores)
+// =============================================================================
+namespace {
+
+// q [num_q_tokens, Hq, 128] of 16-bit elements viewed as 4-D: x = 64 elements,
+// y = head_dim half (128 bytes apart), z = query head, w = token.  A box of
+// 64 x 1 x G x (128 / G) lands as 128 rows (token-major, then head) of 128
+// bytes, 128-byte swizzled: the A operand of S = Q · Kᵀ.
+int make_prefill_q_map(CUtensorMap* m, const void* q, int dtype, int32_t num_q_tokens, int32_t num_q_heads,
+                       int32_t group) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[4] = {64, 2, static_cast<cuuint64_t>(num_q_heads), static_cast<cuuint64_t>(num_q_tokens)};
+  const cuuint64_t strides[3] = {128, 256, static_cast<cuuint64_t>(num_q_heads) * 256};
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(group), static_cast<cuuint32_t>(128 / group)};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+                   const_cast<void*>(q), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled (prefill q) failed (%d)", static_cast<int>(r));
+  return PKV_OK;
+}
+
+// Pool of 16-bit elements, head_dim 128, viewed as in make_pool_map but with
+// a box of one head_dim half: 64 x block_size x 1, so the halves of a chunk's
+// blocks land in two separate 128-row slabs.
+int make_prefill_pool_map(CUtensorMap* m, const void* pool, int dtype, int64_t rows, int32_t block_size) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), 2};
+  const cuuint64_t strides[2] = {256, 128};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(block_size), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                   const_cast<void*>(pool), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled (prefill pool) failed (%d)", static_cast<int>(r));
+  return PKV_OK;
+}
+
+template <typename T, int G>
+int launch_prefill(const pkv::PrefillParams& p, const void* q, const void* k_pool, const void* v_pool, int dtype,
+                   cudaStream_t stream) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  auto kern = pkv::prefill_tc_kernel<T, G>;
+  static std::atomic<bool> configured[kMaxDevices];
+  if (dev >= kMaxDevices || !configured[dev].load(std::memory_order_relaxed)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(pkv::pf::kSmemBytes));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill)");
+    if (dev < kMaxDevices) configured[dev].store(true, std::memory_order_relaxed);
+  }
+  CUtensorMap mq, mk, mv;
+  int rc = make_prefill_q_map(&mq, q, dtype, p.num_q_tokens, p.num_q_heads, G);
+  if (rc) return rc;
+  const int64_t rows = int64_t(p.num_blocks) * p.num_kv_heads * p.block_size;
+  rc = make_prefill_pool_map(&mk, k_pool, dtype, rows, p.block_size);
+  if (rc) return rc;
+  rc = make_prefill_pool_map(&mv, v_pool, dtype, rows, p.block_size);
+  if (rc) return rc;
+  const int64_t grid = int64_t(p.n_tiles) * p.num_seqs * p.num_kv_heads;
+  kern<<<static_cast<unsigned>(grid), pkv::pf::kThreads, pkv::pf::kSmemBytes, stream>>>(p, mq, mk, mv);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
+  return pkv::ok();
+}
+
+template <typename T>
+int dispatch_prefill(int32_t group, const pkv::PrefillParams& p, const void* q, const void* k_pool, const void* v_pool,
+                     int dtype, cudaStream_t s) {
+  if (group == 1) return launch_prefill<T, 1>(p, q, k_pool, v_pool, dtype, s);
+  if (group == 2) return launch_prefill<T, 2>(p, q, k_pool, v_pool, dtype, s);
+  if (group == 4) return launch_prefill<T, 4>(p, q, k_pool, v_pool, dtype, s);
+  return launch_prefill<T, 8>(p, q, k_pool, v_pool, dtype, s);
+}
+
+}  // namespace
+
+extern "C" int pkv_paged_attention_prefill(const void* q, const void* k_pool, const void* v_pool,
+                                           const int32_t* block_tables, const int32_t* seq_lens,
+                                           const int32_t* q_start, int32_t num_seqs, int32_t num_q_tokens,
+                                           int32_t max_q_len, int32_t num_q_heads, int32_t num_kv_heads,
+                                           int32_t head_dim, int32_t num_blocks, int32_t max_blocks_per_seq,
+                                           int32_t block_size, float scale, int32_t dtype, float* out,
+                                           void* stream) {
+  const char* fn = "pkv_paged_attention_prefill";
+  if (dtype != PKV_BF16 && dtype != PKV_F16)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: dtype %d not supported (bf16 or f16)", fn, dtype);
+  int rc = check_common(num_kv_heads, head_dim, block_size, dtype, fn);
+  if (rc) return rc;
+  if (head_dim != 128) return fail(PKV_ERR_UNSUPPORTED, "%s: head_dim %d not supported (128)", fn, head_dim);
+  if (num_seqs < 0 || num_q_tokens < 0 || max_q_len < 0 || num_q_heads <= 0 || num_blocks <= 0 ||
+      max_blocks_per_seq < 0)
+    return fail(PKV_ERR_INVALID_ARG, "%s: bad sizes", fn);
+  if (num_q_heads % num_kv_heads != 0)
+    return fail(PKV_ERR_INVALID_ARG, "%s: num_q_heads %d not a multiple of num_kv_heads %d", fn, num_q_heads,
+                num_kv_heads);
+  const int32_t group = num_q_heads / num_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: group size %d not supported (1, 2, 4 or 8)", fn, group);
+  if (!std::isfinite(scale)) return fail(PKV_ERR_INVALID_ARG, "%s: scale is not finite", fn);
+  if (num_seqs == 0 || num_q_tokens == 0 || max_q_len == 0) return pkv::ok();
+  if (!q || !k_pool || !v_pool || !block_tables || !seq_lens || !q_start || !out)
+    return fail(PKV_ERR_INVALID_ARG, "%s: NULL pointer", fn);
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out))
+    return fail(PKV_ERR_INVALID_ARG, "%s: q, pools and out must be 16-byte aligned", fn);
+  if (int64_t(num_blocks) * num_kv_heads * block_size >= (int64_t(1) << 31))
+    return fail(PKV_ERR_INVALID_ARG, "%s: pool rows exceed 2^31", fn);
+  if (int64_t(max_blocks_per_seq) * block_size >= (int64_t(1) << 31))
+    return fail(PKV_ERR_INVALID_ARG, "%s: max_blocks_per_seq * block_size exceeds 2^31", fn);
+  const int32_t qt = 128 / group;
+  const int64_t n_tiles = (int64_t(max_q_len) + qt - 1) / qt;
+  const int64_t grid = n_tiles * num_seqs * num_kv_heads;
+  if (grid >= (int64_t(1) << 31)) return fail(PKV_ERR_INVALID_ARG, "%s: too many tiles (%lld)", fn, (long long)grid);
+  pkv::PrefillParams p{};
+  p.block_tables = block_tables;
+  p.seq_lens = seq_lens;
+  p.q_start = q_start;
+  p.out = out;
+  p.num_seqs = num_seqs;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.num_blocks = num_blocks;
+  p.max_blocks = max_blocks_per_seq;
+  p.block_size = block_size;
+  p.num_q_tokens = num_q_tokens;
+  p.max_q_len = max_q_len;
+  p.n_tiles = static_cast<int32_t>(n_tiles);
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == PKV_BF16) return dispatch_prefill<__nv_bfloat16>(group, p, q, k_pool, v_pool, dtype, s);
+  return dispatch_prefill<__half>(group, p, q, k_pool, v_pool, dtype, s);
 }

@@ -1,0 +1,415 @@
+// Paged prefill attention on the fifth-generation tensor cores (tcgen05).
+//
+// What it computes (vLLM production page §2 and optimisation-overview page
+// §2.3: chunked prefill): sequence b brings n_b new query rows (packed in q
+// from q_start[b]); their K/V are already in the pool, which holds
+// seq_lens[b] = L_b tokens.  Row i sits at position L_b - n_b + i and attends
+// causally to tokens 0 .. that position through the block table (vLLM paging
+// page §3 phase 2), KV head h / G, fp32 output.
+//
+// One CTA computes one tile: 128 rows = 128/G query tokens x the G query heads
+// of one KV head, so a GQA group turns into a full M = 128 MMA tile even for
+// short chunks.  Keys come in chunks of 128 tokens (128/block_size physical
+// blocks, one TMA box per block and head_dim half).  Per chunk j:
+//
+//   S_j = Q · K_jᵀ        tcgen05.mma, 128x128x128, fp32 in tensor memory
+//   P_j = 2^(S_j·scale·log2e - m)   4 softmax warps, one row per thread
+//   O  += P_j · V_j       tcgen05.mma, P split into bf16 (or f16) hi + lo
+//
+// Warp roles (192 threads): warps 0-3 softmax (thread = row = TMEM lane),
+// warp 4 TMA producer, warp 5 MMA issuer (lane 0) and TMEM owner.  Tensor
+// memory (512 columns): S double buffer at columns 0 and 128, O at 256.
+// Shared memory: Q 32 KB, K and V rings of two 32 KB stages, P hi + lo 64 KB.
+//
+// Pipeline: the MMA warp issues S_0, S_1, then per chunk PV_j followed by
+// S_{j+2}, so q·Kᵀ of the next chunks runs while the softmax warps work on
+// the current one; the softmax warps compute chunk j's exponentials while
+// PV_{j-1} is still running and only wait for it before overwriting P.
+// The running max moves lazily (only by more than 8 in log2 units), as in the
+// decode kernels; a move rescales that row's O in tensor memory.
+//
+// P precision: a single bf16 P misses the 2e-3 output tolerance at early
+// positions (few keys of comparable weight); hi + lo halves keep it within
+// about 1e-5, at the cost of a second P·V pass (one MMA per half).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdint>
+#include <type_traits>
+
+#include "device_common.cuh"
+#include "tcgen05.cuh"
+
+namespace pkv {
+
+struct PrefillParams {
+  const int32_t* block_tables;  // [num_seqs, max_blocks]
+  const int32_t* seq_lens;      // [num_seqs] tokens in the pool, chunk included
+  const int32_t* q_start;       // [num_seqs + 1] first q row of each sequence
+  float* out;                   // [num_q_tokens, num_q_heads, 128]
+  int32_t num_seqs, num_q_heads, num_kv_heads, num_blocks, max_blocks, block_size;
+  int32_t num_q_tokens, max_q_len, n_tiles;
+  float scale_log2;  // scale · log2(e)
+};
+
+namespace pf {
+constexpr int kRows = 128;              // MMA M: query rows per tile
+constexpr int kKeys = 128;              // keys per chunk (S columns, P·V contraction)
+constexpr int kHeadDim = 128;
+constexpr uint32_t kSlab = 128 * 128;   // 128 rows x 64 elements x 2 bytes
+constexpr uint32_t kTile = 2 * kSlab;   // 128 rows x head_dim 128
+constexpr int kStages = 2;
+constexpr int kThreads = 192;
+constexpr int kProducerWarp = 4, kMmaWarp = 5;
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffK = kOffQ + kTile;
+constexpr uint32_t kOffV = kOffK + kStages * kTile;
+constexpr uint32_t kOffP = kOffV + kStages * kTile;  // hi tile, then lo tile
+constexpr uint32_t kOffBar = kOffP + 2 * kTile;
+constexpr size_t kSmemBytes = kOffBar + 256 + 1024;  // barriers, flags; 1024 B alignment slack
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0, kColO = 256;
+constexpr float kRescale = 8.0f;
+constexpr unsigned kAll = 0xffffffffu;
+// mbarrier slots
+enum : int { kQFull = 0, kKFull = 1, kKEmpty = 3, kVFull = 5, kVEmpty = 7, kSFull = 9, kPFull = 11, kPVDone = 12,
+             kDrain = 13, kNumBars = 14 };
+}  // namespace pf
+
+__device__ __forceinline__ void tma_load_3d_nohint(uint32_t dst, const void* tmap, int32_t x, int32_t y, int32_t z,
+                                                   uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, int32_t x, int32_t y, int32_t z, int32_t w,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
+      : "memory");
+}
+
+// Waits (bounded by time only) for a phase; used to drain copies and MMAs in
+// flight before the CTA exits or frees tensor memory.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity) && global_timer_ns() - t0 < kWaitLimitNs) {
+  }
+}
+
+template <typename T, int G>
+__global__ void __launch_bounds__(pf::kThreads, 1)
+    prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_q,
+                      const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v) {
+  static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
+  constexpr int QT = pf::kRows / G;  // query tokens per tile
+  constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+
+  // ---- the tile: (sequence b, KV head g, tile of QT query tokens); the
+  // tiles with the most keys (highest index) are launched first ----
+  const int per_tile = p.num_seqs * p.num_kv_heads;
+  const int tile = p.n_tiles - 1 - static_cast<int>(blockIdx.x) / per_tile;
+  const int rest = static_cast<int>(blockIdx.x) % per_tile;
+  const int b = rest / p.num_kv_heads, g = rest % p.num_kv_heads;
+  const int q0 = p.q_start[b], q1 = p.q_start[b + 1];
+  const int n = q1 - q0, L = p.seq_lens[b];
+  if (n < 0 || q0 < 0 || q1 > p.num_q_tokens || n > L || n > p.max_q_len ||
+      L > p.max_blocks * p.block_size) {
+    if (threadIdx.x == 0 && tile == 0) record_error(PKV_ERR_INVALID_ARG);
+    return;
+  }
+  const int tok0 = tile * QT;  // chunk-relative first token of the tile
+  if (tok0 >= n) return;       // uniform across the CTA: nothing allocated yet
+  const int ctx = L - n;
+  const int pos_min = ctx + tok0;
+  const int pos_max = min(L - 1, ctx + tok0 + QT - 1);
+  const int nc = pos_max / pf::kKeys + 1;  // key chunks this tile attends to
+  const int BS = p.block_size;
+  const int nblk = (L + BS - 1) / BS;
+
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t base = smem_addr(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + pf::kOffBar);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + pf::kNumBars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + pf::kNumBars) + 1;
+  auto bar = [&](int i) { return smem_addr(bars + i); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < pf::kNumBars; ++i) mbar_init(bar(i), i == pf::kPFull ? 128u : 1u);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == pf::kMmaWarp) {
+    tc::tmem_alloc(smem_addr(tmem_slot), pf::kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == pf::kProducerWarp) {
+    // ------------------------------ TMA producer ------------------------------
+    bool ok = true;
+    if (lane == 0) {
+      prefetch_tensormap(&tmap_q);
+      prefetch_tensormap(&tmap_k);
+      prefetch_tensormap(&tmap_v);
+      // Q tile: rows token * G + h, one box per head_dim half
+      mbar_arrive_expect_tx(bar(pf::kQFull), pf::kTile);
+      tma_load_4d(base + pf::kOffQ, &tmap_q, 0, 0, g * G, q0 + tok0, bar(pf::kQFull));
+      tma_load_4d(base + pf::kOffQ + pf::kSlab, &tmap_q, 0, 1, g * G, q0 + tok0, bar(pf::kQFull));
+    }
+    const int32_t* trow = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
+    const int nbc = pf::kKeys / BS;                              // blocks per chunk
+    const uint32_t box_bytes = static_cast<uint32_t>(BS) * 128;  // one block, one head_dim half
+    int issued[2] = {0, 0};  // chunks whose K (V) fill was issued
+    for (int j = 0; j < nc && ok; ++j) {
+      const int s = j & 1;
+      const uint32_t ph = ((j >> 1) & 1) ^ 1;
+      const int jb = j * nbc;
+      const int nload = min(nbc, nblk - jb);  // blocks past the sequence end are not read
+      int phys = 0;
+      if (lane < nload) {
+        phys = trow[jb + lane];
+        if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_blocks)) {
+          record_error(PKV_ERR_BAD_BLOCK);
+          phys = 0;
+        }
+      }
+      const int32_t y = (phys * p.num_kv_heads + g) * BS;
+      for (int kv = 0; kv < 2; ++kv) {
+        const uint32_t full = bar((kv ? pf::kVFull : pf::kKFull) + s);
+        ok = __all_sync(pf::kAll, mbar_wait(bar((kv ? pf::kVEmpty : pf::kKEmpty) + s), ph, abort_flag));
+        if (!ok) break;
+        if (lane == 0) mbar_arrive_expect_tx(full, static_cast<uint32_t>(nload) * 2u * box_bytes);
+        __syncwarp();
+        if (lane < nload) {
+          const uint32_t dst = base + (kv ? pf::kOffV : pf::kOffK) + s * pf::kTile + lane * box_bytes;
+          const void* map = kv ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k);
+          tma_load_3d_nohint(dst, map, 0, y, 0, full);
+          tma_load_3d_nohint(dst + pf::kSlab, map, 0, y, 1, full);
+        }
+        ++issued[kv];
+      }
+    }
+    if (!ok && lane == 0) {
+      record_error(PKV_ERR_DEVICE_TIMEOUT);
+      *abort_flag = 1;
+    }
+    // no copy may still be landing when the CTA exits: wait (bounded) for the
+    // last fill of each stage and for Q
+    if (lane == 0) {
+      drain_wait(bar(pf::kQFull), 0);
+      for (int kv = 0; kv < 2; ++kv) {
+        for (int s = 0; s < pf::kStages && s < issued[kv]; ++s) {
+          const int last = issued[kv] - 1 - ((issued[kv] - 1 - s) & 1);  // last chunk that used stage s
+          drain_wait(bar((kv ? pf::kVFull : pf::kKFull) + s), (last >> 1) & 1);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == pf::kMmaWarp) {
+    // ------------------------------- MMA issuer -------------------------------
+    if (lane == 0) {
+      const uint32_t id_s = tc::idesc_f16(kBf16, false, pf::kRows, pf::kKeys);
+      const uint32_t id_o = tc::idesc_f16(kBf16, true, pf::kRows, pf::kHeadDim);
+      auto issue_s = [&](int j) -> bool {
+        const int s = j & 1;
+        if (!mbar_wait(bar(pf::kKFull + s), (j >> 1) & 1, abort_flag)) return false;
+        tc::fence_after_sync();
+        const uint32_t kst = base + pf::kOffK + s * pf::kTile;
+#pragma unroll
+        for (int kk = 0; kk < pf::kHeadDim / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * pf::kSlab + (kk & 3) * 32;
+          tc::mma_f16_ss(tmem + pf::kColS + s * pf::kKeys, tc::sw128_desc(base + pf::kOffQ + off, 16, 1024),
+                         tc::sw128_desc(kst + off, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+        }
+        tc::commit(bar(pf::kKEmpty + s));
+        tc::commit(bar(pf::kSFull + s));
+        return true;
+      };
+      bool ok = mbar_wait(bar(pf::kQFull), 0, abort_flag);
+      if (ok) ok = issue_s(0);
+      if (ok && nc > 1) ok = issue_s(1);
+      for (int j = 0; j < nc && ok; ++j) {
+        const int s = j & 1;
+        ok = mbar_wait(bar(pf::kPFull), j & 1, abort_flag) && mbar_wait(bar(pf::kVFull + s), (j >> 1) & 1, abort_flag);
+        if (!ok) break;
+        tc::fence_after_sync();
+        const uint32_t vst = base + pf::kOffV + s * pf::kTile;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+#pragma unroll
+          for (int kk = 0; kk < pf::kKeys / 16; ++kk) {
+            const uint32_t a = base + pf::kOffP + part * pf::kTile + (kk >> 2) * pf::kSlab + (kk & 3) * 32;
+            const uint32_t bv = vst + kk * 16 * 128;  // 16 keys of 128-byte rows
+            tc::mma_f16_ss(tmem + pf::kColO, tc::sw128_desc(a, 16, 1024), tc::sw128_desc(bv, pf::kSlab, 1024), id_o,
+                           (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        tc::commit(bar(pf::kVEmpty + s));
+        tc::commit(bar(pf::kPVDone));
+        if (j + 2 < nc) ok = issue_s(j + 2);
+      }
+      if (!ok) {
+        record_error(PKV_ERR_DEVICE_TIMEOUT);
+        *abort_flag = 1;
+      }
+      // every MMA issued so far completes before tensor memory is freed
+      tc::commit(bar(pf::kDrain));
+      drain_wait(bar(pf::kDrain), 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------ softmax warps ------------------------------
+    const int r = threadIdx.x;  // tile row and TMEM lane
+    const int tok = tok0 + r / G;
+    const bool valid = tok < n;
+    const int pos = min(ctx + tok, L - 1);  // rows past the chunk end compute a copy of the last row
+    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t p_row = base + pf::kOffP + r * 128;
+    unsigned char* vzero = smem + pf::kOffV;
+    const float sl = p.scale_log2;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nc && ok; ++j) {
+      const int s = j & 1;
+      ok = __all_sync(pf::kAll, mbar_wait(bar(pf::kSFull + s), (j >> 1) & 1, abort_flag));
+      if (!ok) break;
+      tc::fence_after_sync();
+      float x[pf::kKeys];
+      {
+        uint32_t raw[4][32];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tc::ld_32x32b_x32(trow + pf::kColS + s * pf::kKeys + 32 * q, raw[q]);
+        tc::wait_ld();
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[32 * q + i] = __uint_as_float(raw[q][i]) * sl;
+      }
+      const int key0 = j * pf::kKeys;
+      if (key0 + pf::kKeys - 1 > pos_min) {  // the diagonal: keys after a row's position are hidden
+#pragma unroll
+        for (int c = 0; c < pf::kKeys; ++c) x[c] = key0 + c <= pos ? x[c] : -INFINITY;
+      }
+      float mc = x[0];
+#pragma unroll
+      for (int c = 1; c < pf::kKeys; ++c) mc = fmaxf(mc, x[c]);
+      float factor = 1.f;
+      bool resc = false;
+      if (j == 0) {
+        m_used = mc;  // key 0 is visible to every row: finite
+      } else if (mc > m_used + pf::kRescale) {
+        factor = fast_exp2(m_used - mc);
+        m_used = mc;
+        resc = true;
+      }
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < pf::kKeys; ++c) {
+        x[c] = fast_exp2(x[c] - m_used);
+        sum += x[c];
+      }
+      l = l * factor + sum;
+
+      if (j > 0) {
+        // P_{j-1} and O are still being read by P·V of the previous chunk
+        ok = __all_sync(pf::kAll, mbar_wait(bar(pf::kPVDone), (j - 1) & 1, abort_flag));
+        if (!ok) break;
+        tc::fence_after_sync();
+        if (__any_sync(pf::kAll, resc)) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t o[32];
+            tc::ld_32x32b_x32(trow + pf::kColO + 32 * q, o);
+            tc::wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
+            tc::st_32x32b_x32(trow + pf::kColO + 32 * q, o);
+          }
+          tc::wait_st();
+        }
+      }
+      if (key0 + pf::kKeys > L) {
+        // V rows past the sequence end hold stale or unwritten bytes: zero
+        // them so that P = 0 there cannot meet a NaN pattern
+        ok = __all_sync(pf::kAll, mbar_wait(bar(pf::kVFull + s), (j >> 1) & 1, abort_flag));
+        if (!ok) break;
+        const int v0 = L - key0;
+        unsigned char* vst = vzero + s * pf::kTile;
+        for (int idx = r; idx < (pf::kKeys - v0) * 16; idx += 128) {
+          const int row = v0 + (idx >> 4), piece = idx & 15;
+          *reinterpret_cast<uint4*>(vst + (piece >> 3) * pf::kSlab + row * 128 + (piece & 7) * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      // P hi and lo into the 128-byte-swizzled K-major layout (row r, keys in
+      // two slabs of 64, 16-byte chunk c at position c ^ (r % 8))
+#pragma unroll
+      for (int slab = 0; slab < 2; ++slab) {
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = slab * 64 + ch * 8 + 2 * e;
+            split_pack<T>(x[c], x[c + 1], hi[e], lo[e]);
+          }
+          const uint32_t off = slab * pf::kSlab + ((ch ^ (r & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(p_row + off), "r"(hi[0]), "r"(hi[1]),
+                       "r"(hi[2]), "r"(hi[3])
+                       : "memory");
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(p_row + pf::kTile + off), "r"(lo[0]),
+                       "r"(lo[1]), "r"(lo[2]), "r"(lo[3])
+                       : "memory");
+        }
+      }
+      fence_proxy_async_smem();  // P (and zeroed V rows) visible to the tensor core
+      tc::fence_before_sync();
+      mbar_arrive(bar(pf::kPFull));
+    }
+    if (ok) ok = __all_sync(pf::kAll, mbar_wait(bar(pf::kPVDone), (nc - 1) & 1, abort_flag));
+    if (ok) {
+      tc::fence_after_sync();
+      const float inv = 1.f / l;
+      float* orow = p.out + (static_cast<int64_t>(q0 + tok) * p.num_q_heads + g * G + r % G) * pf::kHeadDim;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t o[32];
+        tc::ld_32x32b_x32(trow + pf::kColO + 32 * q, o);
+        tc::wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(orow + 32 * q + i) =
+                make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
+                            __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+        }
+      }
+    } else if (lane == 0) {
+      record_error(PKV_ERR_DEVICE_TIMEOUT);
+      *abort_flag = 1;
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == pf::kMmaWarp) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, pf::kTmemCols);
+  }
+}
+
+}  // namespace pkv

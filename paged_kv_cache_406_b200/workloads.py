@@ -1,4 +1,4 @@
-"""Seeded synthetic workloads for the paged decode path.
+"""Seeded synthetic workloads for the paged decode and prefill paths.
 
 This module only draws inputs: sequence lengths, the order in which physical
 blocks leave the free list, and N(0, 1) values for q / K / V.  It holds none
@@ -40,6 +40,7 @@ class Workload:
     prefix_tokens: int = 0     # tokens shared by every sequence (refcount = num_seqs)
     pool_slack: float = 1.2    # pool size as a multiple of the blocks needed
     kv_scale: float = 1.0 / 32  # e4m3 pools: value = kv_scale * code value (K and V)
+    chunk_tokens: int = 0      # prefill workloads: new query rows per sequence (0: a decode workload)
 
     @property
     def torch_dtype(self) -> torch.dtype:
@@ -74,6 +75,14 @@ WORKLOADS = {
     "long_splitk": Workload("long_splitk", 8, 32, 8, 128, 16, "bf16", 406004, partition_tokens=512),
     # 7B MHA at high concurrency: 256 lognormal(median 1000, sigma 1) lengths in [16, 8192], 50 steps
     "mha_7b": Workload("mha_7b", 256, 32, 32, 128, 16, "f16", 406005, steps=50),
+    # chunked prefill on the Llama-3-8B layer: 16 sequences, a 512-token chunk
+    # each on top of U[0, 3584] cached tokens (so 512 .. 4096 tokens in all)
+    "prefill_llama3_8b": Workload("prefill_llama3_8b", 16, 32, 8, 128, 16, "bf16", 406006, chunk_tokens=512),
+    # the optimisation-overview page's traffic mix for adaptive block sizes:
+    # 80 % of 64 sequences below 1024 tokens, the rest 1024..8191, one >= 8192
+    "adaptive_mix": Workload("adaptive_mix", 64, 32, 8, 128, 16, "bf16", 406008),
+    # whole 2048-token prompts from an empty cache, 8 sequences
+    "prefill_prompt_2k": Workload("prefill_prompt_2k", 8, 32, 8, 128, 16, "bf16", 406007, chunk_tokens=2048),
 }
 
 
@@ -85,7 +94,8 @@ def scaled(w: Workload, **kw) -> Workload:
 def seq_lens(w: Workload) -> np.ndarray:
     """Per-sequence token counts before the first decode step (int64).
 
-    For prefix-shared workloads this is prefix + tail."""
+    For prefix-shared workloads this is prefix + tail; for prefill workloads
+    the context cached before the chunk of ``chunk_tokens`` new rows."""
     rng = np.random.Generator(np.random.PCG64(w.seed))
     n = w.num_seqs
     if w.name == "tiny":
@@ -97,6 +107,16 @@ def seq_lens(w: Workload) -> np.ndarray:
     if w.name.startswith("long_splitk"):
         base = np.array([32768] * 7 + [131072], dtype=np.int64)
         return base[:n] if n <= 8 else np.resize(base, n)
+    if w.name.startswith("adaptive_mix"):
+        short = int(round(0.8 * n))
+        long_ = max(0, n - short - 1)
+        return np.concatenate([rng.integers(128, 1023, size=short, endpoint=True),
+                               rng.integers(1024, 8191, size=long_, endpoint=True),
+                               rng.integers(8192, 16384, size=n - short - long_, endpoint=True)]).astype(np.int64)
+    if w.name.startswith("prefill_llama3_8b"):  # cached context before the chunk
+        return rng.integers(0, 3584, size=n, endpoint=True).astype(np.int64)
+    if w.name.startswith("prefill_prompt"):
+        return np.zeros(n, dtype=np.int64)
     if w.name.startswith("mha_7b"):
         x = rng.lognormal(mean=math.log(1000.0), sigma=1.0, size=n)
         return np.clip(np.rint(x), 16, 8192).astype(np.int64)

@@ -1,0 +1,204 @@
+"""GPU parity: causal paged prefill attention through the C-ABI against the
+fp64 oracle (B200, tcgen05 kernel).
+
+Tolerance: |gpu - oracle| <= 2e-3 * max(1, |oracle|) elementwise for bf16 /
+fp16 K/V (fp32 output).  Every pool slot that no sequence owns (the tail of a
+partial block, spare blocks) holds NaN, so a kernel that lets an unowned row
+into the result cannot pass.
+"""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+from helpers import DT, assert_close, raw
+from oracle import paged_attention as pa
+from oracle.block_allocator import BlockAllocatorModel
+
+pytestmark = pytest.mark.gpu
+
+import paged_kv_cache_406_b200 as pkv  # noqa: E402
+
+D = 128
+
+
+@pytest.fixture(autouse=True)
+def _clean_status(native):
+    pkv.pkv_device_status(clear=True)
+    yield
+    assert pkv.pkv_device_status(clear=True) == 0, "a kernel recorded a device error"
+
+
+class PrefillCase:
+    """Sequences of ``lens`` tokens whose last ``q_lens`` are the new chunk."""
+
+    def __init__(self, lens, q_lens, hq, hkv, bs, dtype, seed, guard=3, k_ramp=0.0):
+        rng = np.random.default_rng(seed)
+        self.lens, self.q_lens = list(lens), list(q_lens)
+        self.hq, self.hkv, self.bs, self.dtype = hq, hkv, bs, dtype
+        need = sum(-(-L // bs) for L in self.lens)
+        self.nb = need + guard
+        model = BlockAllocatorModel(self.nb, bs, rng.permutation(self.nb))
+        for b, L in enumerate(self.lens):
+            model.add(b, L)
+        self.maxb = max(1, max(len(model.block_table(b)) for b in range(len(self.lens))))
+        self.tables = np.full((len(self.lens), self.maxb), -1, dtype=np.int32)
+        shape = (self.nb, hkv, bs, D)
+        k = torch.full(shape, float("nan"), dtype=torch.float32)
+        v = torch.full(shape, float("nan"), dtype=torch.float32)
+        for b, L in enumerate(self.lens):
+            t = model.block_table(b)
+            self.tables[b, :len(t)] = t
+            kr = torch.from_numpy(rng.standard_normal((L, hkv, D), dtype=np.float32))
+            vr = torch.from_numpy(rng.standard_normal((L, hkv, D), dtype=np.float32))
+            if k_ramp:
+                # scores that keep growing along the sequence: the running max
+                # moves by more than the lazy-rescale threshold chunk after chunk
+                kr = kr * 0.25 + k_ramp * torch.linspace(0, 1, L)[:, None, None]
+            for i in range(L):
+                k[t[i // bs], :, i % bs] = kr[i]
+                v[t[i // bs], :, i % bs] = vr[i]
+        self.k_pool, self.v_pool = k.to(DT[dtype]), v.to(DT[dtype])
+        T = sum(self.q_lens)
+        q = rng.standard_normal((T, hq, D), dtype=np.float32)
+        if k_ramp:
+            q = np.abs(q) * 0.5 + 1.0
+        self.q = torch.from_numpy(q).to(DT[dtype])
+        self.q_start = np.concatenate([[0], np.cumsum(self.q_lens)]).astype(np.int32)
+        self.scale = 1.0 / np.sqrt(D)
+
+    def oracle(self):
+        return pa.paged_prefill_attention(raw(self.q), raw(self.k_pool), raw(self.v_pool), self.tables,
+                                          np.array(self.lens), np.array(self.q_lens), self.scale, self.dtype)
+
+    def run(self, max_q_len=None, out=None):
+        dev = "cuda"
+        res = pkv.pkv_paged_attention_prefill(
+            self.q.to(dev), self.k_pool.to(dev), self.v_pool.to(dev), torch.from_numpy(self.tables).to(dev),
+            torch.tensor(self.lens, dtype=torch.int32, device=dev), torch.from_numpy(self.q_start).to(dev),
+            max(self.q_lens) if max_q_len is None else max_q_len, self.scale, out=out)
+        torch.cuda.synchronize()
+        return res
+
+
+def _seed(*k):
+    return zlib.crc32("-".join(map(str, k)).encode()) % 100000
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("g", [1, 2, 4, 8])
+@pytest.mark.parametrize("bs", [8, 16, 32])
+def test_prefill_matches_oracle(dtype, g, bs):
+    """Whole prompts, chunks behind earlier context, ragged tiles and chunks,
+    lengths around the 128-key chunk edges."""
+    lens = [1, 130, 300, 129, 517, 64]
+    q_lens = [1, 130, 77, 1, 45, 64]
+    case = PrefillCase(lens, q_lens, 2 * g, 2, bs, dtype, _seed(dtype, g, bs))
+    out = case.run()
+    assert_close(out, case.oracle(), dtype, f"prefill {dtype} G{g} bs{bs}")
+
+
+@pytest.mark.parametrize("g", [1, 4])
+def test_long_context_and_many_tiles(g):
+    lens, q_lens = [1500, 700], [300, 700]
+    case = PrefillCase(lens, q_lens, 2 * g, 2, 16, "bf16", _seed("long", g))
+    assert_close(case.run(), case.oracle(), "bf16", f"long G{g}")
+
+
+def test_growing_scores_rescale_the_accumulator():
+    """Scores rise along the sequence so the running max moves by more than
+    the lazy threshold in many chunks: every such move rescales O."""
+    case = PrefillCase([900, 400], [200, 400], 8, 2, 16, "bf16", _seed("ramp"), k_ramp=12.0)
+    ref = case.oracle()
+    assert_close(case.run(), ref, "bf16", "rescaled")
+
+
+def test_one_row_chunks_agree_with_decode():
+    lens = [1, 15, 16, 17, 200, 1000]
+    case = PrefillCase(lens, [1] * len(lens), 8, 2, 16, "bf16", _seed("decode"))
+    pre = case.run()
+    dec = pkv.pkv_paged_attention_decode(case.q.cuda(), case.k_pool.cuda(), case.v_pool.cuda(),
+                                         torch.from_numpy(case.tables).cuda(),
+                                         torch.tensor(lens, dtype=torch.int32, device="cuda"), case.scale)
+    torch.cuda.synchronize()
+    ref = case.oracle()
+    assert_close(pre, ref, "bf16", "prefill n=1")
+    assert_close(dec, ref, "bf16", "decode")
+
+
+def test_chunked_prefill_equals_one_shot():
+    """A 600-token prompt fed as chunks of 128, 1, 300 and 171 tokens (each
+    call seeing the pool as written so far) reproduces the one-shot rows."""
+    L = 600
+    whole = PrefillCase([L], [L], 8, 2, 16, "bf16", _seed("chunks"))
+    ref = whole.oracle()
+    full = whole.run()
+    dev = "cuda"
+    kp, vp, q = whole.k_pool.to(dev), whole.v_pool.to(dev), whole.q.to(dev)
+    tables = torch.from_numpy(whole.tables).to(dev)
+    pieces, start = [], 0
+    for n in (128, 1, 300, 171):
+        end = start + n
+        out = pkv.pkv_paged_attention_prefill(q[start:end].contiguous(), kp, vp, tables,
+                                              torch.tensor([end], dtype=torch.int32, device=dev),
+                                              torch.tensor([0, n], dtype=torch.int32, device=dev), n, whole.scale)
+        pieces.append(out)
+        start = end
+    torch.cuda.synchronize()
+    chunked = torch.cat(pieces)
+    assert_close(full, ref, "bf16", "one shot")
+    assert_close(chunked, ref, "bf16", "chunked")
+
+
+def test_empty_chunks_uncovered_rows_and_slack_tiles():
+    """n = 0 sequences, rows no chunk owns (left untouched) and a max_q_len
+    far above every chunk (the extra tiles exit)."""
+    case = PrefillCase([40, 7, 90], [3, 0, 20], 8, 2, 8, "f16", _seed("empty"))
+    dev = "cuda"
+    T = sum(case.q_lens)
+    q = torch.cat([case.q, torch.zeros((5, 8, D), dtype=case.q.dtype)]).to(dev)  # 5 rows owned by nobody
+    out = torch.full((T + 5, 8, D), 7.0, dtype=torch.float32, device=dev)
+    pkv.pkv_paged_attention_prefill(q, case.k_pool.to(dev), case.v_pool.to(dev),
+                                    torch.from_numpy(case.tables).to(dev),
+                                    torch.tensor(case.lens, dtype=torch.int32, device=dev),
+                                    torch.from_numpy(case.q_start).to(dev), 1000, case.scale, out=out)
+    torch.cuda.synchronize()
+    assert_close(out[:T], case.oracle(), "f16", "owned rows")
+    assert bool((out[T:] == 7.0).all()), "rows outside every chunk were written"
+
+
+def test_chunk_longer_than_sequence_is_recorded():
+    case = PrefillCase([10, 20], [5, 5], 4, 1, 16, "bf16", _seed("bad"))
+    dev = "cuda"
+    out = torch.full((10, 4, D), 3.0, device=dev)
+    pkv.pkv_paged_attention_prefill(case.q.to(dev), case.k_pool.to(dev), case.v_pool.to(dev),
+                                    torch.from_numpy(case.tables).to(dev),
+                                    torch.tensor([3, 20], dtype=torch.int32, device=dev),  # 5 rows > 3 tokens
+                                    torch.from_numpy(case.q_start).to(dev), 5, case.scale, out=out)
+    torch.cuda.synchronize()
+    assert pkv.pkv_device_status(clear=True) == pkv._native.PKV_ERR_INVALID_ARG
+    assert bool((out[:5] == 3.0).all())
+    ref = PrefillCase([10, 20], [5, 5], 4, 1, 16, "bf16", _seed("bad")).oracle()
+    assert_close(out[5:], ref[5:], "bf16", "the valid sequence")
+
+
+def test_unsupported_arguments_are_refused():
+    dev = "cuda"
+    kp = torch.zeros((4, 1, 16, D), dtype=torch.bfloat16, device=dev)
+    tables = torch.zeros((1, 1), dtype=torch.int32, device=dev)
+    lens = torch.ones(1, dtype=torch.int32, device=dev)
+    qs = torch.tensor([0, 1], dtype=torch.int32, device=dev)
+    with pytest.raises(pkv.PagedKVError) as e:  # fp32 pools: tensor cores take 16-bit operands only
+        pkv.pkv_paged_attention_prefill(torch.zeros((1, 1, D), device=dev), kp.float(), kp.float(), tables, lens,
+                                        qs, 1, 1.0)
+    assert e.value.code == -4
+    k64 = torch.zeros((4, 1, 16, 64), dtype=torch.bfloat16, device=dev)
+    with pytest.raises(pkv.PagedKVError) as e:
+        pkv.pkv_paged_attention_prefill(torch.zeros((1, 1, 64), dtype=torch.bfloat16, device=dev), k64, k64,
+                                        tables, lens, qs, 1, 1.0)
+    assert e.value.code == -4
+    with pytest.raises(pkv.PagedKVError) as e:  # group size 3
+        pkv.pkv_paged_attention_prefill(torch.zeros((1, 3, D), dtype=torch.bfloat16, device=dev), kp, kp, tables,
+                                        lens, qs, 1, 1.0)
+    assert e.value.code == -4
