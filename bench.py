@@ -40,10 +40,11 @@ STAGED_STEPS = 16  # distinct steps of metadata resident on the device, cycled
 
 # DRAM traffic of one pkv_paged_attention_decode call on the default workload,
 # from the ncu capture summarised in profiles/ (dram__bytes_read.sum +
-# dram__bytes_write.sum over its kernels).  Valid only while the kernel
-# sources hash to TRAFFIC_SOURCE_SHA; otherwise reported as null.
-TRAFFIC_BYTES = 607263488  # plan + decode + merge kernels, mean of two captured calls
-TRAFFIC_SOURCE_SHA = "62c7be410db53362"
+# dram__bytes_write.sum over its plan, decode and merge kernels, mean of two
+# captured calls).  Valid only while the decode sources hash to
+# TRAFFIC_SOURCE_SHA (kernel_source_sha()); otherwise reported as null.
+TRAFFIC_BYTES = 606448512
+TRAFFIC_SOURCE_SHA = "679a323a3900964d"
 
 
 SEQ_LEN_RECIPES = {
@@ -57,14 +58,17 @@ SEQ_LEN_RECIPES = {
 }
 
 
-def kernel_source_sha() -> str:
-    """Hash of the device sources (every .cu / .cuh file of the library)."""
+DECODE_SOURCES = ("decode.cuh", "decode_mma.cuh", "device_common.cuh")
+PREFILL_SOURCES = ("prefill.cuh", "tcgen05.cuh", "device_common.cuh")
+
+
+def kernel_source_sha(names=DECODE_SOURCES) -> str:
+    """Hash of the device sources a kernel is built from (csrc files)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_406_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(f.read())
+    for name in names:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -668,7 +672,7 @@ def run_prefill(args, w0):
                          "traffic": None, "algorithmic_flops_per_launch": flops,
                          "tensor_flops_issued_per_launch": "1.5x algorithmic (P·V runs on P hi and P lo) plus the "
                                                           "masked part of diagonal chunks",
-                         "avg_launch_ms": round(attn_ms, 5), "kernel_source_sha": kernel_source_sha()},
+                         "avg_launch_ms": round(attn_ms, 5), "kernel_source_sha": kernel_source_sha(PREFILL_SOURCES)},
             "gpu_launches": launches, "clocks": clk, "cpu_baseline": cpu, "e2e": e2e,
         }
         print(json.dumps(res), flush=True)
