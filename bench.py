@@ -681,10 +681,10 @@ def run_prefill(args, w0):
 
 
 def run_adaptive(args, w):
-    """Adaptive block size (optimisation-overview page §3.3) against one
-    fixed 16-token pool on the same batch: a step appends one token per
-    sequence and runs paged decode attention; the adaptive arm does that
-    once per block-size class (32 / 16 / 8)."""
+    """Adaptive block size (optimisation-overview page §3.3) against single
+    pools of 16-, 32- and 8-token blocks on the same batch: a step appends one
+    token per sequence and runs paged decode attention; the adaptive arm does
+    that once per block-size class (32 / 16 / 8)."""
     import paged_kv_cache_406_b200 as P
     from paged_kv_cache_406_b200 import workloads as W
     from paged_kv_cache_406_b200.cache import AdaptivePagedKVCache, PagedKVCache, block_size_for
@@ -703,15 +703,18 @@ def run_adaptive(args, w):
         per_class[bs] = per_class.get(bs, 0) + -(-(int(L) + horizon) // bs)
     per_class = {bs: int(np.ceil(1.2 * nb)) for bs, nb in per_class.items()}
     ad = AdaptivePagedKVCache(per_class, hkv, d, w.torch_dtype, maxtok, device=dev, seed=w.seed)
-    nb16 = int(np.ceil(1.2 * sum(-(-(int(L) + horizon) // 16) for L in lens0)))
-    fixed = PagedKVCache(nb16, hkv, d, 16, w.torch_dtype, -(-maxtok // 16), device=dev,
-                         free_order=W.free_order(nb16, w.seed))
-    for k, c in enumerate(list(ad.caches.values()) + [fixed]):
+    fixed = {}
+    for fbs in (16, 32, 8):  # one pool of a single block size for the whole batch
+        nbf = int(np.ceil(1.2 * sum(-(-(int(L) + horizon) // fbs) for L in lens0)))
+        fixed[fbs] = PagedKVCache(nbf, hkv, d, fbs, w.torch_dtype, -(-maxtok // fbs), device=dev,
+                                  free_order=W.free_order(nbf, w.seed))
+    for k, c in enumerate(list(ad.caches.values()) + list(fixed.values())):
         c.k_pool.copy_(W.normal(c.k_pool.shape, w.torch_dtype, W.pool_seed(w, 0) + 17 * k, device=dev))
         c.v_pool.copy_(W.normal(c.v_pool.shape, w.torch_dtype, W.pool_seed(w, 1) + 17 * k, device=dev))
     for i, L in enumerate(lens0):
         ad.add(i, int(L))
-        fixed.add(i, int(L))
+        for c in fixed.values():
+            c.add(i, int(L))
     ids = ad.order()
     e = torch.tensor([], dtype=w.torch_dtype).element_size()
     q = W.normal((B, hq, d), w.torch_dtype, W.step_seed(w, 0, 0), device=dev)
@@ -728,7 +731,7 @@ def run_adaptive(args, w):
         wsb = P.pkv_decode_workspace_size(len(members), hq, hkv, d, cache.max_blocks, cache.block_size, 0)
         return out, torch.empty(wsb, dtype=torch.uint8, device=dev)
 
-    arms = {"adaptive": [], "fixed_bs16": []}
+    arms = {"adaptive": [], "fixed_bs16": [], "fixed_bs32": [], "fixed_bs8": []}
     a = 0
     for bs in ad.CLASSES:
         members = [i for i in ids if ad.cls[i] == bs]
@@ -736,8 +739,9 @@ def run_adaptive(args, w):
             st, wsp = stage(ad.caches[bs], members)
             arms["adaptive"].append((ad.caches[bs], st, wsp, slice(a, a + len(members))))
             a += len(members)
-    st, wsp = stage(fixed, ids)
-    arms["fixed_bs16"].append((fixed, st, wsp, slice(0, B)))
+    for fbs, c in fixed.items():
+        st, wsp = stage(c, ids)
+        arms[f"fixed_bs{fbs}"].append((c, st, wsp, slice(0, B)))
     out = torch.empty((B, hq, d), dtype=torch.float32, device=dev)
 
     def step(arm, i):

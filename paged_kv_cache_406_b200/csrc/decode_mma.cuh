@@ -45,8 +45,6 @@ struct MmaLayout {
   static constexpr int kRingHalves = D * kKVBytes / 128;            // 128-byte column halves of a stored row
   static constexpr int kRingTileBytes = kChunkTokens * D * kKVBytes;  // stored 16-token chunk in the ring
   static constexpr int kStageBytes = 2 * kRingTileBytes;
-  // e4m3 chunks are widened into a per-warp 16-bit K and V tile
-  static constexpr int kStagingBytes = kKVBytes == 1 ? 2 * kTileBytes : 0;
 };
 
 template <typename T, int D, int G, int kKVBytes = 2>
@@ -54,7 +52,7 @@ struct MmaSmem {
   using L = MmaLayout<D, kKVBytes>;
   static constexpr int kMergeFloats = G * D + 2 * G;
   __host__ __device__ static size_t ring_bytes(int ns) {
-    return size_t(ns) * L::kStageBytes + size_t(kConsumerWarps) * L::kStagingBytes;
+    return size_t(ns) * L::kStageBytes;
   }
   __host__ __device__ static size_t bytes(int ns) {
     // + 1024: the dynamic shared memory base is aligned up to the 1024-byte swizzle atom
@@ -70,18 +68,6 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t codes) {
   return r;
 }
 
-// 16 e4m3 codes (one 16-byte chunk) widened exactly to 16 f16 values.
-__device__ __forceinline__ void widen_e4m3x16(const uint4& in, uint4& lo, uint4& hi) {
-  lo.x = e4m3x2_to_f16x2(static_cast<uint16_t>(in.x));
-  lo.y = e4m3x2_to_f16x2(static_cast<uint16_t>(in.x >> 16));
-  lo.z = e4m3x2_to_f16x2(static_cast<uint16_t>(in.y));
-  lo.w = e4m3x2_to_f16x2(static_cast<uint16_t>(in.y >> 16));
-  hi.x = e4m3x2_to_f16x2(static_cast<uint16_t>(in.z));
-  hi.y = e4m3x2_to_f16x2(static_cast<uint16_t>(in.z >> 16));
-  hi.z = e4m3x2_to_f16x2(static_cast<uint16_t>(in.w));
-  hi.w = e4m3x2_to_f16x2(static_cast<uint16_t>(in.w >> 16));
-}
-
 // A chunk tile in shared memory is built from TMA boxes of `br` rows (br = 16,
 // or 8 when block_size is 8 and a chunk spans two blocks).  Each box holds,
 // for every 128-byte column half h, br rows of 128 B with the 128-byte
@@ -93,8 +79,10 @@ __device__ __forceinline__ uint32_t row_offset(int r, int h, int br_shift, int h
 }
 
 // kKVBytes = 1: the pools hold e4m3 codes (T must be __half: e4m3 widens to
-// f16 exactly); the consumer warp widens each landed chunk into its own
-// 16-bit staging tile and frees the ring stage before the MMAs.
+// f16 exactly).  A consumer warp loads the codes it needs as 32-bit words,
+// frees the ring stage at once and widens them into mma fragments in
+// registers; the contraction order of q·Kᵀ and the output dims of P·V are
+// permuted within each step so every word feeds whole fragment registers.
 template <typename T, int D, int G, int kKVBytes = 2>
 __global__ void __launch_bounds__(kMmaThreads) decode_mma_kernel(const DecodeParams p,
                                                                     const __grid_constant__ CUtensorMap tmap_k,
@@ -222,16 +210,14 @@ __global__ void __launch_bounds__(kMmaThreads) decode_mma_kernel(const DecodePar
   // ldmatrix row addresses of this lane: K chunk (A operand) and V chunk (A = Vᵀ via .trans)
   const int ra = (lane & 7) + ((lane >> 3) & 1) * 8, ca = lane >> 4;
   const int rv = (lane & 7) + (lane >> 4) * 8, cv = (lane >> 3) & 1;
-  // the tiles the MMAs read: the ring chunk itself (16-bit pools, boxes of
-  // br rows) or the warp's staging tile (e4m3 pools, always 16-row layout)
-  const int tile_shift = kFp8 ? 4 : br_shift;
+  // 16-bit pools: the MMAs read the ring chunk itself, built from boxes of br rows
+  const int tile_shift = br_shift;
   uint32_t offa[kHalves], offv[kHalves];
 #pragma unroll
   for (int h = 0; h < kHalves; ++h) {
     offa[h] = row_offset(ra, h, tile_shift, kHalves);
     offv[h] = row_offset(rv, h, tile_shift, kHalves);
   }
-  const uint32_t staging = ring_s + NS * L::kStageBytes + warp * L::kStagingBytes;
   const int xa = ra & 7, xv = rv & 7;
   const int src0 = 4 * (2 * tq) + (gq >> 1), src1 = src0 + 4;  // Pᵀ transpose sources
   const uint32_t sel = (gq & 1) ? 0x7632u : 0x5410u;
@@ -249,8 +235,16 @@ __global__ void __launch_bounds__(kMmaThreads) decode_mma_kernel(const DecodePar
       const T* qrow = static_cast<const T*>(p.q) + (static_cast<int64_t>(u.b) * p.num_q_heads + u.g * G + gq) * D;
 #pragma unroll
       for (int ks = 0; ks < kSteps; ++ks) {
-        qb[ks][0] = gq < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq)) : 0u;
-        qb[ks][1] = gq < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq + 8)) : 0u;
+        if constexpr (kFp8) {
+          // e4m3 K fragments hold dims 16ks + 4tq .. +3 (one 32-bit word of
+          // codes); q follows the same order of the contraction
+          const uint2 v = gq < G ? __ldg(reinterpret_cast<const uint2*>(qrow + 16 * ks + 4 * tq)) : make_uint2(0u, 0u);
+          qb[ks][0] = v.x;
+          qb[ks][1] = v.y;
+        } else {
+          qb[ks][0] = gq < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq)) : 0u;
+          qb[ks][1] = gq < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq + 8)) : 0u;
+        }
       }
     }
     float acc[kSteps][4];
@@ -274,48 +268,50 @@ __global__ void __launch_bounds__(kMmaThreads) decode_mma_kernel(const DecodePar
       uint32_t kbase = ring_s + s * L::kStageBytes;
       uint32_t vbase = kbase + L::kRingTileBytes;
       const int nv = min(kChunkTokens, u.t1 - (u.t0 + k * kChunkTokens));
+      // ---- scores: S^T = K · Qᵀ ----
+      float sc[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t vw[kFp8 ? D / 32 : 1][4];  // e4m3 V words: tokens 2tq, 2tq+1, 2tq+8, 2tq+9
       if constexpr (kFp8) {
-        // widen the e4m3 chunk (rows of 128 B, 128-byte swizzle) into the
-        // 16-bit staging layout, then hand the ring stage back at once; plain
-        // shared-memory accesses so all eight loads are in flight together
-        const unsigned char* ksrc = smem + (kbase - ring_s);
-        const unsigned char* vsrc = smem + (vbase - ring_s);
-        unsigned char* dst = smem + (staging - ring_s);
-        uint4 rk[4], rv[4];
-        uint32_t d0[4], d1[4];
+        // e4m3 rows are 128 B (one swizzle row): token r, 16-byte chunk c at
+        // position c ^ (r % 8).  Every code the warp needs is loaded as 32-bit
+        // words (bank-conflict free), then the ring stage goes back to the
+        // producer before any arithmetic.
+        uint32_t kw[kSteps][2];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int i = lane + 32 * j, row = i >> 3, c = i & 7;  // 16 codes: dims 16c .. 16c+15
-          const int src = row * 128 + ((c ^ (row & 7)) << 4);
-          rk[j] = *reinterpret_cast<const uint4*>(ksrc + src);
-          rv[j] = *reinterpret_cast<const uint4*>(vsrc + src);
-          const uint32_t base = row_offset(row, c >> 2, 4, kHalves);
-          d0[j] = base + ((((c & 3) << 1) ^ (row & 7)) << 4);
-          d1[j] = base + (((((c & 3) << 1) + 1) ^ (row & 7)) << 4);
+        for (int ks = 0; ks < kSteps; ++ks) {
+          const uint32_t a = kbase + gq * 128 + ((ks ^ gq) << 4) + 4 * tq;  // token gq; gq + 8 has the same swizzle
+          asm volatile("ld.shared.b32 %0, [%1];" : "=r"(kw[ks][0]) : "r"(a));
+          asm volatile("ld.shared.b32 %0, [%1];" : "=r"(kw[ks][1]) : "r"(a + 8 * 128));
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint4 lo, hi;
-          widen_e4m3x16(rk[j], lo, hi);
-          *reinterpret_cast<uint4*>(dst + d0[j]) = lo;
-          *reinterpret_cast<uint4*>(dst + d1[j]) = hi;
-          widen_e4m3x16(rv[j], lo, hi);
-          *reinterpret_cast<uint4*>(dst + L::kTileBytes + d0[j]) = lo;
-          *reinterpret_cast<uint4*>(dst + L::kTileBytes + d1[j]) = hi;
+        for (int pp = 0; pp < D / 32; ++pp) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int t = 2 * tq + (i & 1) + (i >> 1) * 8;
+            const uint32_t a = vbase + t * 128 + (((2 * pp + (gq >> 2)) ^ (t & 7)) << 4) + 4 * (gq & 3);
+            asm volatile("ld.shared.b32 %0, [%1];" : "=r"(vw[pp][i]) : "r"(a));
+          }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_addr(empty + s));
-        kbase = staging;
-        vbase = staging + L::kTileBytes;
-      }
-
-      // ---- scores: S^T = K · Qᵀ ----
-      float sc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int ks = 0; ks < kSteps; ++ks) {
-        uint32_t a[4];
-        ldmatrix_x4(kbase + offa[ks / 4] + (((2 * (ks % 4) + ca) ^ xa) << 4), a);
-        mma_16816<T>(sc, a, qb[ks][0], qb[ks][1]);
+        for (int ks = 0; ks < kSteps; ++ks) {
+          // contraction order within the step: K dims 16ks + 4tq + {0,1 | 2,3}
+          // stand at fragment columns {2tq, 2tq+1 | 2tq+8, 2tq+9}
+          uint32_t a[4];
+          a[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(kw[ks][0]));
+          a[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(kw[ks][0] >> 16));
+          a[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(kw[ks][1]));
+          a[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(kw[ks][1] >> 16));
+          mma_16816<T>(sc, a, qb[ks][0], qb[ks][1]);
+        }
+      } else {
+#pragma unroll
+        for (int ks = 0; ks < kSteps; ++ks) {
+          uint32_t a[4];
+          ldmatrix_x4(kbase + offa[ks / 4] + (((2 * (ks % 4) + ca) ^ xa) << 4), a);
+          mma_16816<T>(sc, a, qb[ks][0], qb[ks][1]);
+        }
       }
       const bool v0 = gq < nv, v1 = gq + 8 < nv;  // tokens gq and gq + 8 of the chunk
       const float s0 = v0 ? sc[0] * sl : -INFINITY, s1 = v0 ? sc[1] * sl : -INFINITY;
@@ -358,6 +354,34 @@ __global__ void __launch_bounds__(kMmaThreads) decode_mma_kernel(const DecodePar
       const uint32_t bl0 = __byte_perm(__shfl_sync(kFull, la, src0), __shfl_sync(kFull, la, src1), sel);
       const uint32_t bl1 = __byte_perm(__shfl_sync(kFull, lb, src0), __shfl_sync(kFull, lb, src1), sel);
 
+      if constexpr (kFp8) {
+        // ---- O^T += V^T · P^T from the e4m3 words.  Output dims are
+        // permuted within each 32-dim group: fragment row gq (+8) of m-tile
+        // 2pp + u is dim 32pp + 4gq + 2u (+1), so one word of a token row
+        // (4 consecutive dims) feeds both m-tiles of the pair.  Tokens past
+        // the sequence end read as zero codes. ----
+#pragma unroll
+        for (int pp = 0; pp < D / 32; ++pp) {
+          uint32_t w[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) w[i] = (2 * tq + (i & 1) + (i >> 1) * 8) < nv ? vw[pp][i] : 0u;
+          const uint32_t x01a = __byte_perm(w[0], w[1], 0x5140), x01b = __byte_perm(w[0], w[1], 0x7362);
+          const uint32_t x89a = __byte_perm(w[2], w[3], 0x5140), x89b = __byte_perm(w[2], w[3], 0x7362);
+          uint32_t a[4];
+          a[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(x01a));
+          a[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(x01a >> 16));
+          a[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(x89a));
+          a[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(x89a >> 16));
+          mma_16816<T>(acc[2 * pp], a, bh0, bh1);
+          mma_16816<T>(acc[2 * pp], a, bl0, bl1);
+          a[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(x01b));
+          a[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(x01b >> 16));
+          a[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(x89b));
+          a[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(x89b >> 16));
+          mma_16816<T>(acc[2 * pp + 1], a, bh0, bh1);
+          mma_16816<T>(acc[2 * pp + 1], a, bl0, bl1);
+        }
+      } else {
       // ---- rows past the sequence end: zero V so stale values cannot reach P·V ----
       if (nv < kChunkTokens) {
         const int per_row = 8 * kHalves;
@@ -378,12 +402,9 @@ __global__ void __launch_bounds__(kMmaThreads) decode_mma_kernel(const DecodePar
         mma_16816<T>(acc[mt], a, bh0, bh1);
         mma_16816<T>(acc[mt], a, bl0, bl1);
       }
-      if (!kFp8) {
-        if (nv < kChunkTokens) fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_addr(empty + s));
-      } else {
-        __syncwarp();  // the staging tile is rewritten by this warp's next chunk
+      if (nv < kChunkTokens) fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(empty + s));
       }
       s += kConsumerWarps;
       if (s >= NS) {
@@ -403,14 +424,16 @@ __global__ void __launch_bounds__(kMmaThreads) decode_mma_kernel(const DecodePar
     const int h0 = 2 * tq, h1 = 2 * tq + 1;
 #pragma unroll
     for (int mt = 0; mt < kSteps; ++mt) {
-      const int d = 16 * mt + gq;
+      // fragment rows gq and gq + 8 of m-tile mt: dims d and d + dd
+      const int d = kFp8 ? 32 * (mt >> 1) + 4 * gq + 2 * (mt & 1) : 16 * mt + gq;
+      const int dd = kFp8 ? 1 : 8;
       if (h0 < G) {
         mb[h0 * D + d] = acc[mt][0];
-        mb[h0 * D + d + 8] = acc[mt][2];
+        mb[h0 * D + d + dd] = acc[mt][2];
       }
       if (h1 < G) {
         mb[h1 * D + d] = acc[mt][1];
-        mb[h1 * D + d + 8] = acc[mt][3];
+        mb[h1 * D + d + dd] = acc[mt][3];
       }
     }
     if (gq == 0) {

@@ -869,7 +869,8 @@ extern "C" int pkv_paged_attention_prefill(const void* q, const void* k_pool, co
   const int32_t group = num_q_heads / num_kv_heads;
   if (group != 1 && group != 2 && group != 4 && group != 8)
     return fail(PKV_ERR_UNSUPPORTED, "%s: group size %d not supported (1, 2, 4 or 8)", fn, group);
-  if (!std::isfinite(scale)) return fail(PKV_ERR_INVALID_ARG, "%s: scale is not finite", fn);
+  if (!std::isfinite(scale) || !(scale > 0.f))
+    return fail(PKV_ERR_INVALID_ARG, "%s: scale must be positive and finite", fn);
   if (num_seqs == 0 || num_q_tokens == 0 || max_q_len == 0) return pkv::ok();
   if (!q || !k_pool || !v_pool || !block_tables || !seq_lens || !q_start || !out)
     return fail(PKV_ERR_INVALID_ARG, "%s: NULL pointer", fn);

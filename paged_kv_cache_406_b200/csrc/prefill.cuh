@@ -12,21 +12,28 @@
 // short chunks.  Keys come in chunks of 128 tokens (128/block_size physical
 // blocks, one TMA box per block and head_dim half).  Per chunk j:
 //
-//   S_j = Q · K_jᵀ        tcgen05.mma, 128x128x128, fp32 in tensor memory
-//   P_j = 2^(S_j·scale·log2e - m)   4 softmax warps, one row per thread
-//   O  += P_j · V_j       tcgen05.mma, P split into bf16 (or f16) hi + lo
+//   S_j = Q · K_jᵀ        tcgen05.mma, 128x128x128, A and B from shared memory,
+//                         fp32 in tensor memory
+//   P_j = 2^(S_j·scale·log2e - m)   4 softmax warps, one row per thread,
+//                         written back over S_j as bf16 (or f16) hi + lo
+//   O  += P_j · V_j       tcgen05.mma, A (P) from tensor memory, B (V) from
+//                         shared memory
 //
 // Warp roles (192 threads): warps 0-3 softmax (thread = row = TMEM lane),
 // warp 4 TMA producer, warp 5 MMA issuer (lane 0) and TMEM owner.  Tensor
-// memory (512 columns): S double buffer at columns 0 and 128, O at 256.
-// Shared memory: Q 32 KB, K and V rings of two 32 KB stages, P hi + lo 64 KB.
+// memory (512 columns): S / P double buffer at columns 0 and 128 (P hi in
+// the first 64 columns of its buffer, P lo in the next 64), O at 256.
+// Shared memory: Q 32 KB and K and V rings of 32 KB stages.  Keeping P in
+// tensor memory spares shared memory 128 KB of traffic per chunk (P written
+// and read back), which bounded the first version of this kernel.
 //
 // Pipeline: the MMA warp issues S_0, S_1, then per chunk PV_j followed by
 // S_{j+2}, so q·Kᵀ of the next chunks runs while the softmax warps work on
-// the current one; the softmax warps compute chunk j's exponentials while
-// PV_{j-1} is still running and only wait for it before overwriting P.
-// The running max moves lazily (only by more than 8 in log2 units), as in the
-// decode kernels; a move rescales that row's O in tensor memory.
+// the current one.  The commit of S_j covers every earlier MMA, so by the
+// time a softmax warp sees S_j, PV_{j-2} (the last reader of that buffer)
+// is done and P_j can overwrite it at once.  The running max moves lazily
+// (only by more than 8 in log2 units), as in the decode kernels; a move
+// rescales that row's O in tensor memory after PV_{j-1} has finished.
 //
 // P precision: a single bf16 P misses the 2e-3 output tolerance at early
 // positions (few keys of comparable weight); hi + lo halves keep it within
@@ -52,8 +59,12 @@ struct PrefillParams {
   float* out;                   // [num_q_tokens, num_q_heads, 128]
   int32_t num_seqs, num_q_heads, num_kv_heads, num_blocks, max_blocks, block_size;
   int32_t num_q_tokens, max_q_len, n_tiles;
-  float scale_log2;  // scale · log2(e)
+  float scale_log2;  // scale · log2(e), positive
 };
+
+#ifndef PKV_PREFILL_STAGES
+#define PKV_PREFILL_STAGES 2
+#endif
 
 namespace pf {
 constexpr int kRows = 128;              // MMA M: query rows per tile
@@ -61,22 +72,22 @@ constexpr int kKeys = 128;              // keys per chunk (S columns, P·V contr
 constexpr int kHeadDim = 128;
 constexpr uint32_t kSlab = 128 * 128;   // 128 rows x 64 elements x 2 bytes
 constexpr uint32_t kTile = 2 * kSlab;   // 128 rows x head_dim 128
-constexpr int kStages = 2;
+constexpr int kStages = PKV_PREFILL_STAGES;  // K and V ring depth
 constexpr int kThreads = 192;
 constexpr int kProducerWarp = 4, kMmaWarp = 5;
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kTile;
 constexpr uint32_t kOffV = kOffK + kStages * kTile;
-constexpr uint32_t kOffP = kOffV + kStages * kTile;  // hi tile, then lo tile
-constexpr uint32_t kOffBar = kOffP + 2 * kTile;
+constexpr uint32_t kOffBar = kOffV + kStages * kTile;
 constexpr size_t kSmemBytes = kOffBar + 256 + 1024;  // barriers, flags; 1024 B alignment slack
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;
 constexpr float kRescale = 8.0f;
 constexpr unsigned kAll = 0xffffffffu;
 // mbarrier slots
-enum : int { kQFull = 0, kKFull = 1, kKEmpty = 3, kVFull = 5, kVEmpty = 7, kSFull = 9, kPFull = 11, kPVDone = 12,
-             kDrain = 13, kNumBars = 14 };
+enum : int { kQFull = 0, kKFull = 1, kKEmpty = kKFull + kStages, kVFull = kKEmpty + kStages,
+             kVEmpty = kVFull + kStages, kSFull = kVEmpty + kStages, kPFull = kSFull + 2, kPVDone = kPFull + 1,
+             kDrain = kPVDone + 1, kNumBars = kDrain + 1 };
 }  // namespace pf
 
 __device__ __forceinline__ void tma_load_3d_nohint(uint32_t dst, const void* tmap, int32_t x, int32_t y, int32_t z,
@@ -105,6 +116,22 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
+// P as two 16-bit halves, packed in pairs (x0 in the low half): hi + lo
+// carries about 16 significant bits.  bf16: hi is the truncated top half of
+// the fp32 value (a byte permute), lo the rounded remainder (exact in fp32).
+template <typename T>
+__device__ __forceinline__ void split_hi_lo(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  split_pack<T>(x0, x1, hi, lo);
+}
+
+template <>
+__device__ __forceinline__ void split_hi_lo<__nv_bfloat16>(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const uint32_t u0 = __float_as_uint(x0), u1 = __float_as_uint(x1);
+  hi = __byte_perm(u0, u1, 0x7632);
+  __nv_bfloat162 l = __floats2bfloat162_rn(x0 - __uint_as_float(u0 & 0xffff0000u), x1 - __uint_as_float(u1 & 0xffff0000u));
+  lo = *reinterpret_cast<uint32_t*>(&l);
+}
+
 template <typename T, int G>
 __global__ void __launch_bounds__(pf::kThreads, 1)
     prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_q,
@@ -113,12 +140,13 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
   constexpr int QT = pf::kRows / G;  // query tokens per tile
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
 
-  // ---- the tile: (sequence b, KV head g, tile of QT query tokens); the
-  // tiles with the most keys (highest index) are launched first ----
-  const int per_tile = p.num_seqs * p.num_kv_heads;
-  const int tile = p.n_tiles - 1 - static_cast<int>(blockIdx.x) / per_tile;
-  const int rest = static_cast<int>(blockIdx.x) % per_tile;
-  const int b = rest / p.num_kv_heads, g = rest % p.num_kv_heads;
+  // ---- the tile: (sequence b, KV head g, tile of QT query tokens).  The
+  // tiles of one (b, g) are launched next to each other, most keys first, so
+  // the CTAs in flight at any time share a few sequences' K/V in L2 (launching
+  // one tile index of every (b, g) together re-read K/V from DRAM about 7x) ----
+  const int bg = static_cast<int>(blockIdx.x) / p.n_tiles;
+  const int tile = p.n_tiles - 1 - static_cast<int>(blockIdx.x) % p.n_tiles;
+  const int b = bg / p.num_kv_heads, g = bg % p.num_kv_heads;
   const int q0 = p.q_start[b], q1 = p.q_start[b + 1];
   const int n = q1 - q0, L = p.seq_lens[b];
   if (n < 0 || q0 < 0 || q1 > p.num_q_tokens || n > L || n > p.max_q_len ||
@@ -175,8 +203,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     const uint32_t box_bytes = static_cast<uint32_t>(BS) * 128;  // one block, one head_dim half
     int issued[2] = {0, 0};  // chunks whose K (V) fill was issued
     for (int j = 0; j < nc && ok; ++j) {
-      const int s = j & 1;
-      const uint32_t ph = ((j >> 1) & 1) ^ 1;
+      const int s = j % pf::kStages;
+      const uint32_t ph = ((j / pf::kStages) & 1) ^ 1;
       const int jb = j * nbc;
       const int nload = min(nbc, nblk - jb);  // blocks past the sequence end are not read
       int phys = 0;
@@ -213,8 +241,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       drain_wait(bar(pf::kQFull), 0);
       for (int kv = 0; kv < 2; ++kv) {
         for (int s = 0; s < pf::kStages && s < issued[kv]; ++s) {
-          const int last = issued[kv] - 1 - ((issued[kv] - 1 - s) & 1);  // last chunk that used stage s
-          drain_wait(bar((kv ? pf::kVFull : pf::kKFull) + s), (last >> 1) & 1);
+          const int last = s + (issued[kv] - 1 - s) / pf::kStages * pf::kStages;  // last chunk that used stage s
+          drain_wait(bar((kv ? pf::kVFull : pf::kKFull) + s), (last / pf::kStages) & 1);
         }
       }
     }
@@ -225,37 +253,38 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       const uint32_t id_s = tc::idesc_f16(kBf16, false, pf::kRows, pf::kKeys);
       const uint32_t id_o = tc::idesc_f16(kBf16, true, pf::kRows, pf::kHeadDim);
       auto issue_s = [&](int j) -> bool {
-        const int s = j & 1;
-        if (!mbar_wait(bar(pf::kKFull + s), (j >> 1) & 1, abort_flag)) return false;
+        const int s = j % pf::kStages;
+        if (!mbar_wait(bar(pf::kKFull + s), (j / pf::kStages) & 1, abort_flag)) return false;
         tc::fence_after_sync();
         const uint32_t kst = base + pf::kOffK + s * pf::kTile;
 #pragma unroll
         for (int kk = 0; kk < pf::kHeadDim / 16; ++kk) {
           const uint32_t off = (kk >> 2) * pf::kSlab + (kk & 3) * 32;
-          tc::mma_f16_ss(tmem + pf::kColS + s * pf::kKeys, tc::sw128_desc(base + pf::kOffQ + off, 16, 1024),
+          tc::mma_f16_ss(tmem + pf::kColS + (j & 1) * pf::kKeys, tc::sw128_desc(base + pf::kOffQ + off, 16, 1024),
                          tc::sw128_desc(kst + off, 16, 1024), id_s, kk > 0 ? 1u : 0u);
         }
         tc::commit(bar(pf::kKEmpty + s));
-        tc::commit(bar(pf::kSFull + s));
+        tc::commit(bar(pf::kSFull + (j & 1)));
         return true;
       };
       bool ok = mbar_wait(bar(pf::kQFull), 0, abort_flag);
       if (ok) ok = issue_s(0);
       if (ok && nc > 1) ok = issue_s(1);
       for (int j = 0; j < nc && ok; ++j) {
-        const int s = j & 1;
-        ok = mbar_wait(bar(pf::kPFull), j & 1, abort_flag) && mbar_wait(bar(pf::kVFull + s), (j >> 1) & 1, abort_flag);
+        const int s = j % pf::kStages;
+        ok = mbar_wait(bar(pf::kPFull), j & 1, abort_flag) &&
+             mbar_wait(bar(pf::kVFull + s), (j / pf::kStages) & 1, abort_flag);
         if (!ok) break;
         tc::fence_after_sync();
         const uint32_t vst = base + pf::kOffV + s * pf::kTile;
+        const uint32_t pt = tmem + pf::kColS + (j & 1) * pf::kKeys;  // P hi: 64 columns, then P lo
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
 #pragma unroll
           for (int kk = 0; kk < pf::kKeys / 16; ++kk) {
-            const uint32_t a = base + pf::kOffP + part * pf::kTile + (kk >> 2) * pf::kSlab + (kk & 3) * 32;
             const uint32_t bv = vst + kk * 16 * 128;  // 16 keys of 128-byte rows
-            tc::mma_f16_ss(tmem + pf::kColO, tc::sw128_desc(a, 16, 1024), tc::sw128_desc(bv, pf::kSlab, 1024), id_o,
-                           (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
+            tc::mma_f16_ts(tmem + pf::kColO, pt + part * (pf::kKeys / 2) + kk * 8, tc::sw128_desc(bv, pf::kSlab, 1024),
+                           id_o, (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
           }
         }
         tc::commit(bar(pf::kVEmpty + s));
@@ -278,35 +307,41 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     const bool valid = tok < n;
     const int pos = min(ctx + tok, L - 1);  // rows past the chunk end compute a copy of the last row
     const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const uint32_t p_row = base + pf::kOffP + r * 128;
     unsigned char* vzero = smem + pf::kOffV;
     const float sl = p.scale_log2;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nc && ok; ++j) {
-      const int s = j & 1;
-      ok = __all_sync(pf::kAll, mbar_wait(bar(pf::kSFull + s), (j >> 1) & 1, abort_flag));
+      const int sb = j & 1;              // S / P buffer
+      const int s = j % pf::kStages;     // K / V stage
+      ok = __all_sync(pf::kAll, mbar_wait(bar(pf::kSFull + sb), (j >> 1) & 1, abort_flag));
       if (!ok) break;
       tc::fence_after_sync();
-      float x[pf::kKeys];
+      float x[pf::kKeys];  // raw scores q·k of this row's 128 keys
       {
         uint32_t raw[4][32];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) tc::ld_32x32b_x32(trow + pf::kColS + s * pf::kKeys + 32 * q, raw[q]);
+        for (int q = 0; q < 4; ++q) tc::ld_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + 32 * q, raw[q]);
         tc::wait_ld();
 #pragma unroll
         for (int q = 0; q < 4; ++q)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) x[32 * q + i] = __uint_as_float(raw[q][i]) * sl;
+          for (int i = 0; i < 32; ++i) x[32 * q + i] = __uint_as_float(raw[q][i]);
       }
       const int key0 = j * pf::kKeys;
       if (key0 + pf::kKeys - 1 > pos_min) {  // the diagonal: keys after a row's position are hidden
 #pragma unroll
         for (int c = 0; c < pf::kKeys; ++c) x[c] = key0 + c <= pos ? x[c] : -INFINITY;
       }
-      float mc = x[0];
+      // row max in eight independent chains; the scale is positive, so the
+      // max of the scaled scores is the scaled max
+      float mx[8];
 #pragma unroll
-      for (int c = 1; c < pf::kKeys; ++c) mc = fmaxf(mc, x[c]);
+      for (int i = 0; i < 8; ++i) mx[i] = x[i];
+#pragma unroll
+      for (int c = 8; c < pf::kKeys; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+      const float mc = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl;
       float factor = 1.f;
       bool resc = false;
       if (j == 0) {
@@ -316,36 +351,37 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         m_used = mc;
         resc = true;
       }
-      float sum = 0.f;
+      float sm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const float neg_m = -m_used;
 #pragma unroll
       for (int c = 0; c < pf::kKeys; ++c) {
-        x[c] = fast_exp2(x[c] - m_used);
-        sum += x[c];
+        x[c] = fast_exp2(fmaf(x[c], sl, neg_m));  // hidden keys: exp2(-inf) = 0
+        sm[c & 7] += x[c];
       }
-      l = l * factor + sum;
+      l = l * factor + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
 
-      if (j > 0) {
-        // P_{j-1} and O are still being read by P·V of the previous chunk
+      if (__any_sync(pf::kAll, resc)) {
+        // O still accumulates PV_{j-1}: wait for it, then rescale the row.
+        // (S_j's commit already covered PV_{j-2}, so this parity wait cannot
+        // see an older phase.)
         ok = __all_sync(pf::kAll, mbar_wait(bar(pf::kPVDone), (j - 1) & 1, abort_flag));
         if (!ok) break;
         tc::fence_after_sync();
-        if (__any_sync(pf::kAll, resc)) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t o[32];
-            tc::ld_32x32b_x32(trow + pf::kColO + 32 * q, o);
-            tc::wait_ld();
+        for (int q = 0; q < 4; ++q) {
+          uint32_t o[32];
+          tc::ld_32x32b_x32(trow + pf::kColO + 32 * q, o);
+          tc::wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
-            tc::st_32x32b_x32(trow + pf::kColO + 32 * q, o);
-          }
-          tc::wait_st();
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
+          tc::st_32x32b_x32(trow + pf::kColO + 32 * q, o);
         }
       }
-      if (key0 + pf::kKeys > L) {
+      const bool zero_v = key0 + pf::kKeys > L;
+      if (zero_v) {
         // V rows past the sequence end hold stale or unwritten bytes: zero
         // them so that P = 0 there cannot meet a NaN pattern
-        ok = __all_sync(pf::kAll, mbar_wait(bar(pf::kVFull + s), (j >> 1) & 1, abort_flag));
+        ok = __all_sync(pf::kAll, mbar_wait(bar(pf::kVFull + s), (j / pf::kStages) & 1, abort_flag));
         if (!ok) break;
         const int v0 = L - key0;
         unsigned char* vst = vzero + s * pf::kTile;
@@ -354,33 +390,24 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
           *reinterpret_cast<uint4*>(vst + (piece >> 3) * pf::kSlab + row * 128 + (piece & 7) * 16) =
               make_uint4(0u, 0u, 0u, 0u);
         }
+        fence_proxy_async_smem();  // zeroed V rows visible to the tensor core
       }
-      // P hi and lo into the 128-byte-swizzled K-major layout (row r, keys in
-      // two slabs of 64, 16-byte chunk c at position c ^ (r % 8))
+      // P hi and lo over S_j in tensor memory: this row's lane, key pair
+      // (2c, 2c+1) in column c (hi) and column 64 + c (lo)
 #pragma unroll
-      for (int slab = 0; slab < 2; ++slab) {
+      for (int h = 0; h < 2; ++h) {
+        uint32_t hi[32], lo[32];
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint32_t hi[4], lo[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = slab * 64 + ch * 8 + 2 * e;
-            split_pack<T>(x[c], x[c + 1], hi[e], lo[e]);
-          }
-          const uint32_t off = slab * pf::kSlab + ((ch ^ (r & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(p_row + off), "r"(hi[0]), "r"(hi[1]),
-                       "r"(hi[2]), "r"(hi[3])
-                       : "memory");
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(p_row + pf::kTile + off), "r"(lo[0]),
-                       "r"(lo[1]), "r"(lo[2]), "r"(lo[3])
-                       : "memory");
-        }
+        for (int c = 0; c < 32; ++c) split_hi_lo<T>(x[64 * h + 2 * c], x[64 * h + 2 * c + 1], hi[c], lo[c]);
+        tc::st_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + 32 * h, hi);
+        tc::st_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + pf::kKeys / 2 + 32 * h, lo);
       }
-      fence_proxy_async_smem();  // P (and zeroed V rows) visible to the tensor core
+      tc::wait_st();
       tc::fence_before_sync();
       mbar_arrive(bar(pf::kPFull));
     }
-    if (ok) ok = __all_sync(pf::kAll, mbar_wait(bar(pf::kPVDone), (nc - 1) & 1, abort_flag));
+    // the MMA warp commits kDrain after its last MMA: every P·V is then done
+    if (ok) ok = __all_sync(pf::kAll, mbar_wait(bar(pf::kDrain), 0, abort_flag));
     if (ok) {
       tc::fence_after_sync();
       const float inv = 1.f / l;

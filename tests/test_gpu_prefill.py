@@ -198,6 +198,11 @@ def test_unsupported_arguments_are_refused():
         pkv.pkv_paged_attention_prefill(torch.zeros((1, 1, 64), dtype=torch.bfloat16, device=dev), k64, k64,
                                         tables, lens, qs, 1, 1.0)
     assert e.value.code == -4
+    for bad in (0.0, -0.5, float("nan")):  # the softmax takes the max of unscaled scores: scale > 0
+        with pytest.raises(pkv.PagedKVError) as e:
+            pkv.pkv_paged_attention_prefill(torch.zeros((1, 1, D), dtype=torch.bfloat16, device=dev), kp, kp,
+                                            tables, lens, qs, 1, bad)
+        assert e.value.code == -1
     with pytest.raises(pkv.PagedKVError) as e:  # group size 3
         pkv.pkv_paged_attention_prefill(torch.zeros((1, 3, D), dtype=torch.bfloat16, device=dev), kp, kp, tables,
                                         lens, qs, 1, 1.0)
