@@ -38,13 +38,15 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_SUSTAINED = 1400.0  # TFLOP/s, dense bf16 under the power cap
 STAGED_STEPS = 16  # distinct steps of metadata resident on the device, cycled
 
-# DRAM traffic of one pkv_paged_attention_decode call on the default workload,
-# from the ncu capture summarised in profiles/ (dram__bytes_read.sum +
-# dram__bytes_write.sum over its plan, decode and merge kernels, mean of two
-# captured calls).  Valid only while the decode sources hash to
-# TRAFFIC_SOURCE_SHA (kernel_source_sha()); otherwise reported as null.
-TRAFFIC_BYTES = 606448512
-TRAFFIC_SOURCE_SHA = "679a323a3900964d"
+# DRAM traffic of one pkv_paged_attention_decode call per workload, from the
+# ncu captures summarised in profiles/ (dram__bytes_read.sum +
+# dram__bytes_write.sum over the plan, decode and merge kernels, mean of two
+# captured calls), with the hash of the decode sources they were taken on
+# (kernel_source_sha()).  A pin whose hash no longer matches is reported as null.
+TRAFFIC = {
+    "llama3_8b": (606395136, "d322101e9d2d9b5d"),
+    "llama3_8b_fp8": (307405568, "d322101e9d2d9b5d"),
+}
 
 
 SEQ_LEN_RECIPES = {
@@ -396,7 +398,8 @@ def run_ours(args):
     dec_avg_ms = float(np.mean(dec_ms))
     achieved = float(np.mean(step_algo)) / (dec_avg_ms * 1e-3) / 1e9
     sha = kernel_source_sha()
-    traffic = TRAFFIC_BYTES if (TRAFFIC_BYTES is not None and sha == TRAFFIC_SOURCE_SHA) else None
+    pin = TRAFFIC.get(w.name)
+    traffic = pin[0] if (pin is not None and sha == pin[1]) else None
 
     # ---- end to end through the public API, host buffers in and out ----
     e2e = None

@@ -259,7 +259,8 @@ int pkv_paged_attention_decode(const void* q, const void* k_pool, const void* v_
  * block_tables / seq_lens as for decode; out: float32[num_q_tokens][num_q_heads][128]
  * (rows outside every chunk are not written).  dtype PKV_BF16 or PKV_F16,
  * head_dim 128, G in {1, 2, 4, 8}, block_size 8, 16 or 32; others return
- * PKV_ERR_UNSUPPORTED.  q, pools and out 16-byte aligned.
+ * PKV_ERR_UNSUPPORTED.  q, pools and out 16-byte aligned; scale positive
+ * and finite (else PKV_ERR_INVALID_ARG).
  * Computed on the tcgen05 tensor cores with fp32 accumulation; P enters the
  * P·V product as two 16-bit halves (hi + lo), so the result stays within
  * about 1e-5 of the exact softmax.  A sequence whose chunk is longer than
