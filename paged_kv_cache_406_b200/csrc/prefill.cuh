@@ -12,8 +12,8 @@
 // short chunks.  Keys come in chunks of 128 tokens (128/block_size physical
 // blocks, one TMA box per block and head_dim half).  Per chunk j:
 //
-//   S_j = Q · K_jᵀ        tcgen05.mma, 128x128x128, A (Q) from tensor memory,
-//                         B (K) from shared memory, fp32 in tensor memory
+//   S_j = Q · K_jᵀ        tcgen05.mma, 128x128x128, A and B from shared memory,
+//                         fp32 in tensor memory
 //   P_j = 2^(S_j·scale·log2e - m)   4 softmax warps, one row per thread,
 //                         written back over S_j as bf16 (or f16) hi + lo
 //   O  += P_j · V_j       tcgen05.mma, A (P) from tensor memory, B (V) from
@@ -22,20 +22,18 @@
 // Warp roles (224 threads): warps 0-3 softmax (thread = row = TMEM lane),
 // warps 4 and 5 TMA producers (K, V), warp 6 MMA issuer (lane 0) and TMEM
 // owner.  Tensor
-// memory (512 columns): S / P double buffer at columns 0 and 128 (P hi in
-// the first 64 columns of its buffer, P lo in the next 64), O at 256, Q at
-// 384 (copied once per tile from the TMA-loaded shared-memory tile: with
-// both operands in shared memory, q·Kᵀ issued at about 180 cycles per MMA
-// against 80 for P·V).
+// memory (512 columns): three S / P buffers at columns 0, 128 and 256 (P hi
+// in the first 64 columns of its buffer, P lo in the next 64), O at 384.
 // Shared memory: Q 32 KB and K and V rings of 32 KB stages.  Keeping P in
 // tensor memory spares shared memory 128 KB of traffic per chunk (P written
 // and read back), which bounded the first version of this kernel.
 //
-// Pipeline: the MMA warp issues S_0, S_1, then per chunk PV_j followed by
-// S_{j+2}, so q·Kᵀ of the next chunks runs while the softmax warps work on
-// the current one.  The commit of S_j covers every earlier MMA, so by the
-// time a softmax warp sees S_j, PV_{j-2} (the last reader of that buffer)
-// is done and P_j can overwrite it at once.  The running max moves lazily
+// Pipeline: the MMA warp issues S_0, S_1, S_2, then per chunk PV_j followed
+// by S_{j+3}, so q·Kᵀ of the next chunks runs while the softmax warps work
+// on the current one and the tensor core has the next chunk's P·V ready
+// while waiting for this one's P.  The commit of S_j covers every earlier
+// MMA, so by the time a softmax warp sees S_j, PV_{j-3} (the last reader of
+// that buffer) is done and P_j can overwrite it at once.  The running max moves lazily
 // (only by more than 8 in log2 units), as in the decode kernels; a move
 // rescales that row's O in tensor memory after PV_{j-1} has finished.
 //
@@ -85,13 +83,17 @@ constexpr uint32_t kOffV = kOffK + kStages * kTile;
 constexpr uint32_t kOffBar = kOffV + kStages * kTile;
 constexpr size_t kSmemBytes = kOffBar + 256 + 1024;  // barriers, flags; 1024 B alignment slack
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColO = 256, kColQ = 384;  // Q: 64 columns (128 bf16 per row)
+constexpr int kSBufs = 3;                    // S / P buffers in tensor memory
+constexpr uint32_t kColS = 0, kColO = 384;   // S / P: 3 x 128 columns, O: 128
 constexpr float kRescale = 8.0f;
 constexpr unsigned kAll = 0xffffffffu;
 // mbarrier slots
 enum : int { kQFull = 0, kKFull = 1, kKEmpty = kKFull + kStages, kVFull = kKEmpty + kStages,
-             kVEmpty = kVFull + kStages, kSFull = kVEmpty + kStages, kPFull = kSFull + 2, kPVDone = kPFull + 1,
-             kDrain = kPVDone + 1, kQTmem = kDrain + 1, kNumBars = kQTmem + 1 };
+             kVEmpty = kVFull + kStages, kSFull = kVEmpty + kStages, kPFull = kSFull + kSBufs,
+             kPVDone = kPFull + kSBufs, kDrain = kPVDone + kSBufs, kNumBars = kDrain + 1 };
+// S-full, P-full and PV-done are one barrier per S / P buffer: a buffer's
+// next phase needs the MMA warp to have moved on (S_{j+3} is issued after
+// PV_j), so no waiter can ever be a whole phase behind
 }  // namespace pf
 
 __device__ __forceinline__ void tma_load_3d_nohint(uint32_t dst, const void* tmap, int32_t x, int32_t y, int32_t z,
@@ -112,6 +114,27 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, int3
       : "memory");
 }
 
+// Waits for the phase of `bar` with the given parity, like mbar_wait, but
+// lets the hardware suspend the thread until the phase completes (up to
+// 20 us per try) instead of re-polling: the producer and MMA warps share
+// their SM sub-partitions with softmax warps, whose issue slots a spinning
+// wait would take.  Gives up once *abort is set or after kWaitLimitNs.
+__device__ __forceinline__ bool pf_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity), "r"(20000u)
+        : "memory");
+    if (done) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
 // Waits (bounded by time only) for a phase; used to drain copies and MMAs in
 // flight before the CTA exits or frees tensor memory.
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
@@ -130,11 +153,47 @@ __device__ __forceinline__ void split_hi_lo(float x0, float x1, uint32_t& hi, ui
 
 template <>
 __device__ __forceinline__ void split_hi_lo<__nv_bfloat16>(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  // hi: the top 16 bits of each fp32 value; lo: the top 16 bits of the
+  // (exact) remainder.  Both truncations are byte permutes on the integer
+  // pipe, which keeps the special-function pipe (busy with the
+  // exponentials) free of conversions; hi + lo is within 2^-16 of x.
   const uint32_t u0 = __float_as_uint(x0), u1 = __float_as_uint(x1);
   hi = __byte_perm(u0, u1, 0x7632);
-  __nv_bfloat162 l = __floats2bfloat162_rn(x0 - __uint_as_float(u0 & 0xffff0000u), x1 - __uint_as_float(u1 & 0xffff0000u));
-  lo = *reinterpret_cast<uint32_t*>(&l);
+  // x - trunc(x), both lanes in one packed FMA (exact: the remainder fits)
+  const float2 r = __ffma2_rn(make_float2(__uint_as_float(u0 & 0xffff0000u), __uint_as_float(u1 & 0xffff0000u)),
+                              make_float2(-1.f, -1.f), make_float2(x0, x1));
+  lo = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
 }
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x on the FMA pipe, for x <= 64 (returns +0 for x <= -127): Cody-Waite
+// reduction x = n + f with n the nearest integer (the 1.5·2^23 rounding trick)
+// and f in [-1/2, 1/2], then 2^f = e^(f ln 2) by its Taylor series to degree 5
+// (truncation error below 2.5e-6 relative), scaled by 2^n through the
+// exponent field.  Takes a share of the softmax exponentials off the
+// special-function pipe.
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -127.f);
+  const float t = x + 12582912.f;
+  const float f = x - (t - 12582912.f);
+  float p = 1.3333558146428443e-3f;           // ln2^5 / 5!
+  p = fmaf(p, f, 9.6181291076284772e-3f);     // ln2^4 / 4!
+  p = fmaf(p, f, 5.5504108664821580e-2f);     // ln2^3 / 3!
+  p = fmaf(p, f, 2.4022650695910071e-1f);     // ln2^2 / 2!
+  p = fmaf(p, f, 6.9314718055994531e-1f);     // ln2
+  p = fmaf(p, f, 1.f);
+  const int n = __float_as_int(t) - 0x4B400000;
+  return __int_as_float(__float_as_int(p) + (n << 23));
+}
+
+#ifndef PKV_PREFILL_POLY_EVERY
+#define PKV_PREFILL_POLY_EVERY 0  // one softmax exponential in this many on the FMA pipe (0: none)
+#endif
 
 template <typename T, int G>
 __global__ void __launch_bounds__(pf::kThreads, 1)
@@ -177,7 +236,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < pf::kNumBars; ++i) mbar_init(bar(i), (i == pf::kPFull || i == pf::kQTmem) ? 128u : 1u);
+    for (int i = 0; i < pf::kNumBars; ++i) mbar_init(bar(i), (i >= pf::kPFull && i < pf::kPFull + pf::kSBufs) ? 128u : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -229,7 +288,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       }
       const int32_t y = (phys * p.num_kv_heads + g) * BS;
       const uint32_t full = full0 + 8 * s;
-      ok = __all_sync(pf::kAll, mbar_wait(empty0 + 8 * s, ph, abort_flag));
+      ok = __all_sync(pf::kAll, pf_wait(empty0 + 8 * s, ph, abort_flag));
       if (!ok) break;
       if (lane == 0) mbar_arrive_expect_tx(full, static_cast<uint32_t>(nload) * 2u * box_bytes);
       __syncwarp();
@@ -261,30 +320,30 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       const uint32_t id_o = tc::idesc_f16(kBf16, true, pf::kRows, pf::kHeadDim);
       auto issue_s = [&](int j) -> bool {
         const int s = j % pf::kStages;
-        if (!mbar_wait(bar(pf::kKFull + s), (j / pf::kStages) & 1, abort_flag)) return false;
+        if (!pf_wait(bar(pf::kKFull + s), (j / pf::kStages) & 1, abort_flag)) return false;
         tc::fence_after_sync();
         const uint32_t kst = base + pf::kOffK + s * pf::kTile;
 #pragma unroll
         for (int kk = 0; kk < pf::kHeadDim / 16; ++kk) {
           const uint32_t off = (kk >> 2) * pf::kSlab + (kk & 3) * 32;
-          tc::mma_f16_ts(tmem + pf::kColS + (j & 1) * pf::kKeys, tmem + pf::kColQ + kk * 8,
-                         tc::sw128_desc(kst + off, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+          tc::mma_f16_ss(tmem + pf::kColS + (j % pf::kSBufs) * pf::kKeys,
+                         tc::sw128_desc(base + pf::kOffQ + off, 16, 1024), tc::sw128_desc(kst + off, 16, 1024), id_s,
+                         kk > 0 ? 1u : 0u);
         }
         tc::commit(bar(pf::kKEmpty + s));
-        tc::commit(bar(pf::kSFull + (j & 1)));
+        tc::commit(bar(pf::kSFull + j % pf::kSBufs));
         return true;
       };
-      bool ok = mbar_wait(bar(pf::kQTmem), 0, abort_flag);  // Q copied into tensor memory
-      if (ok) ok = issue_s(0);
-      if (ok && nc > 1) ok = issue_s(1);
+      bool ok = pf_wait(bar(pf::kQFull), 0, abort_flag);
+      for (int j = 0; j < pf::kSBufs && j < nc && ok; ++j) ok = issue_s(j);
       for (int j = 0; j < nc && ok; ++j) {
         const int s = j % pf::kStages;
-        ok = mbar_wait(bar(pf::kPFull), j & 1, abort_flag) &&
-             mbar_wait(bar(pf::kVFull + s), (j / pf::kStages) & 1, abort_flag);
+        ok = pf_wait(bar(pf::kPFull + j % pf::kSBufs), (j / pf::kSBufs) & 1, abort_flag) &&
+             pf_wait(bar(pf::kVFull + s), (j / pf::kStages) & 1, abort_flag);
         if (!ok) break;
         tc::fence_after_sync();
         const uint32_t vst = base + pf::kOffV + s * pf::kTile;
-        const uint32_t pt = tmem + pf::kColS + (j & 1) * pf::kKeys;  // P hi: 64 columns, then P lo
+        const uint32_t pt = tmem + pf::kColS + (j % pf::kSBufs) * pf::kKeys;  // P hi: 64 columns, then P lo
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
 #pragma unroll
@@ -295,8 +354,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
           }
         }
         tc::commit(bar(pf::kVEmpty + s));
-        tc::commit(bar(pf::kPVDone));
-        if (j + 2 < nc) ok = issue_s(j + 2);
+        tc::commit(bar(pf::kPVDone + j % pf::kSBufs));
+        if (j + pf::kSBufs < nc) ok = issue_s(j + pf::kSBufs);
       }
       if (!ok) {
         record_error(PKV_ERR_DEVICE_TIMEOUT);
@@ -317,33 +376,11 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     unsigned char* vzero = smem + pf::kOffV;
     const float sl = p.scale_log2;
     float m_used = -INFINITY, l = 0.f;
-    // Q is the A operand of every S MMA of this tile: copy this row once from
-    // the TMA-written shared-memory tile (128-byte swizzle) into tensor
-    // memory, dims (2c, 2c+1) in column kColQ + c
-    bool ok = __all_sync(pf::kAll, mbar_wait(bar(pf::kQFull), 0, abort_flag));
-    if (ok) {
-      const unsigned char* qs = smem + pf::kOffQ + r * 128;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t w[32];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 v = *reinterpret_cast<const uint4*>(qs + h * pf::kSlab + ((c ^ (r & 7)) << 4));
-          w[4 * c] = v.x;
-          w[4 * c + 1] = v.y;
-          w[4 * c + 2] = v.z;
-          w[4 * c + 3] = v.w;
-        }
-        tc::st_32x32b_x32(trow + pf::kColQ + 32 * h, w);
-      }
-      tc::wait_st();
-      tc::fence_before_sync();
-      mbar_arrive(bar(pf::kQTmem));
-    }
+    bool ok = true;
     for (int j = 0; j < nc && ok; ++j) {
-      const int sb = j & 1;              // S / P buffer
+      const int sb = j % pf::kSBufs;     // S / P buffer
       const int s = j % pf::kStages;     // K / V stage
-      ok = __all_sync(pf::kAll, mbar_wait(bar(pf::kSFull + sb), (j >> 1) & 1, abort_flag));
+      ok = __all_sync(pf::kAll, pf_wait(bar(pf::kSFull + sb), (j / pf::kSBufs) & 1, abort_flag));
       if (!ok) break;
       tc::fence_after_sync();
       float x[pf::kKeys];  // raw scores q·k of this row's 128 keys
@@ -362,15 +399,19 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
 #pragma unroll
         for (int c = 0; c < pf::kKeys; ++c) x[c] = key0 + c <= pos ? x[c] : -INFINITY;
       }
-      // row max in eight independent chains; the scale is positive, so the
-      // max of the scaled scores is the scaled max
-      float mx[8];
+      // row max with three-input maxima in four independent chains; the
+      // scale is positive, so the max of the scaled scores is the scaled max
+      float mx[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = x[i];
-#pragma unroll
-      for (int c = 8; c < pf::kKeys; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
-      const float mc = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl;
+      for (int c = 4; c + 8 <= pf::kKeys; c += 8) {
+        mx[0] = max3f(mx[0], x[c], x[c + 1]);
+        mx[1] = max3f(mx[1], x[c + 2], x[c + 3]);
+        mx[2] = max3f(mx[2], x[c + 4], x[c + 5]);
+        mx[3] = max3f(mx[3], x[c + 6], x[c + 7]);
+      }
+      mx[0] = max3f(mx[0], x[pf::kKeys - 4], x[pf::kKeys - 3]);
+      mx[1] = max3f(mx[1], x[pf::kKeys - 2], x[pf::kKeys - 1]);
+      const float mc = fmaxf(max3f(mx[0], mx[1], mx[2]), mx[3]) * sl;
       float factor = 1.f;
       bool resc = false;
       if (j == 0) {
@@ -380,20 +421,28 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         m_used = mc;
         resc = true;
       }
-      float sm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      const float neg_m = -m_used;
+      // exponentials: arguments and sums two lanes at a time (packed f32x2)
+      float2 sm[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(-m_used, -m_used);
 #pragma unroll
-      for (int c = 0; c < pf::kKeys; ++c) {
-        x[c] = fast_exp2(fmaf(x[c], sl, neg_m));  // hidden keys: exp2(-inf) = 0
-        sm[c & 7] += x[c];
+      for (int c = 0; c < pf::kKeys; c += 2) {
+        const float2 a = __ffma2_rn(make_float2(x[c], x[c + 1]), sl2, nm2);  // hidden keys: -inf -> 0
+        constexpr int kEvery = PKV_PREFILL_POLY_EVERY > 0 ? PKV_PREFILL_POLY_EVERY : 1;
+        x[c] = (PKV_PREFILL_POLY_EVERY > 0 && c % kEvery == kEvery - 1) ? exp2_fma(a.x) : fast_exp2(a.x);
+        x[c + 1] = fast_exp2(a.y);
+        sm[(c >> 1) & 3] = __fadd2_rn(sm[(c >> 1) & 3], make_float2(x[c], x[c + 1]));
       }
-      l = l * factor + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
+      const float2 s01 = __fadd2_rn(sm[0], sm[1]), s23 = __fadd2_rn(sm[2], sm[3]);
+      const float2 st = __fadd2_rn(s01, s23);
+      l = l * factor + (st.x + st.y);
 
       if (__any_sync(pf::kAll, resc)) {
         // O still accumulates PV_{j-1}: wait for it, then rescale the row.
-        // (S_j's commit already covered PV_{j-2}, so this parity wait cannot
-        // see an older phase.)
-        ok = __all_sync(pf::kAll, mbar_wait(bar(pf::kPVDone), (j - 1) & 1, abort_flag));
+        // PV_{j-1} commits to the barrier of its buffer, whose previous
+        // phase (PV_{j-4}) was covered by S_j's commit, so the parity wait
+        // cannot see an older phase.
+        const int pj = j - 1;
+        ok = __all_sync(pf::kAll, pf_wait(bar(pf::kPVDone + pj % pf::kSBufs), (pj / pf::kSBufs) & 1, abort_flag));
         if (!ok) break;
         tc::fence_after_sync();
 #pragma unroll
@@ -410,7 +459,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       if (zero_v) {
         // V rows past the sequence end hold stale or unwritten bytes: zero
         // them so that P = 0 there cannot meet a NaN pattern
-        ok = __all_sync(pf::kAll, mbar_wait(bar(pf::kVFull + s), (j / pf::kStages) & 1, abort_flag));
+        ok = __all_sync(pf::kAll, pf_wait(bar(pf::kVFull + s), (j / pf::kStages) & 1, abort_flag));
         if (!ok) break;
         const int v0 = L - key0;
         unsigned char* vst = vzero + s * pf::kTile;
@@ -433,10 +482,10 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       }
       tc::wait_st();
       tc::fence_before_sync();
-      mbar_arrive(bar(pf::kPFull));
+      mbar_arrive(bar(pf::kPFull + sb));
     }
     // the MMA warp commits kDrain after its last MMA: every P·V is then done
-    if (ok) ok = __all_sync(pf::kAll, mbar_wait(bar(pf::kDrain), 0, abort_flag));
+    if (ok) ok = __all_sync(pf::kAll, pf_wait(bar(pf::kDrain), 0, abort_flag));
     if (ok) {
       tc::fence_after_sync();
       const float inv = 1.f / l;
