@@ -410,13 +410,15 @@ def run_ours(args):
             host_in.append(tuple(W.normal(shape, w.io_dtype, W.step_seed(w, 100 + s, k)).pin_memory()
                                  for k, shape in ((0, (B, hq, d)), (1, (B, hkv, d)), (2, (B, hkv, d)))))
         out_host = torch.empty((B, hq, d), dtype=torch.float32, pin_memory=True)
+        ids_np = np.arange(B, dtype=np.int64)
         for s in range(3):  # warm-up
             qh, kh, vh = host_in[s % len(host_in)]
-            o = cache.decode_step(ids, qh, kh, vh, w.scale, partition_tokens=w.partition_tokens)
-            out_host.copy_(o, non_blocking=True)
+            cache.decode_step_host(ids_np, qh, kh, vh, w.scale, out_host=out_host,
+                                   partition_tokens=w.partition_tokens)
         torch.cuda.synchronize()
-        e_lens = []
-        meta_bytes = 0
+        # lengths after the warm-up: each timed step adds one token per sequence
+        base_tokens = sum(cache.alloc.seq_len(i) for i in range(B))
+        meta_bytes = int(P.lib().pkv_step_meta_bytes(B, cache.max_blocks))
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if ws > 1:
             dist.barrier()
@@ -424,20 +426,20 @@ def run_ours(args):
         e0.record()
         for s in range(E):
             qh, kh, vh = host_in[s % len(host_in)]
-            o = cache.decode_step(ids, qh, kh, vh, w.scale, partition_tokens=w.partition_tokens)
-            out_host.copy_(o, non_blocking=True)
-            e_lens.append(kv_bytes(cache._meta_np[B:2 * B]))
-            meta_bytes += B * (4 + cache.max_blocks) * 4
+            cache.decode_step_host(ids_np, qh, kh, vh, w.scale, out_host=out_host,
+                                   partition_tokens=w.partition_tokens)
         e1.record()
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
-        e2e_ms_all, e2e_bytes_all, _ = combine_ranks(e2e_ms, float(sum(e_lens)), float(B * E), dev)
-        h2d = (B * hq * d + 2 * B * hkv * d) * qsz + meta_bytes // E
+        e_bytes = sum((base_tokens + B * (s + 1)) * hkv * d * 2 * esz for s in range(E))
+        e2e_ms_all, e2e_bytes_all, _ = combine_ranks(e2e_ms, float(e_bytes), float(B * E), dev)
+        h2d = (B * hq * d + 2 * B * hkv * d) * qsz + meta_bytes
         e2e = {"value": round(e2e_bytes_all / (e2e_ms_all * 1e-3) / 1e9, 2), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(B * hq * d * 4),
                "ms_per_step": round(e2e_ms_all / E, 4),
                "tokens_per_s_per_layer": round(ws * B * E / (e2e_ms_all * 1e-3), 1),
-               "includes": "host slot reservation, pinned H2D of q/K/V rows and metadata, kernels, D2H of out"}
+               "includes": "one pkv_decode_step_host call per step: host slot reservation, pinned H2D of q/K/V rows and "
+                           "metadata, kernels, D2H of out"}
 
     st_a = cache.stats()
     alloc_stats = {"used_blocks": st_a["used_blocks"], "free_blocks": st_a["free_blocks"],

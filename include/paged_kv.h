@@ -241,6 +241,62 @@ int pkv_paged_attention_decode(const void* q, const void* k_pool, const void* v_
                                int32_t partition_tokens, void* workspace, size_t workspace_bytes,
                                float* out, void* stream);
 
+/* One whole decode step from host buffers in a single call (vLLM paging page
+ * §3: phase 1 reservation, phase 3 copy-on-write, phase 2 attention), for
+ * serving loops that want one crossing of the library boundary per step:
+ *   1. wait for buf->wait_event (if not NULL) - the copy that last read
+ *      buf->meta_host is done;
+ *   2. pkv_seq_append_slots + pkv_block_tables for seq_ids into
+ *      buf->meta_host, laid out as int32 slots[n] | seq_lens[n] | cow[2n] |
+ *      tables[n][max_blocks_per_seq] (pkv_step_meta_bytes(n, max_blocks));
+ *   3. host-to-device copies (cudaMemcpyAsync on `stream`) of that metadata
+ *      to buf->meta_dev and of the new rows q_host [n][Hq][D],
+ *      k_host / v_host [n][Hkv][D] to q_dev / k_dev / v_dev (element type:
+ *      dtype, or float16 for e4m3 pools); then record buf->done_event (if
+ *      not NULL);
+ *   4. pkv_copy_blocks for the copy-on-write pairs, pkv_kv_append (or
+ *      pkv_kv_append_fp8) and pkv_paged_attention_decode (or _fp8) into
+ *      buf->out_dev [n][Hq][D] float32;
+ *   5. if buf->out_host is not NULL, copy out_dev to it (device to host).
+ * Every host buffer should be pinned for the copies to be asynchronous.
+ * k_scale / v_scale are used for e4m3 pools only.
+ * Overlap (optional): with h2d_stream set, the host-to-device copies run on
+ * it after it waits for compute_done (the previous kernels that read these
+ * device buffers), and `stream` waits for done_event before the kernels; with
+ * d2h_stream set, `stream` records compute_done after the kernels, the copy
+ * back runs on d2h_stream after it, and d2h_done is recorded there (the
+ * next use of out_dev waits for it).  Alternating two buffer sets then lets
+ * the copies of neighbouring steps run under this step's kernels.   Errors: those of the
+ * calls above; argument errors leave the allocator unchanged, but once the
+ * slots are reserved (step 2) a later device error leaves them reserved. */
+typedef struct pkv_step_buffers {
+  void* meta_host;
+  void* meta_dev;
+  const void* q_host;
+  const void* k_host;
+  const void* v_host;
+  void* q_dev;
+  void* k_dev;
+  void* v_dev;
+  float* out_dev;
+  float* out_host;
+  void* wait_event;
+  void* done_event;
+  void* h2d_stream;   /* cudaStream_t or NULL */
+  void* d2h_stream;   /* cudaStream_t or NULL */
+  void* compute_done; /* cudaEvent_t; needed with either stream */
+  void* d2h_done;     /* cudaEvent_t; needed with d2h_stream */
+} pkv_step_buffers_t;
+
+size_t pkv_step_meta_bytes(int32_t n, int32_t max_blocks_per_seq);
+
+int pkv_decode_step_host(pkv_alloc_t* a, const int64_t* seq_ids, int32_t n, const pkv_step_buffers_t* buf,
+                         void* k_pool, void* v_pool, int32_t num_blocks, int32_t num_q_heads,
+                         int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                         int32_t max_blocks_per_seq, float scale, int32_t dtype, float k_scale,
+                         float v_scale, int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
 /* Paged prefill attention (chunked prefill: vLLM production page §2;
  * optimisation-overview page §2.3): sequence b brings
  * n_b = q_start[b+1] - q_start[b] new query rows, stored at rows

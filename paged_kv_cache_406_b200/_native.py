@@ -63,9 +63,19 @@ SIGNATURES = {
                                          _vp]),
     "pkv_paged_attention_decode_fp8": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                                                       _i32, _f32, _f32, _f32, _i32, _vp, _sz, _vp, _vp]),
+    "pkv_step_meta_bytes": (ctypes.c_size_t, [_i32, _i32]),
+    "pkv_decode_step_host": (ctypes.c_int, [_vp, _pi64, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32,
+                                            _i32, _f32, _f32, _i32, _vp, _sz, _vp]),
     "pkv_paged_attention_prefill": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                                                    _i32, _i32, _i32, _f32, _i32, _vp, _vp]),
 }
+
+
+class StepBuffers(ctypes.Structure):
+    """pkv_step_buffers_t: the host and device buffers of one pkv_decode_step_host call."""
+    _fields_ = [(name, ctypes.c_void_p) for name in (
+        "meta_host", "meta_dev", "q_host", "k_host", "v_host", "q_dev", "k_dev", "v_dev", "out_dev", "out_host",
+        "wait_event", "done_event", "h2d_stream", "d2h_stream", "compute_done", "d2h_done")]
 
 
 class PagedKVError(RuntimeError):

@@ -22,7 +22,7 @@ import numpy as np
 import torch
 
 from . import binding as B
-from ._native import check, lib
+from ._native import StepBuffers, check, lib
 
 
 class PagedKVCache:
@@ -143,6 +143,76 @@ class PagedKVCache:
         B.pkv_kv_append(k_new, v_new, slots, self.k_pool, self.v_pool)
         return B.pkv_paged_attention_decode(q, self.k_pool, self.v_pool, tables, lens, scale, out=out,
                                             workspace=ws, partition_tokens=partition_tokens)
+
+    # -- the decode step in one library call -------------------------------
+    def decode_step_host(self, seq_ids: np.ndarray, q_host: torch.Tensor, k_host: torch.Tensor,
+                         v_host: torch.Tensor, scale: float, out_host: Optional[torch.Tensor] = None,
+                         partition_tokens: int = 0, overlap: bool = True) -> torch.Tensor:
+        """The decode step of :meth:`decode_step` as one pkv_decode_step_host
+        call: slot reservation, metadata and row copies from host memory,
+        copy-on-write, append, attention and (with ``out_host``) the copy of
+        the result back to the host.  ``seq_ids``: int64 numpy array;
+        ``q_host`` [n, Hq, D], ``k_host`` / ``v_host`` [n, Hkv, D] pinned host
+        tensors (float16 for e4m3 pools, else the pool dtype).  Two metadata
+        staging buffers alternate, so a step only waits for the copy two steps
+        back before overwriting one.  Returns the device output (valid until
+        the next step) or ``out_host``.  With ``overlap`` the host-to-device
+        and device-to-host copies run on two copy streams of this cache, so
+        they proceed under the neighbouring steps' kernels (two sets of device
+        buffers alternate); ``out_host`` is then complete once the current
+        stream and the copy streams have been synchronised."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = int(ids.size)
+        hq = q_host.shape[1]
+        self._ensure_step(n, hq)
+        k = self._step_k
+        self._step_k ^= 1
+        ws, _ = self._buffers(n, hq, partition_tokens)
+        b = self._step_bufs[k]
+        out = self._step_out[k]
+        b.q_host, b.k_host, b.v_host = q_host.data_ptr(), k_host.data_ptr(), v_host.data_ptr()
+        b.out_host = out_host.data_ptr() if out_host is not None else None
+        b.h2d_stream = self._h2d_stream.cuda_stream if overlap else None
+        b.d2h_stream = self._d2h_stream.cuda_stream if overlap else None
+        check(lib().pkv_decode_step_host(
+            self.alloc._h, ids.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n, ctypes.byref(b),
+            self.k_pool.data_ptr(), self.v_pool.data_ptr(), self.num_blocks, hq, self.num_kv_heads, self.head_dim,
+            self.block_size, self.max_blocks, float(scale), B._dtype_code(self.k_pool), self.k_scale, self.v_scale,
+            int(partition_tokens), ws.data_ptr(), ws.numel(), torch.cuda.current_stream(self.device).cuda_stream))
+        return out_host if out_host is not None else out
+
+    def _ensure_step(self, n: int, hq: int) -> None:
+        key = (n, hq)
+        if getattr(self, "_step_key", None) == key:
+            return
+        nbytes = int(lib().pkv_step_meta_bytes(n, self.max_blocks))
+        io = torch.float16 if self.fp8 else self.dtype
+        self._step_hold = []
+        self._step_bufs = []
+        self._step_out = []
+        self._h2d_stream = torch.cuda.Stream(self.device)
+        self._d2h_stream = torch.cuda.Stream(self.device)
+        # per buffer set: copies in done (host may rewrite the staging), kernels
+        # done (the set's device buffers may be rewritten), copy back done
+        self._step_events = [[torch.cuda.Event() for _ in range(3)] for _ in range(2)]
+        for k in range(2):
+            mh = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+            md = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+            qd = torch.empty((n, hq, self.head_dim), dtype=io, device=self.device)
+            kd = torch.empty((n, self.num_kv_heads, self.head_dim), dtype=io, device=self.device)
+            vd = torch.empty_like(kd)
+            od = torch.empty((n, hq, self.head_dim), dtype=torch.float32, device=self.device)
+            self._step_hold += [mh, md, qd, kd, vd]
+            self._step_out.append(od)
+            for ev in self._step_events[k]:
+                ev.record()  # completed events: the first waits return at once
+            h2d, kern, d2h = (ev.cuda_event for ev in self._step_events[k])
+            b = StepBuffers(meta_host=mh.data_ptr(), meta_dev=md.data_ptr(), q_dev=qd.data_ptr(),
+                            k_dev=kd.data_ptr(), v_dev=vd.data_ptr(), out_dev=od.data_ptr(),
+                            wait_event=h2d, done_event=h2d, compute_done=kern, d2h_done=d2h)
+            self._step_bufs.append(b)
+        self._step_k = 0
+        self._step_key = key
 
     def stats(self) -> dict:
         return self.alloc.stats()

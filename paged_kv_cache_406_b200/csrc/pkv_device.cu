@@ -903,3 +903,100 @@ extern "C" int pkv_paged_attention_prefill(const void* q, const void* k_pool, co
   if (dtype == PKV_BF16) return dispatch_prefill<__nv_bfloat16>(group, p, q, k_pool, v_pool, dtype, s);
   return dispatch_prefill<__half>(group, p, q, k_pool, v_pool, dtype, s);
 }
+
+// =============================================================================
+// A whole decode step from host buffers
+// =============================================================================
+extern "C" size_t pkv_step_meta_bytes(int32_t n, int32_t max_blocks_per_seq) {
+  if (n <= 0 || max_blocks_per_seq < 0) return 0;
+  return size_t(n) * (4 + size_t(max_blocks_per_seq)) * sizeof(int32_t);
+}
+
+extern "C" int pkv_decode_step_host(pkv_alloc_t* a, const int64_t* seq_ids, int32_t n, const pkv_step_buffers_t* buf,
+                                    void* k_pool, void* v_pool, int32_t num_blocks, int32_t num_q_heads,
+                                    int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                    int32_t max_blocks_per_seq, float scale, int32_t dtype, float k_scale,
+                                    float v_scale, int32_t partition_tokens, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  const char* fn = "pkv_decode_step_host";
+  if (!a || !buf || n < 0 || max_blocks_per_seq <= 0 || num_kv_heads <= 0 || num_q_heads <= 0 || head_dim <= 0)
+    return fail(PKV_ERR_INVALID_ARG, "%s: bad arguments", fn);
+  if (n == 0) return pkv::ok();
+  if (!seq_ids || !buf->meta_host || !buf->meta_dev || !buf->q_host || !buf->k_host || !buf->v_host ||
+      !buf->q_dev || !buf->k_dev || !buf->v_dev || !buf->out_dev)
+    return fail(PKV_ERR_INVALID_ARG, "%s: NULL buffer", fn);
+  if ((buf->h2d_stream && (!buf->done_event || !buf->compute_done)) ||
+      (buf->d2h_stream && (!buf->compute_done || !buf->d2h_done)))
+    return fail(PKV_ERR_INVALID_ARG, "%s: a copy stream needs its events", fn);
+  const bool fp8 = dtype == PKV_FP8_E4M3;
+  if (!fp8 && dtype != PKV_F32 && dtype != PKV_BF16 && dtype != PKV_F16)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: dtype %d not supported", fn, dtype);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (buf->wait_event) {
+    e = cudaEventSynchronize(static_cast<cudaEvent_t>(buf->wait_event));
+    if (e != cudaSuccess) return cuda_fail(e, "pkv_decode_step_host: cudaEventSynchronize");
+  }
+  int32_t* m = static_cast<int32_t*>(buf->meta_host);
+  int32_t* slots = m;
+  int32_t* lens = m + n;
+  int32_t* cow = m + 2 * n;
+  int32_t* tables = m + 4 * n;
+  int32_t ncow = 0;
+  int rc = pkv_seq_append_slots(a, seq_ids, n, slots, cow, n, &ncow);
+  if (rc) return rc;
+  rc = pkv_block_tables(a, seq_ids, n, max_blocks_per_seq, tables, lens);
+  if (rc) return rc;
+  const size_t io = fp8 ? 2 : elem_size(dtype);  // bytes per element of q and of the new rows
+  const size_t qb = size_t(n) * num_q_heads * head_dim * io, kb = size_t(n) * num_kv_heads * head_dim * io;
+  cudaStream_t hs = buf->h2d_stream ? static_cast<cudaStream_t>(buf->h2d_stream) : s;
+  cudaEvent_t compute_done = static_cast<cudaEvent_t>(buf->compute_done);
+  e = cudaSuccess;
+  if (buf->h2d_stream) e = cudaStreamWaitEvent(hs, compute_done, 0);  // the device buffers' last readers are done
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(buf->meta_dev, buf->meta_host, pkv_step_meta_bytes(n, max_blocks_per_seq),
+                        cudaMemcpyHostToDevice, hs);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(buf->q_dev, buf->q_host, qb, cudaMemcpyHostToDevice, hs);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(buf->k_dev, buf->k_host, kb, cudaMemcpyHostToDevice, hs);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(buf->v_dev, buf->v_host, kb, cudaMemcpyHostToDevice, hs);
+  if (e == cudaSuccess && buf->done_event) e = cudaEventRecord(static_cast<cudaEvent_t>(buf->done_event), hs);
+  if (e == cudaSuccess && buf->h2d_stream) e = cudaStreamWaitEvent(s, static_cast<cudaEvent_t>(buf->done_event), 0);
+  if (e == cudaSuccess && buf->d2h_stream) e = cudaStreamWaitEvent(s, static_cast<cudaEvent_t>(buf->d2h_done), 0);
+  if (e != cudaSuccess) return cuda_fail(e, "pkv_decode_step_host: host-to-device copies");
+  const int32_t* md = static_cast<const int32_t*>(buf->meta_dev);
+  if (ncow) {
+    rc = pkv_copy_blocks(k_pool, v_pool, md + 2 * n, ncow, num_blocks, num_kv_heads, head_dim, block_size, dtype,
+                         stream);
+    if (rc) return rc;
+  }
+  if (fp8) {
+    rc = pkv_kv_append_fp8(buf->k_dev, buf->v_dev, PKV_F16, md, n, k_pool, v_pool, num_blocks, num_kv_heads,
+                           head_dim, block_size, k_scale, v_scale, stream);
+    if (rc) return rc;
+    rc = pkv_paged_attention_decode_fp8(buf->q_dev, k_pool, v_pool, md + 4 * n, md + n, n, num_q_heads, num_kv_heads,
+                                        head_dim, num_blocks, max_blocks_per_seq, block_size, scale, k_scale, v_scale,
+                                        partition_tokens, workspace, workspace_bytes, buf->out_dev, stream);
+  } else {
+    rc = pkv_kv_append(buf->k_dev, buf->v_dev, md, n, k_pool, v_pool, num_blocks, num_kv_heads, head_dim, block_size,
+                       dtype, stream);
+    if (rc) return rc;
+    rc = pkv_paged_attention_decode(buf->q_dev, k_pool, v_pool, md + 4 * n, md + n, n, num_q_heads, num_kv_heads,
+                                    head_dim, num_blocks, max_blocks_per_seq, block_size, scale, dtype,
+                                    partition_tokens, workspace, workspace_bytes, buf->out_dev, stream);
+  }
+  if (rc) return rc;
+  if (buf->h2d_stream || buf->d2h_stream) {
+    e = cudaEventRecord(compute_done, s);
+    if (e != cudaSuccess) return cuda_fail(e, "pkv_decode_step_host: cudaEventRecord");
+  }
+  if (buf->out_host) {
+    cudaStream_t ds = buf->d2h_stream ? static_cast<cudaStream_t>(buf->d2h_stream) : s;
+    e = buf->d2h_stream ? cudaStreamWaitEvent(ds, compute_done, 0) : cudaSuccess;
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(buf->out_host, buf->out_dev, size_t(n) * num_q_heads * head_dim * sizeof(float),
+                          cudaMemcpyDeviceToHost, ds);
+    if (e == cudaSuccess && buf->d2h_stream) e = cudaEventRecord(static_cast<cudaEvent_t>(buf->d2h_done), ds);
+    if (e != cudaSuccess) return cuda_fail(e, "pkv_decode_step_host: device-to-host copy");
+  }
+  return pkv::ok();
+}

@@ -421,16 +421,27 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         m_used = mc;
         resc = true;
       }
-      // exponentials: arguments and sums two lanes at a time (packed f32x2)
+      // exponentials (arguments and sums two lanes at a time, packed f32x2),
+      // each half of the row written as P hi and lo over S_j in tensor memory
+      // as soon as it is done (the stores complete while the next half is
+      // computed): key pair (2c, 2c+1) in column c (hi) and 64 + c (lo)
       float2 sm[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(-m_used, -m_used);
 #pragma unroll
-      for (int c = 0; c < pf::kKeys; c += 2) {
-        const float2 a = __ffma2_rn(make_float2(x[c], x[c + 1]), sl2, nm2);  // hidden keys: -inf -> 0
-        constexpr int kEvery = PKV_PREFILL_POLY_EVERY > 0 ? PKV_PREFILL_POLY_EVERY : 1;
-        x[c] = (PKV_PREFILL_POLY_EVERY > 0 && c % kEvery == kEvery - 1) ? exp2_fma(a.x) : fast_exp2(a.x);
-        x[c + 1] = fast_exp2(a.y);
-        sm[(c >> 1) & 3] = __fadd2_rn(sm[(c >> 1) & 3], make_float2(x[c], x[c + 1]));
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int c = 64 * h; c < 64 * h + 64; c += 2) {
+          const float2 a = __ffma2_rn(make_float2(x[c], x[c + 1]), sl2, nm2);  // hidden keys: -inf -> 0
+          constexpr int kEvery = PKV_PREFILL_POLY_EVERY > 0 ? PKV_PREFILL_POLY_EVERY : 1;
+          x[c] = (PKV_PREFILL_POLY_EVERY > 0 && c % kEvery == kEvery - 1) ? exp2_fma(a.x) : fast_exp2(a.x);
+          x[c + 1] = fast_exp2(a.y);
+          sm[(c >> 1) & 3] = __fadd2_rn(sm[(c >> 1) & 3], make_float2(x[c], x[c + 1]));
+        }
+        uint32_t hi[32], lo[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) split_hi_lo<T>(x[64 * h + 2 * c], x[64 * h + 2 * c + 1], hi[c], lo[c]);
+        tc::st_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + 32 * h, hi);
+        tc::st_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + pf::kKeys / 2 + 32 * h, lo);
       }
       const float2 s01 = __fadd2_rn(sm[0], sm[1]), s23 = __fadd2_rn(sm[2], sm[3]);
       const float2 st = __fadd2_rn(s01, s23);
@@ -469,16 +480,6 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
               make_uint4(0u, 0u, 0u, 0u);
         }
         fence_proxy_async_smem();  // zeroed V rows visible to the tensor core
-      }
-      // P hi and lo over S_j in tensor memory: this row's lane, key pair
-      // (2c, 2c+1) in column c (hi) and column 64 + c (lo)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t hi[32], lo[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) split_hi_lo<T>(x[64 * h + 2 * c], x[64 * h + 2 * c + 1], hi[c], lo[c]);
-        tc::st_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + 32 * h, hi);
-        tc::st_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + pf::kKeys / 2 + 32 * h, lo);
       }
       tc::wait_st();
       tc::fence_before_sync();

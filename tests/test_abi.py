@@ -110,3 +110,29 @@ def test_copy_blocks_rejects_bad_arguments_before_launch(native):
     assert native.pkv_copy_blocks(FAKE, FAKE, FAKE, 2, 8, 8, 128, 16, 5, None) == N.PKV_ERR_UNSUPPORTED
     assert native.pkv_copy_blocks(FAKE + 4, FAKE, FAKE, 2, 8, 8, 128, 16, N.PKV_F16, None) == N.PKV_ERR_INVALID_ARG
     assert native.pkv_copy_blocks(FAKE, FAKE, 0, 2, 8, 8, 128, 16, N.PKV_F16, None) == N.PKV_ERR_INVALID_ARG
+
+
+def test_step_meta_bytes_and_step_argument_checks(native):
+    """pkv_step_meta_bytes is the documented layout (slots, lengths, copy
+    pairs, tables: n * (4 + max_blocks) int32); the one-call step refuses bad
+    arguments before it touches the allocator or the GPU."""
+    assert native.pkv_step_meta_bytes(64, 256) == 64 * (4 + 256) * 4
+    assert native.pkv_step_meta_bytes(0, 256) == 0 and native.pkv_step_meta_bytes(-1, 8) == 0
+    buf = N.StepBuffers()
+    assert native.pkv_decode_step_host(None, None, 1, ctypes.byref(buf), FAKE, FAKE, 8, 32, 8, 128, 16, 4, 0.1,
+                                       N.PKV_BF16, 1.0, 1.0, 0, FAKE, 0, None) == N.PKV_ERR_INVALID_ARG
+    a = ctypes.c_void_p()
+    assert native.pkv_alloc_create(16, 16, None, ctypes.byref(a)) == 0
+    ids = (ctypes.c_int64 * 1)(0)
+    try:
+        # a NULL staging buffer: refused, and nothing reserved
+        assert native.pkv_seq_add(a, 0, 5) == 0
+        rc = native.pkv_decode_step_host(a, ids, 1, ctypes.byref(buf), FAKE, FAKE, 16, 32, 8, 128, 16, 4, 0.1,
+                                         N.PKV_BF16, 1.0, 1.0, 0, FAKE, 0, None)
+        assert rc == N.PKV_ERR_INVALID_ARG
+        n = ctypes.c_int32()
+        assert native.pkv_seq_len(a, 0, ctypes.byref(n)) == 0 and n.value == 5
+        assert native.pkv_decode_step_host(a, ids, 0, ctypes.byref(buf), FAKE, FAKE, 16, 32, 8, 128, 16, 4, 0.1,
+                                           N.PKV_BF16, 1.0, 1.0, 0, FAKE, 0, None) == 0
+    finally:
+        native.pkv_alloc_destroy(a)

@@ -207,3 +207,41 @@ def test_unsupported_arguments_are_refused():
         pkv.pkv_paged_attention_prefill(torch.zeros((1, 3, D), dtype=torch.bfloat16, device=dev), kp, kp, tables,
                                         lens, qs, 1, 1.0)
     assert e.value.code == -4
+
+
+def test_full_size_chunked_prefill_sampled_rows():
+    """The measured chunked-prefill batch (16 sequences, 512-row chunks behind
+    U[0, 3584] cached tokens, 32 / 8 heads, bf16, block size 16), launched as
+    the bench launches it; 48 sampled (row, head) outputs against the oracle,
+    each as the one-row chunk at its position."""
+    from paged_kv_cache_406_b200 import workloads as W
+    w = W.WORKLOADS["prefill_llama3_8b"]
+    dev = "cuda"
+    B, hq, hkv, d, bs, n = w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, w.chunk_tokens
+    ctx = W.seq_lens(w)
+    L = ctx + n
+    nb = W.pool_blocks(w, L)
+    kp = W.pool_values((nb, hkv, bs, d), w, 0, device=dev)
+    vp = W.pool_values((nb, hkv, bs, d), w, 1, device=dev)
+    alloc = pkv.Allocator(nb, bs, W.free_order(nb, w.seed))
+    for b in range(B):
+        alloc.add(b, int(L[b]))
+    maxb = -(-int(L.max()) // bs)
+    tables, lens = alloc.block_tables(list(range(B)), maxb)
+    q = W.normal((B * n, hq, d), w.torch_dtype, W.step_seed(w, 0, 0), device=dev)
+    out = pkv.pkv_paged_attention_prefill(q, kp, vp, torch.from_numpy(tables).to(dev), torch.from_numpy(lens).to(dev),
+                                          torch.arange(0, B * n + 1, n, dtype=torch.int32, device=dev), n, w.scale)
+    torch.cuda.synchronize()
+    kc, vc, qc = raw(kp), raw(vp), raw(q)
+    rng = np.random.default_rng(406)
+    G = hq // hkv
+    for _ in range(48):
+        b, i, h = int(rng.integers(B)), int(rng.integers(n)), int(rng.integers(hq))
+        pos = int(ctx[b]) + i
+        g = h // G
+        blocks = tables[b, :pos // bs + 1]
+        ref = pa.paged_prefill_attention(qc[b * n + i:b * n + i + 1, g * G:(g + 1) * G], kc[blocks][:, g:g + 1],
+                                         vc[blocks][:, g:g + 1], np.arange(len(blocks))[None], np.array([pos + 1]),
+                                         np.array([1]), w.scale, "bf16")
+        got = out[b * n + i, g * G:(g + 1) * G].unsqueeze(0)
+        assert_close(got, ref, "bf16", f"row {b}/{i} heads {g * G}..{g * G + G - 1}")
