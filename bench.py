@@ -47,6 +47,11 @@ TRAFFIC = {
     "llama3_8b": (606395136, "d322101e9d2d9b5d"),
     "llama3_8b_fp8": (307405568, "d322101e9d2d9b5d"),
 }
+# the same for one pkv_paged_attention_prefill call (prefill_tc_kernel), keyed
+# by the hash of the prefill sources (kernel_source_sha(PREFILL_SOURCES))
+TRAFFIC_PREFILL = {
+    "prefill_llama3_8b": (330831488, "af3a520664f50605"),
+}
 
 
 SEQ_LEN_RECIPES = {
@@ -593,6 +598,9 @@ def run_prefill(args, w0):
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_BF16_SUSTAINED))
     peak_kind = "measured bf16_tflops_sustained" if "bf16_tflops_sustained" in peaks else "fallback sustained"
     achieved = flops / (attn_ms * 1e-3) / 1e12
+    pf_sha = kernel_source_sha(PREFILL_SOURCES)
+    pin = TRAFFIC_PREFILL.get(w.name)
+    traffic = pin[0] if (pin is not None and pf_sha == pin[1]) else None
 
     # ---- end to end: host q / K / V rows and metadata in, out back to host ----
     e2e = None
@@ -674,10 +682,11 @@ def run_prefill(args, w0):
                          "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(achieved / peak, 4), "peak_source": peak_kind,
                          "burst_peak": peaks.get("bf16_tflops"),
-                         "traffic": None, "algorithmic_flops_per_launch": flops,
+                         "traffic": traffic, "traffic_unit": "bytes (DRAM read + write per launch)",
+                         "algorithmic_flops_per_launch": flops,
                          "tensor_flops_issued_per_launch": "1.5x algorithmic (P·V runs on P hi and P lo) plus the "
                                                           "masked part of diagonal chunks",
-                         "avg_launch_ms": round(attn_ms, 5), "kernel_source_sha": kernel_source_sha(PREFILL_SOURCES)},
+                         "avg_launch_ms": round(attn_ms, 5), "kernel_source_sha": pf_sha},
             "gpu_launches": launches, "clocks": clk, "cpu_baseline": cpu, "e2e": e2e,
         }
         print(json.dumps(res), flush=True)
