@@ -807,6 +807,62 @@ def run_adaptive(args, w):
         print(json.dumps(res), flush=True)
 
 
+def run_prefix_cache(args, w):
+    """Hash-based prefix caching in the host allocator (vLLM paging page §3
+    phase 3; production page §5: reuse saves memory, hashing costs CPU time).
+    Admits the workload's requests three ways - plain pkv_seq_add, and
+    pkv_seq_add_cached with shared system prompts and with all-distinct
+    prompts - and reports host time per admission, reuse and blocks held."""
+    import paged_kv_cache_406_b200 as P
+    from paged_kv_cache_406_b200 import workloads as W
+    rng = np.random.default_rng(w.seed)
+    suffix = W.seq_lens(w)
+    systems = [rng.integers(0, 32000, size=w.prefix_tokens, dtype=np.int32) for _ in range(4)]
+    prompts = [np.concatenate([systems[i % 4], rng.integers(0, 32000, size=int(suffix[i]), dtype=np.int32)])
+               for i in range(w.num_seqs)]
+    distinct = [rng.integers(0, 32000, size=len(p), dtype=np.int32) for p in prompts]
+    bs = w.block_size
+    nb = sum(-(-len(p) // bs) for p in prompts) + 16
+    reps = max(1, min(args.steps, 50))
+
+    def arm(kind, data):
+        times, stats = [], None
+        for _ in range(reps):
+            a = P.Allocator(nb, bs, W.free_order(nb, w.seed))
+            t0 = time.perf_counter()
+            if kind == "add":
+                for i, p in enumerate(data):
+                    a.add(i, len(p))
+            else:
+                for i, p in enumerate(data):
+                    a.add_cached(i, p)
+            times.append(time.perf_counter() - t0)
+            stats = a.stats()
+        us = float(np.median(times)) / len(data) * 1e6
+        return {"us_per_admission": round(us, 3), "used_blocks": stats["used_blocks"],
+                "cache_hits": stats["cache_hits"], "cache_queries": stats["cache_queries"],
+                "hit_rate": round(stats["cache_hits"] / max(1, stats["cache_queries"]), 4)}
+
+    res_arms = {"plain_add": arm("add", prompts), "cached_shared_prompts": arm("cached", prompts),
+                "cached_distinct_prompts": arm("cached", distinct)}
+    c, plain = res_arms["cached_shared_prompts"], res_arms["plain_add"]
+    res = {"metric": "prefix caching: host admission time per sequence, KV blocks held", "value": c["us_per_admission"],
+           "unit": "us/sequence", "n_gpus": 0, "steps": reps, "warmup": 0, "ms_per_step": None,
+           "higher_is_better": False, "scaling": None, "vs_baseline": None, "dtype": "int32 token ids",
+           "data": "synthetic",
+           "config": {"workload": w.name, "requests": w.num_seqs, "system_prompts": 4,
+                      "system_prompt_tokens": w.prefix_tokens, "suffix_tokens": "U[16,512]", "block_size": bs,
+                      "timing": "median over repetitions of admitting every request into a fresh allocator, "
+                                "through the Python binding (one ctypes call per request)"},
+           "blocks_saved": plain["used_blocks"] - c["used_blocks"],
+           "blocks_saved_frac": round(1 - c["used_blocks"] / plain["used_blocks"], 4),
+           "hashing_overhead_us": round(res_arms["cached_distinct_prompts"]["us_per_admission"] -
+                                        plain["us_per_admission"], 3),
+           "arms": res_arms, "gpu_launches": 0, "clocks": None, "cpu_baseline": None, "e2e": None,
+           "device": "host only: the C++ allocator (no kernel on this path)"}
+    print(json.dumps(res), flush=True)
+
+
 def run_reference(args):
     """The reference arm: the fp64 CPU oracle, on this arm's workload, each
     step a bounded sample of it (rank 0 only)."""
@@ -905,6 +961,9 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "prefix_cache":
+        from paged_kv_cache_406_b200 import workloads as W
+        run_prefix_cache(args, W.WORKLOADS["prefix_cache"])
     else:
         if not torch.cuda.is_available():
             raise SystemExit("bench.py needs a CUDA GPU (B200); use --impl reference for the CPU oracle")

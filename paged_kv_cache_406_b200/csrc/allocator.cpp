@@ -46,10 +46,12 @@ struct Undo {
 constexpr uint64_t kFnvBasis = 14695981039346656037ull;  // FNV-1a 64-bit offset basis
 constexpr uint64_t kFnvPrime = 1099511628211ull;
 
-uint64_t fnv1a(uint64_t h, const void* data, size_t n) {
-  const unsigned char* p = static_cast<const unsigned char*>(data);
+// FNV-1a over 32-bit token ids (one xor-multiply step per token rather than
+// per byte).  Identities are verified against the stored tokens, so the hash
+// only has to spread keys, not to be collision-free.
+uint64_t fnv1a(uint64_t h, const int32_t* tokens, size_t n) {
   for (size_t i = 0; i < n; ++i) {
-    h ^= p[i];
+    h ^= static_cast<uint32_t>(tokens[i]);
     h *= kFnvPrime;
   }
   return h;
@@ -201,14 +203,17 @@ extern "C" int pkv_seq_add_cached(pkv_alloc_t* a, int64_t seq_id, const int32_t*
     return fail(PKV_ERR_INVALID_ARG, "pkv_seq_add_cached: bad arguments");
   if (a->seqs.count(seq_id)) return fail(PKV_ERR_SEQ_EXISTS, "pkv_seq_add_cached: sequence %lld exists", (long long)seq_id);
   const int32_t bs = a->block_size;
-  if (a->block_tokens.empty()) a->block_tokens.assign(static_cast<size_t>(a->num_blocks) * bs, 0);
+  if (a->block_tokens.empty()) {  // first use of the prefix cache
+    a->block_tokens.assign(static_cast<size_t>(a->num_blocks) * bs, 0);
+    a->cache.reserve(static_cast<size_t>(a->num_blocks));
+  }
   const int32_t nfull = n_tokens / bs;
   const int32_t nblk = (n_tokens + bs - 1) / bs;
   // chain hashes of the full blocks; the leading run found in the cache
   std::vector<uint64_t> h(nfull);
   uint64_t prev = kFnvBasis;
   for (int32_t i = 0; i < nfull; ++i) {
-    h[i] = fnv1a(prev, tokens + static_cast<int64_t>(i) * bs, sizeof(int32_t) * bs);
+    h[i] = fnv1a(prev, tokens + static_cast<int64_t>(i) * bs, static_cast<size_t>(bs));
     prev = h[i];
   }
   std::vector<int32_t> hit_blocks;

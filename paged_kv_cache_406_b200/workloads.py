@@ -81,6 +81,9 @@ WORKLOADS = {
     # the optimisation-overview page's traffic mix for adaptive block sizes:
     # 80 % of 64 sequences below 1024 tokens, the rest 1024..8191, one >= 8192
     "adaptive_mix": Workload("adaptive_mix", 64, 32, 8, 128, 16, "bf16", 406008),
+    # prefix caching (host allocator): 256 requests, each one of 4 shared
+    # 1024-token system prompts plus its own U[16, 512]-token suffix
+    "prefix_cache": Workload("prefix_cache", 256, 32, 8, 128, 16, "bf16", 406009, prefix_tokens=1024),
     # whole 2048-token prompts from an empty cache, 8 sequences
     "prefill_prompt_2k": Workload("prefill_prompt_2k", 8, 32, 8, 128, 16, "bf16", 406007, chunk_tokens=2048),
 }
@@ -113,6 +116,8 @@ def seq_lens(w: Workload) -> np.ndarray:
         return np.concatenate([rng.integers(128, 1023, size=short, endpoint=True),
                                rng.integers(1024, 8191, size=long_, endpoint=True),
                                rng.integers(8192, 16384, size=n - short - long_, endpoint=True)]).astype(np.int64)
+    if w.name == "prefix_cache":  # suffix lengths (the shared prompt comes on top)
+        return rng.integers(16, 512, size=n, endpoint=True).astype(np.int64)
     if w.name.startswith("prefill_llama3_8b"):  # cached context before the chunk
         return rng.integers(0, 3584, size=n, endpoint=True).astype(np.int64)
     if w.name.startswith("prefill_prompt"):
