@@ -38,14 +38,15 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_SUSTAINED = 1400.0  # TFLOP/s, dense bf16 under the power cap
 STAGED_STEPS = 16  # distinct steps of metadata resident on the device, cycled
 
-# DRAM traffic of one pkv_paged_attention_decode call per workload, from the
-# ncu captures summarised in profiles/ (dram__bytes_read.sum +
-# dram__bytes_write.sum over the plan, decode and merge kernels, mean of two
-# captured calls), with the hash of the decode sources they were taken on
-# (kernel_source_sha()).  A pin whose hash no longer matches is reported as null.
+# DRAM traffic of one pkv_append_and_decode call per workload, from the ncu
+# captures summarised in profiles/ (dram__bytes_read.sum +
+# dram__bytes_write.sum over the append + plan, decode and merge kernels, mean
+# of two captured calls), with the hash of the decode sources they were taken
+# on (kernel_source_sha()).  A pin whose hash no longer matches is reported as
+# null.
 TRAFFIC = {
-    "llama3_8b": (606395136, "d322101e9d2d9b5d"),
-    "llama3_8b_fp8": (307405568, "d322101e9d2d9b5d"),
+    "llama3_8b": (606710016, "eb907b967a95bff5"),
+    "llama3_8b_fp8": (307467008, "eb907b967a95bff5"),
 }
 # the same for one pkv_paged_attention_prefill call (prefill_tc_kernel), keyed
 # by the hash of the prefill sources (kernel_source_sha(PREFILL_SOURCES))
@@ -65,7 +66,7 @@ SEQ_LEN_RECIPES = {
 }
 
 
-DECODE_SOURCES = ("decode.cuh", "decode_mma.cuh", "device_common.cuh")
+DECODE_SOURCES = ("append.cuh", "decode.cuh", "decode_mma.cuh", "device_common.cuh")
 PREFILL_SOURCES = ("prefill.cuh", "tcgen05.cuh", "device_common.cuh")
 
 
@@ -280,9 +281,10 @@ def setup(w, device, horizon):
 
 
 def decode_launches(max_blocks: int, block_size: int, partition_tokens: int) -> int:
-    """Kernels one pkv_paged_attention_decode call launches: the plan and
-    decode kernels, plus the partition merge when a sequence of the table's
-    capacity can span more than one partition."""
+    """Kernels one pkv_paged_attention_decode (or pkv_append_and_decode) call
+    launches: the plan (or append + plan) and decode kernels, plus the
+    partition merge when a sequence of the table's capacity can span more than
+    one partition."""
     pt = partition_tokens or 512
     return 2 + (1 if max_blocks * block_size > pt else 0)
 
@@ -334,10 +336,12 @@ def run_ours(args):
 
     def algo_bytes(lens):
         # K/V rows once per (sequence, KV head) + block-table entries + q + out,
-        # + the split-partition partials (m, l, o per query head), written once and read once
+        # + the split-partition partials (m, l, o per query head), written once and read once,
+        # + the new rows of the append (read as given, written as stored) and their slots
         tab = int(sum(-(-int(L) // bs) for L in lens)) * 4
         parts = int(sum(-(-int(L) // pt_eff) for L in lens if L > pt_eff))
-        return kv_bytes(lens) + tab + B * hq * d * qsz + B * hq * d * 4 + 2 * parts * hq * (d + 2) * 4
+        append = 2 * B * hkv * d * (qsz + esz) + B * 4
+        return kv_bytes(lens) + tab + B * hq * d * qsz + B * hq * d * 4 + 2 * parts * hq * (d + 2) * 4 + append
 
     launches_per = []
 
@@ -347,20 +351,18 @@ def run_ours(args):
         if st["ncow"]:
             P.pkv_copy_blocks(cache.k_pool, cache.v_pool, st["cow"])
             n += 1
-        if fp8:
-            P.pkv_kv_append_fp8(st["kn"], st["vn"], st["slots"], cache.k_pool, cache.v_pool, w.kv_scale, w.kv_scale)
-        else:
-            P.pkv_kv_append(st["kn"], st["vn"], st["slots"], cache.k_pool, cache.v_pool)
-        n += 1
         if ev is not None:
             ev[0].record()
+        # the append and the decode of the step in one call (the new rows are
+        # written by the launch that plans the decode)
         if fp8:
-            P.pkv_paged_attention_decode_fp8(st["q"], cache.k_pool, cache.v_pool, st["tables"], st["lens"], w.scale,
-                                             w.kv_scale, w.kv_scale, out=out, workspace=workspace,
-                                             partition_tokens=w.partition_tokens)
+            P.pkv_append_and_decode_fp8(st["kn"], st["vn"], st["slots"], st["q"], cache.k_pool, cache.v_pool,
+                                        st["tables"], st["lens"], w.scale, w.kv_scale, w.kv_scale, out=out,
+                                        workspace=workspace, partition_tokens=w.partition_tokens)
         else:
-            P.pkv_paged_attention_decode(st["q"], cache.k_pool, cache.v_pool, st["tables"], st["lens"], w.scale,
-                                         out=out, workspace=workspace, partition_tokens=w.partition_tokens)
+            P.pkv_append_and_decode(st["kn"], st["vn"], st["slots"], st["q"], cache.k_pool, cache.v_pool,
+                                    st["tables"], st["lens"], w.scale, out=out, workspace=workspace,
+                                    partition_tokens=w.partition_tokens)
         if ev is not None:
             ev[1].record()
         return n + decode_launches(cache.max_blocks, bs, w.partition_tokens)
@@ -480,7 +482,7 @@ def run_ours(args):
                        "l2": "inputs larger than L2: %.0f MB of K/V read per step vs 126 MB L2, no flush"
                              % (np.mean(step_kv) / 1e6),
                        "parallelism": f"replicas x{ws} (independent batches per GPU)"},
-            "roofline": {"kernel": "pkv_paged_attention_decode (plan + decode + partition-merge kernels)",
+            "roofline": {"kernel": "pkv_append_and_decode (append + plan, decode and partition-merge kernels)",
                          "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
                          "traffic": traffic, "algorithmic_bytes_per_launch": int(np.mean(step_algo)),
@@ -761,10 +763,9 @@ def run_adaptive(args, w):
     def step(arm, i):
         for cache, st, wsp, sl in arms[arm]:
             slots, tables, lens, _ = st[i % STAGED_STEPS]
-            P.pkv_kv_append(kn[sl], vn[sl], slots, cache.k_pool, cache.v_pool)
-            P.pkv_paged_attention_decode(q[sl], cache.k_pool, cache.v_pool, tables, lens, w.scale, out=out[sl],
-                                         workspace=wsp)
-        return sum(1 + decode_launches(c.max_blocks, c.block_size, 0) for c, _, _, _ in arms[arm])
+            P.pkv_append_and_decode(kn[sl], vn[sl], slots, q[sl], cache.k_pool, cache.v_pool, tables, lens, w.scale,
+                                    out=out[sl], workspace=wsp)
+        return sum(decode_launches(c.max_blocks, c.block_size, 0) for c, _, _, _ in arms[arm])
 
     res_arms = {}
     clocks = ClockSampler(local, not args.no_clocks)

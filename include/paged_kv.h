@@ -241,6 +241,25 @@ int pkv_paged_attention_decode(const void* q, const void* k_pool, const void* v_
                                int32_t partition_tokens, void* workspace, size_t workspace_bytes,
                                float* out, void* stream);
 
+/* KV append and decode of one step in one call: the result of
+ * pkv_kv_append(k_new, v_new, slot_mapping, n_tokens, ...) followed by
+ * pkv_paged_attention_decode(q, ...) on the same stream, every argument
+ * meaning what it means there (vLLM paging page §3, phases 1 and 2 of a
+ * decode step).  The new rows are written by the launch that builds the
+ * decode work list, so a step pays for one launch fewer; the decode kernel
+ * starts reading only after that launch has finished.  Pool contents and
+ * outputs are bit-identical to the two-call form.  n_tokens = 0 skips the
+ * append; num_seqs = 0 skips the decode.  Every argument is checked before
+ * anything is launched; errors as for the two calls.  Copy-on-write pairs of
+ * the step (pkv_copy_blocks) must be copied before this call. */
+int pkv_append_and_decode(const void* k_new, const void* v_new, const int32_t* slot_mapping,
+                          int32_t n_tokens, const void* q, void* k_pool, void* v_pool,
+                          const int32_t* block_tables, const int32_t* seq_lens, int32_t num_seqs,
+                          int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                          int32_t num_blocks, int32_t max_blocks_per_seq, int32_t block_size,
+                          float scale, int32_t dtype, int32_t partition_tokens, void* workspace,
+                          size_t workspace_bytes, float* out, void* stream);
+
 /* One whole decode step from host buffers in a single call (vLLM paging page
  * §3: phase 1 reservation, phase 3 copy-on-write, phase 2 attention), for
  * serving loops that want one crossing of the library boundary per step:
@@ -254,9 +273,8 @@ int pkv_paged_attention_decode(const void* q, const void* k_pool, const void* v_
  *      k_host / v_host [n][Hkv][D] to q_dev / k_dev / v_dev (element type:
  *      dtype, or float16 for e4m3 pools); then record buf->done_event (if
  *      not NULL);
- *   4. pkv_copy_blocks for the copy-on-write pairs, pkv_kv_append (or
- *      pkv_kv_append_fp8) and pkv_paged_attention_decode (or _fp8) into
- *      buf->out_dev [n][Hq][D] float32;
+ *   4. pkv_copy_blocks for the copy-on-write pairs, then
+ *      pkv_append_and_decode (or _fp8) into buf->out_dev [n][Hq][D] float32;
  *   5. if buf->out_host is not NULL, copy out_dev to it (device to host).
  * Every host buffer should be pinned for the copies to be asynchronous.
  * k_scale / v_scale are used for e4m3 pools only.
@@ -396,6 +414,19 @@ int pkv_paged_attention_decode_fp8(const void* q, const void* k_pool, const void
                                    int32_t max_blocks_per_seq, int32_t block_size, float scale, float k_scale,
                                    float v_scale, int32_t partition_tokens, void* workspace, size_t workspace_bytes,
                                    float* out, void* stream);
+
+/* e4m3 form of pkv_append_and_decode: pkv_kv_append_fp8(k_new, v_new,
+ * src_dtype, slot_mapping, n_tokens, ..., k_scale, v_scale) followed by
+ * pkv_paged_attention_decode_fp8(q, ...), in one call with the same
+ * launches saved and the same guarantees (bit-identical codes and outputs). */
+int pkv_append_and_decode_fp8(const void* k_new, const void* v_new, int32_t src_dtype,
+                              const int32_t* slot_mapping, int32_t n_tokens, const void* q,
+                              void* k_pool, void* v_pool, const int32_t* block_tables,
+                              const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads,
+                              int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks,
+                              int32_t max_blocks_per_seq, int32_t block_size, float scale,
+                              float k_scale, float v_scale, int32_t partition_tokens,
+                              void* workspace, size_t workspace_bytes, float* out, void* stream);
 
 /* Synchronise `stream`, then read the device status word of the current
  * device into *status: PKV_OK, or the first PKV_ERR_BAD_BLOCK /

@@ -6,7 +6,8 @@ host block allocator, C ABI in ``include/paged_kv.h``); this package is its
 thin Python binding.  Build the library with
 ``python -m paged_kv_cache_406_b200.build``.
 """
-from .binding import (Allocator, PagedKVError, pkv_copy_blocks, pkv_decode_workspace_size,  # noqa: F401
+from .binding import (Allocator, PagedKVError, pkv_append_and_decode, pkv_append_and_decode_fp8,  # noqa: F401
+                      pkv_copy_blocks, pkv_decode_workspace_size,
                       pkv_device_status, pkv_kv_append, pkv_kv_append_fp8, pkv_paged_attention_decode,
                       pkv_paged_attention_decode_fp8, pkv_paged_attention_decode_static,
                       pkv_paged_attention_prefill)

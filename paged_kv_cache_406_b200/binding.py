@@ -122,6 +122,63 @@ def pkv_paged_attention_decode(q: torch.Tensor, k_pool: torch.Tensor, v_pool: to
     return out
 
 
+def _new_rows(k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: torch.Tensor, hkv: int, d: int,
+              dtype=None) -> int:
+    for name, t in (("k_new", k_new), ("v_new", v_new)):
+        _cuda(t, name, dtype)
+        if t.dim() != 3 or t.shape[1:] != (hkv, d):
+            raise ValueError(f"{name} must be [n_tokens, {hkv}, {d}]")
+    if k_new.shape != v_new.shape or k_new.dtype != v_new.dtype:
+        raise ValueError("k_new and v_new differ in shape or dtype")
+    _cuda(slot_mapping, "slot_mapping", torch.int32)
+    if slot_mapping.numel() != k_new.shape[0]:
+        raise ValueError("slot_mapping must hold one slot per new token")
+    return k_new.shape[0]
+
+
+def _decode_io(q: torch.Tensor, hkv: int, d: int, bs: int, block_tables: torch.Tensor, seq_lens: torch.Tensor,
+               out: Optional[torch.Tensor], workspace: Optional[torch.Tensor], partition_tokens: int):
+    if q.dim() != 3 or q.shape[2] != d:
+        raise ValueError(f"q must be [num_seqs, num_q_heads, {d}]")
+    B, hq, _ = q.shape
+    _cuda(block_tables, "block_tables", torch.int32)
+    _cuda(seq_lens, "seq_lens", torch.int32)
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.numel() != B:
+        raise ValueError("block_tables must be [num_seqs, max_blocks_per_seq] and seq_lens [num_seqs]")
+    maxb = block_tables.shape[1]
+    if out is None:
+        out = torch.empty((B, hq, d), dtype=torch.float32, device=q.device)
+    else:
+        _cuda(out, "out", torch.float32)
+        if tuple(out.shape) != (B, hq, d):
+            raise ValueError("out has the wrong shape")
+    need = pkv_decode_workspace_size(B, hq, hkv, d, maxb, bs, partition_tokens)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    else:
+        _cuda(workspace, "workspace", torch.uint8)
+    return B, hq, maxb, out, workspace
+
+
+def pkv_append_and_decode(k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: torch.Tensor, q: torch.Tensor,
+                          k_pool: torch.Tensor, v_pool: torch.Tensor, block_tables: torch.Tensor,
+                          seq_lens: torch.Tensor, scale: float, out: Optional[torch.Tensor] = None,
+                          workspace: Optional[torch.Tensor] = None, partition_tokens: int = 0) -> torch.Tensor:
+    """:func:`pkv_kv_append` then :func:`pkv_paged_attention_decode` in one
+    library call (the new rows are written by the launch that plans the
+    decode); returns ``out``."""
+    nb, hkv, bs, d = _pool_dims(_cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"))
+    n = _new_rows(k_new, v_new, slot_mapping, hkv, d, k_pool.dtype)
+    _cuda(q, "q", k_pool.dtype)
+    B, hq, maxb, out, workspace = _decode_io(q, hkv, d, bs, block_tables, seq_lens, out, workspace, partition_tokens)
+    check(lib().pkv_append_and_decode(k_new.data_ptr(), v_new.data_ptr(), slot_mapping.data_ptr(), n, q.data_ptr(),
+                                      k_pool.data_ptr(), v_pool.data_ptr(), block_tables.data_ptr(),
+                                      seq_lens.data_ptr(), B, hq, hkv, d, nb, maxb, bs, float(scale),
+                                      _dtype_code(k_pool), partition_tokens, workspace.data_ptr(), workspace.numel(),
+                                      out.data_ptr(), _stream()))
+    return out
+
+
 def pkv_paged_attention_prefill(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
                                 block_tables: torch.Tensor, seq_lens: torch.Tensor, q_start: torch.Tensor,
                                 max_q_len: int, scale: float, out: Optional[torch.Tensor] = None) -> torch.Tensor:
@@ -243,6 +300,30 @@ def pkv_paged_attention_decode_fp8(q: torch.Tensor, k_pool: torch.Tensor, v_pool
     return out
 
 
+def pkv_append_and_decode_fp8(k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: torch.Tensor,
+                              q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                              block_tables: torch.Tensor, seq_lens: torch.Tensor, scale: float, k_scale: float,
+                              v_scale: float, out: Optional[torch.Tensor] = None,
+                              workspace: Optional[torch.Tensor] = None, partition_tokens: int = 0) -> torch.Tensor:
+    """:func:`pkv_kv_append_fp8` then :func:`pkv_paged_attention_decode_fp8`
+    in one library call; returns ``out``."""
+    _fp8_pool(k_pool, "k_pool")
+    _fp8_pool(v_pool, "v_pool")
+    if k_pool.dim() != 4 or k_pool.shape != v_pool.shape:
+        raise ValueError("pools must be [num_blocks, num_kv_heads, block_size, head_dim]")
+    nb, hkv, bs, d = k_pool.shape
+    n = _new_rows(k_new, v_new, slot_mapping, hkv, d)
+    _cuda(q, "q", torch.float16)
+    B, hq, maxb, out, workspace = _decode_io(q, hkv, d, bs, block_tables, seq_lens, out, workspace, partition_tokens)
+    check(lib().pkv_append_and_decode_fp8(k_new.data_ptr(), v_new.data_ptr(), _dtype_code(k_new),
+                                          slot_mapping.data_ptr(), n, q.data_ptr(), k_pool.data_ptr(),
+                                          v_pool.data_ptr(), block_tables.data_ptr(), seq_lens.data_ptr(), B, hq, hkv,
+                                          d, nb, maxb, bs, float(scale), float(k_scale), float(v_scale),
+                                          partition_tokens, workspace.data_ptr(), workspace.numel(), out.data_ptr(),
+                                          _stream()))
+    return out
+
+
 def pkv_device_status(clear: bool = True) -> int:
     """Synchronise the current stream and return the device status word."""
     st = ctypes.c_int32(0)
@@ -346,4 +427,5 @@ class Allocator:
 
 __all__ = ["Allocator", "PagedKVError", "pkv_kv_append", "pkv_copy_blocks", "pkv_decode_workspace_size",
            "pkv_paged_attention_decode", "pkv_paged_attention_decode_static", "pkv_device_status",
-           "pkv_kv_append_fp8", "pkv_paged_attention_decode_fp8"]
+           "pkv_kv_append_fp8", "pkv_paged_attention_decode_fp8", "pkv_append_and_decode",
+           "pkv_append_and_decode_fp8"]

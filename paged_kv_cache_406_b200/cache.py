@@ -9,9 +9,9 @@ step for one layer ("vLLM's 'memory paging' — PagedAttention illustrated", §3
 2. one host→device copy of the step's metadata (slots, copy pairs, block
    tables, lengths) from pinned memory;
 3. pkv_copy_blocks for the copy-on-write pairs, if any;
-4. pkv_kv_append of the new tokens' K/V;
-5. pkv_paged_attention_decode (plus its partition merge) over every sequence,
-   new token included.
+4. pkv_append_and_decode: the new tokens' K/V written into their slots by the
+   launch that plans the decode, then PagedAttention decode (plus its
+   partition merge) over every sequence, new token included.
 """
 from __future__ import annotations
 
@@ -136,13 +136,11 @@ class PagedKVCache:
         ws, own = self._buffers(n, q.shape[1], partition_tokens)
         out = own if out is None else out
         if self.fp8:
-            B.pkv_kv_append_fp8(k_new, v_new, slots, self.k_pool, self.v_pool, self.k_scale, self.v_scale)
-            return B.pkv_paged_attention_decode_fp8(q, self.k_pool, self.v_pool, tables, lens, scale, self.k_scale,
-                                                    self.v_scale, out=out, workspace=ws,
-                                                    partition_tokens=partition_tokens)
-        B.pkv_kv_append(k_new, v_new, slots, self.k_pool, self.v_pool)
-        return B.pkv_paged_attention_decode(q, self.k_pool, self.v_pool, tables, lens, scale, out=out,
-                                            workspace=ws, partition_tokens=partition_tokens)
+            return B.pkv_append_and_decode_fp8(k_new, v_new, slots, q, self.k_pool, self.v_pool, tables, lens, scale,
+                                               self.k_scale, self.v_scale, out=out, workspace=ws,
+                                               partition_tokens=partition_tokens)
+        return B.pkv_append_and_decode(k_new, v_new, slots, q, self.k_pool, self.v_pool, tables, lens, scale,
+                                       out=out, workspace=ws, partition_tokens=partition_tokens)
 
     # -- the decode step in one library call -------------------------------
     def decode_step_host(self, seq_ids: np.ndarray, q_host: torch.Tensor, k_host: torch.Tensor,

@@ -56,13 +56,11 @@ struct DecodeParams {
 // ---------------------------------------------------------------------------
 // plan: seq_lens -> work list, partitions sorted by block count, largest first
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ seq_lens, int32_t num_seqs,
-                                                    int32_t max_tokens, int32_t part_tokens, int32_t block_size,
-                                                    int4* __restrict__ items, int32_t* __restrict__ n_items) {
-  // the decode grid may be scheduled now; it waits for this grid's results
-  // (griddepcontrol.wait) before reading them
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  extern __shared__ int32_t hist[];  // [kmax + 1] counts, then [kmax + 1] cursors
+// One CTA builds the list; `hist` is 2 * (part_tokens / block_size + 1) ints of
+// shared memory.
+__device__ __forceinline__ void plan_body(const int32_t* __restrict__ seq_lens, int32_t num_seqs, int32_t max_tokens,
+                                          int32_t part_tokens, int32_t block_size, int4* __restrict__ items,
+                                          int32_t* __restrict__ n_items, int32_t* hist) {
   const int kmax = part_tokens / block_size;
   int32_t* cursor = hist + kmax + 1;
   for (int i = threadIdx.x; i <= kmax; i += blockDim.x) hist[i] = 0;
@@ -106,6 +104,16 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
       items[pos] = make_int4(b, 0, 1, 0);
     }
   }
+}
+
+__global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ seq_lens, int32_t num_seqs,
+                                                    int32_t max_tokens, int32_t part_tokens, int32_t block_size,
+                                                    int4* __restrict__ items, int32_t* __restrict__ n_items) {
+  // the decode grid may be scheduled now; it waits for this grid's results
+  // (griddepcontrol.wait) before reading them
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  extern __shared__ int32_t hist[];  // [kmax + 1] counts, then [kmax + 1] cursors
+  plan_body(seq_lens, num_seqs, max_tokens, part_tokens, block_size, items, n_items, hist);
 }
 
 // ---------------------------------------------------------------------------

@@ -1,6 +1,7 @@
 // Device entry points of libpagedkv (sm_100a): KV append, block copy,
-// PagedAttention decode (plan, decode and partition-merge kernels) and the
-// device status word.
+// PagedAttention decode (plan, decode and partition-merge kernels), append and
+// decode in one call, paged prefill, the one-call step from host buffers and
+// the device status word.  The kernels live in the .cuh files.
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -10,132 +11,12 @@
 
 #include <cuda_fp8.h>
 
+#include "append.cuh"
 #include "decode.cuh"
 #include "decode_mma.cuh"
 #include "device_common.cuh"
 #include "prefill.cuh"
 #include "pkv_internal.h"
-
-namespace pkv {
-
-// ---------------------------------------------------------------------------
-// KV append: one thread per 16-byte chunk of one (token, kv head) row, K and V.
-// vLLM paging page §3 phase 1: the new token is written into its slot.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) kv_append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
-                                                        const int32_t* __restrict__ slots, int64_t n_chunks,
-                                                        uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
-                                                        int32_t num_blocks, int32_t num_kv_heads, int32_t row_chunks,
-                                                        int32_t block_size) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= n_chunks) return;
-  const int32_t chunk = static_cast<int32_t>(i % row_chunks);
-  const int64_t row = i / row_chunks;  // token * num_kv_heads + head
-  const int32_t h = static_cast<int32_t>(row % num_kv_heads);
-  const int64_t tok = row / num_kv_heads;
-  const int32_t slot = slots[tok];
-  if (slot < 0) return;  // padding token
-  const int32_t blk = slot / block_size, off = slot - blk * block_size;
-  if (blk >= num_blocks) {
-    if (chunk == 0 && h == 0) record_error(PKV_ERR_BAD_BLOCK);
-    return;
-  }
-  const int64_t dst = ((static_cast<int64_t>(blk) * num_kv_heads + h) * block_size + off) * row_chunks + chunk;
-  k_pool[dst] = k_new[i];
-  v_pool[dst] = v_new[i];
-}
-
-// ---------------------------------------------------------------------------
-// Block copy for copy-on-write (vLLM paging page §3 phase 3): pair y copies
-// one whole block of K and of V, every head and offset.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
-                                                          const int32_t* __restrict__ pairs, int32_t num_blocks,
-                                                          int64_t block_chunks) {
-  const int32_t src = pairs[2 * blockIdx.y], dst = pairs[2 * blockIdx.y + 1];
-  if (static_cast<unsigned>(src) >= static_cast<unsigned>(num_blocks) ||
-      static_cast<unsigned>(dst) >= static_cast<unsigned>(num_blocks)) {
-    if (blockIdx.x == 0 && threadIdx.x == 0) record_error(PKV_ERR_BAD_BLOCK);
-    return;
-  }
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < block_chunks;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    k_pool[dst * block_chunks + i] = k_pool[src * block_chunks + i];
-    v_pool[dst * block_chunks + i] = v_pool[src * block_chunks + i];
-  }
-}
-
-// ---------------------------------------------------------------------------
-// KV append into e4m3 pools: each thread quantises 8 elements of one (token,
-// head) row, x * (1 / scale) in fp32, rounded to nearest e4m3 (ties to even,
-// saturating to +-448), and stores 8 bytes.
-// ---------------------------------------------------------------------------
-template <typename Src>
-__device__ __forceinline__ void load8_f32(const Src* p, float (&x)[8]);
-
-template <>
-__device__ __forceinline__ void load8_f32<float>(const float* p, float (&x)[8]) {
-  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
-  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-}
-
-template <>
-__device__ __forceinline__ void load8_f32<__nv_bfloat16>(const __nv_bfloat16* p, float (&x)[8]) {
-  const uint4 r = *reinterpret_cast<const uint4*>(p);
-  float2 f[4];
-  Elem<__nv_bfloat16>::widen(r, f);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) { x[2 * i] = f[i].x; x[2 * i + 1] = f[i].y; }
-}
-
-template <>
-__device__ __forceinline__ void load8_f32<__half>(const __half* p, float (&x)[8]) {
-  const uint4 r = *reinterpret_cast<const uint4*>(p);
-  float2 f[4];
-  Elem<__half>::widen(r, f);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) { x[2 * i] = f[i].x; x[2 * i + 1] = f[i].y; }
-}
-
-template <typename Src>
-__global__ void __launch_bounds__(256) kv_append_fp8_kernel(const Src* __restrict__ k_new, const Src* __restrict__ v_new,
-                                                            const int32_t* __restrict__ slots, int64_t n_groups,
-                                                            uint8_t* __restrict__ k_pool, uint8_t* __restrict__ v_pool,
-                                                            int32_t num_blocks, int32_t num_kv_heads, int32_t head_dim,
-                                                            int32_t block_size, float k_inv, float v_inv) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= n_groups) return;
-  const int32_t per_row = head_dim / 8;
-  const int32_t grp = static_cast<int32_t>(i % per_row);
-  const int64_t row = i / per_row;  // token * num_kv_heads + head
-  const int32_t h = static_cast<int32_t>(row % num_kv_heads);
-  const int64_t tok = row / num_kv_heads;
-  const int32_t slot = slots[tok];
-  if (slot < 0) return;
-  const int32_t blk = slot / block_size, off = slot - blk * block_size;
-  if (blk >= num_blocks) {
-    if (grp == 0 && h == 0) record_error(PKV_ERR_BAD_BLOCK);
-    return;
-  }
-  const int64_t dst = ((static_cast<int64_t>(blk) * num_kv_heads + h) * block_size + off) * head_dim + grp * 8;
-  const int64_t src = row * head_dim + grp * 8;
-#pragma unroll
-  for (int kv = 0; kv < 2; ++kv) {
-    float x[8];
-    load8_f32<Src>((kv ? v_new : k_new) + src, x);
-    const float inv = kv ? v_inv : k_inv;
-    uint32_t packed[2] = {0u, 0u};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const __nv_fp8x2_storage_t q2 =
-          __nv_cvt_float2_to_fp8x2(make_float2(x[2 * j] * inv, x[2 * j + 1] * inv), __NV_SATFINITE, __NV_E4M3);
-      packed[j >> 1] |= static_cast<uint32_t>(q2) << (16 * (j & 1));
-    }
-    *reinterpret_cast<uint2*>((kv ? v_pool : k_pool) + dst) = make_uint2(packed[0], packed[1]);
-  }
-}
-
-}  // namespace pkv
 
 // ===========================================================================
 // host side
@@ -235,16 +116,48 @@ cudaError_t launch_pdl(Kernel kern, dim3 grid, dim3 block, size_t smem, cudaStre
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-// plan kernel -> decode kernel -> merge kernel (the last only when some
-// sequence can span more than one partition)
+// New K/V rows to write in the same launch as the plan kernel (the append of
+// a decode step), already checked by the caller.  src_dtype < 0: 16-byte row
+// copies into a 16-bit or fp32 pool; otherwise the source dtype of rows
+// quantised into an e4m3 pool.
+struct PendingAppend {
+  pkv::AppendArgs args;
+  int src_dtype;
+};
+
+// plan kernel (or append + plan) -> decode kernel -> merge kernel (the last
+// only when some sequence can span more than one partition)
 template <int D, typename Kernel, typename... Args>
 int launch_plan_decode_merge(const pkv::DecodeParams& p, const int32_t* seq_lens, int32_t num_seqs,
-                             int32_t max_tokens, Kernel kern, int grid, int threads, size_t smem, cudaStream_t stream,
-                             Args... args) {
+                             int32_t max_tokens, const PendingAppend* ap, Kernel kern, int grid, int threads,
+                             size_t smem, cudaStream_t stream, Args... args) {
   const int kmax = p.partition_tokens / p.block_size;
-  pkv::plan_kernel<<<1, 1024, 2 * (kmax + 1) * sizeof(int32_t), stream>>>(
-      seq_lens, num_seqs, max_tokens, p.partition_tokens, p.block_size, const_cast<int4*>(p.items),
-      const_cast<int32_t*>(p.n_items));
+  const size_t plan_smem = 2 * (kmax + 1) * sizeof(int32_t);
+  int4* items = const_cast<int4*>(p.items);
+  int32_t* n_items = const_cast<int32_t*>(p.n_items);
+  if (ap) {
+    const unsigned g = static_cast<unsigned>(1 + (ap->args.n_units + 255) / 256);
+    switch (ap->src_dtype) {
+      case -1:
+        pkv::append_plan_kernel<void><<<g, 256, plan_smem, stream>>>(ap->args, seq_lens, num_seqs, max_tokens,
+                                                                     p.partition_tokens, p.block_size, items, n_items);
+        break;
+      case PKV_F32:
+        pkv::append_plan_kernel<float><<<g, 256, plan_smem, stream>>>(ap->args, seq_lens, num_seqs, max_tokens,
+                                                                      p.partition_tokens, p.block_size, items, n_items);
+        break;
+      case PKV_BF16:
+        pkv::append_plan_kernel<__nv_bfloat16><<<g, 256, plan_smem, stream>>>(
+            ap->args, seq_lens, num_seqs, max_tokens, p.partition_tokens, p.block_size, items, n_items);
+        break;
+      default:
+        pkv::append_plan_kernel<__half><<<g, 256, plan_smem, stream>>>(ap->args, seq_lens, num_seqs, max_tokens,
+                                                                       p.partition_tokens, p.block_size, items, n_items);
+    }
+  } else {
+    pkv::plan_kernel<<<1, 1024, plan_smem, stream>>>(seq_lens, num_seqs, max_tokens, p.partition_tokens, p.block_size,
+                                                     items, n_items);
+  }
   cudaError_t e = launch_pdl(kern, dim3(grid), dim3(threads), smem, stream, p, args...);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   if (p.max_parts > 1) {
@@ -262,7 +175,7 @@ int launch_plan_decode_merge(const pkv::DecodeParams& p, const int32_t* seq_lens
 
 template <typename T, int D, int G>
 int launch_decode(const pkv::DecodeParams& base, const int32_t* seq_lens, int32_t num_seqs, int32_t max_tokens,
-                  cudaStream_t stream) {
+                  const PendingAppend* ap, cudaStream_t stream) {
   pkv::DecodeParams p = base;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -292,7 +205,8 @@ int launch_decode(const pkv::DecodeParams& base, const int32_t* seq_lens, int32_
 
   const int64_t work_upper = int64_t(num_seqs) * p.max_parts * p.num_kv_heads;
   const int grid = static_cast<int>(std::min<int64_t>(int64_t(sm_count(dev)) * occ, work_upper));
-  return launch_plan_decode_merge<D>(p, seq_lens, num_seqs, max_tokens, kern, grid, pkv::kDecodeThreads, smem, stream);
+  return launch_plan_decode_merge<D>(p, seq_lens, num_seqs, max_tokens, ap, kern, grid, pkv::kDecodeThreads, smem,
+                                     stream);
 }
 
 // ---- tensor maps over the K/V pools for the tensor-core kernel ----
@@ -375,7 +289,7 @@ int pool_map(CUtensorMap* out, const void* pool, int dtype, int64_t rows, int he
 
 template <typename T, int D, int G, int kKVBytes = 2>
 int launch_decode_mma(const pkv::DecodeParams& base, const int32_t* seq_lens, int32_t num_seqs, int32_t max_tokens,
-                      int dtype, cudaStream_t stream) {
+                      int dtype, const PendingAppend* ap, cudaStream_t stream) {
   pkv::DecodeParams p = base;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -405,34 +319,34 @@ int launch_decode_mma(const pkv::DecodeParams& base, const int32_t* seq_lens, in
 
   const int64_t work_upper = int64_t(num_seqs) * p.max_parts * p.num_kv_heads;
   const int grid = static_cast<int>(std::min<int64_t>(int64_t(sm_count(dev)) * occ, work_upper));
-  return launch_plan_decode_merge<D>(p, seq_lens, num_seqs, max_tokens, kern, grid, pkv::kMmaThreads, smem, stream, mk,
-                                     mv);
+  return launch_plan_decode_merge<D>(p, seq_lens, num_seqs, max_tokens, ap, kern, grid, pkv::kMmaThreads, smem, stream,
+                                     mk, mv);
 }
 
 template <typename T>
 int dispatch_decode_mma(int32_t head_dim, int32_t group, const pkv::DecodeParams& p, const int32_t* seq_lens,
-                        int32_t num_seqs, int32_t max_tokens, int dtype, cudaStream_t s) {
+                        int32_t num_seqs, int32_t max_tokens, int dtype, const PendingAppend* ap, cudaStream_t s) {
   if (head_dim == 128) {
-    if (group == 2) return launch_decode_mma<T, 128, 2>(p, seq_lens, num_seqs, max_tokens, dtype, s);
-    if (group == 4) return launch_decode_mma<T, 128, 4>(p, seq_lens, num_seqs, max_tokens, dtype, s);
-    return launch_decode_mma<T, 128, 8>(p, seq_lens, num_seqs, max_tokens, dtype, s);
+    if (group == 2) return launch_decode_mma<T, 128, 2>(p, seq_lens, num_seqs, max_tokens, dtype, ap, s);
+    if (group == 4) return launch_decode_mma<T, 128, 4>(p, seq_lens, num_seqs, max_tokens, dtype, ap, s);
+    return launch_decode_mma<T, 128, 8>(p, seq_lens, num_seqs, max_tokens, dtype, ap, s);
   }
-  if (group == 2) return launch_decode_mma<T, 64, 2>(p, seq_lens, num_seqs, max_tokens, dtype, s);
-  if (group == 4) return launch_decode_mma<T, 64, 4>(p, seq_lens, num_seqs, max_tokens, dtype, s);
-  return launch_decode_mma<T, 64, 8>(p, seq_lens, num_seqs, max_tokens, dtype, s);
+  if (group == 2) return launch_decode_mma<T, 64, 2>(p, seq_lens, num_seqs, max_tokens, dtype, ap, s);
+  if (group == 4) return launch_decode_mma<T, 64, 4>(p, seq_lens, num_seqs, max_tokens, dtype, ap, s);
+  return launch_decode_mma<T, 64, 8>(p, seq_lens, num_seqs, max_tokens, dtype, ap, s);
 }
 
 template <typename T>
 int dispatch_decode(int32_t head_dim, int32_t group, const pkv::DecodeParams& p, const int32_t* seq_lens,
-                    int32_t num_seqs, int32_t max_tokens, cudaStream_t s) {
+                    int32_t num_seqs, int32_t max_tokens, const PendingAppend* ap, cudaStream_t s) {
   if (head_dim == 128) {
-    if (group == 1) return launch_decode<T, 128, 1>(p, seq_lens, num_seqs, max_tokens, s);
-    if (group == 2) return launch_decode<T, 128, 2>(p, seq_lens, num_seqs, max_tokens, s);
-    return launch_decode<T, 128, 4>(p, seq_lens, num_seqs, max_tokens, s);
+    if (group == 1) return launch_decode<T, 128, 1>(p, seq_lens, num_seqs, max_tokens, ap, s);
+    if (group == 2) return launch_decode<T, 128, 2>(p, seq_lens, num_seqs, max_tokens, ap, s);
+    return launch_decode<T, 128, 4>(p, seq_lens, num_seqs, max_tokens, ap, s);
   }
-  if (group == 1) return launch_decode<T, 64, 1>(p, seq_lens, num_seqs, max_tokens, s);
-  if (group == 2) return launch_decode<T, 64, 2>(p, seq_lens, num_seqs, max_tokens, s);
-  return launch_decode<T, 64, 4>(p, seq_lens, num_seqs, max_tokens, s);
+  if (group == 1) return launch_decode<T, 64, 1>(p, seq_lens, num_seqs, max_tokens, ap, s);
+  if (group == 2) return launch_decode<T, 64, 2>(p, seq_lens, num_seqs, max_tokens, ap, s);
+  return launch_decode<T, 64, 4>(p, seq_lens, num_seqs, max_tokens, ap, s);
 }
 
 }  // namespace
@@ -451,9 +365,9 @@ extern "C" int pkv_kv_append(const void* k_new, const void* v_new, const int32_t
   const int32_t row_chunks = static_cast<int32_t>(head_dim * elem_size(dtype) / 16);
   const int64_t n_chunks = int64_t(n_tokens) * num_kv_heads * row_chunks;
   const int64_t blocks = (n_chunks + 255) / 256;
-  pkv::kv_append_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), slot_mapping, n_chunks,
-      static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), num_blocks, num_kv_heads, row_chunks, block_size);
+  const pkv::AppendArgs a{k_new, v_new, slot_mapping, n_chunks, k_pool,     v_pool,
+                          num_blocks, num_kv_heads, row_chunks, block_size, 1.0f, 1.0f};
+  pkv::kv_append_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pkv_kv_append launch");
   return pkv::ok();
@@ -495,13 +409,29 @@ extern "C" int pkv_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, 
   return pkv::ok();
 }
 
-extern "C" int pkv_paged_attention_decode(const void* q, const void* k_pool, const void* v_pool,
-                                          const int32_t* block_tables, const int32_t* seq_lens, int32_t num_seqs,
-                                          int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
-                                          int32_t num_blocks, int32_t max_blocks_per_seq, int32_t block_size,
-                                          float scale, int32_t dtype, int32_t partition_tokens, void* workspace,
-                                          size_t workspace_bytes, float* out, void* stream) {
-  const char* fn = "pkv_paged_attention_decode";
+namespace {
+
+// The new rows alone (a step whose batch is empty).
+int launch_append_only(const PendingAppend& ap, cudaStream_t s) {
+  const unsigned blocks = static_cast<unsigned>((ap.args.n_units + 255) / 256);
+  switch (ap.src_dtype) {
+    case -1: pkv::kv_append_kernel<<<blocks, 256, 0, s>>>(ap.args); break;
+    case PKV_F32: pkv::kv_append_fp8_kernel<float><<<blocks, 256, 0, s>>>(ap.args); break;
+    case PKV_BF16: pkv::kv_append_fp8_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(ap.args); break;
+    default: pkv::kv_append_fp8_kernel<__half><<<blocks, 256, 0, s>>>(ap.args);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  return pkv::ok();
+}
+
+// Decode over 16-bit or fp32 pools; with `ap`, the step's new rows are
+// written by the plan launch first.
+int decode_16(const char* fn, const void* q, const void* k_pool, const void* v_pool, const int32_t* block_tables,
+              const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+              int32_t num_blocks, int32_t max_blocks_per_seq, int32_t block_size, float scale, int32_t dtype,
+              int32_t partition_tokens, void* workspace, size_t workspace_bytes, float* out,
+              const PendingAppend* ap, void* stream) {
   int rc = check_common(num_kv_heads, head_dim, block_size, dtype, fn);
   if (rc) return rc;
   if (num_seqs < 0 || num_q_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq < 0)
@@ -518,7 +448,7 @@ extern "C" int pkv_paged_attention_decode(const void* q, const void* k_pool, con
   int32_t pt = 0;
   rc = resolve_partition(partition_tokens, block_size, &pt);
   if (rc) return rc;
-  if (num_seqs == 0) return pkv::ok();
+  if (num_seqs == 0) return ap ? launch_append_only(*ap, static_cast<cudaStream_t>(stream)) : pkv::ok();
   if (!q || !k_pool || !v_pool || !block_tables || !seq_lens || !workspace || !out)
     return fail(PKV_ERR_INVALID_ARG, "%s: NULL pointer", fn);
   if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out))
@@ -559,15 +489,54 @@ extern "C" int pkv_paged_attention_decode(const void* q, const void* k_pool, con
   if (dtype != PKV_F32 && group >= 2 && pt % pkv::kChunkTokens == 0) {
     if (int64_t(num_blocks) * num_kv_heads * block_size > INT32_MAX)
       return fail(PKV_ERR_INVALID_ARG, "%s: pool has more than 2^31 token rows", fn);
-    if (dtype == PKV_BF16) return dispatch_decode_mma<__nv_bfloat16>(head_dim, group, p, seq_lens, num_seqs, mt, dtype, s);
-    return dispatch_decode_mma<__half>(head_dim, group, p, seq_lens, num_seqs, mt, dtype, s);
+    if (dtype == PKV_BF16)
+      return dispatch_decode_mma<__nv_bfloat16>(head_dim, group, p, seq_lens, num_seqs, mt, dtype, ap, s);
+    return dispatch_decode_mma<__half>(head_dim, group, p, seq_lens, num_seqs, mt, dtype, ap, s);
   }
   if (group == 8) return fail(PKV_ERR_UNSUPPORTED, "%s: group size 8 needs partition_tokens %% 16 == 0", fn);
   switch (dtype) {
-    case PKV_F32: return dispatch_decode<float>(head_dim, group, p, seq_lens, num_seqs, mt, s);
-    case PKV_BF16: return dispatch_decode<__nv_bfloat16>(head_dim, group, p, seq_lens, num_seqs, mt, s);
-    default: return dispatch_decode<__half>(head_dim, group, p, seq_lens, num_seqs, mt, s);
+    case PKV_F32: return dispatch_decode<float>(head_dim, group, p, seq_lens, num_seqs, mt, ap, s);
+    case PKV_BF16: return dispatch_decode<__nv_bfloat16>(head_dim, group, p, seq_lens, num_seqs, mt, ap, s);
+    default: return dispatch_decode<__half>(head_dim, group, p, seq_lens, num_seqs, mt, ap, s);
   }
+}
+
+}  // namespace
+
+extern "C" int pkv_paged_attention_decode(const void* q, const void* k_pool, const void* v_pool,
+                                          const int32_t* block_tables, const int32_t* seq_lens, int32_t num_seqs,
+                                          int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                          int32_t num_blocks, int32_t max_blocks_per_seq, int32_t block_size,
+                                          float scale, int32_t dtype, int32_t partition_tokens, void* workspace,
+                                          size_t workspace_bytes, float* out, void* stream) {
+  return decode_16("pkv_paged_attention_decode", q, k_pool, v_pool, block_tables, seq_lens, num_seqs, num_q_heads,
+                   num_kv_heads, head_dim, num_blocks, max_blocks_per_seq, block_size, scale, dtype, partition_tokens,
+                   workspace, workspace_bytes, out, nullptr, stream);
+}
+
+extern "C" int pkv_append_and_decode(const void* k_new, const void* v_new, const int32_t* slot_mapping,
+                                     int32_t n_tokens, const void* q, void* k_pool, void* v_pool,
+                                     const int32_t* block_tables, const int32_t* seq_lens, int32_t num_seqs,
+                                     int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks,
+                                     int32_t max_blocks_per_seq, int32_t block_size, float scale, int32_t dtype,
+                                     int32_t partition_tokens, void* workspace, size_t workspace_bytes, float* out,
+                                     void* stream) {
+  const char* fn = "pkv_append_and_decode";
+  int rc = check_common(num_kv_heads, head_dim, block_size, dtype, fn);
+  if (rc) return rc;
+  if (n_tokens < 0 || num_blocks <= 0) return fail(PKV_ERR_INVALID_ARG, "%s: n_tokens/num_blocks", fn);
+  if (n_tokens > 0) {
+    if (!k_new || !v_new || !slot_mapping || !k_pool || !v_pool) return fail(PKV_ERR_INVALID_ARG, "%s: NULL pointer", fn);
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pool) || !aligned16(v_pool))
+      return fail(PKV_ERR_INVALID_ARG, "%s: K/V buffers must be 16-byte aligned", fn);
+  }
+  const int32_t row_chunks = static_cast<int32_t>(head_dim * elem_size(dtype) / 16);
+  PendingAppend ap{{k_new, v_new, slot_mapping, int64_t(n_tokens) * num_kv_heads * row_chunks, k_pool, v_pool,
+                    num_blocks, num_kv_heads, row_chunks, block_size, 1.0f, 1.0f},
+                   -1};
+  return decode_16(fn, q, k_pool, v_pool, block_tables, seq_lens, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                   num_blocks, max_blocks_per_seq, block_size, scale, dtype, partition_tokens, workspace,
+                   workspace_bytes, out, n_tokens > 0 ? &ap : nullptr, stream);
 }
 
 extern "C" int pkv_device_status(void* stream, int32_t* status, int32_t clear) {
@@ -608,38 +577,25 @@ extern "C" int pkv_kv_append_fp8(const void* k_new, const void* v_new, int32_t s
   const int64_t n_groups = int64_t(n_tokens) * num_kv_heads * (head_dim / 8);
   const unsigned blocks = static_cast<unsigned>((n_groups + 255) / 256);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint8_t* kp = static_cast<uint8_t*>(k_pool);
-  uint8_t* vp = static_cast<uint8_t*>(v_pool);
+  const pkv::AppendArgs a{k_new,      v_new,        slot_mapping, n_groups,   k_pool, v_pool,
+                          num_blocks, num_kv_heads, head_dim / 8, block_size, k_inv,  v_inv};
   switch (src_dtype) {
-    case PKV_F32:
-      pkv::kv_append_fp8_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(k_new),
-                                                              static_cast<const float*>(v_new), slot_mapping, n_groups,
-                                                              kp, vp, num_blocks, num_kv_heads, head_dim, block_size,
-                                                              k_inv, v_inv);
-      break;
-    case PKV_BF16:
-      pkv::kv_append_fp8_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
-          static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new), slot_mapping, n_groups,
-          kp, vp, num_blocks, num_kv_heads, head_dim, block_size, k_inv, v_inv);
-      break;
-    default:
-      pkv::kv_append_fp8_kernel<__half><<<blocks, 256, 0, s>>>(static_cast<const __half*>(k_new),
-                                                               static_cast<const __half*>(v_new), slot_mapping,
-                                                               n_groups, kp, vp, num_blocks, num_kv_heads, head_dim,
-                                                               block_size, k_inv, v_inv);
+    case PKV_F32: pkv::kv_append_fp8_kernel<float><<<blocks, 256, 0, s>>>(a); break;
+    case PKV_BF16: pkv::kv_append_fp8_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(a); break;
+    default: pkv::kv_append_fp8_kernel<__half><<<blocks, 256, 0, s>>>(a);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pkv_kv_append_fp8 launch");
   return pkv::ok();
 }
 
-extern "C" int pkv_paged_attention_decode_fp8(const void* q, const void* k_pool, const void* v_pool,
-                                              const int32_t* block_tables, const int32_t* seq_lens, int32_t num_seqs,
-                                              int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
-                                              int32_t num_blocks, int32_t max_blocks_per_seq, int32_t block_size,
-                                              float scale, float k_scale, float v_scale, int32_t partition_tokens,
-                                              void* workspace, size_t workspace_bytes, float* out, void* stream) {
-  const char* fn = "pkv_paged_attention_decode_fp8";
+namespace {
+
+int decode_fp8(const char* fn, const void* q, const void* k_pool, const void* v_pool, const int32_t* block_tables,
+               const int32_t* seq_lens, int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+               int32_t head_dim, int32_t num_blocks, int32_t max_blocks_per_seq, int32_t block_size, float scale,
+               float k_scale, float v_scale, int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+               float* out, const PendingAppend* ap, void* stream) {
   int rc = check_common(num_kv_heads, head_dim, block_size, PKV_F16, fn);
   if (rc) return rc;
   if (head_dim != 128) return fail(PKV_ERR_UNSUPPORTED, "%s: e4m3 pools need head_dim 128", fn);
@@ -656,7 +612,7 @@ extern "C" int pkv_paged_attention_decode_fp8(const void* q, const void* k_pool,
   rc = resolve_partition(partition_tokens, block_size, &pt);
   if (rc) return rc;
   if (pt % pkv::kChunkTokens != 0) return fail(PKV_ERR_INVALID_ARG, "%s: partition_tokens must be a multiple of 16", fn);
-  if (num_seqs == 0) return pkv::ok();
+  if (num_seqs == 0) return ap ? launch_append_only(*ap, static_cast<cudaStream_t>(stream)) : pkv::ok();
   if (!q || !k_pool || !v_pool || !block_tables || !seq_lens || !workspace || !out)
     return fail(PKV_ERR_INVALID_ARG, "%s: NULL pointer", fn);
   if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out))
@@ -695,11 +651,53 @@ extern "C" int pkv_paged_attention_decode_fp8(const void* q, const void* k_pool,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int32_t mt = static_cast<int32_t>(max_tokens);
   switch (group) {
-    case 1: return launch_decode_mma<__half, 128, 1, 1>(p, seq_lens, num_seqs, mt, PKV_FP8_E4M3, s);
-    case 2: return launch_decode_mma<__half, 128, 2, 1>(p, seq_lens, num_seqs, mt, PKV_FP8_E4M3, s);
-    case 4: return launch_decode_mma<__half, 128, 4, 1>(p, seq_lens, num_seqs, mt, PKV_FP8_E4M3, s);
-    default: return launch_decode_mma<__half, 128, 8, 1>(p, seq_lens, num_seqs, mt, PKV_FP8_E4M3, s);
+    case 1: return launch_decode_mma<__half, 128, 1, 1>(p, seq_lens, num_seqs, mt, PKV_FP8_E4M3, ap, s);
+    case 2: return launch_decode_mma<__half, 128, 2, 1>(p, seq_lens, num_seqs, mt, PKV_FP8_E4M3, ap, s);
+    case 4: return launch_decode_mma<__half, 128, 4, 1>(p, seq_lens, num_seqs, mt, PKV_FP8_E4M3, ap, s);
+    default: return launch_decode_mma<__half, 128, 8, 1>(p, seq_lens, num_seqs, mt, PKV_FP8_E4M3, ap, s);
   }
+}
+
+}  // namespace
+
+extern "C" int pkv_paged_attention_decode_fp8(const void* q, const void* k_pool, const void* v_pool,
+                                              const int32_t* block_tables, const int32_t* seq_lens, int32_t num_seqs,
+                                              int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                              int32_t num_blocks, int32_t max_blocks_per_seq, int32_t block_size,
+                                              float scale, float k_scale, float v_scale, int32_t partition_tokens,
+                                              void* workspace, size_t workspace_bytes, float* out, void* stream) {
+  return decode_fp8("pkv_paged_attention_decode_fp8", q, k_pool, v_pool, block_tables, seq_lens, num_seqs,
+                    num_q_heads, num_kv_heads, head_dim, num_blocks, max_blocks_per_seq, block_size, scale, k_scale,
+                    v_scale, partition_tokens, workspace, workspace_bytes, out, nullptr, stream);
+}
+
+extern "C" int pkv_append_and_decode_fp8(const void* k_new, const void* v_new, int32_t src_dtype,
+                                         const int32_t* slot_mapping, int32_t n_tokens, const void* q, void* k_pool,
+                                         void* v_pool, const int32_t* block_tables, const int32_t* seq_lens,
+                                         int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                         int32_t head_dim, int32_t num_blocks, int32_t max_blocks_per_seq,
+                                         int32_t block_size, float scale, float k_scale, float v_scale,
+                                         int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                                         float* out, void* stream) {
+  const char* fn = "pkv_append_and_decode_fp8";
+  int rc = check_common(num_kv_heads, head_dim, block_size, src_dtype, fn);
+  if (rc) return rc;
+  if (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
+    return fail(PKV_ERR_INVALID_ARG, "%s: scales must be positive and finite", fn);
+  if (n_tokens < 0 || num_blocks <= 0) return fail(PKV_ERR_INVALID_ARG, "%s: n_tokens/num_blocks", fn);
+  if (n_tokens > 0) {
+    if (!k_new || !v_new || !slot_mapping || !k_pool || !v_pool) return fail(PKV_ERR_INVALID_ARG, "%s: NULL pointer", fn);
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pool) || !aligned16(v_pool))
+      return fail(PKV_ERR_INVALID_ARG, "%s: buffers must be 16-byte aligned", fn);
+  }
+  const float k_inv = static_cast<float>(1.0 / static_cast<double>(k_scale));
+  const float v_inv = static_cast<float>(1.0 / static_cast<double>(v_scale));
+  PendingAppend ap{{k_new, v_new, slot_mapping, int64_t(n_tokens) * num_kv_heads * (head_dim / 8), k_pool, v_pool,
+                    num_blocks, num_kv_heads, head_dim / 8, block_size, k_inv, v_inv},
+                   src_dtype};
+  return decode_fp8(fn, q, k_pool, v_pool, block_tables, seq_lens, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                    num_blocks, max_blocks_per_seq, block_size, scale, k_scale, v_scale, partition_tokens, workspace,
+                    workspace_bytes, out, n_tokens > 0 ? &ap : nullptr, stream);
 }
 
 // ===========================================================================
@@ -970,19 +968,14 @@ extern "C" int pkv_decode_step_host(pkv_alloc_t* a, const int64_t* seq_ids, int3
     if (rc) return rc;
   }
   if (fp8) {
-    rc = pkv_kv_append_fp8(buf->k_dev, buf->v_dev, PKV_F16, md, n, k_pool, v_pool, num_blocks, num_kv_heads,
-                           head_dim, block_size, k_scale, v_scale, stream);
-    if (rc) return rc;
-    rc = pkv_paged_attention_decode_fp8(buf->q_dev, k_pool, v_pool, md + 4 * n, md + n, n, num_q_heads, num_kv_heads,
-                                        head_dim, num_blocks, max_blocks_per_seq, block_size, scale, k_scale, v_scale,
-                                        partition_tokens, workspace, workspace_bytes, buf->out_dev, stream);
+    rc = pkv_append_and_decode_fp8(buf->k_dev, buf->v_dev, PKV_F16, md, n, buf->q_dev, k_pool, v_pool, md + 4 * n,
+                                   md + n, n, num_q_heads, num_kv_heads, head_dim, num_blocks, max_blocks_per_seq,
+                                   block_size, scale, k_scale, v_scale, partition_tokens, workspace, workspace_bytes,
+                                   buf->out_dev, stream);
   } else {
-    rc = pkv_kv_append(buf->k_dev, buf->v_dev, md, n, k_pool, v_pool, num_blocks, num_kv_heads, head_dim, block_size,
-                       dtype, stream);
-    if (rc) return rc;
-    rc = pkv_paged_attention_decode(buf->q_dev, k_pool, v_pool, md + 4 * n, md + n, n, num_q_heads, num_kv_heads,
-                                    head_dim, num_blocks, max_blocks_per_seq, block_size, scale, dtype,
-                                    partition_tokens, workspace, workspace_bytes, buf->out_dev, stream);
+    rc = pkv_append_and_decode(buf->k_dev, buf->v_dev, md, n, buf->q_dev, k_pool, v_pool, md + 4 * n, md + n, n,
+                               num_q_heads, num_kv_heads, head_dim, num_blocks, max_blocks_per_seq, block_size, scale,
+                               dtype, partition_tokens, workspace, workspace_bytes, buf->out_dev, stream);
   }
   if (rc) return rc;
   if (buf->h2d_stream || buf->d2h_stream) {
