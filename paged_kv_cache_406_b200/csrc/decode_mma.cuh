@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(kMmaThreads) decode_mma_kernel(const DecodePar
     uint32_t ph = 0, issued = 0;
     uint32_t cg = 0;      // CTA-wide chunk index of the unit's first chunk
     bool ok = true;
-    for (int w = blockIdx.x; w < n_work && ok; w += gridDim.x) {
+    for (int r = 0, w = unit_index(0); w < n_work && ok; w = unit_index(++r)) {
       const WorkUnit u = load_unit(p, w);
       const int32_t* trow = p.block_tables + static_cast<int64_t>(u.b) * p.max_blocks + (u.t0 >> bs_shift);
       const int nch = (u.t1 - u.t0 + kChunkTokens - 1) / kChunkTokens;
@@ -225,7 +225,7 @@ __global__ void __launch_bounds__(kMmaThreads) decode_mma_kernel(const DecodePar
   uint32_t c = 0;
   int iter = 0;
   bool ok = true;
-  for (int w = blockIdx.x; w < n_work; w += gridDim.x, ++iter) {
+  for (int w = unit_index(0); w < n_work; w = unit_index(++iter)) {
     const WorkUnit u = load_unit(p, w);
     const int nch = (u.t1 - u.t0 + kChunkTokens - 1) / kChunkTokens;
 
