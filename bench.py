@@ -50,8 +50,8 @@ EVENT_EVERY = 16
 # on (kernel_source_sha()).  A pin whose hash no longer matches is reported as
 # null.
 TRAFFIC = {
-    "llama3_8b": (606710016, "eb907b967a95bff5"),
-    "llama3_8b_fp8": (307467008, "eb907b967a95bff5"),
+    "llama3_8b": (606696320, "85a57a9f50886783"),
+    "llama3_8b_fp8": (307867264, "85a57a9f50886783"),
 }
 # the same for one pkv_paged_attention_prefill call (prefill_tc_kernel), keyed
 # by the hash of the prefill sources (kernel_source_sha(PREFILL_SOURCES))
