@@ -15,7 +15,7 @@
 //   S_j = Q · K_jᵀ        tcgen05.mma, 128x128x128, A and B from shared memory,
 //                         fp32 in tensor memory
 //   P_j = 2^(S_j·scale·log2e - m)   4 softmax warps, one row per thread,
-//                         written back over S_j as bf16 (or f16) hi + lo
+//                         written back over S_j as bf16 hi + lo, or one f16
 //   O  += P_j · V_j       tcgen05.mma, A (P) from tensor memory, B (V) from
 //                         shared memory
 //
@@ -23,7 +23,8 @@
 // warps 4 and 5 TMA producers (K, V), warp 6 MMA issuer (lane 0) and TMEM
 // owner.  Tensor
 // memory (512 columns): three S / P buffers at columns 0, 128 and 256 (P hi
-// in the first 64 columns of its buffer, P lo in the next 64), O at 384.
+// in the first 64 columns of its buffer, P lo in the next 64; a single f16 P
+// in the first 64), O at 384.
 // Shared memory: Q 32 KB and K and V rings of 32 KB stages.  Keeping P in
 // tensor memory spares shared memory 128 KB of traffic per chunk (P written
 // and read back), which bounded the first version of this kernel.
@@ -37,9 +38,12 @@
 // (only by more than 8 in log2 units), as in the decode kernels; a move
 // rescales that row's O in tensor memory after PV_{j-1} has finished.
 //
-// P precision: a single bf16 P misses the 2e-3 output tolerance at early
-// positions (few keys of comparable weight); hi + lo halves keep it within
-// about 1e-5, at the cost of a second P·V pass (one MMA per half).
+// P precision: a single bf16 P (8 significant bits) misses the 2e-3 output
+// tolerance at early positions (few keys of comparable weight), so for bf16
+// pools P is stored as hi + lo halves (about 16 bits, within about 1e-5) at
+// the cost of a second P·V pass (one MMA per half).  For f16 pools a single
+// f16 P (11 bits: weights within 2^-11 relative, outputs within about 5e-4
+// of the output scale) meets the tolerance, and P·V is one pass.
 #pragma once
 
 #include <cuda.h>
@@ -202,6 +206,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
   constexpr int QT = pf::kRows / G;  // query tokens per tile
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+  constexpr int kParts = kBf16 ? 2 : 1;  // P halves: hi + lo (bf16) or one f16 P
 
   // ---- the tile: (sequence b, KV head g, tile of QT query tokens).  The
   // tiles of one (b, g) are launched next to each other, most keys first, so
@@ -345,7 +350,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         const uint32_t vst = base + pf::kOffV + s * pf::kTile;
         const uint32_t pt = tmem + pf::kColS + (j % pf::kSBufs) * pf::kKeys;  // P hi: 64 columns, then P lo
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
+        for (int part = 0; part < kParts; ++part) {
 #pragma unroll
           for (int kk = 0; kk < pf::kKeys / 16; ++kk) {
             const uint32_t bv = vst + kk * 16 * 128;  // 16 keys of 128-byte rows
@@ -437,11 +442,21 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
           x[c + 1] = fast_exp2(a.y);
           sm[(c >> 1) & 3] = __fadd2_rn(sm[(c >> 1) & 3], make_float2(x[c], x[c + 1]));
         }
-        uint32_t hi[32], lo[32];
+        if constexpr (kBf16) {
+          uint32_t hi[32], lo[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) split_hi_lo<T>(x[64 * h + 2 * c], x[64 * h + 2 * c + 1], hi[c], lo[c]);
-        tc::st_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + 32 * h, hi);
-        tc::st_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + pf::kKeys / 2 + 32 * h, lo);
+          for (int c = 0; c < 32; ++c) split_hi_lo<T>(x[64 * h + 2 * c], x[64 * h + 2 * c + 1], hi[c], lo[c]);
+          tc::st_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + 32 * h, hi);
+          tc::st_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + pf::kKeys / 2 + 32 * h, lo);
+        } else {
+          uint32_t ph[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const __half2 v = __floats2half2_rn(x[64 * h + 2 * c], x[64 * h + 2 * c + 1]);
+            ph[c] = *reinterpret_cast<const uint32_t*>(&v);
+          }
+          tc::st_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + 32 * h, ph);
+        }
       }
       const float2 s01 = __fadd2_rn(sm[0], sm[1]), s23 = __fadd2_rn(sm[2], sm[3]);
       const float2 st = __fadd2_rn(s01, s23);

@@ -99,19 +99,22 @@ def test_prefill_matches_oracle(dtype, g, bs):
     assert_close(out, case.oracle(), dtype, f"prefill {dtype} G{g} bs{bs}")
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
 @pytest.mark.parametrize("g", [1, 4])
-def test_long_context_and_many_tiles(g):
+def test_long_context_and_many_tiles(g, dtype):
+    """bf16 pools take P as hi + lo halves, f16 pools a single f16 P."""
     lens, q_lens = [1500, 700], [300, 700]
-    case = PrefillCase(lens, q_lens, 2 * g, 2, 16, "bf16", _seed("long", g))
-    assert_close(case.run(), case.oracle(), "bf16", f"long G{g}")
+    case = PrefillCase(lens, q_lens, 2 * g, 2, 16, dtype, _seed("long", g, dtype))
+    assert_close(case.run(), case.oracle(), dtype, f"long {dtype} G{g}")
 
 
-def test_growing_scores_rescale_the_accumulator():
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_growing_scores_rescale_the_accumulator(dtype):
     """Scores rise along the sequence so the running max moves by more than
     the lazy threshold in many chunks: every such move rescales O."""
-    case = PrefillCase([900, 400], [200, 400], 8, 2, 16, "bf16", _seed("ramp"), k_ramp=12.0)
+    case = PrefillCase([900, 400], [200, 400], 8, 2, 16, dtype, _seed("ramp", dtype), k_ramp=12.0)
     ref = case.oracle()
-    assert_close(case.run(), ref, "bf16", "rescaled")
+    assert_close(case.run(), ref, dtype, f"rescaled {dtype}")
 
 
 def test_one_row_chunks_agree_with_decode():
