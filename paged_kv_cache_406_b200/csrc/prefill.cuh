@@ -375,7 +375,6 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     // ------------------------------ softmax warps ------------------------------
     const int r = threadIdx.x;  // tile row and TMEM lane
     const int tok = tok0 + r / G;
-    const bool valid = tok < n;
     const int pos = min(ctx + tok, L - 1);  // rows past the chunk end compute a copy of the last row
     const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     unsigned char* vzero = smem + pf::kOffV;
@@ -505,18 +504,33 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     if (ok) {
       tc::fence_after_sync();
       const float inv = 1.f / l;
-      float* orow = p.out + (static_cast<int64_t>(q0 + tok) * p.num_q_heads + g * G + r % G) * pf::kHeadDim;
+      // O goes out through shared memory (Q and the K ring are free once every
+      // MMA is done): each thread parks its row, then each warp writes its 32
+      // rows one 512-byte row per store instruction, instead of 32 rows per
+      // instruction straight from the tensor-memory layout.  The 16-byte piece
+      // c of row r sits at slot c ^ (r mod 8) of the row, so the row-wise
+      // writes and the piece-wise reads are both free of bank conflicts.
+      float4* stage = reinterpret_cast<float4*>(smem + pf::kOffQ);
+      float4* srow = stage + r * (pf::kHeadDim / 4);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t o[32];
         tc::ld_32x32b_x32(trow + pf::kColO + 32 * q, o);
         tc::wait_ld();
-        if (valid) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(orow + 32 * q + i) =
-                make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
-                            __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+        for (int i = 0; i < 8; ++i)
+          srow[(8 * q + i) ^ (r & 7)] =
+              make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
+                          __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+      }
+      __syncwarp();
+      for (int k = 0; k < 32; ++k) {
+        const int rr = warp * 32 + k;  // a row this warp parked
+        const int tk = tok0 + rr / G;
+        if (tk < n) {                  // rows past the chunk end are not written
+          float4* orow = reinterpret_cast<float4*>(
+              p.out + (static_cast<int64_t>(q0 + tk) * p.num_q_heads + g * G + rr % G) * pf::kHeadDim);
+          orow[lane] = stage[rr * (pf::kHeadDim / 4) + (lane ^ (rr & 7))];
         }
       }
     } else if (lane == 0) {
