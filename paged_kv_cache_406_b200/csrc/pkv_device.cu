@@ -806,6 +806,35 @@ int make_prefill_pool_map(CUtensorMap* m, const void* pool, int dtype, int64_t r
   return PKV_OK;
 }
 
+// Tile counters of the persistent prefill kernel.  A launch draws its tiles
+// from one slot and its last CTA re-arms the slot to zero; successive
+// launches take successive slots, so launches that overlap on the GPU (up to
+// kPrefillSlots of them) never share one.
+constexpr int kPrefillSlots = 64;
+__device__ unsigned int g_prefill_tiles[kPrefillSlots][2];
+
+int prefill_counter(unsigned int** out) {
+  static std::mutex mu;
+  static void* base[kMaxDevices] = {};
+  static std::atomic<unsigned> next{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev >= kMaxDevices) return fail(PKV_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kMaxDevices);
+  {
+    std::lock_guard<std::mutex> g(mu);
+    if (!base[dev]) {
+      void* ptr = nullptr;
+      e = cudaGetSymbolAddress(&ptr, g_prefill_tiles);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(prefill tile counters)");
+      base[dev] = ptr;
+    }
+  }
+  const unsigned slot = next.fetch_add(1, std::memory_order_relaxed) % kPrefillSlots;
+  *out = static_cast<unsigned int*>(base[dev]) + 2 * slot;
+  return PKV_OK;
+}
+
 template <typename T, int G>
 int launch_prefill(const pkv::PrefillParams& p, const void* q, const void* k_pool, const void* v_pool, int dtype,
                    cudaStream_t stream) {
@@ -827,8 +856,12 @@ int launch_prefill(const pkv::PrefillParams& p, const void* q, const void* k_poo
   if (rc) return rc;
   rc = make_prefill_pool_map(&mv, v_pool, dtype, rows, p.block_size);
   if (rc) return rc;
-  const int64_t grid = int64_t(p.n_tiles) * p.num_seqs * p.num_kv_heads;
-  kern<<<static_cast<unsigned>(grid), pkv::pf::kThreads, pkv::pf::kSmemBytes, stream>>>(p, mq, mk, mv);
+  const int64_t tiles = int64_t(p.n_tiles) * p.num_seqs * p.num_kv_heads;
+  const int64_t grid = std::min<int64_t>(sm_count(dev), tiles);  // persistent: one CTA per SM
+  unsigned int* ctr = nullptr;
+  rc = prefill_counter(&ctr);
+  if (rc) return rc;
+  kern<<<static_cast<unsigned>(grid), pkv::pf::kThreads, pkv::pf::kSmemBytes, stream>>>(p, mq, mk, mv, ctr);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
   return pkv::ok();

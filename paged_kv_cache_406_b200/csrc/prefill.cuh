@@ -202,34 +202,12 @@ __device__ __forceinline__ float exp2_fma(float x) {
 template <typename T, int G>
 __global__ void __launch_bounds__(pf::kThreads, 1)
     prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_q,
-                      const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v) {
+                      const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                      unsigned int* __restrict__ tile_ctr) {
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
   constexpr int QT = pf::kRows / G;  // query tokens per tile
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr int kParts = kBf16 ? 2 : 1;  // P halves: hi + lo (bf16) or one f16 P
-
-  // ---- the tile: (sequence b, KV head g, tile of QT query tokens).  The
-  // tiles of one (b, g) are launched next to each other, most keys first, so
-  // the CTAs in flight at any time share a few sequences' K/V in L2 (launching
-  // one tile index of every (b, g) together re-read K/V from DRAM about 7x) ----
-  const int bg = static_cast<int>(blockIdx.x) / p.n_tiles;
-  const int tile = p.n_tiles - 1 - static_cast<int>(blockIdx.x) % p.n_tiles;
-  const int b = bg / p.num_kv_heads, g = bg % p.num_kv_heads;
-  const int q0 = p.q_start[b], q1 = p.q_start[b + 1];
-  const int n = q1 - q0, L = p.seq_lens[b];
-  if (n < 0 || q0 < 0 || q1 > p.num_q_tokens || n > L || n > p.max_q_len ||
-      L > p.max_blocks * p.block_size) {
-    if (threadIdx.x == 0 && tile == 0) record_error(PKV_ERR_INVALID_ARG);
-    return;
-  }
-  const int tok0 = tile * QT;  // chunk-relative first token of the tile
-  if (tok0 >= n) return;       // uniform across the CTA: nothing allocated yet
-  const int ctx = L - n;
-  const int pos_min = ctx + tok0;
-  const int pos_max = min(L - 1, ctx + tok0 + QT - 1);
-  const int nc = pos_max / pf::kKeys + 1;  // key chunks this tile attends to
-  const int BS = p.block_size;
-  const int nblk = (L + BS - 1) / BS;
 
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -237,6 +215,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + pf::kOffBar);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + pf::kNumBars);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + pf::kNumBars) + 1;
+  volatile int* tile_slot = reinterpret_cast<volatile int*>(bars + pf::kNumBars) + 2;  // two slots
   auto bar = [&](int i) { return smem_addr(bars + i); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -249,301 +228,360 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     tc::tmem_alloc(smem_addr(tmem_slot), pf::kTmemCols);
     tc::tmem_relinquish();
   }
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
-  const uint32_t tmem = *tmem_slot;
+  if (warp == pf::kProducerK && lane == 0) {
+    prefetch_tensormap(&tmap_q);
+    prefetch_tensormap(&tmap_k);
+    prefetch_tensormap(&tmap_v);
+  }
+  const int total = p.n_tiles * p.num_seqs * p.num_kv_heads;
 
-  if (warp == pf::kProducerK || warp == pf::kProducerV) {
-    // ----------------------------- TMA producers -----------------------------
-    // One warp streams K chunks, the other V chunks, each through its own
-    // ring: K runs ahead of V (q·Kᵀ of chunk j+2 is issued right after P·V
-    // of chunk j, while V's stages free only as P·V completes; a single
-    // producer alternating K and V held K behind V's refills).
-    const int kv = warp == pf::kProducerV ? 1 : 0;
-    bool ok = true;
-    if (lane == 0 && kv == 0) {
-      prefetch_tensormap(&tmap_q);
-      prefetch_tensormap(&tmap_k);
-      prefetch_tensormap(&tmap_v);
-      // Q tile: rows token * G + h, one box per head_dim half
-      mbar_arrive_expect_tx(bar(pf::kQFull), pf::kTile);
-      tma_load_4d(base + pf::kOffQ, &tmap_q, 0, 0, g * G, q0 + tok0, bar(pf::kQFull));
-      tma_load_4d(base + pf::kOffQ + pf::kSlab, &tmap_q, 0, 1, g * G, q0 + tok0, bar(pf::kQFull));
+  // Persistent CTAs (one per SM) take tiles from a counter until it passes
+  // the last one: a CTA's tensor memory, barriers and tensor maps are set up
+  // once, and no CTA launch separates two tiles on an SM.  Tile t is the
+  // (sequence b, KV head g, tile of QT query tokens) of the launch order used
+  // before: the tiles of one (b, g) come one after another, most keys first,
+  // so the tiles in flight at any time share a few sequences' K/V in L2
+  // (taking one tile index of every (b, g) together re-read K/V from DRAM
+  // about 7x); taking them from a counter balances the SMs as they finish.
+  // The barriers keep counting phases across tiles: gc is the number of key
+  // chunks, ti the number of tiles this CTA has done before the current one
+  // (the same in every warp), and chunk j of a tile is chunk gc + j of the CTA.
+  int gc = 0, ti = 0;
+  int issued = 0, q_issued = 0;  // producers: fills issued (chunks, Q tiles) in the CTA's count
+  for (int it = 0;; ++it) {
+    if (threadIdx.x == 0) {
+      const unsigned ticket = *abort_flag ? static_cast<unsigned>(total) : atomicAdd(tile_ctr, 1u);
+      tile_slot[it & 1] = ticket >= static_cast<unsigned>(total) ? total : static_cast<int>(ticket);
     }
-    const int32_t* trow = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
-    const int nbc = pf::kKeys / BS;                              // blocks per chunk
-    const uint32_t box_bytes = static_cast<uint32_t>(BS) * 128;  // one block, one head_dim half
-    int issued = 0;  // chunks whose fill this warp issued
-    const uint32_t full0 = bar(kv ? pf::kVFull : pf::kKFull), empty0 = bar(kv ? pf::kVEmpty : pf::kKEmpty);
-    const void* map = kv ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k);
-    const uint32_t ring = base + (kv ? pf::kOffV : pf::kOffK);
-    for (int j = 0; j < nc && ok; ++j) {
-      const int s = j % pf::kStages;
-      const uint32_t ph = ((j / pf::kStages) & 1) ^ 1;
-      const int jb = j * nbc;
-      const int nload = min(nbc, nblk - jb);  // blocks past the sequence end are not read
-      int phys = 0;
-      if (lane < nload) {
-        phys = trow[jb + lane];
-        if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_blocks)) {
-          record_error(PKV_ERR_BAD_BLOCK);
-          phys = 0;
-        }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const int t = tile_slot[it & 1];
+    if (t >= total) break;
+    const uint32_t tmem = *tmem_slot;
+
+    const int bg = t / p.n_tiles;
+    const int tile = p.n_tiles - 1 - t % p.n_tiles;
+    const int b = bg / p.num_kv_heads, g = bg % p.num_kv_heads;
+    const int q0 = p.q_start[b], q1 = p.q_start[b + 1];
+    const int n = q1 - q0, L = p.seq_lens[b];
+    if (n < 0 || q0 < 0 || q1 > p.num_q_tokens || n > L || n > p.max_q_len ||
+        L > p.max_blocks * p.block_size) {
+      if (threadIdx.x == 0 && tile == 0) record_error(PKV_ERR_INVALID_ARG);
+      continue;
+    }
+    const int tok0 = tile * QT;  // chunk-relative first token of the tile
+    if (tok0 >= n) continue;     // uniform across the CTA
+    const int ctx = L - n;
+    const int pos_min = ctx + tok0;
+    const int pos_max = min(L - 1, ctx + tok0 + QT - 1);
+    const int nc = pos_max / pf::kKeys + 1;  // key chunks this tile attends to
+    const int BS = p.block_size;
+    const int nblk = (L + BS - 1) / BS;
+
+    if (warp == pf::kProducerK || warp == pf::kProducerV) {
+      // ----------------------------- TMA producers -----------------------------
+      // One warp streams K chunks, the other V chunks, each through its own
+      // ring: K runs ahead of V (q·Kᵀ of chunk j+2 is issued right after P·V
+      // of chunk j, while V's stages free only as P·V completes; a single
+      // producer alternating K and V held K behind V's refills).
+      const int kv = warp == pf::kProducerV ? 1 : 0;
+      bool ok = true;
+      q_issued = ti + 1;
+      if (lane == 0 && kv == 0) {
+        // Q tile: rows token * G + h, one box per head_dim half
+        mbar_arrive_expect_tx(bar(pf::kQFull), pf::kTile);
+        tma_load_4d(base + pf::kOffQ, &tmap_q, 0, 0, g * G, q0 + tok0, bar(pf::kQFull));
+        tma_load_4d(base + pf::kOffQ + pf::kSlab, &tmap_q, 0, 1, g * G, q0 + tok0, bar(pf::kQFull));
       }
-      const int32_t y = (phys * p.num_kv_heads + g) * BS;
-      const uint32_t full = full0 + 8 * s;
-      ok = __all_sync(pf::kAll, pf_wait(empty0 + 8 * s, ph, abort_flag));
-      if (!ok) break;
-      if (lane == 0) mbar_arrive_expect_tx(full, static_cast<uint32_t>(nload) * 2u * box_bytes);
-      __syncwarp();
-      if (lane < nload) {
-        const uint32_t dst = ring + s * pf::kTile + lane * box_bytes;
-        tma_load_3d_nohint(dst, map, 0, y, 0, full);
-        tma_load_3d_nohint(dst + pf::kSlab, map, 0, y, 1, full);
-      }
-      ++issued;
-    }
-    if (!ok && lane == 0) {
-      record_error(PKV_ERR_DEVICE_TIMEOUT);
-      *abort_flag = 1;
-    }
-    // no copy may still be landing when the CTA exits: wait (bounded) for the
-    // last fill of each stage and for Q
-    if (lane == 0) {
-      if (kv == 0) drain_wait(bar(pf::kQFull), 0);
-      for (int s = 0; s < pf::kStages && s < issued; ++s) {
-        const int last = s + (issued - 1 - s) / pf::kStages * pf::kStages;  // last chunk that used stage s
-        drain_wait(full0 + 8 * s, (last / pf::kStages) & 1);
-      }
-    }
-    __syncwarp();
-  } else if (warp == pf::kMmaWarp) {
-    // ------------------------------- MMA issuer -------------------------------
-    if (lane == 0) {
-      const uint32_t id_s = tc::idesc_f16(kBf16, false, pf::kRows, pf::kKeys);
-      const uint32_t id_o = tc::idesc_f16(kBf16, true, pf::kRows, pf::kHeadDim);
-      auto issue_s = [&](int j) -> bool {
-        const int s = j % pf::kStages;
-        if (!pf_wait(bar(pf::kKFull + s), (j / pf::kStages) & 1, abort_flag)) return false;
-        tc::fence_after_sync();
-        const uint32_t kst = base + pf::kOffK + s * pf::kTile;
-#pragma unroll
-        for (int kk = 0; kk < pf::kHeadDim / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * pf::kSlab + (kk & 3) * 32;
-          tc::mma_f16_ss(tmem + pf::kColS + (j % pf::kSBufs) * pf::kKeys,
-                         tc::sw128_desc(base + pf::kOffQ + off, 16, 1024), tc::sw128_desc(kst + off, 16, 1024), id_s,
-                         kk > 0 ? 1u : 0u);
-        }
-        tc::commit(bar(pf::kKEmpty + s));
-        tc::commit(bar(pf::kSFull + j % pf::kSBufs));
-        return true;
-      };
-      bool ok = pf_wait(bar(pf::kQFull), 0, abort_flag);
-      for (int j = 0; j < pf::kSBufs && j < nc && ok; ++j) ok = issue_s(j);
+      const int32_t* trow = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
+      const int nbc = pf::kKeys / BS;                              // blocks per chunk
+      const uint32_t box_bytes = static_cast<uint32_t>(BS) * 128;  // one block, one head_dim half
+      const uint32_t full0 = bar(kv ? pf::kVFull : pf::kKFull), empty0 = bar(kv ? pf::kVEmpty : pf::kKEmpty);
+      const void* map = kv ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k);
+      const uint32_t ring = base + (kv ? pf::kOffV : pf::kOffK);
       for (int j = 0; j < nc && ok; ++j) {
-        const int s = j % pf::kStages;
-        ok = pf_wait(bar(pf::kPFull + j % pf::kSBufs), (j / pf::kSBufs) & 1, abort_flag) &&
-             pf_wait(bar(pf::kVFull + s), (j / pf::kStages) & 1, abort_flag);
-        if (!ok) break;
-        tc::fence_after_sync();
-        const uint32_t vst = base + pf::kOffV + s * pf::kTile;
-        const uint32_t pt = tmem + pf::kColS + (j % pf::kSBufs) * pf::kKeys;  // P hi: 64 columns, then P lo
-#pragma unroll
-        for (int part = 0; part < kParts; ++part) {
-#pragma unroll
-          for (int kk = 0; kk < pf::kKeys / 16; ++kk) {
-            const uint32_t bv = vst + kk * 16 * 128;  // 16 keys of 128-byte rows
-            tc::mma_f16_ts(tmem + pf::kColO, pt + part * (pf::kKeys / 2) + kk * 8, tc::sw128_desc(bv, pf::kSlab, 1024),
-                           id_o, (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
+        const int s = (gc + j) % pf::kStages;
+        const uint32_t ph = (((gc + j) / pf::kStages) & 1) ^ 1;
+        const int jb = j * nbc;
+        const int nload = min(nbc, nblk - jb);  // blocks past the sequence end are not read
+        int phys = 0;
+        if (lane < nload) {
+          phys = trow[jb + lane];
+          if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_blocks)) {
+            record_error(PKV_ERR_BAD_BLOCK);
+            phys = 0;
           }
         }
-        tc::commit(bar(pf::kVEmpty + s));
-        tc::commit(bar(pf::kPVDone + j % pf::kSBufs));
-        if (j + pf::kSBufs < nc) ok = issue_s(j + pf::kSBufs);
+        const int32_t y = (phys * p.num_kv_heads + g) * BS;
+        const uint32_t full = full0 + 8 * s;
+        ok = __all_sync(pf::kAll, pf_wait(empty0 + 8 * s, ph, abort_flag));
+        if (!ok) break;
+        if (lane == 0) mbar_arrive_expect_tx(full, static_cast<uint32_t>(nload) * 2u * box_bytes);
+        __syncwarp();
+        if (lane < nload) {
+          const uint32_t dst = ring + s * pf::kTile + lane * box_bytes;
+          tma_load_3d_nohint(dst, map, 0, y, 0, full);
+          tma_load_3d_nohint(dst + pf::kSlab, map, 0, y, 1, full);
+        }
+        issued = gc + j + 1;
       }
-      if (!ok) {
+      if (!ok && lane == 0) {
         record_error(PKV_ERR_DEVICE_TIMEOUT);
         *abort_flag = 1;
       }
-      // every MMA issued so far completes before tensor memory is freed
-      tc::commit(bar(pf::kDrain));
-      drain_wait(bar(pf::kDrain), 0);
-    }
-    __syncwarp();
-  } else {
-    // ------------------------------ softmax warps ------------------------------
-    const int r = threadIdx.x;  // tile row and TMEM lane
-    const int tok = tok0 + r / G;
-    const int pos = min(ctx + tok, L - 1);  // rows past the chunk end compute a copy of the last row
-    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    unsigned char* vzero = smem + pf::kOffV;
-    const float sl = p.scale_log2;
-    float m_used = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < nc && ok; ++j) {
-      const int sb = j % pf::kSBufs;     // S / P buffer
-      const int s = j % pf::kStages;     // K / V stage
-      ok = __all_sync(pf::kAll, pf_wait(bar(pf::kSFull + sb), (j / pf::kSBufs) & 1, abort_flag));
-      if (!ok) break;
-      tc::fence_after_sync();
-      float x[pf::kKeys];  // raw scores q·k of this row's 128 keys
-      {
-        uint32_t raw[4][32];
+      __syncwarp();
+    } else if (warp == pf::kMmaWarp) {
+      // ------------------------------- MMA issuer -------------------------------
+      if (lane == 0) {
+        const uint32_t id_s = tc::idesc_f16(kBf16, false, pf::kRows, pf::kKeys);
+        const uint32_t id_o = tc::idesc_f16(kBf16, true, pf::kRows, pf::kHeadDim);
+        auto issue_s = [&](int j) -> bool {  // j: chunk of the tile; gc + j: chunk of the CTA
+          const int s = (gc + j) % pf::kStages;
+          if (!pf_wait(bar(pf::kKFull + s), ((gc + j) / pf::kStages) & 1, abort_flag)) return false;
+          tc::fence_after_sync();
+          const uint32_t kst = base + pf::kOffK + s * pf::kTile;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) tc::ld_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + 32 * q, raw[q]);
-        tc::wait_ld();
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-#pragma unroll
-          for (int i = 0; i < 32; ++i) x[32 * q + i] = __uint_as_float(raw[q][i]);
-      }
-      const int key0 = j * pf::kKeys;
-      if (key0 + pf::kKeys - 1 > pos_min) {  // the diagonal: keys after a row's position are hidden
-#pragma unroll
-        for (int c = 0; c < pf::kKeys; ++c) x[c] = key0 + c <= pos ? x[c] : -INFINITY;
-      }
-      // row max with three-input maxima in four independent chains; the
-      // scale is positive, so the max of the scaled scores is the scaled max
-      float mx[4] = {x[0], x[1], x[2], x[3]};
-#pragma unroll
-      for (int c = 4; c + 8 <= pf::kKeys; c += 8) {
-        mx[0] = max3f(mx[0], x[c], x[c + 1]);
-        mx[1] = max3f(mx[1], x[c + 2], x[c + 3]);
-        mx[2] = max3f(mx[2], x[c + 4], x[c + 5]);
-        mx[3] = max3f(mx[3], x[c + 6], x[c + 7]);
-      }
-      mx[0] = max3f(mx[0], x[pf::kKeys - 4], x[pf::kKeys - 3]);
-      mx[1] = max3f(mx[1], x[pf::kKeys - 2], x[pf::kKeys - 1]);
-      const float mc = fmaxf(max3f(mx[0], mx[1], mx[2]), mx[3]) * sl;
-      float factor = 1.f;
-      bool resc = false;
-      if (j == 0) {
-        m_used = mc;  // key 0 is visible to every row: finite
-      } else if (mc > m_used + pf::kRescale) {
-        factor = fast_exp2(m_used - mc);
-        m_used = mc;
-        resc = true;
-      }
-      // exponentials (arguments and sums two lanes at a time, packed f32x2),
-      // each half of the row written as P hi and lo over S_j in tensor memory
-      // as soon as it is done (the stores complete while the next half is
-      // computed): key pair (2c, 2c+1) in column c (hi) and 64 + c (lo)
-      float2 sm[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(-m_used, -m_used);
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-#pragma unroll
-        for (int c = 64 * h; c < 64 * h + 64; c += 2) {
-          const float2 a = __ffma2_rn(make_float2(x[c], x[c + 1]), sl2, nm2);  // hidden keys: -inf -> 0
-          constexpr int kEvery = PKV_PREFILL_POLY_EVERY > 0 ? PKV_PREFILL_POLY_EVERY : 1;
-          x[c] = (PKV_PREFILL_POLY_EVERY > 0 && c % kEvery == kEvery - 1) ? exp2_fma(a.x) : fast_exp2(a.x);
-          x[c + 1] = fast_exp2(a.y);
-          sm[(c >> 1) & 3] = __fadd2_rn(sm[(c >> 1) & 3], make_float2(x[c], x[c + 1]));
-        }
-        if constexpr (kBf16) {
-          uint32_t hi[32], lo[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) split_hi_lo<T>(x[64 * h + 2 * c], x[64 * h + 2 * c + 1], hi[c], lo[c]);
-          tc::st_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + 32 * h, hi);
-          tc::st_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + pf::kKeys / 2 + 32 * h, lo);
-        } else {
-          uint32_t ph[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const __half2 v = __floats2half2_rn(x[64 * h + 2 * c], x[64 * h + 2 * c + 1]);
-            ph[c] = *reinterpret_cast<const uint32_t*>(&v);
+          for (int kk = 0; kk < pf::kHeadDim / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * pf::kSlab + (kk & 3) * 32;
+            tc::mma_f16_ss(tmem + pf::kColS + ((gc + j) % pf::kSBufs) * pf::kKeys,
+                           tc::sw128_desc(base + pf::kOffQ + off, 16, 1024), tc::sw128_desc(kst + off, 16, 1024), id_s,
+                           kk > 0 ? 1u : 0u);
           }
-          tc::st_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + 32 * h, ph);
+          tc::commit(bar(pf::kKEmpty + s));
+          tc::commit(bar(pf::kSFull + (gc + j) % pf::kSBufs));
+          return true;
+        };
+        bool ok = pf_wait(bar(pf::kQFull), ti & 1, abort_flag);
+        for (int j = 0; j < pf::kSBufs && j < nc && ok; ++j) ok = issue_s(j);
+        for (int j = 0; j < nc && ok; ++j) {
+          const int gj = gc + j;
+          const int s = gj % pf::kStages;
+          ok = pf_wait(bar(pf::kPFull + gj % pf::kSBufs), (gj / pf::kSBufs) & 1, abort_flag) &&
+               pf_wait(bar(pf::kVFull + s), (gj / pf::kStages) & 1, abort_flag);
+          if (!ok) break;
+          tc::fence_after_sync();
+          const uint32_t vst = base + pf::kOffV + s * pf::kTile;
+          const uint32_t pt = tmem + pf::kColS + (gj % pf::kSBufs) * pf::kKeys;  // P hi: 64 columns, then P lo
+#pragma unroll
+          for (int part = 0; part < kParts; ++part) {
+#pragma unroll
+            for (int kk = 0; kk < pf::kKeys / 16; ++kk) {
+              const uint32_t bv = vst + kk * 16 * 128;  // 16 keys of 128-byte rows
+              tc::mma_f16_ts(tmem + pf::kColO, pt + part * (pf::kKeys / 2) + kk * 8, tc::sw128_desc(bv, pf::kSlab, 1024),
+                             id_o, (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          tc::commit(bar(pf::kVEmpty + s));
+          tc::commit(bar(pf::kPVDone + gj % pf::kSBufs));
+          if (j + pf::kSBufs < nc) ok = issue_s(j + pf::kSBufs);
         }
+        if (!ok) {
+          record_error(PKV_ERR_DEVICE_TIMEOUT);
+          *abort_flag = 1;
+        }
+        // every MMA of the tile completes before O is read and before the next
+        // tile's loads reuse Q and the rings
+        tc::commit(bar(pf::kDrain));
+        drain_wait(bar(pf::kDrain), ti & 1);
       }
-      const float2 s01 = __fadd2_rn(sm[0], sm[1]), s23 = __fadd2_rn(sm[2], sm[3]);
-      const float2 st = __fadd2_rn(s01, s23);
-      l = l * factor + (st.x + st.y);
-
-      if (__any_sync(pf::kAll, resc)) {
-        // O still accumulates PV_{j-1}: wait for it, then rescale the row.
-        // PV_{j-1} commits to the barrier of its buffer, whose previous
-        // phase (PV_{j-4}) was covered by S_j's commit, so the parity wait
-        // cannot see an older phase.
-        const int pj = j - 1;
-        ok = __all_sync(pf::kAll, pf_wait(bar(pf::kPVDone + pj % pf::kSBufs), (pj / pf::kSBufs) & 1, abort_flag));
+      __syncwarp();
+    } else {
+      // ------------------------------ softmax warps ------------------------------
+      const int r = threadIdx.x;  // tile row and TMEM lane
+      const int tok = tok0 + r / G;
+      const int pos = min(ctx + tok, L - 1);  // rows past the chunk end compute a copy of the last row
+      const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+      unsigned char* vzero = smem + pf::kOffV;
+      const float sl = p.scale_log2;
+      float m_used = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < nc && ok; ++j) {
+        const int gj = gc + j;              // chunk of the CTA
+        const int sb = gj % pf::kSBufs;     // S / P buffer
+        const int s = gj % pf::kStages;     // K / V stage
+        ok = __all_sync(pf::kAll, pf_wait(bar(pf::kSFull + sb), (gj / pf::kSBufs) & 1, abort_flag));
         if (!ok) break;
         tc::fence_after_sync();
+        float x[pf::kKeys];  // raw scores q·k of this row's 128 keys
+        {
+          uint32_t raw[4][32];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) tc::ld_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + 32 * q, raw[q]);
+          tc::wait_ld();
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[32 * q + i] = __uint_as_float(raw[q][i]);
+        }
+        const int key0 = j * pf::kKeys;
+        if (key0 + pf::kKeys - 1 > pos_min) {  // the diagonal: keys after a row's position are hidden
+#pragma unroll
+          for (int c = 0; c < pf::kKeys; ++c) x[c] = key0 + c <= pos ? x[c] : -INFINITY;
+        }
+        // row max with three-input maxima in four independent chains; the
+        // scale is positive, so the max of the scaled scores is the scaled max
+        float mx[4] = {x[0], x[1], x[2], x[3]};
+#pragma unroll
+        for (int c = 4; c + 8 <= pf::kKeys; c += 8) {
+          mx[0] = max3f(mx[0], x[c], x[c + 1]);
+          mx[1] = max3f(mx[1], x[c + 2], x[c + 3]);
+          mx[2] = max3f(mx[2], x[c + 4], x[c + 5]);
+          mx[3] = max3f(mx[3], x[c + 6], x[c + 7]);
+        }
+        mx[0] = max3f(mx[0], x[pf::kKeys - 4], x[pf::kKeys - 3]);
+        mx[1] = max3f(mx[1], x[pf::kKeys - 2], x[pf::kKeys - 1]);
+        const float mc = fmaxf(max3f(mx[0], mx[1], mx[2]), mx[3]) * sl;
+        float factor = 1.f;
+        bool resc = false;
+        if (j == 0) {
+          m_used = mc;  // key 0 is visible to every row: finite
+        } else if (mc > m_used + pf::kRescale) {
+          factor = fast_exp2(m_used - mc);
+          m_used = mc;
+          resc = true;
+        }
+        // exponentials (arguments and sums two lanes at a time, packed f32x2),
+        // each half of the row written as P hi and lo over S_j in tensor memory
+        // as soon as it is done (the stores complete while the next half is
+        // computed): key pair (2c, 2c+1) in column c (hi) and 64 + c (lo)
+        float2 sm[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(-m_used, -m_used);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int c = 64 * h; c < 64 * h + 64; c += 2) {
+            const float2 a = __ffma2_rn(make_float2(x[c], x[c + 1]), sl2, nm2);  // hidden keys: -inf -> 0
+            constexpr int kEvery = PKV_PREFILL_POLY_EVERY > 0 ? PKV_PREFILL_POLY_EVERY : 1;
+            x[c] = (PKV_PREFILL_POLY_EVERY > 0 && c % kEvery == kEvery - 1) ? exp2_fma(a.x) : fast_exp2(a.x);
+            x[c + 1] = fast_exp2(a.y);
+            sm[(c >> 1) & 3] = __fadd2_rn(sm[(c >> 1) & 3], make_float2(x[c], x[c + 1]));
+          }
+          if constexpr (kBf16) {
+            uint32_t hi[32], lo[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) split_hi_lo<T>(x[64 * h + 2 * c], x[64 * h + 2 * c + 1], hi[c], lo[c]);
+            tc::st_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + 32 * h, hi);
+            tc::st_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + pf::kKeys / 2 + 32 * h, lo);
+          } else {
+            uint32_t ph[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const __half2 v = __floats2half2_rn(x[64 * h + 2 * c], x[64 * h + 2 * c + 1]);
+              ph[c] = *reinterpret_cast<const uint32_t*>(&v);
+            }
+            tc::st_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + 32 * h, ph);
+          }
+        }
+        const float2 s01 = __fadd2_rn(sm[0], sm[1]), s23 = __fadd2_rn(sm[2], sm[3]);
+        const float2 st = __fadd2_rn(s01, s23);
+        l = l * factor + (st.x + st.y);
+
+        if (__any_sync(pf::kAll, resc)) {
+          // O still accumulates PV_{j-1}: wait for it, then rescale the row.
+          // PV_{j-1} commits to the barrier of its buffer, whose previous
+          // phase (PV_{j-4}) was covered by S_j's commit, so the parity wait
+          // cannot see an older phase.
+          const int pj = gj - 1;
+          ok = __all_sync(pf::kAll, pf_wait(bar(pf::kPVDone + pj % pf::kSBufs), (pj / pf::kSBufs) & 1, abort_flag));
+          if (!ok) break;
+          tc::fence_after_sync();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t o[32];
+            tc::ld_32x32b_x32(trow + pf::kColO + 32 * q, o);
+            tc::wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
+            tc::st_32x32b_x32(trow + pf::kColO + 32 * q, o);
+          }
+        }
+        const bool zero_v = key0 + pf::kKeys > L;
+        if (zero_v) {
+          // V rows past the sequence end hold stale or unwritten bytes: zero
+          // them so that P = 0 there cannot meet a NaN pattern
+          ok = __all_sync(pf::kAll, pf_wait(bar(pf::kVFull + s), (gj / pf::kStages) & 1, abort_flag));
+          if (!ok) break;
+          const int v0 = L - key0;
+          unsigned char* vst = vzero + s * pf::kTile;
+          for (int idx = r; idx < (pf::kKeys - v0) * 16; idx += 128) {
+            const int row = v0 + (idx >> 4), piece = idx & 15;
+            *reinterpret_cast<uint4*>(vst + (piece >> 3) * pf::kSlab + row * 128 + (piece & 7) * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();  // zeroed V rows visible to the tensor core
+        }
+        tc::wait_st();
+        tc::fence_before_sync();
+        mbar_arrive(bar(pf::kPFull + sb));
+      }
+      // the MMA warp commits kDrain after its last MMA: every P·V is then done
+      if (ok) ok = __all_sync(pf::kAll, pf_wait(bar(pf::kDrain), ti & 1, abort_flag));
+      if (ok) {
+        tc::fence_after_sync();
+        const float inv = 1.f / l;
+        // O goes out through shared memory (Q and the K ring are free once every
+        // MMA is done): each thread parks its row, then each warp writes its 32
+        // rows one 512-byte row per store instruction, instead of 32 rows per
+        // instruction straight from the tensor-memory layout.  The 16-byte piece
+        // c of row r sits at slot c ^ (r mod 8) of the row, so the row-wise
+        // writes and the piece-wise reads are both free of bank conflicts.
+        float4* stage = reinterpret_cast<float4*>(smem + pf::kOffQ);
+        float4* srow = stage + r * (pf::kHeadDim / 4);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint32_t o[32];
           tc::ld_32x32b_x32(trow + pf::kColO + 32 * q, o);
           tc::wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
-          tc::st_32x32b_x32(trow + pf::kColO + 32 * q, o);
+          for (int i = 0; i < 8; ++i)
+            srow[(8 * q + i) ^ (r & 7)] =
+                make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
+                            __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
         }
-      }
-      const bool zero_v = key0 + pf::kKeys > L;
-      if (zero_v) {
-        // V rows past the sequence end hold stale or unwritten bytes: zero
-        // them so that P = 0 there cannot meet a NaN pattern
-        ok = __all_sync(pf::kAll, pf_wait(bar(pf::kVFull + s), (j / pf::kStages) & 1, abort_flag));
-        if (!ok) break;
-        const int v0 = L - key0;
-        unsigned char* vst = vzero + s * pf::kTile;
-        for (int idx = r; idx < (pf::kKeys - v0) * 16; idx += 128) {
-          const int row = v0 + (idx >> 4), piece = idx & 15;
-          *reinterpret_cast<uint4*>(vst + (piece >> 3) * pf::kSlab + row * 128 + (piece & 7) * 16) =
-              make_uint4(0u, 0u, 0u, 0u);
+        __syncwarp();
+        for (int k = 0; k < 32; ++k) {
+          const int rr = warp * 32 + k;  // a row this warp parked
+          const int tk = tok0 + rr / G;
+          if (tk < n) {                  // rows past the chunk end are not written
+            float4* orow = reinterpret_cast<float4*>(
+                p.out + (static_cast<int64_t>(q0 + tk) * p.num_q_heads + g * G + rr % G) * pf::kHeadDim);
+            orow[lane] = stage[rr * (pf::kHeadDim / 4) + (lane ^ (rr & 7))];
+          }
         }
-        fence_proxy_async_smem();  // zeroed V rows visible to the tensor core
+      } else if (lane == 0) {
+        record_error(PKV_ERR_DEVICE_TIMEOUT);
+        *abort_flag = 1;
       }
-      tc::wait_st();
-      tc::fence_before_sync();
-      mbar_arrive(bar(pf::kPFull + sb));
     }
-    // the MMA warp commits kDrain after its last MMA: every P·V is then done
-    if (ok) ok = __all_sync(pf::kAll, pf_wait(bar(pf::kDrain), 0, abort_flag));
-    if (ok) {
-      tc::fence_after_sync();
-      const float inv = 1.f / l;
-      // O goes out through shared memory (Q and the K ring are free once every
-      // MMA is done): each thread parks its row, then each warp writes its 32
-      // rows one 512-byte row per store instruction, instead of 32 rows per
-      // instruction straight from the tensor-memory layout.  The 16-byte piece
-      // c of row r sits at slot c ^ (r mod 8) of the row, so the row-wise
-      // writes and the piece-wise reads are both free of bank conflicts.
-      float4* stage = reinterpret_cast<float4*>(smem + pf::kOffQ);
-      float4* srow = stage + r * (pf::kHeadDim / 4);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t o[32];
-        tc::ld_32x32b_x32(trow + pf::kColO + 32 * q, o);
-        tc::wait_ld();
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          srow[(8 * q + i) ^ (r & 7)] =
-              make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
-                          __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
-      }
-      __syncwarp();
-      for (int k = 0; k < 32; ++k) {
-        const int rr = warp * 32 + k;  // a row this warp parked
-        const int tk = tok0 + rr / G;
-        if (tk < n) {                  // rows past the chunk end are not written
-          float4* orow = reinterpret_cast<float4*>(
-              p.out + (static_cast<int64_t>(q0 + tk) * p.num_q_heads + g * G + rr % G) * pf::kHeadDim);
-          orow[lane] = stage[rr * (pf::kHeadDim / 4) + (lane ^ (rr & 7))];
-        }
-      }
-    } else if (lane == 0) {
-      record_error(PKV_ERR_DEVICE_TIMEOUT);
-      *abort_flag = 1;
+
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    gc += nc;
+    ++ti;
+  }  // tiles
+
+  // no copy may still be landing when the CTA exits (a timeout can leave
+  // fills unconsumed): wait (bounded) for the last fill of each stage and Q
+  if ((warp == pf::kProducerK || warp == pf::kProducerV) && lane == 0) {
+    const uint32_t full0 = bar(warp == pf::kProducerV ? pf::kVFull : pf::kKFull);
+    if (warp == pf::kProducerK && q_issued > 0) drain_wait(bar(pf::kQFull), (q_issued - 1) & 1);
+    for (int s = 0; s < pf::kStages && s < issued; ++s) {
+      const int last = s + (issued - 1 - s) / pf::kStages * pf::kStages;  // last chunk that used stage s
+      drain_wait(full0 + 8 * s, (last / pf::kStages) & 1);
     }
   }
-
-  tc::fence_before_sync();
-  __syncthreads();
-  if (warp == pf::kMmaWarp) {
-    tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, pf::kTmemCols);
+  if (warp == pf::kMmaWarp) tc::tmem_dealloc(*tmem_slot, pf::kTmemCols);
+  if (threadIdx.x == 0) {
+    // the last CTA to finish re-arms the counter for the next launch that
+    // uses this slot: every CTA has drawn its last ticket before it counts
+    // itself done
+    __threadfence();
+    if (atomicAdd(tile_ctr + 1, 1u) == gridDim.x - 1) {
+      atomicExch(tile_ctr, 0u);
+      atomicExch(tile_ctr + 1, 0u);
+    }
   }
 }
 
