@@ -84,7 +84,8 @@ constexpr int kThreads = 224;
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kTile;
 constexpr uint32_t kOffV = kOffK + kStages * kTile;
-constexpr uint32_t kOffBar = kOffV + kStages * kTile;
+constexpr uint32_t kOffStage = kOffV + kStages * kTile;  // output rows on their way out (128 x 512 B)
+constexpr uint32_t kOffBar = kOffStage + kRows * kHeadDim * 4;
 constexpr size_t kSmemBytes = kOffBar + 256 + 1024;  // barriers, flags; 1024 B alignment slack
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSBufs = 3;                    // S / P buffers in tensor memory
@@ -92,9 +93,18 @@ constexpr uint32_t kColS = 0, kColO = 384;   // S / P: 3 x 128 columns, O: 128
 constexpr float kRescale = 8.0f;
 constexpr unsigned kAll = 0xffffffffu;
 // mbarrier slots
-enum : int { kQFull = 0, kKFull = 1, kKEmpty = kKFull + kStages, kVFull = kKEmpty + kStages,
+enum : int { kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = kKFull + kStages, kVFull = kKEmpty + kStages,
              kVEmpty = kVFull + kStages, kSFull = kVEmpty + kStages, kPFull = kSFull + kSBufs,
-             kPVDone = kPFull + kSBufs, kDrain = kPVDone + kSBufs, kNumBars = kDrain + 1 };
+             kPVDone = kPFull + kSBufs, kODone = kPVDone + kSBufs, kOFree = kODone + 1, kTileReady = kOFree + 1,
+             kTileFree = kTileReady + 2, kDrain = kTileFree + 2, kNumBars = kDrain + 1 };
+static_assert(kNumBars * 8 + 16 <= 256, "barriers, flags and tile slots fit the reserved 256 bytes");
+// arrivals per phase: P-full and O-free by the 128 softmax threads, tile-free
+// by lane 0 of the V producer, the MMA warp and the four softmax warps
+__host__ __device__ constexpr uint32_t bar_count(int i) {
+  return (i >= kPFull && i < kPFull + kSBufs) || i == kOFree ? 128u
+         : (i >= kTileFree && i < kTileFree + 2)           ? 6u
+                                                             : 1u;
+}
 // S-full, P-full and PV-done are one barrier per S / P buffer: a buffer's
 // next phase needs the MMA warp to have moved on (S_{j+3} is issued after
 // PV_j), so no waiter can ever be a whole phase behind
@@ -220,7 +230,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < pf::kNumBars; ++i) mbar_init(bar(i), (i >= pf::kPFull && i < pf::kPFull + pf::kSBufs) ? 128u : 1u);
+    for (int i = 0; i < pf::kNumBars; ++i) mbar_init(bar(i), pf::bar_count(i));
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -233,66 +243,111 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     prefetch_tensormap(&tmap_k);
     prefetch_tensormap(&tmap_v);
   }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
   const int total = p.n_tiles * p.num_seqs * p.num_kv_heads;
 
-  // Persistent CTAs (one per SM) take tiles from a counter until it passes
-  // the last one: a CTA's tensor memory, barriers and tensor maps are set up
-  // once, and no CTA launch separates two tiles on an SM.  Tile t is the
-  // (sequence b, KV head g, tile of QT query tokens) of the launch order used
-  // before: the tiles of one (b, g) come one after another, most keys first,
-  // so the tiles in flight at any time share a few sequences' K/V in L2
-  // (taking one tile index of every (b, g) together re-read K/V from DRAM
-  // about 7x); taking them from a counter balances the SMs as they finish.
-  // The barriers keep counting phases across tiles: gc is the number of key
-  // chunks, ti the number of tiles this CTA has done before the current one
-  // (the same in every warp), and chunk j of a tile is chunk gc + j of the CTA.
-  int gc = 0, ti = 0;
-  int issued = 0, q_issued = 0;  // producers: fills issued (chunks, Q tiles) in the CTA's count
-  for (int it = 0;; ++it) {
-    if (threadIdx.x == 0) {
-      const unsigned ticket = *abort_flag ? static_cast<unsigned>(total) : atomicAdd(tile_ctr, 1u);
-      tile_slot[it & 1] = ticket >= static_cast<unsigned>(total) ? total : static_cast<int>(ticket);
-    }
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    const int t = tile_slot[it & 1];
-    if (t >= total) break;
-    const uint32_t tmem = *tmem_slot;
-
+  // Persistent CTAs (one per SM).  The K producer draws tile numbers from a
+  // counter and publishes each in one of two slots (tile-ready barrier); the
+  // other roles read it and hand the slot back (tile-free barrier).  Tile t
+  // is the (sequence b, KV head g, tile of QT query tokens) of the order: the
+  // tiles of one (b, g) one after another, most keys first, so the tiles in
+  // flight at any time share a few sequences' K/V in L2 (taking one tile
+  // index of every (b, g) together re-read K/V from DRAM about 7x); drawing
+  // them from a counter balances the SMs as they finish.  Each role moves on
+  // to the next tile as soon as its own part is done, so the next tile's Q
+  // and K loads and its first q·Kᵀ run during this tile's last P·V and
+  // output; only the next tile's first P·V waits for the output to have left
+  // tensor memory (O-free), and the next Q load for the last q·Kᵀ (Q-empty).
+  // The barriers count phases across tiles: gc is the number of key chunks
+  // and tv the number of tiles a role has done before the current one (the
+  // same sequence in every role); chunk j of a tile is chunk gc + j.
+  struct Tile {
+    int b, g, q0, n, L, tok0, ctx, pos_min, nc, nblk;
+    bool valid;
+  };
+  auto tile_of = [&](int t) {
+    Tile d{};
     const int bg = t / p.n_tiles;
     const int tile = p.n_tiles - 1 - t % p.n_tiles;
-    const int b = bg / p.num_kv_heads, g = bg % p.num_kv_heads;
-    const int q0 = p.q_start[b], q1 = p.q_start[b + 1];
-    const int n = q1 - q0, L = p.seq_lens[b];
-    if (n < 0 || q0 < 0 || q1 > p.num_q_tokens || n > L || n > p.max_q_len ||
-        L > p.max_blocks * p.block_size) {
-      if (threadIdx.x == 0 && tile == 0) record_error(PKV_ERR_INVALID_ARG);
-      continue;
+    d.b = bg / p.num_kv_heads;
+    d.g = bg % p.num_kv_heads;
+    d.q0 = p.q_start[d.b];
+    const int q1 = p.q_start[d.b + 1];
+    d.n = q1 - d.q0;
+    d.L = p.seq_lens[d.b];
+    d.tok0 = tile * QT;  // chunk-relative first token of the tile
+    const bool args_ok = !(d.n < 0 || d.q0 < 0 || q1 > p.num_q_tokens || d.n > d.L || d.n > p.max_q_len ||
+                           d.L > p.max_blocks * p.block_size);
+    if (!args_ok && tile == 0 && warp == pf::kProducerK && lane == 0) record_error(PKV_ERR_INVALID_ARG);
+    d.valid = args_ok && d.tok0 < d.n;
+    if (!d.valid) return d;
+    d.ctx = d.L - d.n;
+    d.pos_min = d.ctx + d.tok0;
+    const int pos_max = min(d.L - 1, d.ctx + d.tok0 + QT - 1);
+    d.nc = pos_max / pf::kKeys + 1;  // key chunks this tile attends to
+    d.nblk = (d.L + p.block_size - 1) / p.block_size;
+    return d;
+  };
+  // the tile number of round ti, for every role but the K producer (which
+  // publishes it): returns total when there are no more tiles (or on abort)
+  auto read_tile = [&](int ti) -> int {
+    int t = total;
+    if (lane == 0) {
+      if (pf_wait(bar(pf::kTileReady + (ti & 1)), (ti >> 1) & 1, abort_flag)) t = tile_slot[ti & 1];
+      mbar_arrive(bar(pf::kTileFree + (ti & 1)));
     }
-    const int tok0 = tile * QT;  // chunk-relative first token of the tile
-    if (tok0 >= n) continue;     // uniform across the CTA
-    const int ctx = L - n;
-    const int pos_min = ctx + tok0;
-    const int pos_max = min(L - 1, ctx + tok0 + QT - 1);
-    const int nc = pos_max / pf::kKeys + 1;  // key chunks this tile attends to
-    const int BS = p.block_size;
-    const int nblk = (L + BS - 1) / BS;
+    return __shfl_sync(pf::kAll, t, 0);
+  };
+  const int BS = p.block_size;
+  int issued = 0, q_issued = 0;  // producers: fills issued (chunks, Q tiles) in the CTA's count
 
-    if (warp == pf::kProducerK || warp == pf::kProducerV) {
-      // ----------------------------- TMA producers -----------------------------
-      // One warp streams K chunks, the other V chunks, each through its own
-      // ring: K runs ahead of V (q·Kᵀ of chunk j+2 is issued right after P·V
-      // of chunk j, while V's stages free only as P·V completes; a single
-      // producer alternating K and V held K behind V's refills).
-      const int kv = warp == pf::kProducerV ? 1 : 0;
-      bool ok = true;
-      q_issued = ti + 1;
-      if (lane == 0 && kv == 0) {
-        // Q tile: rows token * G + h, one box per head_dim half
-        mbar_arrive_expect_tx(bar(pf::kQFull), pf::kTile);
-        tma_load_4d(base + pf::kOffQ, &tmap_q, 0, 0, g * G, q0 + tok0, bar(pf::kQFull));
-        tma_load_4d(base + pf::kOffQ + pf::kSlab, &tmap_q, 0, 1, g * G, q0 + tok0, bar(pf::kQFull));
+  if (warp == pf::kProducerK || warp == pf::kProducerV) {
+    // ----------------------------- TMA producers -----------------------------
+    // One warp streams K chunks (and Q), the other V chunks, each through its
+    // own ring: K runs ahead of V (q·Kᵀ of chunk j+2 is issued right after
+    // P·V of chunk j, while V's stages free only as P·V completes; a single
+    // producer alternating K and V held K behind V's refills).
+    const int kv = warp == pf::kProducerV ? 1 : 0;
+    bool ok = true;
+    int gc = 0, tv = 0;
+    for (int ti = 0; ok; ++ti) {
+      int t;
+      if (kv == 0) {
+        t = total;
+        if (lane == 0) {
+          // the slot's previous tile has been read by every other role
+          const bool free = ti < 2 || pf_wait(bar(pf::kTileFree + (ti & 1)), ((ti >> 1) - 1) & 1, abort_flag);
+          if (!free && !*abort_flag) {
+            record_error(PKV_ERR_DEVICE_TIMEOUT);
+            *abort_flag = 1;
+          }
+          const unsigned ticket = (!free || *abort_flag) ? static_cast<unsigned>(total) : atomicAdd(tile_ctr, 1u);
+          t = ticket >= static_cast<unsigned>(total) ? total : static_cast<int>(ticket);
+          tile_slot[ti & 1] = t;
+          mbar_arrive(bar(pf::kTileReady + (ti & 1)));
+        }
+        t = __shfl_sync(pf::kAll, t, 0);
+      } else {
+        t = read_tile(ti);
+      }
+      if (t >= total) break;
+      const Tile d = tile_of(t);
+      if (!d.valid) continue;
+      const int b = d.b, g = d.g, nc = d.nc, nblk = d.nblk;
+      if (kv == 0) {
+        // Q of the previous tile is no longer read once its last q·Kᵀ is done
+        if (tv > 0) ok = __all_sync(pf::kAll, pf_wait(bar(pf::kQEmpty), (tv - 1) & 1, abort_flag));
+        if (!ok) break;
+        if (lane == 0) {
+          // Q tile: rows token * G + h, one box per head_dim half
+          mbar_arrive_expect_tx(bar(pf::kQFull), pf::kTile);
+          tma_load_4d(base + pf::kOffQ, &tmap_q, 0, 0, g * G, d.q0 + d.tok0, bar(pf::kQFull));
+          tma_load_4d(base + pf::kOffQ + pf::kSlab, &tmap_q, 0, 1, g * G, d.q0 + d.tok0, bar(pf::kQFull));
+        }
+        q_issued = tv + 1;
       }
       const int32_t* trow = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
       const int nbc = pf::kKeys / BS;                              // blocks per chunk
@@ -326,16 +381,37 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         }
         issued = gc + j + 1;
       }
-      if (!ok && lane == 0) {
-        record_error(PKV_ERR_DEVICE_TIMEOUT);
-        *abort_flag = 1;
+      gc += nc;
+      ++tv;
+    }
+    if (!ok && lane == 0) {
+      record_error(PKV_ERR_DEVICE_TIMEOUT);
+      *abort_flag = 1;
+    }
+    // no copy may still be landing when the CTA exits (a timeout can leave
+    // fills unconsumed): wait (bounded) for the last fill of each stage and Q
+    if (lane == 0) {
+      const uint32_t full0 = bar(kv ? pf::kVFull : pf::kKFull);
+      if (kv == 0 && q_issued > 0) drain_wait(bar(pf::kQFull), (q_issued - 1) & 1);
+      for (int s = 0; s < pf::kStages && s < issued; ++s) {
+        const int last = s + (issued - 1 - s) / pf::kStages * pf::kStages;  // last chunk that used stage s
+        drain_wait(full0 + 8 * s, (last / pf::kStages) & 1);
       }
-      __syncwarp();
-    } else if (warp == pf::kMmaWarp) {
-      // ------------------------------- MMA issuer -------------------------------
+    }
+    __syncwarp();
+  } else if (warp == pf::kMmaWarp) {
+    // ------------------------------- MMA issuer -------------------------------
+    const uint32_t id_s = tc::idesc_f16(kBf16, false, pf::kRows, pf::kKeys);
+    const uint32_t id_o = tc::idesc_f16(kBf16, true, pf::kRows, pf::kHeadDim);
+    bool ok = true;
+    int gc = 0, tv = 0;
+    for (int ti = 0; ok; ++ti) {
+      const int t = read_tile(ti);
+      if (t >= total) break;
+      const Tile d = tile_of(t);
+      if (!d.valid) continue;
+      const int nc = d.nc;
       if (lane == 0) {
-        const uint32_t id_s = tc::idesc_f16(kBf16, false, pf::kRows, pf::kKeys);
-        const uint32_t id_o = tc::idesc_f16(kBf16, true, pf::kRows, pf::kHeadDim);
         auto issue_s = [&](int j) -> bool {  // j: chunk of the tile; gc + j: chunk of the CTA
           const int s = (gc + j) % pf::kStages;
           if (!pf_wait(bar(pf::kKFull + s), ((gc + j) / pf::kStages) & 1, abort_flag)) return false;
@@ -352,8 +428,11 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
           tc::commit(bar(pf::kSFull + (gc + j) % pf::kSBufs));
           return true;
         };
-        bool ok = pf_wait(bar(pf::kQFull), ti & 1, abort_flag);
+        ok = pf_wait(bar(pf::kQFull), tv & 1, abort_flag);
         for (int j = 0; j < pf::kSBufs && j < nc && ok; ++j) ok = issue_s(j);
+        if (ok && nc <= pf::kSBufs) tc::commit(bar(pf::kQEmpty));  // the tile's last q·Kᵀ is issued
+        // the previous tile's O has been read out of tensor memory
+        if (ok && tv > 0) ok = pf_wait(bar(pf::kOFree), (tv - 1) & 1, abort_flag);
         for (int j = 0; j < nc && ok; ++j) {
           const int gj = gc + j;
           const int s = gj % pf::kStages;
@@ -374,28 +453,44 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
           }
           tc::commit(bar(pf::kVEmpty + s));
           tc::commit(bar(pf::kPVDone + gj % pf::kSBufs));
-          if (j + pf::kSBufs < nc) ok = issue_s(j + pf::kSBufs);
+          if (j + pf::kSBufs < nc) {
+            ok = issue_s(j + pf::kSBufs);
+            if (ok && j + pf::kSBufs == nc - 1) tc::commit(bar(pf::kQEmpty));  // the tile's last q·Kᵀ
+          }
         }
-        if (!ok) {
-          record_error(PKV_ERR_DEVICE_TIMEOUT);
-          *abort_flag = 1;
-        }
-        // every MMA of the tile completes before O is read and before the next
-        // tile's loads reuse Q and the rings
-        tc::commit(bar(pf::kDrain));
-        drain_wait(bar(pf::kDrain), ti & 1);
+        if (ok) tc::commit(bar(pf::kODone));  // the tile's O is complete once its last P·V is
       }
-      __syncwarp();
-    } else {
-      // ------------------------------ softmax warps ------------------------------
-      const int r = threadIdx.x;  // tile row and TMEM lane
+      ok = __shfl_sync(pf::kAll, ok, 0);
+      gc += nc;
+      ++tv;
+    }
+    if (lane == 0) {
+      if (!ok) {
+        record_error(PKV_ERR_DEVICE_TIMEOUT);
+        *abort_flag = 1;
+      }
+      // every MMA issued completes before tensor memory is freed
+      tc::commit(bar(pf::kDrain));
+      drain_wait(bar(pf::kDrain), 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------ softmax warps ------------------------------
+    const int r = threadIdx.x;  // tile row and TMEM lane
+    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    unsigned char* vzero = smem + pf::kOffV;
+    const float sl = p.scale_log2;
+    bool ok = true;
+    int gc = 0, tv = 0;
+    for (int ti = 0; ok; ++ti) {
+      const int t = read_tile(ti);
+      if (t >= total) break;
+      const Tile d = tile_of(t);
+      if (!d.valid) continue;
+      const int nc = d.nc, L = d.L, n = d.n, tok0 = d.tok0, pos_min = d.pos_min;
       const int tok = tok0 + r / G;
-      const int pos = min(ctx + tok, L - 1);  // rows past the chunk end compute a copy of the last row
-      const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-      unsigned char* vzero = smem + pf::kOffV;
-      const float sl = p.scale_log2;
+      const int pos = min(d.ctx + tok, L - 1);  // rows past the chunk end compute a copy of the last row
       float m_used = -INFINITY, l = 0.f;
-      bool ok = true;
       for (int j = 0; j < nc && ok; ++j) {
         const int gj = gc + j;              // chunk of the CTA
         const int sb = gj % pf::kSBufs;     // S / P buffer
@@ -515,64 +610,59 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         tc::fence_before_sync();
         mbar_arrive(bar(pf::kPFull + sb));
       }
-      // the MMA warp commits kDrain after its last MMA: every P·V is then done
-      if (ok) ok = __all_sync(pf::kAll, pf_wait(bar(pf::kDrain), ti & 1, abort_flag));
-      if (ok) {
-        tc::fence_after_sync();
-        const float inv = 1.f / l;
-        // O goes out through shared memory (Q and the K ring are free once every
-        // MMA is done): each thread parks its row, then each warp writes its 32
-        // rows one 512-byte row per store instruction, instead of 32 rows per
-        // instruction straight from the tensor-memory layout.  The 16-byte piece
-        // c of row r sits at slot c ^ (r mod 8) of the row, so the row-wise
-        // writes and the piece-wise reads are both free of bank conflicts.
-        float4* stage = reinterpret_cast<float4*>(smem + pf::kOffQ);
-        float4* srow = stage + r * (pf::kHeadDim / 4);
+      // the MMA warp commits O-done after the tile's last P·V
+      if (ok) ok = __all_sync(pf::kAll, pf_wait(bar(pf::kODone), tv & 1, abort_flag));
+      if (!ok) break;
+      tc::fence_after_sync();
+      // O leaves tensor memory first (the next tile's P·V may then overwrite
+      // it), then goes out through shared memory: each thread parks its row,
+      // and each warp writes its 32 rows one 512-byte row per store
+      // instruction, instead of 32 rows per instruction straight from the
+      // tensor-memory layout.  The 16-byte piece c of row r sits at slot
+      // c ^ (r mod 8) of the row, so the row-wise writes and the piece-wise
+      // reads are both free of bank conflicts.
+      uint32_t o[4][32];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t o[32];
-          tc::ld_32x32b_x32(trow + pf::kColO + 32 * q, o);
-          tc::wait_ld();
+      for (int q = 0; q < 4; ++q) tc::ld_32x32b_x32(trow + pf::kColO + 32 * q, o[q]);
+      tc::wait_ld();
+      tc::fence_before_sync();
+      mbar_arrive(bar(pf::kOFree));
+      const float inv = 1.f / l;
+      float4* stage = reinterpret_cast<float4*>(smem + pf::kOffStage);
+      float4* srow = stage + r * (pf::kHeadDim / 4);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            srow[(8 * q + i) ^ (r & 7)] =
-                make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
-                            __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          srow[(8 * q + i) ^ (r & 7)] =
+              make_float4(__uint_as_float(o[q][4 * i]) * inv, __uint_as_float(o[q][4 * i + 1]) * inv,
+                          __uint_as_float(o[q][4 * i + 2]) * inv, __uint_as_float(o[q][4 * i + 3]) * inv);
+      __syncwarp();
+      for (int k = 0; k < 32; ++k) {
+        const int rr = warp * 32 + k;  // a row this warp parked
+        const int tk = tok0 + rr / G;
+        if (tk < n) {                  // rows past the chunk end are not written
+          float4* orow = reinterpret_cast<float4*>(
+              p.out + (static_cast<int64_t>(d.q0 + tk) * p.num_q_heads + d.g * G + rr % G) * pf::kHeadDim);
+          orow[lane] = stage[rr * (pf::kHeadDim / 4) + (lane ^ (rr & 7))];
         }
-        __syncwarp();
-        for (int k = 0; k < 32; ++k) {
-          const int rr = warp * 32 + k;  // a row this warp parked
-          const int tk = tok0 + rr / G;
-          if (tk < n) {                  // rows past the chunk end are not written
-            float4* orow = reinterpret_cast<float4*>(
-                p.out + (static_cast<int64_t>(q0 + tk) * p.num_q_heads + g * G + rr % G) * pf::kHeadDim);
-            orow[lane] = stage[rr * (pf::kHeadDim / 4) + (lane ^ (rr & 7))];
-          }
-        }
-      } else if (lane == 0) {
-        record_error(PKV_ERR_DEVICE_TIMEOUT);
-        *abort_flag = 1;
       }
+      __syncwarp();  // this warp's rows are out of the staging area before the next tile's
+      gc += nc;
+      ++tv;
     }
-
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    gc += nc;
-    ++ti;
-  }  // tiles
-
-  // no copy may still be landing when the CTA exits (a timeout can leave
-  // fills unconsumed): wait (bounded) for the last fill of each stage and Q
-  if ((warp == pf::kProducerK || warp == pf::kProducerV) && lane == 0) {
-    const uint32_t full0 = bar(warp == pf::kProducerV ? pf::kVFull : pf::kKFull);
-    if (warp == pf::kProducerK && q_issued > 0) drain_wait(bar(pf::kQFull), (q_issued - 1) & 1);
-    for (int s = 0; s < pf::kStages && s < issued; ++s) {
-      const int last = s + (issued - 1 - s) / pf::kStages * pf::kStages;  // last chunk that used stage s
-      drain_wait(full0 + 8 * s, (last / pf::kStages) & 1);
+    if (!ok && lane == 0) {
+      record_error(PKV_ERR_DEVICE_TIMEOUT);
+      *abort_flag = 1;
     }
   }
-  if (warp == pf::kMmaWarp) tc::tmem_dealloc(*tmem_slot, pf::kTmemCols);
+
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == pf::kMmaWarp) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, pf::kTmemCols);
+  }
   if (threadIdx.x == 0) {
     // the last CTA to finish re-arms the counter for the next launch that
     // uses this slot: every CTA has drawn its last ticket before it counts
