@@ -340,7 +340,10 @@ int pkv_decode_step_host(pkv_alloc_t* a, const int64_t* seq_ids, int32_t n, cons
  * about 1e-5 of the exact softmax.  A sequence whose chunk is longer than
  * seq_lens[b] or max_q_len is skipped and recorded as PKV_ERR_INVALID_ARG;
  * table entries outside [0, num_blocks) as PKV_ERR_BAD_BLOCK (block 0 read
- * instead), both in the device status. */
+ * instead), both in the device status.  The kernel runs one CTA per SM,
+ * which draws tiles from a counter inside the library; calls take the
+ * library's 64 counters in turn, so up to 64 calls may overlap on the GPU
+ * (for instance on different streams). */
 int pkv_paged_attention_prefill(const void* q, const void* k_pool, const void* v_pool,
                                 const int32_t* block_tables, const int32_t* seq_lens,
                                 const int32_t* q_start, int32_t num_seqs, int32_t num_q_tokens,

@@ -7,10 +7,11 @@
 // causally to tokens 0 .. that position through the block table (vLLM paging
 // page §3 phase 2), KV head h / G, fp32 output.
 //
-// One CTA computes one tile: 128 rows = 128/G query tokens x the G query heads
-// of one KV head, so a GQA group turns into a full M = 128 MMA tile even for
-// short chunks.  Keys come in chunks of 128 tokens (128/block_size physical
-// blocks, one TMA box per block and head_dim half).  Per chunk j:
+// A tile is 128 rows = 128/G query tokens x the G query heads of one KV head,
+// so a GQA group turns into a full M = 128 MMA tile even for short chunks;
+// persistent CTAs (one per SM) take tiles one after another.  Keys come in
+// chunks of 128 tokens (128/block_size physical blocks, one TMA box per block
+// and head_dim half).  Per chunk j:
 //
 //   S_j = Q · K_jᵀ        tcgen05.mma, 128x128x128, A and B from shared memory,
 //                         fp32 in tensor memory
@@ -25,9 +26,10 @@
 // memory (512 columns): three S / P buffers at columns 0, 128 and 256 (P hi
 // in the first 64 columns of its buffer, P lo in the next 64; a single f16 P
 // in the first 64), O at 384.
-// Shared memory: Q 32 KB and K and V rings of 32 KB stages.  Keeping P in
-// tensor memory spares shared memory 128 KB of traffic per chunk (P written
-// and read back), which bounded the first version of this kernel.
+// Shared memory: Q 32 KB, K and V rings of 32 KB stages and a 64 KB staging
+// buffer for the output rows.  Keeping P in tensor memory spares shared
+// memory 128 KB of traffic per chunk (P written and read back), which bounded
+// the first version of this kernel.
 //
 // Pipeline: the MMA warp issues S_0, S_1, S_2, then per chunk PV_j followed
 // by S_{j+3}, so q·Kᵀ of the next chunks runs while the softmax warps work
