@@ -83,8 +83,13 @@ __device__ __forceinline__ uint32_t row_offset(int r, int h, int br_shift, int h
 // frees the ring stage at once and widens them into mma fragments in
 // registers; the contraction order of q·Kᵀ and the output dims of P·V are
 // permuted within each step so every word feeds whole fragment registers.
+// The e4m3 kernel is held to 3 CTAs per SM (96 registers instead of 158, no
+// spills): its consumers are bound by latency, not issue, and 12 consumer
+// warps per SM instead of 8 take its decode call from 77.3 to 74.8 us on the
+// Llama-3-8B-shaped batch (4 CTAs would spill).  The 16-bit kernels keep the
+// compiler's own choice (127 registers, 2 CTAs per SM).
 template <typename T, int D, int G, int kKVBytes = 2>
-__global__ void __launch_bounds__(kMmaThreads) decode_mma_kernel(const DecodeParams p,
+__global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0) decode_mma_kernel(const DecodeParams p,
                                                                     const __grid_constant__ CUtensorMap tmap_k,
                                                                     const __grid_constant__ CUtensorMap tmap_v) {
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
