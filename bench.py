@@ -50,13 +50,13 @@ EVENT_EVERY = 16
 # on (kernel_source_sha()).  A pin whose hash no longer matches is reported as
 # null.
 TRAFFIC = {
-    "llama3_8b": (606696320, "85a57a9f50886783"),
-    "llama3_8b_fp8": (307867264, "85a57a9f50886783"),
+    "llama3_8b": (607126912, "2b1003ee67f78fc4"),
+    "llama3_8b_fp8": (307347840, "2b1003ee67f78fc4"),
 }
 # the same for one pkv_paged_attention_prefill call (prefill_tc_kernel), keyed
 # by the hash of the prefill sources (kernel_source_sha(PREFILL_SOURCES))
 TRAFFIC_PREFILL = {
-    "prefill_llama3_8b": (330831488, "af3a520664f50605"),
+    "prefill_llama3_8b": (332099840, "99f76280f1c3819b"),
 }
 
 
