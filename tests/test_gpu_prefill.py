@@ -248,3 +248,56 @@ def test_full_size_chunked_prefill_sampled_rows():
                                          np.array([1]), w.scale, "bf16")
         got = out[b * n + i, g * G:(g + 1) * G].unsqueeze(0)
         assert_close(got, ref, "bf16", f"row {b}/{i} heads {g * G}..{g * G + G - 1}")
+
+
+def test_repeated_concurrent_and_captured_calls():
+    """The persistent kernel draws tiles from counters inside the library
+    that each launch's last CTA re-arms: 70 calls in a row (more than the
+    64 counters), two calls overlapping on two streams, and a captured graph
+    replayed five times all give the single call's result bit for bit."""
+    a = PrefillCase([300, 129, 517], [300, 1, 45], 8, 2, 16, "bf16", _seed("repeat", "a"))
+    b = PrefillCase([700, 64], [128, 64], 8, 2, 16, "f16", _seed("repeat", "b"))
+
+    def args(c):
+        dev = "cuda"
+        return (c.q.to(dev), c.k_pool.to(dev), c.v_pool.to(dev), torch.from_numpy(c.tables).to(dev),
+                torch.tensor(c.lens, dtype=torch.int32, device=dev), torch.from_numpy(c.q_start).to(dev),
+                max(c.q_lens), c.scale)
+
+    xa, xb = args(a), args(b)
+    ref_a = pkv.pkv_paged_attention_prefill(*xa).clone()
+    ref_b = pkv.pkv_paged_attention_prefill(*xb).clone()
+    torch.cuda.synchronize()
+    assert_close(ref_a, a.oracle(), "bf16", "single call a")
+    assert_close(ref_b, b.oracle(), "f16", "single call b")
+
+    out = torch.empty_like(ref_a)
+    for _ in range(70):
+        pkv.pkv_paged_attention_prefill(*xa, out=out)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref_a), "70 calls in a row"
+
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    oa, ob = torch.empty_like(ref_a), torch.empty_like(ref_b)
+    torch.cuda.synchronize()
+    for _ in range(5):
+        with torch.cuda.stream(s1):
+            pkv.pkv_paged_attention_prefill(*xa, out=oa)
+        with torch.cuda.stream(s2):
+            pkv.pkv_paged_attention_prefill(*xb, out=ob)
+    torch.cuda.synchronize()
+    assert torch.equal(oa, ref_a) and torch.equal(ob, ref_b), "calls on two streams"
+
+    og = torch.zeros_like(ref_a)
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        pkv.pkv_paged_attention_prefill(*xa, out=og)  # first call outside the capture
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            pkv.pkv_paged_attention_prefill(*xa, out=og)
+    for _ in range(5):
+        og.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(og, ref_a), "graph replay"
