@@ -89,6 +89,7 @@ constexpr uint32_t kOffV = kOffK + kStages * kTile;
 constexpr uint32_t kOffStage = kOffV + kStages * kTile;  // output rows on their way out (128 x 512 B)
 constexpr uint32_t kOffBar = kOffStage + kRows * kHeadDim * 4;
 constexpr size_t kSmemBytes = kOffBar + 256 + 1024;  // barriers, flags; 1024 B alignment slack
+static_assert(kSmemBytes <= 227 * 1024, "one CTA's shared memory (227 KB at most on sm_100)");
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSBufs = 3;                    // S / P buffers in tensor memory
 constexpr uint32_t kColS = 0, kColO = 384;   // S / P: 3 x 128 columns, O: 128
@@ -186,30 +187,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
 }
-
-// 2^x on the FMA pipe, for x <= 64 (returns +0 for x <= -127): Cody-Waite
-// reduction x = n + f with n the nearest integer (the 1.5·2^23 rounding trick)
-// and f in [-1/2, 1/2], then 2^f = e^(f ln 2) by its Taylor series to degree 5
-// (truncation error below 2.5e-6 relative), scaled by 2^n through the
-// exponent field.  Takes a share of the softmax exponentials off the
-// special-function pipe.
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -127.f);
-  const float t = x + 12582912.f;
-  const float f = x - (t - 12582912.f);
-  float p = 1.3333558146428443e-3f;           // ln2^5 / 5!
-  p = fmaf(p, f, 9.6181291076284772e-3f);     // ln2^4 / 4!
-  p = fmaf(p, f, 5.5504108664821580e-2f);     // ln2^3 / 3!
-  p = fmaf(p, f, 2.4022650695910071e-1f);     // ln2^2 / 2!
-  p = fmaf(p, f, 6.9314718055994531e-1f);     // ln2
-  p = fmaf(p, f, 1.f);
-  const int n = __float_as_int(t) - 0x4B400000;
-  return __int_as_float(__float_as_int(p) + (n << 23));
-}
-
-#ifndef PKV_PREFILL_POLY_EVERY
-#define PKV_PREFILL_POLY_EVERY 0  // one softmax exponential in this many on the FMA pipe (0: none)
-#endif
 
 template <typename T, int G>
 __global__ void __launch_bounds__(pf::kThreads, 1)
@@ -549,8 +526,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
 #pragma unroll
           for (int c = 64 * h; c < 64 * h + 64; c += 2) {
             const float2 a = __ffma2_rn(make_float2(x[c], x[c + 1]), sl2, nm2);  // hidden keys: -inf -> 0
-            constexpr int kEvery = PKV_PREFILL_POLY_EVERY > 0 ? PKV_PREFILL_POLY_EVERY : 1;
-            x[c] = (PKV_PREFILL_POLY_EVERY > 0 && c % kEvery == kEvery - 1) ? exp2_fma(a.x) : fast_exp2(a.x);
+            x[c] = fast_exp2(a.x);
             x[c + 1] = fast_exp2(a.y);
             sm[(c >> 1) & 3] = __fadd2_rn(sm[(c >> 1) & 3], make_float2(x[c], x[c + 1]));
           }
