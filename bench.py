@@ -56,7 +56,7 @@ TRAFFIC = {
 # the same for one pkv_paged_attention_prefill call (prefill_tc_kernel), keyed
 # by the hash of the prefill sources (kernel_source_sha(PREFILL_SOURCES))
 TRAFFIC_PREFILL = {
-    "prefill_llama3_8b": (332099840, "99f76280f1c3819b"),
+    "prefill_llama3_8b": (332073216, "7a47bcbddd2fb32c"),
 }
 
 
