@@ -89,39 +89,6 @@ def pkv_decode_workspace_size(num_seqs: int, num_q_heads: int, num_kv_heads: int
     return out.value
 
 
-def pkv_paged_attention_decode(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
-                               block_tables: torch.Tensor, seq_lens: torch.Tensor, scale: float,
-                               out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                               partition_tokens: int = 0) -> torch.Tensor:
-    """PagedAttention decode; returns ``out`` (float32 ``[num_seqs, num_q_heads, head_dim]``)."""
-    nb, hkv, bs, d = _pool_dims(_cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"))
-    _cuda(q, "q", k_pool.dtype)
-    if q.dim() != 3 or q.shape[2] != d:
-        raise ValueError(f"q must be [num_seqs, num_q_heads, {d}]")
-    B, hq, _ = q.shape
-    _cuda(block_tables, "block_tables", torch.int32)
-    _cuda(seq_lens, "seq_lens", torch.int32)
-    if block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.numel() != B:
-        raise ValueError("block_tables must be [num_seqs, max_blocks_per_seq] and seq_lens [num_seqs]")
-    maxb = block_tables.shape[1]
-    if out is None:
-        out = torch.empty((B, hq, d), dtype=torch.float32, device=q.device)
-    else:
-        _cuda(out, "out", torch.float32)
-        if tuple(out.shape) != (B, hq, d):
-            raise ValueError("out has the wrong shape")
-    need = pkv_decode_workspace_size(B, hq, hkv, d, maxb, bs, partition_tokens)
-    if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    else:
-        _cuda(workspace, "workspace", torch.uint8)
-    check(lib().pkv_paged_attention_decode(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
-                                           block_tables.data_ptr(), seq_lens.data_ptr(), B, hq, hkv, d, nb, maxb,
-                                           bs, float(scale), _dtype_code(k_pool), partition_tokens,
-                                           workspace.data_ptr(), workspace.numel(), out.data_ptr(), _stream()))
-    return out
-
-
 def _new_rows(k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: torch.Tensor, hkv: int, d: int,
               dtype=None) -> int:
     for name, t in (("k_new", k_new), ("v_new", v_new)):
@@ -158,6 +125,21 @@ def _decode_io(q: torch.Tensor, hkv: int, d: int, bs: int, block_tables: torch.T
     else:
         _cuda(workspace, "workspace", torch.uint8)
     return B, hq, maxb, out, workspace
+
+
+def pkv_paged_attention_decode(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                               block_tables: torch.Tensor, seq_lens: torch.Tensor, scale: float,
+                               out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                               partition_tokens: int = 0) -> torch.Tensor:
+    """PagedAttention decode; returns ``out`` (float32 ``[num_seqs, num_q_heads, head_dim]``)."""
+    nb, hkv, bs, d = _pool_dims(_cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"))
+    _cuda(q, "q", k_pool.dtype)
+    B, hq, maxb, out, workspace = _decode_io(q, hkv, d, bs, block_tables, seq_lens, out, workspace, partition_tokens)
+    check(lib().pkv_paged_attention_decode(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
+                                           block_tables.data_ptr(), seq_lens.data_ptr(), B, hq, hkv, d, nb, maxb,
+                                           bs, float(scale), _dtype_code(k_pool), partition_tokens,
+                                           workspace.data_ptr(), workspace.numel(), out.data_ptr(), _stream()))
+    return out
 
 
 def pkv_append_and_decode(k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: torch.Tensor, q: torch.Tensor,
@@ -278,21 +260,11 @@ def pkv_paged_attention_decode_fp8(q: torch.Tensor, k_pool: torch.Tensor, v_pool
     """PagedAttention decode over e4m3 pools (q float16); float32 output."""
     _fp8_pool(k_pool, "k_pool")
     _fp8_pool(v_pool, "v_pool")
+    if k_pool.dim() != 4 or k_pool.shape != v_pool.shape:
+        raise ValueError("pools must be [num_blocks, num_kv_heads, block_size, head_dim]")
     nb, hkv, bs, d = k_pool.shape
     _cuda(q, "q", torch.float16)
-    B, hq, _ = q.shape
-    _cuda(block_tables, "block_tables", torch.int32)
-    _cuda(seq_lens, "seq_lens", torch.int32)
-    if block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.numel() != B:
-        raise ValueError("block_tables must be [num_seqs, max_blocks_per_seq] and seq_lens [num_seqs]")
-    maxb = block_tables.shape[1]
-    if out is None:
-        out = torch.empty((B, hq, d), dtype=torch.float32, device=q.device)
-    else:
-        _cuda(out, "out", torch.float32)
-    need = pkv_decode_workspace_size(B, hq, hkv, d, maxb, bs, partition_tokens)
-    if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    B, hq, maxb, out, workspace = _decode_io(q, hkv, d, bs, block_tables, seq_lens, out, workspace, partition_tokens)
     check(lib().pkv_paged_attention_decode_fp8(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
                                                block_tables.data_ptr(), seq_lens.data_ptr(), B, hq, hkv, d, nb, maxb,
                                                bs, float(scale), float(k_scale), float(v_scale), partition_tokens,
