@@ -335,9 +335,11 @@ int pkv_decode_step_host(pkv_alloc_t* a, const int64_t* seq_ids, int32_t n, cons
  * head_dim 128, G in {1, 2, 4, 8}, block_size 8, 16 or 32; others return
  * PKV_ERR_UNSUPPORTED.  q, pools and out 16-byte aligned; scale positive
  * and finite (else PKV_ERR_INVALID_ARG).
- * Computed on the tcgen05 tensor cores with fp32 accumulation; P enters the
- * P·V product as two 16-bit halves (hi + lo), so the result stays within
- * about 1e-5 of the exact softmax.  A sequence whose chunk is longer than
+ * Computed on the tcgen05 tensor cores with fp32 accumulation.  The
+ * softmax weights P enter the P·V product as two bf16 halves (hi + lo) for
+ * bf16 pools, within about 1e-5 of the exact softmax, and as one f16 value
+ * for f16 pools (relative error 2^-11 per weight; the output within about
+ * 5e-4 of the output scale).  A sequence whose chunk is longer than
  * seq_lens[b] or max_q_len is skipped and recorded as PKV_ERR_INVALID_ARG;
  * table entries outside [0, num_blocks) as PKV_ERR_BAD_BLOCK (block 0 read
  * instead), both in the device status.  The kernel runs one CTA per SM,
