@@ -136,3 +136,71 @@ def test_step_meta_bytes_and_step_argument_checks(native):
                                            N.PKV_BF16, 1.0, 1.0, 0, FAKE, 0, None) == 0
     finally:
         native.pkv_alloc_destroy(a)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=7), N.PKV_ERR_UNSUPPORTED),
+    (dict(n=-1), N.PKV_ERR_INVALID_ARG),
+    (dict(kn=FAKE + 8), N.PKV_ERR_INVALID_ARG),         # misaligned new rows
+    (dict(slots=0), N.PKV_ERR_INVALID_ARG),
+    (dict(hq=24, hkv=8), N.PKV_ERR_UNSUPPORTED),        # group size 3: the decode half refuses
+    (dict(scale=float("nan")), N.PKV_ERR_INVALID_ARG),
+    (dict(ws_bytes=16), N.PKV_ERR_INVALID_ARG),
+    (dict(pt=100), N.PKV_ERR_INVALID_ARG),
+])
+def test_append_and_decode_rejects_bad_arguments_before_launch(native, kw, code):
+    """The one-call append + decode checks both halves' arguments before it
+    launches anything (nothing here reaches the GPU)."""
+    a = dict(kn=FAKE, vn=FAKE, slots=FAKE, n=4, q=FAKE, k=FAKE, v=FAKE, t=FAKE, l=FAKE, B=4, hq=32, hkv=8,
+             head_dim=128, nb=64, maxb=8, block_size=16, scale=0.1, dtype=N.PKV_BF16, pt=0, ws=FAKE,
+             ws_bytes=1 << 30, out=FAKE)
+    a.update(kw)
+    rc = native.pkv_append_and_decode(a["kn"], a["vn"], a["slots"], a["n"], a["q"], a["k"], a["v"], a["t"], a["l"],
+                                      a["B"], a["hq"], a["hkv"], a["head_dim"], a["nb"], a["maxb"], a["block_size"],
+                                      a["scale"], a["dtype"], a["pt"], a["ws"], a["ws_bytes"], a["out"], None)
+    assert rc == code, native.pkv_last_error_string()
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(src=7), N.PKV_ERR_UNSUPPORTED),
+    (dict(k_scale=0.0), N.PKV_ERR_INVALID_ARG),
+    (dict(v_scale=float("inf")), N.PKV_ERR_INVALID_ARG),
+    (dict(head_dim=64), N.PKV_ERR_UNSUPPORTED),         # e4m3 pools need head_dim 128
+    (dict(pt=264), N.PKV_ERR_INVALID_ARG),              # not a multiple of 16
+])
+def test_append_and_decode_fp8_rejects_bad_arguments_before_launch(native, kw, code):
+    a = dict(kn=FAKE, vn=FAKE, src=N.PKV_F16, slots=FAKE, n=4, q=FAKE, k=FAKE, v=FAKE, t=FAKE, l=FAKE, B=4,
+             hq=32, hkv=8, head_dim=128, nb=64, maxb=64, block_size=8, scale=0.1, k_scale=0.5, v_scale=0.5,
+             pt=0, ws=FAKE, ws_bytes=1 << 30, out=FAKE)
+    a.update(kw)
+    rc = native.pkv_append_and_decode_fp8(a["kn"], a["vn"], a["src"], a["slots"], a["n"], a["q"], a["k"], a["v"],
+                                          a["t"], a["l"], a["B"], a["hq"], a["hkv"], a["head_dim"], a["nb"],
+                                          a["maxb"], a["block_size"], a["scale"], a["k_scale"], a["v_scale"],
+                                          a["pt"], a["ws"], a["ws_bytes"], a["out"], None)
+    assert rc == code, native.pkv_last_error_string()
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=N.PKV_F32), N.PKV_ERR_UNSUPPORTED),    # the tensor-core prefill takes 16-bit K/V
+    (dict(head_dim=64), N.PKV_ERR_UNSUPPORTED),
+    (dict(hq=24, hkv=8), N.PKV_ERR_UNSUPPORTED),
+    (dict(hq=30, hkv=8), N.PKV_ERR_INVALID_ARG),
+    (dict(scale=0.0), N.PKV_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), N.PKV_ERR_INVALID_ARG),
+    (dict(q=FAKE + 4), N.PKV_ERR_INVALID_ARG),
+    (dict(qs=0), N.PKV_ERR_INVALID_ARG),
+    (dict(T=-1), N.PKV_ERR_INVALID_ARG),
+])
+def test_prefill_rejects_bad_arguments_before_launch(native, kw, code):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, t=FAKE, l=FAKE, qs=FAKE, B=2, T=64, maxq=32, hq=32, hkv=8, head_dim=128,
+             nb=64, maxb=8, block_size=16, scale=0.1, dtype=N.PKV_BF16, out=FAKE)
+    a.update(kw)
+    rc = native.pkv_paged_attention_prefill(a["q"], a["k"], a["v"], a["t"], a["l"], a["qs"], a["B"], a["T"],
+                                            a["maxq"], a["hq"], a["hkv"], a["head_dim"], a["nb"], a["maxb"],
+                                            a["block_size"], a["scale"], a["dtype"], a["out"], None)
+    assert rc == code, native.pkv_last_error_string()
+
+
+def test_prefill_empty_batch_is_a_no_op(native):
+    assert native.pkv_paged_attention_prefill(None, None, None, None, None, None, 0, 0, 0, 32, 8, 128, 64, 8, 16,
+                                              0.1, N.PKV_BF16, None, None) == 0
