@@ -50,8 +50,8 @@ EVENT_EVERY = 16
 # on (kernel_source_sha()).  A pin whose hash no longer matches is reported as
 # null.
 TRAFFIC = {
-    "llama3_8b": (607126912, "2b1003ee67f78fc4"),
-    "llama3_8b_fp8": (307347840, "2b1003ee67f78fc4"),
+    "llama3_8b": (606657152, "54f1a7f0c4803227"),
+    "llama3_8b_fp8": (307465728, "54f1a7f0c4803227"),
 }
 # the same for one pkv_paged_attention_prefill call (prefill_tc_kernel), keyed
 # by the hash of the prefill sources (kernel_source_sha(PREFILL_SOURCES))

@@ -8,9 +8,12 @@
 //
 // How (B200 design, not the page's):
 //   plan kernel    one CTA turns seq_lens into a work list of partitions of
-//                  `partition_tokens` tokens, largest first;
+//                  `partition_tokens` tokens, largest first (in a decode step
+//                  the launch that builds it also writes the step's new K/V
+//                  rows: append_plan_kernel);
 //   decode kernel  persistent CTAs (grid = SMs x resident CTAs) walk the list
-//                  with a stride; per work unit (sequence, partition, KV
+//                  in rounds of alternating direction (unit_index); per work
+//                  unit (sequence, partition, KV
 //                  head) a producer warp streams each block's K and V tiles
 //                  (one contiguous block_size x head_dim tile each) into a
 //                  shared-memory ring with 1-D bulk copies completing on
