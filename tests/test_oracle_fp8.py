@@ -79,3 +79,123 @@ def test_fp8_attention_is_the_definition_on_dequantised_values():
     want = pa.paged_decode_attention(q.astype(np.float32), (fp8.e4m3_decode(kc) * 0.25).astype(np.float32),
                                      (fp8.e4m3_decode(vc) * 0.5).astype(np.float32), tables, lens, 0.2, "f32")
     assert np.max(np.abs(got - want)) < 1e-12  # all dequantised values are exact in fp32
+
+
+# ---------------------------------------------------------------------------
+# kv_append_fp8: the quantising append ("LLM inference optimisation:
+# principles overview" §5.1, an FP8 KV cache), pinned against codes worked out
+# by hand from the e4m3 definition (sign << 7 | exponent field << 3 | mantissa,
+# bias 7; subnormals m/8 * 2^-6; 0x7E = 448 the largest finite).
+# ---------------------------------------------------------------------------
+_NB, _HKV, _BS, _D = 3, 2, 4, 4
+_K_SCALE, _V_SCALE = 0.5, 0.125  # the append multiplies by 2 (K) and by 8 (V): exact in fp32
+_SLOTS = np.array([6, -1, 9])    # token 0 -> block 1 offset 2; token 1 is padding; token 2 -> block 2 offset 1
+_SENTINEL = 0x55
+
+_K_ROWS = np.array([
+    [[0.5, -0.75, 1.0, 224.0], [0.53125, -0.0, 2.0 ** -10, 1000.0]],
+    [[9.0, 9.0, 9.0, 9.0], [9.0, 9.0, 9.0, 9.0]],  # padding row: never written
+    [[1.75, 8.5, -0.375, 0.59375], [-224.0, 0.125, 0.1875, 4.0]],
+], dtype=np.float32)
+# 2x: 1, -1.5, 2, 448 | 1.0625 (tie -> even mantissa 0), -0, 2^-9 (smallest subnormal), 2000 (saturates)
+#     3.5, 17 (tie -> even), -0.75, 1.1875 (tie -> even mantissa 2) | -448, 0.25, 0.375, 8
+_K_CODES = {0: [[0x38, 0xBC, 0x40, 0x7E], [0x38, 0x80, 0x01, 0x7E]],
+            2: [[0x46, 0x58, 0xB4, 0x3A], [0xFE, 0x28, 0x2C, 0x50]]}
+
+_V_ROWS = np.array([
+    [[0.25, 0.1875, -0.4375, 0.09375], [0.01171875, -56.0, 2.0 ** -12, 0.0]],
+    [[-9.0, -9.0, -9.0, -9.0], [-9.0, -9.0, -9.0, -9.0]],
+    [[1.0, -2.0, 0.5, 0.15625], [3.0, 0.0390625, -0.0078125, 60.0]],
+], dtype=np.float32)
+# 8x: 2, 1.5, -3.5, 0.75 | 0.09375 = 1.5 * 2^-4, -448, 2^-9, 0
+#     8, -16, 4, 1.25 | 24, 0.3125, -0.0625, 480 (saturates)
+_V_CODES = {0: [[0x40, 0x3C, 0xC6, 0x34], [0x1C, 0xFE, 0x01, 0x00]],
+            2: [[0x50, 0xD8, 0x48, 0x3A], [0x5C, 0x2A, 0x98, 0x7E]]}
+
+
+def _check_append_fp8(append):
+    """Runs ``append`` (kv_append_fp8's signature) on the hand-worked case and
+    asserts every byte of both pools."""
+    kc = np.full((_NB, _HKV, _BS, _D), _SENTINEL, dtype=np.uint8)
+    vc = np.full((_NB, _HKV, _BS, _D), _SENTINEL, dtype=np.uint8)
+    k_out, v_out = append(kc, vc, _K_ROWS, _V_ROWS, _SLOTS, _K_SCALE, _V_SCALE)
+    want_k = np.full_like(kc, _SENTINEL)
+    want_v = np.full_like(vc, _SENTINEL)
+    for tok, slot in ((0, 6), (2, 9)):
+        blk, off = slot // _BS, slot % _BS
+        want_k[blk, :, off, :] = np.array(_K_CODES[tok], dtype=np.uint8)
+        want_v[blk, :, off, :] = np.array(_V_CODES[tok], dtype=np.uint8)
+    assert np.array_equal(k_out, want_k), "K pool bytes differ from the hand-worked codes"
+    assert np.array_equal(v_out, want_v), "V pool bytes differ from the hand-worked codes"
+    assert np.array_equal(kc, np.full_like(kc, _SENTINEL)), "the input pool was modified in place"
+
+
+def test_kv_append_fp8_matches_hand_worked_codes():
+    _check_append_fp8(fp8.kv_append_fp8)
+
+
+def test_kv_append_fp8_planted_mistakes_are_caught(monkeypatch):
+    """Plausible slips in the quantising append, each planted into the oracle
+    and each turning the hand-worked pin red."""
+    orig_append = fp8.kv_append_fp8
+    mutants = {
+        "K and V scales swapped": lambda kc, vc, k, v, s, ks, vs: orig_append(kc, vc, k, v, s, vs, ks),
+        "K rows into the V pool": lambda kc, vc, k, v, s, ks, vs: orig_append(kc, vc, v, k, s, vs, ks),
+        "multiply by the scale instead of dividing": lambda kc, vc, k, v, s, ks, vs: orig_append(
+            kc, vc, k, v, s, 1.0 / ks, 1.0 / vs),
+    }
+
+    def block_and_offset_swapped(kc, vc, k, v, slots, ks, vs):
+        kq, vq = fp8.quantize_rows(k, ks), fp8.quantize_rows(v, vs)
+        ko, vo = kc.copy(), vc.copy()
+        for i, s in enumerate(slots.tolist()):
+            if s >= 0:
+                off, blk = divmod(int(s), _BS)
+                ko[blk % _NB, :, off % _BS, :] = kq[i]
+                vo[blk % _NB, :, off % _BS, :] = vq[i]
+        return ko, vo
+
+    def padding_written(kc, vc, k, v, slots, ks, vs):
+        kq, vq = fp8.quantize_rows(k, ks), fp8.quantize_rows(v, vs)
+        ko, vo = kc.copy(), vc.copy()
+        for i, s in enumerate(slots.tolist()):
+            blk, off = divmod(int(s), _BS)  # slot -1 lands in the last block, offset 3
+            ko[blk, :, off, :] = kq[i]
+            vo[blk, :, off, :] = vq[i]
+        return ko, vo
+
+    mutants["block and offset swapped"] = block_and_offset_swapped
+    mutants["padding slot written"] = padding_written
+
+    # rounding slips inside the encoder the append uses
+    orig_encode = fp8.e4m3_encode
+    mags = fp8.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+
+    def truncating(x):
+        x = np.asarray(x, dtype=np.float64)
+        out = [int(np.searchsorted(mags, min(abs(v), 448.0), side="right")) - 1 | (0x80 if np.signbit(v) else 0)
+               for v in x.reshape(-1).tolist()]
+        return np.array(out, dtype=np.uint8).reshape(x.shape)
+
+    encode_mutants = {
+        "ties away from zero": lambda x: orig_encode(np.asarray(x, dtype=np.float64) * (1 + 2.0 ** -40)),
+        "no saturation (overflow to NaN)": lambda x: np.where(np.abs(np.asarray(x, dtype=np.float64)) > 448,
+                                                               np.uint8(0x7F), orig_encode(x)).astype(np.uint8),
+        "truncation instead of rounding": truncating,
+    }
+    survivors = []
+    for name, fn in mutants.items():
+        try:
+            _check_append_fp8(fn)
+            survivors.append(name)
+        except AssertionError:
+            pass
+    for name, fn in encode_mutants.items():
+        monkeypatch.setattr(fp8, "e4m3_encode", fn)
+        try:
+            _check_append_fp8(fp8.kv_append_fp8)
+            survivors.append(name)
+        except AssertionError:
+            pass
+        monkeypatch.setattr(fp8, "e4m3_encode", orig_encode)
+    assert not survivors, f"mutants that survived the pin: {survivors}"
