@@ -122,12 +122,14 @@ def test_fp8_rejects_unsupported_shapes():
 
 def test_llama3_8b_fp8_decode_step_full_size(native):
     """One append + attend step of the Llama-3-8B-shaped batch with an e4m3 KV
-    cache through PagedKVCache: slots equal the allocator model's; for sampled
-    sequences the GPU blocks equal the oracle's (pristine pool + the oracle's
-    quantising append) byte for byte and attention is within tolerance."""
+    cache through PagedKVCache, with distinct K and V scales: slots equal the
+    allocator model's; both pools equal the oracle's (pristine pool + the
+    oracle's quantising append for every sequence) byte for byte; attention
+    of every sequence and head is within tolerance."""
     from paged_kv_cache_406_b200 import workloads as W
     from paged_kv_cache_406_b200.cache import PagedKVCache
     w = W.WORKLOADS["llama3_8b_fp8"]
+    k_scale, v_scale = w.kv_scale, 2 * w.kv_scale
     lens = W.seq_lens(w)
     nb = W.pool_blocks(w, lens)
     order = W.free_order(nb, w.seed)
@@ -136,7 +138,7 @@ def test_llama3_8b_fp8_decode_step_full_size(native):
     v0 = W.pool_values(shape, w, 1, device="cuda")
     maxb = -(-(int(lens.max()) + 1) // w.block_size)
     cache = PagedKVCache(nb, w.num_kv_heads, w.head_dim, w.block_size, w.torch_dtype, maxb, free_order=order,
-                         k_pool=k0.clone(), v_pool=v0.clone(), k_scale=w.kv_scale, v_scale=w.kv_scale)
+                         k_pool=k0.clone(), v_pool=v0.clone(), k_scale=k_scale, v_scale=v_scale)
     model = BlockAllocatorModel(nb, w.block_size, order)
     ids = list(range(w.num_seqs))
     for b in ids:
@@ -145,24 +147,19 @@ def test_llama3_8b_fp8_decode_step_full_size(native):
     q = W.normal((w.num_seqs, w.num_q_heads, w.head_dim), w.io_dtype, W.step_seed(w, 0, 0))
     kn = W.normal((w.num_seqs, w.num_kv_heads, w.head_dim), w.io_dtype, W.step_seed(w, 0, 1))
     vn = W.normal((w.num_seqs, w.num_kv_heads, w.head_dim), w.io_dtype, W.step_seed(w, 0, 2))
-    out = cache.decode_step(ids, q, kn, vn, w.scale)
+    out = cache.decode_step(ids, q, kn, vn, w.scale).cpu()
     torch.cuda.synchronize()
     slots, _ = model.append_slots(ids)
     assert cache._meta_dev[:w.num_seqs].cpu().numpy().tolist() == slots
-    order_len = np.argsort(lens)
-    G = w.group
-    for b in sorted({int(order_len[0]), int(order_len[-1]), 17}):
-        tab = model.block_table(b)
-        idx = torch.tensor(tab, device="cuda")
-        kc = k0[idx].view(torch.uint8).cpu().numpy()
-        vc = v0[idx].view(torch.uint8).cpu().numpy()
-        slot_local = tab.index(slots[b] // w.block_size) * w.block_size + slots[b] % w.block_size
-        kc, vc = fp8.kv_append_fp8(kc, vc, kn[b:b + 1].float().numpy(), vn[b:b + 1].float().numpy(),
-                                   np.array([slot_local]), w.kv_scale, w.kv_scale)
-        assert np.array_equal(cache.k_pool[idx].view(torch.uint8).cpu().numpy(), kc)
-        assert np.array_equal(cache.v_pool[idx].view(torch.uint8).cpu().numpy(), vc)
+    kc, vc = fp8.kv_append_fp8(k0.view(torch.uint8).cpu().numpy(), v0.view(torch.uint8).cpu().numpy(),
+                               kn.float().numpy(), vn.float().numpy(), np.array(slots), k_scale, v_scale)
+    assert np.array_equal(cache.k_pool.view(torch.uint8).cpu().numpy(), kc), "K pool differs from the oracle's"
+    assert np.array_equal(cache.v_pool.view(torch.uint8).cpu().numpy(), vc), "V pool differs from the oracle's"
+    qr = raw(q)
+    for b in ids:
+        tab = np.asarray(model.block_table(b))
         local = np.arange(len(tab), dtype=np.int32)[None]
-        ref = fp8.paged_decode_attention_fp8(raw(q[b:b + 1]), kc, vc, local, np.array([model.seq_len(b)]), w.scale,
-                                             w.kv_scale, w.kv_scale)
+        ref = fp8.paged_decode_attention_fp8(qr[b:b + 1], kc[tab], vc[tab], local, np.array([model.seq_len(b)]),
+                                             w.scale, k_scale, v_scale)
         assert_close(out[b:b + 1], ref, "f16", f"fp8 llama3 seq {b}")
-    assert G == 4
+    assert w.group == 4

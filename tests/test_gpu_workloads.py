@@ -1,8 +1,13 @@
 """GPU parity on the five seeded workloads at their full sizes (B200).
 
-Every step's slot mapping must equal the allocator model's; sampled sequences'
-pool blocks must equal the oracle's byte for byte, and their attention output
-must be within tolerance of the fp64 oracle.
+Every step's slot mapping must equal the allocator model's; the checked
+sequences' pool blocks must equal the oracle's byte for byte, and their
+attention output, for every KV head, must be within tolerance of the fp64
+oracle.  The Llama-3-8B-shaped, prefix-shared and long split-K batches are
+checked in full (every sequence, every head); the 50-step MHA batch in full at
+its first and last step and on a rotating eighth of its sequences at every
+step in between, so a work-assignment slip that touches only some (sequence,
+partition, head) units cannot hide.
 """
 import pytest
 
@@ -14,10 +19,7 @@ pytestmark = pytest.mark.gpu
 
 def test_llama3_8b_decode_layer(native):
     w = W.WORKLOADS["llama3_8b"]
-    lens = W.seq_lens(w)
-    order = sorted(range(w.num_seqs), key=lambda b: lens[b])
-    sample = {order[0], order[1], order[len(order) // 2], order[-2], order[-1], 7}
-    st = run_workload(w, sample, check=lambda step, b: True)
+    st = run_workload(w, None, check=lambda step, b: True)
     assert st["num_seqs"] == 64
 
 
@@ -34,14 +36,13 @@ def test_prefix_shared_batch(native, bs, prefix):
 
 def test_long_context_split_k(native):
     w = W.WORKLOADS["long_splitk"]
-    run_workload(w, {0, 7}, check=lambda step, b: True, heads=[0, 5])
+    run_workload(w, None, check=lambda step, b: True)
 
 
 def test_mha_7b_fifty_steps(native):
-    """Steps 0 and 49 checked for four sequences (the longest among them),
-    and one sequence at every step."""
+    """All 256 sequences and 32 heads at steps 0 and 49; at every step in
+    between, the sequences b with b % 8 == step % 8 (each sequence checked
+    six times over the run)."""
     w = W.WORKLOADS["mha_7b"]
-    lens = W.seq_lens(w)
-    longest = int(lens.argmax())
-    sample = {0, 100, 200, longest}
-    run_workload(w, sample, check=lambda step, b: step in (0, w.steps - 1) or b == 100, heads=[0, 13, 31])
+    last = w.steps - 1
+    run_workload(w, None, check=lambda step, b: step in (0, last) or b % 8 == step % 8)

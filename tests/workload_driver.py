@@ -1,10 +1,13 @@
 """Runs a seeded workload through the library (PagedKVCache) and mirrors every
-step on the oracle side for a sample of sequences.
+step on the oracle side.
 
-The oracle side never reads a value the CUDA path produced: its pool blocks
-come from the pristine initial pool (torch's seeded generator), its slots and
-tables from the oracle's own allocator model, and its appended rows from the
-step's seeded inputs.  GPU results are compared after each checked step.
+The oracle side never reads a value the CUDA path produced: its pool starts as
+a host copy of the pristine initial pool (torch's seeded generator), its slots,
+tables and copy-on-write pairs come from the oracle's own allocator model, and
+its appended rows from the step's seeded inputs.  The host pool is kept up to
+date for every sequence (copy-on-write copies and appends applied in place, as
+the oracle's ``copy_blocks`` and ``kv_append`` define them), so any checked
+sequence can be compared at any step.
 """
 from __future__ import annotations
 
@@ -19,40 +22,42 @@ from paged_kv_cache_406_b200 import workloads as W
 from paged_kv_cache_406_b200.cache import PagedKVCache
 
 
-class Mirror:
-    """Host copies of the blocks the sampled sequences use (compact ids)."""
+class HostPool:
+    """The oracle's copy of both pools, raw storage, updated in place."""
 
-    def __init__(self, k0: torch.Tensor, v0: torch.Tensor):
-        self.k0, self.v0 = k0, v0
-        self.ids: dict[int, int] = {}
-        self.k: list[np.ndarray] = []
-        self.v: list[np.ndarray] = []
+    def __init__(self, k0: torch.Tensor, v0: torch.Tensor, bs: int):
+        self.k, self.v, self.bs = raw(k0).copy(), raw(v0).copy(), bs
 
-    def block(self, phys: int) -> int:
-        if phys not in self.ids:
-            self.ids[phys] = len(self.k)
-            self.k.append(raw(self.k0[phys]).copy())
-            self.v.append(raw(self.v0[phys]).copy())
-        return self.ids[phys]
+    def copy(self, pairs) -> None:
+        # copy_blocks: whole blocks src -> dst, in order
+        for src, dst in pairs:
+            self.k[dst] = self.k[src]
+            self.v[dst] = self.v[src]
 
-    def append(self, slot: int, krow: np.ndarray, vrow: np.ndarray, bs: int) -> None:
-        blk, off = divmod(int(slot), bs)
-        c = self.block(blk)
-        self.k[c][:, off, :] = krow
-        self.v[c][:, off, :] = vrow
+    def append(self, slots, krows: np.ndarray, vrows: np.ndarray) -> None:
+        # kv_append: row i into block slot // bs at offset slot % bs; slot < 0 writes nothing
+        for i, s in enumerate(slots):
+            if s < 0:
+                continue
+            blk, off = divmod(int(s), self.bs)
+            self.k[blk, :, off, :] = krows[i]
+            self.v[blk, :, off, :] = vrows[i]
 
-    def copy(self, src: int, dst: int) -> None:
-        s, d = self.block(src), self.block(dst)
-        self.k[d] = self.k[s].copy()
-        self.v[d] = self.v[s].copy()
 
+def compare_pools(cache: PagedKVCache, host: HostPool, what: str) -> None:
+    """Every byte of both device pools against the oracle's host pools."""
+    assert np.array_equal(raw(cache.k_pool), host.k), f"{what}: K pool differs from the oracle's"
+    assert np.array_equal(raw(cache.v_pool), host.v), f"{what}: V pool differs from the oracle's"
 
 
 def run_workload(w: W.Workload, sample, check, steps=None, prefix_tokens=None, heads=None):
-    """Runs ``steps`` decode steps of ``w``; after each step, for every sampled
-    sequence b with ``check(step, b)`` true, compares its blocks byte for byte
-    and its attention output (KV heads ``heads``, all if None) with the oracle.
-    ``sample``: sequence indices mirrored on the host (None = all).
+    """Runs ``steps`` decode steps of ``w``.  After each step the slot
+    mapping is compared with the allocator model's, and for every sequence b
+    in ``sample`` (None = all) with ``check(step, b)`` true the attention
+    output (KV heads ``heads``, None = all) is compared with the fp64 oracle.
+    Both pools are compared byte for byte in full after the prefix phase,
+    after the first step and after the last one (pools only grow, so a wrong
+    write at any step is still there at the end).
     Returns the allocator stats after the last step."""
     steps = w.steps if steps is None else steps
     dt = w.torch_dtype
@@ -68,10 +73,11 @@ def run_workload(w: W.Workload, sample, check, steps=None, prefix_tokens=None, h
     v0 = W.normal(shape, dt, W.pool_seed(w, 1), device="cuda")
     maxb = -(-(int(lens.max()) + steps) // bs)
     cache = PagedKVCache(nb, hkv, d, bs, dt, maxb, free_order=order, k_pool=k0.clone(), v_pool=v0.clone())
+    host = HostPool(k0, v0, bs)
+    del k0, v0
     model = BlockAllocatorModel(nb, bs, order)
     B = w.num_seqs
     sample = set(range(B)) if sample is None else set(sample)
-    mirror = Mirror(k0, v0)
     rng = np.random.default_rng(w.seed + 77)
 
     # ---- admit the batch (shared prefix: one sequence, forked, then tails) ----
@@ -93,13 +99,11 @@ def run_workload(w: W.Workload, sample, check, steps=None, prefix_tokens=None, h
             vn = W.normal((len(ids), hkv, d), dt, int(rng.integers(1 << 30)))
             if ncow:
                 pkv_copy_blocks(cache.k_pool, cache.v_pool, dcow[:2 * ncow].view(ncow, 2))
-                for s_, d_ in mcow:
-                    mirror.copy(s_, d_)
+                host.copy(mcow)
             pkv_kv_append(kn.cuda(), vn.cuda(), dslots, cache.k_pool, cache.v_pool)
-            kr, vr = raw(kn), raw(vn)
-            for i, b in enumerate(ids):
-                if b in sample:
-                    mirror.append(mslots[i], kr[i], vr[i], bs)
+            host.append(mslots, raw(kn), raw(vn))
+        torch.cuda.synchronize()
+        compare_pools(cache, host, f"{w.name} after the prefix phase")
     else:
         for b in range(B):
             cache.add(b, int(lens[b]))
@@ -108,8 +112,7 @@ def run_workload(w: W.Workload, sample, check, steps=None, prefix_tokens=None, h
     for step in range(steps):
         ids = list(range(B))
         mslots, mcow = model.append_slots(ids)
-        for s_, d_ in mcow:
-            mirror.copy(s_, d_)
+        host.copy(mcow)
         q = W.normal((B, hq, d), dt, W.step_seed(w, step, 0))
         kn = W.normal((B, hkv, d), dt, W.step_seed(w, step, 1))
         vn = W.normal((B, hkv, d), dt, W.step_seed(w, step, 2))
@@ -117,24 +120,22 @@ def run_workload(w: W.Workload, sample, check, steps=None, prefix_tokens=None, h
         torch.cuda.synchronize()
         gslots = cache._meta_dev[:B].cpu().numpy()
         assert gslots.tolist() == mslots, f"step {step}: slot mapping differs from the allocator model"
-        kr, vr, qr = raw(kn), raw(vn), raw(q)
-        for b in sample:
-            mirror.append(mslots[b], kr[b], vr[b], bs)
+        qr = raw(q)
+        host.append(mslots, raw(kn), raw(vn))
+        if step in (0, steps - 1):
+            compare_pools(cache, host, f"{w.name} step {step}")
+        out_h = out.cpu()
         for b in sorted(sample):
             if not check(step, b):
                 continue
-            tab = model.block_table(b)
+            tab = np.asarray(model.block_table(b))
             L = model.seq_len(b)
-            ks = np.stack([mirror.k[mirror.block(p)] for p in tab])
-            vs = np.stack([mirror.v[mirror.block(p)] for p in tab])
-            idx = torch.tensor(tab, device="cuda")
-            assert np.array_equal(raw(cache.k_pool[idx]), ks), f"K blocks of seq {b} differ at step {step}"
-            assert np.array_equal(raw(cache.v_pool[idx]), vs), f"V blocks of seq {b} differ at step {step}"
             local = np.arange(len(tab), dtype=np.int32)[None]
+            ks, vs = host.k[tab], host.v[tab]
             for g in (range(hkv) if heads is None else heads):
                 ref = pa.paged_decode_attention(qr[b:b + 1, g * G:(g + 1) * G], ks[:, g:g + 1], vs[:, g:g + 1],
                                                 local, np.array([L]), w.scale, w.dtype)
-                assert_close(out[b:b + 1, g * G:(g + 1) * G], ref, w.dtype,
+                assert_close(out_h[b:b + 1, g * G:(g + 1) * G], ref, w.dtype,
                              f"{w.name} step {step} seq {b} kv head {g}")
     assert pkv_device_status(clear=True) == 0
     return cache.stats()
