@@ -199,3 +199,39 @@ def test_kv_append_fp8_planted_mistakes_are_caught(monkeypatch):
             pass
         monkeypatch.setattr(fp8, "e4m3_encode", orig_encode)
     assert not survivors, f"mutants that survived the pin: {survivors}"
+
+
+def test_decode_over_full_range_codes_needs_p_as_hi_and_lo():
+    """Why the e4m3 decode kernel feeds the softmax weights P to its f16
+    tensor-core products as two halves (hi + lo) rather than one f16 value:
+    over pools whose codes span the whole e4m3 range (V up to 448 * v_scale),
+    a single f16 P (11 significant bits) misses the 2e-3 output tolerance,
+    while hi + lo (about 22 bits) stays far inside it.  Both products are
+    simulated here in float64 from the rounded weights, the sum of weights in
+    fp32 as the kernel keeps it; the reference is the oracle's definition."""
+    rng = np.random.default_rng(5)
+
+    def codes(shape):
+        c = rng.integers(0, 256, size=shape).astype(np.uint8)
+        c[(c & 0x7F) == 0x7F] ^= 1  # no NaN codes
+        return c
+
+    worst_single, worst_pair = 0.0, 0.0
+    for _ in range(60):
+        L = int(rng.integers(1, 2000))
+        kc, vc = codes((1, 1, L, 128)), codes((1, 1, L, 128))
+        q = rng.standard_normal((1, 1, 128)).astype(np.float16)
+        ref = fp8.paged_decode_attention_fp8(q, kc, vc, np.zeros((1, 1), np.int32), np.array([L]), 1 / np.sqrt(128),
+                                             0.25, 0.5)[0, 0]
+        K = fp8.e4m3_decode(kc[0, 0]) * 0.25
+        V = fp8.e4m3_decode(vc[0, 0]) * 0.5
+        s = K @ q[0, 0].astype(np.float64) / np.sqrt(128)
+        p = np.exp(s - s.max()).astype(np.float32)
+        hi = p.astype(np.float16).astype(np.float64)
+        lo = (p.astype(np.float64) - hi).astype(np.float16).astype(np.float64)
+        den = float(p.astype(np.float64).sum())
+        tol = 2e-3 * np.maximum(1.0, np.abs(ref))
+        worst_single = max(worst_single, float(np.max(np.abs(hi @ V / den - ref) / tol)))
+        worst_pair = max(worst_pair, float(np.max(np.abs((hi + lo) @ V / den - ref) / tol)))
+    assert worst_single > 1.0, "a single f16 P would meet the tolerance here: the lo half would be unnecessary"
+    assert worst_pair < 0.05
