@@ -25,6 +25,8 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
+import threading
 import time
 
 import numpy as np
@@ -37,10 +39,14 @@ METRIC = "paged decode attention: KV GB/s (fraction of B200 HBM peak), tokens/s 
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_SUSTAINED = 1400.0  # TFLOP/s, dense bf16 under the power cap
 STAGED_STEPS = 16  # distinct steps of metadata resident on the device, cycled
-# The library call inside a step is bracketed by CUDA events on every
-# EVENT_EVERY-th timed step only (its average duration is the roofline's
-# `avg_launch_ms`): a pair of timing events on every step added about 5 us to
-# a 103 us decode step, and the step rate is the headline number.
+# Where a step holds more than the timed library call (copy-on-write copies,
+# the prefill's append), the call is bracketed by its own CUDA events on every
+# EVENT_EVERY-th timed step from the second on, or on every step from the
+# second on when there are fewer than 4 such samples (a pair of timing events
+# on every step added about 5 us to a 103 us decode step).  Where the call is
+# the whole step, one event after the first step and the end event bracket
+# steps 2..K: the first step starts on an idle GPU right after a synchronise
+# and carries the host's launch latency.
 EVENT_EVERY = 16
 
 # DRAM traffic of one pkv_append_and_decode call per workload, from the ncu
@@ -97,7 +103,21 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the CPU oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--num-seqs", type=int, default=0,
+                    help="a smaller batch of the workload's shape (for profiler captures); 0: the workload's own")
     return ap.parse_args()
+
+
+def workload_of(args):
+    """The named workload, with the batch cut to --num-seqs when given."""
+    from dataclasses import replace
+    from paged_kv_cache_406_b200 import workloads as W
+    w = W.WORKLOADS[args.workload]
+    if args.num_seqs > 0:
+        w = replace(w, num_seqs=args.num_seqs)
+    if getattr(args, "partition_tokens", -1) >= 0:
+        w = replace(w, partition_tokens=args.partition_tokens)
+    return w
 
 
 def dist_env():
@@ -147,51 +167,140 @@ def measured_peaks():
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, power and clock-event reasons of this process's GPU during
+    the timed region, read through NVML (the library nvidia-smi reads): a
+    background thread samples from the start of the region, pausing
+    ``period_s`` between readings, and :meth:`sample` takes one reading on
+    the calling thread, which the timed loops do right after their last
+    launch, while the GPU still works through its queue.  One reading takes
+    milliseconds, so the launching thread never samples mid-region: that
+    starved the GPU of a 20-step region for the reading's duration.  Without
+    the NVML binding, ``nvidia-smi -lms 200`` writes into a temporary file."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+    SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int, enabled: bool):
-        self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+    def __init__(self, device_index: int, enabled: bool, period_s: float = 0.005):
+        self.readings = []  # (sm MHz, reason bits, power W)
+        self.nv = self.h = self.thread = self.proc = None
+        self.max_mhz = None
         if not enabled:
             return
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = self._handle(device_index)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self.bits = {name: int(getattr(pynvml, attr, 0)) for name, attr in self.REASONS}
+        except Exception:
+            self.nv = self.h = None
+            self._start_smi(device_index)
+            return
+        self.stop_ev = threading.Event()
+        self.go = threading.Event()
+        self.period = period_s
+        self.thread = threading.Thread(target=self._loop, daemon=True)
+        self.thread.start()
+
+    def begin(self):
+        """Called right after the timed region's start event: readings start."""
+        if self.thread is not None:
+            self.go.set()
+
+    def _handle(self, device_index: int):
+        nv = self.nv
+        props = torch.cuda.get_device_properties(device_index)
+        uuid = str(getattr(props, "uuid", ""))
+        for u in (uuid, "GPU-" + uuid):
+            try:
+                return nv.nvmlDeviceGetHandleByUUID(u)
+            except Exception:
+                pass
+        try:
+            bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(device_index)
+
+    def sample(self):
+        if self.h is None:
+            return
+        nv = self.nv
+        try:
+            mhz = float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+            bits = int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            watts = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+        except Exception:
+            return
+        self.readings.append((mhz, bits, watts))
+
+    def _loop(self):
+        while not self.go.wait(0.05):
+            if self.stop_ev.is_set():
+                return
+        while not self.stop_ev.is_set():
+            self.sample()
+            self.stop_ev.wait(self.period)
+
+    def _start_smi(self, device_index: int):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="pkv_clocks_", suffix=".csv")
+            self.f = os.fdopen(fd, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
-                 "-i", str(gpu_index)], stdout=self.f, stderr=subprocess.DEVNULL)
+                ["nvidia-smi", f"--query-gpu={self.SMI_FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(device_index)], stdout=self.f, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
 
-    def stop(self):
-        if self.proc is None:
-            return None
+    def _stop_smi(self):
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.f.close()
-        sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
+        sm, smax, reasons = [], [], set()
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": "nvidia-smi"}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvidia-smi -lms 200"}
+
+    def stop(self):
+        if self.proc is not None:
+            return self._stop_smi()
+        if self.h is None:
+            return None
+        self.stop_ev.set()
+        self.go.set()
+        self.thread.join(timeout=5)
+        r = list(self.readings)
+        reasons = sorted({name for _, bits, _ in r for name, bit in self.bits.items() if bit and bits & bit})
+        return {"sm_mhz": statistics.median(m for m, _, _ in r) if r else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(r),
+                "power_w": round(statistics.median(w for _, _, w in r), 1) if r else None,
+                "source": "NVML during the timed region (a thread reading from its start, %.0f ms between "
+                          "readings, plus one read right after the last launch)" % (self.period * 1e3)}
 
 
 # ---------------------------------------------------------------------------
@@ -285,6 +394,14 @@ def setup(w, device, horizon):
     return w, cache, lens
 
 
+def sampled_steps(K: int) -> list:
+    """Timed steps whose call gets its own event pair: every EVENT_EVERY-th
+    from the second on, or every step from the second on when that would give
+    fewer than 4 samples."""
+    every = list(range(1, K, EVENT_EVERY))
+    return every if len(every) >= 4 else list(range(1, K)) or [0]
+
+
 def decode_launches(max_blocks: int, block_size: int, partition_tokens: int) -> int:
     """Kernels one pkv_paged_attention_decode (or pkv_append_and_decode) call
     launches: the plan (or append + plan) and decode kernels, plus the
@@ -305,10 +422,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    w0 = W.WORKLOADS[args.workload]
-    if args.partition_tokens >= 0:
-        from dataclasses import replace
-        w0 = replace(w0, partition_tokens=args.partition_tokens)
+    w0 = workload_of(args)
     horizon = STAGED_STEPS + 3 + max(0, args.e2e_steps) + 8
     w, cache, lens0 = setup(rank_workload(w0, rank), dev, horizon)
     B, hq, hkv, d, bs = w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size
@@ -378,24 +492,42 @@ def run_ours(args):
     assert P.pkv_device_status(clear=True) == 0
 
     K = args.steps
-    sampled = list(range(0, K, EVENT_EVERY))
+    # roofline timing of the call (see EVENT_EVERY): the call is the whole
+    # step unless the step also copies blocks for copy-on-write
+    cow_in_steps = any(staged[(args.warmup + i) % STAGED_STEPS]["ncow"] for i in range(K))
+    sampled = sampled_steps(K) if cow_in_steps else []
     evs = {i: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for i in sampled}
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    after_first = torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local, not args.no_clocks)
     if ws > 1:
         dist.barrier()
     torch.cuda.synchronize()
     start.record()
+    clocks.begin()
     launches = 0
     for i in range(K):
         launches += step(args.warmup + i, evs.get(i))
+        if i == 0:
+            after_first.record()
     end.record()
+    clocks.sample()
     torch.cuda.synchronize()
     if ws > 1:
         dist.barrier()
     clk = clocks.stop()
     elapsed_ms = start.elapsed_time(end)
-    dec_ms = [evs[i][0].elapsed_time(evs[i][1]) for i in sampled]
+    if sampled:
+        dec_ms = [evs[i][0].elapsed_time(evs[i][1]) for i in sampled]
+        launch_timing = f"event pairs around the call on timed steps {sampled[:3]}... ({len(sampled)} samples)"
+    elif K > 1:
+        dec_ms = [after_first.elapsed_time(end) / (K - 1)]
+        sampled = list(range(1, K))
+        launch_timing = f"one event pair around timed steps 2..{K} (the call is the whole step)"
+    else:
+        dec_ms = [elapsed_ms]
+        sampled = [0]
+        launch_timing = "the single timed step"
     status = P.pkv_device_status(clear=True)
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
@@ -409,6 +541,8 @@ def run_ours(args):
 
     peak, peak_kind = measured_peaks()
     dec_avg_ms = float(np.mean(dec_ms))
+    # the call cannot outlast the step it is part of (a check on the timing itself)
+    assert dec_avg_ms <= elapsed_ms / K * 1.02, (dec_avg_ms, elapsed_ms / K)
     achieved = float(np.mean(step_algo)) / (dec_avg_ms * 1e-3) / 1e9
     sha = kernel_source_sha()
     pin = TRAFFIC.get(w.name)
@@ -441,6 +575,7 @@ def run_ours(args):
             qh, kh, vh = host_in[s % len(host_in)]
             cache.decode_step_host(ids_np, qh, kh, vh, w.scale, out_host=out_host,
                                    partition_tokens=w.partition_tokens)
+        cache.wait_copies()  # the last step's result copy back is inside the timed region
         e1.record()
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
@@ -493,7 +628,7 @@ def run_ours(args):
                          "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
                          "traffic": traffic, "algorithmic_bytes_per_launch": int(np.mean(step_algo)),
                          "avg_launch_ms": round(dec_avg_ms, 5), "launch_samples": len(sampled),
-                         "kernel_source_sha": sha},
+                         "launch_timing": launch_timing, "kernel_source_sha": sha},
             "gpu_launches": launches, "clocks": clk, "cpu_baseline": cpu, "e2e": e2e,
             "allocator": alloc_stats,
         }
@@ -565,15 +700,20 @@ def run_prefill(args, w0):
     kn = W.normal((T, hkv, d), w.torch_dtype, W.step_seed(w, 0, 1), device=dev)
     vn = W.normal((T, hkv, d), w.torch_dtype, W.step_seed(w, 0, 2), device=dev)
     out = torch.empty((T, hq, d), dtype=torch.float32, device=dev)
+    # bf16 pools: V of the batch staged as f16 once per call (one f16 P·V pass)
+    pf_ws = torch.empty(max(1, P.pkv_prefill_workspace_size(B, hkv, d, maxb, bs, w.torch_dtype)), dtype=torch.uint8,
+                        device=dev)
+    staged = w.torch_dtype == torch.bfloat16
 
     def step(ev=None):
         P.pkv_kv_append(kn, vn, slot_d, cache.k_pool, cache.v_pool)
         if ev is not None:
             ev[0].record()
-        P.pkv_paged_attention_prefill(q, cache.k_pool, cache.v_pool, tables_d, lens_d, q_start, n, w.scale, out=out)
+        P.pkv_paged_attention_prefill(q, cache.k_pool, cache.v_pool, tables_d, lens_d, q_start, n, w.scale, out=out,
+                                      workspace=pf_ws)
         if ev is not None:
             ev[1].record()
-        return 2
+        return 3 if staged else 2
 
     for _ in range(args.warmup):
         step()
@@ -581,17 +721,19 @@ def run_prefill(args, w0):
     assert P.pkv_device_status(clear=True) == 0
     K = args.steps
     evs = {i: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for i in range(0, K, EVENT_EVERY)}
+           for i in sampled_steps(K)}
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local, not args.no_clocks)
     if ws > 1:
         dist.barrier()
     torch.cuda.synchronize()
     start.record()
+    clocks.begin()
     launches = 0
     for i in range(K):
         launches += step(evs.get(i))
     end.record()
+    clocks.sample()
     torch.cuda.synchronize()
     if ws > 1:
         dist.barrier()
@@ -631,7 +773,8 @@ def run_prefill(args, w0):
             vd.copy_(hv_in, non_blocking=True)
             P.pkv_kv_append(kd, vd, meta_d[:ns], cache.k_pool, cache.v_pool)
             P.pkv_paged_attention_prefill(qd, cache.k_pool, cache.v_pool, meta_d[ns:ns + nt].view(B, maxb),
-                                          meta_d[ns + nt:ns + nt + B], meta_d[ns + nt + B:], n, w.scale, out=out)
+                                          meta_d[ns + nt:ns + nt + B], meta_d[ns + nt + B:], n, w.scale, out=out,
+                                          workspace=pf_ws)
             out_h.copy_(out, non_blocking=True)
 
         for _ in range(3):
@@ -688,14 +831,15 @@ def run_prefill(args, w0):
                        "l2": "inputs larger than L2: %.0f MB of K/V + %.0f MB of q and out per step, no flush"
                              % (int(L.sum()) * hkv * d * 4 / 1e6, T * hq * d * 6 / 1e6),
                        "parallelism": f"replicas x{ws} (independent batches per GPU)"},
-            "roofline": {"kernel": "pkv_paged_attention_prefill (prefill_tc_kernel)", "bound": "tensor",
+            "roofline": {"kernel": "pkv_paged_attention_prefill (stage_v_f16_kernel for bf16 pools, prefill_tc_kernel)",
+                         "bound": "tensor",
                          "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(achieved / peak, 4), "peak_source": peak_kind,
                          "burst_peak": peaks.get("bf16_tflops"),
                          "traffic": traffic, "traffic_unit": "bytes (DRAM read + write per launch)",
                          "algorithmic_flops_per_launch": flops,
-                         "tensor_flops_issued_per_launch": "1.5x algorithmic (P·V runs on P hi and P lo) plus the "
-                                                          "masked part of diagonal chunks",
+                         "tensor_flops_issued_per_launch": "algorithmic plus the masked part of diagonal chunks "
+                                                          "(one f16 P·V pass; bf16 V staged as f16 by the call)",
                          "avg_launch_ms": round(attn_ms, 5), "launch_samples": len(evs),
                          "kernel_source_sha": pf_sha},
             "gpu_launches": launches, "clocks": clk, "cpu_baseline": cpu, "e2e": e2e,
@@ -756,20 +900,35 @@ def run_adaptive(args, w):
         wsb = P.pkv_decode_workspace_size(len(members), hq, hkv, d, cache.max_blocks, cache.block_size, 0)
         return out, torch.empty(wsb, dtype=torch.uint8, device=dev)
 
-    arms = {"adaptive": [], "fixed_bs16": [], "fixed_bs32": [], "fixed_bs8": []}
+    # "adaptive": every class in one pkv_append_and_decode_pools call per step;
+    # "adaptive_per_class": one pkv_append_and_decode call per class (same
+    # staged metadata); "fixed_bsN": one pool of N-token blocks for the batch
+    arms = {"adaptive": [], "adaptive_per_class": [], "fixed_bs16": [], "fixed_bs32": [], "fixed_bs8": []}
     a = 0
     for bs in ad.CLASSES:
         members = [i for i in ids if ad.cls[i] == bs]
         if members:
             st, wsp = stage(ad.caches[bs], members)
-            arms["adaptive"].append((ad.caches[bs], st, wsp, slice(a, a + len(members))))
+            arms["adaptive_per_class"].append((ad.caches[bs], st, wsp, slice(a, a + len(members))))
             a += len(members)
     for fbs, c in fixed.items():
         st, wsp = stage(c, ids)
         arms[f"fixed_bs{fbs}"].append((c, st, wsp, slice(0, B)))
+    per_class = arms["adaptive_per_class"]
+    one_call = []
+    for k in range(STAGED_STEPS):
+        pools = [(c.k_pool, c.v_pool, st[k][1], sl.stop - sl.start) for c, st, _, sl in per_class]
+        one_call.append((pools, torch.cat([st[k][0] for _, st, _, _ in per_class]),
+                         torch.cat([st[k][2] for _, st, _, _ in per_class])))
+    pools_ws = torch.empty(P.pkv_decode_pools_workspace_size(one_call[0][0], hq), dtype=torch.uint8, device=dev)
+    arms["adaptive"] = [(c, st, None, sl) for c, st, _, sl in per_class]  # for the byte and block accounting
     out = torch.empty((B, hq, d), dtype=torch.float32, device=dev)
 
     def step(arm, i):
+        if arm == "adaptive":
+            pools, slots, lens = one_call[i % STAGED_STEPS]
+            P.pkv_append_and_decode_pools(pools, kn, vn, slots, q, lens, w.scale, out=out, workspace=pools_ws)
+            return decode_launches(max(c.max_blocks * c.block_size for c, _, _, _ in per_class) // 16, 16, 0)
         for cache, st, wsp, sl in arms[arm]:
             slots, tables, lens, _ = st[i % STAGED_STEPS]
             P.pkv_append_and_decode(kn[sl], vn[sl], slots, q[sl], cache.k_pool, cache.v_pool, tables, lens, w.scale,
@@ -785,16 +944,18 @@ def run_adaptive(args, w):
         torch.cuda.synchronize()
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s0.record()
+        clocks.begin()
         for i in range(args.steps):
             launches += step(arm, args.warmup + i)
         s1.record()
+        clocks.sample()
         torch.cuda.synchronize()
         ms = s0.elapsed_time(s1)
         nbytes = sum(int(st[(args.warmup + i) % STAGED_STEPS][3].astype(np.int64).sum()) * hkv * d * 2 * e
                      for i in range(args.steps) for _, st, _, _ in arms[arm])
         res_arms[arm] = {"kv_gb_s": round(nbytes / (ms * 1e-3) / 1e9, 1), "ms_per_step": round(ms / args.steps, 5),
                          "tokens_per_s_per_layer": round(B * args.steps / (ms * 1e-3), 1),
-                         "calls_per_step": len(arms[arm]),
+                         "calls_per_step": 1 if arm == "adaptive" else len(arms[arm]),
                          "pool_blocks": {str(c.block_size): c.num_blocks for c, _, _, _ in arms[arm]},
                          "waste_tokens": sum(c.stats()["waste_tokens"] for c, _, _, _ in arms[arm])}
     clk = clocks.stop()
@@ -880,7 +1041,7 @@ def run_reference(args):
     if rank != 0:
         return
     from paged_kv_cache_406_b200 import workloads as W
-    w = W.WORKLOADS[args.workload]
+    w = workload_of(args)
     if w.chunk_tokens:
         return run_reference_prefill(args, w, ws)
     lens = W.seq_lens(w)
@@ -977,8 +1138,7 @@ def main():
     else:
         if not torch.cuda.is_available():
             raise SystemExit("bench.py needs a CUDA GPU (B200); use --impl reference for the CPU oracle")
-        from paged_kv_cache_406_b200 import workloads as W
-        w = W.WORKLOADS[args.workload]
+        w = workload_of(args)
         if w.chunk_tokens:
             run_prefill(args, w)
         elif w.name == "adaptive_mix":

@@ -336,10 +336,19 @@ int pkv_decode_step_host(pkv_alloc_t* a, const int64_t* seq_ids, int32_t n, cons
  * PKV_ERR_UNSUPPORTED.  q, pools and out 16-byte aligned; scale positive
  * and finite (else PKV_ERR_INVALID_ARG).
  * Computed on the tcgen05 tensor cores with fp32 accumulation.  The
- * softmax weights P enter the P·V product as two bf16 halves (hi + lo) for
- * bf16 pools, within about 1e-5 of the exact softmax, and as one f16 value
- * for f16 pools (relative error 2^-11 per weight; the output within about
- * 5e-4 of the output scale).  A sequence whose chunk is longer than
+ * softmax weights P enter the P·V product as one f16 value (relative error
+ * 2^-11 per weight; the output within about 5e-4 of the output scale) for
+ * f16 pools, and for bf16 pools given a workspace: the call then first
+ * copies V of every block the batch reaches into the workspace as f16 (exact
+ * for bf16 magnitudes in [2^-14, 65504], smaller ones rounded to f16
+ * subnormals, absolute error at most 2^-25) and the P·V product reads the
+ * copy.  Without a workspace (NULL), or if some V value of the batch lies
+ * beyond the f16 range, bf16 pools take two bf16 passes (P as hi + lo
+ * halves, within about 1e-5 of the exact softmax) over the pool's own V.
+ * workspace: at least pkv_prefill_workspace_size() bytes of device memory,
+ * 256-byte aligned, owned by the caller and overwritten by the call (NULL or
+ * ignored for f16 pools); calls that overlap on the GPU need their own.  A
+ * sequence whose chunk is longer than
  * seq_lens[b] or max_q_len is skipped and recorded as PKV_ERR_INVALID_ARG;
  * table entries outside [0, num_blocks) as PKV_ERR_BAD_BLOCK (block 0 read
  * instead), both in the device status.  The kernel runs one CTA per SM,
@@ -351,8 +360,17 @@ int pkv_paged_attention_prefill(const void* q, const void* k_pool, const void* v
                                 const int32_t* q_start, int32_t num_seqs, int32_t num_q_tokens,
                                 int32_t max_q_len, int32_t num_q_heads, int32_t num_kv_heads,
                                 int32_t head_dim, int32_t num_blocks, int32_t max_blocks_per_seq,
-                                int32_t block_size, float scale, int32_t dtype, float* out,
-                                void* stream);
+                                int32_t block_size, float scale, int32_t dtype, void* workspace,
+                                size_t workspace_bytes, float* out, void* stream);
+
+/* Bytes of the workspace pkv_paged_attention_prefill takes for a batch of
+ * num_seqs sequences with tables of max_blocks_per_seq entries: for bf16
+ * pools a 256-byte record plus the f16 copy of V,
+ * [num_seqs][max_blocks_per_seq][num_kv_heads][block_size][head_dim]
+ * (2 bytes per element); 0 for f16 pools.  Host only, no device access. */
+int pkv_prefill_workspace_size(int32_t num_seqs, int32_t num_kv_heads, int32_t head_dim,
+                               int32_t max_blocks_per_seq, int32_t block_size, int32_t dtype,
+                               size_t* bytes);
 
 /* PagedAttention decode exactly as pkv_paged_attention_decode, for callers
  * that cannot allocate device memory when they decode: serving runtimes that
@@ -420,6 +438,47 @@ int pkv_paged_attention_decode_fp8(const void* q, const void* k_pool, const void
                                    float v_scale, int32_t partition_tokens, void* workspace, size_t workspace_bytes,
                                    float* out, void* stream);
 
+/* One pool of a batch that spans several pools (adaptive block size,
+ * "LLM inference optimisation: principles overview" §3.3: pools of 32-, 16-
+ * and 8-token blocks for short, medium and long sequences).  The pool's
+ * sequences are the next num_seqs rows of the batch, in pool order; row r of
+ * block_tables is the pool's r-th sequence.  Layouts as for a single pool. */
+typedef struct pkv_pool {
+  void* k_pool;                 /* [num_blocks][num_kv_heads][block_size][head_dim] */
+  void* v_pool;
+  const int32_t* block_tables;  /* [num_seqs][max_blocks_per_seq], physical blocks of this pool */
+  int32_t num_blocks;
+  int32_t block_size;           /* 8, 16 or 32 */
+  int32_t max_blocks_per_seq;
+  int32_t num_seqs;             /* may be 0 */
+} pkv_pool_t;
+
+/* Workspace bytes of pkv_append_and_decode_pools for these pools (sizes
+ * only; the pointers are not read).  Host only. */
+int pkv_decode_pools_workspace_size(const pkv_pool_t* pools, int32_t n_pools, int32_t num_q_heads,
+                                    int32_t num_kv_heads, int32_t head_dim, int32_t partition_tokens,
+                                    size_t* bytes);
+
+/* pkv_append_and_decode over a batch whose sequences live in up to 3 pools of
+ * different block sizes, in one launch sequence (append + plan, decode,
+ * merge) instead of one call per pool.  Row b of k_new / v_new [N][Hkv][D],
+ * slot_mapping [N], q [N][Hq][D], seq_lens [N] and out [N][Hq][D] belongs to
+ * pool c for sum_{i<c} num_seqs_i <= b < sum_{i<=c} num_seqs_i (N = the sum
+ * over the pools); slot_mapping[b] is a slot of that pool (< 0: nothing
+ * written), seq_lens[b] counts its tokens after the append.  Every sequence
+ * gets the result pkv_append_and_decode would give on its own pool (equal
+ * within rounding: the work of a batch is shared out differently).  dtype
+ * PKV_BF16 or PKV_F16, head_dim 128, num_q_heads / num_kv_heads in {2, 4, 8},
+ * 1 <= n_pools <= 3, partition_tokens (0 = 512) a multiple of 16 and of
+ * every pool's block_size; others return PKV_ERR_UNSUPPORTED or
+ * PKV_ERR_INVALID_ARG before any launch.  workspace: at least
+ * pkv_decode_pools_workspace_size() bytes, 256-byte aligned. */
+int pkv_append_and_decode_pools(const pkv_pool_t* pools, int32_t n_pools, const void* k_new,
+                                const void* v_new, const int32_t* slot_mapping, const void* q,
+                                const int32_t* seq_lens, int32_t num_q_heads, int32_t num_kv_heads,
+                                int32_t head_dim, float scale, int32_t dtype, int32_t partition_tokens,
+                                void* workspace, size_t workspace_bytes, float* out, void* stream);
+
 /* e4m3 form of pkv_append_and_decode: pkv_kv_append_fp8(k_new, v_new,
  * src_dtype, slot_mapping, n_tokens, ..., k_scale, v_scale) followed by
  * pkv_paged_attention_decode_fp8(q, ...), in one call with the same
@@ -438,6 +497,22 @@ int pkv_append_and_decode_fp8(const void* k_new, const void* v_new, int32_t src_
  * PKV_ERR_DEVICE_TIMEOUT a kernel recorded since the last clear.  clear != 0
  * resets it to PKV_OK.  Returns PKV_ERR_CUDA if the synchronisation failed. */
 int pkv_device_status(void* stream, int32_t* status, int32_t clear);
+
+/* Test support for the decode kernels' bounded waits (no counterpart in the
+ * pages; failure detection).  Every wait of a decode consumer for a chunk of
+ * K/V gives up after a limit, records PKV_ERR_DEVICE_TIMEOUT in the status
+ * word and lets the CTA finish, so a stalled copy costs an error code instead
+ * of a hung GPU.  This call makes that path run on demand: for the decode
+ * launches that follow (pkv_paged_attention_decode, _fp8, _static and the
+ * append-and-decode forms), the producer of CTA `cta` skips the copies of
+ * that CTA's first work unit, so their consumers wait for chunks that never
+ * arrive; `consumer_wait_ns` (0 = the normal 1 s) is how long a consumer
+ * waits for a chunk before it gives up.  The producer still waits, with the
+ * normal limit, for every copy it did issue before its CTA exits.  cta < 0
+ * restores normal operation (the default).  Outputs of a stalled call are
+ * unspecified; the pools are not written by decode.  Process-wide setting,
+ * read at each launch; always returns PKV_OK. */
+int pkv_debug_stall_decode(int32_t cta, uint64_t consumer_wait_ns);
 
 #ifdef __cplusplus
 }

@@ -37,6 +37,15 @@ class pkv_stats_t(ctypes.Structure):
         "logical_tokens", "waste_tokens", "cached_blocks", "cache_queries", "cache_hits")]
 
 
+class pkv_pool_t(ctypes.Structure):
+    """One pool of a batch spread over several pools (pkv_append_and_decode_pools)."""
+    _fields_ = [("k_pool", ctypes.c_void_p), ("v_pool", ctypes.c_void_p), ("block_tables", ctypes.c_void_p),
+                ("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
+                ("max_blocks_per_seq", ctypes.c_int32), ("num_seqs", ctypes.c_int32)]
+
+
+_ppool = ctypes.POINTER(pkv_pool_t)
+
 SIGNATURES = {
     "pkv_last_error_string": (ctypes.c_char_p, []),
     "pkv_version": (ctypes.c_char_p, []),
@@ -56,6 +65,7 @@ SIGNATURES = {
     "pkv_paged_attention_decode": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                                                   _i32, _f32, _i32, _i32, _vp, _sz, _vp, _vp]),
     "pkv_device_status": (ctypes.c_int, [_vp, _pi32, _i32]),
+    "pkv_debug_stall_decode": (ctypes.c_int, [_i32, ctypes.c_uint64]),
     "pkv_paged_attention_decode_static": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                                                          _i32, _i32, _f32, _i32, _i32, _vp, _vp]),
     "pkv_static_workspace_bytes": (ctypes.c_size_t, []),
@@ -71,7 +81,11 @@ SIGNATURES = {
     "pkv_decode_step_host": (ctypes.c_int, [_vp, _pi64, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32,
                                             _i32, _f32, _f32, _i32, _vp, _sz, _vp]),
     "pkv_paged_attention_prefill": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
-                                                   _i32, _i32, _i32, _f32, _i32, _vp, _vp]),
+                                                   _i32, _i32, _i32, _f32, _i32, _vp, _sz, _vp, _vp]),
+    "pkv_prefill_workspace_size": (ctypes.c_int, [_i32, _i32, _i32, _i32, _i32, _i32, ctypes.POINTER(_sz)]),
+    "pkv_decode_pools_workspace_size": (ctypes.c_int, [_ppool, _i32, _i32, _i32, _i32, _i32, ctypes.POINTER(_sz)]),
+    "pkv_append_and_decode_pools": (ctypes.c_int, [_ppool, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _f32, _i32,
+                                                   _i32, _vp, _sz, _vp, _vp]),
 }
 
 

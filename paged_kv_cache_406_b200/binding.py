@@ -161,13 +161,29 @@ def pkv_append_and_decode(k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping
     return out
 
 
+def pkv_prefill_workspace_size(num_seqs: int, num_kv_heads: int, head_dim: int, max_blocks_per_seq: int,
+                               block_size: int, dtype: torch.dtype) -> int:
+    """Bytes of the prefill workspace (the f16 copy of V for bf16 pools; 0
+    for f16 pools)."""
+    out = ctypes.c_size_t(0)
+    code = N.PKV_BF16 if dtype == torch.bfloat16 else N.PKV_F16
+    check(lib().pkv_prefill_workspace_size(num_seqs, num_kv_heads, head_dim, max_blocks_per_seq, block_size, code,
+                                           ctypes.byref(out)))
+    return out.value
+
+
 def pkv_paged_attention_prefill(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
                                 block_tables: torch.Tensor, seq_lens: torch.Tensor, q_start: torch.Tensor,
-                                max_q_len: int, scale: float, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                                max_q_len: int, scale: float, out: Optional[torch.Tensor] = None,
+                                workspace: Optional[torch.Tensor] = None, stage_v: bool = True) -> torch.Tensor:
     """Causal paged prefill attention; returns ``out`` (float32
     ``[num_q_tokens, num_q_heads, head_dim]``).  Sequence ``b`` owns q rows
     ``q_start[b] .. q_start[b+1]-1`` (int32 ``[num_seqs + 1]`` on the device);
-    ``max_q_len`` bounds every chunk length."""
+    ``max_q_len`` bounds every chunk length.  For bf16 pools with
+    ``stage_v`` the call first copies V into ``workspace`` as f16 (a uint8
+    device tensor of :func:`pkv_prefill_workspace_size` bytes, allocated here
+    if None) so that P·V runs as one f16 pass; ``stage_v=False`` keeps the
+    two bf16 passes (P hi and lo) over the pool's own V."""
     nb, hkv, bs, d = _pool_dims(_cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"))
     _cuda(q, "q", k_pool.dtype)
     if q.dim() != 3 or q.shape[2] != d:
@@ -186,10 +202,19 @@ def pkv_paged_attention_prefill(q: torch.Tensor, k_pool: torch.Tensor, v_pool: t
         _cuda(out, "out", torch.float32)
         if tuple(out.shape) != (T, hq, d):
             raise ValueError("out has the wrong shape")
+    ws_ptr, ws_bytes = None, 0
+    if stage_v and k_pool.dtype == torch.bfloat16:
+        need = pkv_prefill_workspace_size(B, hkv, d, maxb, bs, k_pool.dtype)
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        _cuda(workspace, "workspace", torch.uint8)
+        if workspace.numel() < need:
+            raise ValueError(f"workspace has {workspace.numel()} bytes, {need} needed")
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
     check(lib().pkv_paged_attention_prefill(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
                                             block_tables.data_ptr(), seq_lens.data_ptr(), q_start.data_ptr(), B, T,
                                             int(max_q_len), hq, hkv, d, nb, maxb, bs, float(scale),
-                                            _dtype_code(k_pool), out.data_ptr(), _stream()))
+                                            _dtype_code(k_pool), ws_ptr, ws_bytes, out.data_ptr(), _stream()))
     return out
 
 
@@ -296,11 +321,81 @@ def pkv_append_and_decode_fp8(k_new: torch.Tensor, v_new: torch.Tensor, slot_map
     return out
 
 
+def _pool_array(pools):
+    """ctypes array of pkv_pool_t from (k_pool, v_pool, block_tables, num_seqs) tuples."""
+    arr = (N.pkv_pool_t * len(pools))()
+    for c, (k_pool, v_pool, tables, n) in enumerate(pools):
+        nb, _, bs, _ = _pool_dims(_cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"))
+        _cuda(tables, "block_tables", torch.int32)
+        if tables.dim() != 2 or tables.shape[0] < n:
+            raise ValueError("each pool's block_tables must be [num_seqs, max_blocks_per_seq]")
+        arr[c] = N.pkv_pool_t(k_pool.data_ptr(), v_pool.data_ptr(), tables.data_ptr(), nb, bs, tables.shape[1], int(n))
+    return arr
+
+
+def pkv_decode_pools_workspace_size(pools, num_q_heads: int, partition_tokens: int = 0) -> int:
+    """Workspace bytes of :func:`pkv_append_and_decode_pools` for ``pools``."""
+    arr = _pool_array(pools)
+    _, hkv, _, d = pools[0][0].shape
+    out = ctypes.c_size_t(0)
+    check(lib().pkv_decode_pools_workspace_size(arr, len(pools), num_q_heads, hkv, d, partition_tokens,
+                                                ctypes.byref(out)))
+    return out.value
+
+
+def pkv_append_and_decode_pools(pools, k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: torch.Tensor,
+                                q: torch.Tensor, seq_lens: torch.Tensor, scale: float,
+                                out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                                partition_tokens: int = 0) -> torch.Tensor:
+    """One decode step (append + attention) over a batch spread across
+    pools of different block sizes.  ``pools``: up to 3 tuples
+    ``(k_pool, v_pool, block_tables, num_seqs)``; the rows of ``k_new``,
+    ``v_new``, ``slot_mapping`` (pool-local slots), ``q`` and ``seq_lens``
+    follow the pools' sequences in pool order."""
+    arr = _pool_array(pools)
+    n = sum(int(x[3]) for x in pools)
+    _, hkv, _, d = pools[0][0].shape
+    _cuda(q, "q", pools[0][0].dtype)
+    if q.dim() != 3 or q.shape[0] != n or q.shape[2] != d:
+        raise ValueError(f"q must be [{n}, num_q_heads, {d}]")
+    hq = q.shape[1]
+    for t, name in ((k_new, "k_new"), (v_new, "v_new")):
+        _cuda(t, name, pools[0][0].dtype)
+        if tuple(t.shape) != (n, hkv, d):
+            raise ValueError(f"{name} must be [{n}, {hkv}, {d}]")
+    _cuda(slot_mapping, "slot_mapping", torch.int32)
+    _cuda(seq_lens, "seq_lens", torch.int32)
+    if slot_mapping.numel() != n or seq_lens.numel() != n:
+        raise ValueError(f"slot_mapping and seq_lens must have {n} entries")
+    need = pkv_decode_pools_workspace_size(pools, hq, partition_tokens)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _cuda(workspace, "workspace", torch.uint8)
+    if out is None:
+        out = torch.empty((n, hq, d), dtype=torch.float32, device=q.device)
+    _cuda(out, "out", torch.float32)
+    if tuple(out.shape) != (n, hq, d):
+        raise ValueError("out has the wrong shape")
+    check(lib().pkv_append_and_decode_pools(arr, len(pools), k_new.data_ptr(), v_new.data_ptr(),
+                                            slot_mapping.data_ptr(), q.data_ptr(), seq_lens.data_ptr(), hq, hkv, d,
+                                            float(scale), _dtype_code(pools[0][0]), partition_tokens,
+                                            workspace.data_ptr(), workspace.numel(), out.data_ptr(), _stream()))
+    return out
+
+
 def pkv_device_status(clear: bool = True) -> int:
     """Synchronise the current stream and return the device status word."""
     st = ctypes.c_int32(0)
     check(lib().pkv_device_status(_stream(), ctypes.byref(st), 1 if clear else 0))
     return st.value
+
+
+def pkv_debug_stall_decode(cta: int = -1, consumer_wait_ns: int = 0) -> None:
+    """Test support for the bounded waits: the decode launches that follow
+    leave CTA ``cta``'s first work unit without copies, and consumers give up
+    a wait after ``consumer_wait_ns`` (0: the normal limit); ``cta < 0``
+    restores normal operation."""
+    check(lib().pkv_debug_stall_decode(int(cta), int(consumer_wait_ns)))
 
 
 # ----------------------------------------------------------------------------
@@ -399,5 +494,7 @@ class Allocator:
 
 __all__ = ["Allocator", "PagedKVError", "pkv_kv_append", "pkv_copy_blocks", "pkv_decode_workspace_size",
            "pkv_paged_attention_decode", "pkv_paged_attention_decode_static", "pkv_device_status",
+           "pkv_debug_stall_decode", "pkv_paged_attention_prefill", "pkv_prefill_workspace_size",
+           "pkv_append_and_decode_pools", "pkv_decode_pools_workspace_size",
            "pkv_kv_append_fp8", "pkv_paged_attention_decode_fp8", "pkv_append_and_decode",
            "pkv_append_and_decode_fp8"]

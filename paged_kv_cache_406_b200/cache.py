@@ -179,6 +179,17 @@ class PagedKVCache:
             int(partition_tokens), ws.data_ptr(), ws.numel(), torch.cuda.current_stream(self.device).cuda_stream))
         return out_host if out_host is not None else out
 
+    def wait_copies(self) -> None:
+        """Makes the current stream wait for the copies that
+        :meth:`decode_step_host` issued on this cache's copy streams (with
+        ``overlap``), so that work recorded next on the current stream - a
+        timing event, a read of ``out_host`` after synchronising it - comes
+        after the last result has reached the host."""
+        cur = torch.cuda.current_stream(self.device)
+        for st in (getattr(self, "_h2d_stream", None), getattr(self, "_d2h_stream", None)):
+            if st is not None:
+                cur.wait_stream(st)
+
     def _ensure_step(self, n: int, hq: int) -> None:
         key = (n, hq)
         if getattr(self, "_step_key", None) == key:
@@ -230,7 +241,8 @@ class AdaptivePagedKVCache:
     """Adaptive block size (optimisation-overview page §3.3): one paged pool
     per block-size class (32, 16, 8 tokens); a sequence joins the class of
     its length at admission and keeps it for life (the page leaves migration
-    open; none is done).  A decode step runs the paged path once per class.
+    open; none is done).  A decode step serves every class in one call
+    (pkv_append_and_decode_pools), or one call per class.
 
     ``seq_ids`` passed to :meth:`decode_step` must be grouped by class in the
     order 32, 16, 8 (:meth:`order` returns live ids that way), so that each
@@ -265,18 +277,65 @@ class AdaptivePagedKVCache:
         return [s for bs in self.CLASSES for s in self.cls if self.cls[s] == bs]
 
     def decode_step(self, seq_ids: Sequence[int], q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
-                    scale: float, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                    scale: float, out: Optional[torch.Tensor] = None, one_call: bool = True) -> torch.Tensor:
+        """Append one token per sequence and attend, over every class.  With
+        ``one_call`` (16-bit pools, head_dim 128, 2 to 8 query heads per KV
+        head) the classes share one pkv_append_and_decode_pools call (one
+        append + plan, decode and merge launch for the whole batch); otherwise
+        each class runs its own decode step."""
         n = len(seq_ids)
         ranks = [self.CLASSES.index(self.cls[s]) for s in seq_ids]
         if any(a > b for a, b in zip(ranks, ranks[1:])):
             raise ValueError("seq_ids must be grouped by block-size class (32, 16, 8)")
+        dev = next(iter(self.caches.values())).device
         if out is None:
-            out = torch.empty((n, q.shape[1], q.shape[2]), dtype=torch.float32, device=next(iter(self.caches.values())).device)
-        a = 0
-        for bs in self.CLASSES:
-            m = sum(1 for r in ranks if self.CLASSES[r] == bs)
-            if m:
-                self.caches[bs].decode_step(seq_ids[a:a + m], q[a:a + m], k_new[a:a + m], v_new[a:a + m], scale,
-                                            out=out[a:a + m])
+            out = torch.empty((n, q.shape[1], q.shape[2]), dtype=torch.float32, device=dev)
+        counts = [sum(1 for r in ranks if self.CLASSES[r] == bs) for bs in self.CLASSES]
+        any_cache = next(iter(self.caches.values()))
+        g = q.shape[1] // any_cache.num_kv_heads
+        if not (one_call and any_cache.dtype in (torch.bfloat16, torch.float16) and any_cache.head_dim == 128
+                and g in (2, 4, 8)):
+            a = 0
+            for bs, m in zip(self.CLASSES, counts):
+                if m:
+                    self.caches[bs].decode_step(seq_ids[a:a + m], q[a:a + m], k_new[a:a + m], v_new[a:a + m],
+                                                scale, out=out[a:a + m])
+                a += m
+            return out
+        # host: slots, copy-on-write and tables per class; the step's slots and
+        # lengths gathered into one pinned buffer and copied up once
+        if getattr(self, "_sl_cap", 0) < n:
+            self._sl_host = torch.empty(2 * n, dtype=torch.int32, pin_memory=True)
+            self._sl_dev = torch.empty(2 * n, dtype=torch.int32, device=dev)
+            self._sl_cap = n
+            self._sl_done = None
+        if self._sl_done is not None:
+            self._sl_done.synchronize()
+        sl = self._sl_host.numpy()
+        pools, a = [], 0
+        for bs, m in zip(self.CLASSES, counts):
+            if bs not in self.caches:
+                continue
+            c = self.caches[bs]
+            if not m:  # a class with no sequence this step: a pool of none
+                pools.append((c.k_pool, c.v_pool, torch.empty((0, c.max_blocks), dtype=torch.int32, device=dev), 0))
+                continue
+            ncow, (slots, lens, _, _) = c.prepare_step(seq_ids[a:a + m])
+            sl[a:a + m] = slots[:m]
+            sl[n + a:n + a + m] = lens[:m]
+            _, _, cow, tables = c.upload_step(m)
+            if ncow:
+                B.pkv_copy_blocks(c.k_pool, c.v_pool, cow[:2 * ncow].view(ncow, 2))
+            pools.append((c.k_pool, c.v_pool, tables, m))
             a += m
-        return out
+        self._sl_dev[:2 * n].copy_(self._sl_host[:2 * n], non_blocking=True)
+        ev = torch.cuda.Event()
+        ev.record()
+        self._sl_done = ev
+        q, k_new, v_new = (t.to(dev, non_blocking=True) for t in (q, k_new, v_new))
+        ws = getattr(self, "_pool_ws", None)
+        need = B.pkv_decode_pools_workspace_size(pools, q.shape[1])
+        if ws is None or ws.numel() < need:
+            ws = self._pool_ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        return B.pkv_append_and_decode_pools(pools, k_new, v_new, self._sl_dev[:n], q, self._sl_dev[n:2 * n], scale,
+                                             out=out, workspace=ws)

@@ -16,31 +16,50 @@ namespace pkv {
 // KV append: one thread per 16-byte chunk of one (token, kv head) row, K and V.
 // vLLM paging page §3 phase 1: the new token is written into its slot.
 // ---------------------------------------------------------------------------
+// Token i's row goes into pool c for tok0[c] <= i < tok0[c + 1] (one pool
+// unless a step spans pools of several block sizes); its slot is pool-local.
 struct AppendArgs {
   const void* k_new;
   const void* v_new;
   const int32_t* slots;
   int64_t n_units;  // 16-byte chunks (copy) or 8-element groups (e4m3) over all (token, head) rows
-  void* k_pool;
-  void* v_pool;
-  int32_t num_blocks, num_kv_heads, row_units, block_size;
+  void* k_pool[kMaxPools];
+  void* v_pool[kMaxPools];
+  int32_t num_blocks[kMaxPools], block_size[kMaxPools], tok0[kMaxPools];
+  int32_t n_pools, num_kv_heads, row_units;
   float k_inv, v_inv;  // e4m3 only: 1 / scale
 };
+
+// The pool of token `tok` and its destination fields.
+struct AppendDst {
+  unsigned char* k_pool;
+  unsigned char* v_pool;
+  int32_t num_blocks, block_size;
+};
+
+__device__ __forceinline__ AppendDst append_dst(const AppendArgs& a, int64_t tok) {
+  int c = 0;
+  if (a.n_pools > 1) c = (tok >= a.tok0[1] ? 1 : 0) + (a.n_pools > 2 && tok >= a.tok0[2] ? 1 : 0);
+  return AppendDst{static_cast<unsigned char*>(pick3(a.k_pool, c)), static_cast<unsigned char*>(pick3(a.v_pool, c)),
+                   pick3(a.num_blocks, c), pick3(a.block_size, c)};
+}
 
 __device__ __forceinline__ void append_chunk(const AppendArgs& a, int64_t i) {
   const uint4* __restrict__ k_new = static_cast<const uint4*>(a.k_new);
   const uint4* __restrict__ v_new = static_cast<const uint4*>(a.v_new);
-  uint4* __restrict__ k_pool = static_cast<uint4*>(a.k_pool);
-  uint4* __restrict__ v_pool = static_cast<uint4*>(a.v_pool);
-  const int32_t row_chunks = a.row_units, num_kv_heads = a.num_kv_heads, block_size = a.block_size;
+  const int32_t row_chunks = a.row_units, num_kv_heads = a.num_kv_heads;
   const int32_t chunk = static_cast<int32_t>(i % row_chunks);
   const int64_t row = i / row_chunks;  // token * num_kv_heads + head
   const int32_t h = static_cast<int32_t>(row % num_kv_heads);
   const int64_t tok = row / num_kv_heads;
   const int32_t slot = a.slots[tok];
   if (slot < 0) return;  // padding token
+  const AppendDst t = append_dst(a, tok);
+  uint4* __restrict__ k_pool = reinterpret_cast<uint4*>(t.k_pool);
+  uint4* __restrict__ v_pool = reinterpret_cast<uint4*>(t.v_pool);
+  const int32_t block_size = t.block_size;
   const int32_t blk = slot / block_size, off = slot - blk * block_size;
-  if (blk >= a.num_blocks) {
+  if (blk >= t.num_blocks) {
     if (chunk == 0 && h == 0) record_error(PKV_ERR_BAD_BLOCK);
     return;
   }
@@ -110,9 +129,7 @@ template <typename Src>
 __device__ __forceinline__ void append_fp8_group(const AppendArgs& a, int64_t i) {
   const Src* __restrict__ k_new = static_cast<const Src*>(a.k_new);
   const Src* __restrict__ v_new = static_cast<const Src*>(a.v_new);
-  uint8_t* __restrict__ k_pool = static_cast<uint8_t*>(a.k_pool);
-  uint8_t* __restrict__ v_pool = static_cast<uint8_t*>(a.v_pool);
-  const int32_t per_row = a.row_units, num_kv_heads = a.num_kv_heads, block_size = a.block_size;
+  const int32_t per_row = a.row_units, num_kv_heads = a.num_kv_heads;
   const int32_t head_dim = per_row * 8;
   const int32_t grp = static_cast<int32_t>(i % per_row);
   const int64_t row = i / per_row;  // token * num_kv_heads + head
@@ -120,8 +137,12 @@ __device__ __forceinline__ void append_fp8_group(const AppendArgs& a, int64_t i)
   const int64_t tok = row / num_kv_heads;
   const int32_t slot = a.slots[tok];
   if (slot < 0) return;
+  const AppendDst t = append_dst(a, tok);
+  uint8_t* __restrict__ k_pool = t.k_pool;
+  uint8_t* __restrict__ v_pool = t.v_pool;
+  const int32_t block_size = t.block_size;
   const int32_t blk = slot / block_size, off = slot - blk * block_size;
-  if (blk >= a.num_blocks) {
+  if (blk >= t.num_blocks) {
     if (grp == 0 && h == 0) record_error(PKV_ERR_BAD_BLOCK);
     return;
   }
@@ -157,14 +178,12 @@ __global__ void __launch_bounds__(256) kv_append_fp8_kernel(const AppendArgs a) 
 // Src = void: 16-byte row copies; otherwise the source type quantised to e4m3.
 // ---------------------------------------------------------------------------
 template <typename Src>
-__global__ void __launch_bounds__(256) append_plan_kernel(const AppendArgs a, const int32_t* __restrict__ seq_lens,
-                                                          int32_t num_seqs, int32_t max_tokens, int32_t part_tokens,
-                                                          int32_t block_size, int4* __restrict__ items,
-                                                          int32_t* __restrict__ n_items) {
+__global__ void __launch_bounds__(256) append_plan_kernel(const AppendArgs a, const PlanArgs pa,
+                                                          int4* __restrict__ items, int32_t* __restrict__ n_items) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (blockIdx.x == 0) {
     extern __shared__ int32_t hist[];
-    plan_body(seq_lens, num_seqs, max_tokens, part_tokens, block_size, items, n_items, hist);
+    plan_body(pa, items, n_items, hist);
     return;
   }
   const int64_t i = static_cast<int64_t>(blockIdx.x - 1) * blockDim.x + threadIdx.x;

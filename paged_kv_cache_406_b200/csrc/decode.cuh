@@ -39,12 +39,23 @@ constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr unsigned kFull = 0xffffffffu;
 
+// A batch may span up to kMaxPools pools of different block sizes (one pool
+// per block-size class): sequences seq0 .. of pool c (up to the next pool's
+// seq0) are rows (b - seq0) of that pool's block table.
+constexpr int kMaxPools = 3;
+
+struct PoolView {
+  const void* k;          // K and V pools [num_blocks][num_kv_heads][block_size][head_dim]
+  const void* v;
+  const int32_t* tables;  // [sequences of the pool][max_blocks]
+  int32_t num_blocks, max_blocks, block_size, seq0;
+};
+
 struct DecodeParams {
   const void* q;
-  const void* k_pool;
-  const void* v_pool;
-  const int32_t* block_tables;
-  int32_t num_q_heads, num_kv_heads, num_blocks, max_blocks, block_size, partition_tokens, max_parts;
+  PoolView pool[kMaxPools];
+  int32_t n_pools;
+  int32_t num_q_heads, num_kv_heads, partition_tokens, max_parts;
   int32_t n_stages;
   float scale_log2;
   float v_scale;  // multiplies the output (e4m3 V pools; 1 otherwise)
@@ -54,29 +65,66 @@ struct DecodeParams {
   float* part_l;
   float* part_o;
   float* out;
+  // Test support for the bounded waits (pkv_debug_stall_decode): the
+  // producer of CTA `stall_cta` skips the copies of that CTA's first work
+  // unit (its consumers' waits then run out), and consumers give up a wait
+  // for a chunk after `consumer_wait_ns`.  stall_cta < 0 in normal calls.
+  int32_t stall_cta;
+  uint64_t consumer_wait_ns;
 };
 
+// Pool of sequence b (0 for single-pool batches).
+__device__ __forceinline__ int pool_of(const PoolView* pool, int n_pools, int b) {
+  return n_pools == 1 ? 0 : (b >= pool[1].seq0 ? 1 : 0) + (n_pools > 2 && b >= pool[2].seq0 ? 1 : 0);
+}
+
+// Element c of a small array held in kernel parameters, by selects (a
+// dynamic index into the parameter space would copy the array to local
+// memory).
+template <typename V>
+__device__ __forceinline__ V pick3(const V (&a)[kMaxPools], int c) {
+  return c == 0 ? a[0] : (c == 1 ? a[1] : a[2]);
+}
+
 // ---------------------------------------------------------------------------
-// plan: seq_lens -> work list, partitions sorted by block count, largest first
+// plan: seq_lens -> work list, partitions sorted by size, largest first
 // ---------------------------------------------------------------------------
-// One CTA builds the list; `hist` is 2 * (part_tokens / block_size + 1) ints of
-// shared memory.
-__device__ __forceinline__ void plan_body(const int32_t* __restrict__ seq_lens, int32_t num_seqs, int32_t max_tokens,
-                                          int32_t part_tokens, int32_t block_size, int4* __restrict__ items,
-                                          int32_t* __restrict__ n_items, int32_t* hist) {
-  const int kmax = part_tokens / block_size;
+struct PlanArgs {
+  const int32_t* seq_lens;
+  int32_t num_seqs, part_tokens;
+  int32_t bin_tokens;  // size classes of the sort: part_tokens / bin_tokens + 1 bins
+  int32_t n_pools;
+  int32_t seq0[kMaxPools];  // first sequence of each pool
+  int32_t cap[kMaxPools];   // tokens a sequence of the pool can hold (max_blocks * block_size)
+};
+
+// One CTA builds the list; `hist` is 2 * (part_tokens / bin_tokens + 1) ints
+// of shared memory.  A length outside [0, its pool's capacity] is recorded
+// and clamped.
+__device__ __forceinline__ int plan_len(const PlanArgs& a, int b, bool record) {
+  int c = 0;
+  if (a.n_pools > 1) c = (b >= a.seq0[1] ? 1 : 0) + (a.n_pools > 2 && b >= a.seq0[2] ? 1 : 0);
+  const int cap = pick3(a.cap, c);
+  int L = a.seq_lens[b];
+  if (L < 0 || L > cap) {
+    if (record) record_error(PKV_ERR_BAD_BLOCK);
+    L = L < 0 ? 0 : cap;
+  }
+  return L;
+}
+
+__device__ __forceinline__ void plan_body(const PlanArgs& a, int4* __restrict__ items, int32_t* __restrict__ n_items,
+                                          int32_t* hist) {
+  const int part_tokens = a.part_tokens, bin = a.bin_tokens;
+  const int kmax = part_tokens / bin;
   int32_t* cursor = hist + kmax + 1;
   for (int i = threadIdx.x; i <= kmax; i += blockDim.x) hist[i] = 0;
   __syncthreads();
-  for (int b = threadIdx.x; b < num_seqs; b += blockDim.x) {
-    int L = seq_lens[b];
-    if (L < 0 || L > max_tokens) {
-      record_error(PKV_ERR_BAD_BLOCK);
-      L = L < 0 ? 0 : max_tokens;
-    }
+  for (int b = threadIdx.x; b < a.num_seqs; b += blockDim.x) {
+    const int L = plan_len(a, b, true);
     const int nfull = L / part_tokens, rem = L % part_tokens;
     if (nfull) atomicAdd(&hist[kmax], nfull);
-    if (rem) atomicAdd(&hist[(rem + block_size - 1) / block_size], 1);
+    if (rem) atomicAdd(&hist[(rem + bin - 1) / bin], 1);
     if (L == 0) atomicAdd(&hist[0], 1);
   }
   __syncthreads();
@@ -89,9 +137,8 @@ __device__ __forceinline__ void plan_body(const int32_t* __restrict__ seq_lens, 
     *n_items = run;
   }
   __syncthreads();
-  for (int b = threadIdx.x; b < num_seqs; b += blockDim.x) {
-    int L = seq_lens[b];
-    L = L < 0 ? 0 : (L > max_tokens ? max_tokens : L);
+  for (int b = threadIdx.x; b < a.num_seqs; b += blockDim.x) {
+    const int L = plan_len(a, b, false);
     const int nfull = L / part_tokens, rem = L % part_tokens;
     if (nfull) {
       int pos = atomicAdd(&cursor[kmax], nfull);
@@ -99,7 +146,7 @@ __device__ __forceinline__ void plan_body(const int32_t* __restrict__ seq_lens, 
         items[pos + p] = make_int4(b, p, nfull + (rem ? 1 : 0), (p + 1) * part_tokens);
     }
     if (rem) {
-      int pos = atomicAdd(&cursor[(rem + block_size - 1) / block_size], 1);
+      int pos = atomicAdd(&cursor[(rem + bin - 1) / bin], 1);
       items[pos] = make_int4(b, nfull, nfull + 1, L);
     }
     if (L == 0) {
@@ -109,14 +156,13 @@ __device__ __forceinline__ void plan_body(const int32_t* __restrict__ seq_lens, 
   }
 }
 
-__global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ seq_lens, int32_t num_seqs,
-                                                    int32_t max_tokens, int32_t part_tokens, int32_t block_size,
-                                                    int4* __restrict__ items, int32_t* __restrict__ n_items) {
+__global__ void __launch_bounds__(1024) plan_kernel(const PlanArgs a, int4* __restrict__ items,
+                                                    int32_t* __restrict__ n_items) {
   // the decode grid may be scheduled now; it waits for this grid's results
   // (griddepcontrol.wait) before reading them
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ int32_t hist[];  // [kmax + 1] counts, then [kmax + 1] cursors
-  plan_body(seq_lens, num_seqs, max_tokens, part_tokens, block_size, items, n_items, hist);
+  plan_body(a, items, n_items, hist);
 }
 
 // ---------------------------------------------------------------------------
@@ -201,7 +247,7 @@ __device__ __forceinline__ float pick(const float (&v)[G], int r8) {
 }
 
 struct WorkUnit {
-  int b, part, nparts, t0, t1, g, nblk;
+  int b, part, nparts, t0, t1, g, nblk, c;  // c: the pool of sequence b
 };
 
 // The work unit this CTA takes in round r of the persistent loop.  Rounds go
@@ -214,6 +260,9 @@ __device__ __forceinline__ int unit_index(int r) {
   return r * static_cast<int>(gridDim.x) + c;
 }
 
+// kMulti: the batch may span several pools (else pool 0 only, known at
+// compile time).
+template <bool kMulti = false>
 __device__ __forceinline__ WorkUnit load_unit(const DecodeParams& p, int w) {
   WorkUnit u;
   const int idx = w / p.num_kv_heads;
@@ -224,7 +273,9 @@ __device__ __forceinline__ WorkUnit load_unit(const DecodeParams& p, int w) {
   u.nparts = it.z;
   u.t0 = it.y * p.partition_tokens;
   u.t1 = it.w;
-  u.nblk = (u.t1 - u.t0 + p.block_size - 1) / p.block_size;
+  u.c = kMulti ? pool_of(p.pool, p.n_pools, u.b) : 0;
+  const int bs = kMulti ? pick3(p.pool, u.c).block_size : p.pool[0].block_size;
+  u.nblk = (u.t1 - u.t0 + bs - 1) / bs;
   return u;
 }
 
@@ -288,7 +339,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
   constexpr int kMF = DecodeSmem<T, D, G>::kMergeFloats;
   static_assert(kChunksPerLane >= 1, "head_dim too small");
 
-  const int BS = p.block_size;
+  const int BS = p.pool[0].block_size;  // one pool: the multi-pool batches take the tensor-core kernel
   const int NS = p.n_stages;
   const uint32_t tile_bytes = BS * D * sizeof(T);
   const uint32_t stage_bytes = 2 * tile_bytes;
@@ -321,16 +372,18 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
     // shared memory; lane 0 alone issues the window's blocks (no warp-wide
     // synchronisation on the per-block path).
     const uint64_t policy = l2_evict_first_policy();
-    const unsigned char* kbase = static_cast<const unsigned char*>(p.k_pool);
-    const unsigned char* vbase = static_cast<const unsigned char*>(p.v_pool);
+    const uint64_t tab_policy = l2_evict_last_policy();
+    const unsigned char* kbase = static_cast<const unsigned char*>(p.pool[0].k);
+    const unsigned char* vbase = static_cast<const unsigned char*>(p.pool[0].v);
     int s = 0;
-    uint32_t ph = 0, issued = 0;
+    uint32_t ph = 0, issued = 0, skipped = 0;  // stage uses so far; the first `skipped` of them issued no copy
     bool ok = true;
     for (int r = 0, w = unit_index(0); w < n_work && ok; w = unit_index(++r)) {
+      const bool stall = r == 0 && p.stall_cta == static_cast<int>(blockIdx.x);
       const WorkUnit u = load_unit(p, w);
-      const int32_t* trow = p.block_tables + static_cast<int64_t>(u.b) * p.max_blocks + u.t0 / BS;
+      const int32_t* trow = p.pool[0].tables + static_cast<int64_t>(u.b) * p.pool[0].max_blocks + u.t0 / BS;
       for (int jb = 0; jb < u.nblk && ok; jb += 32) {
-        tab[lane] = jb + lane < u.nblk ? trow[jb + lane] : 0;
+        tab[lane] = jb + lane < u.nblk ? ld_table(trow + jb + lane, tab_policy) : 0;
         __syncwarp();
         if (lane == 0) {
           const int cnt = min(32, u.nblk - jb);
@@ -342,15 +395,19 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
               break;
             }
             int phys = tab[j];
-            if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_blocks)) {
+            if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.pool[0].num_blocks)) {
               record_error(PKV_ERR_BAD_BLOCK);
               phys = 0;
             }
             const size_t off = (static_cast<size_t>(phys) * p.num_kv_heads + u.g) * tile_bytes;
             const uint32_t bar = smem_addr(full + s);
-            mbar_arrive_expect_tx(bar, stage_bytes);
-            bulk_g2s(ring_s + s * stage_bytes, kbase + off, tile_bytes, bar, policy);
-            bulk_g2s(ring_s + s * stage_bytes + tile_bytes, vbase + off, tile_bytes, bar, policy);
+            if (!stall) {
+              mbar_arrive_expect_tx(bar, stage_bytes);
+              bulk_g2s(ring_s + s * stage_bytes, kbase + off, tile_bytes, bar, policy);
+              bulk_g2s(ring_s + s * stage_bytes + tile_bytes, vbase + off, tile_bytes, bar, policy);
+            } else {
+              ++skipped;  // nothing will land in this stage: its consumer's wait runs out
+            }
             ++issued;
             if (++s == NS) {
               s = 0;
@@ -363,10 +420,12 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
       }
     }
     // Before the CTA exits no copy may still be landing in its shared memory:
-    // wait (bounded) for the last phase issued into every stage.
+    // wait (bounded) for the last phase issued into every stage whose last use
+    // carried a copy.
     if (lane == 0) {
       for (int st = 0; st < NS && st < static_cast<int>(issued); ++st) {
         const uint32_t uses = (issued - st + NS - 1) / NS;
+        if (st + NS * (uses - 1) < skipped) continue;
         const uint64_t t0 = global_timer_ns();
         while (!mbar_try_wait(smem_addr(full + st), (uses - 1) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
         }
@@ -417,7 +476,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
     int s = (c + j0) % NS;
     uint32_t ph = ((c + j0) / NS) & 1;
     for (int j = j0; j < u.nblk && ok; j += kConsumerWarps) {
-      const bool landed = __all_sync(kFull, mbar_wait(smem_addr(full + s), ph, abort_flag));
+      const bool landed = __all_sync(kFull, mbar_wait(smem_addr(full + s), ph, abort_flag, p.consumer_wait_ns));
       if (!landed) {
         if (lane == 0) {
           record_error(PKV_ERR_DEVICE_TIMEOUT);

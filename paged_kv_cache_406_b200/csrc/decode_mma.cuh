@@ -88,10 +88,23 @@ __device__ __forceinline__ uint32_t row_offset(int r, int h, int br_shift, int h
 // warps per SM instead of 8 take its decode call from 77.3 to 74.8 us on the
 // Llama-3-8B-shaped batch (4 CTAs would spill).  The 16-bit kernels keep the
 // compiler's own choice (127 registers, 2 CTAs per SM).
-template <typename T, int D, int G, int kKVBytes = 2>
+// Tensor maps of the K and V pools of a batch (pool c: k[c], v[c]).
+struct PoolMaps {
+  CUtensorMap k[kMaxPools];
+  CUtensorMap v[kMaxPools];
+};
+
+// Block size of a pool as shifts: log2(block_size) and log2(rows per TMA box)
+// (8 rows for 8-token blocks, else 16: a 16-token chunk is one box, two
+// boxes of 8-token blocks, or half a 32-token block).
+__device__ __forceinline__ int bs_shift_of(int bs) { return bs == 8 ? 3 : (bs == 16 ? 4 : 5); }
+__device__ __forceinline__ int br_shift_of(int bs) { return bs == 8 ? 3 : 4; }
+
+// kMulti: the batch spans up to kMaxPools pools of different block sizes
+// (each work unit reads its sequence's pool); otherwise pool 0 only.
+template <typename T, int D, int G, int kKVBytes = 2, bool kMulti = false>
 __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0) decode_mma_kernel(const DecodeParams p,
-                                                                    const __grid_constant__ CUtensorMap tmap_k,
-                                                                    const __grid_constant__ CUtensorMap tmap_v) {
+                                                                    const __grid_constant__ PoolMaps maps) {
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
   static_assert(kKVBytes == 2 || (kKVBytes == 1 && D == 128), "e4m3 pools need head_dim 128");
   using L = MmaLayout<D, kKVBytes>;
@@ -102,10 +115,7 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0) decode_mma
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
-  const int BS = p.block_size;
   const int NS = p.n_stages;
-  const int bs_shift = BS == 8 ? 3 : (BS == 16 ? 4 : 5);
-  const int br_shift = BS == 8 ? 3 : 4;  // rows per TMA box: 8 or 16
   float* merge = reinterpret_cast<float*>(smem + MmaSmem<T, D, G, kKVBytes>::ring_bytes(NS));
   uint64_t* full = reinterpret_cast<uint64_t*>(merge + 2 * kConsumerWarps * kMF);
   uint64_t* empty = full + NS;
@@ -136,24 +146,30 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0) decode_mma
     // synchronisation.
     const int pr = warp - kConsumerWarps;
     int32_t* mytab = tab + 32 * pr;
-    if (lane == 0) {
-      prefetch_tensormap(&tmap_k);
-      prefetch_tensormap(&tmap_v);
+    if (lane < (kMulti ? p.n_pools : 1)) {
+      prefetch_tensormap(&maps.k[lane]);
+      prefetch_tensormap(&maps.v[lane]);
     }
     const uint64_t policy = l2_evict_first_policy();
-    const uint32_t box_bytes = (1u << br_shift) * D * kKVBytes;        // one K (or V) box
-    const uint32_t blk_off = L::kRingHalves * (1u << br_shift) * 128;  // second box of a chunk (block_size 8)
+    const uint64_t tab_policy = l2_evict_last_policy();
     int s = pr;           // this producer's stages: pr, pr + 2, ...
-    uint32_t ph = 0, issued = 0;
+    uint32_t ph = 0, issued = 0, skipped = 0;  // stage uses so far; the first `skipped` of them issued no copy
     uint32_t cg = 0;      // CTA-wide chunk index of the unit's first chunk
     bool ok = true;
     for (int r = 0, w = unit_index(0); w < n_work && ok; w = unit_index(++r)) {
-      const WorkUnit u = load_unit(p, w);
-      const int32_t* trow = p.block_tables + static_cast<int64_t>(u.b) * p.max_blocks + (u.t0 >> bs_shift);
+      const bool stall = r == 0 && p.stall_cta == static_cast<int>(blockIdx.x);
+      const WorkUnit u = load_unit<kMulti>(p, w);
+      const PoolView pv = kMulti ? pick3(p.pool, u.c) : p.pool[0];
+      const int BS = pv.block_size, bs_shift = bs_shift_of(BS), br_shift = br_shift_of(BS);
+      const uint32_t box_bytes = (1u << br_shift) * D * kKVBytes;        // one K (or V) box
+      const uint32_t blk_off = L::kRingHalves * (1u << br_shift) * 128;  // second box of a chunk (block_size 8)
+      const CUtensorMap* tmap_k = &maps.k[kMulti ? u.c : 0];
+      const CUtensorMap* tmap_v = &maps.v[kMulti ? u.c : 0];
+      const int32_t* trow = pv.tables + static_cast<int64_t>(u.b - pv.seq0) * pv.max_blocks + (u.t0 >> bs_shift);
       const int nch = (u.t1 - u.t0 + kChunkTokens - 1) / kChunkTokens;
       const int ybase = u.g * BS;
       for (int wb = 0; wb < u.nblk && ok; wb += 32) {
-        mytab[lane] = wb + lane < u.nblk ? trow[wb + lane] : 0;
+        mytab[lane] = wb + lane < u.nblk ? ld_table(trow + wb + lane, tab_policy) : 0;
         __syncwarp();
         if (lane == 0) {
           const int k_begin = (wb << bs_shift) >> 4;
@@ -170,16 +186,17 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0) decode_mma
             const int row0 = BS == 32 ? (k & 1) << 4 : 0;
             const uint32_t bar = smem_addr(full + s);
             const uint32_t kdst = ring_s + s * L::kStageBytes;
-            mbar_arrive_expect_tx(bar, nb_here * 2 * box_bytes);
-            for (int i = 0; i < nb_here; ++i) {
+            if (!stall) mbar_arrive_expect_tx(bar, nb_here * 2 * box_bytes);
+            else ++skipped;  // nothing will land in this stage: its consumer's wait runs out
+            for (int i = 0; i < nb_here && !stall; ++i) {
               int phys = mytab[jb - wb + i];
-              if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_blocks)) {
+              if (static_cast<unsigned>(phys) >= static_cast<unsigned>(pv.num_blocks)) {
                 record_error(PKV_ERR_BAD_BLOCK);
                 phys = 0;
               }
               const int32_t y = phys * p.num_kv_heads * BS + ybase + row0;
-              tma_load_3d(kdst + i * blk_off, &tmap_k, 0, y, 0, bar, policy);
-              tma_load_3d(kdst + L::kRingTileBytes + i * blk_off, &tmap_v, 0, y, 0, bar, policy);
+              tma_load_3d(kdst + i * blk_off, tmap_k, 0, y, 0, bar, policy);
+              tma_load_3d(kdst + L::kRingTileBytes + i * blk_off, tmap_v, 0, y, 0, bar, policy);
             }
             ++issued;
             s += kMmaProducers;
@@ -200,6 +217,7 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0) decode_mma
       const int mine = NS / kMmaProducers;  // stages pr, pr + 2, ...
       for (int j = 0; j < mine && j < static_cast<int>(issued); ++j) {
         const uint32_t uses = (issued - j + mine - 1) / mine;
+        if (j + mine * (uses - 1) < skipped) continue;  // its last use carried no copy
         const int st = pr + kMmaProducers * j;
         const uint64_t t0 = global_timer_ns();
         while (!mbar_try_wait(smem_addr(full + st), (uses - 1) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
@@ -215,14 +233,6 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0) decode_mma
   // ldmatrix row addresses of this lane: K chunk (A operand) and V chunk (A = Vᵀ via .trans)
   const int ra = (lane & 7) + ((lane >> 3) & 1) * 8, ca = lane >> 4;
   const int rv = (lane & 7) + (lane >> 4) * 8, cv = (lane >> 3) & 1;
-  // 16-bit pools: the MMAs read the ring chunk itself, built from boxes of br rows
-  const int tile_shift = br_shift;
-  uint32_t offa[kHalves], offv[kHalves];
-#pragma unroll
-  for (int h = 0; h < kHalves; ++h) {
-    offa[h] = row_offset(ra, h, tile_shift, kHalves);
-    offv[h] = row_offset(rv, h, tile_shift, kHalves);
-  }
   const int xa = ra & 7, xv = rv & 7;
   const int src0 = 4 * (2 * tq) + (gq >> 1), src1 = src0 + 4;  // Pᵀ transpose sources
   const uint32_t sel = (gq & 1) ? 0x7632u : 0x5410u;
@@ -231,8 +241,17 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0) decode_mma
   int iter = 0;
   bool ok = true;
   for (int w = unit_index(0); w < n_work; w = unit_index(++iter)) {
-    const WorkUnit u = load_unit(p, w);
+    const WorkUnit u = load_unit<kMulti>(p, w);
     const int nch = (u.t1 - u.t0 + kChunkTokens - 1) / kChunkTokens;
+    // 16-bit pools: the MMAs read the ring chunk itself, built from boxes of
+    // br rows (the unit's pool decides br)
+    const int tile_shift = br_shift_of(kMulti ? pick3(p.pool, u.c).block_size : p.pool[0].block_size);
+    uint32_t offa[kHalves], offv[kHalves];
+#pragma unroll
+    for (int h = 0; h < kHalves; ++h) {
+      offa[h] = row_offset(ra, h, tile_shift, kHalves);
+      offv[h] = row_offset(rv, h, tile_shift, kHalves);
+    }
 
     // B fragments of Qᵀ: column n = head gq (zero for the padding heads >= G)
     uint32_t qb[kSteps][2];
@@ -261,7 +280,7 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0) decode_mma
     int s = (c + k0) % NS;
     uint32_t ph = ((c + k0) / NS) & 1;
     for (int k = k0; k < nch && ok; k += kConsumerWarps) {
-      const bool landed = __all_sync(kFull, mbar_wait(smem_addr(full + s), ph, abort_flag));
+      const bool landed = __all_sync(kFull, mbar_wait(smem_addr(full + s), ph, abort_flag, p.consumer_wait_ns));
       if (!landed) {
         if (lane == 0) {
           record_error(PKV_ERR_DEVICE_TIMEOUT);

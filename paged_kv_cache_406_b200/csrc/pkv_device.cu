@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include <cuda_fp8.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "append.cuh"
 #include "decode.cuh"
@@ -24,6 +25,15 @@
 namespace {
 
 using pkv::fail;
+
+// An NVTX range around one library call, so that a profiler's timeline shows
+// each step and each entry point by name (a no-op without a tool attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 constexpr int kMaxDevices = 64;
 constexpr int kAutoPartitionTokens = 512;
@@ -125,38 +135,83 @@ struct PendingAppend {
   int src_dtype;
 };
 
+// Test support for the decode kernels' bounded waits (pkv_debug_stall_decode):
+// a CTA whose first work unit gets no copies, and the consumers' wait limit.
+std::atomic<int> g_stall_cta{-1};
+std::atomic<uint64_t> g_consumer_wait_ns{pkv::kWaitLimitNs};
+
+void apply_debug(pkv::DecodeParams& p) {
+  p.stall_cta = g_stall_cta.load(std::memory_order_relaxed);
+  p.consumer_wait_ns = g_consumer_wait_ns.load(std::memory_order_relaxed);
+}
+
+// The one pool of a single-pool batch.
+void set_single_pool(pkv::DecodeParams& p, const void* k_pool, const void* v_pool, const int32_t* block_tables,
+                     int32_t num_blocks, int32_t max_blocks, int32_t block_size) {
+  p.pool[0] = pkv::PoolView{k_pool, v_pool, block_tables, num_blocks, max_blocks, block_size, 0};
+  p.n_pools = 1;
+}
+
+// Append arguments for rows that all go into one pool.
+pkv::AppendArgs single_append(const void* k_new, const void* v_new, const int32_t* slots, int64_t n_units,
+                              void* k_pool, void* v_pool, int32_t num_blocks, int32_t num_kv_heads,
+                              int32_t row_units, int32_t block_size, float k_inv, float v_inv) {
+  pkv::AppendArgs a{};
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.slots = slots;
+  a.n_units = n_units;
+  a.k_pool[0] = k_pool;
+  a.v_pool[0] = v_pool;
+  a.num_blocks[0] = num_blocks;
+  a.block_size[0] = block_size;
+  a.n_pools = 1;
+  a.num_kv_heads = num_kv_heads;
+  a.row_units = row_units;
+  a.k_inv = k_inv;
+  a.v_inv = v_inv;
+  return a;
+}
+
+// Plan arguments of a batch: the sort bins are blocks of a single pool, or
+// 16-token chunks when the pools' block sizes differ.
+pkv::PlanArgs plan_args(const pkv::DecodeParams& p, const int32_t* seq_lens, int32_t num_seqs) {
+  pkv::PlanArgs a{};
+  a.seq_lens = seq_lens;
+  a.num_seqs = num_seqs;
+  a.part_tokens = p.partition_tokens;
+  a.bin_tokens = p.n_pools == 1 ? p.pool[0].block_size : pkv::kChunkTokens;
+  a.n_pools = p.n_pools;
+  for (int c = 0; c < p.n_pools; ++c) {
+    a.seq0[c] = p.pool[c].seq0;
+    a.cap[c] = p.pool[c].max_blocks * p.pool[c].block_size;
+  }
+  return a;
+}
+
 // plan kernel (or append + plan) -> decode kernel -> merge kernel (the last
 // only when some sequence can span more than one partition)
 template <int D, typename Kernel, typename... Args>
 int launch_plan_decode_merge(const pkv::DecodeParams& p, const int32_t* seq_lens, int32_t num_seqs,
                              int32_t max_tokens, const PendingAppend* ap, Kernel kern, int grid, int threads,
                              size_t smem, cudaStream_t stream, Args... args) {
-  const int kmax = p.partition_tokens / p.block_size;
+  const pkv::PlanArgs pa = plan_args(p, seq_lens, num_seqs);
+  const int kmax = pa.part_tokens / pa.bin_tokens;
   const size_t plan_smem = 2 * (kmax + 1) * sizeof(int32_t);
   int4* items = const_cast<int4*>(p.items);
   int32_t* n_items = const_cast<int32_t*>(p.n_items);
   if (ap) {
     const unsigned g = static_cast<unsigned>(1 + (ap->args.n_units + 255) / 256);
     switch (ap->src_dtype) {
-      case -1:
-        pkv::append_plan_kernel<void><<<g, 256, plan_smem, stream>>>(ap->args, seq_lens, num_seqs, max_tokens,
-                                                                     p.partition_tokens, p.block_size, items, n_items);
-        break;
-      case PKV_F32:
-        pkv::append_plan_kernel<float><<<g, 256, plan_smem, stream>>>(ap->args, seq_lens, num_seqs, max_tokens,
-                                                                      p.partition_tokens, p.block_size, items, n_items);
-        break;
+      case -1: pkv::append_plan_kernel<void><<<g, 256, plan_smem, stream>>>(ap->args, pa, items, n_items); break;
+      case PKV_F32: pkv::append_plan_kernel<float><<<g, 256, plan_smem, stream>>>(ap->args, pa, items, n_items); break;
       case PKV_BF16:
-        pkv::append_plan_kernel<__nv_bfloat16><<<g, 256, plan_smem, stream>>>(
-            ap->args, seq_lens, num_seqs, max_tokens, p.partition_tokens, p.block_size, items, n_items);
+        pkv::append_plan_kernel<__nv_bfloat16><<<g, 256, plan_smem, stream>>>(ap->args, pa, items, n_items);
         break;
-      default:
-        pkv::append_plan_kernel<__half><<<g, 256, plan_smem, stream>>>(ap->args, seq_lens, num_seqs, max_tokens,
-                                                                       p.partition_tokens, p.block_size, items, n_items);
+      default: pkv::append_plan_kernel<__half><<<g, 256, plan_smem, stream>>>(ap->args, pa, items, n_items);
     }
   } else {
-    pkv::plan_kernel<<<1, 1024, plan_smem, stream>>>(seq_lens, num_seqs, max_tokens, p.partition_tokens, p.block_size,
-                                                     items, n_items);
+    pkv::plan_kernel<<<1, 1024, plan_smem, stream>>>(pa, items, n_items);
   }
   cudaError_t e = launch_pdl(kern, dim3(grid), dim3(threads), smem, stream, p, args...);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
@@ -177,17 +232,19 @@ template <typename T, int D, int G>
 int launch_decode(const pkv::DecodeParams& base, const int32_t* seq_lens, int32_t num_seqs, int32_t max_tokens,
                   const PendingAppend* ap, cudaStream_t stream) {
   pkv::DecodeParams p = base;
+  apply_debug(p);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  p.n_stages = ring_stages(size_t(2) * p.block_size * D * sizeof(T));
-  const size_t smem = pkv::DecodeSmem<T, D, G>::bytes(p.block_size, p.n_stages);
+  const int32_t bs = p.pool[0].block_size;
+  p.n_stages = ring_stages(size_t(2) * bs * D * sizeof(T));
+  const size_t smem = pkv::DecodeSmem<T, D, G>::bytes(bs, p.n_stages);
   auto kern = pkv::decode_kernel<T, D, G>;
 
   // per device: opt in to the largest dynamic shared memory any block size
   // needs (once), then cache resident CTAs per SM for this block size
   static std::atomic<int> occ_cache[kMaxDevices][3];
-  const int bs_idx = p.block_size == 8 ? 0 : (p.block_size == 16 ? 1 : 2);
+  const int bs_idx = bs == 8 ? 0 : (bs == 16 ? 1 : 2);
   int occ = dev < kMaxDevices ? occ_cache[dev][bs_idx].load(std::memory_order_relaxed) : 0;
   if (occ == 0) {
     size_t smem_max = 0;
@@ -259,7 +316,8 @@ int make_pool_map(CUtensorMap* m, const void* pool, int dtype, int64_t rows, int
   return PKV_OK;
 }
 
-// Small cache of encoded maps: a decode step reuses the same pools every call.
+// Small cache of encoded maps: a decode step reuses the same pools every call
+// (up to 16 pools' K and V maps: several caches, or several block-size pools).
 struct MapCacheEntry {
   const void* pool;
   int64_t rows;
@@ -269,7 +327,7 @@ struct MapCacheEntry {
 
 int pool_map(CUtensorMap* out, const void* pool, int dtype, int64_t rows, int head_dim, int box_rows) {
   static std::mutex mu;
-  static MapCacheEntry cache[8];
+  static MapCacheEntry cache[16];
   static int next = 0, used = 0;
   std::lock_guard<std::mutex> g(mu);
   for (int i = 0; i < used; ++i) {
@@ -282,21 +340,22 @@ int pool_map(CUtensorMap* out, const void* pool, int dtype, int64_t rows, int he
   int rc = make_pool_map(out, pool, dtype, rows, head_dim, box_rows);
   if (rc) return rc;
   cache[next] = MapCacheEntry{pool, rows, dtype, head_dim, box_rows, *out};
-  next = (next + 1) % 8;
-  used = used < 8 ? used + 1 : 8;
+  next = (next + 1) % 16;
+  used = used < 16 ? used + 1 : 16;
   return PKV_OK;
 }
 
-template <typename T, int D, int G, int kKVBytes = 2>
+template <typename T, int D, int G, int kKVBytes = 2, bool kMulti = false>
 int launch_decode_mma(const pkv::DecodeParams& base, const int32_t* seq_lens, int32_t num_seqs, int32_t max_tokens,
                       int dtype, const PendingAppend* ap, cudaStream_t stream) {
   pkv::DecodeParams p = base;
+  apply_debug(p);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   p.n_stages = 8;
   const size_t smem = pkv::MmaSmem<T, D, G, kKVBytes>::bytes(p.n_stages);
-  auto kern = pkv::decode_mma_kernel<T, D, G, kKVBytes>;
+  auto kern = pkv::decode_mma_kernel<T, D, G, kKVBytes, kMulti>;
   static std::atomic<int> occ_cache[kMaxDevices];
   int occ = dev < kMaxDevices ? occ_cache[dev].load(std::memory_order_relaxed) : 0;
   if (occ == 0) {
@@ -309,18 +368,22 @@ int launch_decode_mma(const pkv::DecodeParams& base, const int32_t* seq_lens, in
     if (occ <= 0) return fail(PKV_ERR_CUDA, "decode_mma kernel does not fit on an SM (smem %zu)", smem);
     if (dev < kMaxDevices) occ_cache[dev].store(occ, std::memory_order_relaxed);
   }
-  const int64_t rows = int64_t(p.num_blocks) * p.num_kv_heads * p.block_size;
-  const int box_rows = p.block_size < pkv::kChunkTokens ? p.block_size : pkv::kChunkTokens;
-  CUtensorMap mk, mv;
-  int rc = pool_map(&mk, p.k_pool, dtype, rows, D, box_rows);
-  if (rc) return rc;
-  rc = pool_map(&mv, p.v_pool, dtype, rows, D, box_rows);
-  if (rc) return rc;
+  pkv::PoolMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  for (int c = 0; c < p.n_pools; ++c) {
+    const pkv::PoolView& pv = p.pool[c];
+    const int64_t rows = int64_t(pv.num_blocks) * p.num_kv_heads * pv.block_size;
+    const int box_rows = pv.block_size < pkv::kChunkTokens ? pv.block_size : pkv::kChunkTokens;
+    int rc = pool_map(&maps.k[c], pv.k, dtype, rows, D, box_rows);
+    if (rc) return rc;
+    rc = pool_map(&maps.v[c], pv.v, dtype, rows, D, box_rows);
+    if (rc) return rc;
+  }
 
   const int64_t work_upper = int64_t(num_seqs) * p.max_parts * p.num_kv_heads;
   const int grid = static_cast<int>(std::min<int64_t>(int64_t(sm_count(dev)) * occ, work_upper));
   return launch_plan_decode_merge<D>(p, seq_lens, num_seqs, max_tokens, ap, kern, grid, pkv::kMmaThreads, smem, stream,
-                                     mk, mv);
+                                     maps);
 }
 
 template <typename T>
@@ -354,6 +417,7 @@ int dispatch_decode(int32_t head_dim, int32_t group, const pkv::DecodeParams& p,
 extern "C" int pkv_kv_append(const void* k_new, const void* v_new, const int32_t* slot_mapping, int32_t n_tokens,
                              void* k_pool, void* v_pool, int32_t num_blocks, int32_t num_kv_heads,
                              int32_t head_dim, int32_t block_size, int32_t dtype, void* stream) {
+  NvtxRange nvtx_range("pkv_kv_append");
   int rc = check_common(num_kv_heads, head_dim, block_size, dtype, "pkv_kv_append");
   if (rc) return rc;
   if (n_tokens < 0 || num_blocks <= 0) return fail(PKV_ERR_INVALID_ARG, "pkv_kv_append: n_tokens/num_blocks");
@@ -365,8 +429,8 @@ extern "C" int pkv_kv_append(const void* k_new, const void* v_new, const int32_t
   const int32_t row_chunks = static_cast<int32_t>(head_dim * elem_size(dtype) / 16);
   const int64_t n_chunks = int64_t(n_tokens) * num_kv_heads * row_chunks;
   const int64_t blocks = (n_chunks + 255) / 256;
-  const pkv::AppendArgs a{k_new, v_new, slot_mapping, n_chunks, k_pool,     v_pool,
-                          num_blocks, num_kv_heads, row_chunks, block_size, 1.0f, 1.0f};
+  const pkv::AppendArgs a = single_append(k_new, v_new, slot_mapping, n_chunks, k_pool, v_pool, num_blocks,
+                                          num_kv_heads, row_chunks, block_size, 1.0f, 1.0f);
   pkv::kv_append_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pkv_kv_append launch");
@@ -376,6 +440,7 @@ extern "C" int pkv_kv_append(const void* k_new, const void* v_new, const int32_t
 extern "C" int pkv_copy_blocks(void* k_pool, void* v_pool, const int32_t* block_pairs, int32_t n_pairs,
                                int32_t num_blocks, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                                int32_t dtype, void* stream) {
+  NvtxRange nvtx_range("pkv_copy_blocks");
   // a byte copy: e4m3 pools are copied like 16-bit ones, at one byte per element
   int rc = check_common(num_kv_heads, head_dim, block_size, dtype == PKV_FP8_E4M3 ? PKV_F16 : dtype, "pkv_copy_blocks");
   if (rc) return rc;
@@ -464,14 +529,9 @@ int decode_16(const char* fn, const void* q, const void* k_pool, const void* v_p
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   pkv::DecodeParams p{};
   p.q = q;
-  p.k_pool = k_pool;
-  p.v_pool = v_pool;
-  p.block_tables = block_tables;
+  set_single_pool(p, k_pool, v_pool, block_tables, num_blocks, max_blocks_per_seq, block_size);
   p.num_q_heads = num_q_heads;
   p.num_kv_heads = num_kv_heads;
-  p.num_blocks = num_blocks;
-  p.max_blocks = max_blocks_per_seq;
-  p.block_size = block_size;
   p.partition_tokens = pt;
   p.max_parts = w.max_parts;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
@@ -509,6 +569,7 @@ extern "C" int pkv_paged_attention_decode(const void* q, const void* k_pool, con
                                           int32_t num_blocks, int32_t max_blocks_per_seq, int32_t block_size,
                                           float scale, int32_t dtype, int32_t partition_tokens, void* workspace,
                                           size_t workspace_bytes, float* out, void* stream) {
+  NvtxRange nvtx_range("pkv_paged_attention_decode");
   return decode_16("pkv_paged_attention_decode", q, k_pool, v_pool, block_tables, seq_lens, num_seqs, num_q_heads,
                    num_kv_heads, head_dim, num_blocks, max_blocks_per_seq, block_size, scale, dtype, partition_tokens,
                    workspace, workspace_bytes, out, nullptr, stream);
@@ -521,6 +582,7 @@ extern "C" int pkv_append_and_decode(const void* k_new, const void* v_new, const
                                      int32_t max_blocks_per_seq, int32_t block_size, float scale, int32_t dtype,
                                      int32_t partition_tokens, void* workspace, size_t workspace_bytes, float* out,
                                      void* stream) {
+  NvtxRange nvtx_range("pkv_append_and_decode");
   const char* fn = "pkv_append_and_decode";
   int rc = check_common(num_kv_heads, head_dim, block_size, dtype, fn);
   if (rc) return rc;
@@ -531,12 +593,18 @@ extern "C" int pkv_append_and_decode(const void* k_new, const void* v_new, const
       return fail(PKV_ERR_INVALID_ARG, "%s: K/V buffers must be 16-byte aligned", fn);
   }
   const int32_t row_chunks = static_cast<int32_t>(head_dim * elem_size(dtype) / 16);
-  PendingAppend ap{{k_new, v_new, slot_mapping, int64_t(n_tokens) * num_kv_heads * row_chunks, k_pool, v_pool,
-                    num_blocks, num_kv_heads, row_chunks, block_size, 1.0f, 1.0f},
+  PendingAppend ap{single_append(k_new, v_new, slot_mapping, int64_t(n_tokens) * num_kv_heads * row_chunks, k_pool,
+                                 v_pool, num_blocks, num_kv_heads, row_chunks, block_size, 1.0f, 1.0f),
                    -1};
   return decode_16(fn, q, k_pool, v_pool, block_tables, seq_lens, num_seqs, num_q_heads, num_kv_heads, head_dim,
                    num_blocks, max_blocks_per_seq, block_size, scale, dtype, partition_tokens, workspace,
                    workspace_bytes, out, n_tokens > 0 ? &ap : nullptr, stream);
+}
+
+extern "C" int pkv_debug_stall_decode(int32_t cta, uint64_t consumer_wait_ns) {
+  g_stall_cta.store(cta < 0 ? -1 : cta, std::memory_order_relaxed);
+  g_consumer_wait_ns.store(consumer_wait_ns == 0 ? pkv::kWaitLimitNs : consumer_wait_ns, std::memory_order_relaxed);
+  return pkv::ok();
 }
 
 extern "C" int pkv_device_status(void* stream, int32_t* status, int32_t clear) {
@@ -556,12 +624,159 @@ extern "C" int pkv_device_status(void* stream, int32_t* status, int32_t clear) {
 }
 
 // ===========================================================================
+// A decode step over a batch spread across pools of different block sizes
+// ===========================================================================
+namespace {
+
+constexpr int kMaxPoolsAbi = pkv::kMaxPools;
+
+// Checks the pool list; on success `total` is the batch size, `max_tokens`
+// the largest per-sequence capacity and `pt` the partition size.
+int check_pools(const char* fn, const pkv_pool_t* pools, int32_t n_pools, int32_t partition_tokens, int64_t* total,
+                int64_t* max_tokens, int32_t* pt) {
+  if (!pools || n_pools < 1 || n_pools > kMaxPoolsAbi)
+    return fail(PKV_ERR_INVALID_ARG, "%s: 1 to %d pools", fn, kMaxPoolsAbi);
+  int32_t part = partition_tokens == 0 ? kAutoPartitionTokens : partition_tokens;
+  if (part <= 0 || part % pkv::kChunkTokens != 0 || part > kMaxPartitionTokens)
+    return fail(PKV_ERR_INVALID_ARG, "%s: partition_tokens %d must be a positive multiple of 16, at most %d", fn,
+                partition_tokens, kMaxPartitionTokens);
+  *total = 0;
+  *max_tokens = 0;
+  for (int c = 0; c < n_pools; ++c) {
+    const pkv_pool_t& q = pools[c];
+    if (q.block_size != 8 && q.block_size != 16 && q.block_size != 32)
+      return fail(PKV_ERR_UNSUPPORTED, "%s: pool %d block_size %d not supported (8, 16 or 32)", fn, c, q.block_size);
+    if (part % q.block_size != 0)
+      return fail(PKV_ERR_INVALID_ARG, "%s: partition_tokens %d is not a multiple of pool %d's block_size %d", fn, part,
+                  c, q.block_size);
+    if (q.num_seqs < 0 || q.num_blocks <= 0 || q.max_blocks_per_seq < 0)
+      return fail(PKV_ERR_INVALID_ARG, "%s: pool %d: bad sizes", fn, c);
+    *total += q.num_seqs;
+    *max_tokens = std::max<int64_t>(*max_tokens, int64_t(q.max_blocks_per_seq) * q.block_size);
+  }
+  if (*total > INT32_MAX / 2) return fail(PKV_ERR_INVALID_ARG, "%s: too many sequences", fn);
+  if (*max_tokens > (int64_t(1) << 30)) return fail(PKV_ERR_INVALID_ARG, "%s: max_blocks_per_seq too large", fn);
+  *pt = part;
+  return PKV_OK;
+}
+
+}  // namespace
+
+extern "C" int pkv_decode_pools_workspace_size(const pkv_pool_t* pools, int32_t n_pools, int32_t num_q_heads,
+                                               int32_t num_kv_heads, int32_t head_dim, int32_t partition_tokens,
+                                               size_t* bytes) {
+  const char* fn = "pkv_decode_pools_workspace_size";
+  if (!bytes) return fail(PKV_ERR_INVALID_ARG, "%s: bytes is NULL", fn);
+  if (num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0) return fail(PKV_ERR_INVALID_ARG, "%s: bad sizes", fn);
+  int64_t total = 0, max_tokens = 0;
+  int32_t pt = 0;
+  int rc = check_pools(fn, pools, n_pools, partition_tokens, &total, &max_tokens, &pt);
+  if (rc) return rc;
+  *bytes = ws_layout(total, num_q_heads, num_kv_heads, head_dim, max_tokens, pt).total;
+  return pkv::ok();
+}
+
+extern "C" int pkv_append_and_decode_pools(const pkv_pool_t* pools, int32_t n_pools, const void* k_new,
+                                           const void* v_new, const int32_t* slot_mapping, const void* q,
+                                           const int32_t* seq_lens, int32_t num_q_heads, int32_t num_kv_heads,
+                                           int32_t head_dim, float scale, int32_t dtype, int32_t partition_tokens,
+                                           void* workspace, size_t workspace_bytes, float* out, void* stream) {
+  const char* fn = "pkv_append_and_decode_pools";
+  NvtxRange nvtx_range(fn);
+  if (dtype != PKV_BF16 && dtype != PKV_F16)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: dtype %d not supported (bf16 or f16)", fn, dtype);
+  if (head_dim != 128) return fail(PKV_ERR_UNSUPPORTED, "%s: head_dim %d not supported (128)", fn, head_dim);
+  if (num_kv_heads <= 0 || num_q_heads <= 0 || num_q_heads % num_kv_heads != 0)
+    return fail(PKV_ERR_INVALID_ARG, "%s: num_q_heads %d must be a positive multiple of num_kv_heads %d", fn,
+                num_q_heads, num_kv_heads);
+  const int32_t group = num_q_heads / num_kv_heads;
+  if (group != 2 && group != 4 && group != 8)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: group size %d not supported (2, 4 or 8)", fn, group);
+  if (!std::isfinite(scale)) return fail(PKV_ERR_INVALID_ARG, "%s: scale is not finite", fn);
+  int64_t total = 0, max_tokens = 0;
+  int32_t pt = 0;
+  int rc = check_pools(fn, pools, n_pools, partition_tokens, &total, &max_tokens, &pt);
+  if (rc) return rc;
+  if (total == 0) return pkv::ok();
+  if (!k_new || !v_new || !slot_mapping || !q || !seq_lens || !workspace || !out)
+    return fail(PKV_ERR_INVALID_ARG, "%s: NULL pointer", fn);
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(q) || !aligned16(out))
+    return fail(PKV_ERR_INVALID_ARG, "%s: q, new rows and out must be 16-byte aligned", fn);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(PKV_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", fn);
+  const int32_t N = static_cast<int32_t>(total);
+  const WsLayout w = ws_layout(N, num_q_heads, num_kv_heads, head_dim, max_tokens, pt);
+  if (workspace_bytes < w.total)
+    return fail(PKV_ERR_INVALID_ARG, "%s: workspace %zu bytes < %zu needed", fn, workspace_bytes, w.total);
+
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  pkv::DecodeParams p{};
+  p.q = q;
+  const int32_t row_chunks = head_dim * 2 / 16;
+  pkv::AppendArgs a{};
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.slots = slot_mapping;
+  a.n_units = int64_t(N) * num_kv_heads * row_chunks;
+  a.n_pools = n_pools;
+  a.num_kv_heads = num_kv_heads;
+  a.row_units = row_chunks;
+  a.k_inv = a.v_inv = 1.0f;
+  int32_t seq0 = 0;
+  for (int c = 0; c < n_pools; ++c) {
+    const pkv_pool_t& pc = pools[c];
+    if (pc.num_seqs > 0) {
+      if (!pc.k_pool || !pc.v_pool || !pc.block_tables) return fail(PKV_ERR_INVALID_ARG, "%s: pool %d: NULL pointer", fn, c);
+      if (!aligned16(pc.k_pool) || !aligned16(pc.v_pool))
+        return fail(PKV_ERR_INVALID_ARG, "%s: pool %d must be 16-byte aligned", fn, c);
+    }
+    if (int64_t(pc.num_blocks) * num_kv_heads * pc.block_size > INT32_MAX)
+      return fail(PKV_ERR_INVALID_ARG, "%s: pool %d has more than 2^31 token rows", fn, c);
+    p.pool[c] = pkv::PoolView{pc.k_pool, pc.v_pool, pc.block_tables, pc.num_blocks, pc.max_blocks_per_seq,
+                              pc.block_size, seq0};
+    a.k_pool[c] = pc.k_pool;
+    a.v_pool[c] = pc.v_pool;
+    a.num_blocks[c] = pc.num_blocks;
+    a.block_size[c] = pc.block_size;
+    a.tok0[c] = seq0;
+    seq0 += pc.num_seqs;
+  }
+  // pools without sequences still count in the thresholds (seq0 equal to the
+  // next pool's), so no sequence maps to them
+  p.n_pools = n_pools;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.partition_tokens = pt;
+  p.max_parts = w.max_parts;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.v_scale = 1.0f;
+  p.items = reinterpret_cast<const int4*>(ws + w.items);
+  p.n_items = reinterpret_cast<const int32_t*>(ws);
+  p.part_m = reinterpret_cast<float*>(ws + w.m);
+  p.part_l = reinterpret_cast<float*>(ws + w.l);
+  p.part_o = reinterpret_cast<float*>(ws + w.o);
+  p.out = out;
+  const PendingAppend ap{a, -1};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int32_t mt = static_cast<int32_t>(max_tokens);
+  if (dtype == PKV_BF16) {
+    if (group == 2) return launch_decode_mma<__nv_bfloat16, 128, 2, 2, true>(p, seq_lens, N, mt, dtype, &ap, s);
+    if (group == 4) return launch_decode_mma<__nv_bfloat16, 128, 4, 2, true>(p, seq_lens, N, mt, dtype, &ap, s);
+    return launch_decode_mma<__nv_bfloat16, 128, 8, 2, true>(p, seq_lens, N, mt, dtype, &ap, s);
+  }
+  if (group == 2) return launch_decode_mma<__half, 128, 2, 2, true>(p, seq_lens, N, mt, dtype, &ap, s);
+  if (group == 4) return launch_decode_mma<__half, 128, 4, 2, true>(p, seq_lens, N, mt, dtype, &ap, s);
+  return launch_decode_mma<__half, 128, 8, 2, true>(p, seq_lens, N, mt, dtype, &ap, s);
+}
+
+// ===========================================================================
 // FP8 (e4m3) KV cache
 // ===========================================================================
 extern "C" int pkv_kv_append_fp8(const void* k_new, const void* v_new, int32_t src_dtype,
                                  const int32_t* slot_mapping, int32_t n_tokens, void* k_pool, void* v_pool,
                                  int32_t num_blocks, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                                  float k_scale, float v_scale, void* stream) {
+  NvtxRange nvtx_range("pkv_kv_append_fp8");
   const char* fn = "pkv_kv_append_fp8";
   int rc = check_common(num_kv_heads, head_dim, block_size, src_dtype, fn);
   if (rc) return rc;
@@ -577,8 +792,8 @@ extern "C" int pkv_kv_append_fp8(const void* k_new, const void* v_new, int32_t s
   const int64_t n_groups = int64_t(n_tokens) * num_kv_heads * (head_dim / 8);
   const unsigned blocks = static_cast<unsigned>((n_groups + 255) / 256);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const pkv::AppendArgs a{k_new,      v_new,        slot_mapping, n_groups,   k_pool, v_pool,
-                          num_blocks, num_kv_heads, head_dim / 8, block_size, k_inv,  v_inv};
+  const pkv::AppendArgs a = single_append(k_new, v_new, slot_mapping, n_groups, k_pool, v_pool, num_blocks,
+                                          num_kv_heads, head_dim / 8, block_size, k_inv, v_inv);
   switch (src_dtype) {
     case PKV_F32: pkv::kv_append_fp8_kernel<float><<<blocks, 256, 0, s>>>(a); break;
     case PKV_BF16: pkv::kv_append_fp8_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(a); break;
@@ -629,14 +844,9 @@ int decode_fp8(const char* fn, const void* q, const void* k_pool, const void* v_
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   pkv::DecodeParams p{};
   p.q = q;
-  p.k_pool = k_pool;
-  p.v_pool = v_pool;
-  p.block_tables = block_tables;
+  set_single_pool(p, k_pool, v_pool, block_tables, num_blocks, max_blocks_per_seq, block_size);
   p.num_q_heads = num_q_heads;
   p.num_kv_heads = num_kv_heads;
-  p.num_blocks = num_blocks;
-  p.max_blocks = max_blocks_per_seq;
-  p.block_size = block_size;
   p.partition_tokens = pt;
   p.max_parts = w.max_parts;
   // scores = scale * k_scale * q·codes; output = v_scale * softmax-weighted codes
@@ -666,6 +876,7 @@ extern "C" int pkv_paged_attention_decode_fp8(const void* q, const void* k_pool,
                                               int32_t num_blocks, int32_t max_blocks_per_seq, int32_t block_size,
                                               float scale, float k_scale, float v_scale, int32_t partition_tokens,
                                               void* workspace, size_t workspace_bytes, float* out, void* stream) {
+  NvtxRange nvtx_range("pkv_paged_attention_decode_fp8");
   return decode_fp8("pkv_paged_attention_decode_fp8", q, k_pool, v_pool, block_tables, seq_lens, num_seqs,
                     num_q_heads, num_kv_heads, head_dim, num_blocks, max_blocks_per_seq, block_size, scale, k_scale,
                     v_scale, partition_tokens, workspace, workspace_bytes, out, nullptr, stream);
@@ -679,6 +890,7 @@ extern "C" int pkv_append_and_decode_fp8(const void* k_new, const void* v_new, i
                                          int32_t block_size, float scale, float k_scale, float v_scale,
                                          int32_t partition_tokens, void* workspace, size_t workspace_bytes,
                                          float* out, void* stream) {
+  NvtxRange nvtx_range("pkv_append_and_decode_fp8");
   const char* fn = "pkv_append_and_decode_fp8";
   int rc = check_common(num_kv_heads, head_dim, block_size, src_dtype, fn);
   if (rc) return rc;
@@ -692,8 +904,8 @@ extern "C" int pkv_append_and_decode_fp8(const void* k_new, const void* v_new, i
   }
   const float k_inv = static_cast<float>(1.0 / static_cast<double>(k_scale));
   const float v_inv = static_cast<float>(1.0 / static_cast<double>(v_scale));
-  PendingAppend ap{{k_new, v_new, slot_mapping, int64_t(n_tokens) * num_kv_heads * (head_dim / 8), k_pool, v_pool,
-                    num_blocks, num_kv_heads, head_dim / 8, block_size, k_inv, v_inv},
+  PendingAppend ap{single_append(k_new, v_new, slot_mapping, int64_t(n_tokens) * num_kv_heads * (head_dim / 8),
+                                 k_pool, v_pool, num_blocks, num_kv_heads, head_dim / 8, block_size, k_inv, v_inv),
                    src_dtype};
   return decode_fp8(fn, q, k_pool, v_pool, block_tables, seq_lens, num_seqs, num_q_heads, num_kv_heads, head_dim,
                     num_blocks, max_blocks_per_seq, block_size, scale, k_scale, v_scale, partition_tokens, workspace,
@@ -747,6 +959,7 @@ extern "C" int pkv_paged_attention_decode_static(const void* q, const void* k_po
                                                  int32_t head_dim, int32_t num_blocks, int32_t max_blocks_per_seq,
                                                  int32_t block_size, float scale, int32_t dtype,
                                                  int32_t partition_tokens, float* out, void* stream) {
+  NvtxRange nvtx_range("pkv_paged_attention_decode_static");
   size_t need = 0;
   int rc = pkv_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, block_size,
                                      partition_tokens, &need);
@@ -835,9 +1048,15 @@ int prefill_counter(unsigned int** out) {
   return PKV_OK;
 }
 
+// Bytes of the staged f16 copy of V (bf16 pools): a 256-byte record, then
+// [num_seqs][max_blocks][Hkv][block_size][128] f16.
+size_t prefill_stage_bytes(int64_t num_seqs, int64_t num_kv_heads, int64_t max_blocks, int64_t block_size) {
+  return 256 + round256(size_t(num_seqs * max_blocks * num_kv_heads * block_size) * 128 * sizeof(__half));
+}
+
 template <typename T, int G>
 int launch_prefill(const pkv::PrefillParams& p, const void* q, const void* k_pool, const void* v_pool, int dtype,
-                   cudaStream_t stream) {
+                   void* v_stage, cudaStream_t stream) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -856,12 +1075,42 @@ int launch_prefill(const pkv::PrefillParams& p, const void* q, const void* k_poo
   if (rc) return rc;
   rc = make_prefill_pool_map(&mv, v_pool, dtype, rows, p.block_size);
   if (rc) return rc;
+  pkv::PrefillParams pp = p;
+  CUtensorMap mvs = mv;
+  if (v_stage) {
+    // V of every sequence's blocks converted to f16 once, then read by the
+    // prefill kernel through its own map (same box shape as the pool's)
+    static std::atomic<uint32_t> epoch{0};
+    pp.epoch = epoch.fetch_add(1, std::memory_order_relaxed) + 1;
+    pp.v_staged = 1;
+    pp.v_range = static_cast<const uint32_t*>(v_stage);
+    unsigned char* copy = static_cast<unsigned char*>(v_stage) + 256;
+    const int64_t srows = int64_t(p.num_seqs) * p.max_blocks * p.num_kv_heads * p.block_size;
+    rc = make_prefill_pool_map(&mvs, copy, PKV_F16, srows, p.block_size);
+    if (rc) return rc;
+    pkv::VStageArgs a{};
+    a.block_tables = p.block_tables;
+    a.seq_lens = p.seq_lens;
+    a.v_pool = static_cast<const uint4*>(v_pool);
+    a.staged = reinterpret_cast<uint4*>(copy);
+    a.range = static_cast<uint32_t*>(v_stage);
+    a.epoch = pp.epoch;
+    a.num_seqs = p.num_seqs;
+    a.num_blocks = p.num_blocks;
+    a.max_blocks = p.max_blocks;
+    a.block_size = p.block_size;
+    a.block_pieces = p.num_kv_heads * p.block_size * 128 / 8;
+    // whole blocks per CTA: about 8 CTAs per SM over the batch
+    const int ny = std::min(p.num_seqs, 65535);
+    const int nx = std::max(1, std::min(p.max_blocks, (8 * sm_count(dev) + ny - 1) / ny));
+    pkv::stage_v_f16_kernel<<<dim3(nx, ny), 256, 0, stream>>>(a);
+  }
   const int64_t tiles = int64_t(p.n_tiles) * p.num_seqs * p.num_kv_heads;
   const int64_t grid = std::min<int64_t>(sm_count(dev), tiles);  // persistent: one CTA per SM
   unsigned int* ctr = nullptr;
   rc = prefill_counter(&ctr);
   if (rc) return rc;
-  kern<<<static_cast<unsigned>(grid), pkv::pf::kThreads, pkv::pf::kSmemBytes, stream>>>(p, mq, mk, mv, ctr);
+  kern<<<static_cast<unsigned>(grid), pkv::pf::kThreads, pkv::pf::kSmemBytes, stream>>>(pp, mq, mk, mv, mvs, ctr);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
   return pkv::ok();
@@ -869,22 +1118,33 @@ int launch_prefill(const pkv::PrefillParams& p, const void* q, const void* k_poo
 
 template <typename T>
 int dispatch_prefill(int32_t group, const pkv::PrefillParams& p, const void* q, const void* k_pool, const void* v_pool,
-                     int dtype, cudaStream_t s) {
-  if (group == 1) return launch_prefill<T, 1>(p, q, k_pool, v_pool, dtype, s);
-  if (group == 2) return launch_prefill<T, 2>(p, q, k_pool, v_pool, dtype, s);
-  if (group == 4) return launch_prefill<T, 4>(p, q, k_pool, v_pool, dtype, s);
-  return launch_prefill<T, 8>(p, q, k_pool, v_pool, dtype, s);
+                     int dtype, void* v_stage, cudaStream_t s) {
+  if (group == 1) return launch_prefill<T, 1>(p, q, k_pool, v_pool, dtype, v_stage, s);
+  if (group == 2) return launch_prefill<T, 2>(p, q, k_pool, v_pool, dtype, v_stage, s);
+  if (group == 4) return launch_prefill<T, 4>(p, q, k_pool, v_pool, dtype, v_stage, s);
+  return launch_prefill<T, 8>(p, q, k_pool, v_pool, dtype, v_stage, s);
 }
 
 }  // namespace
+
+extern "C" int pkv_prefill_workspace_size(int32_t num_seqs, int32_t num_kv_heads, int32_t head_dim,
+                                          int32_t max_blocks_per_seq, int32_t block_size, int32_t dtype,
+                                          size_t* bytes) {
+  if (!bytes) return fail(PKV_ERR_INVALID_ARG, "pkv_prefill_workspace_size: bytes is NULL");
+  if (num_seqs < 0 || num_kv_heads <= 0 || head_dim <= 0 || max_blocks_per_seq < 0 || block_size <= 0)
+    return fail(PKV_ERR_INVALID_ARG, "pkv_prefill_workspace_size: bad sizes");
+  *bytes = dtype == PKV_BF16 ? prefill_stage_bytes(num_seqs, num_kv_heads, max_blocks_per_seq, block_size) : 0;
+  return pkv::ok();
+}
 
 extern "C" int pkv_paged_attention_prefill(const void* q, const void* k_pool, const void* v_pool,
                                            const int32_t* block_tables, const int32_t* seq_lens,
                                            const int32_t* q_start, int32_t num_seqs, int32_t num_q_tokens,
                                            int32_t max_q_len, int32_t num_q_heads, int32_t num_kv_heads,
                                            int32_t head_dim, int32_t num_blocks, int32_t max_blocks_per_seq,
-                                           int32_t block_size, float scale, int32_t dtype, float* out,
-                                           void* stream) {
+                                           int32_t block_size, float scale, int32_t dtype, void* workspace,
+                                           size_t workspace_bytes, float* out, void* stream) {
+  NvtxRange nvtx_range("pkv_paged_attention_prefill");
   const char* fn = "pkv_paged_attention_prefill";
   if (dtype != PKV_BF16 && dtype != PKV_F16)
     return fail(PKV_ERR_UNSUPPORTED, "%s: dtype %d not supported (bf16 or f16)", fn, dtype);
@@ -930,9 +1190,20 @@ extern "C" int pkv_paged_attention_prefill(const void* q, const void* k_pool, co
   p.max_q_len = max_q_len;
   p.n_tiles = static_cast<int32_t>(n_tiles);
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  void* v_stage = nullptr;
+  if (dtype == PKV_BF16 && workspace) {
+    const size_t need = prefill_stage_bytes(num_seqs, num_kv_heads, max_blocks_per_seq, block_size);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      return fail(PKV_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", fn);
+    if (workspace_bytes < need)
+      return fail(PKV_ERR_INVALID_ARG, "%s: workspace %zu bytes < %zu needed", fn, workspace_bytes, need);
+    if (int64_t(num_seqs) * max_blocks_per_seq * num_kv_heads * block_size >= (int64_t(1) << 31))
+      return fail(PKV_ERR_INVALID_ARG, "%s: staged V rows exceed 2^31", fn);
+    v_stage = workspace;
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (dtype == PKV_BF16) return dispatch_prefill<__nv_bfloat16>(group, p, q, k_pool, v_pool, dtype, s);
-  return dispatch_prefill<__half>(group, p, q, k_pool, v_pool, dtype, s);
+  if (dtype == PKV_BF16) return dispatch_prefill<__nv_bfloat16>(group, p, q, k_pool, v_pool, dtype, v_stage, s);
+  return dispatch_prefill<__half>(group, p, q, k_pool, v_pool, dtype, nullptr, s);
 }
 
 // =============================================================================
@@ -949,6 +1220,7 @@ extern "C" int pkv_decode_step_host(pkv_alloc_t* a, const int64_t* seq_ids, int3
                                     int32_t max_blocks_per_seq, float scale, int32_t dtype, float k_scale,
                                     float v_scale, int32_t partition_tokens, void* workspace,
                                     size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("pkv_decode_step_host");
   const char* fn = "pkv_decode_step_host";
   if (!a || !buf || n < 0 || max_blocks_per_seq <= 0 || num_kv_heads <= 0 || num_q_heads <= 0 || head_dim <= 0)
     return fail(PKV_ERR_INVALID_ARG, "%s: bad arguments", fn);

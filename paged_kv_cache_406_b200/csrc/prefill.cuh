@@ -68,6 +68,13 @@ struct PrefillParams {
   int32_t num_seqs, num_q_heads, num_kv_heads, num_blocks, max_blocks, block_size;
   int32_t num_q_tokens, max_q_len, n_tiles;
   float scale_log2;  // scale · log2(e), positive
+  // bf16 pools with a staged f16 copy of V (v_staged != 0): P·V runs as one
+  // f16 pass over the copy (tmap_vs), unless the staging recorded a value
+  // beyond the f16 range (*v_range == epoch), in which case it runs as the
+  // two bf16 passes (P hi and lo) over the pool's V
+  int32_t v_staged;
+  uint32_t epoch;
+  const uint32_t* v_range;
 };
 
 #ifndef PKV_PREFILL_STAGES
@@ -188,15 +195,90 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return r;
 }
 
+// ---------------------------------------------------------------------------
+// V staged as f16 for bf16 pools (one pass per call, before the prefill
+// kernel).  bf16 carries 8 significant bits and f16 11, so every bf16 value
+// of magnitude in [2^-14, 65504] converts exactly; smaller ones round to f16
+// subnormals (absolute error at most 2^-25).  A finite value above 65504 has
+// no f16 counterpart: the kernel then writes the call's epoch into *range and
+// the prefill kernel keeps the bf16 hi + lo path over the pool's own V.
+// Layout of the copy: [num_seqs][max_blocks][Hkv][block_size][128] f16; the
+// blocks of sequence b past ceil(seq_lens[b] / block_size) are not written.
+// Grid: y strides over the sequences, x over the blocks of one; a CTA copies
+// whole blocks (one table read each), four 16-byte pieces per thread in
+// flight.
+// ---------------------------------------------------------------------------
+struct VStageArgs {
+  const int32_t* block_tables;
+  const int32_t* seq_lens;
+  const uint4* v_pool;  // bf16 pool, 16 bytes = 8 elements
+  uint4* staged;        // f16 copy
+  uint32_t* range;
+  uint32_t epoch;
+  int32_t num_seqs, num_blocks, max_blocks, block_size, block_pieces;  // pieces: Hkv * block_size * 128 / 8
+};
+
+// Eight bf16 values (16 bytes) to eight f16 values; `over` is set if a finite
+// value lies beyond the f16 range.
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4 w, bool& over) {
+  const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+  uint32_t res[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    // bf16 is the top half of an fp32: widening is a shift
+    const float lo = __uint_as_float(in[k] << 16), hi = __uint_as_float(in[k] & 0xffff0000u);
+    over |= (fabsf(lo) > 65504.f && fabsf(lo) != INFINITY) || (fabsf(hi) > 65504.f && fabsf(hi) != INFINITY);
+    const __half2 h = __floats2half2_rn(lo, hi);
+    res[k] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  return make_uint4(res[0], res[1], res[2], res[3]);
+}
+
+__global__ void __launch_bounds__(256) stage_v_f16_kernel(const VStageArgs a) {
+  constexpr int kUnroll = 4;
+  bool over = false;
+  const int pieces = a.block_pieces;
+  for (int b = blockIdx.y; b < a.num_seqs; b += gridDim.y) {
+    int L = a.seq_lens[b];
+    L = L < 0 ? 0 : min(L, a.max_blocks * a.block_size);
+    const int nblk = (L + a.block_size - 1) / a.block_size;
+    const int32_t* trow = a.block_tables + static_cast<int64_t>(b) * a.max_blocks;
+    for (int j = blockIdx.x; j < nblk; j += gridDim.x) {
+      int phys = trow[j];
+      if (static_cast<unsigned>(phys) >= static_cast<unsigned>(a.num_blocks)) {
+        if (threadIdx.x == 0) record_error(PKV_ERR_BAD_BLOCK);
+        phys = 0;
+      }
+      const uint4* src = a.v_pool + static_cast<int64_t>(phys) * pieces;
+      uint4* dst = a.staged + (static_cast<int64_t>(b) * a.max_blocks + j) * pieces;
+      int i = threadIdx.x;
+      for (; i + (kUnroll - 1) * 256 < pieces; i += kUnroll * 256) {
+        uint4 w[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) w[u] = src[i + u * 256];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) dst[i + u * 256] = bf16x8_to_f16x8(w[u], over);
+      }
+      for (; i < pieces; i += 256) dst[i] = bf16x8_to_f16x8(src[i], over);
+    }
+  }
+  if (__any_sync(0xffffffffu, over) && (threadIdx.x & 31) == 0) atomicExch(a.range, a.epoch);
+}
+
 template <typename T, int G>
 __global__ void __launch_bounds__(pf::kThreads, 1)
     prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_q,
                       const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
-                      unsigned int* __restrict__ tile_ctr) {
+                      const __grid_constant__ CUtensorMap tmap_vs, unsigned int* __restrict__ tile_ctr) {
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
   constexpr int QT = pf::kRows / G;  // query tokens per tile
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
-  constexpr int kParts = kBf16 ? 2 : 1;  // P halves: hi + lo (bf16) or one f16 P
+  // One f16 P and one P·V pass (f16 pools, or bf16 pools whose V was staged
+  // as f16 within range), else P as bf16 hi + lo halves and two passes.
+  // Uniform over the launch: every thread reads the same staging record.
+  bool f16p = !kBf16;
+  if constexpr (kBf16) f16p = p.v_staged != 0 && *p.v_range != p.epoch;
+  const bool v_from_stage = kBf16 && f16p;
 
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -332,7 +414,10 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       const int nbc = pf::kKeys / BS;                              // blocks per chunk
       const uint32_t box_bytes = static_cast<uint32_t>(BS) * 128;  // one block, one head_dim half
       const uint32_t full0 = bar(kv ? pf::kVFull : pf::kKFull), empty0 = bar(kv ? pf::kVEmpty : pf::kKEmpty);
-      const void* map = kv ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k);
+      // V from the staged f16 copy: block j of sequence b sits at b * max_blocks + j, no table lookup
+      const bool staged = kv && v_from_stage;
+      const void* map = kv ? (staged ? static_cast<const void*>(&tmap_vs) : static_cast<const void*>(&tmap_v))
+                           : static_cast<const void*>(&tmap_k);
       const uint32_t ring = base + (kv ? pf::kOffV : pf::kOffK);
       for (int j = 0; j < nc && ok; ++j) {
         const int s = (gc + j) % pf::kStages;
@@ -341,10 +426,14 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         const int nload = min(nbc, nblk - jb);  // blocks past the sequence end are not read
         int phys = 0;
         if (lane < nload) {
-          phys = trow[jb + lane];
-          if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_blocks)) {
-            record_error(PKV_ERR_BAD_BLOCK);
-            phys = 0;
+          if (staged) {
+            phys = b * p.max_blocks + jb + lane;
+          } else {
+            phys = trow[jb + lane];
+            if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_blocks)) {
+              record_error(PKV_ERR_BAD_BLOCK);
+              phys = 0;
+            }
           }
         }
         const int32_t y = (phys * p.num_kv_heads + g) * BS;
@@ -381,7 +470,9 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
   } else if (warp == pf::kMmaWarp) {
     // ------------------------------- MMA issuer -------------------------------
     const uint32_t id_s = tc::idesc_f16(kBf16, false, pf::kRows, pf::kKeys);
-    const uint32_t id_o = tc::idesc_f16(kBf16, true, pf::kRows, pf::kHeadDim);
+    // P·V: f16 P and f16 V in one pass, or bf16 P hi and lo over bf16 V
+    const uint32_t id_o = tc::idesc_f16(kBf16 && !f16p, true, pf::kRows, pf::kHeadDim);
+    const int parts = f16p ? 1 : 2;
     bool ok = true;
     int gc = 0, tv = 0;
     for (int ti = 0; ok; ++ti) {
@@ -421,8 +512,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
           tc::fence_after_sync();
           const uint32_t vst = base + pf::kOffV + s * pf::kTile;
           const uint32_t pt = tmem + pf::kColS + (gj % pf::kSBufs) * pf::kKeys;  // P hi: 64 columns, then P lo
-#pragma unroll
-          for (int part = 0; part < kParts; ++part) {
+          for (int part = 0; part < parts; ++part) {
 #pragma unroll
             for (int kk = 0; kk < pf::kKeys / 16; ++kk) {
               const uint32_t bv = vst + kk * 16 * 128;  // 16 keys of 128-byte rows
@@ -530,7 +620,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
             x[c + 1] = fast_exp2(a.y);
             sm[(c >> 1) & 3] = __fadd2_rn(sm[(c >> 1) & 3], make_float2(x[c], x[c + 1]));
           }
-          if constexpr (kBf16) {
+          if (!f16p) {
             uint32_t hi[32], lo[32];
 #pragma unroll
             for (int c = 0; c < 32; ++c) split_hi_lo<T>(x[64 * h + 2 * c], x[64 * h + 2 * c + 1], hi[c], lo[c]);

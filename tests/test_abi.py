@@ -190,17 +190,76 @@ def test_append_and_decode_fp8_rejects_bad_arguments_before_launch(native, kw, c
     (dict(q=FAKE + 4), N.PKV_ERR_INVALID_ARG),
     (dict(qs=0), N.PKV_ERR_INVALID_ARG),
     (dict(T=-1), N.PKV_ERR_INVALID_ARG),
+    (dict(ws=FAKE + 16, ws_bytes=1 << 30), N.PKV_ERR_INVALID_ARG),  # the V staging area: 256-byte aligned
+    (dict(ws=FAKE, ws_bytes=4096), N.PKV_ERR_INVALID_ARG),          # and large enough
 ])
 def test_prefill_rejects_bad_arguments_before_launch(native, kw, code):
     a = dict(q=FAKE, k=FAKE, v=FAKE, t=FAKE, l=FAKE, qs=FAKE, B=2, T=64, maxq=32, hq=32, hkv=8, head_dim=128,
-             nb=64, maxb=8, block_size=16, scale=0.1, dtype=N.PKV_BF16, out=FAKE)
+             nb=64, maxb=8, block_size=16, scale=0.1, dtype=N.PKV_BF16, ws=None, ws_bytes=0, out=FAKE)
     a.update(kw)
     rc = native.pkv_paged_attention_prefill(a["q"], a["k"], a["v"], a["t"], a["l"], a["qs"], a["B"], a["T"],
                                             a["maxq"], a["hq"], a["hkv"], a["head_dim"], a["nb"], a["maxb"],
-                                            a["block_size"], a["scale"], a["dtype"], a["out"], None)
+                                            a["block_size"], a["scale"], a["dtype"], a["ws"], a["ws_bytes"], a["out"],
+                                            None)
     assert rc == code, native.pkv_last_error_string()
 
 
 def test_prefill_empty_batch_is_a_no_op(native):
     assert native.pkv_paged_attention_prefill(None, None, None, None, None, None, 0, 0, 0, 32, 8, 128, 64, 8, 16,
-                                              0.1, N.PKV_BF16, None, None) == 0
+                                              0.1, N.PKV_BF16, None, 0, None, None) == 0
+
+
+def test_prefill_workspace_size(native):
+    out = ctypes.c_size_t(0)
+    # bf16: a 256-byte record + [num_seqs][max_blocks][Hkv][block_size][128] f16
+    assert native.pkv_prefill_workspace_size(16, 8, 128, 256, 16, N.PKV_BF16, ctypes.byref(out)) == 0
+    assert out.value == 256 + 16 * 256 * 8 * 16 * 128 * 2
+    assert native.pkv_prefill_workspace_size(16, 8, 128, 256, 16, N.PKV_F16, ctypes.byref(out)) == 0
+    assert out.value == 0  # f16 pools need no staging
+    assert native.pkv_prefill_workspace_size(-1, 8, 128, 256, 16, N.PKV_BF16, ctypes.byref(out)) == N.PKV_ERR_INVALID_ARG
+
+
+def _pools(*specs):
+    """pkv_pool_t array from (num_blocks, block_size, max_blocks, num_seqs); fake pointers (never read)."""
+    arr = (N.pkv_pool_t * len(specs))()
+    for c, (nb, bs, maxb, n) in enumerate(specs):
+        arr[c] = N.pkv_pool_t(FAKE, FAKE, FAKE, nb, bs, maxb, n)
+    return arr
+
+
+def test_pools_workspace_size_matches_the_single_pool_layout(native):
+    out, ref = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    # 50 + 13 + 1 sequences; the largest capacity is 256 blocks of 16 = 512 blocks of 8 = 4096 tokens
+    pools = _pools((1000, 32, 32, 50), (2000, 16, 256, 13), (3000, 8, 512, 1))
+    assert native.pkv_decode_pools_workspace_size(pools, 3, 32, 8, 128, 0, ctypes.byref(out)) == 0
+    assert native.pkv_decode_workspace_size(64, 32, 8, 128, 256, 16, 0, ctypes.byref(ref)) == 0
+    assert out.value == ref.value
+
+
+@pytest.mark.parametrize("specs,kw,code", [
+    ((), {}, N.PKV_ERR_INVALID_ARG),                                                   # no pool
+    (((64, 16, 8, 1),) * 4, {}, N.PKV_ERR_INVALID_ARG),                               # four pools
+    (((64, 24, 8, 1),), {}, N.PKV_ERR_UNSUPPORTED),                                   # block size 24
+    (((64, 32, 8, 1),), dict(pt=48), N.PKV_ERR_INVALID_ARG),                         # 48 % 32 != 0
+    (((64, 16, 8, 1),), dict(pt=24), N.PKV_ERR_INVALID_ARG),                         # not a multiple of 16
+    (((64, 16, 8, 1),), dict(dtype=N.PKV_F32), N.PKV_ERR_UNSUPPORTED),               # tensor cores only
+    (((64, 16, 8, 1),), dict(hq=8, hkv=8), N.PKV_ERR_UNSUPPORTED),                   # one query head per KV head
+    (((64, 16, 8, 1),), dict(head_dim=64), N.PKV_ERR_UNSUPPORTED),
+    (((64, 16, 8, 1),), dict(ws_bytes=256), N.PKV_ERR_INVALID_ARG),                  # workspace too small
+    (((64, 16, 8, 1),), dict(q=FAKE + 8), N.PKV_ERR_INVALID_ARG),                    # misaligned q
+    (((64, 16, 8, -1),), {}, N.PKV_ERR_INVALID_ARG),                                  # negative count
+])
+def test_pools_call_rejects_bad_arguments_before_launch(native, specs, kw, code):
+    a = dict(q=FAKE, hq=32, hkv=8, head_dim=128, scale=0.1, dtype=N.PKV_BF16, pt=0, ws_bytes=1 << 30)
+    a.update(kw)
+    pools = _pools(*specs) if specs else None
+    rc = native.pkv_append_and_decode_pools(pools, len(specs), FAKE, FAKE, FAKE, a["q"], FAKE, a["hq"], a["hkv"],
+                                            a["head_dim"], a["scale"], a["dtype"], a["pt"], FAKE, a["ws_bytes"], FAKE,
+                                            None)
+    assert rc == code, native.pkv_last_error_string()
+
+
+def test_pools_call_with_no_sequences_is_a_no_op(native):
+    pools = _pools((64, 16, 8, 0), (64, 8, 8, 0))
+    assert native.pkv_append_and_decode_pools(pools, 2, None, None, None, None, None, 32, 8, 128, 0.1, N.PKV_BF16,
+                                              0, None, 0, None, None) == 0

@@ -72,12 +72,13 @@ class PrefillCase:
         return pa.paged_prefill_attention(raw(self.q), raw(self.k_pool), raw(self.v_pool), self.tables,
                                           np.array(self.lens), np.array(self.q_lens), self.scale, self.dtype)
 
-    def run(self, max_q_len=None, out=None):
+    def run(self, max_q_len=None, out=None, stage_v=True, workspace=None):
         dev = "cuda"
         res = pkv.pkv_paged_attention_prefill(
             self.q.to(dev), self.k_pool.to(dev), self.v_pool.to(dev), torch.from_numpy(self.tables).to(dev),
             torch.tensor(self.lens, dtype=torch.int32, device=dev), torch.from_numpy(self.q_start).to(dev),
-            max(self.q_lens) if max_q_len is None else max_q_len, self.scale, out=out)
+            max(self.q_lens) if max_q_len is None else max_q_len, self.scale, out=out, stage_v=stage_v,
+            workspace=workspace)
         torch.cuda.synchronize()
         return res
 
@@ -86,35 +87,62 @@ def _seed(*k):
     return zlib.crc32("-".join(map(str, k)).encode()) % 100000
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("dtype,stage_v", [("bf16", True), ("bf16", False), ("f16", True)])
 @pytest.mark.parametrize("g", [1, 2, 4, 8])
 @pytest.mark.parametrize("bs", [8, 16, 32])
-def test_prefill_matches_oracle(dtype, g, bs):
+def test_prefill_matches_oracle(dtype, stage_v, g, bs):
     """Whole prompts, chunks behind earlier context, ragged tiles and chunks,
-    lengths around the 128-key chunk edges."""
+    lengths around the 128-key chunk edges; bf16 pools both with V staged as
+    f16 (one f16 P·V pass) and without (P hi + lo over bf16 V)."""
     lens = [1, 130, 300, 129, 517, 64]
     q_lens = [1, 130, 77, 1, 45, 64]
     case = PrefillCase(lens, q_lens, 2 * g, 2, bs, dtype, _seed(dtype, g, bs))
-    out = case.run()
-    assert_close(out, case.oracle(), dtype, f"prefill {dtype} G{g} bs{bs}")
+    out = case.run(stage_v=stage_v)
+    assert_close(out, case.oracle(), dtype, f"prefill {dtype} G{g} bs{bs} stage_v={stage_v}")
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_bf16_v_beyond_f16_range_keeps_the_bf16_path():
+    """A V value above 65504 has no f16 counterpart: the staged call must fall
+    back to the two bf16 passes over the pool (bit for bit the unstaged
+    result), and the next call on the same workspace, with values in range,
+    must take the f16 pass again (its result then differs in the last bits
+    from the unstaged one) - both within tolerance of the oracle."""
+    lens, q_lens = [700, 300], [200, 300]
+    big = PrefillCase(lens, q_lens, 8, 2, 16, "bf16", _seed("range"))
+    t = big.tables[0, 1]
+    big.v_pool[t, 0, 3, 5] = 131072.0  # token 19 of sequence 0, KV head 0, dim 5
+    ws = torch.empty(pkv.pkv_prefill_workspace_size(2, 2, D, big.maxb, 16, torch.bfloat16), dtype=torch.uint8,
+                     device="cuda")
+    staged = big.run(workspace=ws)
+    plain = big.run(stage_v=False)
+    assert torch.equal(staged, plain), "an out-of-range V must keep the bf16 hi + lo path"
+    assert_close(staged, big.oracle(), "bf16", "V beyond the f16 range")
+    small = PrefillCase(lens, q_lens, 8, 2, 16, "bf16", _seed("range"))
+    staged = small.run(workspace=ws)
+    plain = small.run(stage_v=False)
+    assert not torch.equal(staged, plain), "values in range take the one-pass f16 P"
+    ref = small.oracle()
+    assert_close(staged, ref, "bf16", "staged after the fallback")
+    assert_close(plain, ref, "bf16", "unstaged")
+
+
+@pytest.mark.parametrize("dtype,stage_v", [("bf16", True), ("bf16", False), ("f16", True)])
 @pytest.mark.parametrize("g", [1, 4])
-def test_long_context_and_many_tiles(g, dtype):
-    """bf16 pools take P as hi + lo halves, f16 pools a single f16 P."""
+def test_long_context_and_many_tiles(g, dtype, stage_v):
+    """bf16 pools take P as hi + lo halves, or one f16 P over V staged as
+    f16; f16 pools a single f16 P."""
     lens, q_lens = [1500, 700], [300, 700]
     case = PrefillCase(lens, q_lens, 2 * g, 2, 16, dtype, _seed("long", g, dtype))
-    assert_close(case.run(), case.oracle(), dtype, f"long {dtype} G{g}")
+    assert_close(case.run(stage_v=stage_v), case.oracle(), dtype, f"long {dtype} G{g} stage_v={stage_v}")
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f16"])
-def test_growing_scores_rescale_the_accumulator(dtype):
+@pytest.mark.parametrize("dtype,stage_v", [("bf16", True), ("bf16", False), ("f16", True)])
+def test_growing_scores_rescale_the_accumulator(dtype, stage_v):
     """Scores rise along the sequence so the running max moves by more than
     the lazy threshold in many chunks: every such move rescales O."""
     case = PrefillCase([900, 400], [200, 400], 8, 2, 16, dtype, _seed("ramp", dtype), k_ramp=12.0)
     ref = case.oracle()
-    assert_close(case.run(), ref, dtype, f"rescaled {dtype}")
+    assert_close(case.run(stage_v=stage_v), ref, dtype, f"rescaled {dtype} stage_v={stage_v}")
 
 
 def test_one_row_chunks_agree_with_decode():
@@ -212,11 +240,13 @@ def test_unsupported_arguments_are_refused():
     assert e.value.code == -4
 
 
-def test_full_size_chunked_prefill_sampled_rows():
+@pytest.mark.parametrize("stage_v", [True, False])
+def test_full_size_chunked_prefill_sampled_rows(stage_v):
     """The measured chunked-prefill batch (16 sequences, 512-row chunks behind
     U[0, 3584] cached tokens, 32 / 8 heads, bf16, block size 16), launched as
-    the bench launches it; 48 sampled (row, head) outputs against the oracle,
-    each as the one-row chunk at its position."""
+    the bench launches it (V staged as f16), and without staging; in every
+    sequence, eight rows at and around the 128-row tile edges, every head,
+    against the oracle, each as the one-row chunk at its position."""
     from paged_kv_cache_406_b200 import workloads as W
     w = W.WORKLOADS["prefill_llama3_8b"]
     dev = "cuda"
@@ -233,21 +263,24 @@ def test_full_size_chunked_prefill_sampled_rows():
     tables, lens = alloc.block_tables(list(range(B)), maxb)
     q = W.normal((B * n, hq, d), w.torch_dtype, W.step_seed(w, 0, 0), device=dev)
     out = pkv.pkv_paged_attention_prefill(q, kp, vp, torch.from_numpy(tables).to(dev), torch.from_numpy(lens).to(dev),
-                                          torch.arange(0, B * n + 1, n, dtype=torch.int32, device=dev), n, w.scale)
+                                          torch.arange(0, B * n + 1, n, dtype=torch.int32, device=dev), n, w.scale,
+                                          stage_v=stage_v)
     torch.cuda.synchronize()
     kc, vc, qc = raw(kp), raw(vp), raw(q)
-    rng = np.random.default_rng(406)
+    out = out.cpu()
     G = hq // hkv
-    for _ in range(48):
-        b, i, h = int(rng.integers(B)), int(rng.integers(n)), int(rng.integers(hq))
-        pos = int(ctx[b]) + i
-        g = h // G
-        blocks = tables[b, :pos // bs + 1]
-        ref = pa.paged_prefill_attention(qc[b * n + i:b * n + i + 1, g * G:(g + 1) * G], kc[blocks][:, g:g + 1],
-                                         vc[blocks][:, g:g + 1], np.arange(len(blocks))[None], np.array([pos + 1]),
-                                         np.array([1]), w.scale, "bf16")
-        got = out[b * n + i, g * G:(g + 1) * G].unsqueeze(0)
-        assert_close(got, ref, "bf16", f"row {b}/{i} heads {g * G}..{g * G + G - 1}")
+    for b in range(B):
+        kb, vb = kc[tables[b, :-(-int(L[b]) // bs)]], vc[tables[b, :-(-int(L[b]) // bs)]]
+        for i in (0, 1, 31, 32, 127, 128, 300, n - 1):
+            pos = int(ctx[b]) + i
+            nblk = pos // bs + 1
+            for g in range(hkv):
+                ref = pa.paged_prefill_attention(qc[b * n + i:b * n + i + 1, g * G:(g + 1) * G],
+                                                 kb[:nblk, g:g + 1], vb[:nblk, g:g + 1],
+                                                 np.arange(nblk)[None], np.array([pos + 1]), np.array([1]),
+                                                 w.scale, "bf16")
+                got = out[b * n + i, g * G:(g + 1) * G].unsqueeze(0)
+                assert_close(got, ref, "bf16", f"row {b}/{i} heads {g * G}..{g * G + G - 1}")
 
 
 def test_repeated_concurrent_and_captured_calls():

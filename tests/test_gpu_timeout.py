@@ -1,0 +1,65 @@
+"""The decode kernels' bounded waits, made to run out on purpose (B200).
+
+Every wait of a decode consumer for a K/V chunk gives up after a limit,
+records PKV_ERR_DEVICE_TIMEOUT in the device status word and lets its CTA
+finish.  Here that path runs without any fault or hang: through
+pkv_debug_stall_decode the producer of CTA 0 skips the copies of its first
+work unit, so that unit's consumers wait for chunks that never arrive; with a
+1 ms limit they give up, the producer stops and, having issued no copy, exits
+at once.  The call must end promptly with the timeout recorded, and the next
+normal call on the same pools must match the oracle.
+"""
+import time
+
+import pytest
+import torch
+
+from helpers import Case, assert_close
+
+pytestmark = pytest.mark.gpu
+
+PKV_ERR_DEVICE_TIMEOUT = -6
+
+
+# bf16 with G = 4: the tensor-core kernel; f32 (G = 4) and f16 with G = 1: the CUDA-core kernel
+@pytest.mark.parametrize("dtype,g", [("bf16", 4), ("f32", 4), ("f16", 1)])
+def test_stalled_unit_times_out_and_next_call_is_correct(native, dtype, g):
+    import paged_kv_cache_406_b200 as P
+    # 4 sequences x 4 partitions of 512 tokens x 2 KV heads = 32 work units, one
+    # per CTA; a unit spans 32 chunks, more than any ring has stages, so the
+    # stalled producer issues no copy at all before it gives up
+    case = Case([2048] * 4, 2 * g, 2, 128, 16, dtype, seed=404 + g)
+    d = case.device()
+    args = (d["q"], d["k_pool"], d["v_pool"], d["block_tables"], d["seq_lens"], case.scale)
+    P.pkv_paged_attention_decode(*args)  # first launch: module load and tensor maps outside the timing
+    assert P.pkv_device_status(clear=True) == 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    P.pkv_debug_stall_decode(0, 1_000_000)
+    try:
+        t0 = time.perf_counter()
+        e0.record()
+        P.pkv_paged_attention_decode(*args)
+        e1.record()
+        status = P.pkv_device_status(clear=True)
+        wall = time.perf_counter() - t0
+    finally:
+        P.pkv_debug_stall_decode(-1, 0)
+    assert status == PKV_ERR_DEVICE_TIMEOUT
+    ms = e0.elapsed_time(e1)
+    # 1 ms of waiting, then every role leaves; nothing waits out the normal 1 s limit
+    assert ms < 200.0, f"the stalled call took {ms:.1f} ms on the device"
+    assert wall < 5.0
+    out = P.pkv_paged_attention_decode(*args)
+    assert P.pkv_device_status(clear=True) == 0
+    assert_close(out, case.oracle(), dtype, f"{dtype} G={g} after the timed-out call")
+
+
+def test_stall_setting_is_off_by_default(native):
+    import paged_kv_cache_406_b200 as P
+    case = Case([700, 1500], 8, 2, 128, 16, "bf16", seed=405)
+    d = case.device()
+    P.pkv_debug_stall_decode(-1, 0)
+    out = P.pkv_paged_attention_decode(d["q"], d["k_pool"], d["v_pool"], d["block_tables"], d["seq_lens"],
+                                       case.scale)
+    assert P.pkv_device_status(clear=True) == 0
+    assert_close(out, case.oracle(), "bf16", "stall off")
