@@ -500,19 +500,18 @@ int pkv_device_status(void* stream, int32_t* status, int32_t clear);
 
 /* Test support for the decode kernels' bounded waits (no counterpart in the
  * pages; failure detection).  Every wait of a decode consumer for a chunk of
- * K/V gives up after a limit, records PKV_ERR_DEVICE_TIMEOUT in the status
- * word and lets the CTA finish, so a stalled copy costs an error code instead
- * of a hung GPU.  This call makes that path run on demand: for the decode
- * launches that follow (pkv_paged_attention_decode, _fp8, _static and the
- * append-and-decode forms), the producer of CTA `cta` skips the copies of
- * that CTA's first work unit, so their consumers wait for chunks that never
- * arrive; `consumer_wait_ns` (0 = the normal 1 s) is how long a consumer
- * waits for a chunk before it gives up.  The producer still waits, with the
- * normal limit, for every copy it did issue before its CTA exits.  cta < 0
+ * K/V gives up after a limit (1 s), records PKV_ERR_DEVICE_TIMEOUT in the
+ * status word and lets the CTA finish, so a stalled copy costs an error code
+ * instead of a hung GPU.  This call makes that path run on demand: for the
+ * decode launches that follow (pkv_paged_attention_decode, _fp8, _static and
+ * the append-and-decode forms), the producer of CTA `cta` skips the copies
+ * of that CTA's first work unit, so their consumers wait for chunks that
+ * never arrive and give up after the limit; the producer still waits, with
+ * the same limit, for every copy it did issue before its CTA exits.  cta < 0
  * restores normal operation (the default).  Outputs of a stalled call are
- * unspecified; the pools are not written by decode.  Process-wide setting,
- * read at each launch; always returns PKV_OK. */
-int pkv_debug_stall_decode(int32_t cta, uint64_t consumer_wait_ns);
+ * unspecified; decode does not write the pools.  Process-wide setting, read
+ * at each launch; always returns PKV_OK. */
+int pkv_debug_stall_decode(int32_t cta);
 
 #ifdef __cplusplus
 }

@@ -161,6 +161,35 @@ def pkv_append_and_decode(k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping
     return out
 
 
+def bind_append_and_decode(k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: torch.Tensor, q: torch.Tensor,
+                           k_pool: torch.Tensor, v_pool: torch.Tensor, block_tables: torch.Tensor,
+                           seq_lens: torch.Tensor, scale: float, out: torch.Tensor, workspace: torch.Tensor,
+                           partition_tokens: int = 0):
+    """:func:`pkv_append_and_decode` checked and marshalled once for a fixed
+    set of buffers; returns a callable that issues the call again (on the
+    stream current at bind time) with no per-call Python work but the C call
+    and its status check.  The buffers must stay alive and keep their shapes;
+    their contents may change between calls (a serving loop that stages each
+    step's rows and metadata into the same tensors)."""
+    nb, hkv, bs, d = _pool_dims(_cuda(k_pool, "k_pool"), _cuda(v_pool, "v_pool"))
+    n = _new_rows(k_new, v_new, slot_mapping, hkv, d, k_pool.dtype)
+    _cuda(q, "q", k_pool.dtype)
+    B, hq, maxb, out, workspace = _decode_io(q, hkv, d, bs, block_tables, seq_lens, out, workspace, partition_tokens)
+    fn = lib().pkv_append_and_decode
+    args = (k_new.data_ptr(), v_new.data_ptr(), slot_mapping.data_ptr(), n, q.data_ptr(), k_pool.data_ptr(),
+            v_pool.data_ptr(), block_tables.data_ptr(), seq_lens.data_ptr(), B, hq, hkv, d, nb, maxb, bs, float(scale),
+            _dtype_code(k_pool), partition_tokens, workspace.data_ptr(), workspace.numel(), out.data_ptr(), _stream())
+    keep = (k_new, v_new, slot_mapping, q, k_pool, v_pool, block_tables, seq_lens, out, workspace)
+
+    def call():
+        rc = fn(*args)
+        if rc:
+            check(rc)
+        return keep[8]
+
+    return call
+
+
 def pkv_prefill_workspace_size(num_seqs: int, num_kv_heads: int, head_dim: int, max_blocks_per_seq: int,
                                block_size: int, dtype: torch.dtype) -> int:
     """Bytes of the prefill workspace (the f16 copy of V for bf16 pools; 0
@@ -390,12 +419,12 @@ def pkv_device_status(clear: bool = True) -> int:
     return st.value
 
 
-def pkv_debug_stall_decode(cta: int = -1, consumer_wait_ns: int = 0) -> None:
+def pkv_debug_stall_decode(cta: int = -1) -> None:
     """Test support for the bounded waits: the decode launches that follow
-    leave CTA ``cta``'s first work unit without copies, and consumers give up
-    a wait after ``consumer_wait_ns`` (0: the normal limit); ``cta < 0``
-    restores normal operation."""
-    check(lib().pkv_debug_stall_decode(int(cta), int(consumer_wait_ns)))
+    leave CTA ``cta``'s first work unit without copies, so its consumers'
+    waits run out (after the normal limit); ``cta < 0`` restores normal
+    operation."""
+    check(lib().pkv_debug_stall_decode(int(cta)))
 
 
 # ----------------------------------------------------------------------------
@@ -495,6 +524,6 @@ class Allocator:
 __all__ = ["Allocator", "PagedKVError", "pkv_kv_append", "pkv_copy_blocks", "pkv_decode_workspace_size",
            "pkv_paged_attention_decode", "pkv_paged_attention_decode_static", "pkv_device_status",
            "pkv_debug_stall_decode", "pkv_paged_attention_prefill", "pkv_prefill_workspace_size",
-           "pkv_append_and_decode_pools", "pkv_decode_pools_workspace_size",
+           "pkv_append_and_decode_pools", "pkv_decode_pools_workspace_size", "bind_append_and_decode",
            "pkv_kv_append_fp8", "pkv_paged_attention_decode_fp8", "pkv_append_and_decode",
            "pkv_append_and_decode_fp8"]

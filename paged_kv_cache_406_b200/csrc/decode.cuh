@@ -67,10 +67,8 @@ struct DecodeParams {
   float* out;
   // Test support for the bounded waits (pkv_debug_stall_decode): the
   // producer of CTA `stall_cta` skips the copies of that CTA's first work
-  // unit (its consumers' waits then run out), and consumers give up a wait
-  // for a chunk after `consumer_wait_ns`.  stall_cta < 0 in normal calls.
+  // unit, so its consumers' waits run out.  stall_cta < 0 in normal calls.
   int32_t stall_cta;
-  uint64_t consumer_wait_ns;
 };
 
 // Pool of sequence b (0 for single-pool batches).
@@ -476,7 +474,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
     int s = (c + j0) % NS;
     uint32_t ph = ((c + j0) / NS) & 1;
     for (int j = j0; j < u.nblk && ok; j += kConsumerWarps) {
-      const bool landed = __all_sync(kFull, mbar_wait(smem_addr(full + s), ph, abort_flag, p.consumer_wait_ns));
+      const bool landed = __all_sync(kFull, mbar_wait(smem_addr(full + s), ph, abort_flag));
       if (!landed) {
         if (lane == 0) {
           record_error(PKV_ERR_DEVICE_TIMEOUT);

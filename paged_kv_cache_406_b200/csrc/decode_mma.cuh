@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0) decode_mma
     int s = (c + k0) % NS;
     uint32_t ph = ((c + k0) / NS) & 1;
     for (int k = k0; k < nch && ok; k += kConsumerWarps) {
-      const bool landed = __all_sync(kFull, mbar_wait(smem_addr(full + s), ph, abort_flag, p.consumer_wait_ns));
+      const bool landed = __all_sync(kFull, mbar_wait(smem_addr(full + s), ph, abort_flag));
       if (!landed) {
         if (lane == 0) {
           record_error(PKV_ERR_DEVICE_TIMEOUT);

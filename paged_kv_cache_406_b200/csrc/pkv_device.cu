@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include <cuda_fp8.h>
 #include <nvtx3/nvToolsExt.h>
@@ -136,14 +137,10 @@ struct PendingAppend {
 };
 
 // Test support for the decode kernels' bounded waits (pkv_debug_stall_decode):
-// a CTA whose first work unit gets no copies, and the consumers' wait limit.
+// a CTA whose first work unit gets no copies.
 std::atomic<int> g_stall_cta{-1};
-std::atomic<uint64_t> g_consumer_wait_ns{pkv::kWaitLimitNs};
 
-void apply_debug(pkv::DecodeParams& p) {
-  p.stall_cta = g_stall_cta.load(std::memory_order_relaxed);
-  p.consumer_wait_ns = g_consumer_wait_ns.load(std::memory_order_relaxed);
-}
+void apply_debug(pkv::DecodeParams& p) { p.stall_cta = g_stall_cta.load(std::memory_order_relaxed); }
 
 // The one pool of a single-pool batch.
 void set_single_pool(pkv::DecodeParams& p, const void* k_pool, const void* v_pool, const int32_t* block_tables,
@@ -601,9 +598,8 @@ extern "C" int pkv_append_and_decode(const void* k_new, const void* v_new, const
                    workspace_bytes, out, n_tokens > 0 ? &ap : nullptr, stream);
 }
 
-extern "C" int pkv_debug_stall_decode(int32_t cta, uint64_t consumer_wait_ns) {
+extern "C" int pkv_debug_stall_decode(int32_t cta) {
   g_stall_cta.store(cta < 0 ? -1 : cta, std::memory_order_relaxed);
-  g_consumer_wait_ns.store(consumer_wait_ns == 0 ? pkv::kWaitLimitNs : consumer_wait_ns, std::memory_order_relaxed);
   return pkv::ok();
 }
 
@@ -1054,19 +1050,36 @@ size_t prefill_stage_bytes(int64_t num_seqs, int64_t num_kv_heads, int64_t max_b
   return 256 + round256(size_t(num_seqs * max_blocks * num_kv_heads * block_size) * 128 * sizeof(__half));
 }
 
+// One launch of the persistent prefill kernel instance <T, G, kF16P>: one
+// CTA per SM, its own tile-counter slot.
+template <typename T, int G, bool kF16P>
+int launch_prefill_instance(const pkv::PrefillParams& p, const CUtensorMap& mq, const CUtensorMap& mk,
+                            const CUtensorMap& mv, int dev, cudaStream_t stream) {
+  auto kern = pkv::prefill_tc_kernel<T, G, kF16P>;
+  static std::atomic<bool> configured[kMaxDevices];
+  if (dev >= kMaxDevices || !configured[dev].load(std::memory_order_relaxed)) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(pkv::pf::kSmemBytes));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill)");
+    if (dev < kMaxDevices) configured[dev].store(true, std::memory_order_relaxed);
+  }
+  const int64_t tiles = int64_t(p.n_tiles) * p.num_seqs * p.num_kv_heads;
+  const int64_t grid = std::min<int64_t>(sm_count(dev), tiles);  // persistent: one CTA per SM
+  unsigned int* ctr = nullptr;
+  int rc = prefill_counter(&ctr);
+  if (rc) return rc;
+  kern<<<static_cast<unsigned>(grid), pkv::pf::kThreads, pkv::pf::kSmemBytes, stream>>>(p, mq, mk, mv, ctr);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
+  return PKV_OK;
+}
+
 template <typename T, int G>
 int launch_prefill(const pkv::PrefillParams& p, const void* q, const void* k_pool, const void* v_pool, int dtype,
                    void* v_stage, cudaStream_t stream) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  auto kern = pkv::prefill_tc_kernel<T, G>;
-  static std::atomic<bool> configured[kMaxDevices];
-  if (dev >= kMaxDevices || !configured[dev].load(std::memory_order_relaxed)) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(pkv::pf::kSmemBytes));
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill)");
-    if (dev < kMaxDevices) configured[dev].store(true, std::memory_order_relaxed);
-  }
   CUtensorMap mq, mk, mv;
   int rc = make_prefill_q_map(&mq, q, dtype, p.num_q_tokens, p.num_q_heads, G);
   if (rc) return rc;
@@ -1105,14 +1118,17 @@ int launch_prefill(const pkv::PrefillParams& p, const void* q, const void* k_poo
     const int nx = std::max(1, std::min(p.max_blocks, (8 * sm_count(dev) + ny - 1) / ny));
     pkv::stage_v_f16_kernel<<<dim3(nx, ny), 256, 0, stream>>>(a);
   }
-  const int64_t tiles = int64_t(p.n_tiles) * p.num_seqs * p.num_kv_heads;
-  const int64_t grid = std::min<int64_t>(sm_count(dev), tiles);  // persistent: one CTA per SM
-  unsigned int* ctr = nullptr;
-  rc = prefill_counter(&ctr);
+  if constexpr (std::is_same<T, __half>::value) {
+    rc = launch_prefill_instance<__half, G, true>(pp, mq, mk, mv, dev, stream);
+  } else if (v_stage) {
+    // the bf16 instance runs only if the staging found a value beyond the
+    // f16 range, the f16 one only if it did not; the other returns at once
+    rc = launch_prefill_instance<__nv_bfloat16, G, false>(pp, mq, mk, mv, dev, stream);
+    if (!rc) rc = launch_prefill_instance<__nv_bfloat16, G, true>(pp, mq, mk, mvs, dev, stream);
+  } else {
+    rc = launch_prefill_instance<__nv_bfloat16, G, false>(pp, mq, mk, mv, dev, stream);
+  }
   if (rc) return rc;
-  kern<<<static_cast<unsigned>(grid), pkv::pf::kThreads, pkv::pf::kSmemBytes, stream>>>(pp, mq, mk, mv, mvs, ctr);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
   return pkv::ok();
 }
 

@@ -69,9 +69,9 @@ struct PrefillParams {
   int32_t num_q_tokens, max_q_len, n_tiles;
   float scale_log2;  // scale · log2(e), positive
   // bf16 pools with a staged f16 copy of V (v_staged != 0): P·V runs as one
-  // f16 pass over the copy (tmap_vs), unless the staging recorded a value
-  // beyond the f16 range (*v_range == epoch), in which case it runs as the
-  // two bf16 passes (P hi and lo) over the pool's V
+  // f16 pass over the copy, unless the staging recorded a value beyond the
+  // f16 range (*v_range == epoch), in which case it runs as the two bf16
+  // passes (P hi and lo) over the pool's V (two launches, see the kernel)
   int32_t v_staged;
   uint32_t epoch;
   const uint32_t* v_range;
@@ -265,20 +265,27 @@ __global__ void __launch_bounds__(256) stage_v_f16_kernel(const VStageArgs a) {
   if (__any_sync(0xffffffffu, over) && (threadIdx.x & 31) == 0) atomicExch(a.range, a.epoch);
 }
 
-template <typename T, int G>
+// kF16P: one f16 P and one P·V pass over f16 V (the pool's own for f16 pools,
+// the staged copy for bf16 pools); otherwise (bf16 only) P as bf16 hi + lo
+// halves, two passes over the pool's bf16 V.  A bf16 call with staged V
+// launches both instances: each reads the staging record first and the one
+// whose case does not hold returns at once (the record says whether some V
+// value lay beyond the f16 range), so each instance carries one P path only.
+template <typename T, int G, bool kF16P>
 __global__ void __launch_bounds__(pf::kThreads, 1)
     prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_q,
                       const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
-                      const __grid_constant__ CUtensorMap tmap_vs, unsigned int* __restrict__ tile_ctr) {
+                      unsigned int* __restrict__ tile_ctr) {
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
   constexpr int QT = pf::kRows / G;  // query tokens per tile
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
-  // One f16 P and one P·V pass (f16 pools, or bf16 pools whose V was staged
-  // as f16 within range), else P as bf16 hi + lo halves and two passes.
-  // Uniform over the launch: every thread reads the same staging record.
-  bool f16p = !kBf16;
-  if constexpr (kBf16) f16p = p.v_staged != 0 && *p.v_range != p.epoch;
-  const bool v_from_stage = kBf16 && f16p;
+  static_assert(kBf16 || kF16P, "f16 pools take the one-pass f16 P");
+  constexpr bool f16p = kF16P;
+  if (kBf16 && p.v_staged) {
+    const bool beyond = *p.v_range == p.epoch;
+    if (beyond == kF16P) return;  // the other instance of this call does the work
+  }
+  constexpr bool v_from_stage = kBf16 && kF16P;  // tmap_v then maps the staged f16 copy
 
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -416,8 +423,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       const uint32_t full0 = bar(kv ? pf::kVFull : pf::kKFull), empty0 = bar(kv ? pf::kVEmpty : pf::kKEmpty);
       // V from the staged f16 copy: block j of sequence b sits at b * max_blocks + j, no table lookup
       const bool staged = kv && v_from_stage;
-      const void* map = kv ? (staged ? static_cast<const void*>(&tmap_vs) : static_cast<const void*>(&tmap_v))
-                           : static_cast<const void*>(&tmap_k);
+      const void* map = kv ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k);
       const uint32_t ring = base + (kv ? pf::kOffV : pf::kOffK);
       for (int j = 0; j < nc && ok; ++j) {
         const int s = (gc + j) % pf::kStages;
@@ -472,7 +478,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     const uint32_t id_s = tc::idesc_f16(kBf16, false, pf::kRows, pf::kKeys);
     // P·V: f16 P and f16 V in one pass, or bf16 P hi and lo over bf16 V
     const uint32_t id_o = tc::idesc_f16(kBf16 && !f16p, true, pf::kRows, pf::kHeadDim);
-    const int parts = f16p ? 1 : 2;
+    constexpr int parts = f16p ? 1 : 2;
     bool ok = true;
     int gc = 0, tv = 0;
     for (int ti = 0; ok; ++ti) {
@@ -512,6 +518,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
           tc::fence_after_sync();
           const uint32_t vst = base + pf::kOffV + s * pf::kTile;
           const uint32_t pt = tmem + pf::kColS + (gj % pf::kSBufs) * pf::kKeys;  // P hi: 64 columns, then P lo
+#pragma unroll
           for (int part = 0; part < parts; ++part) {
 #pragma unroll
             for (int kk = 0; kk < pf::kKeys / 16; ++kk) {
@@ -620,7 +627,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
             x[c + 1] = fast_exp2(a.y);
             sm[(c >> 1) & 3] = __fadd2_rn(sm[(c >> 1) & 3], make_float2(x[c], x[c + 1]));
           }
-          if (!f16p) {
+          if constexpr (!f16p) {
             uint32_t hi[32], lo[32];
 #pragma unroll
             for (int c = 0; c < 32; ++c) split_hi_lo<T>(x[64 * h + 2 * c], x[64 * h + 2 * c + 1], hi[c], lo[c]);

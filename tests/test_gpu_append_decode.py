@@ -162,3 +162,30 @@ def test_append_and_decode_fp8_matches_oracle_and_two_calls(g, bs):
     assert torch.equal(fk, tk) and torch.equal(fv, tv)
     assert torch.equal(out, two)
     assert_close(out, ref, "f16", f"append+decode e4m3 G{g} bs{bs}")
+
+
+def test_bound_call_equals_the_plain_call():
+    """bind_append_and_decode: the call checked and marshalled once, issued
+    twice, gives the plain call's pools and outputs bit for bit."""
+    case = Case([5, 300, 1030, 2049], 8, 2, 128, 16, "bf16", seed=71)
+    slots, tables, lens = _grow(case)
+    rng = np.random.default_rng(72)
+    kn, vn = randn((case.B, 2, 128), "bf16", rng), randn((case.B, 2, 128), "bf16", rng)
+    dev = "cuda"
+    args = dict(k_new=kn.to(dev), v_new=vn.to(dev), slot_mapping=torch.from_numpy(slots).to(dev), q=case.q.to(dev),
+                block_tables=torch.from_numpy(tables).to(dev), seq_lens=torch.from_numpy(lens.astype(np.int32)).to(dev))
+    kp1, vp1 = case.k_pool.to(dev), case.v_pool.to(dev)
+    kp2, vp2 = kp1.clone(), vp1.clone()
+    want = pkv.pkv_append_and_decode(args["k_new"], args["v_new"], args["slot_mapping"], args["q"], kp1, vp1,
+                                     args["block_tables"], args["seq_lens"], case.scale)
+    ws = torch.empty(pkv.pkv_decode_workspace_size(case.B, 8, 2, 128, tables.shape[1], 16, 0), dtype=torch.uint8,
+                     device=dev)
+    out = torch.full_like(want, float("nan"))
+    call = pkv.bind_append_and_decode(args["k_new"], args["v_new"], args["slot_mapping"], args["q"], kp2, vp2,
+                                      args["block_tables"], args["seq_lens"], case.scale, out, ws)
+    for _ in range(2):
+        got = call()
+        torch.cuda.synchronize()
+        assert got is out
+        assert torch.equal(out, want)
+    assert torch.equal(kp1, kp2) and torch.equal(vp1, vp2)

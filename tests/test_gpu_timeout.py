@@ -1,13 +1,14 @@
 """The decode kernels' bounded waits, made to run out on purpose (B200).
 
-Every wait of a decode consumer for a K/V chunk gives up after a limit,
+Every wait of a decode consumer for a K/V chunk gives up after a limit (1 s),
 records PKV_ERR_DEVICE_TIMEOUT in the device status word and lets its CTA
 finish.  Here that path runs without any fault or hang: through
 pkv_debug_stall_decode the producer of CTA 0 skips the copies of its first
-work unit, so that unit's consumers wait for chunks that never arrive; with a
-1 ms limit they give up, the producer stops and, having issued no copy, exits
-at once.  The call must end promptly with the timeout recorded, and the next
-normal call on the same pools must match the oracle.
+work unit, so that unit's consumers wait for chunks that never arrive; they
+give up after the limit, the producer stops and, having issued no copy,
+exits at once.  The call must end within the limit plus a margin, with the
+timeout recorded, and the next normal call on the same pools must match the
+oracle.
 """
 import time
 
@@ -34,7 +35,7 @@ def test_stalled_unit_times_out_and_next_call_is_correct(native, dtype, g):
     P.pkv_paged_attention_decode(*args)  # first launch: module load and tensor maps outside the timing
     assert P.pkv_device_status(clear=True) == 0
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    P.pkv_debug_stall_decode(0, 1_000_000)
+    P.pkv_debug_stall_decode(0)
     try:
         t0 = time.perf_counter()
         e0.record()
@@ -43,12 +44,13 @@ def test_stalled_unit_times_out_and_next_call_is_correct(native, dtype, g):
         status = P.pkv_device_status(clear=True)
         wall = time.perf_counter() - t0
     finally:
-        P.pkv_debug_stall_decode(-1, 0)
+        P.pkv_debug_stall_decode(-1)
     assert status == PKV_ERR_DEVICE_TIMEOUT
     ms = e0.elapsed_time(e1)
-    # 1 ms of waiting, then every role leaves; nothing waits out the normal 1 s limit
-    assert ms < 200.0, f"the stalled call took {ms:.1f} ms on the device"
-    assert wall < 5.0
+    # one wait limit (1 s) for the stalled consumers, then every role leaves;
+    # no second limit is waited out (the producer issued no copy to drain)
+    assert 900.0 < ms < 1600.0, f"the stalled call took {ms:.1f} ms on the device"
+    assert wall < 10.0
     out = P.pkv_paged_attention_decode(*args)
     assert P.pkv_device_status(clear=True) == 0
     assert_close(out, case.oracle(), dtype, f"{dtype} G={g} after the timed-out call")
@@ -58,7 +60,7 @@ def test_stall_setting_is_off_by_default(native):
     import paged_kv_cache_406_b200 as P
     case = Case([700, 1500], 8, 2, 128, 16, "bf16", seed=405)
     d = case.device()
-    P.pkv_debug_stall_decode(-1, 0)
+    P.pkv_debug_stall_decode(-1)
     out = P.pkv_paged_attention_decode(d["q"], d["k_pool"], d["v_pool"], d["block_tables"], d["seq_lens"],
                                        case.scale)
     assert P.pkv_device_status(clear=True) == 0
