@@ -277,25 +277,25 @@ __device__ __forceinline__ WorkUnit load_unit(const DecodeParams& p, int w) {
   return u;
 }
 
-// Final merge of one work unit: the kConsumerWarps per-warp records in `rec`
+// Final merge of one work unit: the kCW per-warp records in `rec`
 // (acc[G][D], m[G], l[G] each, taken against each warp's own running max)
 // are rescaled to their common max and either normalised into `out` (the
 // sequence has one partition) or stored as the partition's (m, l, o) partial
-// for merge_kernel.  Called by the consumer threads (0 .. kConsumerWarps*32-1)
+// for merge_kernel.  Called by the consumer threads (0 .. kCW*32-1)
 // after the named barrier that publishes the records.
-template <int G, int D>
+template <int G, int D, int kCW = kConsumerWarps>
 __device__ __forceinline__ void merge_store(const float* rec, const WorkUnit& u, const DecodeParams& p) {
   constexpr int kMF = G * D + 2 * G;
   const bool single = u.nparts == 1;
-  for (int idx = threadIdx.x; idx < G * D; idx += kConsumerWarps * 32) {
+  for (int idx = threadIdx.x; idx < G * D; idx += kCW * 32) {
     const int h = idx / D, d = idx - h * D;
     float M = -INFINITY;
 #pragma unroll
-    for (int w2 = 0; w2 < kConsumerWarps; ++w2) M = fmaxf(M, rec[w2 * kMF + G * D + h]);
+    for (int w2 = 0; w2 < kCW; ++w2) M = fmaxf(M, rec[w2 * kMF + G * D + h]);
     float num = 0.f, den = 0.f;
     if (M != -INFINITY) {
 #pragma unroll
-      for (int w2 = 0; w2 < kConsumerWarps; ++w2) {
+      for (int w2 = 0; w2 < kCW; ++w2) {
         const float f = fast_exp2(rec[w2 * kMF + G * D + h] - M);
         num += f * rec[w2 * kMF + h * D + d];
         den += f * rec[w2 * kMF + G * D + G + h];
@@ -328,7 +328,9 @@ struct DecodeSmem {
   }
 };
 
-template <typename T, int D, int G>
+// kStall: the instance that honours DecodeParams::stall_cta (the test of the
+// bounded waits); production launches use the instance without the check.
+template <typename T, int D, int G, bool kStall = false>
 __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr int kVec = Elem<T>::kVec;       // elements per 16-byte chunk
@@ -377,7 +379,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
     uint32_t ph = 0, issued = 0, skipped = 0;  // stage uses so far; the first `skipped` of them issued no copy
     bool ok = true;
     for (int r = 0, w = unit_index(0); w < n_work && ok; w = unit_index(++r)) {
-      const bool stall = r == 0 && p.stall_cta == static_cast<int>(blockIdx.x);
+      const bool stall = kStall && r == 0 && p.stall_cta == static_cast<int>(blockIdx.x);
       const WorkUnit u = load_unit(p, w);
       const int32_t* trow = p.pool[0].tables + static_cast<int64_t>(u.b) * p.pool[0].max_blocks + u.t0 / BS;
       for (int jb = 0; jb < u.nblk && ok; jb += 32) {

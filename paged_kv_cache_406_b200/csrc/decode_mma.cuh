@@ -37,6 +37,7 @@ constexpr int kChunkTokens = 16;
 constexpr int kMmaProducers = 2;
 constexpr int kMmaThreads = (kConsumerWarps + kMmaProducers) * 32;
 
+
 // kKVBytes = bytes per stored K/V element: 2 (bf16 / f16) or 1 (e4m3).
 template <int D, int kKVBytes = 2>
 struct MmaLayout {
@@ -50,22 +51,27 @@ struct MmaLayout {
 template <typename T, int D, int G, int kKVBytes = 2>
 struct MmaSmem {
   using L = MmaLayout<D, kKVBytes>;
+  static constexpr int kCW = kConsumerWarps;
+  static constexpr int kThreads = kMmaThreads;
   static constexpr int kMergeFloats = G * D + 2 * G;
   __host__ __device__ static size_t ring_bytes(int ns) {
     return size_t(ns) * L::kStageBytes;
   }
   __host__ __device__ static size_t bytes(int ns) {
     // + 1024: the dynamic shared memory base is aligned up to the 1024-byte swizzle atom
-    return 1024 + ring_bytes(ns) + 2 * kConsumerWarps * kMergeFloats * sizeof(float) + 2 * ns * sizeof(uint64_t) +
-           16 + kMmaProducers * 128;
+    return 1024 + ring_bytes(ns) + 2 * kCW * kMergeFloats * sizeof(float) + 2 * ns * sizeof(uint64_t) + 16 +
+           kMmaProducers * 128;
   }
 };
 
-// Two e4m3 codes (low byte first) widened exactly to a packed f16 pair.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t codes) {
-  uint32_t r;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(codes));
-  return r;
+// Four e4m3 codes (one word, code i in byte i) widened exactly to two packed
+// f16 pairs: codes 0, 1 into lo and codes 2, 3 into hi.  The word is split
+// into its 16-bit halves by a register-pair move rather than a shift (one
+// ALU instruction fewer per pair: the e4m3 kernel is bound by its ALU pipe).
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %2;\n cvt.rn.f16x2.e4m3x2 %0, l;\n cvt.rn.f16x2.e4m3x2 %1, h;\n}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
 }
 
 // A chunk tile in shared memory is built from TMA boxes of `br` rows (br = 16,
@@ -102,13 +108,16 @@ __device__ __forceinline__ int br_shift_of(int bs) { return bs == 8 ? 3 : 4; }
 
 // kMulti: the batch spans up to kMaxPools pools of different block sizes
 // (each work unit reads its sequence's pool); otherwise pool 0 only.
-template <typename T, int D, int G, int kKVBytes = 2, bool kMulti = false>
-__global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0) decode_mma_kernel(const DecodeParams p,
-                                                                    const __grid_constant__ PoolMaps maps) {
+// kStall: the instance that honours DecodeParams::stall_cta (the test of the
+// bounded waits); production launches use the instance without the check.
+template <typename T, int D, int G, int kKVBytes = 2, bool kMulti = false, bool kStall = false>
+__global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0)
+    decode_mma_kernel(const DecodeParams p, const __grid_constant__ PoolMaps maps) {
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
   static_assert(kKVBytes == 2 || (kKVBytes == 1 && D == 128), "e4m3 pools need head_dim 128");
   using L = MmaLayout<D, kKVBytes>;
   constexpr bool kFp8 = kKVBytes == 1;
+  constexpr int kCW = kConsumerWarps;
   constexpr int kSteps = D / 16;  // k-steps of q·Kᵀ and m-tiles of P·V
   constexpr int kHalves = L::kHalves;
   constexpr int kMF = MmaSmem<T, D, G, kKVBytes>::kMergeFloats;
@@ -117,7 +126,7 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0) decode_mma
 
   const int NS = p.n_stages;
   float* merge = reinterpret_cast<float*>(smem + MmaSmem<T, D, G, kKVBytes>::ring_bytes(NS));
-  uint64_t* full = reinterpret_cast<uint64_t*>(merge + 2 * kConsumerWarps * kMF);
+  uint64_t* full = reinterpret_cast<uint64_t*>(merge + 2 * kCW * kMF);
   uint64_t* empty = full + NS;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + NS);
   int32_t* tab = reinterpret_cast<int32_t*>(empty + NS) + 4;  // 32 block-table entries per producer
@@ -138,13 +147,13 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0) decode_mma
 
   const int n_work = *p.n_items * p.num_kv_heads;
 
-  if (warp >= kConsumerWarps) {
+  if (warp >= kCW) {
     // ----------------------------- producers -----------------------------
     // Both producer warps walk every unit and refill their own 32-entry
     // block-table window; lane 0 of producer pr alone issues the window's
     // chunks of parity pr, so the per-chunk path has no warp-wide
     // synchronisation.
-    const int pr = warp - kConsumerWarps;
+    const int pr = warp - kCW;
     int32_t* mytab = tab + 32 * pr;
     if (lane < (kMulti ? p.n_pools : 1)) {
       prefetch_tensormap(&maps.k[lane]);
@@ -157,7 +166,7 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0) decode_mma
     uint32_t cg = 0;      // CTA-wide chunk index of the unit's first chunk
     bool ok = true;
     for (int r = 0, w = unit_index(0); w < n_work && ok; w = unit_index(++r)) {
-      const bool stall = r == 0 && p.stall_cta == static_cast<int>(blockIdx.x);
+      const bool stall = kStall && r == 0 && p.stall_cta == static_cast<int>(blockIdx.x);
       const WorkUnit u = load_unit<kMulti>(p, w);
       const PoolView pv = kMulti ? pick3(p.pool, u.c) : p.pool[0];
       const int BS = pv.block_size, bs_shift = bs_shift_of(BS), br_shift = br_shift_of(BS);
@@ -276,10 +285,10 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0) decode_mma
     for (int mt = 0; mt < kSteps; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // heads 2tq, 2tq+1
 
-    const int k0 = (warp - static_cast<int>(c % kConsumerWarps) + kConsumerWarps) % kConsumerWarps;
+    const int k0 = (warp - static_cast<int>(c % kCW) + kCW) % kCW;
     int s = (c + k0) % NS;
     uint32_t ph = ((c + k0) / NS) & 1;
-    for (int k = k0; k < nch && ok; k += kConsumerWarps) {
+    for (int k = k0; k < nch && ok; k += kCW) {
       const bool landed = __all_sync(kFull, mbar_wait(smem_addr(full + s), ph, abort_flag));
       if (!landed) {
         if (lane == 0) {
@@ -323,10 +332,8 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0) decode_mma
           // contraction order within the step: K dims 16ks + 4tq + {0,1 | 2,3}
           // stand at fragment columns {2tq, 2tq+1 | 2tq+8, 2tq+9}
           uint32_t a[4];
-          a[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(kw[ks][0]));
-          a[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(kw[ks][0] >> 16));
-          a[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(kw[ks][1]));
-          a[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(kw[ks][1] >> 16));
+          e4m3x4_to_f16x2x2(kw[ks][0], a[0], a[2]);
+          e4m3x4_to_f16x2x2(kw[ks][1], a[1], a[3]);
           mma_16816<T>(sc, a, qb[ks][0], qb[ks][1]);
         }
       } else {
@@ -386,22 +393,20 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0) decode_mma
         // the sequence end read as zero codes. ----
 #pragma unroll
         for (int pp = 0; pp < D / 32; ++pp) {
-          uint32_t w[4];
+          uint32_t w[4] = {vw[pp][0], vw[pp][1], vw[pp][2], vw[pp][3]};
+          if (nv < kChunkTokens) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) w[i] = (2 * tq + (i & 1) + (i >> 1) * 8) < nv ? vw[pp][i] : 0u;
+            for (int i = 0; i < 4; ++i) w[i] = (2 * tq + (i & 1) + (i >> 1) * 8) < nv ? w[i] : 0u;
+          }
           const uint32_t x01a = __byte_perm(w[0], w[1], 0x5140), x01b = __byte_perm(w[0], w[1], 0x7362);
           const uint32_t x89a = __byte_perm(w[2], w[3], 0x5140), x89b = __byte_perm(w[2], w[3], 0x7362);
           uint32_t a[4];
-          a[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(x01a));
-          a[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(x01a >> 16));
-          a[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(x89a));
-          a[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(x89a >> 16));
+          e4m3x4_to_f16x2x2(x01a, a[0], a[1]);
+          e4m3x4_to_f16x2x2(x89a, a[2], a[3]);
           mma_16816<T>(acc[2 * pp], a, bh0, bh1);
           mma_16816<T>(acc[2 * pp], a, bl0, bl1);
-          a[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(x01b));
-          a[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(x01b >> 16));
-          a[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(x89b));
-          a[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(x89b >> 16));
+          e4m3x4_to_f16x2x2(x01b, a[0], a[1]);
+          e4m3x4_to_f16x2x2(x89b, a[2], a[3]);
           mma_16816<T>(acc[2 * pp + 1], a, bh0, bh1);
           mma_16816<T>(acc[2 * pp + 1], a, bl0, bl1);
         }
@@ -430,7 +435,7 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0) decode_mma
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_addr(empty + s));
       }
-      s += kConsumerWarps;
+      s += kCW;
       if (s >= NS) {
         s -= NS;
         ph ^= 1;
@@ -444,7 +449,7 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0) decode_mma
       l0 += __shfl_xor_sync(kFull, l0, o);
       l1 += __shfl_xor_sync(kFull, l1, o);
     }
-    float* mb = merge + ((iter & 1) * kConsumerWarps + warp) * kMF;
+    float* mb = merge + ((iter & 1) * kCW + warp) * kMF;
     const int h0 = 2 * tq, h1 = 2 * tq + 1;
 #pragma unroll
     for (int mt = 0; mt < kSteps; ++mt) {
@@ -470,8 +475,8 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0) decode_mma
         mb[G * D + G + h1] = l1;
       }
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
-    merge_store<G, D>(merge + (iter & 1) * kConsumerWarps * kMF, u, p);
+    asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
+    merge_store<G, D, kCW>(merge + (iter & 1) * kCW * kMF, u, p);
   }
 }
 

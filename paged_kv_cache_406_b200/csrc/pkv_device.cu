@@ -237,6 +237,7 @@ int launch_decode(const pkv::DecodeParams& base, const int32_t* seq_lens, int32_
   p.n_stages = ring_stages(size_t(2) * bs * D * sizeof(T));
   const size_t smem = pkv::DecodeSmem<T, D, G>::bytes(bs, p.n_stages);
   auto kern = pkv::decode_kernel<T, D, G>;
+  auto kern_stall = pkv::decode_kernel<T, D, G, true>;
 
   // per device: opt in to the largest dynamic shared memory any block size
   // needs (once), then cache resident CTAs per SM for this block size
@@ -247,10 +248,12 @@ int launch_decode(const pkv::DecodeParams& base, const int32_t* seq_lens, int32_
     size_t smem_max = 0;
     for (int bs : {8, 16, 32})
       smem_max = std::max(smem_max, pkv::DecodeSmem<T, D, G>::bytes(bs, ring_stages(size_t(2) * bs * D * sizeof(T))));
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_max));
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(carveout)");
+    for (auto k : {kern, kern_stall}) {
+      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_max));
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
+      e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(carveout)");
+    }
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, pkv::kDecodeThreads, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
     if (occ <= 0) return fail(PKV_ERR_CUDA, "decode kernel does not fit on an SM (smem %zu)", smem);
@@ -259,8 +262,8 @@ int launch_decode(const pkv::DecodeParams& base, const int32_t* seq_lens, int32_
 
   const int64_t work_upper = int64_t(num_seqs) * p.max_parts * p.num_kv_heads;
   const int grid = static_cast<int>(std::min<int64_t>(int64_t(sm_count(dev)) * occ, work_upper));
-  return launch_plan_decode_merge<D>(p, seq_lens, num_seqs, max_tokens, ap, kern, grid, pkv::kDecodeThreads, smem,
-                                     stream);
+  return launch_plan_decode_merge<D>(p, seq_lens, num_seqs, max_tokens, ap, p.stall_cta >= 0 ? kern_stall : kern,
+                                     grid, pkv::kDecodeThreads, smem, stream);
 }
 
 // ---- tensor maps over the K/V pools for the tensor-core kernel ----
@@ -350,17 +353,22 @@ int launch_decode_mma(const pkv::DecodeParams& base, const int32_t* seq_lens, in
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  using Smem = pkv::MmaSmem<T, D, G, kKVBytes>;
   p.n_stages = 8;
-  const size_t smem = pkv::MmaSmem<T, D, G, kKVBytes>::bytes(p.n_stages);
+  const size_t smem = Smem::bytes(p.n_stages);
   auto kern = pkv::decode_mma_kernel<T, D, G, kKVBytes, kMulti>;
+  // the bounded-wait test instance exists for single-pool batches only
+  auto kern_stall = pkv::decode_mma_kernel<T, D, G, kKVBytes, kMulti, !kMulti>;
   static std::atomic<int> occ_cache[kMaxDevices];
   int occ = dev < kMaxDevices ? occ_cache[dev].load(std::memory_order_relaxed) : 0;
   if (occ == 0) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_mma)");
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(carveout)");
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, pkv::kMmaThreads, smem);
+    for (auto k : {kern, kern_stall}) {
+      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_mma)");
+      e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(carveout)");
+    }
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, Smem::kThreads, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
     if (occ <= 0) return fail(PKV_ERR_CUDA, "decode_mma kernel does not fit on an SM (smem %zu)", smem);
     if (dev < kMaxDevices) occ_cache[dev].store(occ, std::memory_order_relaxed);
@@ -379,8 +387,8 @@ int launch_decode_mma(const pkv::DecodeParams& base, const int32_t* seq_lens, in
 
   const int64_t work_upper = int64_t(num_seqs) * p.max_parts * p.num_kv_heads;
   const int grid = static_cast<int>(std::min<int64_t>(int64_t(sm_count(dev)) * occ, work_upper));
-  return launch_plan_decode_merge<D>(p, seq_lens, num_seqs, max_tokens, ap, kern, grid, pkv::kMmaThreads, smem, stream,
-                                     maps);
+  return launch_plan_decode_merge<D>(p, seq_lens, num_seqs, max_tokens, ap, p.stall_cta >= 0 ? kern_stall : kern,
+                                     grid, Smem::kThreads, smem, stream, maps);
 }
 
 template <typename T>
