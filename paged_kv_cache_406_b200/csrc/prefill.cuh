@@ -138,35 +138,6 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, int3
       : "memory");
 }
 
-// Waits for the phase of `bar` with the given parity, like mbar_wait, but
-// lets the hardware suspend the thread until the phase completes (up to
-// 20 us per try) instead of re-polling: the producer and MMA warps share
-// their SM sub-partitions with softmax warps, whose issue slots a spinning
-// wait would take.  Gives up once *abort is set or after kWaitLimitNs.
-__device__ __forceinline__ bool pf_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (;;) {
-    uint32_t done;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
-        : "=r"(done)
-        : "r"(bar), "r"(parity), "r"(20000u)
-        : "memory");
-    if (done) return true;
-    if (*abort) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
-  }
-}
-
-// Waits (bounded by time only) for a phase; used to drain copies and MMAs in
-// flight before the CTA exits or frees tensor memory.
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity) && global_timer_ns() - t0 < kWaitLimitNs) {
-  }
-}
-
 // P as two 16-bit halves, packed in pairs (x0 in the low half): hi + lo
 // carries about 16 significant bits.  bf16: hi is the truncated top half of
 // the fp32 value (a byte permute), lo the rounded remainder (exact in fp32).
@@ -364,7 +335,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
   auto read_tile = [&](int ti) -> int {
     int t = total;
     if (lane == 0) {
-      if (pf_wait(bar(pf::kTileReady + (ti & 1)), (ti >> 1) & 1, abort_flag)) t = tile_slot[ti & 1];
+      if (mbar_wait_sleep(bar(pf::kTileReady + (ti & 1)), (ti >> 1) & 1, abort_flag)) t = tile_slot[ti & 1];
       mbar_arrive(bar(pf::kTileFree + (ti & 1)));
     }
     return __shfl_sync(pf::kAll, t, 0);
@@ -387,7 +358,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         t = total;
         if (lane == 0) {
           // the slot's previous tile has been read by every other role
-          const bool free = ti < 2 || pf_wait(bar(pf::kTileFree + (ti & 1)), ((ti >> 1) - 1) & 1, abort_flag);
+          const bool free = ti < 2 || mbar_wait_sleep(bar(pf::kTileFree + (ti & 1)), ((ti >> 1) - 1) & 1, abort_flag);
           if (!free && !*abort_flag) {
             record_error(PKV_ERR_DEVICE_TIMEOUT);
             *abort_flag = 1;
@@ -407,7 +378,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       const int b = d.b, g = d.g, nc = d.nc, nblk = d.nblk;
       if (kv == 0) {
         // Q of the previous tile is no longer read once its last q·Kᵀ is done
-        if (tv > 0) ok = __all_sync(pf::kAll, pf_wait(bar(pf::kQEmpty), (tv - 1) & 1, abort_flag));
+        if (tv > 0) ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kQEmpty), (tv - 1) & 1, abort_flag));
         if (!ok) break;
         if (lane == 0) {
           // Q tile: rows token * G + h, one box per head_dim half
@@ -444,7 +415,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         }
         const int32_t y = (phys * p.num_kv_heads + g) * BS;
         const uint32_t full = full0 + 8 * s;
-        ok = __all_sync(pf::kAll, pf_wait(empty0 + 8 * s, ph, abort_flag));
+        ok = __all_sync(pf::kAll, mbar_wait_sleep(empty0 + 8 * s, ph, abort_flag));
         if (!ok) break;
         if (lane == 0) mbar_arrive_expect_tx(full, static_cast<uint32_t>(nload) * 2u * box_bytes);
         __syncwarp();
@@ -466,10 +437,10 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     // fills unconsumed): wait (bounded) for the last fill of each stage and Q
     if (lane == 0) {
       const uint32_t full0 = bar(kv ? pf::kVFull : pf::kKFull);
-      if (kv == 0 && q_issued > 0) drain_wait(bar(pf::kQFull), (q_issued - 1) & 1);
+      if (kv == 0 && q_issued > 0) mbar_drain(bar(pf::kQFull), (q_issued - 1) & 1);
       for (int s = 0; s < pf::kStages && s < issued; ++s) {
         const int last = s + (issued - 1 - s) / pf::kStages * pf::kStages;  // last chunk that used stage s
-        drain_wait(full0 + 8 * s, (last / pf::kStages) & 1);
+        mbar_drain(full0 + 8 * s, (last / pf::kStages) & 1);
       }
     }
     __syncwarp();
@@ -490,7 +461,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       if (lane == 0) {
         auto issue_s = [&](int j) -> bool {  // j: chunk of the tile; gc + j: chunk of the CTA
           const int s = (gc + j) % pf::kStages;
-          if (!pf_wait(bar(pf::kKFull + s), ((gc + j) / pf::kStages) & 1, abort_flag)) return false;
+          if (!mbar_wait_sleep(bar(pf::kKFull + s), ((gc + j) / pf::kStages) & 1, abort_flag)) return false;
           tc::fence_after_sync();
           const uint32_t kst = base + pf::kOffK + s * pf::kTile;
 #pragma unroll
@@ -504,16 +475,16 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
           tc::commit(bar(pf::kSFull + (gc + j) % pf::kSBufs));
           return true;
         };
-        ok = pf_wait(bar(pf::kQFull), tv & 1, abort_flag);
+        ok = mbar_wait_sleep(bar(pf::kQFull), tv & 1, abort_flag);
         for (int j = 0; j < pf::kSBufs && j < nc && ok; ++j) ok = issue_s(j);
         if (ok && nc <= pf::kSBufs) tc::commit(bar(pf::kQEmpty));  // the tile's last q·Kᵀ is issued
         // the previous tile's O has been read out of tensor memory
-        if (ok && tv > 0) ok = pf_wait(bar(pf::kOFree), (tv - 1) & 1, abort_flag);
+        if (ok && tv > 0) ok = mbar_wait_sleep(bar(pf::kOFree), (tv - 1) & 1, abort_flag);
         for (int j = 0; j < nc && ok; ++j) {
           const int gj = gc + j;
           const int s = gj % pf::kStages;
-          ok = pf_wait(bar(pf::kPFull + gj % pf::kSBufs), (gj / pf::kSBufs) & 1, abort_flag) &&
-               pf_wait(bar(pf::kVFull + s), (gj / pf::kStages) & 1, abort_flag);
+          ok = mbar_wait_sleep(bar(pf::kPFull + gj % pf::kSBufs), (gj / pf::kSBufs) & 1, abort_flag) &&
+               mbar_wait_sleep(bar(pf::kVFull + s), (gj / pf::kStages) & 1, abort_flag);
           if (!ok) break;
           tc::fence_after_sync();
           const uint32_t vst = base + pf::kOffV + s * pf::kTile;
@@ -547,7 +518,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       }
       // every MMA issued completes before tensor memory is freed
       tc::commit(bar(pf::kDrain));
-      drain_wait(bar(pf::kDrain), 0);
+      mbar_drain(bar(pf::kDrain), 0);
     }
     __syncwarp();
   } else {
@@ -571,7 +542,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         const int gj = gc + j;              // chunk of the CTA
         const int sb = gj % pf::kSBufs;     // S / P buffer
         const int s = gj % pf::kStages;     // K / V stage
-        ok = __all_sync(pf::kAll, pf_wait(bar(pf::kSFull + sb), (gj / pf::kSBufs) & 1, abort_flag));
+        ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kSFull + sb), (gj / pf::kSBufs) & 1, abort_flag));
         if (!ok) break;
         tc::fence_after_sync();
         float x[pf::kKeys];  // raw scores q·k of this row's 128 keys
@@ -653,7 +624,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
           // phase (PV_{j-4}) was covered by S_j's commit, so the parity wait
           // cannot see an older phase.
           const int pj = gj - 1;
-          ok = __all_sync(pf::kAll, pf_wait(bar(pf::kPVDone + pj % pf::kSBufs), (pj / pf::kSBufs) & 1, abort_flag));
+          ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kPVDone + pj % pf::kSBufs), (pj / pf::kSBufs) & 1, abort_flag));
           if (!ok) break;
           tc::fence_after_sync();
 #pragma unroll
@@ -670,7 +641,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         if (zero_v) {
           // V rows past the sequence end hold stale or unwritten bytes: zero
           // them so that P = 0 there cannot meet a NaN pattern
-          ok = __all_sync(pf::kAll, pf_wait(bar(pf::kVFull + s), (gj / pf::kStages) & 1, abort_flag));
+          ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kVFull + s), (gj / pf::kStages) & 1, abort_flag));
           if (!ok) break;
           const int v0 = L - key0;
           unsigned char* vst = vzero + s * pf::kTile;
@@ -686,7 +657,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         mbar_arrive(bar(pf::kPFull + sb));
       }
       // the MMA warp commits O-done after the tile's last P·V
-      if (ok) ok = __all_sync(pf::kAll, pf_wait(bar(pf::kODone), tv & 1, abort_flag));
+      if (ok) ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kODone), tv & 1, abort_flag));
       if (!ok) break;
       tc::fence_after_sync();
       // O leaves tensor memory first (the next tile's P·V may then overwrite
