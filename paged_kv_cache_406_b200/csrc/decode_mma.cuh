@@ -38,19 +38,16 @@ constexpr int kMmaProducers = 2;
 constexpr int kMmaThreads = (kConsumerWarps + kMmaProducers) * 32;
 
 
-// kKVBytes = bytes per stored K/V element: 2 (bf16 / f16) or 1 (e4m3).
-template <int D, int kKVBytes = 2>
+template <int D>
 struct MmaLayout {
-  static constexpr int kHalves = D / 64;                           // 128-byte column halves of a 16-bit row
-  static constexpr int kTileBytes = kChunkTokens * D * 2;           // 16-bit 16-token K (or V) chunk
-  static constexpr int kRingHalves = D * kKVBytes / 128;            // 128-byte column halves of a stored row
-  static constexpr int kRingTileBytes = kChunkTokens * D * kKVBytes;  // stored 16-token chunk in the ring
-  static constexpr int kStageBytes = 2 * kRingTileBytes;
+  static constexpr int kHalves = D / 64;                   // 128-byte column halves of a 16-bit row
+  static constexpr int kTileBytes = kChunkTokens * D * 2;  // 16-token K (or V) chunk
+  static constexpr int kStageBytes = 2 * kTileBytes;
 };
 
-template <typename T, int D, int G, int kKVBytes = 2>
+template <typename T, int D, int G>
 struct MmaSmem {
-  using L = MmaLayout<D, kKVBytes>;
+  using L = MmaLayout<D>;
   static constexpr int kCW = kConsumerWarps;
   static constexpr int kThreads = kMmaThreads;
   static constexpr int kMergeFloats = G * D + 2 * G;
@@ -64,16 +61,6 @@ struct MmaSmem {
   }
 };
 
-// Four e4m3 codes (one word, code i in byte i) widened exactly to two packed
-// f16 pairs: codes 0, 1 into lo and codes 2, 3 into hi.  The word is split
-// into its 16-bit halves by a register-pair move rather than a shift (one
-// ALU instruction fewer per pair: the e4m3 kernel is bound by its ALU pipe).
-__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %2;\n cvt.rn.f16x2.e4m3x2 %0, l;\n cvt.rn.f16x2.e4m3x2 %1, h;\n}"
-      : "=r"(lo), "=r"(hi)
-      : "r"(w));
-}
-
 // A chunk tile in shared memory is built from TMA boxes of `br` rows (br = 16,
 // or 8 when block_size is 8 and a chunk spans two blocks).  Each box holds,
 // for every 128-byte column half h, br rows of 128 B with the 128-byte
@@ -84,16 +71,6 @@ __device__ __forceinline__ uint32_t row_offset(int r, int h, int br_shift, int h
   return static_cast<uint32_t>(((r >> br_shift) * halves * br + h * br + (r & (br - 1))) * 128);
 }
 
-// kKVBytes = 1: the pools hold e4m3 codes (T must be __half: e4m3 widens to
-// f16 exactly).  A consumer warp loads the codes it needs as 32-bit words,
-// frees the ring stage at once and widens them into mma fragments in
-// registers; the contraction order of q·Kᵀ and the output dims of P·V are
-// permuted within each step so every word feeds whole fragment registers.
-// The e4m3 kernel is held to 3 CTAs per SM (96 registers instead of 158, no
-// spills): its consumers are bound by latency, not issue, and 12 consumer
-// warps per SM instead of 8 take its decode call from 77.3 to 74.8 us on the
-// Llama-3-8B-shaped batch (4 CTAs would spill).  The 16-bit kernels keep the
-// compiler's own choice (127 registers, 2 CTAs per SM).
 // Tensor maps of the K and V pools of a batch (pool c: k[c], v[c]).
 struct PoolMaps {
   CUtensorMap k[kMaxPools];
@@ -106,26 +83,27 @@ struct PoolMaps {
 __device__ __forceinline__ int bs_shift_of(int bs) { return bs == 8 ? 3 : (bs == 16 ? 4 : 5); }
 __device__ __forceinline__ int br_shift_of(int bs) { return bs == 8 ? 3 : 4; }
 
+// Two CTAs fit an SM (shared memory); declaring it lets the compiler use up
+// to 170 registers (146 for head_dim 128) instead of its own choice of 96,
+// which was 1-2 % slower.
 // kMulti: the batch spans up to kMaxPools pools of different block sizes
 // (each work unit reads its sequence's pool); otherwise pool 0 only.
 // kStall: the instance that honours DecodeParams::stall_cta (the test of the
 // bounded waits); production launches use the instance without the check.
-template <typename T, int D, int G, int kKVBytes = 2, bool kMulti = false, bool kStall = false>
-__global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0)
+template <typename T, int D, int G, bool kMulti = false, bool kStall = false>
+__global__ void __launch_bounds__(kMmaThreads, 2)
     decode_mma_kernel(const DecodeParams p, const __grid_constant__ PoolMaps maps) {
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
-  static_assert(kKVBytes == 2 || (kKVBytes == 1 && D == 128), "e4m3 pools need head_dim 128");
-  using L = MmaLayout<D, kKVBytes>;
-  constexpr bool kFp8 = kKVBytes == 1;
+  using L = MmaLayout<D>;
   constexpr int kCW = kConsumerWarps;
   constexpr int kSteps = D / 16;  // k-steps of q·Kᵀ and m-tiles of P·V
   constexpr int kHalves = L::kHalves;
-  constexpr int kMF = MmaSmem<T, D, G, kKVBytes>::kMergeFloats;
+  constexpr int kMF = MmaSmem<T, D, G>::kMergeFloats;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
   const int NS = p.n_stages;
-  float* merge = reinterpret_cast<float*>(smem + MmaSmem<T, D, G, kKVBytes>::ring_bytes(NS));
+  float* merge = reinterpret_cast<float*>(smem + MmaSmem<T, D, G>::ring_bytes(NS));
   uint64_t* full = reinterpret_cast<uint64_t*>(merge + 2 * kCW * kMF);
   uint64_t* empty = full + NS;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + NS);
@@ -170,8 +148,8 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0)
       const WorkUnit u = load_unit<kMulti>(p, w);
       const PoolView pv = kMulti ? pick3(p.pool, u.c) : p.pool[0];
       const int BS = pv.block_size, bs_shift = bs_shift_of(BS), br_shift = br_shift_of(BS);
-      const uint32_t box_bytes = (1u << br_shift) * D * kKVBytes;        // one K (or V) box
-      const uint32_t blk_off = L::kRingHalves * (1u << br_shift) * 128;  // second box of a chunk (block_size 8)
+      const uint32_t box_bytes = (1u << br_shift) * D * 2;               // one K (or V) box
+      const uint32_t blk_off = L::kHalves * (1u << br_shift) * 128;  // second box of a chunk (block_size 8)
       const CUtensorMap* tmap_k = &maps.k[kMulti ? u.c : 0];
       const CUtensorMap* tmap_v = &maps.v[kMulti ? u.c : 0];
       const int32_t* trow = pv.tables + static_cast<int64_t>(u.b - pv.seq0) * pv.max_blocks + (u.t0 >> bs_shift);
@@ -205,7 +183,7 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0)
               }
               const int32_t y = phys * p.num_kv_heads * BS + ybase + row0;
               tma_load_3d(kdst + i * blk_off, tmap_k, 0, y, 0, bar, policy);
-              tma_load_3d(kdst + L::kRingTileBytes + i * blk_off, tmap_v, 0, y, 0, bar, policy);
+              tma_load_3d(kdst + L::kTileBytes + i * blk_off, tmap_v, 0, y, 0, bar, policy);
             }
             ++issued;
             s += kMmaProducers;
@@ -268,16 +246,8 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0)
       const T* qrow = static_cast<const T*>(p.q) + (static_cast<int64_t>(u.b) * p.num_q_heads + u.g * G + gq) * D;
 #pragma unroll
       for (int ks = 0; ks < kSteps; ++ks) {
-        if constexpr (kFp8) {
-          // e4m3 K fragments hold dims 16ks + 4tq .. +3 (one 32-bit word of
-          // codes); q follows the same order of the contraction
-          const uint2 v = gq < G ? __ldg(reinterpret_cast<const uint2*>(qrow + 16 * ks + 4 * tq)) : make_uint2(0u, 0u);
-          qb[ks][0] = v.x;
-          qb[ks][1] = v.y;
-        } else {
-          qb[ks][0] = gq < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq)) : 0u;
-          qb[ks][1] = gq < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq + 8)) : 0u;
-        }
+        qb[ks][0] = gq < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq)) : 0u;
+        qb[ks][1] = gq < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq + 8)) : 0u;
       }
     }
     float acc[kSteps][4];
@@ -299,50 +269,15 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0)
         break;
       }
       uint32_t kbase = ring_s + s * L::kStageBytes;
-      uint32_t vbase = kbase + L::kRingTileBytes;
+      uint32_t vbase = kbase + L::kTileBytes;
       const int nv = min(kChunkTokens, u.t1 - (u.t0 + k * kChunkTokens));
       // ---- scores: S^T = K · Qᵀ ----
       float sc[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t vw[kFp8 ? D / 32 : 1][4];  // e4m3 V words: tokens 2tq, 2tq+1, 2tq+8, 2tq+9
-      if constexpr (kFp8) {
-        // e4m3 rows are 128 B (one swizzle row): token r, 16-byte chunk c at
-        // position c ^ (r % 8).  Every code the warp needs is loaded as 32-bit
-        // words (bank-conflict free), then the ring stage goes back to the
-        // producer before any arithmetic.
-        uint32_t kw[kSteps][2];
 #pragma unroll
-        for (int ks = 0; ks < kSteps; ++ks) {
-          const uint32_t a = kbase + gq * 128 + ((ks ^ gq) << 4) + 4 * tq;  // token gq; gq + 8 has the same swizzle
-          asm volatile("ld.shared.b32 %0, [%1];" : "=r"(kw[ks][0]) : "r"(a));
-          asm volatile("ld.shared.b32 %0, [%1];" : "=r"(kw[ks][1]) : "r"(a + 8 * 128));
-        }
-#pragma unroll
-        for (int pp = 0; pp < D / 32; ++pp) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int t = 2 * tq + (i & 1) + (i >> 1) * 8;
-            const uint32_t a = vbase + t * 128 + (((2 * pp + (gq >> 2)) ^ (t & 7)) << 4) + 4 * (gq & 3);
-            asm volatile("ld.shared.b32 %0, [%1];" : "=r"(vw[pp][i]) : "r"(a));
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_addr(empty + s));
-#pragma unroll
-        for (int ks = 0; ks < kSteps; ++ks) {
-          // contraction order within the step: K dims 16ks + 4tq + {0,1 | 2,3}
-          // stand at fragment columns {2tq, 2tq+1 | 2tq+8, 2tq+9}
-          uint32_t a[4];
-          e4m3x4_to_f16x2x2(kw[ks][0], a[0], a[2]);
-          e4m3x4_to_f16x2x2(kw[ks][1], a[1], a[3]);
-          mma_16816<T>(sc, a, qb[ks][0], qb[ks][1]);
-        }
-      } else {
-#pragma unroll
-        for (int ks = 0; ks < kSteps; ++ks) {
-          uint32_t a[4];
-          ldmatrix_x4(kbase + offa[ks / 4] + (((2 * (ks % 4) + ca) ^ xa) << 4), a);
-          mma_16816<T>(sc, a, qb[ks][0], qb[ks][1]);
-        }
+      for (int ks = 0; ks < kSteps; ++ks) {
+        uint32_t a[4];
+        ldmatrix_x4(kbase + offa[ks / 4] + (((2 * (ks % 4) + ca) ^ xa) << 4), a);
+        mma_16816<T>(sc, a, qb[ks][0], qb[ks][1]);
       }
       const bool v0 = gq < nv, v1 = gq + 8 < nv;  // tokens gq and gq + 8 of the chunk
       const float s0 = v0 ? sc[0] * sl : -INFINITY, s1 = v0 ? sc[1] * sl : -INFINITY;
@@ -385,32 +320,6 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0)
       const uint32_t bl0 = __byte_perm(__shfl_sync(kFull, la, src0), __shfl_sync(kFull, la, src1), sel);
       const uint32_t bl1 = __byte_perm(__shfl_sync(kFull, lb, src0), __shfl_sync(kFull, lb, src1), sel);
 
-      if constexpr (kFp8) {
-        // ---- O^T += V^T · P^T from the e4m3 words.  Output dims are
-        // permuted within each 32-dim group: fragment row gq (+8) of m-tile
-        // 2pp + u is dim 32pp + 4gq + 2u (+1), so one word of a token row
-        // (4 consecutive dims) feeds both m-tiles of the pair.  Tokens past
-        // the sequence end read as zero codes. ----
-#pragma unroll
-        for (int pp = 0; pp < D / 32; ++pp) {
-          uint32_t w[4] = {vw[pp][0], vw[pp][1], vw[pp][2], vw[pp][3]};
-          if (nv < kChunkTokens) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) w[i] = (2 * tq + (i & 1) + (i >> 1) * 8) < nv ? w[i] : 0u;
-          }
-          const uint32_t x01a = __byte_perm(w[0], w[1], 0x5140), x01b = __byte_perm(w[0], w[1], 0x7362);
-          const uint32_t x89a = __byte_perm(w[2], w[3], 0x5140), x89b = __byte_perm(w[2], w[3], 0x7362);
-          uint32_t a[4];
-          e4m3x4_to_f16x2x2(x01a, a[0], a[1]);
-          e4m3x4_to_f16x2x2(x89a, a[2], a[3]);
-          mma_16816<T>(acc[2 * pp], a, bh0, bh1);
-          mma_16816<T>(acc[2 * pp], a, bl0, bl1);
-          e4m3x4_to_f16x2x2(x01b, a[0], a[1]);
-          e4m3x4_to_f16x2x2(x89b, a[2], a[3]);
-          mma_16816<T>(acc[2 * pp + 1], a, bh0, bh1);
-          mma_16816<T>(acc[2 * pp + 1], a, bl0, bl1);
-        }
-      } else {
       // ---- rows past the sequence end: zero V so stale values cannot reach P·V ----
       if (nv < kChunkTokens) {
         const int per_row = 8 * kHalves;
@@ -434,7 +343,6 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0)
       if (nv < kChunkTokens) fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_addr(empty + s));
-      }
       s += kCW;
       if (s >= NS) {
         s -= NS;
@@ -454,15 +362,14 @@ __global__ void __launch_bounds__(kMmaThreads, kKVBytes == 1 ? 3 : 0)
 #pragma unroll
     for (int mt = 0; mt < kSteps; ++mt) {
       // fragment rows gq and gq + 8 of m-tile mt: dims d and d + dd
-      const int d = kFp8 ? 32 * (mt >> 1) + 4 * gq + 2 * (mt & 1) : 16 * mt + gq;
-      const int dd = kFp8 ? 1 : 8;
+      const int d = 16 * mt + gq;
       if (h0 < G) {
         mb[h0 * D + d] = acc[mt][0];
-        mb[h0 * D + d + dd] = acc[mt][2];
+        mb[h0 * D + d + 8] = acc[mt][2];
       }
       if (h1 < G) {
         mb[h1 * D + d] = acc[mt][1];
-        mb[h1 * D + d + dd] = acc[mt][3];
+        mb[h1 * D + d + 8] = acc[mt][3];
       }
     }
     if (gq == 0) {

@@ -54,17 +54,19 @@ constexpr uint32_t kStageBytes = 2 * kTileBytes;  // K then V
 constexpr uint32_t kTmemCols = 128;
 constexpr uint32_t kColS = 0, kColO = 64;  // S^T buffers at columns 0 and 32, O^T at 64
 constexpr float kThreshold = 8.0f;
-constexpr uint32_t kPBuf = 4096;  // one P-terms buffer
 
 // N of the two MMAs: terms x heads, rounded up to the shape rules
 __host__ __device__ constexpr int n_s(int g) { return (kTermsQ * g + 7) / 8 * 8; }
 __host__ __device__ constexpr int n_o(int g) { return (kTermsP * g + 15) / 16 * 16; }
 
-// shared memory (from a 1024-byte aligned base) for a ring of NSt stages
-template <int NSt>
+// shared memory (from a 1024-byte aligned base) for a ring of NSt stages and
+// G query heads per KV head
+template <int NSt, int G>
 struct Layout {
-  static constexpr uint32_t kOffQ = NSt * kStageBytes;  // q terms: up to 24 rows x 128 B, swizzled
-  static constexpr uint32_t kOffP = kOffQ + 3 * 1024;   // P terms: 2 buffers x [group][token][16 B]
+  static constexpr uint32_t kPBuf = n_o(G) / 16 * 2048;  // P terms of one chunk: [group][token][16 B]
+  static constexpr uint32_t kOffQ = NSt * kStageBytes;   // q terms: n_s(G) rows x 128 B, swizzled
+  static constexpr uint32_t kQBytes = n_s(G) / 8 * 1024;
+  static constexpr uint32_t kOffP = kOffQ + kQBytes;     // two P-terms buffers
   static constexpr uint32_t kOffRed = kOffP + 2 * kPBuf;  // [3][4 warps][8 heads]: chunk maxima (2), row sums
   static constexpr uint32_t kOffQs = kOffRed + 3 * 4 * 8 * 4;
   static constexpr uint32_t kOffBar = kOffQs + 8 * 4;
@@ -107,10 +109,44 @@ __device__ __forceinline__ float warp_max(float x) {
   return x;
 }
 
-__device__ __forceinline__ float warp_sum(float x) {
+// Reduce-scatter of G per-lane values over the warp: lane l returns the
+// reduction (max, or sum) of head (l >> (5 - log2 G)) over all 32 lanes.
+// The first log2 G steps halve each lane's list (the half a lane keeps is
+// chosen by its lane bit), so G heads cost 5 + G - 1 - log2 G shuffles
+// (6 for G = 4) instead of 5 G.
+template <int G, bool kMax>
+__device__ __forceinline__ float reduce_scatter(const float (&v)[G], int lane) {
+  float a[G];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-  return x;
+  for (int i = 0; i < G; ++i) a[i] = v[i];
+  int o = 16;
+#pragma unroll
+  for (int n = G; n > 1; n >>= 1, o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < n / 2; ++i) {
+      const float keep = up ? a[i + n / 2] : a[i], give = up ? a[i] : a[i + n / 2];
+      const float other = __shfl_xor_sync(0xffffffffu, give, o);
+      a[i] = kMax ? fmaxf(keep, other) : keep + other;
+    }
+  }
+#pragma unroll
+  for (; o > 0; o >>= 1) {
+    const float other = __shfl_xor_sync(0xffffffffu, a[0], o);
+    a[0] = kMax ? fmaxf(a[0], other) : a[0] + other;
+  }
+  return a[0];
+}
+
+// The head whose reduction lane l holds after reduce_scatter<G>, and whether
+// l is the first lane holding it.
+template <int G>
+__device__ __forceinline__ int scatter_head(int lane) {
+  return G == 1 ? 0 : (lane >> (G == 2 ? 4 : (G == 4 ? 3 : 2))) & (G - 1);
+}
+template <int G>
+__device__ __forceinline__ bool scatter_first(int lane) {
+  return (lane & (32 / G - 1)) == 0;
 }
 
 // Two fp32 values rounded to e4m3 (nearest, ties to even; no value here
@@ -127,12 +163,12 @@ __device__ __forceinline__ uint32_t e4m3_pair(float x0, float x1, float& d0, flo
 }  // namespace t8
 
 template <int G, int NSt>
-__global__ void __launch_bounds__(t8::kThreads, NSt <= 3 ? 2 : 1)
+__global__ void __launch_bounds__(t8::kThreads, NSt <= 2 ? 3 : (NSt == 3 ? 2 : 1))
     decode_tc8_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v) {
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
   constexpr int NS_ = t8::n_s(G), NO = t8::n_o(G);
-  using L = t8::Layout<NSt>;
+  using L = t8::Layout<NSt, G>;
   static_assert(NS_ <= 32 && NO <= 32, "S^T and O^T columns");
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -152,9 +188,9 @@ __global__ void __launch_bounds__(t8::kThreads, NSt <= 3 ? 2 : 1)
   if (warp < 4) {
     // q-term rows past kTermsQ * G are never written: zero them (and the rest) once
     uint4* q = reinterpret_cast<uint4*>(smem + L::kOffQ);
-    for (int i = threadIdx.x; i < 3 * 1024 / 16; i += 128) q[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = threadIdx.x; i < static_cast<int>(L::kQBytes) / 16; i += 128) q[i] = make_uint4(0u, 0u, 0u, 0u);
     uint4* pz = reinterpret_cast<uint4*>(smem + L::kOffP);
-    for (int i = threadIdx.x; i < 2 * static_cast<int>(t8::kPBuf) / 16; i += 128) pz[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = threadIdx.x; i < 2 * static_cast<int>(L::kPBuf) / 16; i += 128) pz[i] = make_uint4(0u, 0u, 0u, 0u);
   }
   if (warp == t8::kMmaWarp) {
     tc::tmem_alloc(smem_addr(tmem_slot), t8::kTmemCols);
@@ -295,7 +331,7 @@ __global__ void __launch_bounds__(t8::kThreads, NSt <= 3 ? 2 : 1)
           tc::fence_after_sync();
           // O^T += V^T (MN-major: V rows as stored) · P terms (MN-major, 16-byte token rows), 4 x 32 tokens
           const uint32_t vst = base + (jj % NSt) * t8::kStageBytes + t8::kTileBytes;
-          const uint32_t pb = base + L::kOffP + (jj & 1) * t8::kPBuf;
+          const uint32_t pb = base + L::kOffP + (jj & 1) * L::kPBuf;
 #pragma unroll
           for (int ks = 0; ks < t8::kTok / 32; ++ks) {
             tc::mma_e4m3_ss(tmem + t8::kColO, tc::sw128_desc(vst + 4096 * ks, 16, 1024),
@@ -424,17 +460,16 @@ __global__ void __launch_bounds__(t8::kThreads, NSt <= 3 ? 2 : 1)
         tc::fence_before_sync();
         mbar_arrive(bar(L::kBSFree + (j & 1)));
         fail |= !got;
-        float s[G], cm[G];
+        float s[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           const float dot = __uint_as_float(sr[h]) + __uint_as_float(sr[G + h]) * 0.0625f +
                             __uint_as_float(sr[2 * G + h]) * 0.00390625f;
           s[h] = (t < nv && got) ? sw[h] * dot : -INFINITY;
-          cm[h] = t8::warp_max(s[h]);
         }
-        if (lane == 0) {
-#pragma unroll
-          for (int h = 0; h < G; ++h) red[(j & 1) * 32 + warp * 8 + h] = cm[h];
+        {
+          const float cm = t8::reduce_scatter<G, true>(s, lane);
+          if (t8::scatter_first<G>(lane)) red[(j & 1) * 32 + warp * 8 + t8::scatter_head<G>(lane)] = cm;
         }
         __syncwarp();
         fail = t8::softmax_bar_any(fail);
@@ -508,7 +543,7 @@ __global__ void __launch_bounds__(t8::kThreads, NSt <= 3 ? 2 : 1)
             }
           }
         }
-        unsigned char* pb = smem + L::kOffP + (j & 1) * t8::kPBuf;
+        unsigned char* pb = smem + L::kOffP + (j & 1) * L::kPBuf;
 #pragma unroll
         for (int g16 = 0; g16 < NO / 16; ++g16) {
           *reinterpret_cast<uint4*>(pb + g16 * 2048 + t * 16) =
@@ -535,13 +570,8 @@ __global__ void __launch_bounds__(t8::kThreads, NSt <= 3 ? 2 : 1)
       // ---- unit epilogue: row sums over the 128 threads, O^T out of tensor memory ----
       float* lsum = red + 64;  // [4 warps][8 heads], after the two chunk-max buffers
       {
-        float ls[G];
-#pragma unroll
-        for (int h = 0; h < G; ++h) ls[h] = t8::warp_sum(l[h]);
-        if (lane == 0) {
-#pragma unroll
-          for (int h = 0; h < G; ++h) lsum[warp * 8 + h] = ls[h];
-        }
+        const float ls = t8::reduce_scatter<G, false>(l, lane);
+        if (t8::scatter_first<G>(lane)) lsum[warp * 8 + t8::scatter_head<G>(lane)] = ls;
       }
       const bool okd =
           __all_sync(0xffffffffu, mbar_wait_sleep(bar(L::kBPFree + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag));

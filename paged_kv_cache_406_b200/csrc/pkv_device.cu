@@ -346,7 +346,7 @@ int pool_map(CUtensorMap* out, const void* pool, int dtype, int64_t rows, int he
   return PKV_OK;
 }
 
-template <typename T, int D, int G, int kKVBytes = 2, bool kMulti = false>
+template <typename T, int D, int G, bool kMulti = false>
 int launch_decode_mma(const pkv::DecodeParams& base, const int32_t* seq_lens, int32_t num_seqs, int32_t max_tokens,
                       int dtype, const PendingAppend* ap, cudaStream_t stream) {
   pkv::DecodeParams p = base;
@@ -354,12 +354,12 @@ int launch_decode_mma(const pkv::DecodeParams& base, const int32_t* seq_lens, in
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  using Smem = pkv::MmaSmem<T, D, G, kKVBytes>;
+  using Smem = pkv::MmaSmem<T, D, G>;
   p.n_stages = 8;
   const size_t smem = Smem::bytes(p.n_stages);
-  auto kern = pkv::decode_mma_kernel<T, D, G, kKVBytes, kMulti>;
+  auto kern = pkv::decode_mma_kernel<T, D, G, kMulti>;
   // the bounded-wait test instance exists for single-pool batches only
-  auto kern_stall = pkv::decode_mma_kernel<T, D, G, kKVBytes, kMulti, !kMulti>;
+  auto kern_stall = pkv::decode_mma_kernel<T, D, G, kMulti, !kMulti>;
   static std::atomic<int> occ_cache[kMaxDevices];
   int occ = dev < kMaxDevices ? occ_cache[dev].load(std::memory_order_relaxed) : 0;
   if (occ == 0) {
@@ -765,19 +765,22 @@ extern "C" int pkv_append_and_decode_pools(const pkv_pool_t* pools, int32_t n_po
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int32_t mt = static_cast<int32_t>(max_tokens);
   if (dtype == PKV_BF16) {
-    if (group == 2) return launch_decode_mma<__nv_bfloat16, 128, 2, 2, true>(p, seq_lens, N, mt, dtype, &ap, s);
-    if (group == 4) return launch_decode_mma<__nv_bfloat16, 128, 4, 2, true>(p, seq_lens, N, mt, dtype, &ap, s);
-    return launch_decode_mma<__nv_bfloat16, 128, 8, 2, true>(p, seq_lens, N, mt, dtype, &ap, s);
+    if (group == 2) return launch_decode_mma<__nv_bfloat16, 128, 2, true>(p, seq_lens, N, mt, dtype, &ap, s);
+    if (group == 4) return launch_decode_mma<__nv_bfloat16, 128, 4, true>(p, seq_lens, N, mt, dtype, &ap, s);
+    return launch_decode_mma<__nv_bfloat16, 128, 8, true>(p, seq_lens, N, mt, dtype, &ap, s);
   }
-  if (group == 2) return launch_decode_mma<__half, 128, 2, 2, true>(p, seq_lens, N, mt, dtype, &ap, s);
-  if (group == 4) return launch_decode_mma<__half, 128, 4, 2, true>(p, seq_lens, N, mt, dtype, &ap, s);
-  return launch_decode_mma<__half, 128, 8, 2, true>(p, seq_lens, N, mt, dtype, &ap, s);
+  if (group == 2) return launch_decode_mma<__half, 128, 2, true>(p, seq_lens, N, mt, dtype, &ap, s);
+  if (group == 4) return launch_decode_mma<__half, 128, 4, true>(p, seq_lens, N, mt, dtype, &ap, s);
+  return launch_decode_mma<__half, 128, 8, true>(p, seq_lens, N, mt, dtype, &ap, s);
 }
 
-// e4m3 pools: the tcgen05 kernel (decode_tc8.cuh), two persistent CTAs per SM,
-// each with a ring of three 128-token chunks (one CTA with six stages: 27 %
-// slower on the Llama-3-8B batch).
-constexpr int kTc8Stages = 3;
+// e4m3 pools: the tcgen05 kernel (decode_tc8.cuh), persistent CTAs with a ring
+// of 128-token chunks: three CTAs per SM with two stages each (G <= 4), two
+// with three (G = 8, whose registers do not fit three CTAs).  On the
+// Llama-3-8B batch 3 x 2 stages ran 4.8 % faster than 2 x 3 and 45 % faster
+// than one CTA with 6: the softmax warps' latency, not the bytes in flight,
+// bounds the kernel, so more of them per SM is what pays.
+__host__ __device__ constexpr int tc8_stages(int g) { return g == 8 ? 3 : 2; }
 
 template <int G>
 int launch_decode_tc8(const pkv::DecodeParams& base, const int32_t* seq_lens, int32_t num_seqs, int32_t max_tokens,
@@ -786,8 +789,9 @@ int launch_decode_tc8(const pkv::DecodeParams& base, const int32_t* seq_lens, in
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  const size_t smem = pkv::t8::Layout<kTc8Stages>::kSmemBytes;
-  auto kern = pkv::decode_tc8_kernel<G, kTc8Stages>;
+  constexpr int NSt = tc8_stages(G);
+  const size_t smem = pkv::t8::Layout<NSt, G>::kSmemBytes;
+  auto kern = pkv::decode_tc8_kernel<G, NSt>;
   static std::atomic<int> occ_cache[kMaxDevices];
   int occ = dev < kMaxDevices ? occ_cache[dev].load(std::memory_order_relaxed) : 0;
   if (occ == 0) {
@@ -796,15 +800,15 @@ int launch_decode_tc8(const pkv::DecodeParams& base, const int32_t* seq_lens, in
     e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(carveout)");
     // CTAs per SM from the SM's shared memory (the occupancy query counts
-    // one CTA where two fit: measured, two are co-resident and run twice as
-    // fast); the launch bounds keep the registers of two CTAs within the SM's
-    // file, and each CTA holds 128 of the 512 tensor-memory columns
+    // one CTA where two fit: measured, two are co-resident and run 1.6x as
+    // fast); the launch bounds keep the registers of that many CTAs within
+    // the SM's file, and each CTA holds 128 of the 512 tensor-memory columns
     int smem_sm = 0, reserved = 0;
     e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute(smem per SM)");
     e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute(reserved smem)");
-    occ = std::min(2, smem_sm / static_cast<int>(smem + static_cast<size_t>(reserved)));
+    occ = std::min(NSt == 2 ? 3 : 2, smem_sm / static_cast<int>(smem + static_cast<size_t>(reserved)));
     if (occ <= 0) return fail(PKV_ERR_CUDA, "decode_tc8 kernel does not fit on an SM (smem %zu)", smem);
     if (dev < kMaxDevices) occ_cache[dev].store(occ, std::memory_order_relaxed);
   }
