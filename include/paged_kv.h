@@ -427,9 +427,9 @@ int pkv_kv_append_fp8(const void* k_new, const void* v_new, int32_t src_dtype, c
 /* PagedAttention decode over e4m3 pools: the result of
  * pkv_paged_attention_decode on the dequantised values (scores
  * scale * k_scale * q·code, output v_scale * the softmax-weighted codes).
- * q is float16 [num_seqs][num_q_heads][head_dim] (e4m3 widens to f16
- * exactly); head_dim must be 128; group sizes 1, 2, 4, 8; partition_tokens a
- * multiple of 16 (0 = automatic).  Workspace as sized by
+ * q is float16 [num_seqs][num_q_heads][head_dim]; head_dim must be 128;
+ * group sizes 1, 2, 4, 8; partition_tokens a multiple of 16 (0 =
+ * automatic).  Workspace as sized by
  * pkv_decode_workspace_size with the same arguments. */
 int pkv_paged_attention_decode_fp8(const void* q, const void* k_pool, const void* v_pool,
                                    const int32_t* block_tables, const int32_t* seq_lens, int32_t num_seqs,

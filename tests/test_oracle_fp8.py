@@ -201,14 +201,15 @@ def test_kv_append_fp8_planted_mistakes_are_caught(monkeypatch):
     assert not survivors, f"mutants that survived the pin: {survivors}"
 
 
-def test_decode_over_full_range_codes_needs_p_as_hi_and_lo():
-    """Why the e4m3 decode kernel feeds the softmax weights P to its f16
-    tensor-core products as two halves (hi + lo) rather than one f16 value:
-    over pools whose codes span the whole e4m3 range (V up to 448 * v_scale),
-    a single f16 P (11 significant bits) misses the 2e-3 output tolerance,
-    while hi + lo (about 22 bits) stays far inside it.  Both products are
+def test_decode_over_full_range_codes_needs_p_beyond_f16():
+    """How precise the softmax weights P must be when they meet e4m3 V in a
+    tensor-core product: over pools whose codes span the whole e4m3 range (V
+    up to 448 * v_scale), a single f16 P (11 significant bits) misses the
+    2e-3 output tolerance, while P as two f16 halves (hi + lo, about 22 bits)
+    stays far inside it.  (The e4m3 decode kernel carries P as four e4m3
+    terms, about 16 bits: tests/test_fp8_terms.py.)  Both products are
     simulated here in float64 from the rounded weights, the sum of weights in
-    fp32 as the kernel keeps it; the reference is the oracle's definition."""
+    fp32; the reference is the oracle's definition."""
     rng = np.random.default_rng(5)
 
     def codes(shape):
@@ -233,5 +234,5 @@ def test_decode_over_full_range_codes_needs_p_as_hi_and_lo():
         tol = 2e-3 * np.maximum(1.0, np.abs(ref))
         worst_single = max(worst_single, float(np.max(np.abs(hi @ V / den - ref) / tol)))
         worst_pair = max(worst_pair, float(np.max(np.abs((hi + lo) @ V / den - ref) / tol)))
-    assert worst_single > 1.0, "a single f16 P would meet the tolerance here: the lo half would be unnecessary"
+    assert worst_single > 1.0, "a single f16 P would meet the tolerance here"
     assert worst_pair < 0.05
