@@ -162,7 +162,10 @@ __device__ __forceinline__ uint32_t e4m3_pair(float x0, float x1, float& d0, flo
 
 }  // namespace t8
 
-template <int G, int NSt>
+// kStall: the instance that honours DecodeParams::stall_cta (the test of the
+// bounded waits: that CTA's producer issues no copy for its first work unit);
+// production launches use the instance without the check.
+template <int G, int NSt, bool kStall = false>
 __global__ void __launch_bounds__(t8::kThreads, NSt <= 2 ? 3 : (NSt == 3 ? 2 : 1))
     decode_tc8_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v) {
@@ -233,8 +236,9 @@ __global__ void __launch_bounds__(t8::kThreads, NSt <= 2 ? 3 : (NSt == 3 ? 2 : 1
     };
     prefetch(unit_index(0));
     bool ok = true;
-    int j = 0;  // chunks issued by this CTA
+    int j = 0, skipped = 0;  // ring uses so far; the first `skipped` of them carried no copy
     for (int r = 0, w = unit_index(0); w < n_work && ok; w = unit_index(++r)) {
+      const bool stall = kStall && r == 0 && p.stall_cta == static_cast<int>(blockIdx.x);
       const WorkUnit u = un;
       int32_t tab = tab_n;
       int wb = 0;
@@ -265,6 +269,11 @@ __global__ void __launch_bounds__(t8::kThreads, NSt <= 2 ? 3 : (NSt == 3 ? 2 : 1
                                    : true,
                          0);
         if (!ok) break;
+        if (stall) {  // nothing lands in this stage: the MMA warp's wait for it runs out
+          ++skipped;
+          ++j;
+          continue;
+        }
         if (lane == 0) mbar_arrive_expect_tx(bar(L::kBFull + s), static_cast<uint32_t>(nbox * box_rows * t8::kD * 2));
         __syncwarp();
         if (lane < nbox) {
@@ -283,6 +292,7 @@ __global__ void __launch_bounds__(t8::kThreads, NSt <= 2 ? 3 : (NSt == 3 ? 2 : 1
       // no copy may still be landing when the CTA exits: the last fill of each stage
       for (int s = 0; s < NSt && s < j; ++s) {
         const int last = s + (j - 1 - s) / NSt * NSt;
+        if (last < skipped) continue;  // its last use carried no copy
         mbar_drain(bar(L::kBFull + s), (last / NSt) & 1);
       }
     }

@@ -786,19 +786,23 @@ template <int G>
 int launch_decode_tc8(const pkv::DecodeParams& base, const int32_t* seq_lens, int32_t num_seqs, int32_t max_tokens,
                       const PendingAppend* ap, cudaStream_t stream) {
   pkv::DecodeParams p = base;
+  apply_debug(p);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   constexpr int NSt = tc8_stages(G);
   const size_t smem = pkv::t8::Layout<NSt, G>::kSmemBytes;
   auto kern = pkv::decode_tc8_kernel<G, NSt>;
+  auto kern_stall = pkv::decode_tc8_kernel<G, NSt, true>;  // the bounded-wait test instance
   static std::atomic<int> occ_cache[kMaxDevices];
   int occ = dev < kMaxDevices ? occ_cache[dev].load(std::memory_order_relaxed) : 0;
   if (occ == 0) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_tc8)");
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(carveout)");
+    for (auto k : {kern, kern_stall}) {
+      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_tc8)");
+      e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(carveout)");
+    }
     // CTAs per SM from the SM's shared memory (the occupancy query counts
     // one CTA where two fit: measured, two are co-resident and run 1.6x as
     // fast); the launch bounds keep the registers of that many CTAs within
@@ -822,8 +826,8 @@ int launch_decode_tc8(const pkv::DecodeParams& base, const int32_t* seq_lens, in
   if (rc) return rc;
   const int64_t work_upper = int64_t(num_seqs) * p.max_parts * p.num_kv_heads;
   const int grid = static_cast<int>(std::min<int64_t>(int64_t(sm_count(dev)) * occ, work_upper));
-  return launch_plan_decode_merge<128>(p, seq_lens, num_seqs, max_tokens, ap, kern, grid, pkv::t8::kThreads, smem,
-                                       stream, mk, mv);
+  return launch_plan_decode_merge<128>(p, seq_lens, num_seqs, max_tokens, ap, p.stall_cta >= 0 ? kern_stall : kern,
+                                       grid, pkv::t8::kThreads, smem, stream, mk, mv);
 }
 
 // ===========================================================================

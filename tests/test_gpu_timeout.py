@@ -56,6 +56,41 @@ def test_stalled_unit_times_out_and_next_call_is_correct(native, dtype, g):
     assert_close(out, case.oracle(), dtype, f"{dtype} G={g} after the timed-out call")
 
 
+def test_stalled_unit_times_out_e4m3_kernel(native):
+    """The same on the tcgen05 e4m3 kernel: the stalled CTA's MMA warp gives up
+    waiting for its first chunk's tiles, raises the abort flag, and the
+    softmax warps and the producer (blocked on a stage that never frees)
+    leave with it."""
+    import numpy as np
+    import paged_kv_cache_406_b200 as P
+    from test_gpu_fp8 import Fp8Case
+    # 4 sequences x 4 partitions of 512 tokens x 2 KV heads = 32 units, one per
+    # CTA; a unit spans 4 chunks of 128 tokens, more than the ring's 2 stages
+    case = Fp8Case([2048] * 4, 8, 2, 16, seed=406)
+    ref = case.oracle()
+    case.gpu()  # first launch: module load and tensor maps outside the timing
+    assert P.pkv_device_status(clear=True) == 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    P.pkv_debug_stall_decode(0)
+    try:
+        t0 = time.perf_counter()
+        e0.record()
+        case.gpu()
+        e1.record()
+        status = P.pkv_device_status(clear=True)
+        wall = time.perf_counter() - t0
+    finally:
+        P.pkv_debug_stall_decode(-1)
+    assert status == PKV_ERR_DEVICE_TIMEOUT
+    ms = e0.elapsed_time(e1)
+    assert 900.0 < ms < 1600.0, f"the stalled call took {ms:.1f} ms on the device"
+    assert wall < 10.0
+    out = case.gpu()
+    assert P.pkv_device_status(clear=True) == 0
+    assert_close(out, ref, "f16", "e4m3 after the timed-out call")
+    assert np.isfinite(out.cpu().numpy()).all()
+
+
 def test_stall_setting_is_off_by_default(native):
     import paged_kv_cache_406_b200 as P
     case = Case([700, 1500], 8, 2, 128, 16, "bf16", seed=405)
