@@ -589,10 +589,12 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize()
         e0.record()
+        h0 = time.perf_counter()
         for s in range(E):
             qh, kh, vh = host_in[s % len(host_in)]
             cache.decode_step_host(ids_np, qh, kh, vh, w.scale, out_host=out_host,
                                    partition_tokens=w.partition_tokens)
+        host_ms = (time.perf_counter() - h0) * 1e3
         cache.wait_copies()  # the last step's result copy back is inside the timed region
         e1.record()
         torch.cuda.synchronize()
@@ -603,6 +605,7 @@ def run_ours(args):
         e2e = {"value": round(e2e_bytes_all / (e2e_ms_all * 1e-3) / 1e9, 2), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(B * hq * d * 4),
                "ms_per_step": round(e2e_ms_all / E, 4),
+               "host_issue_ms_per_step": round(host_ms / E, 4),
                "tokens_per_s_per_layer": round(ws * B * E / (e2e_ms_all * 1e-3), 1),
                "includes": "one pkv_decode_step_host call per step: host slot reservation, pinned H2D of q/K/V rows and "
                            "metadata, kernels, D2H of out"}
