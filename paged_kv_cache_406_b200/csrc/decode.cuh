@@ -711,4 +711,94 @@ __global__ void __launch_bounds__(256) merge_kernel(const int32_t* __restrict__ 
   for (int i = 0; i < kPer; ++i) dst[i] = acc[i] * inv;
 }
 
+// ---------------------------------------------------------------------------
+// merge for batches whose sequences can span more than 32 partitions (long
+// contexts): one CTA per (sequence, query head), its 8 warps each merging a
+// contiguous eighth of the partitions against their own max, then warp 0
+// combining the 8 records (max, sum, row) the same way.  A warp per row
+// walked the 256 partitions of a 128K-token sequence one after another.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) merge_wide_kernel(const int32_t* __restrict__ seq_lens, int32_t num_seqs,
+                                                         int32_t num_q_heads, int32_t max_tokens, int32_t part_tokens,
+                                                         int32_t max_parts, const float* __restrict__ part_m,
+                                                         const float* __restrict__ part_l,
+                                                         const float* __restrict__ part_o, float* __restrict__ out) {
+  constexpr int kPer = D / 32;
+  __shared__ float rec_m[8], rec_l[8];
+  __shared__ float rec_o[8][D];
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int row = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (row >= num_seqs * num_q_heads) return;
+  int L = seq_lens[row / num_q_heads];
+  L = L < 0 ? 0 : (L > max_tokens ? max_tokens : L);
+  if (L <= part_tokens) return;  // one partition: written by the decode kernel (uniform over the CTA)
+  const int np = (L + part_tokens - 1) / part_tokens;
+  const int per = (np + 7) / 8, q0 = warp * per, q1 = min(np, q0 + per);  // this warp's partitions
+  const int64_t base = static_cast<int64_t>(row) * max_parts;
+  float M = -INFINITY;
+  for (int q = q0 + lane; q < q1; q += 32) M = fmaxf(M, part_m[base + q]);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+  float acc[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) acc[i] = 0.f;
+  float den = 0.f;
+  for (int g0 = q0; g0 < q1; g0 += 32) {
+    const int nq = min(32, q1 - g0);
+    const float f_mine = lane < nq ? fast_exp2(part_m[base + g0 + lane] - M) : 0.f;
+    den += lane < nq ? f_mine * part_l[base + g0 + lane] : 0.f;
+    const float* o = part_o + (base + g0) * D + lane * kPer;
+    int j = 0;
+    for (; j + 4 <= nq; j += 4) {
+      float v[4][kPer];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) v[t][i] = o[(j + t) * D + i];
+      }
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float f = __shfl_sync(kFull, f_mine, j + t);
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) acc[i] += f * v[t][i];
+      }
+    }
+    for (; j < nq; ++j) {
+      const float f = __shfl_sync(kFull, f_mine, j);
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) acc[i] += f * o[j * D + i];
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(kFull, den, o);
+  if (lane == 0) {
+    rec_m[warp] = M;  // -inf for a warp without partitions
+    rec_l[warp] = den;
+  }
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) rec_o[warp][lane * kPer + i] = acc[i];
+  __syncthreads();
+  if (warp != 0) return;
+  float Mt = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) Mt = fmaxf(Mt, rec_m[w]);
+  float res[kPer], dt = 0.f;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) res[i] = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    const float f = rec_m[w] == -INFINITY ? 0.f : fast_exp2(rec_m[w] - Mt);
+    dt += f * rec_l[w];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) res[i] += f * rec_o[w][lane * kPer + i];
+  }
+  const float inv = dt > 0.f ? 1.f / dt : 0.f;
+  float* dst = out + static_cast<int64_t>(row) * D + lane * kPer;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) dst[i] = res[i] * inv;
+}
+
 }  // namespace pkv

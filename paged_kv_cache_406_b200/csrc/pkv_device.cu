@@ -224,10 +224,13 @@ int launch_plan_decode_merge(const pkv::DecodeParams& p, const int32_t* seq_lens
   e = launch_pdl(kern, dim3(grid), dim3(threads), smem, stream, p, args...);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   if (p.max_parts > 1) {
+    // a warp per (sequence, query head), or a CTA when a sequence can span
+    // more than 32 partitions
     const int rows = num_seqs * p.num_q_heads;
-    e = launch_pdl(pkv::merge_kernel<D>, dim3((rows + 7) / 8), dim3(256), 0, stream, seq_lens, num_seqs,
-                   p.num_q_heads, max_tokens, p.partition_tokens, p.max_parts,
-                   static_cast<const float*>(p.part_m), static_cast<const float*>(p.part_l),
+    const bool wide = p.max_parts > 32;
+    e = launch_pdl(wide ? pkv::merge_wide_kernel<D> : pkv::merge_kernel<D>, dim3(wide ? rows : (rows + 7) / 8),
+                   dim3(256), 0, stream, seq_lens, num_seqs, p.num_q_heads, max_tokens, p.partition_tokens,
+                   p.max_parts, static_cast<const float*>(p.part_m), static_cast<const float*>(p.part_l),
                    static_cast<const float*>(p.part_o), p.out);
     if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   }
