@@ -15,30 +15,42 @@
 //
 //   S_j = Q · K_jᵀ        tcgen05.mma, 128x128x128, A and B from shared memory,
 //                         fp32 in tensor memory
-//   P_j = 2^(S_j·scale·log2e - m)   4 softmax warps, one row per thread,
-//                         written back over S_j as bf16 hi + lo, or one f16
-//   O  += P_j · V_j       tcgen05.mma, A (P) from tensor memory, B (V) from
-//                         shared memory
+//   P_j = 2^(S_j·scale·log2e - m_h)   8 softmax warps in two warpgroups: warp-
+//                         group h takes keys [64h, 64h + 64) of every chunk,
+//                         one row per thread, with its own running max m_h;
+//                         P written back over its half of S_j as bf16 hi +
+//                         lo, or one f16
+//   O_h += P_j,h · V_j,h  tcgen05.mma per half, A (P) from tensor memory, B
+//                         (V rows of that half) from shared memory; two
+//                         accumulators, combined once per tile:
+//                         O = (2^(m_0-M) O_0 + 2^(m_1-M) O_1) / (2^(m_0-M) l_0 + 2^(m_1-M) l_1)
 //
-// Warp roles (224 threads): warps 0-3 softmax (thread = row = TMEM lane),
-// warps 4 and 5 TMA producers (K, V), warp 6 MMA issuer (lane 0) and TMEM
-// owner.  Tensor
-// memory (512 columns): three S / P buffers at columns 0, 128 and 256 (P hi
-// in the first 64 columns of its buffer, P lo in the next 64; a single f16 P
-// in the first 64), O at 384.
-// Shared memory: Q 32 KB, K and V rings of 32 KB stages and a 64 KB staging
-// buffer for the output rows.  Keeping P in tensor memory spares shared
-// memory 128 KB of traffic per chunk (P written and read back), which bounded
-// the first version of this kernel.
+// The two halves share nothing during a tile (no exchange of maxima per
+// chunk), and two softmax warps per SM sub-partition hide each other's
+// latencies: the per-row chain (tensor-memory load, max, 64 exponentials, P
+// store) was the bound with one warp per sub-partition and all 128 keys per
+// row.
 //
-// Pipeline: the MMA warp issues S_0, S_1, S_2, then per chunk PV_j followed
-// by S_{j+3}, so q·Kᵀ of the next chunks runs while the softmax warps work
-// on the current one and the tensor core has the next chunk's P·V ready
-// while waiting for this one's P.  The commit of S_j covers every earlier
-// MMA, so by the time a softmax warp sees S_j, PV_{j-3} (the last reader of
-// that buffer) is done and P_j can overwrite it at once.  The running max moves lazily
-// (only by more than 8 in log2 units), as in the decode kernels; a move
-// rescales that row's O in tensor memory after PV_{j-1} has finished.
+// Warp roles (352 threads): warps 0-7 softmax (thread = row = TMEM lane of
+// its warp's lane quarter, warp mod 4), warps 8 and 9 TMA producers (K, V),
+// warp 10 MMA issuer (lane 0) and TMEM owner.  Tensor memory (512 columns):
+// two S / P buffers at columns 0 and 128 (half h in columns 64h .. 64h + 63
+// of a buffer: P hi in the first 32, P lo in the next 32; a single f16 P in
+// the first 32), O_0 at 256, O_1 at 384.
+// Shared memory: Q 32 KB, K and V rings of 32 KB stages, a 64 KB staging
+// buffer for the output rows and 1 KB through which the two warpgroups
+// exchange (max, sum) per row at the end of a tile.  Keeping P in tensor
+// memory spares shared memory 128 KB of traffic per chunk (P written and read
+// back), which bounded the first version of this kernel.
+//
+// Pipeline: the MMA warp issues S_0, S_1, then per chunk PV_j (each half as
+// soon as its P is written) followed by S_{j+2}, so q·Kᵀ of the next chunk
+// runs while the softmax warps work on the current one.  The commit of S_j
+// covers every earlier MMA, so by the time a softmax warp sees S_j, PV_{j-2}
+// (the last reader of that buffer) is done and P_j can overwrite it at once.
+// The running max moves lazily (only by more than 8 in log2 units), as in the
+// decode kernels; a move rescales that half's O in tensor memory after
+// PV_{j-1} has finished.
 //
 // P precision: a single bf16 P (8 significant bits) misses the 2e-3 output
 // tolerance at early positions (few keys of comparable weight), so for bf16
@@ -88,36 +100,42 @@ constexpr int kHeadDim = 128;
 constexpr uint32_t kSlab = 128 * 128;   // 128 rows x 64 elements x 2 bytes
 constexpr uint32_t kTile = 2 * kSlab;   // 128 rows x head_dim 128
 constexpr int kStages = PKV_PREFILL_STAGES;  // K and V ring depth
-constexpr int kProducerK = 4, kProducerV = 5, kMmaWarp = 6;
-constexpr int kThreads = 224;
+constexpr int kHalf = kKeys / 2;        // keys of one softmax warpgroup per chunk
+constexpr int kSoftmaxThreads = 256;    // warps 0-7
+constexpr int kProducerK = 8, kProducerV = 9, kMmaWarp = 10;
+constexpr int kThreads = 352;
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kTile;
 constexpr uint32_t kOffV = kOffK + kStages * kTile;
 constexpr uint32_t kOffStage = kOffV + kStages * kTile;  // output rows on their way out (128 x 512 B)
 constexpr uint32_t kOffBar = kOffStage + kRows * kHeadDim * 4;
-constexpr size_t kSmemBytes = kOffBar + 256 + 1024;  // barriers, flags; 1024 B alignment slack
+constexpr uint32_t kOffXchg = kOffBar + 256;  // 128 rows x (float, float): the halves' (max, sum), then weights
+constexpr size_t kSmemBytes = kOffXchg + 1024 + 1024;  // barriers, flags, exchange; 1024 B alignment slack
 static_assert(kSmemBytes <= 227 * 1024, "one CTA's shared memory (227 KB at most on sm_100)");
 constexpr uint32_t kTmemCols = 512;
-constexpr int kSBufs = 3;                    // S / P buffers in tensor memory
-constexpr uint32_t kColS = 0, kColO = 384;   // S / P: 3 x 128 columns, O: 128
+constexpr int kSBufs = 2;                    // S / P buffers in tensor memory
+constexpr uint32_t kColS = 0, kColO = 256;   // S / P: 2 x 128 columns; O_h at 256 + 128 h
 constexpr float kRescale = 8.0f;
 constexpr unsigned kAll = 0xffffffffu;
 // mbarrier slots
 enum : int { kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = kKFull + kStages, kVFull = kKEmpty + kStages,
              kVEmpty = kVFull + kStages, kSFull = kVEmpty + kStages, kPFull = kSFull + kSBufs,
-             kPVDone = kPFull + kSBufs, kODone = kPVDone + kSBufs, kOFree = kODone + 1, kTileReady = kOFree + 1,
-             kTileFree = kTileReady + 2, kDrain = kTileFree + 2, kNumBars = kDrain + 1 };
+             kPVDone = kPFull + 2 * kSBufs, kODone = kPVDone + kSBufs, kOFree = kODone + 1, kXFull = kOFree + 1,
+             kXBack = kXFull + 1, kTileReady = kXBack + 1, kTileFree = kTileReady + 2, kDrain = kTileFree + 2,
+             kNumBars = kDrain + 1 };
 static_assert(kNumBars * 8 + 16 <= 256, "barriers, flags and tile slots fit the reserved 256 bytes");
-// arrivals per phase: P-full and O-free by the 128 softmax threads, tile-free
-// by lane 0 of the V producer, the MMA warp and the four softmax warps
+// arrivals per phase: P-full (one per buffer and half) and the exchange by
+// one warpgroup's 128 threads, O-free by all 256 softmax threads, tile-free by
+// lane 0 of the V producer, the MMA warp and the eight softmax warps
 __host__ __device__ constexpr uint32_t bar_count(int i) {
-  return (i >= kPFull && i < kPFull + kSBufs) || i == kOFree ? 128u
-         : (i >= kTileFree && i < kTileFree + 2)           ? 6u
-                                                             : 1u;
+  return (i >= kPFull && i < kPFull + 2 * kSBufs) || i == kXFull || i == kXBack ? 128u
+         : i == kOFree                                                         ? 256u
+         : (i >= kTileFree && i < kTileFree + 2)                               ? 10u
+                                                                               : 1u;
 }
-// S-full, P-full and PV-done are one barrier per S / P buffer: a buffer's
-// next phase needs the MMA warp to have moved on (S_{j+3} is issued after
-// PV_j), so no waiter can ever be a whole phase behind
+// S-full, P-full and PV-done are barriers per S / P buffer: a buffer's next
+// phase needs the MMA warp to have moved on (S_{j+2} is issued after PV_j),
+// so no waiter can ever be a whole phase behind
 }  // namespace pf
 
 __device__ __forceinline__ void tma_load_3d_nohint(uint32_t dst, const void* tmap, int32_t x, int32_t y, int32_t z,
@@ -483,21 +501,27 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         for (int j = 0; j < nc && ok; ++j) {
           const int gj = gc + j;
           const int s = gj % pf::kStages;
-          ok = mbar_wait_sleep(bar(pf::kPFull + gj % pf::kSBufs), (gj / pf::kSBufs) & 1, abort_flag) &&
-               mbar_wait_sleep(bar(pf::kVFull + s), (gj / pf::kStages) & 1, abort_flag);
-          if (!ok) break;
-          tc::fence_after_sync();
+          ok = mbar_wait_sleep(bar(pf::kVFull + s), (gj / pf::kStages) & 1, abort_flag);
           const uint32_t vst = base + pf::kOffV + s * pf::kTile;
-          const uint32_t pt = tmem + pf::kColS + (gj % pf::kSBufs) * pf::kKeys;  // P hi: 64 columns, then P lo
+          const uint32_t pt = tmem + pf::kColS + (gj % pf::kSBufs) * pf::kKeys;
+          // each half's P·V as soon as its warpgroup has written P (P hi in
+          // the half's first 32 columns, P lo in the next 32)
 #pragma unroll
-          for (int part = 0; part < parts; ++part) {
+          for (int hf = 0; hf < 2 && ok; ++hf) {
+            ok = mbar_wait_sleep(bar(pf::kPFull + 2 * (gj % pf::kSBufs) + hf), (gj / pf::kSBufs) & 1, abort_flag);
+            if (!ok) break;
+            tc::fence_after_sync();
 #pragma unroll
-            for (int kk = 0; kk < pf::kKeys / 16; ++kk) {
-              const uint32_t bv = vst + kk * 16 * 128;  // 16 keys of 128-byte rows
-              tc::mma_f16_ts(tmem + pf::kColO, pt + part * (pf::kKeys / 2) + kk * 8, tc::sw128_desc(bv, pf::kSlab, 1024),
-                             id_o, (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
+            for (int part = 0; part < parts; ++part) {
+#pragma unroll
+              for (int kk = 0; kk < pf::kHalf / 16; ++kk) {
+                const uint32_t bv = vst + (hf * pf::kHalf + kk * 16) * 128;  // 16 keys of 128-byte rows
+                tc::mma_f16_ts(tmem + pf::kColO + hf * pf::kHeadDim, pt + hf * pf::kHalf + part * (pf::kHalf / 2) + kk * 8,
+                               tc::sw128_desc(bv, pf::kSlab, 1024), id_o, (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
+              }
             }
           }
+          if (!ok) break;
           tc::commit(bar(pf::kVEmpty + s));
           tc::commit(bar(pf::kPVDone + gj % pf::kSBufs));
           if (j + pf::kSBufs < nc) {
@@ -523,9 +547,15 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------ softmax warps ------------------------------
-    const int r = threadIdx.x;  // tile row and TMEM lane
-    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    // warpgroup hf takes keys [64 hf, 64 hf + 64) of every chunk of the tile
+    const int hf = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;  // tile row and TMEM lane
+    const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t tsp = trow + pf::kColS + hf * pf::kHalf;     // this half's S / P columns in buffer 0
+    const uint32_t to = trow + pf::kColO + hf * pf::kHeadDim;   // this half's O
+    const uint32_t to_cols = trow + pf::kColO + hf * pf::kHalf;  // output columns [64 hf, 64 hf + 64) of O_0
     unsigned char* vzero = smem + pf::kOffV;
+    float2* xch = reinterpret_cast<float2*>(smem + pf::kOffXchg) + r;
     const float sl = p.scale_log2;
     bool ok = true;
     int gc = 0, tv = 0;
@@ -537,6 +567,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       const int nc = d.nc, L = d.L, n = d.n, tok0 = d.tok0, pos_min = d.pos_min;
       const int tok = tok0 + r / G;
       const int pos = min(d.ctx + tok, L - 1);  // rows past the chunk end compute a copy of the last row
+      // running max (-inf until a key of this half is visible to the row) and sum
       float m_used = -INFINITY, l = 0.f;
       for (int j = 0; j < nc && ok; ++j) {
         const int gj = gc + j;              // chunk of the CTA
@@ -545,73 +576,76 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kSFull + sb), (gj / pf::kSBufs) & 1, abort_flag));
         if (!ok) break;
         tc::fence_after_sync();
-        float x[pf::kKeys];  // raw scores q·k of this row's 128 keys
+        float x[pf::kHalf];  // raw scores q·k of this row's 64 keys
         {
-          uint32_t raw[4][32];
+          uint32_t raw[2][32];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) tc::ld_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + 32 * q, raw[q]);
+          for (int q = 0; q < 2; ++q) tc::ld_32x32b_x32(tsp + sb * pf::kKeys + 32 * q, raw[q]);
           tc::wait_ld();
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
+          for (int q = 0; q < 2; ++q)
 #pragma unroll
             for (int i = 0; i < 32; ++i) x[32 * q + i] = __uint_as_float(raw[q][i]);
         }
-        const int key0 = j * pf::kKeys;
-        if (key0 + pf::kKeys - 1 > pos_min) {  // the diagonal: keys after a row's position are hidden
+        const int key0 = j * pf::kKeys + hf * pf::kHalf;  // this half's first key
+        if (key0 + pf::kHalf - 1 > pos_min) {  // the diagonal: keys after a row's position are hidden
 #pragma unroll
-          for (int c = 0; c < pf::kKeys; ++c) x[c] = key0 + c <= pos ? x[c] : -INFINITY;
+          for (int c = 0; c < pf::kHalf; ++c) x[c] = key0 + c <= pos ? x[c] : -INFINITY;
         }
         // row max with three-input maxima in four independent chains; the
         // scale is positive, so the max of the scaled scores is the scaled max
         float mx[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-        for (int c = 4; c + 8 <= pf::kKeys; c += 8) {
+        for (int c = 4; c + 8 <= pf::kHalf; c += 8) {
           mx[0] = max3f(mx[0], x[c], x[c + 1]);
           mx[1] = max3f(mx[1], x[c + 2], x[c + 3]);
           mx[2] = max3f(mx[2], x[c + 4], x[c + 5]);
           mx[3] = max3f(mx[3], x[c + 6], x[c + 7]);
         }
-        mx[0] = max3f(mx[0], x[pf::kKeys - 4], x[pf::kKeys - 3]);
-        mx[1] = max3f(mx[1], x[pf::kKeys - 2], x[pf::kKeys - 1]);
-        const float mc = fmaxf(max3f(mx[0], mx[1], mx[2]), mx[3]) * sl;
+        mx[0] = max3f(mx[0], x[pf::kHalf - 4], x[pf::kHalf - 3]);
+        mx[1] = max3f(mx[1], x[pf::kHalf - 2], x[pf::kHalf - 1]);
+        const float mc = fmaxf(max3f(mx[0], mx[1], mx[2]), mx[3]) * sl;  // -inf: no visible key here
         float factor = 1.f;
         bool resc = false;
-        if (j == 0) {
-          m_used = mc;  // key 0 is visible to every row: finite
-        } else if (mc > m_used + pf::kRescale) {
-          factor = fast_exp2(m_used - mc);
+        if (mc > m_used + pf::kRescale) {
+          // the first visible keys of this half only set the max (O_h and l
+          // are still zero); later moves rescale both
+          resc = m_used != -INFINITY;
+          if (resc) factor = fast_exp2(m_used - mc);
           m_used = mc;
-          resc = true;
         }
         // exponentials (arguments and sums two lanes at a time, packed f32x2),
-        // each half of the row written as P hi and lo over S_j in tensor memory
-        // as soon as it is done (the stores complete while the next half is
-        // computed): key pair (2c, 2c+1) in column c (hi) and 64 + c (lo)
+        // each quarter of the row written as P over S_j in tensor memory as
+        // soon as it is done (the stores complete while the next quarter is
+        // computed): key pair (2c, 2c+1) of the half in column c (hi) and
+        // 32 + c (lo) of the half's columns
         float2 sm[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(-m_used, -m_used);
+        const float2 sl2 = make_float2(sl, sl);
+        const float nm = m_used == -INFINITY ? 0.f : -m_used;  // no visible key: every argument stays -inf
+        const float2 nm2 = make_float2(nm, nm);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
 #pragma unroll
-          for (int c = 64 * h; c < 64 * h + 64; c += 2) {
+          for (int c = 32 * h; c < 32 * h + 32; c += 2) {
             const float2 a = __ffma2_rn(make_float2(x[c], x[c + 1]), sl2, nm2);  // hidden keys: -inf -> 0
             x[c] = fast_exp2(a.x);
             x[c + 1] = fast_exp2(a.y);
             sm[(c >> 1) & 3] = __fadd2_rn(sm[(c >> 1) & 3], make_float2(x[c], x[c + 1]));
           }
           if constexpr (!f16p) {
-            uint32_t hi[32], lo[32];
+            uint32_t hi[16], lo[16];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) split_hi_lo<T>(x[64 * h + 2 * c], x[64 * h + 2 * c + 1], hi[c], lo[c]);
-            tc::st_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + 32 * h, hi);
-            tc::st_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + pf::kKeys / 2 + 32 * h, lo);
+            for (int c = 0; c < 16; ++c) split_hi_lo<T>(x[32 * h + 2 * c], x[32 * h + 2 * c + 1], hi[c], lo[c]);
+            tc::st_32x32b_x16(tsp + sb * pf::kKeys + 16 * h, hi);
+            tc::st_32x32b_x16(tsp + sb * pf::kKeys + pf::kHalf / 2 + 16 * h, lo);
           } else {
-            uint32_t ph[32];
+            uint32_t ph[16];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const __half2 v = __floats2half2_rn(x[64 * h + 2 * c], x[64 * h + 2 * c + 1]);
+            for (int c = 0; c < 16; ++c) {
+              const __half2 v = __floats2half2_rn(x[32 * h + 2 * c], x[32 * h + 2 * c + 1]);
               ph[c] = *reinterpret_cast<const uint32_t*>(&v);
             }
-            tc::st_32x32b_x32(trow + pf::kColS + sb * pf::kKeys + 32 * h, ph);
+            tc::st_32x32b_x16(tsp + sb * pf::kKeys + 16 * h, ph);
           }
         }
         const float2 s01 = __fadd2_rn(sm[0], sm[1]), s23 = __fadd2_rn(sm[2], sm[3]);
@@ -619,10 +653,10 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         l = l * factor + (st.x + st.y);
 
         if (__any_sync(pf::kAll, resc)) {
-          // O still accumulates PV_{j-1}: wait for it, then rescale the row.
+          // O_h still accumulates PV_{j-1}: wait for it, then rescale the row.
           // PV_{j-1} commits to the barrier of its buffer, whose previous
-          // phase (PV_{j-4}) was covered by S_j's commit, so the parity wait
-          // cannot see an older phase.
+          // phase (PV_{j-3}) was covered by S_{j-1}'s commit, so the parity
+          // wait cannot see an older phase.
           const int pj = gj - 1;
           ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kPVDone + pj % pf::kSBufs), (pj / pf::kSBufs) & 1, abort_flag));
           if (!ok) break;
@@ -630,22 +664,22 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             uint32_t o[32];
-            tc::ld_32x32b_x32(trow + pf::kColO + 32 * q, o);
+            tc::ld_32x32b_x32(to + 32 * q, o);
             tc::wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
-            tc::st_32x32b_x32(trow + pf::kColO + 32 * q, o);
+            tc::st_32x32b_x32(to + 32 * q, o);
           }
         }
-        const bool zero_v = key0 + pf::kKeys > L;
-        if (zero_v) {
-          // V rows past the sequence end hold stale or unwritten bytes: zero
-          // them so that P = 0 there cannot meet a NaN pattern
+        const int vend = j * pf::kKeys + (hf + 1) * pf::kHalf;  // one past this half's last key
+        if (vend > L) {
+          // V rows of this half past the sequence end hold stale or unwritten
+          // bytes: zero them so that P = 0 there cannot meet a NaN pattern
           ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kVFull + s), (gj / pf::kStages) & 1, abort_flag));
           if (!ok) break;
-          const int v0 = L - key0;
+          const int v0 = max(L - j * pf::kKeys, hf * pf::kHalf);  // first row to zero, chunk-relative
           unsigned char* vst = vzero + s * pf::kTile;
-          for (int idx = r; idx < (pf::kKeys - v0) * 16; idx += 128) {
+          for (int idx = r; idx < ((hf + 1) * pf::kHalf - v0) * 16; idx += 128) {
             const int row = v0 + (idx >> 4), piece = idx & 15;
             *reinterpret_cast<uint4*>(vst + (piece >> 3) * pf::kSlab + row * 128 + (piece & 7) * 16) =
                 make_uint4(0u, 0u, 0u, 0u);
@@ -654,46 +688,79 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         }
         tc::wait_st();
         tc::fence_before_sync();
-        mbar_arrive(bar(pf::kPFull + sb));
+        mbar_arrive(bar(pf::kPFull + 2 * sb + hf));
       }
       // the MMA warp commits O-done after the tile's last P·V
       if (ok) ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kODone), tv & 1, abort_flag));
       if (!ok) break;
       tc::fence_after_sync();
-      // O leaves tensor memory first (the next tile's P·V may then overwrite
-      // it), then goes out through shared memory: each thread parks its row,
-      // and each warp writes its 32 rows one 512-byte row per store
-      // instruction, instead of 32 rows per instruction straight from the
-      // tensor-memory layout.  The 16-byte piece c of row r sits at slot
-      // c ^ (r mod 8) of the row, so the row-wise writes and the piece-wise
-      // reads are both free of bank conflicts.
-      uint32_t o[4][32];
+      // this warpgroup writes output columns [64 hf, 64 hf + 64) of its rows:
+      // both accumulators leave tensor memory first (the next tile's P·V may
+      // then overwrite them)
+      uint32_t o0[2][32], o1[2][32];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) tc::ld_32x32b_x32(trow + pf::kColO + 32 * q, o[q]);
+      for (int q = 0; q < 2; ++q) {
+        tc::ld_32x32b_x32(to_cols + 32 * q, o0[q]);
+        tc::ld_32x32b_x32(to_cols + pf::kHeadDim + 32 * q, o1[q]);
+      }
       tc::wait_ld();
       tc::fence_before_sync();
       mbar_arrive(bar(pf::kOFree));
-      const float inv = 1.f / l;
+      // weights of the two halves: warpgroup 1 hands its (max, sum) to
+      // warpgroup 0 through shared memory, which returns both weights with
+      // the normalisation folded in; key 0 is visible to every row, so m_0
+      // is finite and the total positive
+      float c0, c1;
+      if (hf == 1) {
+        *xch = make_float2(m_used, l);
+        mbar_arrive(bar(pf::kXFull));
+        ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kXBack), tv & 1, abort_flag));
+        if (!ok) break;
+        const float2 w = *xch;
+        c0 = w.x;
+        c1 = w.y;
+      } else {
+        ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kXFull), tv & 1, abort_flag));
+        if (!ok) break;
+        const float2 o = *xch;
+        const float mm = fmaxf(m_used, o.x);
+        const float w0 = fast_exp2(m_used - mm), w1 = fast_exp2(o.x - mm);  // m_1 = -inf: w1 = 0
+        const float inv = 1.f / (l * w0 + o.y * w1);
+        c0 = w0 * inv;
+        c1 = w1 * inv;
+        *xch = make_float2(c0, c1);
+        mbar_arrive(bar(pf::kXBack));
+      }
+      // then out through shared memory: each thread parks its half row, and
+      // each warp writes its 32 half rows two per store instruction, instead
+      // of 32 rows per instruction straight from the tensor-memory layout.
+      // The 16-byte piece c of row r sits at slot c ^ (r mod 8) of the row,
+      // so the row-wise writes and the piece-wise reads are both free of bank
+      // conflicts.
       float4* stage = reinterpret_cast<float4*>(smem + pf::kOffStage);
       float4* srow = stage + r * (pf::kHeadDim / 4);
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
+      for (int q = 0; q < 2; ++q)
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          srow[(8 * q + i) ^ (r & 7)] =
-              make_float4(__uint_as_float(o[q][4 * i]) * inv, __uint_as_float(o[q][4 * i + 1]) * inv,
-                          __uint_as_float(o[q][4 * i + 2]) * inv, __uint_as_float(o[q][4 * i + 3]) * inv);
+        for (int i = 0; i < 8; ++i) {
+          float v[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            v[e] = __uint_as_float(o0[q][4 * i + e]) * c0 + __uint_as_float(o1[q][4 * i + e]) * c1;
+          srow[(16 * hf + 8 * q + i) ^ (r & 7)] = make_float4(v[0], v[1], v[2], v[3]);
+        }
       __syncwarp();
-      for (int k = 0; k < 32; ++k) {
-        const int rr = warp * 32 + k;  // a row this warp parked
+      for (int k = 0; k < 16; ++k) {
+        const int rr = (warp & 3) * 32 + 2 * k + (lane >> 4);  // a row this warp parked
+        const int piece = 16 * hf + (lane & 15);
         const int tk = tok0 + rr / G;
-        if (tk < n) {                  // rows past the chunk end are not written
+        if (tk < n) {  // rows past the chunk end are not written
           float4* orow = reinterpret_cast<float4*>(
               p.out + (static_cast<int64_t>(d.q0 + tk) * p.num_q_heads + d.g * G + rr % G) * pf::kHeadDim);
-          orow[lane] = stage[rr * (pf::kHeadDim / 4) + (lane ^ (rr & 7))];
+          orow[piece] = stage[rr * (pf::kHeadDim / 4) + (piece ^ (rr & 7))];
         }
       }
-      __syncwarp();  // this warp's rows are out of the staging area before the next tile's
+      __syncwarp();  // this warp's half rows are out of the staging area before the next tile's
       gc += nc;
       ++tv;
     }
