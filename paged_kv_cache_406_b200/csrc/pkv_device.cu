@@ -1265,7 +1265,7 @@ extern "C" int pkv_paged_attention_prefill(const void* q, const void* k_pool, co
     return fail(PKV_ERR_INVALID_ARG, "%s: pool rows exceed 2^31", fn);
   if (int64_t(max_blocks_per_seq) * block_size >= (int64_t(1) << 31))
     return fail(PKV_ERR_INVALID_ARG, "%s: max_blocks_per_seq * block_size exceeds 2^31", fn);
-  const int32_t qt = 128 / group;
+  const int32_t qt = pkv::pf::kTileRows / group;  // query tokens per tile
   const int64_t n_tiles = (int64_t(max_q_len) + qt - 1) / qt;
   const int64_t grid = n_tiles * num_seqs * num_kv_heads;
   if (grid >= (int64_t(1) << 31)) return fail(PKV_ERR_INVALID_ARG, "%s: too many tiles (%lld)", fn, (long long)grid);

@@ -7,50 +7,46 @@
 // causally to tokens 0 .. that position through the block table (vLLM paging
 // page §3 phase 2), KV head h / G, fp32 output.
 //
-// A tile is 128 rows = 128/G query tokens x the G query heads of one KV head,
-// so a GQA group turns into a full M = 128 MMA tile even for short chunks;
-// persistent CTAs (one per SM) take tiles one after another.  Keys come in
-// chunks of 128 tokens (128/block_size physical blocks, one TMA box per block
-// and head_dim half).  Per chunk j:
+// A tile is 256 rows = 256/G query tokens x the G query heads of one KV head,
+// in two halves A and B of 128 rows (one M = 128 MMA tile each), so a GQA
+// group turns into full MMA tiles even for short chunks; persistent CTAs (one
+// per SM) take tiles one after another.  Keys come in chunks of 128 tokens
+// (128/block_size physical blocks, one TMA box per block and head_dim half),
+// each loaded once for both halves.  Per chunk j and half h:
 //
-//   S_j = Q · K_jᵀ        tcgen05.mma, 128x128x128, A and B from shared memory,
+//   S_h = Q_h · K_jᵀ      tcgen05.mma, 128x128x128, A and B from shared memory,
 //                         fp32 in tensor memory
-//   P_j = 2^(S_j·scale·log2e - m_h)   8 softmax warps in two warpgroups: warp-
-//                         group h takes keys [64h, 64h + 64) of every chunk,
-//                         one row per thread, with its own running max m_h;
-//                         P written back over its half of S_j as bf16 hi +
-//                         lo, or one f16
-//   O_h += P_j,h · V_j,h  tcgen05.mma per half, A (P) from tensor memory, B
-//                         (V rows of that half) from shared memory; two
-//                         accumulators, combined once per tile:
-//                         O = (2^(m_0-M) O_0 + 2^(m_1-M) O_1) / (2^(m_0-M) l_0 + 2^(m_1-M) l_1)
+//   P_h = 2^(S_h·scale·log2e - m)   4 softmax warps per half, one row per
+//                         thread, written back over S_h as bf16 hi + lo, or one
+//                         f16
+//   O_h += P_h · V_j      tcgen05.mma, A (P) from tensor memory, B (V) from
+//                         shared memory
 //
-// The two halves share nothing during a tile (no exchange of maxima per
-// chunk), and two softmax warps per SM sub-partition hide each other's
-// latencies: the per-row chain (tensor-memory load, max, 64 exponentials, P
-// store) was the bound with one warp per sub-partition and all 128 keys per
-// row.
+// The halves ping-pong: the MMA warp issues P·V of one half and q·Kᵀ of its
+// next chunk as soon as that half's P is written, so the tensor core works on
+// one half while the other half's softmax runs.  With a single 128-row tile,
+// each chunk's P·V waited for the S -> softmax -> P round trip of the same
+// tile, and the tensor core idled half of the time even with no softmax work
+// at all; two halves also load K/V once per 256 rows.
 //
-// Warp roles (352 threads): warps 0-7 softmax (thread = row = TMEM lane of
-// its warp's lane quarter, warp mod 4), warps 8 and 9 TMA producers (K, V),
-// warp 10 MMA issuer (lane 0) and TMEM owner.  Tensor memory (512 columns):
-// two S / P buffers at columns 0 and 128 (half h in columns 64h .. 64h + 63
-// of a buffer: P hi in the first 32, P lo in the next 32; a single f16 P in
-// the first 32), O_0 at 256, O_1 at 384.
-// Shared memory: Q 32 KB, K and V rings of 32 KB stages, a 64 KB staging
-// buffer for the output rows and 1 KB through which the two warpgroups
-// exchange (max, sum) per row at the end of a tile.  Keeping P in tensor
-// memory spares shared memory 128 KB of traffic per chunk (P written and read
-// back), which bounded the first version of this kernel.
+// Warp roles (352 threads): warps 0-3 softmax of half A, 4-7 of half B
+// (thread = row = TMEM lane of its warp's lane quarter, warp mod 4), warps 8
+// and 9 TMA producers (K with Q, V), warp 10 MMA issuer (lane 0) and TMEM
+// owner.  Tensor memory (512 columns): S / P of half h at column 128 h (P hi
+// in the first 64 columns, P lo in the next 64; a single f16 P in the first
+// 64), O of half h at 256 + 128 h.
+// Shared memory: Q of both halves 64 KB, K and V rings of 32 KB stages, and
+// 4 KB per softmax warp through which its output rows leave in 128-byte
+// pieces.  Keeping P in tensor memory spares shared memory 128 KB of traffic
+// per chunk (P written and read back), which bounded the first version of
+// this kernel.
 //
-// Pipeline: the MMA warp issues S_0, S_1, then per chunk PV_j (each half as
-// soon as its P is written) followed by S_{j+2}, so q·Kᵀ of the next chunk
-// runs while the softmax warps work on the current one.  The commit of S_j
-// covers every earlier MMA, so by the time a softmax warp sees S_j, PV_{j-2}
-// (the last reader of that buffer) is done and P_j can overwrite it at once.
-// The running max moves lazily (only by more than 8 in log2 units), as in the
-// decode kernels; a move rescales that half's O in tensor memory after
-// PV_{j-1} has finished.
+// Pipeline per chunk j: P·V_A(j), q·Kᵀ_A(j+1), P·V_B(j), q·Kᵀ_B(j+1).  A half
+// has one S / P buffer: q·Kᵀ of its next chunk overwrites P only after the
+// P·V that reads it (the tensor core runs a thread's MMAs in order), and the
+// commit of S_h(j) covers P·V_h(j-1), so a softmax warp that sees S_h(j) may
+// rescale O_h at once.  The running max moves lazily (only by more than 8 in
+// log2 units), as in the decode kernels.
 //
 // P precision: a single bf16 P (8 significant bits) misses the 2e-3 output
 // tolerance at early positions (few keys of comparable weight), so for bf16
@@ -94,48 +90,45 @@ struct PrefillParams {
 #endif
 
 namespace pf {
-constexpr int kRows = 128;              // MMA M: query rows per tile
+constexpr int kRows = 128;              // MMA M: query rows per half tile
+constexpr int kTileRows = 256;          // query rows per tile (halves A and B)
 constexpr int kKeys = 128;              // keys per chunk (S columns, P·V contraction)
 constexpr int kHeadDim = 128;
 constexpr uint32_t kSlab = 128 * 128;   // 128 rows x 64 elements x 2 bytes
 constexpr uint32_t kTile = 2 * kSlab;   // 128 rows x head_dim 128
 constexpr int kStages = PKV_PREFILL_STAGES;  // K and V ring depth
-constexpr int kHalf = kKeys / 2;        // keys of one softmax warpgroup per chunk
 constexpr int kSoftmaxThreads = 256;    // warps 0-7
 constexpr int kProducerK = 8, kProducerV = 9, kMmaWarp = 10;
 constexpr int kThreads = 352;
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kTile;
+constexpr uint32_t kOffQ = 0;                              // Q of half h at h * kTile
+constexpr uint32_t kOffK = kOffQ + 2 * kTile;
 constexpr uint32_t kOffV = kOffK + kStages * kTile;
-constexpr uint32_t kOffStage = kOffV + kStages * kTile;  // output rows on their way out (128 x 512 B)
-constexpr uint32_t kOffBar = kOffStage + kRows * kHeadDim * 4;
-constexpr uint32_t kOffXchg = kOffBar + 256;  // 128 rows x (float, float): the halves' (max, sum), then weights
-constexpr size_t kSmemBytes = kOffXchg + 1024 + 1024;  // barriers, flags, exchange; 1024 B alignment slack
+constexpr uint32_t kStageWarp = 32 * 32 * 4;               // a warp's 32 rows x 32 fp32 output columns
+constexpr uint32_t kOffStage = kOffV + kStages * kTile;
+constexpr uint32_t kOffBar = kOffStage + 8 * kStageWarp;
+constexpr size_t kSmemBytes = kOffBar + 256 + 1024;  // barriers, flags; 1024 B alignment slack
 static_assert(kSmemBytes <= 227 * 1024, "one CTA's shared memory (227 KB at most on sm_100)");
 constexpr uint32_t kTmemCols = 512;
-constexpr int kSBufs = 2;                    // S / P buffers in tensor memory
-constexpr uint32_t kColS = 0, kColO = 256;   // S / P: 2 x 128 columns; O_h at 256 + 128 h
+constexpr uint32_t kColS = 0, kColO = 256;   // S / P of half h at 128 h, O of half h at 256 + 128 h
 constexpr float kRescale = 8.0f;
 constexpr unsigned kAll = 0xffffffffu;
-// mbarrier slots
-enum : int { kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = kKFull + kStages, kVFull = kKEmpty + kStages,
-             kVEmpty = kVFull + kStages, kSFull = kVEmpty + kStages, kPFull = kSFull + kSBufs,
-             kPVDone = kPFull + 2 * kSBufs, kODone = kPVDone + kSBufs, kOFree = kODone + 1, kXFull = kOFree + 1,
-             kXBack = kXFull + 1, kTileReady = kXBack + 1, kTileFree = kTileReady + 2, kDrain = kTileFree + 2,
+// mbarrier slots; Q, S, P, O-done and O-free come once per half
+enum : int { kQFull = 0, kQEmpty = 2, kKFull = 4, kKEmpty = kKFull + kStages, kVFull = kKEmpty + kStages,
+             kVEmpty = kVFull + kStages, kSFull = kVEmpty + kStages, kPFull = kSFull + 2, kODone = kPFull + 2,
+             kOFree = kODone + 2, kTileReady = kOFree + 2, kTileFree = kTileReady + 2, kDrain = kTileFree + 2,
              kNumBars = kDrain + 1 };
 static_assert(kNumBars * 8 + 16 <= 256, "barriers, flags and tile slots fit the reserved 256 bytes");
-// arrivals per phase: P-full (one per buffer and half) and the exchange by
-// one warpgroup's 128 threads, O-free by all 256 softmax threads, tile-free by
-// lane 0 of the V producer, the MMA warp and the eight softmax warps
+// arrivals per phase: P-full and O-free by a half's 128 softmax threads,
+// tile-free by lane 0 of the V producer, the MMA warp and the eight softmax
+// warps
 __host__ __device__ constexpr uint32_t bar_count(int i) {
-  return (i >= kPFull && i < kPFull + 2 * kSBufs) || i == kXFull || i == kXBack ? 128u
-         : i == kOFree                                                         ? 256u
-         : (i >= kTileFree && i < kTileFree + 2)                               ? 10u
-                                                                               : 1u;
+  return (i >= kPFull && i < kPFull + 2) || (i >= kOFree && i < kOFree + 2) ? 128u
+         : (i >= kTileFree && i < kTileFree + 2)                            ? 10u
+                                                                            : 1u;
 }
-// S-full, P-full and PV-done are barriers per S / P buffer: a buffer's next
-// phase needs the MMA warp to have moved on (S_{j+2} is issued after PV_j),
-// so no waiter can ever be a whole phase behind
+// S-full and P-full of a half complete once per chunk and O-done / O-free
+// once per tile; a half's next phase needs the MMA warp or the softmax warps
+// of that half to have moved on, so no waiter can ever be a whole phase behind
 }  // namespace pf
 
 __device__ __forceinline__ void tma_load_3d_nohint(uint32_t dst, const void* tmap, int32_t x, int32_t y, int32_t z,
@@ -266,7 +259,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
                       const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                       unsigned int* __restrict__ tile_ctr) {
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
-  constexpr int QT = pf::kRows / G;  // query tokens per tile
+  constexpr int QT = pf::kRows / G;  // query tokens per half tile
+  constexpr int QT2 = 2 * QT;        // query tokens per tile
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   static_assert(kBf16 || kF16P, "f16 pools take the one-pass f16 P");
   constexpr bool f16p = kF16P;
@@ -309,7 +303,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
   // Persistent CTAs (one per SM).  The K producer draws tile numbers from a
   // counter and publishes each in one of two slots (tile-ready barrier); the
   // other roles read it and hand the slot back (tile-free barrier).  Tile t
-  // is the (sequence b, KV head g, tile of QT query tokens) of the order: the
+  // is the (sequence b, KV head g, tile of QT2 query tokens) of the order: the
   // tiles of one (b, g) one after another, most keys first, so the tiles in
   // flight at any time share a few sequences' K/V in L2 (taking one tile
   // index of every (b, g) together re-read K/V from DRAM about 7x); drawing
@@ -335,7 +329,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     const int q1 = p.q_start[d.b + 1];
     d.n = q1 - d.q0;
     d.L = p.seq_lens[d.b];
-    d.tok0 = tile * QT;  // chunk-relative first token of the tile
+    d.tok0 = tile * QT2;  // chunk-relative first token of the tile
     const bool args_ok = !(d.n < 0 || d.q0 < 0 || q1 > p.num_q_tokens || d.n > d.L || d.n > p.max_q_len ||
                            d.L > p.max_blocks * p.block_size);
     if (!args_ok && tile == 0 && warp == pf::kProducerK && lane == 0) record_error(PKV_ERR_INVALID_ARG);
@@ -343,7 +337,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     if (!d.valid) return d;
     d.ctx = d.L - d.n;
     d.pos_min = d.ctx + d.tok0;
-    const int pos_max = min(d.L - 1, d.ctx + d.tok0 + QT - 1);
+    const int pos_max = min(d.L - 1, d.ctx + d.tok0 + QT2 - 1);
     d.nc = pos_max / pf::kKeys + 1;  // key chunks this tile attends to
     d.nblk = (d.L + p.block_size - 1) / p.block_size;
     return d;
@@ -359,7 +353,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     return __shfl_sync(pf::kAll, t, 0);
   };
   const int BS = p.block_size;
-  int issued = 0, q_issued = 0;  // producers: fills issued (chunks, Q tiles) in the CTA's count
+  int issued = 0, q_issued[2] = {0, 0};  // producers: fills issued (chunks, Q tiles of each half) in the CTA's count
 
   if (warp == pf::kProducerK || warp == pf::kProducerV) {
     // ----------------------------- TMA producers -----------------------------
@@ -395,16 +389,21 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       if (!d.valid) continue;
       const int b = d.b, g = d.g, nc = d.nc, nblk = d.nblk;
       if (kv == 0) {
-        // Q of the previous tile is no longer read once its last q·Kᵀ is done
-        if (tv > 0) ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kQEmpty), (tv - 1) & 1, abort_flag));
-        if (!ok) break;
-        if (lane == 0) {
-          // Q tile: rows token * G + h, one box per head_dim half
-          mbar_arrive_expect_tx(bar(pf::kQFull), pf::kTile);
-          tma_load_4d(base + pf::kOffQ, &tmap_q, 0, 0, g * G, d.q0 + d.tok0, bar(pf::kQFull));
-          tma_load_4d(base + pf::kOffQ + pf::kSlab, &tmap_q, 0, 1, g * G, d.q0 + d.tok0, bar(pf::kQFull));
+        // Q of a half of the previous tile is no longer read once that half's
+        // last q·Kᵀ is done; half h holds tokens tok0 + h * QT .. + QT - 1
+        // (rows token * G + head; tokens past q's end read as zeros)
+        for (int h = 0; h < 2 && ok; ++h) {
+          if (tv > 0) ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kQEmpty + h), (tv - 1) & 1, abort_flag));
+          if (!ok) break;
+          if (lane == 0) {
+            const uint32_t dst = base + pf::kOffQ + h * pf::kTile;
+            mbar_arrive_expect_tx(bar(pf::kQFull + h), pf::kTile);
+            tma_load_4d(dst, &tmap_q, 0, 0, g * G, d.q0 + d.tok0 + h * QT, bar(pf::kQFull + h));
+            tma_load_4d(dst + pf::kSlab, &tmap_q, 0, 1, g * G, d.q0 + d.tok0 + h * QT, bar(pf::kQFull + h));
+          }
+          q_issued[h] = tv + 1;
         }
-        q_issued = tv + 1;
+        if (!ok) break;
       }
       const int32_t* trow = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
       const int nbc = pf::kKeys / BS;                              // blocks per chunk
@@ -455,7 +454,9 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     // fills unconsumed): wait (bounded) for the last fill of each stage and Q
     if (lane == 0) {
       const uint32_t full0 = bar(kv ? pf::kVFull : pf::kKFull);
-      if (kv == 0 && q_issued > 0) mbar_drain(bar(pf::kQFull), (q_issued - 1) & 1);
+      if (kv == 0)
+        for (int h = 0; h < 2; ++h)
+          if (q_issued[h] > 0) mbar_drain(bar(pf::kQFull + h), (q_issued[h] - 1) & 1);
       for (int s = 0; s < pf::kStages && s < issued; ++s) {
         const int last = s + (issued - 1 - s) / pf::kStages * pf::kStages;  // last chunk that used stage s
         mbar_drain(full0 + 8 * s, (last / pf::kStages) & 1);
@@ -477,59 +478,81 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       if (!d.valid) continue;
       const int nc = d.nc;
       if (lane == 0) {
-        auto issue_s = [&](int j) -> bool {  // j: chunk of the tile; gc + j: chunk of the CTA
-          const int s = (gc + j) % pf::kStages;
-          if (!mbar_wait_sleep(bar(pf::kKFull + s), ((gc + j) / pf::kStages) & 1, abort_flag)) return false;
-          tc::fence_after_sync();
-          const uint32_t kst = base + pf::kOffK + s * pf::kTile;
+        // S_h = Q_h · K_jᵀ into half h's S / P columns; the K stage has landed
+        auto issue_s = [&](int h, int j) {
+          const uint32_t kst = base + pf::kOffK + ((gc + j) % pf::kStages) * pf::kTile;
+          const uint32_t qh = base + pf::kOffQ + h * pf::kTile;
 #pragma unroll
           for (int kk = 0; kk < pf::kHeadDim / 16; ++kk) {
             const uint32_t off = (kk >> 2) * pf::kSlab + (kk & 3) * 32;
-            tc::mma_f16_ss(tmem + pf::kColS + ((gc + j) % pf::kSBufs) * pf::kKeys,
-                           tc::sw128_desc(base + pf::kOffQ + off, 16, 1024), tc::sw128_desc(kst + off, 16, 1024), id_s,
-                           kk > 0 ? 1u : 0u);
+            tc::mma_f16_ss(tmem + pf::kColS + h * pf::kKeys, tc::sw128_desc(qh + off, 16, 1024),
+                           tc::sw128_desc(kst + off, 16, 1024), id_s, kk > 0 ? 1u : 0u);
           }
-          tc::commit(bar(pf::kKEmpty + s));
-          tc::commit(bar(pf::kSFull + (gc + j) % pf::kSBufs));
-          return true;
+          tc::commit(bar(pf::kSFull + h));
         };
-        ok = mbar_wait_sleep(bar(pf::kQFull), tv & 1, abort_flag);
-        for (int j = 0; j < pf::kSBufs && j < nc && ok; ++j) ok = issue_s(j);
-        if (ok && nc <= pf::kSBufs) tc::commit(bar(pf::kQEmpty));  // the tile's last q·Kᵀ is issued
-        // the previous tile's O has been read out of tensor memory
-        if (ok && tv > 0) ok = mbar_wait_sleep(bar(pf::kOFree), (tv - 1) & 1, abort_flag);
+        // O_h += P_h · V_j (P hi in the first 64 columns of the half's buffer, P lo in the next 64)
+        auto issue_pv = [&](int h, int j) {
+          const uint32_t vst = base + pf::kOffV + ((gc + j) % pf::kStages) * pf::kTile;
+          const uint32_t pt = tmem + pf::kColS + h * pf::kKeys;
+#pragma unroll
+          for (int part = 0; part < parts; ++part) {
+#pragma unroll
+            for (int kk = 0; kk < pf::kKeys / 16; ++kk) {
+              const uint32_t bv = vst + kk * 16 * 128;  // 16 keys of 128-byte rows
+              tc::mma_f16_ts(tmem + pf::kColO + h * pf::kHeadDim, pt + part * (pf::kKeys / 2) + kk * 8,
+                             tc::sw128_desc(bv, pf::kSlab, 1024), id_o, (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+        };
+        auto wait_k = [&](int j) {
+          const int gj = gc + j;
+          const bool r = mbar_wait_sleep(bar(pf::kKFull + gj % pf::kStages), (gj / pf::kStages) & 1, abort_flag);
+          tc::fence_after_sync();
+          return r;
+        };
+        // the tile's first q·Kᵀ of both halves
+        ok = mbar_wait_sleep(bar(pf::kQFull), tv & 1, abort_flag) &&
+             mbar_wait_sleep(bar(pf::kQFull + 1), tv & 1, abort_flag) && wait_k(0);
+        if (ok) {
+          issue_s(0, 0);
+          if (nc == 1) tc::commit(bar(pf::kQEmpty));  // half A's last q·Kᵀ
+          issue_s(1, 0);
+          if (nc == 1) tc::commit(bar(pf::kQEmpty + 1));
+          tc::commit(bar(pf::kKEmpty + gc % pf::kStages));
+        }
         for (int j = 0; j < nc && ok; ++j) {
           const int gj = gc + j;
           const int s = gj % pf::kStages;
           ok = mbar_wait_sleep(bar(pf::kVFull + s), (gj / pf::kStages) & 1, abort_flag);
-          const uint32_t vst = base + pf::kOffV + s * pf::kTile;
-          const uint32_t pt = tmem + pf::kColS + (gj % pf::kSBufs) * pf::kKeys;
-          // each half's P·V as soon as its warpgroup has written P (P hi in
-          // the half's first 32 columns, P lo in the next 32)
-#pragma unroll
-          for (int hf = 0; hf < 2 && ok; ++hf) {
-            ok = mbar_wait_sleep(bar(pf::kPFull + 2 * (gj % pf::kSBufs) + hf), (gj / pf::kSBufs) & 1, abort_flag);
-            if (!ok) break;
-            tc::fence_after_sync();
-#pragma unroll
-            for (int part = 0; part < parts; ++part) {
-#pragma unroll
-              for (int kk = 0; kk < pf::kHalf / 16; ++kk) {
-                const uint32_t bv = vst + (hf * pf::kHalf + kk * 16) * 128;  // 16 keys of 128-byte rows
-                tc::mma_f16_ts(tmem + pf::kColO + hf * pf::kHeadDim, pt + hf * pf::kHalf + part * (pf::kHalf / 2) + kk * 8,
-                               tc::sw128_desc(bv, pf::kSlab, 1024), id_o, (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
-              }
-            }
-          }
+          // half A: its P·V (after the previous tile's O_A has left tensor
+          // memory), then its next q·Kᵀ, which waits for the next K stage
+          if (ok && j == 0 && tv > 0) ok = mbar_wait_sleep(bar(pf::kOFree), (tv - 1) & 1, abort_flag);
+          if (ok) ok = mbar_wait_sleep(bar(pf::kPFull), gj & 1, abort_flag);
           if (!ok) break;
+          tc::fence_after_sync();
+          issue_pv(0, j);
+          if (j + 1 < nc) {
+            if (!(ok = wait_k(j + 1))) break;
+            issue_s(0, j + 1);
+            if (j + 1 == nc - 1) tc::commit(bar(pf::kQEmpty));
+          } else {
+            tc::commit(bar(pf::kODone));  // O_A is complete once its last P·V is
+          }
+          // half B likewise; V_j and K_{j+1} are then free
+          if (j == 0 && tv > 0) ok = mbar_wait_sleep(bar(pf::kOFree + 1), (tv - 1) & 1, abort_flag);
+          if (ok) ok = mbar_wait_sleep(bar(pf::kPFull + 1), gj & 1, abort_flag);
+          if (!ok) break;
+          tc::fence_after_sync();
+          issue_pv(1, j);
           tc::commit(bar(pf::kVEmpty + s));
-          tc::commit(bar(pf::kPVDone + gj % pf::kSBufs));
-          if (j + pf::kSBufs < nc) {
-            ok = issue_s(j + pf::kSBufs);
-            if (ok && j + pf::kSBufs == nc - 1) tc::commit(bar(pf::kQEmpty));  // the tile's last q·Kᵀ
+          if (j + 1 < nc) {
+            issue_s(1, j + 1);
+            tc::commit(bar(pf::kKEmpty + (gj + 1) % pf::kStages));
+            if (j + 1 == nc - 1) tc::commit(bar(pf::kQEmpty + 1));
+          } else {
+            tc::commit(bar(pf::kODone + 1));
           }
         }
-        if (ok) tc::commit(bar(pf::kODone));  // the tile's O is complete once its last P·V is
       }
       ok = __shfl_sync(pf::kAll, ok, 0);
       gc += nc;
@@ -547,15 +570,14 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------ softmax warps ------------------------------
-    // warpgroup hf takes keys [64 hf, 64 hf + 64) of every chunk of the tile
-    const int hf = warp >> 2;
-    const int r = (warp & 3) * 32 + lane;  // tile row and TMEM lane
+    const int hh = warp >> 2;               // half of the tile
+    const int r = (warp & 3) * 32 + lane;   // row of the half and TMEM lane
+    const int R = hh * pf::kRows + r;       // row of the tile
     const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const uint32_t tsp = trow + pf::kColS + hf * pf::kHalf;     // this half's S / P columns in buffer 0
-    const uint32_t to = trow + pf::kColO + hf * pf::kHeadDim;   // this half's O
-    const uint32_t to_cols = trow + pf::kColO + hf * pf::kHalf;  // output columns [64 hf, 64 hf + 64) of O_0
+    const uint32_t ts = trow + pf::kColS + hh * pf::kKeys;     // this half's S / P
+    const uint32_t to = trow + pf::kColO + hh * pf::kHeadDim;  // this half's O
     unsigned char* vzero = smem + pf::kOffV;
-    float2* xch = reinterpret_cast<float2*>(smem + pf::kOffXchg) + r;
+    float4* wstage = reinterpret_cast<float4*>(smem + pf::kOffStage + warp * pf::kStageWarp);
     const float sl = p.scale_log2;
     bool ok = true;
     int gc = 0, tv = 0;
@@ -565,66 +587,62 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       const Tile d = tile_of(t);
       if (!d.valid) continue;
       const int nc = d.nc, L = d.L, n = d.n, tok0 = d.tok0, pos_min = d.pos_min;
-      const int tok = tok0 + r / G;
+      const int tok = tok0 + R / G;
       const int pos = min(d.ctx + tok, L - 1);  // rows past the chunk end compute a copy of the last row
-      // running max (-inf until a key of this half is visible to the row) and sum
       float m_used = -INFINITY, l = 0.f;
       for (int j = 0; j < nc && ok; ++j) {
-        const int gj = gc + j;              // chunk of the CTA
-        const int sb = gj % pf::kSBufs;     // S / P buffer
-        const int s = gj % pf::kStages;     // K / V stage
-        ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kSFull + sb), (gj / pf::kSBufs) & 1, abort_flag));
+        const int gj = gc + j;           // chunk of the CTA
+        const int s = gj % pf::kStages;  // K / V stage
+        ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kSFull + hh), gj & 1, abort_flag));
         if (!ok) break;
         tc::fence_after_sync();
-        float x[pf::kHalf];  // raw scores q·k of this row's 64 keys
+        float x[pf::kKeys];  // raw scores q·k of this row's 128 keys
         {
-          uint32_t raw[2][32];
+          uint32_t raw[4][32];
 #pragma unroll
-          for (int q = 0; q < 2; ++q) tc::ld_32x32b_x32(tsp + sb * pf::kKeys + 32 * q, raw[q]);
+          for (int q = 0; q < 4; ++q) tc::ld_32x32b_x32(ts + 32 * q, raw[q]);
           tc::wait_ld();
 #pragma unroll
-          for (int q = 0; q < 2; ++q)
+          for (int q = 0; q < 4; ++q)
 #pragma unroll
             for (int i = 0; i < 32; ++i) x[32 * q + i] = __uint_as_float(raw[q][i]);
         }
-        const int key0 = j * pf::kKeys + hf * pf::kHalf;  // this half's first key
-        if (key0 + pf::kHalf - 1 > pos_min) {  // the diagonal: keys after a row's position are hidden
+        const int key0 = j * pf::kKeys;
+        if (key0 + pf::kKeys - 1 > pos_min) {  // the diagonal: keys after a row's position are hidden
 #pragma unroll
-          for (int c = 0; c < pf::kHalf; ++c) x[c] = key0 + c <= pos ? x[c] : -INFINITY;
+          for (int c = 0; c < pf::kKeys; ++c) x[c] = key0 + c <= pos ? x[c] : -INFINITY;
         }
         // row max with three-input maxima in four independent chains; the
         // scale is positive, so the max of the scaled scores is the scaled max
         float mx[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-        for (int c = 4; c + 8 <= pf::kHalf; c += 8) {
+        for (int c = 4; c + 8 <= pf::kKeys; c += 8) {
           mx[0] = max3f(mx[0], x[c], x[c + 1]);
           mx[1] = max3f(mx[1], x[c + 2], x[c + 3]);
           mx[2] = max3f(mx[2], x[c + 4], x[c + 5]);
           mx[3] = max3f(mx[3], x[c + 6], x[c + 7]);
         }
-        mx[0] = max3f(mx[0], x[pf::kHalf - 4], x[pf::kHalf - 3]);
-        mx[1] = max3f(mx[1], x[pf::kHalf - 2], x[pf::kHalf - 1]);
-        const float mc = fmaxf(max3f(mx[0], mx[1], mx[2]), mx[3]) * sl;  // -inf: no visible key here
+        mx[0] = max3f(mx[0], x[pf::kKeys - 4], x[pf::kKeys - 3]);
+        mx[1] = max3f(mx[1], x[pf::kKeys - 2], x[pf::kKeys - 1]);
+        const float mc = fmaxf(max3f(mx[0], mx[1], mx[2]), mx[3]) * sl;
         float factor = 1.f;
         bool resc = false;
-        if (mc > m_used + pf::kRescale) {
-          // the first visible keys of this half only set the max (O_h and l
-          // are still zero); later moves rescale both
-          resc = m_used != -INFINITY;
-          if (resc) factor = fast_exp2(m_used - mc);
+        if (j == 0) {
+          m_used = mc;  // key 0 is visible to every row: finite
+        } else if (mc > m_used + pf::kRescale) {
+          factor = fast_exp2(m_used - mc);
           m_used = mc;
+          resc = true;
         }
         // exponentials (arguments and sums two lanes at a time, packed f32x2),
-        // each quarter of the row written as P over S_j in tensor memory as
-        // soon as it is done (the stores complete while the next quarter is
-        // computed): key pair (2c, 2c+1) of the half in column c (hi) and
-        // 32 + c (lo) of the half's columns
+        // each quarter of the row written as P hi and lo over S in tensor
+        // memory as soon as it is done (the stores complete while the next
+        // quarter is computed): key pair (2c, 2c+1) in column c (hi) and
+        // 64 + c (lo)
         float2 sm[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        const float2 sl2 = make_float2(sl, sl);
-        const float nm = m_used == -INFINITY ? 0.f : -m_used;  // no visible key: every argument stays -inf
-        const float2 nm2 = make_float2(nm, nm);
+        const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(-m_used, -m_used);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < 4; ++h) {
 #pragma unroll
           for (int c = 32 * h; c < 32 * h + 32; c += 2) {
             const float2 a = __ffma2_rn(make_float2(x[c], x[c + 1]), sl2, nm2);  // hidden keys: -inf -> 0
@@ -636,8 +654,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
             uint32_t hi[16], lo[16];
 #pragma unroll
             for (int c = 0; c < 16; ++c) split_hi_lo<T>(x[32 * h + 2 * c], x[32 * h + 2 * c + 1], hi[c], lo[c]);
-            tc::st_32x32b_x16(tsp + sb * pf::kKeys + 16 * h, hi);
-            tc::st_32x32b_x16(tsp + sb * pf::kKeys + pf::kHalf / 2 + 16 * h, lo);
+            tc::st_32x32b_x16(ts + 16 * h, hi);
+            tc::st_32x32b_x16(ts + pf::kKeys / 2 + 16 * h, lo);
           } else {
             uint32_t ph[16];
 #pragma unroll
@@ -645,7 +663,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
               const __half2 v = __floats2half2_rn(x[32 * h + 2 * c], x[32 * h + 2 * c + 1]);
               ph[c] = *reinterpret_cast<const uint32_t*>(&v);
             }
-            tc::st_32x32b_x16(tsp + sb * pf::kKeys + 16 * h, ph);
+            tc::st_32x32b_x16(ts + 16 * h, ph);
           }
         }
         const float2 s01 = __fadd2_rn(sm[0], sm[1]), s23 = __fadd2_rn(sm[2], sm[3]);
@@ -653,14 +671,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         l = l * factor + (st.x + st.y);
 
         if (__any_sync(pf::kAll, resc)) {
-          // O_h still accumulates PV_{j-1}: wait for it, then rescale the row.
-          // PV_{j-1} commits to the barrier of its buffer, whose previous
-          // phase (PV_{j-3}) was covered by S_{j-1}'s commit, so the parity
-          // wait cannot see an older phase.
-          const int pj = gj - 1;
-          ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kPVDone + pj % pf::kSBufs), (pj / pf::kSBufs) & 1, abort_flag));
-          if (!ok) break;
-          tc::fence_after_sync();
+          // O still holds the sum up to chunk j-1: the commit of S(j), seen
+          // above, covers P·V(j-1), which the MMA warp issued before it
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             uint32_t o[32];
@@ -671,15 +683,15 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
             tc::st_32x32b_x32(to + 32 * q, o);
           }
         }
-        const int vend = j * pf::kKeys + (hf + 1) * pf::kHalf;  // one past this half's last key
-        if (vend > L) {
-          // V rows of this half past the sequence end hold stale or unwritten
-          // bytes: zero them so that P = 0 there cannot meet a NaN pattern
+        if (hh == 0 && key0 + pf::kKeys > L) {
+          // V rows past the sequence end hold stale or unwritten bytes: half
+          // A zeroes them (before its P-full, so before either half's P·V
+          // reads them) so that P = 0 there cannot meet a NaN pattern
           ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kVFull + s), (gj / pf::kStages) & 1, abort_flag));
           if (!ok) break;
-          const int v0 = max(L - j * pf::kKeys, hf * pf::kHalf);  // first row to zero, chunk-relative
+          const int v0 = L - key0;
           unsigned char* vst = vzero + s * pf::kTile;
-          for (int idx = r; idx < ((hf + 1) * pf::kHalf - v0) * 16; idx += 128) {
+          for (int idx = r; idx < (pf::kKeys - v0) * 16; idx += 128) {
             const int row = v0 + (idx >> 4), piece = idx & 15;
             *reinterpret_cast<uint4*>(vst + (piece >> 3) * pf::kSlab + row * 128 + (piece & 7) * 16) =
                 make_uint4(0u, 0u, 0u, 0u);
@@ -688,79 +700,48 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         }
         tc::wait_st();
         tc::fence_before_sync();
-        mbar_arrive(bar(pf::kPFull + 2 * sb + hf));
+        mbar_arrive(bar(pf::kPFull + hh));
       }
-      // the MMA warp commits O-done after the tile's last P·V
-      if (ok) ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kODone), tv & 1, abort_flag));
+      // the MMA warp commits O-done after the half's last P·V
+      if (ok) ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kODone + hh), tv & 1, abort_flag));
       if (!ok) break;
       tc::fence_after_sync();
-      // this warpgroup writes output columns [64 hf, 64 hf + 64) of its rows:
-      // both accumulators leave tensor memory first (the next tile's P·V may
-      // then overwrite them)
-      uint32_t o0[2][32], o1[2][32];
+      // O goes out 32 columns at a time through this warp's 4 KB of shared
+      // memory: each thread parks 128 bytes of its row, then each store
+      // instruction writes 4 rows' 128-byte pieces, instead of 32 rows' 16
+      // bytes straight from the tensor-memory layout.  The 16-byte piece c of
+      // parked row k sits at slot c ^ (k mod 8), so the parking and the
+      // row-wise reads are both free of bank conflicts.  Once the last
+      // columns are loaded, O may be overwritten by the next tile's P·V.
+      const float inv = 1.f / l;
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        tc::ld_32x32b_x32(to_cols + 32 * q, o0[q]);
-        tc::ld_32x32b_x32(to_cols + pf::kHeadDim + 32 * q, o1[q]);
-      }
-      tc::wait_ld();
-      tc::fence_before_sync();
-      mbar_arrive(bar(pf::kOFree));
-      // weights of the two halves: warpgroup 1 hands its (max, sum) to
-      // warpgroup 0 through shared memory, which returns both weights with
-      // the normalisation folded in; key 0 is visible to every row, so m_0
-      // is finite and the total positive
-      float c0, c1;
-      if (hf == 1) {
-        *xch = make_float2(m_used, l);
-        mbar_arrive(bar(pf::kXFull));
-        ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kXBack), tv & 1, abort_flag));
-        if (!ok) break;
-        const float2 w = *xch;
-        c0 = w.x;
-        c1 = w.y;
-      } else {
-        ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kXFull), tv & 1, abort_flag));
-        if (!ok) break;
-        const float2 o = *xch;
-        const float mm = fmaxf(m_used, o.x);
-        const float w0 = fast_exp2(m_used - mm), w1 = fast_exp2(o.x - mm);  // m_1 = -inf: w1 = 0
-        const float inv = 1.f / (l * w0 + o.y * w1);
-        c0 = w0 * inv;
-        c1 = w1 * inv;
-        *xch = make_float2(c0, c1);
-        mbar_arrive(bar(pf::kXBack));
-      }
-      // then out through shared memory: each thread parks its half row, and
-      // each warp writes its 32 half rows two per store instruction, instead
-      // of 32 rows per instruction straight from the tensor-memory layout.
-      // The 16-byte piece c of row r sits at slot c ^ (r mod 8) of the row,
-      // so the row-wise writes and the piece-wise reads are both free of bank
-      // conflicts.
-      float4* stage = reinterpret_cast<float4*>(smem + pf::kOffStage);
-      float4* srow = stage + r * (pf::kHeadDim / 4);
-#pragma unroll
-      for (int q = 0; q < 2; ++q)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float v[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            v[e] = __uint_as_float(o0[q][4 * i + e]) * c0 + __uint_as_float(o1[q][4 * i + e]) * c1;
-          srow[(16 * hf + 8 * q + i) ^ (r & 7)] = make_float4(v[0], v[1], v[2], v[3]);
+      for (int q = 0; q < 4; ++q) {
+        uint32_t o[32];
+        tc::ld_32x32b_x32(to + 32 * q, o);
+        tc::wait_ld();
+        if (q == 3) {
+          tc::fence_before_sync();
+          mbar_arrive(bar(pf::kOFree + hh));
         }
-      __syncwarp();
-      for (int k = 0; k < 16; ++k) {
-        const int rr = (warp & 3) * 32 + 2 * k + (lane >> 4);  // a row this warp parked
-        const int piece = 16 * hf + (lane & 15);
-        const int tk = tok0 + rr / G;
-        if (tk < n) {  // rows past the chunk end are not written
-          float4* orow = reinterpret_cast<float4*>(
-              p.out + (static_cast<int64_t>(d.q0 + tk) * p.num_q_heads + d.g * G + rr % G) * pf::kHeadDim);
-          orow[piece] = stage[rr * (pf::kHeadDim / 4) + (piece ^ (rr & 7))];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          wstage[lane * 8 + (i ^ (lane & 7))] =
+              make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
+                          __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int kr = 4 * k + (lane >> 3), piece = lane & 7;  // parked row and its 16-byte piece
+          const int rr = hh * pf::kRows + (warp & 3) * 32 + kr;    // row of the tile
+          const int tk = tok0 + rr / G;
+          if (tk < n) {  // rows past the chunk end are not written
+            float4* orow = reinterpret_cast<float4*>(
+                p.out + (static_cast<int64_t>(d.q0 + tk) * p.num_q_heads + d.g * G + rr % G) * pf::kHeadDim);
+            orow[8 * q + piece] = wstage[kr * 8 + (piece ^ (kr & 7))];
+          }
         }
+        __syncwarp();  // the pieces are out before the next columns are parked
       }
-      __syncwarp();  // this warp's half rows are out of the staging area before the next tile's
       gc += nc;
       ++tv;
     }
