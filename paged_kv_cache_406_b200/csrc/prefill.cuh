@@ -29,12 +29,13 @@
 // tile, and the tensor core idled half of the time even with no softmax work
 // at all; two halves also load K/V once per 256 rows.
 //
-// Warp roles (352 threads): warps 0-3 softmax of half A, 4-7 of half B
+// Warp roles (384 threads): warps 0-3 softmax of half A, 4-7 of half B
 // (thread = row = TMEM lane of its warp's lane quarter, warp mod 4), warps 8
 // and 9 TMA producers (K with Q, V), warp 10 MMA issuer (lane 0) and TMEM
-// owner.  Tensor memory (512 columns): S / P of half h at column 128 h (P hi
-// in the first 64 columns, P lo in the next 64; a single f16 P in the first
-// 64), O of half h at 256 + 128 h.
+// owner, warp 11 idle (it completes the fourth warpgroup, whose registers go
+// to the softmax warpgroups).  Tensor memory (512 columns): S / P of half h
+// at column 128 h (P hi in the first 64 columns, P lo in the next 64; a single
+// f16 P in the first 64), O of half h at 256 + 128 h.
 // Shared memory: Q of both halves 64 KB, K and V rings of 32 KB stages, and
 // 4 KB per softmax warp through which its output rows leave in 128-byte
 // pieces.  Keeping P in tensor memory spares shared memory 128 KB of traffic
@@ -99,7 +100,7 @@ constexpr uint32_t kTile = 2 * kSlab;   // 128 rows x head_dim 128
 constexpr int kStages = PKV_PREFILL_STAGES;  // K and V ring depth
 constexpr int kSoftmaxThreads = 256;    // warps 0-7
 constexpr int kProducerK = 8, kProducerV = 9, kMmaWarp = 10;
-constexpr int kThreads = 352;
+constexpr int kThreads = 384;  // warp 11 only completes the producer warpgroup
 constexpr uint32_t kOffQ = 0;                              // Q of half h at h * kTile
 constexpr uint32_t kOffK = kOffQ + 2 * kTile;
 constexpr uint32_t kOffV = kOffK + kStages * kTile;
@@ -118,11 +119,12 @@ enum : int { kQFull = 0, kQEmpty = 2, kKFull = 4, kKEmpty = kKFull + kStages, kV
              kOFree = kODone + 2, kTileReady = kOFree + 2, kTileFree = kTileReady + 2, kDrain = kTileFree + 2,
              kNumBars = kDrain + 1 };
 static_assert(kNumBars * 8 + 16 <= 256, "barriers, flags and tile slots fit the reserved 256 bytes");
-// arrivals per phase: P-full and O-free by a half's 128 softmax threads,
+// arrivals per phase: P-full and O-free by lane 0 of each of a half's four
+// softmax warps, once the whole warp's tensor-memory accesses are done;
 // tile-free by lane 0 of the V producer, the MMA warp and the eight softmax
 // warps
 __host__ __device__ constexpr uint32_t bar_count(int i) {
-  return (i >= kPFull && i < kPFull + 2) || (i >= kOFree && i < kOFree + 2) ? 128u
+  return (i >= kPFull && i < kPFull + 2) || (i >= kOFree && i < kOFree + 2) ? 4u
          : (i >= kTileFree && i < kTileFree + 2)                            ? 10u
                                                                             : 1u;
 }
@@ -355,220 +357,229 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
   const int BS = p.block_size;
   int issued = 0, q_issued[2] = {0, 0};  // producers: fills issued (chunks, Q tiles of each half) in the CTA's count
 
-  if (warp == pf::kProducerK || warp == pf::kProducerV) {
-    // ----------------------------- TMA producers -----------------------------
-    // One warp streams K chunks (and Q), the other V chunks, each through its
-    // own ring: K runs ahead of V (q·Kᵀ of chunk j+2 is issued right after
-    // P·V of chunk j, while V's stages free only as P·V completes; a single
-    // producer alternating K and V held K behind V's refills).
-    const int kv = warp == pf::kProducerV ? 1 : 0;
-    bool ok = true;
-    int gc = 0, tv = 0;
-    for (int ti = 0; ok; ++ti) {
-      int t;
-      if (kv == 0) {
-        t = total;
-        if (lane == 0) {
-          // the slot's previous tile has been read by every other role
-          const bool free = ti < 2 || mbar_wait_sleep(bar(pf::kTileFree + (ti & 1)), ((ti >> 1) - 1) & 1, abort_flag);
-          if (!free && !*abort_flag) {
-            record_error(PKV_ERR_DEVICE_TIMEOUT);
-            *abort_flag = 1;
-          }
-          const unsigned ticket = (!free || *abort_flag) ? static_cast<unsigned>(total) : atomicAdd(tile_ctr, 1u);
-          t = ticket >= static_cast<unsigned>(total) ? total : static_cast<int>(ticket);
-          tile_slot[ti & 1] = t;
-          mbar_arrive(bar(pf::kTileReady + (ti & 1)));
-        }
-        t = __shfl_sync(pf::kAll, t, 0);
-      } else {
-        t = read_tile(ti);
-      }
-      if (t >= total) break;
-      const Tile d = tile_of(t);
-      if (!d.valid) continue;
-      const int b = d.b, g = d.g, nc = d.nc, nblk = d.nblk;
-      if (kv == 0) {
-        // Q of a half of the previous tile is no longer read once that half's
-        // last q·Kᵀ is done; half h holds tokens tok0 + h * QT .. + QT - 1
-        // (rows token * G + head; tokens past q's end read as zeros)
-        for (int h = 0; h < 2 && ok; ++h) {
-          if (tv > 0) ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kQEmpty + h), (tv - 1) & 1, abort_flag));
-          if (!ok) break;
+  // Registers: the kernel is launched at 168 a thread (384 x 168 = 64512);
+  // the producer / MMA warpgroup (warps 8-11) drops to 112 and the two softmax
+  // warpgroups rise to 184 (128 x 112 + 256 x 184 = 61440, within the launch's
+  // total, so the increase never waits for long): the softmax rows (128
+  // scores a thread) then fit in registers without spilling.
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 112;\n" ::: "memory");
+    if (warp == pf::kProducerK || warp == pf::kProducerV) {
+      // ----------------------------- TMA producers -----------------------------
+      // One warp streams K chunks (and Q), the other V chunks, each through its
+      // own ring: K runs ahead of V (q·Kᵀ of chunk j+2 is issued right after
+      // P·V of chunk j, while V's stages free only as P·V completes; a single
+      // producer alternating K and V held K behind V's refills).
+      const int kv = warp == pf::kProducerV ? 1 : 0;
+      bool ok = true;
+      int gc = 0, tv = 0;
+      for (int ti = 0; ok; ++ti) {
+        int t;
+        if (kv == 0) {
+          t = total;
           if (lane == 0) {
-            const uint32_t dst = base + pf::kOffQ + h * pf::kTile;
-            mbar_arrive_expect_tx(bar(pf::kQFull + h), pf::kTile);
-            tma_load_4d(dst, &tmap_q, 0, 0, g * G, d.q0 + d.tok0 + h * QT, bar(pf::kQFull + h));
-            tma_load_4d(dst + pf::kSlab, &tmap_q, 0, 1, g * G, d.q0 + d.tok0 + h * QT, bar(pf::kQFull + h));
-          }
-          q_issued[h] = tv + 1;
-        }
-        if (!ok) break;
-      }
-      const int32_t* trow = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
-      const int nbc = pf::kKeys / BS;                              // blocks per chunk
-      const uint32_t box_bytes = static_cast<uint32_t>(BS) * 128;  // one block, one head_dim half
-      const uint32_t full0 = bar(kv ? pf::kVFull : pf::kKFull), empty0 = bar(kv ? pf::kVEmpty : pf::kKEmpty);
-      // V from the staged f16 copy: block j of sequence b sits at b * max_blocks + j, no table lookup
-      const bool staged = kv && v_from_stage;
-      const void* map = kv ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k);
-      const uint32_t ring = base + (kv ? pf::kOffV : pf::kOffK);
-      for (int j = 0; j < nc && ok; ++j) {
-        const int s = (gc + j) % pf::kStages;
-        const uint32_t ph = (((gc + j) / pf::kStages) & 1) ^ 1;
-        const int jb = j * nbc;
-        const int nload = min(nbc, nblk - jb);  // blocks past the sequence end are not read
-        int phys = 0;
-        if (lane < nload) {
-          if (staged) {
-            phys = b * p.max_blocks + jb + lane;
-          } else {
-            phys = trow[jb + lane];
-            if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_blocks)) {
-              record_error(PKV_ERR_BAD_BLOCK);
-              phys = 0;
+            // the slot's previous tile has been read by every other role
+            const bool free = ti < 2 || mbar_wait_sleep(bar(pf::kTileFree + (ti & 1)), ((ti >> 1) - 1) & 1, abort_flag);
+            if (!free && !*abort_flag) {
+              record_error(PKV_ERR_DEVICE_TIMEOUT);
+              *abort_flag = 1;
             }
+            const unsigned ticket = (!free || *abort_flag) ? static_cast<unsigned>(total) : atomicAdd(tile_ctr, 1u);
+            t = ticket >= static_cast<unsigned>(total) ? total : static_cast<int>(ticket);
+            tile_slot[ti & 1] = t;
+            mbar_arrive(bar(pf::kTileReady + (ti & 1)));
           }
+          t = __shfl_sync(pf::kAll, t, 0);
+        } else {
+          t = read_tile(ti);
         }
-        const int32_t y = (phys * p.num_kv_heads + g) * BS;
-        const uint32_t full = full0 + 8 * s;
-        ok = __all_sync(pf::kAll, mbar_wait_sleep(empty0 + 8 * s, ph, abort_flag));
-        if (!ok) break;
-        if (lane == 0) mbar_arrive_expect_tx(full, static_cast<uint32_t>(nload) * 2u * box_bytes);
-        __syncwarp();
-        if (lane < nload) {
-          const uint32_t dst = ring + s * pf::kTile + lane * box_bytes;
-          tma_load_3d_nohint(dst, map, 0, y, 0, full);
-          tma_load_3d_nohint(dst + pf::kSlab, map, 0, y, 1, full);
-        }
-        issued = gc + j + 1;
-      }
-      gc += nc;
-      ++tv;
-    }
-    if (!ok && lane == 0) {
-      record_error(PKV_ERR_DEVICE_TIMEOUT);
-      *abort_flag = 1;
-    }
-    // no copy may still be landing when the CTA exits (a timeout can leave
-    // fills unconsumed): wait (bounded) for the last fill of each stage and Q
-    if (lane == 0) {
-      const uint32_t full0 = bar(kv ? pf::kVFull : pf::kKFull);
-      if (kv == 0)
-        for (int h = 0; h < 2; ++h)
-          if (q_issued[h] > 0) mbar_drain(bar(pf::kQFull + h), (q_issued[h] - 1) & 1);
-      for (int s = 0; s < pf::kStages && s < issued; ++s) {
-        const int last = s + (issued - 1 - s) / pf::kStages * pf::kStages;  // last chunk that used stage s
-        mbar_drain(full0 + 8 * s, (last / pf::kStages) & 1);
-      }
-    }
-    __syncwarp();
-  } else if (warp == pf::kMmaWarp) {
-    // ------------------------------- MMA issuer -------------------------------
-    const uint32_t id_s = tc::idesc_f16(kBf16, false, pf::kRows, pf::kKeys);
-    // P·V: f16 P and f16 V in one pass, or bf16 P hi and lo over bf16 V
-    const uint32_t id_o = tc::idesc_f16(kBf16 && !f16p, true, pf::kRows, pf::kHeadDim);
-    constexpr int parts = f16p ? 1 : 2;
-    bool ok = true;
-    int gc = 0, tv = 0;
-    for (int ti = 0; ok; ++ti) {
-      const int t = read_tile(ti);
-      if (t >= total) break;
-      const Tile d = tile_of(t);
-      if (!d.valid) continue;
-      const int nc = d.nc;
-      if (lane == 0) {
-        // S_h = Q_h · K_jᵀ into half h's S / P columns; the K stage has landed
-        auto issue_s = [&](int h, int j) {
-          const uint32_t kst = base + pf::kOffK + ((gc + j) % pf::kStages) * pf::kTile;
-          const uint32_t qh = base + pf::kOffQ + h * pf::kTile;
-#pragma unroll
-          for (int kk = 0; kk < pf::kHeadDim / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * pf::kSlab + (kk & 3) * 32;
-            tc::mma_f16_ss(tmem + pf::kColS + h * pf::kKeys, tc::sw128_desc(qh + off, 16, 1024),
-                           tc::sw128_desc(kst + off, 16, 1024), id_s, kk > 0 ? 1u : 0u);
-          }
-          tc::commit(bar(pf::kSFull + h));
-        };
-        // O_h += P_h · V_j (P hi in the first 64 columns of the half's buffer, P lo in the next 64)
-        auto issue_pv = [&](int h, int j) {
-          const uint32_t vst = base + pf::kOffV + ((gc + j) % pf::kStages) * pf::kTile;
-          const uint32_t pt = tmem + pf::kColS + h * pf::kKeys;
-#pragma unroll
-          for (int part = 0; part < parts; ++part) {
-#pragma unroll
-            for (int kk = 0; kk < pf::kKeys / 16; ++kk) {
-              const uint32_t bv = vst + kk * 16 * 128;  // 16 keys of 128-byte rows
-              tc::mma_f16_ts(tmem + pf::kColO + h * pf::kHeadDim, pt + part * (pf::kKeys / 2) + kk * 8,
-                             tc::sw128_desc(bv, pf::kSlab, 1024), id_o, (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
+        if (t >= total) break;
+        const Tile d = tile_of(t);
+        if (!d.valid) continue;
+        const int b = d.b, g = d.g, nc = d.nc, nblk = d.nblk;
+        if (kv == 0) {
+          // Q of a half of the previous tile is no longer read once that half's
+          // last q·Kᵀ is done; half h holds tokens tok0 + h * QT .. + QT - 1
+          // (rows token * G + head; tokens past q's end read as zeros)
+          for (int h = 0; h < 2 && ok; ++h) {
+            if (tv > 0) ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kQEmpty + h), (tv - 1) & 1, abort_flag));
+            if (!ok) break;
+            if (lane == 0) {
+              const uint32_t dst = base + pf::kOffQ + h * pf::kTile;
+              mbar_arrive_expect_tx(bar(pf::kQFull + h), pf::kTile);
+              tma_load_4d(dst, &tmap_q, 0, 0, g * G, d.q0 + d.tok0 + h * QT, bar(pf::kQFull + h));
+              tma_load_4d(dst + pf::kSlab, &tmap_q, 0, 1, g * G, d.q0 + d.tok0 + h * QT, bar(pf::kQFull + h));
             }
+            q_issued[h] = tv + 1;
           }
-        };
-        auto wait_k = [&](int j) {
-          const int gj = gc + j;
-          const bool r = mbar_wait_sleep(bar(pf::kKFull + gj % pf::kStages), (gj / pf::kStages) & 1, abort_flag);
-          tc::fence_after_sync();
-          return r;
-        };
-        // the tile's first q·Kᵀ of both halves
-        ok = mbar_wait_sleep(bar(pf::kQFull), tv & 1, abort_flag) &&
-             mbar_wait_sleep(bar(pf::kQFull + 1), tv & 1, abort_flag) && wait_k(0);
-        if (ok) {
-          issue_s(0, 0);
-          if (nc == 1) tc::commit(bar(pf::kQEmpty));  // half A's last q·Kᵀ
-          issue_s(1, 0);
-          if (nc == 1) tc::commit(bar(pf::kQEmpty + 1));
-          tc::commit(bar(pf::kKEmpty + gc % pf::kStages));
+          if (!ok) break;
         }
+        const int32_t* trow = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
+        const int nbc = pf::kKeys / BS;                              // blocks per chunk
+        const uint32_t box_bytes = static_cast<uint32_t>(BS) * 128;  // one block, one head_dim half
+        const uint32_t full0 = bar(kv ? pf::kVFull : pf::kKFull), empty0 = bar(kv ? pf::kVEmpty : pf::kKEmpty);
+        // V from the staged f16 copy: block j of sequence b sits at b * max_blocks + j, no table lookup
+        const bool staged = kv && v_from_stage;
+        const void* map = kv ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k);
+        const uint32_t ring = base + (kv ? pf::kOffV : pf::kOffK);
         for (int j = 0; j < nc && ok; ++j) {
-          const int gj = gc + j;
-          const int s = gj % pf::kStages;
-          ok = mbar_wait_sleep(bar(pf::kVFull + s), (gj / pf::kStages) & 1, abort_flag);
-          // half A: its P·V (after the previous tile's O_A has left tensor
-          // memory), then its next q·Kᵀ, which waits for the next K stage
-          if (ok && j == 0 && tv > 0) ok = mbar_wait_sleep(bar(pf::kOFree), (tv - 1) & 1, abort_flag);
-          if (ok) ok = mbar_wait_sleep(bar(pf::kPFull), gj & 1, abort_flag);
-          if (!ok) break;
-          tc::fence_after_sync();
-          issue_pv(0, j);
-          if (j + 1 < nc) {
-            if (!(ok = wait_k(j + 1))) break;
-            issue_s(0, j + 1);
-            if (j + 1 == nc - 1) tc::commit(bar(pf::kQEmpty));
-          } else {
-            tc::commit(bar(pf::kODone));  // O_A is complete once its last P·V is
+          const int s = (gc + j) % pf::kStages;
+          const uint32_t ph = (((gc + j) / pf::kStages) & 1) ^ 1;
+          const int jb = j * nbc;
+          const int nload = min(nbc, nblk - jb);  // blocks past the sequence end are not read
+          int phys = 0;
+          if (lane < nload) {
+            if (staged) {
+              phys = b * p.max_blocks + jb + lane;
+            } else {
+              phys = trow[jb + lane];
+              if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_blocks)) {
+                record_error(PKV_ERR_BAD_BLOCK);
+                phys = 0;
+              }
+            }
           }
-          // half B likewise; V_j and K_{j+1} are then free
-          if (j == 0 && tv > 0) ok = mbar_wait_sleep(bar(pf::kOFree + 1), (tv - 1) & 1, abort_flag);
-          if (ok) ok = mbar_wait_sleep(bar(pf::kPFull + 1), gj & 1, abort_flag);
+          const int32_t y = (phys * p.num_kv_heads + g) * BS;
+          const uint32_t full = full0 + 8 * s;
+          ok = __all_sync(pf::kAll, mbar_wait_sleep(empty0 + 8 * s, ph, abort_flag));
           if (!ok) break;
-          tc::fence_after_sync();
-          issue_pv(1, j);
-          tc::commit(bar(pf::kVEmpty + s));
-          if (j + 1 < nc) {
-            issue_s(1, j + 1);
-            tc::commit(bar(pf::kKEmpty + (gj + 1) % pf::kStages));
-            if (j + 1 == nc - 1) tc::commit(bar(pf::kQEmpty + 1));
-          } else {
-            tc::commit(bar(pf::kODone + 1));
+          if (lane == 0) mbar_arrive_expect_tx(full, static_cast<uint32_t>(nload) * 2u * box_bytes);
+          __syncwarp();
+          if (lane < nload) {
+            const uint32_t dst = ring + s * pf::kTile + lane * box_bytes;
+            tma_load_3d_nohint(dst, map, 0, y, 0, full);
+            tma_load_3d_nohint(dst + pf::kSlab, map, 0, y, 1, full);
           }
+          issued = gc + j + 1;
         }
+        gc += nc;
+        ++tv;
       }
-      ok = __shfl_sync(pf::kAll, ok, 0);
-      gc += nc;
-      ++tv;
-    }
-    if (lane == 0) {
-      if (!ok) {
+      if (!ok && lane == 0) {
         record_error(PKV_ERR_DEVICE_TIMEOUT);
         *abort_flag = 1;
       }
-      // every MMA issued completes before tensor memory is freed
-      tc::commit(bar(pf::kDrain));
-      mbar_drain(bar(pf::kDrain), 0);
+      // no copy may still be landing when the CTA exits (a timeout can leave
+      // fills unconsumed): wait (bounded) for the last fill of each stage and Q
+      if (lane == 0) {
+        const uint32_t full0 = bar(kv ? pf::kVFull : pf::kKFull);
+        if (kv == 0)
+          for (int h = 0; h < 2; ++h)
+            if (q_issued[h] > 0) mbar_drain(bar(pf::kQFull + h), (q_issued[h] - 1) & 1);
+        for (int s = 0; s < pf::kStages && s < issued; ++s) {
+          const int last = s + (issued - 1 - s) / pf::kStages * pf::kStages;  // last chunk that used stage s
+          mbar_drain(full0 + 8 * s, (last / pf::kStages) & 1);
+        }
+      }
+      __syncwarp();
+    } else if (warp == pf::kMmaWarp) {
+      // ------------------------------- MMA issuer -------------------------------
+      const uint32_t id_s = tc::idesc_f16(kBf16, false, pf::kRows, pf::kKeys);
+      // P·V: f16 P and f16 V in one pass, or bf16 P hi and lo over bf16 V
+      const uint32_t id_o = tc::idesc_f16(kBf16 && !f16p, true, pf::kRows, pf::kHeadDim);
+      constexpr int parts = f16p ? 1 : 2;
+      bool ok = true;
+      int gc = 0, tv = 0;
+      for (int ti = 0; ok; ++ti) {
+        const int t = read_tile(ti);
+        if (t >= total) break;
+        const Tile d = tile_of(t);
+        if (!d.valid) continue;
+        const int nc = d.nc;
+        if (lane == 0) {
+          // S_h = Q_h · K_jᵀ into half h's S / P columns; the K stage has landed
+          auto issue_s = [&](int h, int j) {
+            const uint32_t kst = base + pf::kOffK + ((gc + j) % pf::kStages) * pf::kTile;
+            const uint32_t qh = base + pf::kOffQ + h * pf::kTile;
+  #pragma unroll
+            for (int kk = 0; kk < pf::kHeadDim / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * pf::kSlab + (kk & 3) * 32;
+              tc::mma_f16_ss(tmem + pf::kColS + h * pf::kKeys, tc::sw128_desc(qh + off, 16, 1024),
+                             tc::sw128_desc(kst + off, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+            }
+            tc::commit(bar(pf::kSFull + h));
+          };
+          // O_h += P_h · V_j (P hi in the first 64 columns of the half's buffer, P lo in the next 64)
+          auto issue_pv = [&](int h, int j) {
+            const uint32_t vst = base + pf::kOffV + ((gc + j) % pf::kStages) * pf::kTile;
+            const uint32_t pt = tmem + pf::kColS + h * pf::kKeys;
+  #pragma unroll
+            for (int part = 0; part < parts; ++part) {
+  #pragma unroll
+              for (int kk = 0; kk < pf::kKeys / 16; ++kk) {
+                const uint32_t bv = vst + kk * 16 * 128;  // 16 keys of 128-byte rows
+                tc::mma_f16_ts(tmem + pf::kColO + h * pf::kHeadDim, pt + part * (pf::kKeys / 2) + kk * 8,
+                               tc::sw128_desc(bv, pf::kSlab, 1024), id_o, (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
+              }
+            }
+          };
+          auto wait_k = [&](int j) {
+            const int gj = gc + j;
+            const bool r = mbar_wait_sleep(bar(pf::kKFull + gj % pf::kStages), (gj / pf::kStages) & 1, abort_flag);
+            tc::fence_after_sync();
+            return r;
+          };
+          // the tile's first q·Kᵀ of both halves
+          ok = mbar_wait_sleep(bar(pf::kQFull), tv & 1, abort_flag) &&
+               mbar_wait_sleep(bar(pf::kQFull + 1), tv & 1, abort_flag) && wait_k(0);
+          if (ok) {
+            issue_s(0, 0);
+            if (nc == 1) tc::commit(bar(pf::kQEmpty));  // half A's last q·Kᵀ
+            issue_s(1, 0);
+            if (nc == 1) tc::commit(bar(pf::kQEmpty + 1));
+            tc::commit(bar(pf::kKEmpty + gc % pf::kStages));
+          }
+          for (int j = 0; j < nc && ok; ++j) {
+            const int gj = gc + j;
+            const int s = gj % pf::kStages;
+            ok = mbar_wait_sleep(bar(pf::kVFull + s), (gj / pf::kStages) & 1, abort_flag);
+            // half A: its P·V (after the previous tile's O_A has left tensor
+            // memory), then its next q·Kᵀ, which waits for the next K stage
+            if (ok && j == 0 && tv > 0) ok = mbar_wait_sleep(bar(pf::kOFree), (tv - 1) & 1, abort_flag);
+            if (ok) ok = mbar_wait_sleep(bar(pf::kPFull), gj & 1, abort_flag);
+            if (!ok) break;
+            tc::fence_after_sync();
+            issue_pv(0, j);
+            if (j + 1 < nc) {
+              if (!(ok = wait_k(j + 1))) break;
+              issue_s(0, j + 1);
+              if (j + 1 == nc - 1) tc::commit(bar(pf::kQEmpty));
+            } else {
+              tc::commit(bar(pf::kODone));  // O_A is complete once its last P·V is
+            }
+            // half B likewise; V_j and K_{j+1} are then free
+            if (j == 0 && tv > 0) ok = mbar_wait_sleep(bar(pf::kOFree + 1), (tv - 1) & 1, abort_flag);
+            if (ok) ok = mbar_wait_sleep(bar(pf::kPFull + 1), gj & 1, abort_flag);
+            if (!ok) break;
+            tc::fence_after_sync();
+            issue_pv(1, j);
+            tc::commit(bar(pf::kVEmpty + s));
+            if (j + 1 < nc) {
+              issue_s(1, j + 1);
+              tc::commit(bar(pf::kKEmpty + (gj + 1) % pf::kStages));
+              if (j + 1 == nc - 1) tc::commit(bar(pf::kQEmpty + 1));
+            } else {
+              tc::commit(bar(pf::kODone + 1));
+            }
+          }
+        }
+        ok = __shfl_sync(pf::kAll, ok, 0);
+        gc += nc;
+        ++tv;
+      }
+      if (lane == 0) {
+        if (!ok) {
+          record_error(PKV_ERR_DEVICE_TIMEOUT);
+          *abort_flag = 1;
+        }
+        // every MMA issued completes before tensor memory is freed
+        tc::commit(bar(pf::kDrain));
+        mbar_drain(bar(pf::kDrain), 0);
+      }
+      __syncwarp();
     }
-    __syncwarp();
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 184;\n" ::: "memory");
     // ------------------------------ softmax warps ------------------------------
     const int hh = warp >> 2;               // half of the tile
     const int r = (warp & 3) * 32 + lane;   // row of the half and TMEM lane
@@ -700,7 +711,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         }
         tc::wait_st();
         tc::fence_before_sync();
-        mbar_arrive(bar(pf::kPFull + hh));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(pf::kPFull + hh));
       }
       // the MMA warp commits O-done after the half's last P·V
       if (ok) ok = __all_sync(pf::kAll, mbar_wait_sleep(bar(pf::kODone + hh), tv & 1, abort_flag));
@@ -721,7 +733,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         tc::wait_ld();
         if (q == 3) {
           tc::fence_before_sync();
-          mbar_arrive(bar(pf::kOFree + hh));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(pf::kOFree + hh));
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i)
