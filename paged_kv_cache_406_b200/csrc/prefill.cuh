@@ -305,11 +305,15 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
   // Persistent CTAs (one per SM).  The K producer draws tile numbers from a
   // counter and publishes each in one of two slots (tile-ready barrier); the
   // other roles read it and hand the slot back (tile-free barrier).  Tile t
-  // is the (sequence b, KV head g, tile of QT2 query tokens) of the order: the
-  // tiles of one (b, g) one after another, most keys first, so the tiles in
-  // flight at any time share a few sequences' K/V in L2 (taking one tile
-  // index of every (b, g) together re-read K/V from DRAM about 7x); drawing
-  // them from a counter balances the SMs as they finish.  Each role moves on
+  // is the (sequence b, KV head g, tile of QT2 query tokens) of the order:
+  // sequence by sequence, and within a sequence tile by tile, most keys
+  // first, each tile for all KV heads.  The tiles in flight at any time then
+  // share a few sequences' K/V in L2 (taking one tile index of every
+  // sequence together re-read K/V from DRAM about 7x), and each sequence
+  // hands out its short tiles last (taking all tiles of one KV head before
+  // the next left the longest tiles of the last sequence's last heads to
+  // the end of the launch, with most SMs idle); drawing them from a counter
+  // balances the SMs as they finish.  Each role moves on
   // to the next tile as soon as its own part is done, so the next tile's Q
   // and K loads and its first q·Kᵀ run during this tile's last P·V and
   // output; only the next tile's first P·V waits for the output to have left
@@ -323,10 +327,11 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
   };
   auto tile_of = [&](int t) {
     Tile d{};
-    const int bg = t / p.n_tiles;
-    const int tile = p.n_tiles - 1 - t % p.n_tiles;
-    d.b = bg / p.num_kv_heads;
-    d.g = bg % p.num_kv_heads;
+    const int per_seq = p.n_tiles * p.num_kv_heads;
+    d.b = t / per_seq;
+    const int w = t - d.b * per_seq;
+    const int tile = p.n_tiles - 1 - w / p.num_kv_heads;  // most keys first
+    d.g = w % p.num_kv_heads;
     d.q0 = p.q_start[d.b];
     const int q1 = p.q_start[d.b + 1];
     d.n = q1 - d.q0;
