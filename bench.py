@@ -64,17 +64,17 @@ def prequeue():
 # DRAM traffic of one pkv_append_and_decode call per workload, from the ncu
 # captures summarised in profiles/ (dram__bytes_read.sum +
 # dram__bytes_write.sum over the append + plan, decode and merge kernels, mean
-# of two captured calls), with the hash of the decode sources they were taken
+# of the captured calls), with the hash of the decode sources they were taken
 # on (kernel_source_sha()).  A pin whose hash no longer matches is reported as
 # null.
 TRAFFIC = {
-    "llama3_8b": (607322368, "9a6d1ec7b8826ff0"),
-    "llama3_8b_fp8": (307472256, "9a6d1ec7b8826ff0"),
+    "llama3_8b": (608189696, "63144cce5d01af9c"),
+    "llama3_8b_fp8": (308448870, "63144cce5d01af9c"),
 }
 # the same for one pkv_paged_attention_prefill call (prefill_tc_kernel), keyed
 # by the hash of the prefill sources (kernel_source_sha(PREFILL_SOURCES))
 TRAFFIC_PREFILL = {
-    "prefill_llama3_8b": (330391680, "9a32dc64e7837fe2"),
+    "prefill_llama3_8b": (329096448, "a84cd42cef03ca0c"),
 }
 
 
