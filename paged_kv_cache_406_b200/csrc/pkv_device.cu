@@ -1191,9 +1191,12 @@ int launch_prefill(const pkv::PrefillParams& p, const void* q, const void* k_poo
     a.max_blocks = p.max_blocks;
     a.block_size = p.block_size;
     a.block_pieces = p.num_kv_heads * p.block_size * 128 / 8;
-    // whole blocks per CTA: about 8 CTAs per SM over the batch
+    // at most two whole blocks per CTA: the CTAs past a sequence's last block
+    // return at once and the block scheduler balances sequences of different
+    // lengths (a fixed ~8 CTAs per SM over the batch left the CTAs of the
+    // longest sequences copying four blocks while the rest had finished)
     const int ny = std::min(p.num_seqs, 65535);
-    const int nx = std::max(1, std::min(p.max_blocks, (8 * sm_count(dev) + ny - 1) / ny));
+    const int nx = std::max(1, (p.max_blocks + 1) / 2);
     pkv::stage_v_f16_kernel<<<dim3(nx, ny), 256, 0, stream>>>(a);
   }
   if constexpr (std::is_same<T, __half>::value) {
