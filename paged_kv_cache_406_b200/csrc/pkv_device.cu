@@ -1132,7 +1132,7 @@ size_t prefill_stage_bytes(int64_t num_seqs, int64_t num_kv_heads, int64_t max_b
 // CTA per SM, its own tile-counter slot.
 template <typename T, int G, bool kF16P>
 int launch_prefill_instance(const pkv::PrefillParams& p, const CUtensorMap& mq, const CUtensorMap& mk,
-                            const CUtensorMap& mv, int dev, cudaStream_t stream) {
+                            const CUtensorMap& mv, int dev, cudaStream_t stream, bool pdl = false) {
   auto kern = pkv::prefill_tc_kernel<T, G, kF16P>;
   static std::atomic<bool> configured[kMaxDevices];
   if (dev >= kMaxDevices || !configured[dev].load(std::memory_order_relaxed)) {
@@ -1146,7 +1146,13 @@ int launch_prefill_instance(const pkv::PrefillParams& p, const CUtensorMap& mq, 
   unsigned int* ctr = nullptr;
   int rc = prefill_counter(&ctr);
   if (rc) return rc;
-  kern<<<static_cast<unsigned>(grid), pkv::pf::kThreads, pkv::pf::kSmemBytes, stream>>>(p, mq, mk, mv, ctr);
+  if (pdl) {
+    const cudaError_t el = launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(pkv::pf::kThreads),
+                                      pkv::pf::kSmemBytes, stream, p, mq, mk, mv, ctr);
+    if (el != cudaSuccess) return cuda_fail(el, "prefill kernel launch");
+  } else {
+    kern<<<static_cast<unsigned>(grid), pkv::pf::kThreads, pkv::pf::kSmemBytes, stream>>>(p, mq, mk, mv, ctr);
+  }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
   return PKV_OK;
@@ -1205,7 +1211,7 @@ int launch_prefill(const pkv::PrefillParams& p, const void* q, const void* k_poo
     // the bf16 instance runs only if the staging found a value beyond the
     // f16 range, the f16 one only if it did not; the other returns at once
     rc = launch_prefill_instance<__nv_bfloat16, G, false>(pp, mq, mk, mv, dev, stream);
-    if (!rc) rc = launch_prefill_instance<__nv_bfloat16, G, true>(pp, mq, mk, mvs, dev, stream);
+    if (!rc) rc = launch_prefill_instance<__nv_bfloat16, G, true>(pp, mq, mk, mvs, dev, stream, true);
   } else {
     rc = launch_prefill_instance<__nv_bfloat16, G, false>(pp, mq, mk, mv, dev, stream);
   }

@@ -266,6 +266,12 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   static_assert(kBf16 || kF16P, "f16 pools take the one-pass f16 P");
   constexpr bool f16p = kF16P;
+  // A staged bf16 call launches the hi + lo instance and then the f16 one
+  // programmatically serialised: the first lets the second be scheduled at
+  // once, and the second waits for the first (so for the staging before it)
+  // before reading the staging record.  Both are no-ops for a plain launch.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (kBf16 && p.v_staged) {
     const bool beyond = *p.v_range == p.epoch;
     if (beyond == kF16P) return;  // the other instance of this call does the work
