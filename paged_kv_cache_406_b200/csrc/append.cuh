@@ -71,6 +71,9 @@ __device__ __forceinline__ void append_chunk(const AppendArgs& a, int64_t i) {
 __global__ void __launch_bounds__(256) kv_append_kernel(const AppendArgs a) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i < a.n_units) append_chunk(a, i);
+  // a programmatically serialised successor (the prefill's V staging) may be
+  // scheduled now; it still waits for this grid's writes before reading
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------

@@ -1203,17 +1203,20 @@ int launch_prefill(const pkv::PrefillParams& p, const void* q, const void* k_poo
     // longest sequences copying four blocks while the rest had finished)
     const int ny = std::min(p.num_seqs, 65535);
     const int nx = std::max(1, (p.max_blocks + 1) / 2);
-    pkv::stage_v_f16_kernel<<<dim3(nx, ny), 256, 0, stream>>>(a);
+    const cudaError_t es = launch_pdl(pkv::stage_v_f16_kernel, dim3(nx, ny), dim3(256), 0, stream, a);
+    if (es != cudaSuccess) return cuda_fail(es, "V staging launch");
   }
+  // every launch programmatically serialised: each kernel waits for its
+  // predecessor (griddepcontrol.wait) before reading anything
   if constexpr (std::is_same<T, __half>::value) {
-    rc = launch_prefill_instance<__half, G, true>(pp, mq, mk, mv, dev, stream);
+    rc = launch_prefill_instance<__half, G, true>(pp, mq, mk, mv, dev, stream, true);
   } else if (v_stage) {
     // the bf16 instance runs only if the staging found a value beyond the
     // f16 range, the f16 one only if it did not; the other returns at once
-    rc = launch_prefill_instance<__nv_bfloat16, G, false>(pp, mq, mk, mv, dev, stream);
+    rc = launch_prefill_instance<__nv_bfloat16, G, false>(pp, mq, mk, mv, dev, stream, true);
     if (!rc) rc = launch_prefill_instance<__nv_bfloat16, G, true>(pp, mq, mk, mvs, dev, stream, true);
   } else {
-    rc = launch_prefill_instance<__nv_bfloat16, G, false>(pp, mq, mk, mv, dev, stream);
+    rc = launch_prefill_instance<__nv_bfloat16, G, false>(pp, mq, mk, mv, dev, stream, true);
   }
   if (rc) return rc;
   return pkv::ok();

@@ -219,6 +219,9 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4 w, bool& over) {
 }
 
 __global__ void __launch_bounds__(256) stage_v_f16_kernel(const VStageArgs a) {
+  // launched programmatically serialised: the previous kernel of the stream
+  // (the append of the chunk's rows) is complete before anything is read
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   constexpr int kUnroll = 4;
   bool over = false;
   const int pieces = a.block_pieces;
@@ -247,6 +250,7 @@ __global__ void __launch_bounds__(256) stage_v_f16_kernel(const VStageArgs a) {
     }
   }
   if (__any_sync(0xffffffffu, over) && (threadIdx.x & 31) == 0) atomicExch(a.range, a.epoch);
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the prefill instances wait for this grid
 }
 
 // kF16P: one f16 P and one P·V pass over f16 V (the pool's own for f16 pools,
@@ -266,10 +270,11 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   static_assert(kBf16 || kF16P, "f16 pools take the one-pass f16 P");
   constexpr bool f16p = kF16P;
-  // A staged bf16 call launches the hi + lo instance and then the f16 one
-  // programmatically serialised: the first lets the second be scheduled at
-  // once, and the second waits for the first (so for the staging before it)
-  // before reading the staging record.  Both are no-ops for a plain launch.
+  // Launched programmatically serialised (behind the V staging, or the other
+  // instance of a staged bf16 call, or whatever the stream ran before): the
+  // next instance may be scheduled at once, and this one waits for the
+  // previous kernel (so for the staging and the append before it) before
+  // reading anything.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   if (kBf16 && p.v_staged) {
