@@ -68,13 +68,13 @@ def prequeue():
 # on (kernel_source_sha()).  A pin whose hash no longer matches is reported as
 # null.
 TRAFFIC = {
-    "llama3_8b": (608189696, "63144cce5d01af9c"),
-    "llama3_8b_fp8": (308448870, "63144cce5d01af9c"),
+    "llama3_8b": (608230758, "7daaec3872a1cfe9"),
+    "llama3_8b_fp8": (308158284, "7daaec3872a1cfe9"),
 }
 # the same for one pkv_paged_attention_prefill call (prefill_tc_kernel), keyed
 # by the hash of the prefill sources (kernel_source_sha(PREFILL_SOURCES))
 TRAFFIC_PREFILL = {
-    "prefill_llama3_8b": (329096448, "a84cd42cef03ca0c"),
+    "prefill_llama3_8b": (328944128, "ae50fc52d00e931f"),
 }
 
 
