@@ -1132,7 +1132,7 @@ size_t prefill_stage_bytes(int64_t num_seqs, int64_t num_kv_heads, int64_t max_b
 // CTA per SM, its own tile-counter slot.
 template <typename T, int G, bool kF16P>
 int launch_prefill_instance(const pkv::PrefillParams& p, const CUtensorMap& mq, const CUtensorMap& mk,
-                            const CUtensorMap& mv, int dev, cudaStream_t stream, bool pdl = false) {
+                            const CUtensorMap& mv, int dev, cudaStream_t stream) {
   auto kern = pkv::prefill_tc_kernel<T, G, kF16P>;
   static std::atomic<bool> configured[kMaxDevices];
   if (dev >= kMaxDevices || !configured[dev].load(std::memory_order_relaxed)) {
@@ -1146,14 +1146,10 @@ int launch_prefill_instance(const pkv::PrefillParams& p, const CUtensorMap& mq, 
   unsigned int* ctr = nullptr;
   int rc = prefill_counter(&ctr);
   if (rc) return rc;
-  if (pdl) {
-    const cudaError_t el = launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(pkv::pf::kThreads),
-                                      pkv::pf::kSmemBytes, stream, p, mq, mk, mv, ctr);
-    if (el != cudaSuccess) return cuda_fail(el, "prefill kernel launch");
-  } else {
-    kern<<<static_cast<unsigned>(grid), pkv::pf::kThreads, pkv::pf::kSmemBytes, stream>>>(p, mq, mk, mv, ctr);
-  }
-  const cudaError_t e = cudaGetLastError();
+  // programmatically serialised: the kernel waits for its predecessor
+  // (griddepcontrol.wait) before reading anything
+  const cudaError_t e = launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(pkv::pf::kThreads),
+                                   pkv::pf::kSmemBytes, stream, p, mq, mk, mv, ctr);
   if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
   return PKV_OK;
 }
@@ -1209,14 +1205,14 @@ int launch_prefill(const pkv::PrefillParams& p, const void* q, const void* k_poo
   // every launch programmatically serialised: each kernel waits for its
   // predecessor (griddepcontrol.wait) before reading anything
   if constexpr (std::is_same<T, __half>::value) {
-    rc = launch_prefill_instance<__half, G, true>(pp, mq, mk, mv, dev, stream, true);
+    rc = launch_prefill_instance<__half, G, true>(pp, mq, mk, mv, dev, stream);
   } else if (v_stage) {
     // the bf16 instance runs only if the staging found a value beyond the
     // f16 range, the f16 one only if it did not; the other returns at once
-    rc = launch_prefill_instance<__nv_bfloat16, G, false>(pp, mq, mk, mv, dev, stream, true);
-    if (!rc) rc = launch_prefill_instance<__nv_bfloat16, G, true>(pp, mq, mk, mvs, dev, stream, true);
+    rc = launch_prefill_instance<__nv_bfloat16, G, false>(pp, mq, mk, mv, dev, stream);
+    if (!rc) rc = launch_prefill_instance<__nv_bfloat16, G, true>(pp, mq, mk, mvs, dev, stream);
   } else {
-    rc = launch_prefill_instance<__nv_bfloat16, G, false>(pp, mq, mk, mv, dev, stream, true);
+    rc = launch_prefill_instance<__nv_bfloat16, G, false>(pp, mq, mk, mv, dev, stream);
   }
   if (rc) return rc;
   return pkv::ok();

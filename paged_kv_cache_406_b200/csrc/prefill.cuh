@@ -327,8 +327,9 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
   // balances the SMs as they finish.  Each role moves on
   // to the next tile as soon as its own part is done, so the next tile's Q
   // and K loads and its first q·Kᵀ run during this tile's last P·V and
-  // output; only the next tile's first P·V waits for the output to have left
-  // tensor memory (O-free), and the next Q load for the last q·Kᵀ (Q-empty).
+  // output; only a half's first P·V of the next tile waits for its output to
+  // have left tensor memory (O-free), and its next Q load for its last q·Kᵀ
+  // (Q-empty).
   // The barriers count phases across tiles: gc is the number of key chunks
   // and tv the number of tiles a role has done before the current one (the
   // same sequence in every role); chunk j of a tile is chunk gc + j.
@@ -383,9 +384,10 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     if (warp == pf::kProducerK || warp == pf::kProducerV) {
       // ----------------------------- TMA producers -----------------------------
       // One warp streams K chunks (and Q), the other V chunks, each through its
-      // own ring: K runs ahead of V (q·Kᵀ of chunk j+2 is issued right after
-      // P·V of chunk j, while V's stages free only as P·V completes; a single
-      // producer alternating K and V held K behind V's refills).
+      // own ring: K runs ahead of V (q·Kᵀ of chunk j+1 is issued right after
+      // each half's P·V of chunk j, while V's stages free only as both halves'
+      // P·V complete; a single producer alternating K and V held K behind V's
+      // refills).
       const int kv = warp == pf::kProducerV ? 1 : 0;
       bool ok = true;
       int gc = 0, tv = 0;
