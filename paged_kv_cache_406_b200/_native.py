@@ -78,7 +78,9 @@ SIGNATURES = {
     "pkv_append_and_decode_fp8": (ctypes.c_int, [_vp, _vp, _i32, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
                                                  _i32, _i32, _i32, _i32, _f32, _f32, _f32, _i32, _vp, _sz, _vp, _vp]),
     "pkv_step_meta_bytes": (ctypes.c_size_t, [_i32, _i32]),
-    "pkv_decode_step_host": (ctypes.c_int, [_vp, _pi64, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32,
+    # seq_ids (const int64_t*) as a plain address: the per-step caller passes
+    # the int64 array's address without building a ctypes pointer object
+    "pkv_decode_step_host": (ctypes.c_int, [_vp, _vp, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32,
                                             _i32, _f32, _f32, _i32, _vp, _sz, _vp]),
     "pkv_paged_attention_prefill": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                                                    _i32, _i32, _i32, _f32, _i32, _vp, _sz, _vp, _vp]),

@@ -165,7 +165,22 @@ class PagedKVCache:
         self._ensure_step(n, hq)
         k = self._step_k
         self._step_k ^= 1
-        ws, _ = self._buffers(n, hq, partition_tokens)
+        # per (n, Hq, partition size): the workspace and the call's fixed
+        # arguments, so that a step marshals only what changes
+        key = (n, hq, int(partition_tokens))
+        fixed = self._step_fixed.get(key) if hasattr(self, "_step_fixed") else None
+        if fixed is None:
+            if not hasattr(self, "_step_fixed"):
+                self._step_fixed = {}
+            ws, _ = self._buffers(n, hq, partition_tokens)
+            fixed = (self.k_pool.data_ptr(), self.v_pool.data_ptr(), self.num_blocks, hq, self.num_kv_heads,
+                     self.head_dim, self.block_size, self.max_blocks)
+            tail = (B._dtype_code(self.k_pool), self.k_scale, self.v_scale, int(partition_tokens), ws.data_ptr(),
+                    ws.numel())
+            dev = self.device.index if self.device.index is not None else torch.cuda.current_device()
+            fixed = (fixed, tail, dev, ws)  # holds ws: its address stays valid
+            self._step_fixed[key] = fixed
+        head, tail, dev, _ = fixed
         b = self._step_bufs[k]
         out = self._step_out[k]
         b.q_host, b.k_host, b.v_host = q_host.data_ptr(), k_host.data_ptr(), v_host.data_ptr()
@@ -173,10 +188,8 @@ class PagedKVCache:
         b.h2d_stream = self._h2d_stream.cuda_stream if overlap else None
         b.d2h_stream = self._d2h_stream.cuda_stream if overlap else None
         check(lib().pkv_decode_step_host(
-            self.alloc._h, ids.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n, ctypes.byref(b),
-            self.k_pool.data_ptr(), self.v_pool.data_ptr(), self.num_blocks, hq, self.num_kv_heads, self.head_dim,
-            self.block_size, self.max_blocks, float(scale), B._dtype_code(self.k_pool), self.k_scale, self.v_scale,
-            int(partition_tokens), ws.data_ptr(), ws.numel(), torch.cuda.current_stream(self.device).cuda_stream))
+            self.alloc._h, ids.ctypes.data, n, ctypes.byref(b), *head, float(scale), *tail,
+            torch._C._cuda_getCurrentRawStream(dev)))
         return out_host if out_host is not None else out
 
     def wait_copies(self) -> None:
