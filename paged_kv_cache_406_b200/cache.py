@@ -165,24 +165,23 @@ class PagedKVCache:
         self._ensure_step(n, hq)
         k = self._step_k
         self._step_k ^= 1
-        # per (n, Hq, partition size): the workspace and the call's fixed
-        # arguments, so that a step marshals only what changes
+        # the call's fixed arguments for the current (n, Hq, partition size),
+        # recomputed when it changes (one entry: batch sizes vary step to step)
         key = (n, hq, int(partition_tokens))
-        fixed = self._step_fixed.get(key) if hasattr(self, "_step_fixed") else None
-        if fixed is None:
-            if not hasattr(self, "_step_fixed"):
-                self._step_fixed = {}
+        fixed = getattr(self, "_step_fixed", None)
+        if fixed is None or fixed[0] != key:
             ws, _ = self._buffers(n, hq, partition_tokens)
-            fixed = (self.k_pool.data_ptr(), self.v_pool.data_ptr(), self.num_blocks, hq, self.num_kv_heads,
-                     self.head_dim, self.block_size, self.max_blocks)
+            head = (self.k_pool.data_ptr(), self.v_pool.data_ptr(), self.num_blocks, hq, self.num_kv_heads,
+                    self.head_dim, self.block_size, self.max_blocks)
             tail = (B._dtype_code(self.k_pool), self.k_scale, self.v_scale, int(partition_tokens), ws.data_ptr(),
                     ws.numel())
             dev = self.device.index if self.device.index is not None else torch.cuda.current_device()
-            fixed = (fixed, tail, dev, ws)  # holds ws: its address stays valid
-            self._step_fixed[key] = fixed
+            fixed = (key, (head, tail, dev, ws))  # holds ws: its address stays valid while cached
+            self._step_fixed = fixed
+        fixed = fixed[1]
         head, tail, dev, _ = fixed
         b = self._step_bufs[k]
-        out = self._step_out[k]
+        out = self._step_out[k][:n]
         b.q_host, b.k_host, b.v_host = q_host.data_ptr(), k_host.data_ptr(), v_host.data_ptr()
         b.out_host = out_host.data_ptr() if out_host is not None else None
         b.h2d_stream = self._h2d_stream.cuda_stream if overlap else None
@@ -204,9 +203,17 @@ class PagedKVCache:
                 cur.wait_stream(st)
 
     def _ensure_step(self, n: int, hq: int) -> None:
-        key = (n, hq)
-        if getattr(self, "_step_key", None) == key:
+        # buffers sized by capacity: a batch of up to the largest n seen so far
+        # reuses them; a larger one (or another head count) allocates anew,
+        # after the device has finished with the old ones (copies in flight on
+        # the copy streams read and write them)
+        cap = getattr(self, "_step_key", None)
+        if cap is not None and cap[1] == hq and n <= cap[0]:
             return
+        if cap is not None:
+            torch.cuda.synchronize(self.device)
+        n = max(n, cap[0] if cap is not None else 0)
+        key = (n, hq)
         nbytes = int(lib().pkv_step_meta_bytes(n, self.max_blocks))
         io = torch.float16 if self.fp8 else self.dtype
         self._step_hold = []

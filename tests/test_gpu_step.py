@@ -98,3 +98,32 @@ def test_one_call_steps_in_a_row(native):
     torch.cuda.synchronize()
     assert torch.equal(a.k_pool, b.k_pool)
     assert pkv.pkv_device_status(clear=True) == 0
+
+
+def test_one_call_steps_with_changing_batches(native):
+    """The batch size and the partition size change from step to step (as a
+    serving loop's do): the one-call step reuses its buffers for smaller
+    batches, grows them for larger ones, re-derives its call arguments, and
+    matches the multi-call step bit for bit, with and without the copy
+    streams."""
+    a, b, _, _, _ = _caches("bf16", nb=128)
+    for c in (a, b):
+        for i in range(6):
+            c.add(i, 5 * i + 2)
+    rng = np.random.default_rng(7)
+    for step, n in enumerate([3, 1, 6, 2, 6, 4, 1, 5, 6, 3, 2, 6]):
+        ids = np.arange(n, dtype=np.int64)
+        pt = (0, 32, 64)[step % 3]
+        q = torch.from_numpy(rng.standard_normal((n, 8, 128), dtype=np.float32)).to(torch.bfloat16)
+        kn = torch.from_numpy(rng.standard_normal((n, 2, 128), dtype=np.float32)).to(torch.bfloat16)
+        vn = torch.from_numpy(rng.standard_normal((n, 2, 128), dtype=np.float32)).to(torch.bfloat16)
+        r = a.decode_step(list(ids), q.cuda(), kn.cuda(), vn.cuda(), 0.1, partition_tokens=pt).clone()
+        pinned = (q.pin_memory(), kn.pin_memory(), vn.pin_memory())  # alive until the copies have run
+        out_host = torch.empty((n, 8, 128), dtype=torch.float32, pin_memory=True)
+        g = b.decode_step_host(ids, *pinned, 0.1, out_host=out_host, partition_tokens=pt, overlap=step % 4 != 3)
+        b.wait_copies()
+        torch.cuda.synchronize()
+        assert torch.equal(r.cpu(), g), f"step {step} (n {n}, partitions of {pt})"
+    torch.cuda.synchronize()
+    assert torch.equal(a.k_pool, b.k_pool) and torch.equal(a.v_pool, b.v_pool)
+    assert pkv.pkv_device_status(clear=True) == 0
