@@ -165,12 +165,15 @@ class PagedKVCache:
         self._ensure_step(n, hq)
         k = self._step_k
         self._step_k ^= 1
-        # the call's fixed arguments for the current (n, Hq, partition size),
-        # recomputed when it changes (one entry: batch sizes vary step to step)
-        key = (n, hq, int(partition_tokens))
+        # the call's fixed arguments for the step buffers' capacity and this
+        # partition size (a workspace sized for the capacity serves every
+        # smaller batch), recomputed when either changes
+        key = (self._step_key, int(partition_tokens))
         fixed = getattr(self, "_step_fixed", None)
         if fixed is None or fixed[0] != key:
-            ws, _ = self._buffers(n, hq, partition_tokens)
+            need = B.pkv_decode_workspace_size(self._step_key[0], hq, self.num_kv_heads, self.head_dim,
+                                               self.max_blocks, self.block_size, partition_tokens)
+            ws = torch.empty(max(1, need), dtype=torch.uint8, device=self.device)
             head = (self.k_pool.data_ptr(), self.v_pool.data_ptr(), self.num_blocks, hq, self.num_kv_heads,
                     self.head_dim, self.block_size, self.max_blocks)
             tail = (B._dtype_code(self.k_pool), self.k_scale, self.v_scale, int(partition_tokens), ws.data_ptr(),
