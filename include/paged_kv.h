@@ -513,6 +513,19 @@ int pkv_device_status(void* stream, int32_t* status, int32_t clear);
  * at each launch; always returns PKV_OK. */
 int pkv_debug_stall_decode(int32_t cta);
 
+/* The same for the prefill kernel (pkv_paged_attention_prefill): every wait
+ * of its roles gives up after the same limit (1 s), records
+ * PKV_ERR_DEVICE_TIMEOUT and sets the CTA's abort flag, after which every
+ * role of the CTA leaves its tile loop.  For the prefill launches that
+ * follow, the K producer of CTA `cta` skips its first chunk of K, so the MMA
+ * warp waits for a chunk that never arrives and gives up after the limit;
+ * the producers still wait, with the same limit, for every copy they did
+ * issue before the CTA exits.  The other CTAs finish their tiles.  cta < 0
+ * restores normal operation (the default).  Outputs of a stalled call are
+ * unspecified; prefill does not write the pools.  Process-wide setting,
+ * read at each call; always returns PKV_OK. */
+int pkv_debug_stall_prefill(int32_t cta);
+
 #ifdef __cplusplus
 }
 #endif

@@ -11,6 +11,7 @@ from .binding import (Allocator, PagedKVError, pkv_append_and_decode, pkv_append
                       pkv_device_status, pkv_kv_append, pkv_kv_append_fp8, pkv_paged_attention_decode,
                       pkv_paged_attention_decode_fp8, pkv_paged_attention_decode_static,
                       pkv_paged_attention_prefill, pkv_prefill_workspace_size, pkv_debug_stall_decode,
+                      pkv_debug_stall_prefill,
                       pkv_append_and_decode_pools, pkv_decode_pools_workspace_size,
                       bind_append_and_decode)
 from ._native import LIB_PATH, lib  # noqa: F401

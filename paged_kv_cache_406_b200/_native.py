@@ -66,6 +66,7 @@ SIGNATURES = {
                                                   _i32, _f32, _i32, _i32, _vp, _sz, _vp, _vp]),
     "pkv_device_status": (ctypes.c_int, [_vp, _pi32, _i32]),
     "pkv_debug_stall_decode": (ctypes.c_int, [_i32]),
+    "pkv_debug_stall_prefill": (ctypes.c_int, [_i32]),
     "pkv_paged_attention_decode_static": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                                                          _i32, _i32, _f32, _i32, _i32, _vp, _vp]),
     "pkv_static_workspace_bytes": (ctypes.c_size_t, []),

@@ -427,6 +427,14 @@ def pkv_debug_stall_decode(cta: int = -1) -> None:
     check(lib().pkv_debug_stall_decode(int(cta)))
 
 
+def pkv_debug_stall_prefill(cta: int = -1) -> None:
+    """Test support for the prefill kernel's bounded waits: in the prefill
+    launches that follow, the K producer of CTA ``cta`` skips its first
+    chunk, so the MMA warp's wait for it runs out (after the normal limit);
+    ``cta < 0`` restores normal operation."""
+    check(lib().pkv_debug_stall_prefill(int(cta)))
+
+
 # ----------------------------------------------------------------------------
 # host block allocator
 # ----------------------------------------------------------------------------
@@ -523,7 +531,7 @@ class Allocator:
 
 __all__ = ["Allocator", "PagedKVError", "pkv_kv_append", "pkv_copy_blocks", "pkv_decode_workspace_size",
            "pkv_paged_attention_decode", "pkv_paged_attention_decode_static", "pkv_device_status",
-           "pkv_debug_stall_decode", "pkv_paged_attention_prefill", "pkv_prefill_workspace_size",
+           "pkv_debug_stall_decode", "pkv_debug_stall_prefill", "pkv_paged_attention_prefill", "pkv_prefill_workspace_size",
            "pkv_append_and_decode_pools", "pkv_decode_pools_workspace_size", "bind_append_and_decode",
            "pkv_kv_append_fp8", "pkv_paged_attention_decode_fp8", "pkv_append_and_decode",
            "pkv_append_and_decode_fp8"]

@@ -140,6 +140,8 @@ struct PendingAppend {
 // Test support for the decode kernels' bounded waits (pkv_debug_stall_decode):
 // a CTA whose first work unit gets no copies.
 std::atomic<int> g_stall_cta{-1};
+// the same for the prefill kernel (pkv_debug_stall_prefill)
+std::atomic<int> g_stall_prefill_cta{-1};
 
 void apply_debug(pkv::DecodeParams& p) { p.stall_cta = g_stall_cta.load(std::memory_order_relaxed); }
 
@@ -618,6 +620,11 @@ extern "C" int pkv_append_and_decode(const void* k_new, const void* v_new, const
   return decode_16(fn, q, k_pool, v_pool, block_tables, seq_lens, num_seqs, num_q_heads, num_kv_heads, head_dim,
                    num_blocks, max_blocks_per_seq, block_size, scale, dtype, partition_tokens, workspace,
                    workspace_bytes, out, n_tokens > 0 ? &ap : nullptr, stream);
+}
+
+extern "C" int pkv_debug_stall_prefill(int32_t cta) {
+  g_stall_prefill_cta.store(cta < 0 ? -1 : cta, std::memory_order_relaxed);
+  return pkv::ok();
 }
 
 extern "C" int pkv_debug_stall_decode(int32_t cta) {
@@ -1292,6 +1299,7 @@ extern "C" int pkv_paged_attention_prefill(const void* q, const void* k_pool, co
   p.max_q_len = max_q_len;
   p.n_tiles = static_cast<int32_t>(n_tiles);
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.stall_cta = g_stall_prefill_cta.load(std::memory_order_relaxed);
   void* v_stage = nullptr;
   if (dtype == PKV_BF16 && workspace) {
     const size_t need = prefill_stage_bytes(num_seqs, num_kv_heads, max_blocks_per_seq, block_size);

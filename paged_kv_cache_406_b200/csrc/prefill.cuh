@@ -84,6 +84,10 @@ struct PrefillParams {
   int32_t v_staged;
   uint32_t epoch;
   const uint32_t* v_range;
+  // Test support for the bounded waits (pkv_debug_stall_prefill): the K
+  // producer of CTA `stall_cta` skips its first K chunk, so the MMA warp's
+  // wait for it runs out.  stall_cta < 0 in normal calls.
+  int32_t stall_cta = -1;
 };
 
 #ifndef PKV_PREFILL_STAGES
@@ -373,6 +377,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
   };
   const int BS = p.block_size;
   int issued = 0, q_issued[2] = {0, 0};  // producers: fills issued (chunks, Q tiles of each half) in the CTA's count
+  int skipped = -1;                       // the K producer's chunk left out by the stall test support
 
   // Registers: the kernel is launched at 168 a thread (384 x 168 = 64512);
   // the producer / MMA warpgroup (warps 8-11) drops to 112 and the two softmax
@@ -461,12 +466,16 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
           const uint32_t full = full0 + 8 * s;
           ok = __all_sync(pf::kAll, mbar_wait_sleep(empty0 + 8 * s, ph, abort_flag));
           if (!ok) break;
-          if (lane == 0) mbar_arrive_expect_tx(full, static_cast<uint32_t>(nload) * 2u * box_bytes);
-          __syncwarp();
-          if (lane < nload) {
-            const uint32_t dst = ring + s * pf::kTile + lane * box_bytes;
-            tma_load_3d_nohint(dst, map, 0, y, 0, full);
-            tma_load_3d_nohint(dst + pf::kSlab, map, 0, y, 1, full);
+          if (kv == 0 && gc + j == 0 && p.stall_cta == static_cast<int>(blockIdx.x)) {
+            skipped = 0;  // test support: the CTA's first K chunk never arrives
+          } else {
+            if (lane == 0) mbar_arrive_expect_tx(full, static_cast<uint32_t>(nload) * 2u * box_bytes);
+            __syncwarp();
+            if (lane < nload) {
+              const uint32_t dst = ring + s * pf::kTile + lane * box_bytes;
+              tma_load_3d_nohint(dst, map, 0, y, 0, full);
+              tma_load_3d_nohint(dst + pf::kSlab, map, 0, y, 1, full);
+            }
           }
           issued = gc + j + 1;
         }
@@ -486,7 +495,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
             if (q_issued[h] > 0) mbar_drain(bar(pf::kQFull + h), (q_issued[h] - 1) & 1);
         for (int s = 0; s < pf::kStages && s < issued; ++s) {
           const int last = s + (issued - 1 - s) / pf::kStages * pf::kStages;  // last chunk that used stage s
-          mbar_drain(full0 + 8 * s, (last / pf::kStages) & 1);
+          if (last != skipped) mbar_drain(full0 + 8 * s, (last / pf::kStages) & 1);  // a skipped fill never lands
         }
       }
       __syncwarp();

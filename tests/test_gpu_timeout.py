@@ -100,3 +100,53 @@ def test_stall_setting_is_off_by_default(native):
                                        case.scale)
     assert P.pkv_device_status(clear=True) == 0
     assert_close(out, case.oracle(), "bf16", "stall off")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_stalled_prefill_times_out_and_next_call_is_correct(native, dtype):
+    """The prefill kernel's bounded waits: through pkv_debug_stall_prefill the
+    K producer of CTA 0 skips its first chunk of K, the MMA warp gives up
+    after the limit, the CTA's abort flag sends every role out of its tile
+    loop, and the producers drain only the copies they issued.  The other
+    CTAs finish their tiles.  The call ends within the limit plus a margin
+    with the timeout recorded, and the next call matches the oracle (bf16:
+    the staged path, whose f16 instance is the one that stalls)."""
+    import paged_kv_cache_406_b200 as P
+    from test_gpu_prefill import PrefillCase
+    # 8 sequences x 16 tiles of 64 tokens x 2 KV heads = 256 tiles, every one
+    # with rows to compute, more than there are persistent CTAs: CTA 0 draws
+    # work (with tiles past a short chunk's end it could draw only those)
+    case = PrefillCase([1536] * 8, [1024] * 8, 8, 2, 16, dtype, seed=405)
+    case.run()  # first call: module load and tensor maps outside the timing
+    assert P.pkv_device_status(clear=True) == 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    P.pkv_debug_stall_prefill(0)
+    try:
+        t0 = time.perf_counter()
+        e0.record()
+        case.run()
+        e1.record()
+        status = P.pkv_device_status(clear=True)
+        wall = time.perf_counter() - t0
+    finally:
+        P.pkv_debug_stall_prefill(-1)
+    assert status == PKV_ERR_DEVICE_TIMEOUT
+    ms = e0.elapsed_time(e1)
+    # one wait limit (1 s) for the MMA warp, then every role of the CTA leaves;
+    # the skipped fill is not waited for again in the drain
+    assert 900.0 < ms < 1600.0, f"the stalled call took {ms:.1f} ms on the device"
+    assert wall < 10.0
+    out = case.run()
+    assert P.pkv_device_status(clear=True) == 0
+    assert_close(out, case.oracle(), dtype, f"{dtype} prefill after the timed-out call")
+
+
+def test_prefill_stall_setting_is_off_by_default(native):
+    """Without the test call, no prefill launch stalls: a normal call records
+    no timeout."""
+    import paged_kv_cache_406_b200 as P
+    from test_gpu_prefill import PrefillCase
+    case = PrefillCase([300, 129], [77, 1], 8, 2, 16, "bf16", seed=406)
+    out = case.run()
+    assert P.pkv_device_status(clear=True) == 0
+    assert_close(out, case.oracle(), "bf16", "prefill with the stall setting off")
