@@ -74,7 +74,7 @@ TRAFFIC = {
 # the same for one pkv_paged_attention_prefill call (prefill_tc_kernel), keyed
 # by the hash of the prefill sources (kernel_source_sha(PREFILL_SOURCES))
 TRAFFIC_PREFILL = {
-    "prefill_llama3_8b": (329763584, "860769eb3a8f6a14"),
+    "prefill_llama3_8b": (329452800, "8e17c4b8b5daa237"),
 }
 
 
